@@ -1,0 +1,382 @@
+"""Benchmark of the Gated DeltaNet hot path on B200.
+
+One step = one pass of the whole layer path over one batch of synthetic input on the
+1024-wide hybrid-model prefill workload (T = 4096, 16 q/k and 16 v heads, d = 128, bf16):
+chunked gated delta-rule scan -> gated RMSNorm * SiLU(z) with the fused NVFP4 activation
+encode -> NVFP4 W4A4 output projection 2048 -> 1024. The decode step (B = 256 sequences,
+16 q/k / 32 v heads, fp32 state [256, 32, 128, 128] updated in place) is timed in the
+same run and reported under "decode".
+
+Launch: python bench.py [--gpus N --steps K --warmup W] (N > 1 under torchrun, one rank
+per GPU, each rank an independent replica of the workload: weak scaling, no collective
+on the data path). `--impl reference` times the CPU oracle on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "GDN prefill tokens/s & decode GB/s (fraction of B200 roofline), 1 GPU"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+CHUNK = 64
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return d, "measured"
+    except OSError:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def scan_flops(w: workloads.Workload) -> float:
+    """Algorithmic FLOPs of the chunked scan (64-token chunks, d = Dk = Dv): per token,
+    Hv * (6 d^2 + 6 C d) for the state products, W, U~ and the intra-chunk output, plus
+    Hk * 4 C d for K K^T and Q K^T (shared by the value heads of a key head)."""
+    d, C = w.D, CHUNK
+    return float(w.T) * (w.Hv * (6 * d * d + 6 * C * d) + w.Hk * 4 * C * d)
+
+
+def scan_bytes(w: workloads.Workload, o_bytes=2) -> float:
+    """Algorithmic HBM bytes of the scan: q, k, v read once (bf16), a, b (fp32), o written,
+    initial/final states when present."""
+    b = w.T * (2 * w.Hk * w.D * 2 + w.Hv * w.D * 2 + 2 * w.Hv * 4 + w.Hv * w.D * o_bytes)
+    if w.s0_std > 0:
+        b += 2 * w.num_seqs * w.Hv * w.D * w.D * 4
+    return float(b)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- GPU arm ----
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import gated_deltanet_03_b200 as g
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    w = workloads.PREFILL_1K
+    x = workloads.generate(w)
+    bf, f32 = torch.bfloat16, torch.float32
+
+    def up(a, dt):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+
+    q, k, v, z = up(x["q"], bf), up(x["k"], bf), up(x["v"], bf), up(x["z"], bf)
+    a, b = up(x["a"], f32), up(x["b"], f32)
+    A_log, dt_bias, nw = up(x["A_log"], f32), up(x["dt_bias"], f32), up(x["norm_weight"], f32)
+    W = up(x["proj_weight"], bf)
+    gw = float(448.0 * 6.0 / W.float().abs().max().item())
+    wq, ws = g.nvfp4_quantize_act(W, gw)           # weights: quantised once, outside timing
+    T, Hv, D, K, N = w.T, w.Hv, w.D, w.K, w.n_out
+    o = torch.empty((T, Hv, D), dtype=bf, device=dev)
+    S = torch.empty((1, Hv, D, D), dtype=f32, device=dev)
+    xq = torch.empty((T, K // 2), dtype=torch.uint8, device=dev)
+    xs = torch.empty((T, K // 16), dtype=torch.uint8, device=dev)
+    Y = torch.empty((T, N), dtype=bf, device=dev)
+    # activation global scale: one calibration pass outside timing
+    g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, final_state=S, o=o)
+    y_cal = g.gdn_gated_rmsnorm_silu(o, z, nw, out_dtype=f32)
+    gx = float(448.0 * 6.0 / y_cal.abs().max().item())
+    alpha = float(np.float32(1.0) / (np.float32(gx) * np.float32(gw)))
+    del y_cal
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=f32, device=dev)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, final_state=S, o=o)
+        if evs:
+            evs[1].record(stream)
+        g.gdn_gated_rmsnorm_silu_nvfp4(o, z, nw, gx, xq=xq, xs=xs)
+        if evs:
+            evs[2].record(stream)
+        g.nvfp4_gemm(xq, xs, wq, ws, alpha, y=Y)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert g.gdn_get_device_status() == 0
+
+    evsets = [[ev() for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()          # L2 flush between timed steps (outside the events)
+            step(evsets[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evsets]
+    scan_ms = [e[0].elapsed_time(e[1]) for e in evsets]
+    tail_ms = [e[1].elapsed_time(e[2]) for e in evsets]
+    gemm_ms = [e[2].elapsed_time(e[3]) for e in evsets]
+    ms = statistics.mean(step_ms)
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    assert g.gdn_get_device_status() == 0
+
+    # end to end through the public API: pinned host inputs in, host result out
+    hq, hk, hv, hz = (t.cpu().pin_memory() for t in (q, k, v, z))
+    ha, hb = a.cpu().pin_memory(), b.cpu().pin_memory()
+    hY = torch.empty((T, N), dtype=bf, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hz, ha, hb))
+    d2h = hY.numel() * hY.element_size()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+        z.copy_(hz, non_blocking=True); a.copy_(ha, non_blocking=True); b.copy_(hb, non_blocking=True)
+        step()
+        hY.copy_(Y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        s0, s1 = ev(), ev()
+        s0.record(stream)
+        e2e_step()
+        s1.record(stream)
+        s1.synchronize()
+        e2e_ms.append(s0.elapsed_time(s1))
+    e2e = statistics.mean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = float(t.item())
+
+    # decode step on the batched-decode workload (state 512 MiB > L2: no flush needed)
+    dw = workloads.DECODE_B256
+    dx = workloads.generate(dw)
+    dq, dk, dv = up(dx["q"], bf), up(dx["k"], bf), up(dx["v"], bf)
+    da, db = up(dx["a"], f32), up(dx["b"], f32)
+    dA, ddt = up(dx["A_log"], f32), up(dx["dt_bias"], f32)
+    dstate = up(dx["initial_state"], f32)
+    dout = torch.empty((dw.num_seqs, dw.Hv, dw.D), dtype=bf, device=dev)
+    for _ in range(max(3, args.warmup)):
+        g.gdn_decode_step(dq, dk, dv, da, db, dA, ddt, dstate, o=dout)
+    torch.cuda.synchronize()
+    dec_ms = []
+    for _ in range(max(args.steps, 10)):
+        s0, s1 = ev(), ev()
+        s0.record(stream)
+        g.gdn_decode_step(dq, dk, dv, da, db, dA, ddt, dstate, o=dout)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        dec_ms.append(s0.elapsed_time(s1))
+    dec = statistics.median(dec_ms)
+    state_bytes = dstate.numel() * 4
+    dec_bytes = 2 * state_bytes + sum(t.numel() * t.element_size() for t in (dq, dk, dv, da, db, dout))
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    pk, pk_kind = peaks()
+    scan_s = statistics.mean(scan_ms) / 1e3
+    fl = scan_flops(w)
+    achieved_tflops = fl / scan_s / 1e12
+    peak_tflops = float(pk["bf16_tflops"])
+    tokens = T * world
+    out = {
+        "metric": METRIC,
+        "value": tokens / (ms_max / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; shapes of the pages' 1024-wide hybrid layer)",
+        "config": {"workload": w.name, "T": T, "Hk": w.Hk, "Hv": Hv, "d": D, "chunk": CHUNK,
+                   "out_proj": "NVFP4 W4A4 %d->%d" % (K, N), "global_batch": 1, "seq_len": T,
+                   "parallelism": "replicas x%d" % world, "l2": "flushed (256 MiB write) between timed steps"},
+        "breakdown_ms": {"scan": statistics.mean(scan_ms), "gated_norm_nvfp4": statistics.mean(tail_ms),
+                         "nvfp4_gemm": statistics.mean(gemm_ms)},
+        "roofline": {"kernel": "gdn prefill scan", "bound": "tensor", "achieved": achieved_tflops,
+                     "peak": peak_tflops, "unit": "TFLOP/s", "frac": achieved_tflops / peak_tflops,
+                     "peak_kind": pk_kind + " (bf16 dense burst; the scan's MMAs are fp16)",
+                     "algorithmic_flops": fl, "algorithmic_bytes": scan_bytes(w),
+                     "hbm_frac": scan_bytes(w) / scan_s / 1e9 / float(pk["hbm_gbs"]),
+                     "traffic": None},
+        "e2e": {"value": tokens / (e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+        "decode": {"workload": dw.name, "ms": dec, "GB/s": dec_bytes / (dec / 1e3) / 1e9,
+                   "frac": dec_bytes / (dec / 1e3) / 1e9 / float(pk["hbm_gbs"]),
+                   "bytes": dec_bytes, "peak_gbs": float(pk["hbm_gbs"]), "peak_kind": pk_kind},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu:
+        out["cpu_baseline"] = cpu_baseline(w, x)
+    print(json.dumps(out))
+
+
+# ----------------------------------------------------------------- CPU arm ----
+
+def cpu_pass(w, x, units=None):
+    """The oracle over the same workload: scan (threaded over heads), gated tail, NVFP4
+    encode and the fp64 GEMM over dequantised operands."""
+    import oracle
+    o, S = oracle.gdn_scan(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                           cu_seqlens=x["cu_seqlens"], units=units)
+    y = oracle.gated_rmsnorm_silu(workloads.round_bf16(o.astype(np.float32)), x["z"], x["norm_weight"])
+    gx = np.float32(448.0 * 6.0 / max(np.abs(y).max(), 1e-30))
+    W = x["proj_weight"]
+    gw = np.float32(448.0 * 6.0 / np.abs(W).max())
+    xq, xs = oracle.nvfp4_quantize(workloads.round_bf16(y.astype(np.float32)), gx)
+    wq, ws = oracle.nvfp4_quantize(W, gw)
+    return oracle.nvfp4_gemm(xq, xs, gx, wq, ws, gw)
+
+
+def cpu_baseline(w, x):
+    import oracle
+    t0 = time.perf_counter()
+    cpu_pass(w, x)
+    dt = time.perf_counter() - t0
+    return {"value": w.T / dt, "unit": "tokens/s", "cores": oracle.default_threads(), "kind": "oracle",
+            "sample": "the whole workload once (all %d heads, all rows)" % w.Hv, "seconds": dt}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = workloads.PREFILL_1K
+    x = workloads.generate(w)
+    for _ in range(args.warmup):
+        cpu_pass(w, x, units=[0])
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        cpu_pass(w, x)
+        times.append(time.perf_counter() - t0)
+    dt = statistics.mean(times)
+    val = w.T / dt
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; shapes of the pages' 1024-wide hybrid layer)",
+        "config": {"workload": w.name, "T": w.T, "Hk": w.Hk, "Hv": w.Hv, "d": w.D},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": oracle.default_threads(), "kind": "oracle",
+                         "sample": "the whole workload per step (all heads, all rows)"},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    args = p.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

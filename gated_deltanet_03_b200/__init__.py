@@ -1,0 +1,209 @@
+"""Python binding of the Gated DeltaNet B200 library (libgdn_b200.so, C ABI in include/gdn.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels.
+PyTorch provides device memory (output tensors are allocated with torch) and the current
+stream. There is no CPU fallback: if the library is missing, importing this package raises.
+
+Functions keep the C names:
+  gdn_prefill_chunked, gdn_decode_step, gdn_gated_rmsnorm_silu,
+  gdn_gated_rmsnorm_silu_nvfp4, nvfp4_quantize_act, nvfp4_gemm,
+  gdn_prefill_workspace_bytes, gdn_get_device_status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn_b200.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, GDN_ERR_WORKSPACE = range(6)
+GDN_BF16, GDN_F32 = 0, 1
+
+# Exported C symbols, in the order include/gdn.h declares them.
+ABI_SYMBOLS = (
+    "gdn_prefill_chunked", "gdn_prefill_workspace_bytes", "gdn_decode_step",
+    "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act",
+    "nvfp4_gemm", "gdn_get_device_status", "gdn_status_string", "gdn_version",
+)
+
+
+class GdnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__("%s failed: %s (status %d)" % (fn, status_string(status), status))
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libgdn_b200.so is not built (run __graft_entry__.build() or "
+                          "python gated_deltanet_03_b200/build.py)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    lib.gdn_prefill_chunked.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32,
+                                        i32, P, P, P, i32, P, sz, P]
+    lib.gdn_prefill_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+    lib.gdn_prefill_workspace_bytes.restype = sz
+    lib.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, P, P,
+                                    i32, P]
+    lib.gdn_gated_rmsnorm_silu.argtypes = [P, P, P, f32, i32, i32, i32, i32, P, i32, P]
+    lib.gdn_gated_rmsnorm_silu_nvfp4.argtypes = [P, P, P, f32, i32, i32, i32, i32, f32, P, P, P]
+    lib.nvfp4_quantize_act.argtypes = [P, i32, i32, i32, f32, P, P, P]
+    lib.nvfp4_gemm.argtypes = [P, P, P, P, f32, i32, i32, i32, i32, P, P]
+    lib.gdn_get_device_status.argtypes = [P]
+    lib.gdn_status_string.argtypes = [i32]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_version.restype = i32
+    for name in ("gdn_prefill_chunked", "gdn_decode_step", "gdn_gated_rmsnorm_silu",
+                 "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_gemm",
+                 "gdn_get_device_status"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+LIB = _load()
+
+
+def status_string(s: int) -> str:
+    return LIB.gdn_status_string(int(s)).decode()
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError("unsupported dtype %s (bf16 or fp32)" % t.dtype)
+
+
+def _dt_of(dtype) -> int:
+    return GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+
+
+def _check(name: str, status: int):
+    if status != GDN_OK:
+        raise GdnError(name, status)
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def gdn_prefill_workspace_bytes(T, num_seqs, Hk, Hv, Dk, Dv) -> int:
+    return int(LIB.gdn_prefill_workspace_bytes(T, num_seqs, Hk, Hv, Dk, Dv))
+
+
+def gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, initial_state=None,
+                        final_state=None, scale: float = 1.0, qk_l2norm: bool = True,
+                        out_dtype=None, o=None, workspace=None, stream=None):
+    """Gated delta rule over packed sequences. q, k [T, Hk, D]; v [T, Hv, D]; a, b [T, Hv] fp32;
+    A_log, dt_bias [Hv] fp32; cu_seqlens int32 [N+1] on the device or None.
+    Returns (o [T, Hv, D], final_state [N, Hv, D, D] fp32)."""
+    T, Hk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    out_dtype = out_dtype or q.dtype
+    if o is None:
+        o = torch.empty((T, Hv, Dv), dtype=out_dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((N, Hv, Dv, Dk), dtype=torch.float32, device=q.device)
+    _contig(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state, final_state, o)
+    ws_bytes = gdn_prefill_workspace_bytes(T, N, Hk, Hv, Dk, Dv)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=q.device)
+    st = LIB.gdn_prefill_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log),
+                                 _ptr(dt_bias), _ptr(cu_seqlens), N, T, Hk, Hv, Dk, Dv,
+                                 float(scale), int(bool(qk_l2norm)), _dt(q), _ptr(initial_state),
+                                 _ptr(final_state), _ptr(o), _dt(o), _ptr(workspace),
+                                 0 if workspace is None else workspace.numel(), _stream(stream))
+    _check("gdn_prefill_chunked", st)
+    return o, final_state
+
+
+def gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1.0,
+                    qk_l2norm: bool = True, out_dtype=None, o=None, stream=None):
+    """One token per sequence; `state` [B, Hv, D, D] fp32 is updated in place. Returns o."""
+    B, Hk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    out_dtype = out_dtype or q.dtype
+    if o is None:
+        o = torch.empty((B, Hv, Dv), dtype=out_dtype, device=q.device)
+    _contig(q, k, v, a, b, A_log, dt_bias, state, o)
+    st = LIB.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
+                             B, Hk, Hv, Dk, Dv, float(scale), int(bool(qk_l2norm)), _dt(q),
+                             _ptr(state), _ptr(o), _dt(o), _stream(stream))
+    _check("gdn_decode_step", st)
+    return o
+
+
+def gdn_gated_rmsnorm_silu(o, z, weight, eps: float = 1e-6, out_dtype=None, y=None, stream=None):
+    """o, z [M, Hv, D] -> y [M, Hv * D]."""
+    M, Hv, D = o.shape
+    out_dtype = out_dtype or o.dtype
+    if y is None:
+        y = torch.empty((M, Hv * D), dtype=out_dtype, device=o.device)
+    _contig(o, z, weight, y)
+    st = LIB.gdn_gated_rmsnorm_silu(_ptr(o), _ptr(z), _ptr(weight), float(eps), M, Hv, D, _dt(o),
+                                    _ptr(y), _dt(y), _stream(stream))
+    _check("gdn_gated_rmsnorm_silu", st)
+    return y
+
+
+def gdn_gated_rmsnorm_silu_nvfp4(o, z, weight, global_scale: float, eps: float = 1e-6,
+                                 xq=None, xs=None, stream=None):
+    """o, z [M, Hv, D] -> (xq [M, K/2] uint8, xs [M, K/16] uint8), K = Hv * D."""
+    M, Hv, D = o.shape
+    K = Hv * D
+    if xq is None:
+        xq = torch.empty((M, K // 2), dtype=torch.uint8, device=o.device)
+    if xs is None:
+        xs = torch.empty((M, K // 16), dtype=torch.uint8, device=o.device)
+    _contig(o, z, weight, xq, xs)
+    st = LIB.gdn_gated_rmsnorm_silu_nvfp4(_ptr(o), _ptr(z), _ptr(weight), float(eps), M, Hv, D, _dt(o),
+                                          float(global_scale), _ptr(xq), _ptr(xs), _stream(stream))
+    _check("gdn_gated_rmsnorm_silu_nvfp4", st)
+    return xq, xs
+
+
+def nvfp4_quantize_act(x, global_scale: float, xq=None, xs=None, stream=None):
+    """x [M, K] bf16/fp32 -> (xq [M, K/2] uint8, xs [M, K/16] uint8)."""
+    M, K = x.shape
+    if xq is None:
+        xq = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    if xs is None:
+        xs = torch.empty((M, K // 16), dtype=torch.uint8, device=x.device)
+    _contig(x, xq, xs)
+    st = LIB.nvfp4_quantize_act(_ptr(x), _dt(x), M, K, float(global_scale), _ptr(xq), _ptr(xs),
+                                _stream(stream))
+    _check("nvfp4_quantize_act", st)
+    return xq, xs
+
+
+def nvfp4_gemm(aq, as_, bq, bs, alpha: float, out_dtype=torch.bfloat16, y=None, stream=None):
+    """(aq [M, K/2], as [M, K/16]) x (bq [N, K/2], bs [N, K/16])^T * alpha -> y [M, N]."""
+    M, K = aq.shape[0], aq.shape[1] * 2
+    N = bq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=aq.device)
+    _contig(aq, as_, bq, bs, y)
+    st = LIB.nvfp4_gemm(_ptr(aq), _ptr(as_), _ptr(bq), _ptr(bs), float(alpha), M, N, K, _dt(y), _ptr(y),
+                        _stream(stream))
+    _check("nvfp4_gemm", st)
+    return y
+
+
+def gdn_get_device_status(stream=None) -> int:
+    return int(LIB.gdn_get_device_status(_stream(stream)))

@@ -1,0 +1,179 @@
+// C entry points declared in include/gdn.h: host-side argument checks, kernel variant
+// selection and launches on the caller's stream. No device memory is allocated here; the
+// only library-owned device object is the status word that bounded waits report into.
+#include <cstdio>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+__device__ int g_device_status = 0;
+
+constexpr int kMaxDevices = 64;
+int *g_status_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the status word on the current device (looked up once per device).
+int *status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<int *>(p);
+    }
+    return g_status_ptr[dev];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_ok(int32_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool dtype_ok(gdn_dtype t) { return t == GDN_BF16 || t == GDN_F32; }
+
+gdn_status launched(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t gdn_version(void) { return 100; }
+
+const char *gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported size or dtype";
+        case GDN_ERR_CUDA: return "CUDA error";
+        case GDN_ERR_TIMEOUT: return "device-side wait timed out";
+        case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+gdn_status gdn_get_device_status(gdn_stream_t stream) {
+    int *p = status_ptr();
+    if (!p) return GDN_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpyAsync(&h, p, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
+    if (h != 0) {
+        const int zero = 0;
+        if (cudaMemcpyAsync(p, &zero, sizeof(int), cudaMemcpyHostToDevice, stream) != cudaSuccess) return GDN_ERR_CUDA;
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    return static_cast<gdn_status>(h);
+}
+
+size_t gdn_prefill_workspace_bytes(int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv, int32_t Dk,
+                                   int32_t Dv) {
+    (void)T; (void)num_seqs; (void)Hk; (void)Hv; (void)Dk; (void)Dv;
+    return 0;
+}
+
+gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v, const float *a, const float *b,
+                               const float *A_log, const float *dt_bias, const int32_t *cu_seqlens,
+                               int32_t num_seqs, int32_t T, int32_t Hk, int32_t Hv, int32_t Dk, int32_t Dv,
+                               float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                               const float *initial_state, float *final_state, void *o,
+                               gdn_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                               gdn_stream_t stream) {
+    (void)workspace; (void)workspace_bytes;
+    if (T < 0 || num_seqs < 1 || Hk < 1 || Hv < 1 || Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens && num_seqs != 1) return GDN_ERR_INVALID_ARG;
+    if (Dk != Dv) return GDN_ERR_UNSUPPORTED;
+    if (!head_ok(Dk)) return GDN_ERR_UNSUPPORTED;
+    if (T > 0) {
+        if (!q || !k || !v || !a || !b || !o) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return GDN_ERR_INVALID_ARG;
+    }
+    if (!A_log || !dt_bias) return GDN_ERR_INVALID_ARG;
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return GDN_ERR_INVALID_ARG;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (Dk == 128 && in_dtype == GDN_BF16 && T > 0) {
+        gdn::ChunkedArgs c{q, k, v, a, b, A_log, dt_bias, cu_seqlens, T, num_seqs, Hk, Hv, scale, qk_l2norm,
+                           out_dtype == GDN_BF16, initial_state, final_state, o, status_ptr()};
+        cudaError_t e = gdn::launch_chunked(c, st);
+        if (e != cudaErrorNotSupported) return launched(e);
+    }
+    gdn::RecurrentArgs r{q, k, v, a, b, A_log, dt_bias, cu_seqlens, T, num_seqs, Hk, Hv, Dk, scale,
+                         qk_l2norm, in_dtype == GDN_BF16, out_dtype == GDN_BF16, initial_state,
+                         final_state, o};
+    return launched(gdn::launch_recurrent(r, st));
+}
+
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const float *a, const float *b,
+                           const float *A_log, const float *dt_bias, int32_t B, int32_t Hk, int32_t Hv,
+                           int32_t Dk, int32_t Dv, float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                           float *state, void *o, gdn_dtype out_dtype, gdn_stream_t stream) {
+    if (B < 0 || Hk < 1 || Hv < 1 || Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
+    if (Dk != Dv || !head_ok(Dk)) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !A_log || !dt_bias || !state || !o) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
+        return GDN_ERR_INVALID_ARG;
+    gdn::RecurrentArgs r{q, k, v, a, b, A_log, dt_bias, nullptr, 1, B, Hk, Hv, Dk, scale, qk_l2norm,
+                         in_dtype == GDN_BF16, out_dtype == GDN_BF16, state, state, o};
+    return launched(gdn::launch_recurrent(r, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static gdn_status tail_check(const void *o, const void *z, const float *weight, float eps, int32_t M,
+                             int32_t Hv, int32_t Dv, gdn_dtype in_dtype) {
+    if (M < 0 || Hv < 1 || !dtype_ok(in_dtype) || !(eps >= 0.0f)) return GDN_ERR_INVALID_ARG;
+    if (!head_ok(Dv)) return GDN_ERR_UNSUPPORTED;
+    if (M > 0 && (!o || !z || !weight || !aligned16(o) || !aligned16(z))) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+gdn_status gdn_gated_rmsnorm_silu(const void *o, const void *z, const float *weight, float eps, int32_t M,
+                                  int32_t Hv, int32_t Dv, gdn_dtype in_dtype, void *y, gdn_dtype out_dtype,
+                                  gdn_stream_t stream) {
+    gdn_status s = tail_check(o, z, weight, eps, M, Hv, Dv, in_dtype);
+    if (s != GDN_OK) return s;
+    if (!dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
+    if (M == 0) return GDN_OK;
+    if (!y || !aligned16(y)) return GDN_ERR_INVALID_ARG;
+    gdn::TailArgs t{o, z, weight, eps, M, Hv, Dv, in_dtype == GDN_BF16, y, out_dtype == GDN_BF16, 0.0f,
+                    nullptr, nullptr};
+    return launched(gdn::launch_gated_rmsnorm(t, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gdn_status gdn_gated_rmsnorm_silu_nvfp4(const void *o, const void *z, const float *weight, float eps,
+                                        int32_t M, int32_t Hv, int32_t Dv, gdn_dtype in_dtype,
+                                        float global_scale, uint8_t *xq, uint8_t *xs, gdn_stream_t stream) {
+    gdn_status s = tail_check(o, z, weight, eps, M, Hv, Dv, in_dtype);
+    if (s != GDN_OK) return s;
+    if (!(global_scale > 0.0f) || !(global_scale < 3.0e38f)) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)Hv * Dv % 32 != 0) return GDN_ERR_UNSUPPORTED;
+    if (M == 0) return GDN_OK;
+    if (!xq || !xs || !aligned16(xq)) return GDN_ERR_INVALID_ARG;
+    gdn::TailArgs t{o, z, weight, eps, M, Hv, Dv, in_dtype == GDN_BF16, nullptr, true, global_scale, xq, xs};
+    return launched(gdn::launch_gated_rmsnorm_nvfp4(t, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gdn_status nvfp4_quantize_act(const void *x, gdn_dtype in_dtype, int32_t M, int32_t K, float global_scale,
+                              uint8_t *xq, uint8_t *xs, gdn_stream_t stream) {
+    if (M < 0 || K < 0 || !dtype_ok(in_dtype)) return GDN_ERR_INVALID_ARG;
+    if (!(global_scale > 0.0f) || !(global_scale < 3.0e38f)) return GDN_ERR_INVALID_ARG;
+    if (K % 32 != 0) return GDN_ERR_UNSUPPORTED;
+    if (M == 0 || K == 0) return GDN_OK;
+    if (!x || !xq || !xs || !aligned16(x) || !aligned16(xq)) return GDN_ERR_INVALID_ARG;
+    return launched(gdn::launch_nvfp4_quantize(x, in_dtype == GDN_BF16, M, K, global_scale, xq, xs,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gdn_status nvfp4_gemm(const uint8_t *aq, const uint8_t *as, const uint8_t *bq, const uint8_t *bs, float alpha,
+                      int32_t M, int32_t N, int32_t K, gdn_dtype out_dtype, void *y, gdn_stream_t stream) {
+    if (M < 0 || N < 0 || K < 0 || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
+    if (K % 32 != 0 || N % 16 != 0) return GDN_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return GDN_OK;
+    if (K == 0) return GDN_ERR_UNSUPPORTED;
+    if (!aq || !as || !bq || !bs || !y) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(aq) || !aligned16(bq) || !aligned16(y)) return GDN_ERR_INVALID_ARG;
+    gdn::GemmArgs g{aq, as, bq, bs, alpha, M, N, K, out_dtype == GDN_BF16, y, status_ptr()};
+    return launched(gdn::launch_nvfp4_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,67 @@
+// Internal launcher interface between the C entry points (api.cu) and the kernels.
+// Every launcher enqueues on the given stream and returns the launch's cudaError_t.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+struct RecurrentArgs {
+    const void *q, *k, *v;
+    const float *a, *b, *A_log, *dt_bias;
+    const int32_t *cu_seqlens;   // device [num_seqs + 1], or null: seq n = [n*T1, (n+1)*T1)
+    int32_t tokens_per_seq;      // T1 when cu_seqlens is null
+    int32_t num_seqs, Hk, Hv, D;
+    float scale;
+    int32_t l2norm;
+    bool in_bf16, out_bf16;
+    const float *S0;             // may be null (zero state); may alias S_out
+    float *S_out;                // may be null
+    void *o;
+};
+cudaError_t launch_recurrent(const RecurrentArgs &r, cudaStream_t st);
+
+struct ChunkedArgs {
+    const void *q, *k, *v;       // bf16
+    const float *a, *b, *A_log, *dt_bias;
+    const int32_t *cu_seqlens;   // may be null (one sequence of T tokens)
+    int32_t T, num_seqs, Hk, Hv;
+    float scale;
+    int32_t l2norm;
+    bool out_bf16;
+    const float *S0;
+    float *S_out;
+    void *o;
+    int *status;
+};
+cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st);
+
+struct TailArgs {
+    const void *o, *z;
+    const float *w;
+    float eps;
+    int32_t M, Hv, D;
+    bool in_bf16;
+    void *y;                     // gated output (plain variant)
+    bool out_bf16;
+    float gs;                    // NVFP4 variant: encode scale, outputs xq/xs
+    uint8_t *xq, *xs;
+};
+cudaError_t launch_gated_rmsnorm(const TailArgs &t, cudaStream_t st);
+cudaError_t launch_gated_rmsnorm_nvfp4(const TailArgs &t, cudaStream_t st);
+
+cudaError_t launch_nvfp4_quantize(const void *x, bool in_bf16, int32_t M, int32_t K, float gs,
+                                  uint8_t *xq, uint8_t *xs, cudaStream_t st);
+
+struct GemmArgs {
+    const uint8_t *aq, *as, *bq, *bs;
+    float alpha;
+    int32_t M, N, K;
+    bool out_bf16;
+    void *y;
+    int *status;
+};
+cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st);
+
+}  // namespace gdn

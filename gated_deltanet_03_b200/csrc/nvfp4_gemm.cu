@@ -1,0 +1,278 @@
+// NVFP4 W4A4 GEMM on the block-scaled FP4 tensor cores (tcgen05 kind::mxf4nvf4, 16-value
+// E4M3 scale blocks, fp32 accumulation in tensor memory):
+//     y[m, n] = alpha * sum_k E2M1(a)[m,k] E4M3(as)[m,k/16] * E2M1(b)[n,k] E4M3(bs)[n,k/16].
+// "Why Gated DeltaNet Survives 4-Bit Quantization", abstract: NVFP4 W4A4 on every linear
+// layer; "Red Lite dev15d - DeltaNet gated tail", Pinned graph semantics, step 6: the output
+// projection (4096 -> 2048 in the 27B-class layer).
+//
+// One CTA computes a 128 x 256 tile of y. Warp roles:
+//   warp 0   TMA producer: A (128 rows x 128 B) and B (256 rows x 128 B) tiles per stage,
+//            128-byte swizzle, into a 4-stage ring;
+//   warp 1   allocates tensor memory; lane 0 issues tcgen05.cp (scales) and tcgen05.mma;
+//   warp 2   scale loader: re-lays the row-major [rows, K/16] E4M3 scales of the stage into
+//            the 32x16-byte blocks the tensor core's scale copy reads (row r of a 128-row
+//            group at byte (r % 32) * 16 + (r / 32) * 4 + j), zero beyond K;
+//   warps 4-7 epilogue: tensor memory -> registers -> alpha * acc -> y.
+// Every barrier wait is bounded (about 1 s); an expired wait records GDN_ERR_TIMEOUT and
+// the CTA finishes without issuing more work.
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gdn {
+namespace {
+
+constexpr int BM = 128, BN = 256;
+constexpr int BK = 256;                    // FP4 values per stage per row (128 bytes)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK / 2;       // 16 KB
+constexpr int B_BYTES = BN * BK / 2;       // 32 KB
+constexpr int SFA_BYTES = (BM / 128) * (BK / 64) * 512;   // 2 KB: 4 k-blocks x one 128-row block
+constexpr int SFB_BYTES = (BN / 128) * (BK / 64) * 512;   // 4 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int THREADS = 256;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_ACC = 0;             // accumulator: 128 lanes x 256 columns fp32
+constexpr uint32_t TM_SFA = 256;           // 4 k-blocks x 4 columns
+constexpr uint32_t TM_SFB = 272;           // 4 k-blocks x 8 columns
+
+// Instruction descriptor, kind::mxf4nvf4 block-scaled: A and B E2M1 (format 1), K-major,
+// scales UE4M3, M = 128, N = 256, dense K = 64 per instruction.
+__host__ __device__ constexpr uint32_t make_idesc() {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+struct Smem {
+    uint8_t *base;
+    __device__ uint8_t *a(int s) const { return base + s * STAGE_BYTES; }
+    __device__ uint8_t *b(int s) const { return base + s * STAGE_BYTES + A_BYTES; }
+    __device__ uint8_t *sfa(int s) const { return base + s * STAGE_BYTES + A_BYTES + B_BYTES; }
+    __device__ uint8_t *sfb(int s) const { return base + s * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES; }
+};
+
+// 16 scale bytes of one row for the k-range of a stage (zero past K or past the last row).
+__device__ __forceinline__ uint4 load_scale_row(const uint8_t *sf, int row, int rows, int kblk16, int nblk16) {
+    uint4 r = make_uint4(0, 0, 0, 0);
+    if (row >= rows || kblk16 >= nblk16) return r;
+    const uint8_t *p = sf + (size_t)row * nblk16 + kblk16;
+    if (nblk16 - kblk16 >= 16 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
+        return __ldg(reinterpret_cast<const uint4 *>(p));
+    }
+    uint8_t tmp[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) tmp[j] = (kblk16 + j < nblk16) ? p[j] : (uint8_t)0;
+    r.x = tmp[0] | (tmp[1] << 8) | (tmp[2] << 16) | ((uint32_t)tmp[3] << 24);
+    r.y = tmp[4] | (tmp[5] << 8) | (tmp[6] << 16) | ((uint32_t)tmp[7] << 24);
+    r.z = tmp[8] | (tmp[9] << 8) | (tmp[10] << 16) | ((uint32_t)tmp[11] << 24);
+    r.w = tmp[12] | (tmp[13] << 8) | (tmp[14] << 16) | ((uint32_t)tmp[15] << 24);
+    return r;
+}
+
+// Scatter one row's 16 scale bytes (4 k-blocks x 4 scales) into the per-k-block scale
+// copies: k-block kb of a group of 128 rows is a 512-byte block, row r at word
+// (r % 32) * 4 + r / 32.
+__device__ __forceinline__ void put_scale_row(uint8_t *dst, int row_in_tile, int groups, uint4 v) {
+    const int grp = row_in_tile / 128, r = row_in_tile % 128;
+    uint32_t *w = reinterpret_cast<uint32_t *>(dst);
+    const int word = (r % 32) * 4 + r / 32;
+    const uint32_t vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) w[(kb * groups + grp) * 128 + word] = vals[kb];
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                  const uint8_t *__restrict__ sfa_g, const uint8_t *__restrict__ sfb_g, float alpha, int M,
+                  int N, int K, int out_bf16, void *__restrict__ y, int *status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem sm{base};
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
+    uint64_t *full = bars, *empty = bars + STAGES, *acc_full = bars + 2 * STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int tile_n = blockIdx.x, tile_m = blockIdx.y;
+    const int num_k = (K + BK - 1) / BK;
+    const int nblk16 = K / 16;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 2);   // TMA producer's expect_tx arrive + scale loader's arrive
+            mbar_init(&empty[s], 1);  // tcgen05.commit of the MMAs that read the stage
+        }
+        mbar_init(acc_full, 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int kt = 0; kt < num_k; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (kt / STAGES) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, status)) break;
+                mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+                tma_load_2d(sm.a(s), &map_a, &full[s], kt * (BK / 2), tile_m * BM);
+                tma_load_2d(sm.b(s), &map_b, &full[s], kt * (BK / 2), tile_n * BN);
+            }
+        }
+    } else if (warp == 2) {
+        for (int kt = 0; kt < num_k; ++kt) {
+            const int s = kt % STAGES;
+            const uint32_t ph = (kt / STAGES) & 1;
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            const int kb16 = kt * (BK / 16);
+            for (int r = lane; r < BM; r += 32)
+                put_scale_row(sm.sfa(s), r, BM / 128, load_scale_row(sfa_g, tile_m * BM + r, M, kb16, nblk16));
+            for (int r = lane; r < BN; r += 32)
+                put_scale_row(sm.sfb(s), r, BN / 128, load_scale_row(sfb_g, tile_n * BN + r, N, kb16, nblk16));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[s]);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = make_idesc();
+            bool ok = true;
+            for (int kt = 0; kt < num_k && ok; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (kt / STAGES) & 1;
+                if (!mbar_wait(&full[s], ph, status)) { ok = false; break; }
+                tc_fence_after();
+                // scales of the 4 k-blocks into tensor memory (one 32x128-bit block each,
+                // broadcast to the four lane quarters)
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    const uint64_t da = smem_desc(smem_u32(sm.sfa(s) + kb * 512), 0, 128, 0);
+                    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem + TM_SFA + kb * 4),
+                                 "l"(da));
+#pragma unroll
+                    for (int g = 0; g < BN / 128; ++g) {
+                        const uint64_t db = smem_desc(smem_u32(sm.sfb(s) + (kb * (BN / 128) + g) * 512), 0, 128, 0);
+                        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(
+                                         tmem + TM_SFB + kb * (BN / 32) + g * 4),
+                                     "l"(db));
+                    }
+                }
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    const uint64_t adesc = smem_desc(smem_u32(sm.a(s)) + kb * 32, 16, 1024, 2);
+                    const uint64_t bdesc = smem_desc(smem_u32(sm.b(s)) + kb * 32, 16, 1024, 2);
+                    const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\t"
+                        "setp.ne.b32 p, %4, 0;\n\t"
+                        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+                        "}" ::"r"(tmem + TM_ACC),
+                        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(tmem + TM_SFA + kb * 4),
+                        "r"(tmem + TM_SFB + kb * (BN / 32)));
+                }
+                tc_commit(&empty[s]);
+            }
+            if (ok) tc_commit(acc_full);
+        }
+    } else if (warp >= 4) {
+        const int quarter = warp - 4;  // == warp % 4: this warp's lane quarter of tensor memory
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(acc_full, 0, status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok) {
+            tc_fence_after();
+            const int row = tile_m * BM + quarter * 32 + lane;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + TM_ACC + ((uint32_t)(quarter * 32) << 16) + c0, r);
+                tmem_ld_wait();
+                const int n0 = tile_n * BN + c0;
+                if (row < M && n0 < N) {
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * alpha;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        if (n0 + j < N) {
+                            const float (&v8)[8] = *reinterpret_cast<const float(*)[8]>(&v[j]);
+                            if (out_bf16) store8<true>(y, (size_t)row * N + n0 + j, v8);
+                            else store8<false>(y, (size_t)row * N + n0 + j, v8);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side ----
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Byte-granular 2-D map over a [rows, row_bytes] matrix, box [box_rows, 128 B], 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {row_bytes, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t elem[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, elem,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, g.aq, (uint64_t)g.M, (uint64_t)g.K / 2, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&mb, g.bq, (uint64_t)g.N, (uint64_t)g.K / 2, BN)) return cudaErrorInvalidValue;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM);
+    nvfp4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, g.as, g.bs, g.alpha, g.M, g.N, g.K,
+                                                         g.out_bf16 ? 1 : 0, g.y, g.status);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -1,0 +1,133 @@
+// The gated tail before the output projection, and the NVFP4 activation encoder.
+//
+// "Red Lite dev15d - DeltaNet gated tail + Q4_K output projection", Pinned graph
+// semantics, steps 1-5: per value head of D values, RMSNorm with one shared weight,
+// times SiLU(z), flattened head-major (which is the identity on the [M, Hv, D] memory).
+// "Why Gated DeltaNet Survives 4-Bit Quantization", abstract, mechanism i: NVFP4 with
+// 16-element block scales (E4M3) over E2M1 values and an fp32 global scale.
+//
+// Both kernels are HBM-bound streams: 16-byte loads, D/8 lanes per head row, the mean of
+// squares as a lane-group shuffle reduction, and (NVFP4) the block maximum over a pair
+// of lanes, then the hardware E4M3 / E2M1 conversions.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gdn {
+
+constexpr int kTailThreads = 256;
+
+template <int D, bool IN_BF16, bool OUT_BF16, bool NVFP4>
+__global__ void __launch_bounds__(kTailThreads)
+gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
+                     const float *__restrict__ w, float eps, int64_t rows,
+                     void *__restrict__ y, float gs, uint8_t *__restrict__ xq,
+                     uint8_t *__restrict__ xs) {
+    constexpr int LANES = D / 8;                 // lanes per head row, 8 values each
+    constexpr int RPB = kTailThreads / LANES;    // head rows per block pass
+    const int lane_in_row = threadIdx.x % LANES;
+    const int col = lane_in_row * 8;
+    float wv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wv[j] = w[col + j];
+    const float inv_d = 1.0f / (float)D;
+
+    for (int64_t row = (int64_t)blockIdx.x * RPB + threadIdx.x / LANES; row - threadIdx.x / LANES < rows;
+         row += (int64_t)gridDim.x * RPB) {
+        const bool live = row < rows;
+        const size_t base = (size_t)(live ? row : 0) * D + col;
+        float ov[8], zv[8];
+        load8<IN_BF16>(o, base, ov);
+        load8<IN_BF16>(z, base, zv);
+        float ss = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss += ov[j] * ov[j];
+        ss = group_sum<LANES>(ss);
+        const float inv_rms = rsqrtf(ss * inv_d + eps);
+        float yv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) yv[j] = ov[j] * inv_rms * wv[j] * (zv[j] * sigmoid_f(zv[j]));
+        if constexpr (!NVFP4) {
+            if (live) store8<OUT_BF16>(y, base, yv);
+        } else {
+            // y as the bf16 tensor the two-call path would hand to the encoder
+#pragma unroll
+            for (int j = 0; j < 8; ++j) yv[j] = round_bf16(yv[j]);
+            float amax = amax8(yv);
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // partner lane: same block
+            float r;
+            const uint32_t sb = nvfp4_block_scale(amax, gs, r);
+            const uint32_t packed = nvfp4_pack8(yv, r);
+            if (live) {
+                reinterpret_cast<uint32_t *>(xq)[base / 8] = packed;
+                if ((lane_in_row & 1) == 0) xs[base / 16] = (uint8_t)sb;
+            }
+        }
+    }
+}
+
+template <int D, bool IN_BF16, bool OUT_BF16, bool NVFP4>
+static cudaError_t launch_tail_t(const TailArgs &t, cudaStream_t st) {
+    const int64_t rows = (int64_t)t.M * t.Hv;
+    if (rows == 0) return cudaSuccess;
+    constexpr int RPB = kTailThreads / (D / 8);
+    int64_t blocks = (rows + RPB - 1) / RPB;
+    const int64_t cap = 148 * 16;
+    if (blocks > cap) blocks = cap;
+    gated_rmsnorm_kernel<D, IN_BF16, OUT_BF16, NVFP4><<<(unsigned)blocks, kTailThreads, 0, st>>>(
+        t.o, t.z, t.w, t.eps, rows, t.y, t.gs, t.xq, t.xs);
+    return cudaGetLastError();
+}
+
+template <bool NVFP4, int D>
+static cudaError_t launch_tail_d(const TailArgs &t, cudaStream_t st) {
+    if (t.in_bf16) {
+        return t.out_bf16 ? launch_tail_t<D, true, true, NVFP4>(t, st) : launch_tail_t<D, true, false, NVFP4>(t, st);
+    }
+    return t.out_bf16 ? launch_tail_t<D, false, true, NVFP4>(t, st) : launch_tail_t<D, false, false, NVFP4>(t, st);
+}
+
+template <bool NVFP4>
+static cudaError_t launch_tail(const TailArgs &t, cudaStream_t st) {
+    switch (t.D) {
+        case 16: return launch_tail_d<NVFP4, 16>(t, st);
+        case 32: return launch_tail_d<NVFP4, 32>(t, st);
+        case 64: return launch_tail_d<NVFP4, 64>(t, st);
+        case 128: return launch_tail_d<NVFP4, 128>(t, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_gated_rmsnorm(const TailArgs &t, cudaStream_t st) { return launch_tail<false>(t, st); }
+cudaError_t launch_gated_rmsnorm_nvfp4(const TailArgs &t, cudaStream_t st) { return launch_tail<true>(t, st); }
+
+// One thread per 16-value block: two 16-byte loads (bf16) or four (fp32), one 8-byte store of
+// codes and one byte of scale.
+template <bool IN_BF16>
+__global__ void __launch_bounds__(256)
+nvfp4_quantize_kernel(const void *__restrict__ x, int64_t nblocks, float gs,
+                      uint8_t *__restrict__ xq, uint8_t *__restrict__ xs) {
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblocks;
+         blk += (int64_t)gridDim.x * blockDim.x) {
+        float lo[8], hi[8];
+        load8<IN_BF16>(x, (size_t)blk * 16, lo);
+        load8<IN_BF16>(x, (size_t)blk * 16 + 8, hi);
+        float r;
+        const uint32_t sb = nvfp4_block_scale(fmaxf(amax8(lo), amax8(hi)), gs, r);
+        uint2 packed = make_uint2(nvfp4_pack8(lo, r), nvfp4_pack8(hi, r));
+        reinterpret_cast<uint2 *>(xq)[blk] = packed;
+        xs[blk] = (uint8_t)sb;
+    }
+}
+
+cudaError_t launch_nvfp4_quantize(const void *x, bool in_bf16, int32_t M, int32_t K, float gs,
+                                  uint8_t *xq, uint8_t *xs, cudaStream_t st) {
+    const int64_t nblocks = (int64_t)M * (K / 16);
+    if (nblocks == 0) return cudaSuccess;
+    int64_t grid = (nblocks + 255) / 256;
+    if (grid > 148 * 8) grid = 148 * 8;
+    if (in_bf16) nvfp4_quantize_kernel<true><<<(unsigned)grid, 256, 0, st>>>(x, nblocks, gs, xq, xs);
+    else nvfp4_quantize_kernel<false><<<(unsigned)grid, 256, 0, st>>>(x, nblocks, gs, xq, xs);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -1,0 +1,174 @@
+/*
+ * gdn.h - C ABI of the Gated DeltaNet token mixer and its NVFP4 gated tail on B200 (sm_100a).
+ *
+ * The operations (page title, section):
+ *   [GDN]  "Why Gated DeltaNet Survives 4-Bit Quantization: NVFP4 W4A4 for the Recurrent
+ *          Half of a Hybrid 27B LLM", abstract. A fixed-size recurrent state per head; a
+ *          decay gate through softplus and an exponential and a write-strength gate through
+ *          a sigmoid (mechanism ii); each write overwrites the state along the current key
+ *          (mechanism iii); NVFP4 W4A4 with 16-element block scaling (mechanism i). The
+ *          explicit recurrence is the gated delta rule (Yang, Kautz, Hatamizadeh, "Gated
+ *          Delta Networks", ICLR 2025):
+ *              S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t q_t,
+ *              alpha_t = exp(-exp(A_log) * softplus(a_t + dt_bias)),  beta_t = sigmoid(b_t).
+ *   [TAIL] "Red Lite dev15d - DeltaNet gated tail + Q4_K output projection", section
+ *          "Pinned graph semantics", steps 1-6: per value head of 128, RMSNorm with one
+ *          shared F32 weight, times SiLU(z), flattened head-major, then the output
+ *          projection (here NVFP4 W4A4 instead of Q4_K).
+ *
+ * Conventions for every entry point:
+ *   - All pointers are DEVICE pointers owned by the caller, row-major and contiguous,
+ *     16-byte aligned (a misaligned pointer is GDN_ERR_INVALID_ARG). The library never
+ *     allocates device memory and keeps no pointer after a call returns.
+ *   - Work is enqueued on `stream` and the call returns without synchronising. Arguments
+ *     are checked on the host before anything is launched; on any error nothing runs.
+ *   - GDN_ERR_CUDA means a launch failed (cudaGetLastError after the launch).
+ *   - Kernels that wait on barriers bound every wait; on expiry they record
+ *     GDN_ERR_TIMEOUT in a device status word and finish without deadlocking. Read (and
+ *     clear) it with gdn_get_device_status().
+ *   - Multi-head layouts: q, k [T, Hk, Dk]; v, o, z [T, Hv, Dv]; value head h reads key
+ *     head h / (Hv / Hk) (contiguous groups). The state is [.., Hv, Dv, Dk] fp32, key index
+ *     contiguous, so that o = S q.
+ */
+#ifndef GDN_B200_H
+#define GDN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *gdn_stream_t; /* the same handle as cudaStream_t */
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or dtype */
+    GDN_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. head size) */
+    GDN_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
+    GDN_ERR_TIMEOUT = 4,     /* a bounded device-side wait expired */
+    GDN_ERR_WORKSPACE = 5    /* workspace missing or too small */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
+
+/* ------------------------------------------------------------------ prefill ----
+ * [GDN]: the gated delta rule over whole sequences, o_t = S_t q_t for every token.
+ *
+ * q, k        [T, Hk, Dk] in `in_dtype`;  v [T, Hv, Dv] in `in_dtype`
+ * a, b        [T, Hv] fp32 gate pre-activations; A_log, dt_bias [Hv] fp32
+ * cu_seqlens  device int32 [num_seqs + 1], cumulative token offsets of the packed
+ *             sequences (cu_seqlens[0] = 0, cu_seqlens[num_seqs] = T); NULL means one
+ *             sequence of T tokens (then num_seqs must be 1). Every sequence starts from
+ *             its own initial state.
+ * scale       multiplies q after normalisation (1.0 = the formula as written)
+ * qk_l2norm   non-zero: q and k are L2-normalised per head inside the path,
+ *             x * (sum x^2 + 1e-6)^-1/2, before use (the delta rule wants unit keys)
+ * initial_state  [num_seqs, Hv, Dv, Dk] fp32, or NULL for zero states
+ * final_state    [num_seqs, Hv, Dv, Dk] fp32 output, or NULL; may alias initial_state
+ * o           [T, Hv, Dv] in `out_dtype`
+ * workspace   device scratch of at least gdn_prefill_workspace_bytes(...) bytes (may be
+ *             NULL when that is 0).
+ * Supported: Dk == Dv in {16, 32, 64, 128}; Hv % Hk == 0; T >= 0 (T == 0 only writes
+ * final_state = initial_state). Dk == Dv == 128 with bf16 inputs runs the tensor-core
+ * chunked kernel (64-token chunks; operands staged in fp16, so |q|, |k|, |v| and the
+ * state must stay below 6.5e4); other sizes run the CUDA-core recurrent kernel.
+ */
+GDN_API gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v,
+                               const float *a, const float *b,
+                               const float *A_log, const float *dt_bias,
+                               const int32_t *cu_seqlens, int32_t num_seqs,
+                               int32_t T, int32_t Hk, int32_t Hv, int32_t Dk, int32_t Dv,
+                               float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                               const float *initial_state, float *final_state,
+                               void *o, gdn_dtype out_dtype,
+                               void *workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/* Scratch bytes gdn_prefill_chunked needs for these sizes (0 when it needs none). */
+GDN_API size_t gdn_prefill_workspace_bytes(int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv,
+                                   int32_t Dk, int32_t Dv);
+
+/* ------------------------------------------------------------------- decode ----
+ * [GDN]: one token per sequence; the state is read once and written once, in place.
+ * q, k [B, Hk, Dk], v [B, Hv, Dv] in `in_dtype`; a, b [B, Hv] fp32; A_log, dt_bias [Hv];
+ * state [B, Hv, Dv, Dk] fp32, updated in place; o [B, Hv, Dv] in `out_dtype`.
+ * Supported: Dk == Dv in {16, 32, 64, 128}, Hv % Hk == 0, B >= 0.
+ */
+GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
+                           const float *a, const float *b,
+                           const float *A_log, const float *dt_bias,
+                           int32_t B, int32_t Hk, int32_t Hv, int32_t Dk, int32_t Dv,
+                           float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                           float *state, void *o, gdn_dtype out_dtype, gdn_stream_t stream);
+
+/* ------------------------------------------------------------ gated RMSNorm ----
+ * [TAIL] steps 1-5: y[m, h*Dv + i] = o[m,h,i] / sqrt(mean_i o[m,h,:]^2 + eps) * w[i]
+ *                                     * z[m,h,i] * sigmoid(z[m,h,i]).
+ * o, z [M, Hv, Dv] in `in_dtype`; weight [Dv] fp32, shared by all heads; y [M, Hv*Dv]
+ * in `out_dtype`. Supported: Dv in {16, 32, 64, 128}; M >= 0.
+ */
+GDN_API gdn_status gdn_gated_rmsnorm_silu(const void *o, const void *z, const float *weight, float eps,
+                                  int32_t M, int32_t Hv, int32_t Dv, gdn_dtype in_dtype,
+                                  void *y, gdn_dtype out_dtype, gdn_stream_t stream);
+
+/* The same tail with its NVFP4 activation quantisation fused in: y is formed as above,
+ * rounded to bf16, and encoded exactly as nvfp4_quantize_act would encode that bf16
+ * tensor (so the two-call and fused paths agree bit for bit). K = Hv * Dv.
+ * xq [M, K/2], xs [M, K/16]: see nvfp4_quantize_act. */
+GDN_API gdn_status gdn_gated_rmsnorm_silu_nvfp4(const void *o, const void *z, const float *weight,
+                                        float eps, int32_t M, int32_t Hv, int32_t Dv,
+                                        gdn_dtype in_dtype, float global_scale,
+                                        uint8_t *xq, uint8_t *xs, gdn_stream_t stream);
+
+/* ------------------------------------------------------------ NVFP4 encode ----
+ * [GDN] mechanism i: NVFP4 with 16-element blocks. For each 16 consecutive values of a
+ * row of x [M, K] (in `in_dtype`), in fp32 with this order of operations:
+ *   amax = max |x_j|;  s = (amax / 6) * global_scale;  sb = E4M3(s) (nearest, ties to
+ *   even, saturating at 448);  r = global_scale / sb (0 when sb == 0);
+ *   code_j = E2M1(x_j * r) (nearest, ties to even, saturating at 6, sign kept).
+ * xq [M, K/2] uint8: element 2j in the low nibble of byte j, 2j+1 in the high nibble.
+ * xs [M, K/16] uint8: the E4M3 block scales, row-major.
+ * global_scale is the caller's calibrated encode scale, typically 448 * 6 / amax(tensor);
+ * it must be finite and > 0. Decoded value: E2M1(code) * E4M3(sb) / global_scale.
+ * Supported: K % 32 == 0, M >= 0.
+ */
+GDN_API gdn_status nvfp4_quantize_act(const void *x, gdn_dtype in_dtype, int32_t M, int32_t K,
+                              float global_scale, uint8_t *xq, uint8_t *xs, gdn_stream_t stream);
+
+/* ------------------------------------------------------------ NVFP4 GEMM ----
+ * [GDN] "NVFP4 W4A4 on all linear layers"; [TAIL] step 6 (ssm_out, 4096 -> 2048):
+ *   y[m, n] = alpha * sum_k E2M1(a)[m,k] E4M3(as)[m,k/16] E2M1(b)[n,k] E4M3(bs)[n,k/16]
+ * with fp32 accumulation on the block-scaled FP4 tensor cores.
+ * aq [M, K/2], as [M, K/16]: the activations as nvfp4_quantize_act writes them;
+ * bq [N, K/2], bs [N, K/16]: the weight [N, K] (K contiguous), quantised the same way;
+ * alpha = 1 / (global_scale_a * global_scale_b); y [M, N] in `out_dtype`.
+ * Supported: K % 32 == 0, N % 16 == 0, M >= 0 (K is zero-padded to the 256-value
+ * tile inside the kernel; ragged M and N tiles are masked).
+ */
+GDN_API gdn_status nvfp4_gemm(const uint8_t *aq, const uint8_t *as, const uint8_t *bq, const uint8_t *bs,
+                      float alpha, int32_t M, int32_t N, int32_t K, gdn_dtype out_dtype, void *y,
+                      gdn_stream_t stream);
+
+/* ----------------------------------------------------------------- helpers ---- */
+
+/* Synchronises `stream`, returns the device status word (GDN_OK or GDN_ERR_TIMEOUT) that
+ * kernels set on an expired bounded wait, and clears it. */
+GDN_API gdn_status gdn_get_device_status(gdn_stream_t stream);
+
+/* Static description of a status code. */
+GDN_API const char *gdn_status_string(gdn_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+GDN_API int32_t gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN_B200_H */

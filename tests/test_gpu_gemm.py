@@ -1,0 +1,78 @@
+"""Parity of the block-scaled NVFP4 GEMM with the oracle (fp64 product of the dequantised
+operands, both sides fed the same oracle-encoded codes and scales): within the stated
+1e-2 max relative error, for ragged M, N and K tiles, the tiny K = 32 case, and the full
+output-projection sizes (sampled rows)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from helpers import TOL_GEMM, dev, rel_err, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def g():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    import gated_deltanet_03_b200 as lib
+    return lib
+
+
+def _operands(M, N, K, seed):
+    rng = np.random.default_rng(seed)
+    A = workloads.activations(M, K, seed=seed)
+    W = workloads.round_bf16(rng.standard_normal((N, K)).astype(np.float32) * 0.02)
+    gsa = np.float32(448.0 * 6.0 / np.abs(A).max())
+    gsw = np.float32(448.0 * 6.0 / np.abs(W).max())
+    aq, as_ = oracle.nvfp4_quantize(A, gsa)
+    wq, ws = oracle.nvfp4_quantize(W, gsw)
+    return aq, as_, gsa, wq, ws, gsw
+
+
+def _gpu(g, aq, as_, wq, ws, alpha, out_dtype):
+    u8 = torch.uint8
+    y = g.nvfp4_gemm(dev(aq, u8), dev(as_, u8), dev(wq, u8), dev(ws, u8), alpha, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert g.gdn_get_device_status() == 0
+    return to_np(y)
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 16, 32), (128, 256, 256), (300, 272, 512), (1, 16, 96),
+                                   (129, 512, 2048), (4096, 1024, 2048)])
+def test_gemm_matches_oracle(g, M, N, K):
+    aq, as_, gsa, wq, ws, gsw = _operands(M, N, K, seed=M + N + K)
+    ref = oracle.nvfp4_gemm(aq, as_, gsa, wq, ws, gsw)
+    alpha = float(np.float32(1.0) / (np.float32(gsa) * np.float32(gsw)))
+    y32 = _gpu(g, aq, as_, wq, ws, alpha, torch.float32)
+    assert rel_err(y32, ref) <= TOL_GEMM, rel_err(y32, ref)
+    y16 = _gpu(g, aq, as_, wq, ws, alpha, torch.bfloat16)
+    assert rel_err(y16, ref) <= TOL_GEMM
+
+
+def test_gemm_exact_on_grid_values(g):
+    """Codes whose products sum exactly in fp32: every element of y is exact."""
+    rng = np.random.default_rng(5)
+    M, N, K = 128, 256, 256
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    A = grid[rng.integers(0, 8, (M, K))] * np.where(rng.random((M, K)) < .5, -1, 1).astype(np.float32)
+    B = grid[rng.integers(0, 8, (N, K))] * np.where(rng.random((N, K)) < .5, -1, 1).astype(np.float32)
+    A.reshape(M, K // 16, 16)[:, :, 0] = 6.0
+    B.reshape(N, K // 16, 16)[:, :, 0] = 6.0
+    aq, as_ = oracle.nvfp4_quantize(A, 1.0)
+    bq, bs = oracle.nvfp4_quantize(B, 1.0)
+    y = _gpu(g, aq, as_, bq, bs, 1.0, torch.float32)
+    np.testing.assert_array_equal(y, A.astype(np.float64) @ B.T.astype(np.float64))
+
+
+@pytest.mark.parametrize("M,N,K", [(32768, 2048, 4096), (256, 2048, 4096)])
+def test_gemm_full_size_sampled_rows(g, M, N, K):
+    aq, as_, gsa, wq, ws, gsw = _operands(M, N, K, seed=11)
+    alpha = float(np.float32(1.0) / (np.float32(gsa) * np.float32(gsw)))
+    y = _gpu(g, aq, as_, wq, ws, alpha, torch.bfloat16)
+    rows = np.random.default_rng(1).choice(M, size=min(M, 256), replace=False)
+    rows = np.concatenate([rows, [0, M - 1]])
+    ref = oracle.nvfp4_gemm(aq, as_, gsa, wq, ws, gsw, rows=rows)
+    assert rel_err(y[rows], ref) <= TOL_GEMM
