@@ -308,6 +308,61 @@ def run_gpu(args):
     print(json.dumps(out))
 
 
+def run_only(args):
+    """One kernel alone, `warmup` + `steps` launches, CUDA-event timed (L2 flushed between)."""
+    import torch
+
+    import gated_deltanet_03_b200 as g
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    bf, f32 = torch.bfloat16, torch.float32
+    names = {wl.name: wl for wl in workloads.WORKLOADS}
+    w = names[args.workload] if args.workload else (workloads.DECODE_B256 if args.only == "decode"
+                                                    else workloads.PREFILL_1K)
+    x = workloads.generate(w)
+
+    def up(a, dt):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+
+    q, k, v, z = up(x["q"], bf), up(x["k"], bf), up(x["v"], bf), up(x["z"], bf)
+    a, b = up(x["a"], f32), up(x["b"], f32)
+    A_log, dt_bias, nw = up(x["A_log"], f32), up(x["dt_bias"], f32), up(x["norm_weight"], f32)
+    cu = up(x["cu_seqlens"], torch.int32) if w.num_seqs > 1 else None
+    S0 = None if x["initial_state"] is None else up(x["initial_state"], f32)
+    o = torch.empty((w.T, w.Hv, w.D), dtype=bf, device=dev)
+    S = torch.empty((w.num_seqs, w.Hv, w.D, w.D), dtype=f32, device=dev)
+    W = up(x["proj_weight"], bf)
+    wq, ws = g.nvfp4_quantize_act(W, 1.0)
+    xq = torch.empty((w.T, w.K // 2), dtype=torch.uint8, device=dev)
+    xs = torch.empty((w.T, w.K // 16), dtype=torch.uint8, device=dev)
+    Y = torch.empty((w.T, w.n_out), dtype=bf, device=dev)
+    g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=cu, initial_state=S0, final_state=S, o=o)
+    g.gdn_gated_rmsnorm_silu_nvfp4(o, z, nw, 1.0, xq=xq, xs=xs)
+    fn = {
+        "scan": lambda: g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=cu, initial_state=S0,
+                                              final_state=S, o=o),
+        "tail": lambda: g.gdn_gated_rmsnorm_silu_nvfp4(o, z, nw, 1.0, xq=xq, xs=xs),
+        "gemm": lambda: g.nvfp4_gemm(xq, xs, wq, ws, 1.0, y=Y),
+        "decode": lambda: g.gdn_decode_step(q, k, v, a, b, A_log, dt_bias, S0, o=o),
+    }[args.only]
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=f32, device=dev)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    assert g.gdn_get_device_status() == 0
+    print(json.dumps({"only": args.only, "workload": w.name, "ms_median": statistics.median(times),
+                      "ms_mean": statistics.mean(times), "steps": args.steps}))
+
+
 # ----------------------------------------------------------------- CPU arm ----
 
 def cpu_pass(w, x, units=None):
@@ -369,11 +424,16 @@ def main():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    p.add_argument("--only", choices=["scan", "tail", "gemm", "decode"],
+                   help="time one kernel alone on its workload (for profiling); prints one JSON line")
+    p.add_argument("--workload", default=None, help="workload name for --only scan (default: 1024-wide prefill)")
     args = p.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.only:
+        run_only(args)
     else:
         run_gpu(args)
 

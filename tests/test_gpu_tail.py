@@ -54,10 +54,10 @@ def test_nvfp4_quantize_bit_exact(g, M, K, io):
 
 def test_e2m1_hardware_rounding_every_bf16_value(g):
     """Blocks [6, v1..v15] with global scale 1: the block scale is exactly 1 (E4M3 0x38), so
-    each code is E2M1(v) of the value itself. Every bf16 value with |v| <= 6.5 is covered."""
+    each code is E2M1(v) of the value itself. Every bf16 value with |v| <= 6 is covered."""
     bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
     vals = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
-    vals = vals[np.isfinite(vals) & (np.abs(vals) <= 6.5)]
+    vals = vals[np.isfinite(vals) & (np.abs(vals) <= 6.0)]
     vals = np.concatenate([vals, np.zeros((-len(vals)) % 15, np.float32)])
     blocks = np.concatenate([np.full((len(vals) // 15, 1), 6.0, np.float32), vals.reshape(-1, 15)], axis=1)
     pad = (-blocks.shape[0]) % 2
