@@ -9,9 +9,10 @@
 //   warp 0   TMA producer: A (128 rows x 128 B) and B (256 rows x 128 B) tiles per stage,
 //            128-byte swizzle, into a 4-stage ring;
 //   warp 1   allocates tensor memory; lane 0 issues tcgen05.cp (scales) and tcgen05.mma;
-//   warp 2   scale loader: re-lays the row-major [rows, K/16] E4M3 scales of the stage into
-//            the 32x16-byte blocks the tensor core's scale copy reads (row r of a 128-row
-//            group at byte (r % 32) * 16 + (r / 32) * 4 + j), zero beyond K;
+//   warp 2   scale re-layout: the stage's row-major [rows, 16 B] E4M3 scales (TMA-loaded with
+//            the tiles when K % 256 == 0, else gathered with plain loads and zero past K) are
+//            permuted in place into the 32x16-byte blocks the tensor core's scale copy reads
+//            (row r of a 128-row group at byte (r % 32) * 16 + (r / 32) * 4 + j);
 //   warps 4-7 epilogue: tensor memory -> registers -> alpha * acc -> y.
 // Every barrier wait is bounded (about 1 s); an expired wait records GDN_ERR_TIMEOUT and
 // the CTA finishes without issuing more work.
@@ -82,16 +83,42 @@ __device__ __forceinline__ void put_scale_row(uint8_t *dst, int row_in_tile, int
     for (int kb = 0; kb < 4; ++kb) w[(kb * groups + grp) * 128 + word] = vals[kb];
 }
 
+// In-place permutation of one stage's scales from [rows][16 B] (row-major, as loaded) into
+// the per-k-block 512-byte blocks: every lane loads all its words first, then stores.
+__device__ __forceinline__ void relayout_scales(uint8_t *sf, int rows, int lane) {
+    uint32_t *w = reinterpret_cast<uint32_t *>(sf);
+    const int groups = rows / 128;
+    uint32_t v[BN / 32][4];
+#pragma unroll
+    for (int i = 0; i < BN / 32; ++i) {
+        if (i < rows / 32) {
+            const uint4 x = reinterpret_cast<const uint4 *>(sf)[i * 32 + lane];
+            v[i][0] = x.x; v[i][1] = x.y; v[i][2] = x.z; v[i][3] = x.w;
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < BN / 32; ++i) {
+        if (i < rows / 32) {
+            const int r = i * 32 + lane, grp = r / 128, rr = r % 128;
+            const int word = (rr % 32) * 4 + rr / 32;
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) w[(kb * groups + grp) * 128 + word] = v[i][kb];
+        }
+    }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                  const uint8_t *__restrict__ sfa_g, const uint8_t *__restrict__ sfb_g, float alpha, int M,
-                  int N, int K, int out_bf16, void *__restrict__ y, int *status) {
+                  const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
+                  int sf_tma, const uint8_t *__restrict__ sfa_g, const uint8_t *__restrict__ sfb_g, float alpha,
+                  int M, int N, int K, int out_bf16, void *__restrict__ y, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Smem sm{base};
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
-    uint64_t *full = bars, *empty = bars + STAGES, *acc_full = bars + 2 * STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 1);
+    uint64_t *full = bars, *empty = bars + STAGES, *sf_ready = bars + 2 * STAGES, *acc_full = bars + 3 * STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int tile_n = blockIdx.x, tile_m = blockIdx.y;
@@ -100,8 +127,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 2);   // TMA producer's expect_tx arrive + scale loader's arrive
-            mbar_init(&empty[s], 1);  // tcgen05.commit of the MMAs that read the stage
+            mbar_init(&full[s], 1);      // TMA producer's expect_tx arrive
+            mbar_init(&empty[s], 1);     // tcgen05.commit of the MMAs that read the stage
+            mbar_init(&sf_ready[s], 1);  // scale warp: the stage's scales are in place
         }
         mbar_init(acc_full, 1);
         fence_barrier_init();
@@ -123,9 +151,13 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 const int s = kt % STAGES;
                 const uint32_t ph = (kt / STAGES) & 1;
                 if (!mbar_wait(&empty[s], ph ^ 1, status)) break;
-                mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+                mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + (sf_tma ? SFA_BYTES + SFB_BYTES : 0));
                 tma_load_2d(sm.a(s), &map_a, &full[s], kt * (BK / 2), tile_m * BM);
                 tma_load_2d(sm.b(s), &map_b, &full[s], kt * (BK / 2), tile_n * BN);
+                if (sf_tma) {
+                    tma_load_2d(sm.sfa(s), &map_sfa, &full[s], kt * (BK / 16), tile_m * BM);
+                    tma_load_2d(sm.sfb(s), &map_sfb, &full[s], kt * (BK / 16), tile_n * BN);
+                }
             }
         }
     } else if (warp == 2) {
@@ -133,17 +165,26 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             const int s = kt % STAGES;
             const uint32_t ph = (kt / STAGES) & 1;
             bool ok = true;
-            if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, status);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            const int kb16 = kt * (BK / 16);
-            for (int r = lane; r < BM; r += 32)
-                put_scale_row(sm.sfa(s), r, BM / 128, load_scale_row(sfa_g, tile_m * BM + r, M, kb16, nblk16));
-            for (int r = lane; r < BN; r += 32)
-                put_scale_row(sm.sfb(s), r, BN / 128, load_scale_row(sfb_g, tile_n * BN + r, N, kb16, nblk16));
+            if (sf_tma) {
+                // scales arrive with the tiles; permute them in place once they land
+                if (lane == 0) ok = mbar_wait(&full[s], ph, status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                relayout_scales(sm.sfa(s), BM, lane);
+                relayout_scales(sm.sfb(s), BN, lane);
+            } else {
+                if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                const int kb16 = kt * (BK / 16);
+                for (int r = lane; r < BM; r += 32)
+                    put_scale_row(sm.sfa(s), r, BM / 128, load_scale_row(sfa_g, tile_m * BM + r, M, kb16, nblk16));
+                for (int r = lane; r < BN; r += 32)
+                    put_scale_row(sm.sfb(s), r, BN / 128, load_scale_row(sfb_g, tile_n * BN + r, N, kb16, nblk16));
+            }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&full[s]);
+            if (lane == 0) mbar_arrive(&sf_ready[s]);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -152,7 +193,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             for (int kt = 0; kt < num_k && ok; ++kt) {
                 const int s = kt % STAGES;
                 const uint32_t ph = (kt / STAGES) & 1;
-                if (!mbar_wait(&full[s], ph, status)) { ok = false; break; }
+                if (!mbar_wait(&full[s], ph, status) || !mbar_wait(&sf_ready[s], ph, status)) { ok = false; break; }
                 tc_fence_after();
                 // scales of the 4 k-blocks into tensor memory (one 32x128-bit block each,
                 // broadcast to the four lane quarters)
@@ -244,25 +285,36 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Byte-granular 2-D map over a [rows, row_bytes] matrix, box [box_rows, 128 B], 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+// Byte-granular 2-D map over a [rows, row_bytes] matrix, box [box_rows, box_bytes].
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t row_bytes, uint32_t box_rows,
+              uint32_t box_bytes = 128, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {row_bytes, rows};
     cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t box[2] = {box_bytes, box_rows};
     cuuint32_t elem[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, elem,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
 cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, msa, msb;
     if (!make_map(&ma, g.aq, (uint64_t)g.M, (uint64_t)g.K / 2, BM)) return cudaErrorInvalidValue;
     if (!make_map(&mb, g.bq, (uint64_t)g.N, (uint64_t)g.K / 2, BN)) return cudaErrorInvalidValue;
+    // scales by TMA when their rows are whole 16-byte multiples per stage and 16-byte aligned
+    const bool sf_tma = (g.K % BK == 0) && ((reinterpret_cast<uintptr_t>(g.as) | reinterpret_cast<uintptr_t>(g.bs)) & 15u) == 0;
+    if (sf_tma) {
+        if (!make_map(&msa, g.as, (uint64_t)g.M, (uint64_t)g.K / 16, BM, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !make_map(&msb, g.bs, (uint64_t)g.N, (uint64_t)g.K / 16, BN, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    } else {
+        msa = ma;   // unused
+        msb = mb;
+    }
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
@@ -270,8 +322,8 @@ cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
         attr_set = true;
     }
     dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM);
-    nvfp4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, g.as, g.bs, g.alpha, g.M, g.N, g.K,
-                                                         g.out_bf16 ? 1 : 0, g.y, g.status);
+    nvfp4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, msa, msb, sf_tma ? 1 : 0, g.as, g.bs, g.alpha, g.M,
+                                                         g.N, g.K, g.out_bf16 ? 1 : 0, g.y, g.status);
     return cudaGetLastError();
 }
 
