@@ -65,8 +65,9 @@ gdn_status gdn_get_device_status(gdn_stream_t stream) {
 
 size_t gdn_prefill_workspace_bytes(int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv, int32_t Dk,
                                    int32_t Dv) {
-    (void)T; (void)num_seqs; (void)Hk; (void)Hv; (void)Dk; (void)Dv;
-    return 0;
+    (void)Hk;
+    if (T <= 0 || num_seqs < 1 || Hv < 1 || Dk != 128 || Dv != 128) return 0;
+    return gdn::chunked_workspace_bytes(T, num_seqs, Hv);
 }
 
 gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v, const float *a, const float *b,
@@ -76,7 +77,6 @@ gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v, cons
                                const float *initial_state, float *final_state, void *o,
                                gdn_dtype out_dtype, void *workspace, size_t workspace_bytes,
                                gdn_stream_t stream) {
-    (void)workspace; (void)workspace_bytes;
     if (T < 0 || num_seqs < 1 || Hk < 1 || Hv < 1 || Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
     if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
     if (!cu_seqlens && num_seqs != 1) return GDN_ERR_INVALID_ARG;
@@ -92,8 +92,10 @@ gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v, cons
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (Dk == 128 && in_dtype == GDN_BF16 && T > 0) {
+        const size_t need = gdn::chunked_workspace_bytes(T, num_seqs, Hv);
+        if (!workspace || workspace_bytes < need || !aligned16(workspace)) return GDN_ERR_WORKSPACE;
         gdn::ChunkedArgs c{q, k, v, a, b, A_log, dt_bias, cu_seqlens, T, num_seqs, Hk, Hv, scale, qk_l2norm,
-                           out_dtype == GDN_BF16, initial_state, final_state, o, status_ptr()};
+                           out_dtype == GDN_BF16, initial_state, final_state, o, workspace, status_ptr()};
         cudaError_t e = gdn::launch_chunked(c, st);
         if (e != cudaErrorNotSupported) return launched(e);
     }

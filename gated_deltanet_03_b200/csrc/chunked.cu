@@ -1,4 +1,6 @@
-// Chunked gated delta-rule prefill on the fifth-generation tensor cores (tcgen05, TMEM).
+// Chunked gated delta-rule prefill on the fifth-generation tensor cores (tcgen05, TMEM),
+// as two kernels: a prep kernel that is parallel over (chunk, value head) and a chain
+// kernel that is sequential over the chunks of each (sequence, value head).
 //
 // "Why Gated DeltaNet Survives 4-Bit Quantization" (abstract, mechanisms ii-iii) describes
 // the recurrence; here it is evaluated 64 tokens at a time in the WY / UT form, which is
@@ -8,63 +10,51 @@
 //   W = T diag(beta gamma) K,   U~ = T diag(beta) V,     U = U~ - W S0^T,
 //   O = diag(gamma) Q S0^T + (Q K^T o Gamma) U,          Gamma_rs = exp(G_r - G_s), s <= r,
 //   S_C = gamma_C S0 + U^T diag(gamma_C / gamma) K.
+// W, U~ and P = (Q K^T o Gamma) do not depend on the state: the prep kernel computes them
+// for every chunk at once and writes them to the caller's workspace; the chain kernel then
+// only runs the four state-dependent products per chunk.
+//
 // The L2 norms of q and k never touch an MMA operand: raw bf16 inputs (exact in fp16) feed
 // the tensor cores and 1/|k|, scale/|q| enter as diagonal factors of the derived operands.
-// Derived operands (T', T'', W, U, P, S0) are staged in fp16 (11-bit significand) with fp32
-// accumulation in tensor memory; the state itself stays fp32 in registers.
+// Derived operands (T', T'', W, U~, U, P, S0) are staged in fp16 (11-bit significand) with
+// fp32 accumulation in tensor memory; the state itself stays fp32 in registers.
 //
-// Everything is computed transposed so that every MMA has M = 128 (the value or key index
-// on the tensor-memory lanes):
-//   MMA1  D1[128 x 64]  = [K; Q] K^T                      (K K^T rows 0-63, Q K^T rows 64-127)
-//   MMA2  D2 = W^T      = K^T T'^T      T' = T diag(beta gamma / |k|)
-//   MMA3  D3 = U~^T     = V^T T''^T     T'' = T diag(beta)
-//   MMA4  D3 -= S0 W^T                  (D3 becomes U^T)
-//   MMA5  D5 = S0 Q^T
-//   MMA6  D6 = U^T P^T                  P = Q K^T o Gamma / (|q| |k|) * scale
-//   MMA7  D7 = U_S^T K                  U_S = U diag(gamma_C / gamma / |k|)
+// Every MMA has M = 128 by working transposed (value or key index on the TMEM lanes):
+//   prep   MMA1  D1[128 x 64] = [K; Q] K^T        (K K^T rows 0-63, Q K^T rows 64-127)
+//          MMA2  D2 = W^T  = K^T T'^T               T'  = T diag(beta gamma / |k|)
+//          MMA3  D3 = U~^T = V^T T''^T              T'' = T diag(beta)
+//   chain  MMA4  D4 = S0 W^T      -> U^T = U~^T - D4
+//          MMA5  D5 = S0 Q^T
+//          MMA7  D7 = U_S^T K     U_S = U diag(gamma_C / gamma / |k|)
+//          MMA6  D6 = U^T P^T     P = Q K^T o Gamma / (|q| |k|) * scale
 // then o^T = D5 diag(gamma * scale / |q|) + D6 and S <- gamma_C S + D7.
 //
-// One CTA (256 threads) owns one (sequence, value head) and walks its chunks in order; the
-// next chunk's q/k/v tiles stream in by TMA (3-D maps over [T, heads, 128]) while the
-// current one is processed. Tensor memory: 448 of 512 columns.
+// Workspace: one 41 KB item per (value head, chunk slot): the W operand image (fp16,
+// [key j][token s], 128-byte swizzled rows), U~ (fp16, [token s][value i]), the P operand
+// image (fp16, [r][s] swizzled) and fp32 vectors (gamma_r scale/|q_r|, gamma_C/gamma_s/|k_s|,
+// gamma_C). Chunk c of sequence n uses slot cu_seqlens[n] / 64 + n + c, so slots never
+// collide and T / 64 + num_seqs slots per head suffice.
 #include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
 
 namespace gdn {
+
+constexpr int kChunk = 64;
+constexpr int kWsItem = 41984;
+constexpr int kWsW = 0, kWsU = 16384, kWsP = 32768, kWsVec = 40960;
+
+size_t chunked_workspace_bytes(int T, int num_seqs, int Hv) {
+    return (size_t)Hv * (size_t)(T / kChunk + num_seqs) * kWsItem;
+}
+
 namespace {
 
-constexpr int C = 64;          // chunk length
+constexpr int C = kChunk;      // chunk length
 constexpr int D = 128;         // head size
-constexpr int NT = 256;        // threads
-
-// shared-memory map (bytes); 1024-byte aligned tiles for the 128-byte swizzle
-constexpr int TILE = C * 128;                  // 64 rows x 128 B (one half of a 64 x 128 fp16/bf16 tile)
-constexpr int OFF_KQ = 0;                      // [K_lo][Q_lo][K_hi][Q_hi] fp16 working tiles
-constexpr int OFF_V = OFF_KQ + 4 * TILE;       // [V_lo][V_hi]
-constexpr int OFF_STG = OFF_V + 2 * TILE;      // bf16 staging of the next chunk, same 6-tile order
-constexpr int OFF_S = OFF_STG + 6 * TILE;      // S0 fp16, [S_lo: 128 rows x 64][S_hi]   (32 KB)
-constexpr int OFF_W = OFF_S + 2 * 2 * TILE;    // W as [j: 128 rows][s: 64] fp16        (16 KB)
-constexpr int OFF_P = OFF_W + 2 * TILE;        // P [r: 64][s: 64] fp16                 (8 KB)
-constexpr int OFF_TP = OFF_P + TILE;           // T'  [s][r] fp16                       (8 KB)
-constexpr int OFF_TPP = OFF_TP + TILE;         // T'' [s][r] fp16                       (8 KB)
-constexpr int OFF_U = OFF_TPP + TILE;          // U_A, U_S [i: 128][s: 64] fp16          (32 KB)
-// fp32 scratch of the (I + A)^-1 step, in areas that are dead while it runs:
-constexpr int OFF_AF = OFF_U;                  //   A [64][65] and X [3][256] in the U area
-constexpr int OFF_XF = OFF_U + 64 * 65 * 4;
-constexpr int OFF_TF = OFF_W;                  //   T [64][64] in the W area
-constexpr int OFF_VEC = OFF_U + 4 * TILE;      // per-chunk vectors
-constexpr int VEC_FLOATS = 8 * 64;
-constexpr int OFF_BAR = OFF_VEC + VEC_FLOATS * 4;
-constexpr int SMEM_USED = OFF_BAR + 64;
-constexpr int SMEM_BYTES = SMEM_USED + 1024;
-static_assert(64 * 65 * 4 + 3 * 256 * 4 <= 4 * TILE, "A and X fit in the U area");
-static_assert(64 * 64 * 4 <= 2 * TILE, "T fits in the W area");
-static_assert(SMEM_BYTES <= 232448, "shared memory per block");
-
-// tensor-memory columns
-constexpr uint32_t TM_D1 = 0, TM_D2 = 64, TM_D3 = 128, TM_D5 = 192, TM_D6 = 256, TM_D7 = 320;
+constexpr int NT = 256;        // threads per CTA
+constexpr int TILE = C * 128;  // 64 rows x 128 B: one half (64 columns) of a 64 x 128 16-bit tile
 
 // kind::f16 instruction descriptor: fp16 A/B, fp32 accumulate, M = 128.
 __host__ __device__ constexpr uint32_t idesc_f16(int N, bool a_mn, bool b_mn, bool neg_a) {
@@ -109,30 +99,339 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 struct Maps {
     CUtensorMap q, k, v;
 };
 
-__global__ void __launch_bounds__(NT, 1)
-gdn_chunked_kernel(const __grid_constant__ Maps maps, const float *__restrict__ ga, const float *__restrict__ gb,
-                   const float *__restrict__ A_log, const float *__restrict__ dt_bias,
-                   const int32_t *__restrict__ cu_seqlens, int32_t T, int32_t Hk, int32_t Hv, float scale,
-                   int32_t l2norm, int32_t out_bf16, const float *S0g, float *S_out, void *__restrict__ o,
-                   int *status) {
+// Convert a staged bf16 tile region to fp16 in place, 16 bytes per step. For the [K; Q]
+// area (4 tiles, rows of 128 B) also returns the thread's share of its row's sum of squares.
+__device__ __forceinline__ float convert16(uint8_t *p) {
+    uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    float f[8], ss = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float2 x = __bfloat1622float2(b2[e]);
+        f[2 * e] = x.x;
+        f[2 * e + 1] = x.y;
+        ss += x.x * x.x + x.y * x.y;
+    }
+    st_h8(p, f);
+    return ss;
+}
+
+// Chunk location: slot `id` of the workspace belongs to sequence n (the last n whose first
+// slot cu[n] / 64 + n is <= id) and is its chunk id - (cu[n] / 64 + n).
+__device__ __forceinline__ void locate(int id, const int32_t *cu, int num_seqs, int T, int &n, int &t_begin,
+                                       int &t_end) {
+    n = 0;
+    t_begin = 0;
+    t_end = T;
+    if (cu) {
+        int lo = 0, hi = num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (cu[mid] / C + mid <= id) lo = mid;
+            else hi = mid - 1;
+        }
+        n = lo;
+        t_begin = cu[n];
+        t_end = cu[n + 1];
+    }
+}
+
+// ===================================================================================
+// Prep kernel: one CTA per (chunk slot, value head); two CTAs per SM.
+// ===================================================================================
+constexpr int P_OFF_KQ = 0;                     // [K_lo][Q_lo][K_hi][Q_hi], bf16 -> fp16 in place
+constexpr int P_OFF_V = 4 * TILE;               // [V_lo][V_hi]
+constexpr int P_OFF_TP = 6 * TILE;              // T'  [s][r] fp16, swizzled
+constexpr int P_OFF_TPP = 7 * TILE;             // T'' [s][r] fp16, swizzled
+constexpr int P_OFF_AF = 8 * TILE;              // A fp32 [64][65]
+constexpr int P_OFF_TF = P_OFF_AF + 64 * 65 * 4;  // T fp32 [64][64]
+constexpr int P_OFF_XF = P_OFF_TF + 64 * 64 * 4;  // X fp32 [3][256]
+constexpr int P_OFF_VEC = P_OFF_XF + 3 * 256 * 4; // G, beta, rk, rq, gamma (64 each), row sums of squares (128)
+constexpr int P_OFF_BAR = P_OFF_VEC + 8 * 64 * 4;
+constexpr int P_SMEM = P_OFF_BAR + 64 + 1024;
+static_assert(P_SMEM * 2 <= 228 * 1024, "two prep CTAs per SM");
+constexpr uint32_t P_TM_D1 = 0, P_TM_D2 = 64, P_TM_D3 = 128;
+
+__global__ void __launch_bounds__(NT, 2)
+gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict__ ga, const float *__restrict__ gb,
+                      const float *__restrict__ A_log, const float *__restrict__ dt_bias,
+                      const int32_t *__restrict__ cu_seqlens, int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv,
+                      int32_t slots, float scale, int32_t l2norm, uint8_t *__restrict__ ws, int *status) {
+    const int id = blockIdx.x, h = blockIdx.y;
+    int n, t_begin, t_end;
+    locate(id, cu_seqlens, num_seqs, T, n, t_begin, t_end);
+    const int t0 = t_begin + (id - (t_begin / C + n)) * C;
+    if (id < t_begin / C + n || t0 >= t_end) return;   // a slot no chunk uses
+    const int L = min(C, t_end - t0);
+    const int hk = h / (Hv / Hk);
+    uint8_t *item = ws + ((size_t)h * slots + id) * kWsItem;
+
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *vec = reinterpret_cast<float *>(sm + OFF_VEC);
-    float *sG = vec, *sBeta = vec + 64, *sRk = vec + 128, *sRq = vec + 192, *sGam = vec + 256;
-    float *sDecS = vec + 320;   // exp(G_last - G_s) / |k_s| for the state update
-    float *sSS = vec + 384;     // row sums of squares of [K; Q] (64 + 64)
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    float *vec = reinterpret_cast<float *>(sm + P_OFF_VEC);
+    float *sG = vec, *sBeta = vec + 64, *sRk = vec + 128, *sRq = vec + 192, *sGam = vec + 256, *sSS = vec + 320;
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + P_OFF_BAR);
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 2);
-    float *Af = reinterpret_cast<float *>(sm + OFF_AF);   // [64][65]
-    float *Tf = reinterpret_cast<float *>(sm + OFF_TF);   // [64][64]
-    float *Xf = reinterpret_cast<float *>(sm + OFF_XF);   // 3 x 256
+    float *Af = reinterpret_cast<float *>(sm + P_OFF_AF);
+    float *Tf = reinterpret_cast<float *>(sm + P_OFF_TF);
+    float *Xf = reinterpret_cast<float *>(sm + P_OFF_XF);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int wg = warp / 4;
+    const int row = (warp % 4) * 32 + lane;
+    const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
+
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(bar_mma, 1);
+        fence_barrier_init();
+        mbar_arrive_expect_tx(bar_tma, 6 * TILE);
+        tma_load_3d(sm + P_OFF_KQ + 0 * TILE, &maps.k, bar_tma, 0, hk, t0);
+        tma_load_3d(sm + P_OFF_KQ + 1 * TILE, &maps.q, bar_tma, 0, hk, t0);
+        tma_load_3d(sm + P_OFF_KQ + 2 * TILE, &maps.k, bar_tma, 64, hk, t0);
+        tma_load_3d(sm + P_OFF_KQ + 3 * TILE, &maps.q, bar_tma, 64, hk, t0);
+        tma_load_3d(sm + P_OFF_V + 0 * TILE, &maps.v, bar_tma, 0, h, t0);
+        tma_load_3d(sm + P_OFF_V + 1 * TILE, &maps.v, bar_tma, 64, h, t0);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    // gates and the warp-local part of the cumulative log decay, while the tiles stream in
+    if (tid < 64) {
+        float g = 0.0f, beta = 0.0f;
+        if (tid < L) gdn_gates(ga[(size_t)(t0 + tid) * Hv + h], gb[(size_t)(t0 + tid) * Hv + h], A_log[h], dt_bias[h], g, beta);
+        float x = g;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        sG[tid] = x;
+        sBeta[tid] = beta;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (tid >= 32 && tid < 64) sG[tid] += sG[31];
+
+    int ok = 1;
+    if (tid == 0) ok = mbar_wait(bar_tma, 0, status) ? 1 : 0;
+    if (!__syncthreads_and(ok)) goto teardown;
+    {
+        // [K;Q] rows: thread -> (row rho = tid / 2, half = tid % 2); V: 4 chunks per thread
+        const int rho = tid >> 1, half = tid & 1;
+        uint8_t *rowp = sm + P_OFF_KQ + half * 2 * TILE + rho * 128;
+        float ss = 0.0f;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) ss += convert16(rowp + ((ch + rho) & 7) * 16);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        if (half == 0) sSS[rho] = ss;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) convert16(sm + P_OFF_V + (tid * 4 + e) * 16);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t id1 = idesc_f16(64, false, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint8_t *abase = sm + P_OFF_KQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
+            mma_f16(tmem + P_TM_D1, kdesc(abase), kdesc(abase), id1, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar_mma);
+    }
+    if (tid < 64) {
+        const bool v = tid < L;
+        sRk[tid] = v ? (l2norm ? rsqrtf(sSS[tid] + 1e-6f) : 1.0f) : 0.0f;
+        sRq[tid] = v ? (l2norm ? rsqrtf(sSS[64 + tid] + 1e-6f) * scale : scale) : 0.0f;
+        sGam[tid] = v ? expf(sG[tid]) : 0.0f;
+    }
+    if (tid == 0) ok = mbar_wait(bar_mma, 0, status) ? 1 : 0;
+    if (!__syncthreads_and(ok)) goto teardown;
+    tc_fence_after();
+    {
+        // A (fp32, for the inverse) from K K^T; P (fp16 operand image, to the workspace) from Q K^T
+        uint32_t r32[32];
+        const int col0 = wg * 32;
+        tmem_ld32(tmem + P_TM_D1 + lane_base + col0, r32);
+        tmem_ld_wait();
+        if (row < 64) {
+            const int r = row;
+            const float Gr = sG[r], br = sBeta[r] * sRk[r];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int s = col0 + j;
+                float a = 0.0f;
+                if (s < r && r < L) a = br * __expf(Gr - sG[s]) * __uint_as_float(r32[j]) * sRk[s];
+                Af[r * 65 + s] = a;
+            }
+        } else {
+            const int r = row - 64;
+            const float Gr = sG[r], rqr = sRq[r];
+            float pv[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int s = col0 + j;
+                pv[j] = (s <= r && r < L) ? __uint_as_float(r32[j]) * rqr * sRk[s] * __expf(Gr - sG[s]) : 0.0f;
+            }
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) st_h8(item + kWsP + swz(r, wg * 4 + ch), &pv[ch * 8]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- T = (I + A)^-1: 16 x 16 diagonal blocks by forward substitution, then the
+    //      off-diagonal blocks level by level, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.
+    if (tid < 64) {
+        const int bi = tid / 16, cc = tid % 16, o0 = bi * 16;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = (r == cc) ? 1.0f : 0.0f;
+#pragma unroll
+            for (int s = 0; s < r; ++s) acc -= Af[(o0 + r) * 65 + o0 + s] * x[s];
+            x[r] = acc;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tf[(o0 + r) * 64 + o0 + cc] = x[r];
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int lvl = 1; lvl < 4; ++lvl) {
+        const int nblk = 4 - lvl;
+        const int er = tid / 16, ec = tid % 16;
+        for (int bj = 0; bj < nblk; ++bj) {
+            const int bi = bj + lvl;
+            float acc = 0.0f;
+            for (int bk = bj; bk < bi; ++bk)
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    acc += Af[(bi * 16 + er) * 65 + bk * 16 + e] * Tf[(bk * 16 + e) * 64 + bj * 16 + ec];
+            Xf[bj * 256 + er * 16 + ec] = acc;
+        }
+        __syncthreads();
+        for (int bj = 0; bj < nblk; ++bj) {
+            const int bi = bj + lvl;
+            float acc = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc += Tf[(bi * 16 + er) * 64 + bi * 16 + e] * Xf[bj * 256 + e * 16 + ec];
+            Tf[(bi * 16 + er) * 64 + bj * 16 + ec] = -acc;
+        }
+        __syncthreads();
+    }
+    {
+        // T' = T diag(beta gamma / |k|), T'' = T diag(beta): fp16 B operands [s][r] (r <= s)
+        const int s = tid / 4, part = tid % 4;
+        float tp[16], tpp[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int r = part * 16 + e;
+            const float t = (r <= s) ? Tf[s * 64 + r] : 0.0f;
+            tpp[e] = t * sBeta[r];
+            tp[e] = tpp[e] * sGam[r] * sRk[r];
+        }
+        st_h8(sm + P_OFF_TP + swz(s, part * 2), tp);
+        st_h8(sm + P_OFF_TP + swz(s, part * 2 + 1), tp + 8);
+        st_h8(sm + P_OFF_TPP + swz(s, part * 2), tpp);
+        st_h8(sm + P_OFF_TPP + swz(s, part * 2 + 1), tpp + 8);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t id_mn = idesc_f16(64, true, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)   // D2 = K^T T'^T  (A: K, MN-major over j)
+            mma_f16(tmem + P_TM_D2, mndesc(sm + P_OFF_KQ + kk * 2048, 2 * TILE), kdesc(sm + P_OFF_TP + kk * 32), id_mn,
+                    kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)   // D3 = V^T T''^T
+            mma_f16(tmem + P_TM_D3, mndesc(sm + P_OFF_V + kk * 2048, TILE), kdesc(sm + P_OFF_TPP + kk * 32), id_mn,
+                    kk > 0);
+        tc_commit(bar_mma);
+    }
+    // vectors for the chain: gamma_r scale/|q_r|, gamma_C/gamma_s/|k_s|, gamma_C
+    if (tid < 64) {
+        float *wv = reinterpret_cast<float *>(item + kWsVec);
+        const float G_last = sG[L - 1];
+        wv[tid] = sGam[tid] * sRq[tid];
+        wv[64 + tid] = tid < L ? __expf(G_last - sG[tid]) * sRk[tid] : 0.0f;
+        if (tid == 0) wv[128] = __expf(G_last);
+    }
+    if (tid == 0) ok = mbar_wait(bar_mma, 1, status) ? 1 : 0;
+    if (!__syncthreads_and(ok)) goto teardown;
+    tc_fence_after();
+    {
+        // W operand image: row j (this thread's TMEM lane), tokens s in 16-byte chunks
+        uint32_t r32[32];
+        tmem_ld32(tmem + P_TM_D2 + lane_base + wg * 32, r32);
+        tmem_ld_wait();
+        float w[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) w[j] = __uint_as_float(r32[j]);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) st_h8(item + kWsW + swz(row, wg * 4 + ch), &w[ch * 8]);
+        // U~ as [s][i]
+        tmem_ld32(tmem + P_TM_D3 + lane_base + wg * 32, r32);
+        tmem_ld_wait();
+        __half *ut = reinterpret_cast<__half *>(item + kWsU);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ut[(wg * 32 + j) * D + row] = __float2half_rn(__uint_as_float(r32[j]));
+    }
+teardown:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ===================================================================================
+// Chain kernel: one CTA per (value head, sequence), chunks in order, double-buffered.
+// ===================================================================================
+constexpr int B_W = 0, B_U = 16384, B_P = 32768, B_VEC = 40960, B_KQ = 41984;   // within a chunk buffer
+constexpr int BUF = B_KQ + 4 * TILE;                                           // 74752 B
+constexpr int CH_OFF_BUF0 = 0;
+constexpr int CH_OFF_S = 2 * BUF;                 // S0 fp16 [S_lo: 128 rows x 64][S_hi]
+constexpr int CH_OFF_UA = CH_OFF_S + 4 * TILE;    // U^T fp16 [i][s]
+constexpr int CH_OFF_US = CH_OFF_UA + 2 * TILE;   // U_S^T fp16 [i][s]
+constexpr int CH_OFF_BAR = CH_OFF_US + 2 * TILE;
+constexpr int CH_SMEM = CH_OFF_BAR + 128 + 1024;
+static_assert(CH_SMEM <= 232448, "chain shared memory");
+static_assert(BUF % 1024 == 0 && B_KQ % 1024 == 0, "1024-byte aligned tiles");
+constexpr uint32_t C_TM_D4 = 0, C_TM_D5 = 64, C_TM_D6 = 128, C_TM_D7 = 192;
+
+__global__ void __launch_bounds__(NT, 1)
+gdn_chunk_chain_kernel(const __grid_constant__ Maps maps, const int32_t *__restrict__ cu_seqlens, int32_t T,
+                       int32_t Hk, int32_t Hv, int32_t slots, int32_t out_bf16, const float *S0g, float *S_out,
+                       void *__restrict__ o, const uint8_t *__restrict__ ws, int *status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CH_OFF_BAR);
+    uint64_t *full = bars, *bar_u = bars + 2, *bar_o5 = bars + 3, *bar_s = bars + 4, *bar_o6 = bars + 5;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int wg = warp / 4;
+    const int row = (warp % 4) * 32 + lane;
+    const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
     const int h = blockIdx.x, n = blockIdx.y;
     const int hk = h / (Hv / Hk);
     int t_begin = 0, t_end = T;
@@ -141,11 +440,16 @@ gdn_chunked_kernel(const __grid_constant__ Maps maps, const float *__restrict__ 
         t_end = cu_seqlens[n + 1];
     }
     const int nchunks = (t_end - t_begin + C - 1) / C;
-    const float Al = A_log[h], db = dt_bias[h];
+    const int slot0 = t_begin / C + n;
+    const uint8_t *ws_h = ws + (size_t)h * slots * kWsItem;
 
     if (tid == 0) {
-        mbar_init(bar_tma, 1);
-        mbar_init(bar_mma, 1);
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_init(bar_u, 1);
+        mbar_init(bar_o5, 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o6, 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -156,34 +460,25 @@ gdn_chunked_kernel(const __grid_constant__ Maps maps, const float *__restrict__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    uint32_t ph_tma = 0, ph_mma = 0;
-    bool alive = true;
 
-    auto issue_loads = [&](int t0) {
-        mbar_arrive_expect_tx(bar_tma, 6 * TILE);
-        uint8_t *stg = sm + OFF_STG;
-        tma_load_3d(stg + 0 * TILE, &maps.k, bar_tma, 0, hk, t0);
-        tma_load_3d(stg + 1 * TILE, &maps.q, bar_tma, 0, hk, t0);
-        tma_load_3d(stg + 2 * TILE, &maps.k, bar_tma, 64, hk, t0);
-        tma_load_3d(stg + 3 * TILE, &maps.q, bar_tma, 64, hk, t0);
-        tma_load_3d(stg + 4 * TILE, &maps.v, bar_tma, 0, h, t0);
-        tma_load_3d(stg + 5 * TILE, &maps.v, bar_tma, 64, h, t0);
+    auto issue_chunk = [&](int c) {
+        uint8_t *buf = sm + CH_OFF_BUF0 + (c & 1) * BUF;
+        uint64_t *bar = &full[c & 1];
+        const uint8_t *item = ws_h + (size_t)(slot0 + c) * kWsItem;
+        const int t0 = t_begin + c * C;
+        mbar_arrive_expect_tx(bar, BUF);
+        bulk_load(buf + B_W, item + kWsW, 16384, bar);
+        bulk_load(buf + B_U, item + kWsU, 16384, bar);
+        bulk_load(buf + B_P, item + kWsP, 8192, bar);
+        bulk_load(buf + B_VEC, item + kWsVec, 1024, bar);
+        tma_load_3d(buf + B_KQ + 0 * TILE, &maps.k, bar, 0, hk, t0);
+        tma_load_3d(buf + B_KQ + 1 * TILE, &maps.q, bar, 0, hk, t0);
+        tma_load_3d(buf + B_KQ + 2 * TILE, &maps.k, bar, 64, hk, t0);
+        tma_load_3d(buf + B_KQ + 3 * TILE, &maps.q, bar, 64, hk, t0);
     };
-    // Wait on an mbarrier phase: one thread polls (bounded), the block learns the outcome
-    // at a barrier, so every thread takes the same branch after a timeout.
-    auto wait_bar = [&](uint64_t *bar, uint32_t &ph) -> bool {
-        int ok = 1;
-        if (tid == 0) ok = mbar_wait(bar, ph, status) ? 1 : 0;
-        ph ^= 1u;
-        return __syncthreads_and(ok) != 0;
-    };
+    if (tid == 0 && nchunks > 0) issue_chunk(0);
 
-    if (tid == 0 && nchunks > 0) issue_loads(t_begin);
-
-    // ---- initial state: thread (lane row i, column half wg) holds S[i][64 wg .. 64 wg + 63]
-    const int wg = warp / 4;                 // column half
-    const int row = (warp % 4) * 32 + lane;  // tensor-memory lane == value index i
-    const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
+    // state: thread (TMEM lane i, column half wg) holds S[i][64 wg .. 64 wg + 63] in fp32
     float S[64];
     {
         const size_t base = (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
@@ -199,261 +494,67 @@ gdn_chunked_kernel(const __grid_constant__ Maps maps, const float *__restrict__ 
         }
     }
     auto write_S_smem = [&]() {
-        uint8_t *half = sm + OFF_S + wg * 2 * TILE;   // 128 rows x 128 B
+        uint8_t *half = sm + CH_OFF_S + wg * 2 * TILE;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) st_h8(half + swz(row, ch), &S[ch * 8]);
     };
     write_S_smem();
 
-    for (int c = 0; c < nchunks && alive; ++c) {
+    bool alive = true;
+    for (int c = 0; c < nchunks; ++c) {
         const int t0 = t_begin + c * C;
         const int L = min(C, t_end - t0);
+        uint8_t *buf = sm + CH_OFF_BUF0 + (c & 1) * BUF;
+        const float *vec = reinterpret_cast<const float *>(buf + B_VEC);
+        const uint32_t ph = (uint32_t)(c & 1);
 
-        // ---------------------------------------------------------------- stage in
-        if (!wait_bar(bar_tma, ph_tma)) { alive = false; break; }
-        {
-            // [K;Q] rows: thread -> (row rho = tid / 2, half = tid % 2): convert and square-sum
-            const int rho = tid >> 1, half = tid & 1;
-            const uint32_t off = (uint32_t)(half * 2 * TILE + rho * 128);
-            float ss = 0.0f;
+        int ok = 1;
+        if (tid == 0) ok = mbar_wait(&full[c & 1], (uint32_t)((c >> 1) & 1), status) ? 1 : 0;
+        if (!__syncthreads_and(ok)) { alive = false; break; }
+        // K and Q tiles to fp16 in place (8 chunks of 16 B per thread)
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint4 u = *reinterpret_cast<const uint4 *>(sm + OFF_STG + off + ch * 16);
-                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
-                float f[8];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float2 x = __bfloat1622float2(b2[e]);
-                    f[2 * e] = x.x; f[2 * e + 1] = x.y;
-                    ss += x.x * x.x + x.y * x.y;
-                }
-                st_h8(sm + OFF_KQ + off + ch * 16, f);
-            }
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            if (half == 0) sSS[rho] = ss;
-            // V: 1024 chunks, 4 per thread
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const uint32_t o16 = (uint32_t)(4 * TILE + (tid * 4 + e) * 16);
-                uint4 u = *reinterpret_cast<const uint4 *>(sm + OFF_STG + o16);
-                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
-                float f[8];
-#pragma unroll
-                for (int q2 = 0; q2 < 4; ++q2) {
-                    float2 x = __bfloat1622float2(b2[q2]);
-                    f[2 * q2] = x.x; f[2 * q2 + 1] = x.y;
-                }
-                st_h8(sm + OFF_KQ + o16, f);
-            }
-        }
-        // gates and the in-chunk cumulative log decay (warps 0-1: token r = tid)
-        if (tid < 64) {
-            const int r = tid;
-            float g = 0.0f, beta = 0.0f;
-            if (r < L) gdn_gates(ga[(size_t)(t0 + r) * Hv + h], gb[(size_t)(t0 + r) * Hv + h], Al, db, g, beta);
-            float x = g;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                float y = __shfl_up_sync(0xffffffffu, x, off);
-                if (lane >= off) x += y;
-            }
-            sG[r] = x;       // warp-local inclusive sums; warp 1 adds warp 0's total below
-            sBeta[r] = beta;
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            // MMA1: D1 = [K; Q] K^T (M = 128, N = 64, K = 128)
-            tc_fence_after();
-            const uint32_t id = idesc_f16(64, false, false, false);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint8_t *abase = sm + OFF_KQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
-                mma_f16(tmem + TM_D1, kdesc(abase), kdesc(abase), id, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(bar_mma);
-            // the staging tiles are free: stream in the next chunk
-            if (c + 1 < nchunks) {
-                fence_proxy_async_smem();
-                issue_loads(t0 + C);
-            }
-        }
-        if (tid >= 32 && tid < 64) sG[tid] += sG[31];
-        __syncthreads();
-        if (tid < 64) {
-            const int r = tid;
-            const float G = sG[r];
-            const bool v = r < L;
-            const float rk = v ? (l2norm ? rsqrtf(sSS[r] + 1e-6f) : 1.0f) : 0.0f;
-            const float rq = v ? (l2norm ? rsqrtf(sSS[64 + r] + 1e-6f) * scale : scale) : 0.0f;
-            sRk[r] = rk;
-            sRq[r] = rq;
-            sGam[r] = v ? expf(G) : 0.0f;
-        }
-        __syncthreads();
-        const float G_last = sG[L - 1];
-        if (tid < 64) sDecS[tid] = tid < L ? expf(G_last - sG[tid]) * sRk[tid] : 0.0f;
-
-        // ---------------------------------------------------- A and P from D1
-        if (!wait_bar(bar_mma, ph_mma)) { alive = false; break; }
-        tc_fence_after();
-        {
-            uint32_t r32[32];
-            const int col0 = wg * 32;
-            tmem_ld32(tmem + TM_D1 + lane_base + col0, r32);
-            tmem_ld_wait();
-            if (row < 64) {
-                const int r = row;
-                const float Gr = sG[r], br = sBeta[r], rkr = sRk[r];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int s = col0 + j;
-                    float a = 0.0f;
-                    if (s < r && r < L) a = br * expf(Gr - sG[s]) * __uint_as_float(r32[j]) * rkr * sRk[s];
-                    Af[r * 65 + s] = a;
-                }
-            } else {
-                const int r = row - 64;
-                const float Gr = sG[r], rqr = sRq[r];
-                float pv[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int s = col0 + j;
-                    float p = 0.0f;
-                    if (s <= r && r < L) p = __uint_as_float(r32[j]) * rqr * sRk[s] * expf(Gr - sG[s]);
-                    pv[j] = p;
-                }
-                uint8_t *P = sm + OFF_P;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) st_h8(P + swz(r, wg * 4 + ch), &pv[ch * 8]);
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ---------------------------------------------------- T = (I + A)^-1, blocked 16 x 16
-        if (tid < 64) {
-            const int bi = tid / 16, cc = tid % 16, o0 = bi * 16;
-            float x[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = (r == cc) ? 1.0f : 0.0f;
-#pragma unroll
-                for (int s = 0; s < r; ++s) acc -= Af[(o0 + r) * 65 + o0 + s] * x[s];
-                x[r] = acc;
-            }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) Tf[(o0 + r) * 64 + o0 + cc] = x[r];
-        }
-        __syncthreads();
-        for (int lvl = 1; lvl < 4; ++lvl) {
-            const int nblk = 4 - lvl;
-            const int er = tid / 16, ec = tid % 16;
-            // X_ij = sum_{k=j}^{i-1} A_ik T_kj   for (i, j) = (j + lvl, j)
-            for (int bj = 0; bj < nblk; ++bj) {
-                const int bi = bj + lvl;
-                float acc = 0.0f;
-                for (int bk = bj; bk < bi; ++bk)
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        acc += Af[(bi * 16 + er) * 65 + bk * 16 + e] * Tf[(bk * 16 + e) * 64 + bj * 16 + ec];
-                Xf[bj * 256 + er * 16 + ec] = acc;
-            }
-            __syncthreads();
-            // T_ij = -T_ii X_ij
-            for (int bj = 0; bj < nblk; ++bj) {
-                const int bi = bj + lvl;
-                float acc = 0.0f;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) acc += Tf[(bi * 16 + er) * 64 + bi * 16 + e] * Xf[bj * 256 + e * 16 + ec];
-                Tf[(bi * 16 + er) * 64 + bj * 16 + ec] = -acc;
-            }
-            __syncthreads();
-        }
-        // T' = T diag(beta gamma rk), T'' = T diag(beta) as fp16 B operands [s][r] (r <= s)
-        {
-            const int s = tid / 4, part = tid % 4;   // 16 columns each
-            float tp[16], tpp[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int r = part * 16 + e;
-                const float t = (r <= s) ? Tf[s * 64 + r] : 0.0f;
-                tp[e] = t * sBeta[r] * sGam[r] * sRk[r];
-                tpp[e] = t * sBeta[r];
-            }
-            st_h8(sm + OFF_TP + swz(s, part * 2), tp);
-            st_h8(sm + OFF_TP + swz(s, part * 2 + 1), tp + 8);
-            st_h8(sm + OFF_TPP + swz(s, part * 2), tpp);
-            st_h8(sm + OFF_TPP + swz(s, part * 2 + 1), tpp + 8);
-        }
+        for (int e = 0; e < 8; ++e) convert16(buf + B_KQ + (tid * 8 + e) * 16);
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            // MMA2: D2 = K^T T'^T (A = K, MN-major over the key index; K-extent = token r)
-            const uint32_t id_mn = idesc_f16(64, true, false, false);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TM_D2, mndesc(sm + OFF_KQ + kk * 2048, 2 * TILE), kdesc(sm + OFF_TP + kk * 32), id_mn,
-                        kk > 0);
-            // MMA3: D3 = V^T T''^T
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TM_D3, mndesc(sm + OFF_V + kk * 2048, TILE), kdesc(sm + OFF_TPP + kk * 32), id_mn, kk > 0);
-            // MMA5: D5 = S0 Q^T (A = S0 K-major over j, B = Q K-major over j)
-            const uint32_t id_kk = idesc_f16(64, false, false, false);
+            if (c + 1 < nchunks) issue_chunk(c + 1);
+            // MMA4: D4 = S0 W^T (A: S0 K-major over j; B: W image, MN-major over s)
+            const uint32_t id4 = idesc_f16(64, false, true, false);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint8_t *a = sm + OFF_S + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
-                const uint8_t *b = sm + OFF_KQ + TILE + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
-                mma_f16(tmem + TM_D5, kdesc(a), kdesc(b), id_kk, kk > 0);
+                const uint8_t *a = sm + CH_OFF_S + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
+                mma_f16(tmem + C_TM_D4, kdesc(a), mndesc(buf + B_W + kk * 2048, 0), id4, kk > 0);
             }
-            tc_commit(bar_mma);
-        }
-        if (!wait_bar(bar_mma, ph_mma)) { alive = false; break; }
-        tc_fence_after();
-        // ---------------------------------------------------- W (fp16, [j][s]) from D2
-        {
-            uint32_t r32[32];
-            tmem_ld32(tmem + TM_D2 + lane_base + wg * 32, r32);
-            tmem_ld_wait();
-            float w[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) w[j] = __uint_as_float(r32[j]);
-            uint8_t *Wt = sm + OFF_W;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) st_h8(Wt + swz(row, wg * 4 + ch), &w[ch * 8]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            // MMA4: D3 -= S0 W^T (B = W, MN-major over the token index s; K-extent = j)
-            const uint32_t id = idesc_f16(64, false, true, true);
+            tc_commit(bar_u);
+            // MMA5: D5 = S0 Q^T
+            const uint32_t id5 = idesc_f16(64, false, false, false);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint8_t *a = sm + OFF_S + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
-                mma_f16(tmem + TM_D3, kdesc(a), mndesc(sm + OFF_W + kk * 2048, 0), id, 1u);
+                const uint8_t *a = sm + CH_OFF_S + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
+                const uint8_t *b = buf + B_KQ + TILE + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
+                mma_f16(tmem + C_TM_D5, kdesc(a), kdesc(b), id5, kk > 0);
             }
-            tc_commit(bar_mma);
+            tc_commit(bar_o5);
         }
-        if (!wait_bar(bar_mma, ph_mma)) { alive = false; break; }
+        if (tid == 0) ok = mbar_wait(bar_u, ph, status) ? 1 : 0;
+        if (!__syncthreads_and(ok)) { alive = false; break; }
         tc_fence_after();
-        // ---------------------------------------------------- U^T rows -> U_A, U_S (fp16 [i][s])
         {
+            // U^T = U~^T - D4 -> U_A = U^T, U_S = U^T diag(gamma_C / gamma / |k|) (fp16 [i][s])
             uint32_t r32[32];
-            tmem_ld32(tmem + TM_D3 + lane_base + wg * 32, r32);
+            tmem_ld32(tmem + C_TM_D4 + lane_base + wg * 32, r32);
             tmem_ld_wait();
+            const __half *ut = reinterpret_cast<const __half *>(buf + B_U);
             float ua[32], us[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int s = wg * 32 + j;
-                const float u = (s < L) ? __uint_as_float(r32[j]) : 0.0f;
+                const float u = (s < L) ? __half2float(ut[s * D + row]) - __uint_as_float(r32[j]) : 0.0f;
                 ua[j] = u;
-                us[j] = u * sDecS[s];
+                us[j] = u * vec[64 + s];
             }
-            uint8_t *UA = sm + OFF_U, *US = sm + OFF_U + 2 * TILE;
+            uint8_t *UA = sm + CH_OFF_UA, *US = sm + CH_OFF_US;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 st_h8(UA + swz(row, wg * 4 + ch), &ua[ch * 8]);
@@ -465,46 +566,52 @@ gdn_chunked_kernel(const __grid_constant__ Maps maps, const float *__restrict__ 
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            // MMA6: D6 = U^T P^T ; MMA7: D7 = U_S^T K (B = K MN-major over j; K-extent = s)
-            const uint32_t id6 = idesc_f16(64, false, false, false);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TM_D6, kdesc(sm + OFF_U + kk * 32), kdesc(sm + OFF_P + kk * 32), id6, kk > 0);
+            // MMA7: D7 = U_S^T K (B: K, MN-major over j); MMA6: D6 = U^T P^T
             const uint32_t id7 = idesc_f16(128, false, true, false);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TM_D7, kdesc(sm + OFF_U + 2 * TILE + kk * 32), mndesc(sm + OFF_KQ + kk * 2048, 2 * TILE),
-                        id7, kk > 0);
-            tc_commit(bar_mma);
+                mma_f16(tmem + C_TM_D7, kdesc(sm + CH_OFF_US + kk * 32), mndesc(buf + B_KQ + kk * 2048, 2 * TILE), id7,
+                        kk > 0);
+            tc_commit(bar_s);
+            const uint32_t id6 = idesc_f16(64, false, false, false);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(tmem + C_TM_D6, kdesc(sm + CH_OFF_UA + kk * 32), kdesc(buf + B_P + kk * 32), id6, kk > 0);
+            tc_commit(bar_o6);
         }
-        if (!wait_bar(bar_mma, ph_mma)) { alive = false; break; }
+        if (tid == 0) ok = mbar_wait(bar_s, ph, status) ? 1 : 0;
+        if (!__syncthreads_and(ok)) { alive = false; break; }
         tc_fence_after();
-        // ---------------------------------------------------- outputs and the state update
+        {
+            const float gC = vec[128];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t r7[32];
+                tmem_ld32(tmem + C_TM_D7 + lane_base + wg * 64 + half * 32, r7);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[half * 32 + j] = gC * S[half * 32 + j] + __uint_as_float(r7[j]);
+            }
+        }
+        if (tid == 0) ok = mbar_wait(bar_o6, ph, status) ? 1 : 0;
+        if (!__syncthreads_and(ok)) { alive = false; break; }
+        tc_fence_after();
+        write_S_smem();   // the next chunk's S0 (MMA4/5 of this chunk are complete)
         {
             uint32_t a5[32], a6[32];
-            tmem_ld32(tmem + TM_D5 + lane_base + wg * 32, a5);
-            tmem_ld32(tmem + TM_D6 + lane_base + wg * 32, a6);
+            tmem_ld32(tmem + C_TM_D5 + lane_base + wg * 32, a5);
+            tmem_ld32(tmem + C_TM_D6 + lane_base + wg * 32, a6);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int r = wg * 32 + j;
                 if (r < L) {
-                    const float val = __uint_as_float(a5[j]) * sGam[r] * sRq[r] + __uint_as_float(a6[j]);
+                    const float val = __uint_as_float(a5[j]) * vec[r] + __uint_as_float(a6[j]);
                     const size_t idx = ((size_t)(t0 + r) * Hv + h) * D + row;
                     if (out_bf16) store1<true>(o, idx, val);
                     else store1<false>(o, idx, val);
                 }
             }
-            const float gC = sGam[L - 1];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r7[32];
-                tmem_ld32(tmem + TM_D7 + lane_base + wg * 64 + half * 32, r7);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) S[half * 32 + j] = gC * S[half * 32 + j] + __uint_as_float(r7[j]);
-            }
-            write_S_smem();
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -564,14 +671,22 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
         return cudaErrorInvalidValue;
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    dim3 grid(c.Hv, c.num_seqs);
-    gdn_chunked_kernel<<<grid, NT, SMEM_BYTES, st>>>(maps, c.a, c.b, c.A_log, c.dt_bias, c.cu_seqlens, c.T, c.Hk, c.Hv,
-                                                      c.scale, c.l2norm, c.out_bf16 ? 1 : 0, c.S0, c.S_out, c.o,
-                                                      c.status);
+    const int slots = c.T / kChunk + c.num_seqs;
+    uint8_t *ws = static_cast<uint8_t *>(c.ws);
+    gdn_chunk_prep_kernel<<<dim3(slots, c.Hv), NT, P_SMEM, st>>>(maps, c.a, c.b, c.A_log, c.dt_bias, c.cu_seqlens, c.T,
+                                                                 c.num_seqs, c.Hk, c.Hv, slots, c.scale, c.l2norm, ws,
+                                                                 c.status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    gdn_chunk_chain_kernel<<<dim3(c.Hv, c.num_seqs), NT, CH_SMEM, st>>>(maps, c.cu_seqlens, c.T, c.Hk, c.Hv, slots,
+                                                                        c.out_bf16 ? 1 : 0, c.S0, c.S_out, c.o, ws,
+                                                                        c.status);
     return cudaGetLastError();
 }
 

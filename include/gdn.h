@@ -74,12 +74,15 @@ typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
  * initial_state  [num_seqs, Hv, Dv, Dk] fp32, or NULL for zero states
  * final_state    [num_seqs, Hv, Dv, Dk] fp32 output, or NULL; may alias initial_state
  * o           [T, Hv, Dv] in `out_dtype`
- * workspace   device scratch of at least gdn_prefill_workspace_bytes(...) bytes (may be
- *             NULL when that is 0).
+ * workspace   device scratch of at least gdn_prefill_workspace_bytes(...) bytes, 16-byte
+ *             aligned, owned by the caller; its contents on entry do not matter and are
+ *             overwritten. GDN_ERR_WORKSPACE if it is needed and missing or too small.
  * Supported: Dk == Dv in {16, 32, 64, 128}; Hv % Hk == 0; T >= 0 (T == 0 only writes
  * final_state = initial_state). Dk == Dv == 128 with bf16 inputs runs the tensor-core
- * chunked kernel (64-token chunks; operands staged in fp16, so |q|, |k|, |v| and the
- * state must stay below 6.5e4); other sizes run the CUDA-core recurrent kernel.
+ * chunked path (64-token chunks; a prep kernel parallel over chunks writes the
+ * state-independent operands to the workspace, a chain kernel walks the chunks of each
+ * sequence; operands are staged in fp16, so |q|, |k|, |v| and the state must stay below
+ * 6.5e4). Other sizes and fp32 inputs run the CUDA-core recurrent kernel (no workspace).
  */
 GDN_API gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v,
                                const float *a, const float *b,
@@ -91,7 +94,8 @@ GDN_API gdn_status gdn_prefill_chunked(const void *q, const void *k, const void 
                                void *o, gdn_dtype out_dtype,
                                void *workspace, size_t workspace_bytes, gdn_stream_t stream);
 
-/* Scratch bytes gdn_prefill_chunked needs for these sizes (0 when it needs none). */
+/* Scratch bytes the tensor-core path of gdn_prefill_chunked needs for these sizes:
+ * Hv * (T / 64 + num_seqs) * 41984 when Dk == Dv == 128, else 0. Host-only, no CUDA call. */
 GDN_API size_t gdn_prefill_workspace_bytes(int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv,
                                    int32_t Dk, int32_t Dv);
 
