@@ -145,7 +145,7 @@ def run_gpu(args):
     A_log, dt_bias, nw = up(x["A_log"], f32), up(x["dt_bias"], f32), up(x["norm_weight"], f32)
     W = up(x["proj_weight"], bf)
     gw = float(448.0 * 6.0 / W.float().abs().max().item())
-    wq, ws = g.nvfp4_quantize_act(W, gw)           # weights: quantised once, outside timing
+    wq, ws_w = g.nvfp4_quantize_act(W, gw)         # weights: quantised once, outside timing
     T, Hv, D, K, N = w.T, w.Hv, w.D, w.K, w.n_out
     o = torch.empty((T, Hv, D), dtype=bf, device=dev)
     S = torch.empty((1, Hv, D, D), dtype=f32, device=dev)
@@ -161,19 +161,21 @@ def run_gpu(args):
     flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=f32, device=dev)
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ws = torch.empty((g.gdn_prefill_workspace_bytes(T, 1, w.Hk, Hv, D, D),), dtype=torch.uint8, device=dev)
 
-    def step(evs=None):
-        if evs:
-            evs[0].record(stream)
-        g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, final_state=S, o=o)
-        if evs:
-            evs[1].record(stream)
+    def scan():
+        g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, final_state=S, o=o, workspace=ws)
+
+    def tail():
         g.gdn_gated_rmsnorm_silu_nvfp4(o, z, nw, gx, xq=xq, xs=xs)
-        if evs:
-            evs[2].record(stream)
-        g.nvfp4_gemm(xq, xs, wq, ws, alpha, y=Y)
-        if evs:
-            evs[3].record(stream)
+
+    def gemm():
+        g.nvfp4_gemm(xq, xs, wq, ws_w, alpha, y=Y)
+
+    def step():
+        scan()
+        tail()
+        gemm()
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -181,22 +183,47 @@ def run_gpu(args):
     torch.cuda.synchronize()
     assert g.gdn_get_device_status() == 0
 
-    evsets = [[ev() for _ in range(4)] for _ in range(args.steps)]
+    # CUDA graphs: the step and each op alone, replayed so the timing is device time only
+    graphs = {}
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for name, fn in (("step", step), ("scan", scan), ("tail", tail), ("gemm", gemm)):
+            fn()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=side):
+                fn()
+            graphs[name] = gr
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+
+    def timed(gr, n):
+        out = []
+        for _ in range(n):
+            flush.zero_()          # L2 flush between timed replays (outside the events)
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            gr.replay()
+            e1.record(stream)
+            out.append((e0, e1))
+        return out
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            flush.zero_()          # L2 flush between timed steps (outside the events)
-            step(evsets[i])
+        step_ev = timed(graphs["step"], args.steps)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms = [e[0].elapsed_time(e[3]) for e in evsets]
-    scan_ms = [e[0].elapsed_time(e[1]) for e in evsets]
-    tail_ms = [e[1].elapsed_time(e[2]) for e in evsets]
-    gemm_ms = [e[2].elapsed_time(e[3]) for e in evsets]
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    parts = {}
+    for name in ("scan", "tail", "gemm"):
+        evs = timed(graphs[name], args.steps)
+        torch.cuda.synchronize()
+        parts[name] = [a.elapsed_time(b) for a, b in evs]
+    scan_ms, tail_ms, gemm_ms = parts["scan"], parts["tail"], parts["gemm"]
     ms = statistics.mean(step_ms)
     ms_max = ms
     if world > 1:
@@ -213,6 +240,7 @@ def run_gpu(args):
     d2h = hY.numel() * hY.element_size()
 
     def e2e_step():
+        # host -> device inputs, the whole path through the public API, result back to host
         q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
         z.copy_(hz, non_blocking=True); a.copy_(ha, non_blocking=True); b.copy_(hb, non_blocking=True)
         step()
@@ -288,8 +316,8 @@ def run_gpu(args):
                    "out_proj": "NVFP4 W4A4 %d->%d" % (K, N), "global_batch": 1, "seq_len": T,
                    "parallelism": "replicas x%d" % world, "l2": "flushed (256 MiB write) between timed steps"},
         "breakdown_ms": {"scan": statistics.mean(scan_ms), "gated_norm_nvfp4": statistics.mean(tail_ms),
-                         "nvfp4_gemm": statistics.mean(gemm_ms)},
-        "roofline": {"kernel": "gdn prefill scan", "bound": "tensor", "achieved": achieved_tflops,
+                         "nvfp4_gemm": statistics.mean(gemm_ms), "timing": "CUDA graph replay per op"},
+        "roofline": {"kernel": "gdn prefill scan (prep + chain kernels of one call)", "bound": "tensor", "achieved": achieved_tflops,
                      "peak": peak_tflops, "unit": "TFLOP/s", "frac": achieved_tflops / peak_tflops,
                      "peak_kind": pk_kind + " (bf16 dense burst; the scan's MMAs are fp16)",
                      "algorithmic_flops": fl, "algorithmic_bytes": scan_bytes(w),
@@ -300,7 +328,7 @@ def run_gpu(args):
         "decode": {"workload": dw.name, "ms": dec, "GB/s": dec_bytes / (dec / 1e3) / 1e9,
                    "frac": dec_bytes / (dec / 1e3) / 1e9 / float(pk["hbm_gbs"]),
                    "bytes": dec_bytes, "peak_gbs": float(pk["hbm_gbs"]), "peak_kind": pk_kind},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 4 * args.steps,
         "clocks": clk.summary(),
     }
     if not args.no_cpu:

@@ -155,8 +155,8 @@ constexpr int P_OFF_V = 4 * TILE;               // [V_lo][V_hi]
 constexpr int P_OFF_TP = 6 * TILE;              // T'  [s][r] fp16, swizzled
 constexpr int P_OFF_TPP = 7 * TILE;             // T'' [s][r] fp16, swizzled
 constexpr int P_OFF_AF = 8 * TILE;              // A fp32 [64][65]
-constexpr int P_OFF_TF = P_OFF_AF + 64 * 65 * 4;  // T fp32 [64][64]
-constexpr int P_OFF_XF = P_OFF_TF + 64 * 64 * 4;  // X fp32 [3][256]
+constexpr int P_OFF_TF = P_OFF_AF + 64 * 65 * 4;  // T fp32 [64][65]
+constexpr int P_OFF_XF = P_OFF_TF + 64 * 65 * 4;  // X fp32 [3][256]
 constexpr int P_OFF_VEC = P_OFF_XF + 3 * 256 * 4; // G, beta, rk, rq, gamma (64 each), row sums of squares (128)
 constexpr int P_OFF_BAR = P_OFF_VEC + 8 * 64 * 4;
 constexpr int P_SMEM = P_OFF_BAR + 64 + 1024;
@@ -241,7 +241,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         ss += __shfl_xor_sync(0xffffffffu, ss, 1);
         if (half == 0) sSS[rho] = ss;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) convert16(sm + P_OFF_V + (tid * 4 + e) * 16);
+        for (int e = 0; e < 4; ++e) convert16(sm + P_OFF_V + (e * NT + tid) * 16);
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -309,7 +309,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             x[r] = acc;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tf[(o0 + r) * 64 + o0 + cc] = x[r];
+        for (int r = 0; r < 16; ++r) Tf[(o0 + r) * 65 + o0 + cc] = x[r];
     }
     __syncthreads();
 #pragma unroll 1
@@ -322,7 +322,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             for (int bk = bj; bk < bi; ++bk)
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    acc += Af[(bi * 16 + er) * 65 + bk * 16 + e] * Tf[(bk * 16 + e) * 64 + bj * 16 + ec];
+                    acc += Af[(bi * 16 + er) * 65 + bk * 16 + e] * Tf[(bk * 16 + e) * 65 + bj * 16 + ec];
             Xf[bj * 256 + er * 16 + ec] = acc;
         }
         __syncthreads();
@@ -330,19 +330,19 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             const int bi = bj + lvl;
             float acc = 0.0f;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) acc += Tf[(bi * 16 + er) * 64 + bi * 16 + e] * Xf[bj * 256 + e * 16 + ec];
-            Tf[(bi * 16 + er) * 64 + bj * 16 + ec] = -acc;
+            for (int e = 0; e < 16; ++e) acc += Tf[(bi * 16 + er) * 65 + bi * 16 + e] * Xf[bj * 256 + e * 16 + ec];
+            Tf[(bi * 16 + er) * 65 + bj * 16 + ec] = -acc;
         }
         __syncthreads();
     }
     {
         // T' = T diag(beta gamma / |k|), T'' = T diag(beta): fp16 B operands [s][r] (r <= s)
-        const int s = tid / 4, part = tid % 4;
+        const int s = tid % 64, part = tid / 64;
         float tp[16], tpp[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int r = part * 16 + e;
-            const float t = (r <= s) ? Tf[s * 64 + r] : 0.0f;
+            const float t = (r <= s) ? Tf[s * 65 + r] : 0.0f;
             tpp[e] = t * sBeta[r];
             tp[e] = tpp[e] * sGam[r] * sRk[r];
         }
@@ -511,9 +511,9 @@ gdn_chunk_chain_kernel(const __grid_constant__ Maps maps, const int32_t *__restr
         int ok = 1;
         if (tid == 0) ok = mbar_wait(&full[c & 1], (uint32_t)((c >> 1) & 1), status) ? 1 : 0;
         if (!__syncthreads_and(ok)) { alive = false; break; }
-        // K and Q tiles to fp16 in place (8 chunks of 16 B per thread)
+        // K and Q tiles to fp16 in place (8 chunks of 16 B per thread, lane-consecutive)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) convert16(buf + B_KQ + (tid * 8 + e) * 16);
+        for (int e = 0; e < 8; ++e) convert16(buf + B_KQ + (e * NT + tid) * 16);
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
@@ -598,19 +598,36 @@ gdn_chunk_chain_kernel(const __grid_constant__ Maps maps, const int32_t *__restr
         tc_fence_after();
         write_S_smem();   // the next chunk's S0 (MMA4/5 of this chunk are complete)
         {
+            // o^T = D5 diag(gamma scale / |q|) + D6, staged as [r][i] in the (now free) U area,
+            // then written with 16-byte row-contiguous stores (rows r < L only)
             uint32_t a5[32], a6[32];
             tmem_ld32(tmem + C_TM_D5 + lane_base + wg * 32, a5);
             tmem_ld32(tmem + C_TM_D6 + lane_base + wg * 32, a6);
             tmem_ld_wait();
+            uint8_t *stage = sm + CH_OFF_UA;
+            if (out_bf16) {
+                __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(stage);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int r = wg * 32 + j;
-                if (r < L) {
-                    const float val = __uint_as_float(a5[j]) * vec[r] + __uint_as_float(a6[j]);
-                    const size_t idx = ((size_t)(t0 + r) * Hv + h) * D + row;
-                    if (out_bf16) store1<true>(o, idx, val);
-                    else store1<false>(o, idx, val);
+                for (int j = 0; j < 32; ++j) {
+                    const int r = wg * 32 + j;
+                    st[r * D + row] = __float2bfloat16_rn(__uint_as_float(a5[j]) * vec[r] + __uint_as_float(a6[j]));
                 }
+            } else {
+                float *st = reinterpret_cast<float *>(stage);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int r = wg * 32 + j;
+                    st[r * D + row] = __uint_as_float(a5[j]) * vec[r] + __uint_as_float(a6[j]);
+                }
+            }
+            __syncthreads();
+            const int row_bytes = out_bf16 ? D * 2 : D * 4;
+            const int per_row = row_bytes / 16;
+            uint8_t *ob = static_cast<uint8_t *>(o);
+            for (int e = tid; e < L * per_row; e += NT) {
+                const int r = e / per_row, ch = e % per_row;
+                const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + ch * 16);
+                *reinterpret_cast<uint4 *>(ob + (((size_t)(t0 + r) * Hv + h) * D) * (row_bytes / D) + ch * 16) = val;
             }
         }
         fence_proxy_async_smem();

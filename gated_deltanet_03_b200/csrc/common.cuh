@@ -94,6 +94,9 @@ GDN_DEV float group_sum(float v) {
 // softplus(x) = log(1 + e^x), stable for large x; library expf / log1pf.
 GDN_DEV float softplus_f(float x) { return x > 20.0f ? x : log1pf(expf(x)); }
 GDN_DEV float sigmoid_f(float x) { return 1.0f / (1.0f + expf(-x)); }
+// z * sigmoid(z) with the fast exponential and division intrinsics (a few ulp; the tail's
+// tolerance is 1e-5 relative): the gated tail runs this once per element.
+GDN_DEV float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // log of the decay gate, g = -exp(A_log) * softplus(a + dt_bias), and the write strength.
 GDN_DEV void gdn_gates(float a, float b, float A_log, float dt_bias, float &g, float &beta) {

@@ -45,7 +45,7 @@ gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
         const float inv_rms = rsqrtf(ss * inv_d + eps);
         float yv[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) yv[j] = ov[j] * inv_rms * wv[j] * (zv[j] * sigmoid_f(zv[j]));
+        for (int j = 0; j < 8; ++j) yv[j] = ov[j] * inv_rms * wv[j] * silu_fast(zv[j]);
         if constexpr (!NVFP4) {
             if (live) store8<OUT_BF16>(y, base, yv);
         } else {
