@@ -65,9 +65,8 @@ gdn_status gdn_get_device_status(gdn_stream_t stream) {
 
 size_t gdn_prefill_workspace_bytes(int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv, int32_t Dk,
                                    int32_t Dv) {
-    (void)Hk;
-    if (T <= 0 || num_seqs < 1 || Hv < 1 || Dk != 128 || Dv != 128) return 0;
-    return gdn::chunked_workspace_bytes(T, num_seqs, Hv);
+    if (T <= 0 || num_seqs < 1 || Hk < 1 || Hv < 1 || Dk != 128 || Dv != 128) return 0;
+    return gdn::chunked_workspace_bytes(T, num_seqs, Hk, Hv);
 }
 
 gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v, const float *a, const float *b,
@@ -92,7 +91,7 @@ gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v, cons
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (Dk == 128 && in_dtype == GDN_BF16 && T > 0) {
-        const size_t need = gdn::chunked_workspace_bytes(T, num_seqs, Hv);
+        const size_t need = gdn::chunked_workspace_bytes(T, num_seqs, Hk, Hv);
         if (!workspace || workspace_bytes < need || !aligned16(workspace)) return GDN_ERR_WORKSPACE;
         gdn::ChunkedArgs c{q, k, v, a, b, A_log, dt_bias, cu_seqlens, T, num_seqs, Hk, Hv, scale, qk_l2norm,
                            out_dtype == GDN_BF16, initial_state, final_state, o, workspace, status_ptr()};

@@ -24,16 +24,18 @@
 //          MMA2  D2 = W^T  = K^T T'^T               T'  = T diag(beta gamma / |k|)
 //          MMA3  D3 = U~^T = V^T T''^T              T'' = T diag(beta)
 //   chain  MMA4  D4 = S0 W^T      -> U^T = U~^T - D4
-//          MMA5  D5 = S0 Q^T
 //          MMA7  D7 = U_S^T K     U_S = U diag(gamma_C / gamma / |k|)
-//          MMA6  D6 = U^T P^T     P = Q K^T o Gamma / (|q| |k|) * scale
-// then o^T = D5 diag(gamma * scale / |q|) + D6 and S <- gamma_C S + D7.
+//          MMA5  D5 = S0 Q'^T     Q' = diag(gamma scale / |q|) Q
+//          MMA6  D5 += U^T P^T    P = Q K^T o Gamma / (|q| |k|) * scale
+// then o^T = D5 and S <- gamma_C S + D7. In the chain the fp16 copies of S0 and U live in
+// tensor memory and are the A operands of their MMAs (no shared-memory round trip).
 //
-// Workspace: one 41 KB item per (value head, chunk slot): the W operand image (fp16,
+// Workspace: one 57 KB item per (value head, chunk slot): the W operand image (fp16,
 // [key j][token s], 128-byte swizzled rows), U~ (fp16, [token s][value i]), the P operand
-// image (fp16, [r][s] swizzled) and fp32 vectors (gamma_r scale/|q_r|, gamma_C/gamma_s/|k_s|,
-// gamma_C). Chunk c of sequence n uses slot cu_seqlens[n] / 64 + n + c, so slots never
-// collide and T / 64 + num_seqs slots per head suffice.
+// image (fp16, [r][s] swizzled), the Q' = diag(gamma scale / |q|) Q operand image and fp32
+// vectors (gamma_C / gamma_s / |k_s|, gamma_C); and one 16 KB fp16 K operand image per (key
+// head, chunk slot). Chunk c of sequence n uses slot cu_seqlens[n] / 64 + n + c, so slots
+// never collide and T / 64 + num_seqs slots per head suffice.
 #include <mutex>
 
 #include "common.cuh"
@@ -42,11 +44,17 @@
 namespace gdn {
 
 constexpr int kChunk = 64;
-constexpr int kWsItem = 41984;
-constexpr int kWsW = 0, kWsU = 16384, kWsP = 32768, kWsVec = 40960;
+// per (value head, slot): W image, U~, P image, Q' image, vectors
+constexpr int kWsItem = 58368;
+constexpr int kWsW = 0, kWsU = 16384, kWsP = 32768, kWsQ = 40960, kWsVec = 57344;
+// per (key head, slot): the fp16 K image
+constexpr int kWsKItem = 16384;
 
-size_t chunked_workspace_bytes(int T, int num_seqs, int Hv) {
+static size_t ws_value_region(int T, int num_seqs, int Hv) {
     return (size_t)Hv * (size_t)(T / kChunk + num_seqs) * kWsItem;
+}
+size_t chunked_workspace_bytes(int T, int num_seqs, int Hk, int Hv) {
+    return ws_value_region(T, num_seqs, Hv) + (size_t)Hk * (size_t)(T / kChunk + num_seqs) * kWsKItem;
 }
 
 namespace {
@@ -167,7 +175,8 @@ __global__ void __launch_bounds__(NT, 2)
 gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict__ ga, const float *__restrict__ gb,
                       const float *__restrict__ A_log, const float *__restrict__ dt_bias,
                       const int32_t *__restrict__ cu_seqlens, int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv,
-                      int32_t slots, float scale, int32_t l2norm, uint8_t *__restrict__ ws, int *status) {
+                      int32_t slots, float scale, int32_t l2norm, uint8_t *__restrict__ ws,
+                      uint8_t *__restrict__ ws_k, int *status) {
     const int id = blockIdx.x, h = blockIdx.y;
     int n, t_begin, t_end;
     locate(id, cu_seqlens, num_seqs, T, n, t_begin, t_end);
@@ -264,6 +273,31 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     if (tid == 0) ok = mbar_wait(bar_mma, 0, status) ? 1 : 0;
     if (!__syncthreads_and(ok)) goto teardown;
     tc_fence_after();
+    {
+        // operand images for the chain: Q' = diag(gamma scale / |q|) Q per value head, and the
+        // fp16 K per key head (written by the first value head of its group)
+        uint8_t *qimg = item + kWsQ;
+        uint8_t *kimg = ws_k + ((size_t)hk * slots + id) * kWsKItem;
+        const bool write_k = (h % (Hv / Hk)) == 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int idx = e * NT + tid, half = idx / 512, within = idx % 512, r = within / 8;
+            uint4 qv = *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + (2 * half + 1) * TILE + within * 16);
+            const __half2 *q2 = reinterpret_cast<const __half2 *>(&qv);
+            const float f = sGam[r] * sRq[r];
+            float qs[8];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float2 x = __half22float2(q2[w]);
+                qs[2 * w] = x.x * f;
+                qs[2 * w + 1] = x.y * f;
+            }
+            st_h8(qimg + half * TILE + within * 16, qs);
+            if (write_k)
+                *reinterpret_cast<uint4 *>(kimg + half * TILE + within * 16) =
+                    *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + 2 * half * TILE + within * 16);
+        }
+    }
     {
         // A (fp32, for the inverse) from K K^T; P (fp16 operand image, to the workspace) from Q K^T
         uint32_t r32[32];
@@ -366,13 +400,12 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                     kk > 0);
         tc_commit(bar_mma);
     }
-    // vectors for the chain: gamma_r scale/|q_r|, gamma_C/gamma_s/|k_s|, gamma_C
+    // vectors for the chain: gamma_C / gamma_s / |k_s| and gamma_C
     if (tid < 64) {
         float *wv = reinterpret_cast<float *>(item + kWsVec);
         const float G_last = sG[L - 1];
-        wv[tid] = sGam[tid] * sRq[tid];
-        wv[64 + tid] = tid < L ? __expf(G_last - sG[tid]) * sRk[tid] : 0.0f;
-        if (tid == 0) wv[128] = __expf(G_last);
+        wv[tid] = tid < L ? __expf(G_last - sG[tid]) * sRk[tid] : 0.0f;
+        if (tid == 0) wv[64] = __expf(G_last);
     }
     if (tid == 0) ok = mbar_wait(bar_mma, 1, status) ? 1 : 0;
     if (!__syncthreads_and(ok)) goto teardown;
@@ -406,27 +439,33 @@ teardown:
 // ===================================================================================
 // Chain kernel: one CTA per (value head, sequence), chunks in order, double-buffered.
 // ===================================================================================
-constexpr int B_W = 0, B_U = 16384, B_P = 32768, B_VEC = 40960, B_KQ = 41984;   // within a chunk buffer
-constexpr int BUF = B_KQ + 4 * TILE;                                           // 74752 B
-constexpr int CH_OFF_BUF0 = 0;
-constexpr int CH_OFF_S = 2 * BUF;                 // S0 fp16 [S_lo: 128 rows x 64][S_hi]
-constexpr int CH_OFF_UA = CH_OFF_S + 4 * TILE;    // U^T fp16 [i][s]
-constexpr int CH_OFF_US = CH_OFF_UA + 2 * TILE;   // U_S^T fp16 [i][s]
-constexpr int CH_OFF_BAR = CH_OFF_US + 2 * TILE;
+constexpr int B_W = 0, B_U = 16384, B_P = 32768, B_Q = 40960, B_VEC = 57344, B_K = 58368;  // within a buffer
+constexpr int BUF = B_K + 2 * TILE;                                                        // 74752 B
+constexpr int CH_OFF_STAGE = 2 * BUF;            // o staging, [r][i] (bf16 or fp32)
+constexpr int CH_OFF_BAR = CH_OFF_STAGE + 64 * 128 * 4;
 constexpr int CH_SMEM = CH_OFF_BAR + 128 + 1024;
 static_assert(CH_SMEM <= 232448, "chain shared memory");
-static_assert(BUF % 1024 == 0 && B_KQ % 1024 == 0, "1024-byte aligned tiles");
-constexpr uint32_t C_TM_D4 = 0, C_TM_D5 = 64, C_TM_D6 = 128, C_TM_D7 = 192;
+static_assert(BUF % 1024 == 0 && B_K % 1024 == 0 && B_Q % 1024 == 0, "1024-byte aligned operand tiles");
+// tensor memory: fp32 accumulators D4 (U), D5 (o), D7 (state update); fp16 A operands
+constexpr uint32_t C_TM_D4 = 0, C_TM_D5 = 64, C_TM_D7 = 128, C_TM_SA = 256 /* x2 */, C_TM_UA = 384, C_TM_US = 416;
+
+// tcgen05.mma kind::f16 with the A operand in tensor memory (M = 128, K-major rows on lanes).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
 
 __global__ void __launch_bounds__(NT, 1)
-gdn_chunk_chain_kernel(const __grid_constant__ Maps maps, const int32_t *__restrict__ cu_seqlens, int32_t T,
-                       int32_t Hk, int32_t Hv, int32_t slots, int32_t out_bf16, const float *S0g, float *S_out,
-                       void *__restrict__ o, const uint8_t *__restrict__ ws, int *status) {
+gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_t Hk, int32_t Hv, int32_t slots,
+                       int32_t out_bf16, const float *S0g, float *S_out, void *__restrict__ o,
+                       const uint8_t *__restrict__ ws, const uint8_t *__restrict__ ws_k, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CH_OFF_BAR);
-    uint64_t *full = bars, *bar_u = bars + 2, *bar_o5 = bars + 3, *bar_s = bars + 4, *bar_o6 = bars + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+    uint64_t *full = bars, *bar_u = bars + 2, *bar_s = bars + 3, *bar_o = bars + 4;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 5);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int wg = warp / 4;
@@ -442,14 +481,14 @@ gdn_chunk_chain_kernel(const __grid_constant__ Maps maps, const int32_t *__restr
     const int nchunks = (t_end - t_begin + C - 1) / C;
     const int slot0 = t_begin / C + n;
     const uint8_t *ws_h = ws + (size_t)h * slots * kWsItem;
+    const uint8_t *ws_kh = ws_k + (size_t)hk * slots * kWsKItem;
 
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
         mbar_init(bar_u, 1);
-        mbar_init(bar_o5, 1);
         mbar_init(bar_s, 1);
-        mbar_init(bar_o6, 1);
+        mbar_init(bar_o, 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -462,19 +501,16 @@ gdn_chunk_chain_kernel(const __grid_constant__ Maps maps, const int32_t *__restr
     const uint32_t tmem = *tmem_slot;
 
     auto issue_chunk = [&](int c) {
-        uint8_t *buf = sm + CH_OFF_BUF0 + (c & 1) * BUF;
+        uint8_t *buf = sm + (c & 1) * BUF;
         uint64_t *bar = &full[c & 1];
         const uint8_t *item = ws_h + (size_t)(slot0 + c) * kWsItem;
-        const int t0 = t_begin + c * C;
         mbar_arrive_expect_tx(bar, BUF);
         bulk_load(buf + B_W, item + kWsW, 16384, bar);
         bulk_load(buf + B_U, item + kWsU, 16384, bar);
         bulk_load(buf + B_P, item + kWsP, 8192, bar);
+        bulk_load(buf + B_Q, item + kWsQ, 16384, bar);
         bulk_load(buf + B_VEC, item + kWsVec, 1024, bar);
-        tma_load_3d(buf + B_KQ + 0 * TILE, &maps.k, bar, 0, hk, t0);
-        tma_load_3d(buf + B_KQ + 1 * TILE, &maps.q, bar, 0, hk, t0);
-        tma_load_3d(buf + B_KQ + 2 * TILE, &maps.k, bar, 64, hk, t0);
-        tma_load_3d(buf + B_KQ + 3 * TILE, &maps.q, bar, 64, hk, t0);
+        bulk_load(buf + B_K, ws_kh + (size_t)(slot0 + c) * kWsKItem, 16384, bar);
     };
     if (tid == 0 && nchunks > 0) issue_chunk(0);
 
@@ -493,97 +529,128 @@ gdn_chunk_chain_kernel(const __grid_constant__ Maps maps, const int32_t *__restr
             for (int c = 0; c < 64; ++c) S[c] = 0.0f;
         }
     }
-    auto write_S_smem = [&]() {
-        uint8_t *half = sm + CH_OFF_S + wg * 2 * TILE;
+    // fp16 copy of S as the A operand (row i on lane i, key index j packed two per column)
+    auto store_S = [&](int b) {
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_h8(half + swz(row, ch), &S[ch * 8]);
+        for (int part = 0; part < 2; ++part) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) pk[w] = pack_h2(S[part * 32 + 2 * w], S[part * 32 + 2 * w + 1]);
+            tmem_st16(tmem + lane_base + C_TM_SA + b * 64 + wg * 32 + part * 16, pk);
+        }
     };
-    write_S_smem();
+    store_S(0);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+
+    // o of a finished chunk: D5 (o^T, fp32) -> [r][i] staging -> 16-byte row stores
+    auto emit_o = [&](int c) {
+        const int t0 = t_begin + c * C;
+        const int L = min(C, t_end - t0);
+        uint32_t a5[32];
+        tmem_ld32(tmem + C_TM_D5 + lane_base + wg * 32, a5);
+        tmem_ld_wait();
+        uint8_t *stage = sm + CH_OFF_STAGE;
+        if (out_bf16) {
+            __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(stage);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) st[(wg * 32 + j) * D + row] = __float2bfloat16_rn(__uint_as_float(a5[j]));
+        } else {
+            float *st = reinterpret_cast<float *>(stage);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) st[(wg * 32 + j) * D + row] = __uint_as_float(a5[j]);
+        }
+        __syncthreads();
+        const int row_bytes = out_bf16 ? D * 2 : D * 4;
+        const int per_row = row_bytes / 16;
+        uint8_t *ob = static_cast<uint8_t *>(o);
+        for (int e = tid; e < L * per_row; e += NT) {
+            const int r = e / per_row, ch = e % per_row;
+            const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + ch * 16);
+            *reinterpret_cast<uint4 *>(ob + (((size_t)(t0 + r) * Hv + h) * D) * (row_bytes / D) + ch * 16) = val;
+        }
+    };
 
     bool alive = true;
+    int ok = 1;
     for (int c = 0; c < nchunks; ++c) {
         const int t0 = t_begin + c * C;
         const int L = min(C, t_end - t0);
-        uint8_t *buf = sm + CH_OFF_BUF0 + (c & 1) * BUF;
+        const int b = c & 1;
+        uint8_t *buf = sm + b * BUF;
         const float *vec = reinterpret_cast<const float *>(buf + B_VEC);
         const uint32_t ph = (uint32_t)(c & 1);
 
-        int ok = 1;
-        if (tid == 0) ok = mbar_wait(&full[c & 1], (uint32_t)((c >> 1) & 1), status) ? 1 : 0;
+        // chunk c's operands have landed; chunk c-1's output products (MMA5/6) are done
+        if (tid == 0) {
+            ok = mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status) ? 1 : 0;
+            if (ok && c > 0) ok = mbar_wait(bar_o, ph ^ 1u, status) ? 1 : 0;
+        }
         if (!__syncthreads_and(ok)) { alive = false; break; }
-        // K and Q tiles to fp16 in place (8 chunks of 16 B per thread, lane-consecutive)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) convert16(buf + B_KQ + (e * NT + tid) * 16);
-        fence_proxy_async_smem();
-        __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            if (c + 1 < nchunks) issue_chunk(c + 1);
-            // MMA4: D4 = S0 W^T (A: S0 K-major over j; B: W image, MN-major over s)
+            // MMA4: D4 = S0 W^T (A: S0 fp16 in TMEM; B: W image, MN-major over the token s)
             const uint32_t id4 = idesc_f16(64, false, true, false);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint8_t *a = sm + CH_OFF_S + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
-                mma_f16(tmem + C_TM_D4, kdesc(a), mndesc(buf + B_W + kk * 2048, 0), id4, kk > 0);
-            }
+            for (int kk = 0; kk < 8; ++kk)
+                mma_f16_ts(tmem + C_TM_D4, tmem + C_TM_SA + b * 64 + kk * 8, mndesc(buf + B_W + kk * 2048, 0), id4, kk > 0);
             tc_commit(bar_u);
-            // MMA5: D5 = S0 Q^T
-            const uint32_t id5 = idesc_f16(64, false, false, false);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint8_t *a = sm + CH_OFF_S + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
-                const uint8_t *b = buf + B_KQ + TILE + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
-                mma_f16(tmem + C_TM_D5, kdesc(a), kdesc(b), id5, kk > 0);
+            if (c + 1 < nchunks) {   // its buffer's last readers (chunk c-1) are done
+                fence_proxy_async_smem();
+                issue_chunk(c + 1);
             }
-            tc_commit(bar_o5);
         }
+        if (c > 0) emit_o(c - 1);   // overlaps MMA4
+
         if (tid == 0) ok = mbar_wait(bar_u, ph, status) ? 1 : 0;
         if (!__syncthreads_and(ok)) { alive = false; break; }
         tc_fence_after();
         {
-            // U^T = U~^T - D4 -> U_A = U^T, U_S = U^T diag(gamma_C / gamma / |k|) (fp16 [i][s])
+            // U^T = U~^T - D4; U_A = U^T and U_S = U^T diag(gamma_C / gamma / |k|) as fp16 A operands
             uint32_t r32[32];
             tmem_ld32(tmem + C_TM_D4 + lane_base + wg * 32, r32);
             tmem_ld_wait();
             const __half *ut = reinterpret_cast<const __half *>(buf + B_U);
-            float ua[32], us[32];
+            uint32_t ua[16], us[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int s = wg * 32 + j;
-                const float u = (s < L) ? __half2float(ut[s * D + row]) - __uint_as_float(r32[j]) : 0.0f;
-                ua[j] = u;
-                us[j] = u * vec[64 + s];
+            for (int w = 0; w < 16; ++w) {
+                const int s0 = wg * 32 + 2 * w;
+                const float u0 = (s0 < L) ? __half2float(ut[s0 * D + row]) - __uint_as_float(r32[2 * w]) : 0.0f;
+                const float u1 = (s0 + 1 < L) ? __half2float(ut[(s0 + 1) * D + row]) - __uint_as_float(r32[2 * w + 1]) : 0.0f;
+                ua[w] = pack_h2(u0, u1);
+                us[w] = pack_h2(u0 * vec[s0], u1 * vec[s0 + 1]);
             }
-            uint8_t *UA = sm + CH_OFF_UA, *US = sm + CH_OFF_US;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                st_h8(UA + swz(row, wg * 4 + ch), &ua[ch * 8]);
-                st_h8(US + swz(row, wg * 4 + ch), &us[ch * 8]);
-            }
+            tmem_st16(tmem + lane_base + C_TM_UA + wg * 16, ua);
+            tmem_st16(tmem + lane_base + C_TM_US + wg * 16, us);
+            tmem_st_wait();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            // MMA7: D7 = U_S^T K (B: K, MN-major over j); MMA6: D6 = U^T P^T
+            // MMA7: D7 = U_S^T K (B: K image, MN-major over j)
             const uint32_t id7 = idesc_f16(128, false, true, false);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + C_TM_D7, kdesc(sm + CH_OFF_US + kk * 32), mndesc(buf + B_KQ + kk * 2048, 2 * TILE), id7,
-                        kk > 0);
+                mma_f16_ts(tmem + C_TM_D7, tmem + C_TM_US + kk * 8, mndesc(buf + B_K + kk * 2048, TILE), id7, kk > 0);
             tc_commit(bar_s);
-            const uint32_t id6 = idesc_f16(64, false, false, false);
+            // MMA5: D5 = S0 Q'^T ; MMA6: D5 += U^T P^T
+            const uint32_t id5 = idesc_f16(64, false, false, false);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_f16_ts(tmem + C_TM_D5, tmem + C_TM_SA + b * 64 + kk * 8,
+                           kdesc(buf + B_Q + (kk < 4 ? 0 : TILE) + (kk & 3) * 32), id5, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + C_TM_D6, kdesc(sm + CH_OFF_UA + kk * 32), kdesc(buf + B_P + kk * 32), id6, kk > 0);
-            tc_commit(bar_o6);
+                mma_f16_ts(tmem + C_TM_D5, tmem + C_TM_UA + kk * 8, kdesc(buf + B_P + kk * 32), id5, 1u);
+            tc_commit(bar_o);
         }
         if (tid == 0) ok = mbar_wait(bar_s, ph, status) ? 1 : 0;
         if (!__syncthreads_and(ok)) { alive = false; break; }
         tc_fence_after();
         {
-            const float gC = vec[128];
+            const float gC = vec[64];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t r7[32];
@@ -592,49 +659,21 @@ gdn_chunk_chain_kernel(const __grid_constant__ Maps maps, const int32_t *__restr
 #pragma unroll
                 for (int j = 0; j < 32; ++j) S[half * 32 + j] = gC * S[half * 32 + j] + __uint_as_float(r7[j]);
             }
+            store_S(b ^ 1);   // S0 of chunk c + 1 (its slot was last read by chunk c-1's MMAs)
+            tmem_st_wait();
         }
-        if (tid == 0) ok = mbar_wait(bar_o6, ph, status) ? 1 : 0;
-        if (!__syncthreads_and(ok)) { alive = false; break; }
-        tc_fence_after();
-        write_S_smem();   // the next chunk's S0 (MMA4/5 of this chunk are complete)
-        {
-            // o^T = D5 diag(gamma scale / |q|) + D6, staged as [r][i] in the (now free) U area,
-            // then written with 16-byte row-contiguous stores (rows r < L only)
-            uint32_t a5[32], a6[32];
-            tmem_ld32(tmem + C_TM_D5 + lane_base + wg * 32, a5);
-            tmem_ld32(tmem + C_TM_D6 + lane_base + wg * 32, a6);
-            tmem_ld_wait();
-            uint8_t *stage = sm + CH_OFF_UA;
-            if (out_bf16) {
-                __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(stage);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int r = wg * 32 + j;
-                    st[r * D + row] = __float2bfloat16_rn(__uint_as_float(a5[j]) * vec[r] + __uint_as_float(a6[j]));
-                }
-            } else {
-                float *st = reinterpret_cast<float *>(stage);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int r = wg * 32 + j;
-                    st[r * D + row] = __uint_as_float(a5[j]) * vec[r] + __uint_as_float(a6[j]);
-                }
-            }
-            __syncthreads();
-            const int row_bytes = out_bf16 ? D * 2 : D * 4;
-            const int per_row = row_bytes / 16;
-            uint8_t *ob = static_cast<uint8_t *>(o);
-            for (int e = tid; e < L * per_row; e += NT) {
-                const int r = e / per_row, ch = e % per_row;
-                const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + ch * 16);
-                *reinterpret_cast<uint4 *>(ob + (((size_t)(t0 + r) * Hv + h) * D) * (row_bytes / D) + ch * 16) = val;
-            }
-        }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
     }
-
+    if (alive && nchunks > 0) {
+        if (tid == 0) ok = mbar_wait(bar_o, (uint32_t)((nchunks - 1) & 1), status) ? 1 : 0;
+        if (__syncthreads_and(ok)) {
+            tc_fence_after();
+            emit_o(nchunks - 1);
+        } else {
+            alive = false;
+        }
+    }
     if (alive && S_out) {
         const size_t base = (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
 #pragma unroll
@@ -696,14 +735,15 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
     }
     const int slots = c.T / kChunk + c.num_seqs;
     uint8_t *ws = static_cast<uint8_t *>(c.ws);
+    uint8_t *ws_k = ws + ws_value_region(c.T, c.num_seqs, c.Hv);
     gdn_chunk_prep_kernel<<<dim3(slots, c.Hv), NT, P_SMEM, st>>>(maps, c.a, c.b, c.A_log, c.dt_bias, c.cu_seqlens, c.T,
                                                                  c.num_seqs, c.Hk, c.Hv, slots, c.scale, c.l2norm, ws,
-                                                                 c.status);
+                                                                 ws_k, c.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    gdn_chunk_chain_kernel<<<dim3(c.Hv, c.num_seqs), NT, CH_SMEM, st>>>(maps, c.cu_seqlens, c.T, c.Hk, c.Hv, slots,
+    gdn_chunk_chain_kernel<<<dim3(c.Hv, c.num_seqs), NT, CH_SMEM, st>>>(c.cu_seqlens, c.T, c.Hk, c.Hv, slots,
                                                                         c.out_bf16 ? 1 : 0, c.S0, c.S_out, c.o, ws,
-                                                                        c.status);
+                                                                        ws_k, c.status);
     return cudaGetLastError();
 }
 

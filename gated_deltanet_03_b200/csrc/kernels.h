@@ -33,10 +33,10 @@ struct ChunkedArgs {
     const float *S0;
     float *S_out;
     void *o;
-    void *ws;                    // workspace of chunked_workspace_bytes(T, num_seqs, Hv) bytes
+    void *ws;                    // workspace of chunked_workspace_bytes(T, num_seqs, Hk, Hv) bytes
     int *status;
 };
-size_t chunked_workspace_bytes(int T, int num_seqs, int Hv);
+size_t chunked_workspace_bytes(int T, int num_seqs, int Hk, int Hv);
 cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st);
 
 struct TailArgs {
