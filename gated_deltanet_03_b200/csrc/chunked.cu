@@ -10,32 +10,30 @@
 //   W = T diag(beta gamma) K,   U~ = T diag(beta) V,     U = U~ - W S0^T,
 //   O = diag(gamma) Q S0^T + (Q K^T o Gamma) U,          Gamma_rs = exp(G_r - G_s), s <= r,
 //   S_C = gamma_C S0 + U^T diag(gamma_C / gamma) K.
-// W, U~ and P = (Q K^T o Gamma) do not depend on the state: the prep kernel computes them
-// for every chunk at once and writes them to the caller's workspace; the chain kernel then
-// only runs the four state-dependent products per chunk.
+// W, U~, P = (Q K^T o Gamma) and the scaled Q and K do not depend on the state: the prep
+// kernel computes them for every chunk at once into the caller's workspace; the chain
+// kernel then runs two state-dependent MMAs per chunk.
 //
 // The L2 norms of q and k never touch an MMA operand: raw bf16 inputs (exact in fp16) feed
 // the tensor cores and 1/|k|, scale/|q| enter as diagonal factors of the derived operands.
-// Derived operands (T', T'', W, U~, U, P, S0) are staged in fp16 (11-bit significand) with
-// fp32 accumulation in tensor memory; the state itself stays fp32 in registers.
+// Derived operands are staged in fp16 (11-bit significand) with fp32 accumulation in tensor
+// memory; the state itself stays fp32 in registers.
 //
-// Every MMA has M = 128 by working transposed (value or key index on the TMEM lanes):
-//   prep   MMA1  D1[128 x 64] = [K; Q] K^T        (K K^T rows 0-63, Q K^T rows 64-127)
-//          MMA2  D2 = W^T  = K^T T'^T               T'  = T diag(beta gamma / |k|)
-//          MMA3  D3 = U~^T = V^T T''^T              T'' = T diag(beta)
-//   chain  MMA4  D4 = S0 W^T      -> U^T = U~^T - D4
-//          MMA7  D7 = U_S^T K     U_S = U diag(gamma_C / gamma / |k|)
-//          MMA5  D5 = S0 Q'^T     Q' = diag(gamma scale / |q|) Q
-//          MMA6  D5 += U^T P^T    P = Q K^T o Gamma / (|q| |k|) * scale
-// then o^T = D5 and S <- gamma_C S + D7. In the chain the fp16 copies of S0 and U live in
-// tensor memory and are the A operands of their MMAs (no shared-memory round trip).
+// Every MMA has M = 128 (value or key index on the TMEM lanes):
+//   prep   MMA1  D1 = [K; Q] [K; Q]^T      (rows 0-63: K K^T | K Q^T)
+//          MMA2  D2 = W^T  = K^T T'^T      T'  = T diag(beta gamma / |k|)
+//          MMA3  D3 = U~^T = V^T T''^T     T'' = T diag(beta)
+//   chain  MMA45 [D4 | D5a] = S0 [W; Q']^T            Q' = diag(gamma scale / |q|) Q
+//          MMA67 [D7 | D5b] = U^T [K''; P^T]^T        K'' = diag(gamma_C / gamma / |k|) K
+//                                                     P^T[s][r] = k_s.q_r Gamma_rs scale / (|q_r| |k_s|)
+//   with U^T = U~^T - D4, S <- gamma_C S + D7, o^T = D5a + D5b. In the chain the fp16 copies of
+//   S0 and U live in tensor memory as the A operands; one warp issues the copies and MMAs,
+//   eight warps do the element-wise work, and they hand over through mbarriers.
 //
-// Workspace: one 57 KB item per (value head, chunk slot): the W operand image (fp16,
-// [key j][token s], 128-byte swizzled rows), U~ (fp16, [token s][value i]), the P operand
-// image (fp16, [r][s] swizzled), the Q' = diag(gamma scale / |q|) Q operand image and fp32
-// vectors (gamma_C / gamma_s / |k_s|, gamma_C); and one 16 KB fp16 K operand image per (key
-// head, chunk slot). Chunk c of sequence n uses slot cu_seqlens[n] / 64 + n + c, so slots
-// never collide and T / 64 + num_seqs slots per head suffice.
+// Workspace: one 73 KB item per (value head, chunk slot): [W; Q'] (fp16, K-major, 128 rows,
+// 128-byte swizzled), [K''; P^T] (fp16, three 64-wide MN-major blocks), U~ (fp16 [s][i]) and
+// gamma_C. Chunk c of sequence n uses slot cu_seqlens[n] / 64 + n + c, so slots never
+// collide and T / 64 + num_seqs slots per head suffice.
 #include <mutex>
 
 #include "common.cuh"
@@ -44,24 +42,19 @@
 namespace gdn {
 
 constexpr int kChunk = 64;
-// per (value head, slot): W image, U~, P image, Q' image, vectors
-constexpr int kWsItem = 58368;
-constexpr int kWsW = 0, kWsU = 16384, kWsP = 32768, kWsQ = 40960, kWsVec = 57344;
-// per (key head, slot): the fp16 K image
-constexpr int kWsKItem = 16384;
+constexpr int kWsItem = 74752;
+constexpr int kWsWQ = 0, kWsKP = 32768, kWsU = 57344, kWsVec = 73728;
 
-static size_t ws_value_region(int T, int num_seqs, int Hv) {
-    return (size_t)Hv * (size_t)(T / kChunk + num_seqs) * kWsItem;
-}
 size_t chunked_workspace_bytes(int T, int num_seqs, int Hk, int Hv) {
-    return ws_value_region(T, num_seqs, Hv) + (size_t)Hk * (size_t)(T / kChunk + num_seqs) * kWsKItem;
+    (void)Hk;
+    return (size_t)Hv * (size_t)(T / kChunk + num_seqs) * kWsItem;
 }
 
 namespace {
 
 constexpr int C = kChunk;      // chunk length
 constexpr int D = 128;         // head size
-constexpr int NT = 256;        // threads per CTA
+constexpr int NT = 256;        // element-wise threads per CTA
 constexpr int TILE = C * 128;  // 64 rows x 128 B: one half (64 columns) of a 64 x 128 16-bit tile
 
 // kind::f16 instruction descriptor: fp16 A/B, fp32 accumulate, M = 128.
@@ -158,25 +151,26 @@ __device__ __forceinline__ void locate(int id, const int32_t *cu, int num_seqs, 
 // ===================================================================================
 // Prep kernel: one CTA per (chunk slot, value head); two CTAs per SM.
 // ===================================================================================
-constexpr int P_OFF_KQ = 0;                     // [K_lo][Q_lo][K_hi][Q_hi], bf16 -> fp16 in place
-constexpr int P_OFF_V = 4 * TILE;               // [V_lo][V_hi]
-constexpr int P_OFF_TP = 6 * TILE;              // T'  [s][r] fp16, swizzled
-constexpr int P_OFF_TPP = 7 * TILE;             // T'' [s][r] fp16, swizzled
-constexpr int P_OFF_AF = 8 * TILE;              // A fp32 [64][65]
+constexpr int P_OFF_KQ = 0;                       // [K_lo][Q_lo][K_hi][Q_hi], bf16 -> fp16 in place
+constexpr int P_OFF_V = 4 * TILE;                 // [V_lo][V_hi]
+constexpr int P_OFF_TP = 6 * TILE;                // T'  [s][r] fp16, swizzled
+constexpr int P_OFF_TPP = 7 * TILE;               // T'' [s][r] fp16, swizzled
+constexpr int P_OFF_AF = 8 * TILE;                // A fp32 [64][65]
 constexpr int P_OFF_TF = P_OFF_AF + 64 * 65 * 4;  // T fp32 [64][65]
 constexpr int P_OFF_XF = P_OFF_TF + 64 * 65 * 4;  // X fp32 [3][256]
-constexpr int P_OFF_VEC = P_OFF_XF + 3 * 256 * 4; // G, beta, rk, rq, gamma (64 each), row sums of squares (128)
+constexpr int P_OFF_STG = P_OFF_AF;               // W and U~ staging once A and T are dead (32 KB)
+constexpr int P_OFF_VEC = P_OFF_XF + 3 * 256 * 4; // G, beta, rk, rq, gamma, decS (64 each), row sums of squares (128)
 constexpr int P_OFF_BAR = P_OFF_VEC + 8 * 64 * 4;
 constexpr int P_SMEM = P_OFF_BAR + 64 + 1024;
 static_assert(P_SMEM * 2 <= 228 * 1024, "two prep CTAs per SM");
-constexpr uint32_t P_TM_D1 = 0, P_TM_D2 = 64, P_TM_D3 = 128;
+static_assert(P_OFF_XF - P_OFF_AF >= 4 * TILE, "staging fits in the A/T scratch");
+constexpr uint32_t P_TM_D1 = 0, P_TM_D2 = 128, P_TM_D3 = 192;
 
 __global__ void __launch_bounds__(NT, 2)
 gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict__ ga, const float *__restrict__ gb,
                       const float *__restrict__ A_log, const float *__restrict__ dt_bias,
                       const int32_t *__restrict__ cu_seqlens, int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv,
-                      int32_t slots, float scale, int32_t l2norm, uint8_t *__restrict__ ws,
-                      uint8_t *__restrict__ ws_k, int *status) {
+                      int32_t slots, float scale, int32_t l2norm, uint8_t *__restrict__ ws, int *status) {
     const int id = blockIdx.x, h = blockIdx.y;
     int n, t_begin, t_end;
     locate(id, cu_seqlens, num_seqs, T, n, t_begin, t_end);
@@ -189,7 +183,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *vec = reinterpret_cast<float *>(sm + P_OFF_VEC);
-    float *sG = vec, *sBeta = vec + 64, *sRk = vec + 128, *sRq = vec + 192, *sGam = vec + 256, *sSS = vec + 320;
+    float *sG = vec, *sBeta = vec + 64, *sRk = vec + 128, *sRq = vec + 192, *sGam = vec + 256, *sDec = vec + 320,
+          *sSS = vec + 384;
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + P_OFF_BAR);
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 2);
@@ -256,7 +251,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     __syncthreads();
     if (tid == 0) {
         tc_fence_after();
-        const uint32_t id1 = idesc_f16(64, false, false, false);
+        const uint32_t id1 = idesc_f16(128, false, false, false);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint8_t *abase = sm + P_OFF_KQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
@@ -270,61 +265,65 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         sRq[tid] = v ? (l2norm ? rsqrtf(sSS[64 + tid] + 1e-6f) * scale : scale) : 0.0f;
         sGam[tid] = v ? expf(sG[tid]) : 0.0f;
     }
+    __syncthreads();
+    if (tid < 64) sDec[tid] = tid < L ? __expf(sG[L - 1] - sG[tid]) * sRk[tid] : 0.0f;
+    if (tid == 0) {
+        float *wv = reinterpret_cast<float *>(item + kWsVec);
+        wv[0] = __expf(sG[L - 1]);   // gamma_C
+    }
     if (tid == 0) ok = mbar_wait(bar_mma, 0, status) ? 1 : 0;
     if (!__syncthreads_and(ok)) goto teardown;
     tc_fence_after();
     {
-        // operand images for the chain: Q' = diag(gamma scale / |q|) Q per value head, and the
-        // fp16 K per key head (written by the first value head of its group)
-        uint8_t *qimg = item + kWsQ;
-        uint8_t *kimg = ws_k + ((size_t)hk * slots + id) * kWsKItem;
-        const bool write_k = (h % (Hv / Hk)) == 0;
+        // Q' rows (64 + r of the [W; Q'] image) and K'' (the first two blocks of [K''; P^T]):
+        // the converted tiles scaled row by row, swizzle positions unchanged
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int idx = e * NT + tid, half = idx / 512, within = idx % 512, r = within / 8;
-            uint4 qv = *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + (2 * half + 1) * TILE + within * 16);
-            const __half2 *q2 = reinterpret_cast<const __half2 *>(&qv);
-            const float f = sGam[r] * sRq[r];
-            float qs[8];
+        for (int e = 0; e < 8; ++e) {
+            const int idx = e * NT + tid;          // 2048 chunks: 1024 of Q, 1024 of K
+            const int isk = idx >> 10, w = idx & 1023, half = w >> 9, within = w & 511, r = within >> 3;
+            const uint8_t *src = sm + P_OFF_KQ + (2 * half + (isk ? 0 : 1)) * TILE + within * 16;
+            const float f = isk ? sDec[r] : sGam[r] * sRq[r];
+            const uint4 hv = *reinterpret_cast<const uint4 *>(src);
+            const __half2 *h2 = reinterpret_cast<const __half2 *>(&hv);
+            float x[8];
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float2 x = __half22float2(q2[w]);
-                qs[2 * w] = x.x * f;
-                qs[2 * w + 1] = x.y * f;
+            for (int q2 = 0; q2 < 4; ++q2) {
+                const float2 t = __half22float2(h2[q2]);
+                x[2 * q2] = t.x * f;
+                x[2 * q2 + 1] = t.y * f;
             }
-            st_h8(qimg + half * TILE + within * 16, qs);
-            if (write_k)
-                *reinterpret_cast<uint4 *>(kimg + half * TILE + within * 16) =
-                    *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + 2 * half * TILE + within * 16);
+            uint8_t *dst = isk ? item + kWsKP + half * TILE + within * 16
+                               : item + kWsWQ + half * 2 * TILE + TILE + within * 16;
+            st_h8(dst, x);
         }
-    }
-    {
-        // A (fp32, for the inverse) from K K^T; P (fp16 operand image, to the workspace) from Q K^T
-        uint32_t r32[32];
-        const int col0 = wg * 32;
-        tmem_ld32(tmem + P_TM_D1 + lane_base + col0, r32);
-        tmem_ld_wait();
+        // rows s of D1 (lanes 0-63): K K^T (warps 0-1) -> column s of A; K Q^T (warps 4-5) -> P^T row s
         if (row < 64) {
-            const int r = row;
-            const float Gr = sG[r], br = sBeta[r] * sRk[r];
+            const int s = row;
+            const float Gs = sG[s], rks = sRk[s];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int s = col0 + j;
-                float a = 0.0f;
-                if (s < r && r < L) a = br * __expf(Gr - sG[s]) * __uint_as_float(r32[j]) * sRk[s];
-                Af[r * 65 + s] = a;
+            for (int hcol = 0; hcol < 2; ++hcol) {
+                uint32_t r32[32];
+                tmem_ld32(tmem + P_TM_D1 + lane_base + wg * 64 + hcol * 32, r32);
+                tmem_ld_wait();
+                if (wg == 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int r = hcol * 32 + j;
+                        float a = 0.0f;
+                        if (s < r && r < L) a = sBeta[r] * __expf(sG[r] - Gs) * __uint_as_float(r32[j]) * sRk[r] * rks;
+                        Af[r * 65 + s] = a;
+                    }
+                } else {
+                    float pv[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int r = hcol * 32 + j;
+                        pv[j] = (s <= r && r < L) ? __uint_as_float(r32[j]) * sRq[r] * rks * __expf(sG[r] - Gs) : 0.0f;
+                    }
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) st_h8(item + kWsKP + 2 * TILE + swz(s, hcol * 4 + ch), &pv[ch * 8]);
+                }
             }
-        } else {
-            const int r = row - 64;
-            const float Gr = sG[r], rqr = sRq[r];
-            float pv[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int s = col0 + j;
-                pv[j] = (s <= r && r < L) ? __uint_as_float(r32[j]) * rqr * sRk[s] * __expf(Gr - sG[s]) : 0.0f;
-            }
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) st_h8(item + kWsP + swz(r, wg * 4 + ch), &pv[ch * 8]);
         }
     }
     tc_fence_before();
@@ -400,32 +399,35 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                     kk > 0);
         tc_commit(bar_mma);
     }
-    // vectors for the chain: gamma_C / gamma_s / |k_s| and gamma_C
-    if (tid < 64) {
-        float *wv = reinterpret_cast<float *>(item + kWsVec);
-        const float G_last = sG[L - 1];
-        wv[tid] = tid < L ? __expf(G_last - sG[tid]) * sRk[tid] : 0.0f;
-        if (tid == 0) wv[64] = __expf(G_last);
-    }
     if (tid == 0) ok = mbar_wait(bar_mma, 1, status) ? 1 : 0;
     if (!__syncthreads_and(ok)) goto teardown;
     tc_fence_after();
     {
-        // W operand image: row j (this thread's TMEM lane), tokens s in 16-byte chunks
-        uint32_t r32[32];
-        tmem_ld32(tmem + P_TM_D2 + lane_base + wg * 32, r32);
+        // W^T (lane j) -> W K-major [s][j] and U~^T (lane i) -> U~ [s][i], transposed through
+        // shared memory (the A/T scratch is dead), then copied out in 16-byte chunks
+        uint8_t *stg = sm + P_OFF_STG;
+        __half *uts = reinterpret_cast<__half *>(stg + 2 * TILE);
+        uint32_t wv32[32], uv32[32];
+        tmem_ld32(tmem + P_TM_D2 + lane_base + wg * 32, wv32);
+        tmem_ld32(tmem + P_TM_D3 + lane_base + wg * 32, uv32);
         tmem_ld_wait();
-        float w[32];
+        const int j = row, hj = j >> 6, jj = j & 63;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) w[j] = __uint_as_float(r32[j]);
+        for (int q = 0; q < 32; ++q) {
+            const int s = wg * 32 + q;
+            *reinterpret_cast<__half *>(stg + hj * TILE + s * 128 + (((jj >> 3) ^ (s & 7)) << 4) + (jj & 7) * 2) =
+                __float2half_rn(__uint_as_float(wv32[q]));
+        }
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) st_h8(item + kWsW + swz(row, wg * 4 + ch), &w[ch * 8]);
-        // U~ as [s][i]
-        tmem_ld32(tmem + P_TM_D3 + lane_base + wg * 32, r32);
-        tmem_ld_wait();
-        __half *ut = reinterpret_cast<__half *>(item + kWsU);
+        for (int q = 0; q < 32; ++q) uts[(wg * 32 + q) * D + row] = __float2half_rn(__uint_as_float(uv32[q]));
+    }
+    __syncthreads();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ut[(wg * 32 + j) * D + row] = __float2half_rn(__uint_as_float(r32[j]));
+    for (int e = 0; e < 8; ++e) {
+        const int idx = e * NT + tid;   // 1024 chunks of W, then 1024 of U~
+        const uint8_t *src = sm + P_OFF_STG + idx * 16;
+        uint8_t *dst = idx < 1024 ? item + kWsWQ + (idx >> 9) * 2 * TILE + (idx & 511) * 16 : item + kWsU + (idx - 1024) * 16;
+        *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
     }
 teardown:
     tc_fence_before();
@@ -438,16 +440,16 @@ teardown:
 
 // ===================================================================================
 // Chain kernel: one CTA per (value head, sequence), chunks in order, double-buffered.
+// Warps 0-7: element-wise work; warp 8: bulk copies and MMA issue.
 // ===================================================================================
-constexpr int B_W = 0, B_U = 16384, B_P = 32768, B_Q = 40960, B_VEC = 57344, B_K = 58368;  // within a buffer
-constexpr int BUF = B_K + 2 * TILE;                                                        // 74752 B
-constexpr int CH_OFF_STAGE = 2 * BUF;            // o staging, [r][i] (bf16 or fp32)
+constexpr int CH_THREADS = NT + 32;
+constexpr int CH_OFF_STAGE = 2 * kWsItem;          // o staging, [r][i] (bf16 or fp32)
 constexpr int CH_OFF_BAR = CH_OFF_STAGE + 64 * 128 * 4;
 constexpr int CH_SMEM = CH_OFF_BAR + 128 + 1024;
 static_assert(CH_SMEM <= 232448, "chain shared memory");
-static_assert(BUF % 1024 == 0 && B_K % 1024 == 0 && B_Q % 1024 == 0, "1024-byte aligned operand tiles");
-// tensor memory: fp32 accumulators D4 (U), D5 (o), D7 (state update); fp16 A operands
-constexpr uint32_t C_TM_D4 = 0, C_TM_D5 = 64, C_TM_D7 = 128, C_TM_SA = 256 /* x2 */, C_TM_UA = 384, C_TM_US = 416;
+static_assert(kWsItem % 1024 == 0 && kWsKP % 1024 == 0, "1024-byte aligned operand tiles");
+// tensor memory: [D4 | D5a] (MMA45), [D7 | D5b] (MMA67), fp16 S0 (two slots) and U as A operands
+constexpr uint32_t C_TM_D45 = 0, C_TM_D67 = 128, C_TM_SA = 320, C_TM_UA = 448;
 
 // tcgen05.mma kind::f16 with the A operand in tensor memory (M = 128, K-major rows on lanes).
 __device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -457,22 +459,31 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t
         "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
 
-__global__ void __launch_bounds__(NT, 1)
-gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_t Hk, int32_t Hv, int32_t slots,
+// Barrier among the 256 element-wise threads only (named barrier 1), with an AND vote.
+__device__ __forceinline__ int workers_and(int pred) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, 1, 256, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred)
+        : "memory");
+    return r;
+}
+__device__ __forceinline__ void workers_sync() { asm volatile("barrier.cta.sync 2, 256;" ::: "memory"); }
+
+__global__ void __launch_bounds__(CH_THREADS, 1)
+gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_t Hv, int32_t slots,
                        int32_t out_bf16, const float *S0g, float *S_out, void *__restrict__ o,
-                       const uint8_t *__restrict__ ws, const uint8_t *__restrict__ ws_k, int *status) {
+                       const uint8_t *__restrict__ ws, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CH_OFF_BAR);
-    uint64_t *full = bars, *bar_u = bars + 2, *bar_s = bars + 3, *bar_o = bars + 4;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 5);
+    uint64_t *full = bars, *bar_u = bars + 2, *bar_s = bars + 3, *bar_uready = bars + 4, *bar_sready = bars + 5;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int wg = warp / 4;
-    const int row = (warp % 4) * 32 + lane;
-    const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
     const int h = blockIdx.x, n = blockIdx.y;
-    const int hk = h / (Hv / Hk);
     int t_begin = 0, t_end = T;
     if (cu_seqlens) {
         t_begin = cu_seqlens[n];
@@ -481,14 +492,14 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
     const int nchunks = (t_end - t_begin + C - 1) / C;
     const int slot0 = t_begin / C + n;
     const uint8_t *ws_h = ws + (size_t)h * slots * kWsItem;
-    const uint8_t *ws_kh = ws_k + (size_t)hk * slots * kWsKItem;
 
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
         mbar_init(bar_u, 1);
         mbar_init(bar_s, 1);
-        mbar_init(bar_o, 1);
+        mbar_init(bar_uready, 8);
+        mbar_init(bar_sready, 8);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -500,185 +511,163 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto issue_chunk = [&](int c) {
-        uint8_t *buf = sm + (c & 1) * BUF;
-        uint64_t *bar = &full[c & 1];
-        const uint8_t *item = ws_h + (size_t)(slot0 + c) * kWsItem;
-        mbar_arrive_expect_tx(bar, BUF);
-        bulk_load(buf + B_W, item + kWsW, 16384, bar);
-        bulk_load(buf + B_U, item + kWsU, 16384, bar);
-        bulk_load(buf + B_P, item + kWsP, 8192, bar);
-        bulk_load(buf + B_Q, item + kWsQ, 16384, bar);
-        bulk_load(buf + B_VEC, item + kWsVec, 1024, bar);
-        bulk_load(buf + B_K, ws_kh + (size_t)(slot0 + c) * kWsKItem, 16384, bar);
-    };
-    if (tid == 0 && nchunks > 0) issue_chunk(0);
-
-    // state: thread (TMEM lane i, column half wg) holds S[i][64 wg .. 64 wg + 63] in fp32
-    float S[64];
-    {
-        const size_t base = (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
-        if (S0g) {
+    if (warp == 8) {
+        // ------------------------------------------------ copy + MMA issue (one thread)
+        if (lane == 0) {
+            auto issue_chunk = [&](int c) {
+                uint64_t *bar = &full[c & 1];
+                mbar_arrive_expect_tx(bar, kWsItem);
+                bulk_load(sm + (c & 1) * kWsItem, ws_h + (size_t)(slot0 + c) * kWsItem, kWsItem, bar);
+            };
+            if (nchunks > 0) issue_chunk(0);
+            const uint32_t id45 = idesc_f16(128, false, false, false);
+            const uint32_t id67 = idesc_f16(192, false, true, false);
+            for (int c = 0; c < nchunks; ++c) {
+                const int b = c & 1;
+                const uint8_t *buf = sm + b * kWsItem;
+                if (!mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status)) break;
+                if (!mbar_wait(bar_sready, (uint32_t)(c & 1), status)) break;
+                tc_fence_after();
+                // [D4 | D5a] = S0 [W; Q']^T   (B: 128 K-major rows, K = 128 key columns)
 #pragma unroll
-            for (int c = 0; c < 64; c += 4) {
-                float4 x = *reinterpret_cast<const float4 *>(S0g + base + c);
-                S[c] = x.x; S[c + 1] = x.y; S[c + 2] = x.z; S[c + 3] = x.w;
-            }
-        } else {
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tmem + C_TM_D45, tmem + C_TM_SA + b * 64 + kk * 8,
+                               kdesc(buf + kWsWQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32), id45, kk > 0);
+                tc_commit(bar_u);
+                if (c + 1 < nchunks) {   // the other buffer's readers (chunk c-1) are done
+                    fence_proxy_async_smem();
+                    issue_chunk(c + 1);
+                }
+                if (!mbar_wait(bar_uready, (uint32_t)(c & 1), status)) break;
+                tc_fence_after();
+                // [D7 | D5b] = U^T [K''; P^T]^T   (B: three MN-major blocks of 64, K = 64 tokens)
 #pragma unroll
-            for (int c = 0; c < 64; ++c) S[c] = 0.0f;
-        }
-    }
-    // fp16 copy of S as the A operand (row i on lane i, key index j packed two per column)
-    auto store_S = [&](int b) {
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int w = 0; w < 16; ++w) pk[w] = pack_h2(S[part * 32 + 2 * w], S[part * 32 + 2 * w + 1]);
-            tmem_st16(tmem + lane_base + C_TM_SA + b * 64 + wg * 32 + part * 16, pk);
-        }
-    };
-    store_S(0);
-    tmem_st_wait();
-    tc_fence_before();
-    __syncthreads();
-
-    // o of a finished chunk: D5 (o^T, fp32) -> [r][i] staging -> 16-byte row stores
-    auto emit_o = [&](int c) {
-        const int t0 = t_begin + c * C;
-        const int L = min(C, t_end - t0);
-        uint32_t a5[32];
-        tmem_ld32(tmem + C_TM_D5 + lane_base + wg * 32, a5);
-        tmem_ld_wait();
-        uint8_t *stage = sm + CH_OFF_STAGE;
-        if (out_bf16) {
-            __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(stage);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) st[(wg * 32 + j) * D + row] = __float2bfloat16_rn(__uint_as_float(a5[j]));
-        } else {
-            float *st = reinterpret_cast<float *>(stage);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) st[(wg * 32 + j) * D + row] = __uint_as_float(a5[j]);
-        }
-        __syncthreads();
-        const int row_bytes = out_bf16 ? D * 2 : D * 4;
-        const int per_row = row_bytes / 16;
-        uint8_t *ob = static_cast<uint8_t *>(o);
-        for (int e = tid; e < L * per_row; e += NT) {
-            const int r = e / per_row, ch = e % per_row;
-            const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + ch * 16);
-            *reinterpret_cast<uint4 *>(ob + (((size_t)(t0 + r) * Hv + h) * D) * (row_bytes / D) + ch * 16) = val;
-        }
-    };
-
-    bool alive = true;
-    int ok = 1;
-    for (int c = 0; c < nchunks; ++c) {
-        const int t0 = t_begin + c * C;
-        const int L = min(C, t_end - t0);
-        const int b = c & 1;
-        uint8_t *buf = sm + b * BUF;
-        const float *vec = reinterpret_cast<const float *>(buf + B_VEC);
-        const uint32_t ph = (uint32_t)(c & 1);
-
-        // chunk c's operands have landed; chunk c-1's output products (MMA5/6) are done
-        if (tid == 0) {
-            ok = mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status) ? 1 : 0;
-            if (ok && c > 0) ok = mbar_wait(bar_o, ph ^ 1u, status) ? 1 : 0;
-        }
-        if (!__syncthreads_and(ok)) { alive = false; break; }
-        if (tid == 0) {
-            tc_fence_after();
-            // MMA4: D4 = S0 W^T (A: S0 fp16 in TMEM; B: W image, MN-major over the token s)
-            const uint32_t id4 = idesc_f16(64, false, true, false);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_f16_ts(tmem + C_TM_D4, tmem + C_TM_SA + b * 64 + kk * 8, mndesc(buf + B_W + kk * 2048, 0), id4, kk > 0);
-            tc_commit(bar_u);
-            if (c + 1 < nchunks) {   // its buffer's last readers (chunk c-1) are done
-                fence_proxy_async_smem();
-                issue_chunk(c + 1);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16_ts(tmem + C_TM_D67, tmem + C_TM_UA + kk * 8, mndesc(buf + kWsKP + kk * 2048, TILE), id67,
+                               kk > 0);
+                tc_commit(bar_s);
             }
         }
-        if (c > 0) emit_o(c - 1);   // overlaps MMA4
-
-        if (tid == 0) ok = mbar_wait(bar_u, ph, status) ? 1 : 0;
-        if (!__syncthreads_and(ok)) { alive = false; break; }
-        tc_fence_after();
+    } else {
+        // ------------------------------------------------ element-wise work (256 threads)
+        const int wg = warp / 4;
+        const int row = (warp % 4) * 32 + lane;   // TMEM lane == value index i
+        const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
+        float S[64];   // S[i][64 wg .. 64 wg + 63], fp32
         {
-            // U^T = U~^T - D4; U_A = U^T and U_S = U^T diag(gamma_C / gamma / |k|) as fp16 A operands
-            uint32_t r32[32];
-            tmem_ld32(tmem + C_TM_D4 + lane_base + wg * 32, r32);
-            tmem_ld_wait();
-            const __half *ut = reinterpret_cast<const __half *>(buf + B_U);
-            uint32_t ua[16], us[16];
+            const size_t base = (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
+            if (S0g) {
 #pragma unroll
-            for (int w = 0; w < 16; ++w) {
-                const int s0 = wg * 32 + 2 * w;
-                const float u0 = (s0 < L) ? __half2float(ut[s0 * D + row]) - __uint_as_float(r32[2 * w]) : 0.0f;
-                const float u1 = (s0 + 1 < L) ? __half2float(ut[(s0 + 1) * D + row]) - __uint_as_float(r32[2 * w + 1]) : 0.0f;
-                ua[w] = pack_h2(u0, u1);
-                us[w] = pack_h2(u0 * vec[s0], u1 * vec[s0 + 1]);
+                for (int c = 0; c < 64; c += 4) {
+                    float4 x = *reinterpret_cast<const float4 *>(S0g + base + c);
+                    S[c] = x.x; S[c + 1] = x.y; S[c + 2] = x.z; S[c + 3] = x.w;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) S[c] = 0.0f;
             }
-            tmem_st16(tmem + lane_base + C_TM_UA + wg * 16, ua);
-            tmem_st16(tmem + lane_base + C_TM_US + wg * 16, us);
+        }
+        // fp16 copy of S as an A operand: row i on lane i, key index j two per column
+        auto store_S = [&](int slot) {
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int w = 0; w < 16; ++w) pk[w] = pack_h2(S[part * 32 + 2 * w], S[part * 32 + 2 * w + 1]);
+                tmem_st16(tmem + lane_base + C_TM_SA + slot * 64 + wg * 32 + part * 16, pk);
+            }
             tmem_st_wait();
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_sready);
+        };
+        store_S(0);
+
+        bool alive = true;
+        for (int c = 0; c < nchunks; ++c) {
+            const int t0 = t_begin + c * C;
+            const int L = min(C, t_end - t0);
+            const int b = c & 1;
+            const uint8_t *buf = sm + b * kWsItem;
+            const uint32_t ph = (uint32_t)(c & 1);
+
+            int ok = 1;
+            if (tid == 0)
+                ok = (mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status) && mbar_wait(bar_u, ph, status)) ? 1 : 0;
+            if (!workers_and(ok)) { alive = false; break; }
             tc_fence_after();
-            // MMA7: D7 = U_S^T K (B: K image, MN-major over j)
-            const uint32_t id7 = idesc_f16(128, false, true, false);
+            {
+                // U^T = U~^T - D4 as the fp16 A operand of MMA67
+                uint32_t r32[32];
+                tmem_ld32(tmem + C_TM_D45 + lane_base + wg * 32, r32);
+                tmem_ld_wait();
+                const __half *ut = reinterpret_cast<const __half *>(buf + kWsU);
+                uint32_t ua[16];
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16_ts(tmem + C_TM_D7, tmem + C_TM_US + kk * 8, mndesc(buf + B_K + kk * 2048, TILE), id7, kk > 0);
-            tc_commit(bar_s);
-            // MMA5: D5 = S0 Q'^T ; MMA6: D5 += U^T P^T
-            const uint32_t id5 = idesc_f16(64, false, false, false);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_f16_ts(tmem + C_TM_D5, tmem + C_TM_SA + b * 64 + kk * 8,
-                           kdesc(buf + B_Q + (kk < 4 ? 0 : TILE) + (kk & 3) * 32), id5, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16_ts(tmem + C_TM_D5, tmem + C_TM_UA + kk * 8, kdesc(buf + B_P + kk * 32), id5, 1u);
-            tc_commit(bar_o);
-        }
-        if (tid == 0) ok = mbar_wait(bar_s, ph, status) ? 1 : 0;
-        if (!__syncthreads_and(ok)) { alive = false; break; }
-        tc_fence_after();
-        {
-            const float gC = vec[64];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r7[32];
-                tmem_ld32(tmem + C_TM_D7 + lane_base + wg * 64 + half * 32, r7);
+                for (int w = 0; w < 16; ++w) {
+                    const int s0 = wg * 32 + 2 * w;
+                    const float u0 = (s0 < L) ? __half2float(ut[s0 * D + row]) - __uint_as_float(r32[2 * w]) : 0.0f;
+                    const float u1 = (s0 + 1 < L) ? __half2float(ut[(s0 + 1) * D + row]) - __uint_as_float(r32[2 * w + 1]) : 0.0f;
+                    ua[w] = pack_h2(u0, u1);
+                }
+                tmem_st16(tmem + lane_base + C_TM_UA + wg * 16, ua);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_uready);
+            }
+            if (tid == 0) ok = mbar_wait(bar_s, ph, status) ? 1 : 0;
+            if (!workers_and(ok)) { alive = false; break; }
+            tc_fence_after();
+            float ov[32];
+            {
+                uint32_t a5[32], b5[32];
+                tmem_ld32(tmem + C_TM_D45 + lane_base + 64 + wg * 32, a5);
+                tmem_ld32(tmem + C_TM_D67 + lane_base + 128 + wg * 32, b5);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) S[half * 32 + j] = gC * S[half * 32 + j] + __uint_as_float(r7[j]);
-            }
-            store_S(b ^ 1);   // S0 of chunk c + 1 (its slot was last read by chunk c-1's MMAs)
-            tmem_st_wait();
-        }
-        tc_fence_before();
-        __syncthreads();
-    }
-    if (alive && nchunks > 0) {
-        if (tid == 0) ok = mbar_wait(bar_o, (uint32_t)((nchunks - 1) & 1), status) ? 1 : 0;
-        if (__syncthreads_and(ok)) {
-            tc_fence_after();
-            emit_o(nchunks - 1);
-        } else {
-            alive = false;
-        }
-    }
-    if (alive && S_out) {
-        const size_t base = (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
+                for (int j = 0; j < 32; ++j) ov[j] = __uint_as_float(a5[j]) + __uint_as_float(b5[j]);
+                const float gC = reinterpret_cast<const float *>(buf + kWsVec)[0];
 #pragma unroll
-        for (int c = 0; c < 64; c += 4)
-            *reinterpret_cast<float4 *>(S_out + base + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r7[32];
+                    tmem_ld32(tmem + C_TM_D67 + lane_base + wg * 64 + half * 32, r7);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) S[half * 32 + j] = gC * S[half * 32 + j] + __uint_as_float(r7[j]);
+                }
+                store_S(b ^ 1);   // S0 of chunk c + 1; releases the MMA warp
+            }
+            {
+                // o rows of this chunk: staged as [r][i], then 16-byte row stores (rows < L)
+                uint8_t *stage = sm + CH_OFF_STAGE;
+                if (out_bf16) {
+                    __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(stage);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) st[(wg * 32 + j) * D + row] = __float2bfloat16_rn(ov[j]);
+                } else {
+                    float *st = reinterpret_cast<float *>(stage);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) st[(wg * 32 + j) * D + row] = ov[j];
+                }
+                workers_sync();
+                const int row_bytes = out_bf16 ? D * 2 : D * 4;
+                const int per_row = row_bytes / 16;
+                uint8_t *ob = static_cast<uint8_t *>(o);
+                for (int e = tid; e < L * per_row; e += NT) {
+                    const int r = e / per_row, ch = e % per_row;
+                    const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + ch * 16);
+                    *reinterpret_cast<uint4 *>(ob + (((size_t)(t0 + r) * Hv + h) * D) * (row_bytes / D) + ch * 16) = val;
+                }
+                workers_sync();
+            }
+        }
+        if (alive && S_out) {
+            const size_t base = (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
+#pragma unroll
+            for (int c = 0; c < 64; c += 4)
+                *reinterpret_cast<float4 *>(S_out + base + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -735,15 +724,13 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
     }
     const int slots = c.T / kChunk + c.num_seqs;
     uint8_t *ws = static_cast<uint8_t *>(c.ws);
-    uint8_t *ws_k = ws + ws_value_region(c.T, c.num_seqs, c.Hv);
     gdn_chunk_prep_kernel<<<dim3(slots, c.Hv), NT, P_SMEM, st>>>(maps, c.a, c.b, c.A_log, c.dt_bias, c.cu_seqlens, c.T,
                                                                  c.num_seqs, c.Hk, c.Hv, slots, c.scale, c.l2norm, ws,
-                                                                 ws_k, c.status);
+                                                                 c.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    gdn_chunk_chain_kernel<<<dim3(c.Hv, c.num_seqs), NT, CH_SMEM, st>>>(c.cu_seqlens, c.T, c.Hk, c.Hv, slots,
-                                                                        c.out_bf16 ? 1 : 0, c.S0, c.S_out, c.o, ws,
-                                                                        ws_k, c.status);
+    gdn_chunk_chain_kernel<<<dim3(c.Hv, c.num_seqs), CH_THREADS, CH_SMEM, st>>>(
+        c.cu_seqlens, c.T, c.Hv, slots, c.out_bf16 ? 1 : 0, c.S0, c.S_out, c.o, ws, c.status);
     return cudaGetLastError();
 }
 

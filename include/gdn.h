@@ -95,8 +95,7 @@ GDN_API gdn_status gdn_prefill_chunked(const void *q, const void *k, const void 
                                void *workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /* Scratch bytes the tensor-core path of gdn_prefill_chunked needs for these sizes:
- * (T / 64 + num_seqs) * (58368 * Hv + 16384 * Hk) when Dk == Dv == 128, else 0. Host-only, no
- * CUDA call. */
+ * Hv * (T / 64 + num_seqs) * 74752 when Dk == Dv == 128, else 0. Host-only, no CUDA call. */
 GDN_API size_t gdn_prefill_workspace_bytes(int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv,
                                    int32_t Dk, int32_t Dv);
 
