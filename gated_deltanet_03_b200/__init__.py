@@ -26,7 +26,8 @@ GDN_BF16, GDN_F32 = 0, 1
 ABI_SYMBOLS = (
     "gdn_prefill_chunked", "gdn_prefill_workspace_bytes", "gdn_decode_step",
     "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act",
-    "nvfp4_gemm", "gdn_get_device_status", "gdn_status_string", "gdn_version",
+    "nvfp4_gemm", "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_status_string",
+    "gdn_version",
 )
 
 
@@ -52,11 +53,13 @@ def _load() -> ctypes.CDLL:
     lib.gdn_gated_rmsnorm_silu_nvfp4.argtypes = [P, P, P, f32, i32, i32, i32, i32, f32, P, P, P]
     lib.nvfp4_quantize_act.argtypes = [P, i32, i32, i32, f32, P, P, P]
     lib.nvfp4_gemm.argtypes = [P, P, P, P, f32, i32, i32, i32, i32, P, P]
+    lib.gdn_prefill_chunked_static_ws.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32,
+                                                  i32, i32, P, P, P, i32, P]
     lib.gdn_get_device_status.argtypes = [P]
     lib.gdn_status_string.argtypes = [i32]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_version.restype = i32
-    for name in ("gdn_prefill_chunked", "gdn_decode_step", "gdn_gated_rmsnorm_silu",
+    for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_static_ws", "gdn_decode_step", "gdn_gated_rmsnorm_silu",
                  "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_gemm",
                  "gdn_get_device_status"):
         getattr(lib, name).restype = ctypes.c_int

@@ -160,6 +160,30 @@ GDN_API gdn_status nvfp4_gemm(const uint8_t *aq, const uint8_t *as, const uint8_
                       float alpha, int32_t M, int32_t N, int32_t K, gdn_dtype out_dtype, void *y,
                       gdn_stream_t stream);
 
+/* ------------------------------------------------- allocation-free prefill ----
+ * No counterpart in the paper. For callers that cannot allocate device memory - code that
+ * runs where cudaMalloc is unavailable or not allowed, or a host framework that owns every
+ * allocation - this is gdn_prefill_chunked without the workspace argument: same inputs,
+ * outputs, layouts and status codes. The tensor-core path uses a fixed scratch array inside
+ * the library instead: 32 MiB (33554432 bytes), held on every GPU that loads the library
+ * until the process exits. Sizes whose workspace (gdn_prefill_workspace_bytes) exceeds
+ * 32 MiB return GDN_ERR_WORKSPACE before anything is launched. It allocates nothing.
+ * The first call on a device looks up the array's device address for that device; make
+ * that first call before any stream capture on the device.
+ * Every call uses the same array: calls that can overlap on the GPU (other streams, other
+ * host threads) race on it and corrupt each other's results, so serialise them. What a
+ * previous call left in the array does not matter: the path writes all it later reads.
+ */
+GDN_API gdn_status gdn_prefill_chunked_static_ws(const void *q, const void *k, const void *v,
+                                                 const float *a, const float *b,
+                                                 const float *A_log, const float *dt_bias,
+                                                 const int32_t *cu_seqlens, int32_t num_seqs,
+                                                 int32_t T, int32_t Hk, int32_t Hv, int32_t Dk,
+                                                 int32_t Dv, float scale, int32_t qk_l2norm,
+                                                 gdn_dtype in_dtype, const float *initial_state,
+                                                 float *final_state, void *o, gdn_dtype out_dtype,
+                                                 gdn_stream_t stream);
+
 /* ----------------------------------------------------------------- helpers ---- */
 
 /* Synchronises `stream`, returns the device status word (GDN_OK or GDN_ERR_TIMEOUT) that
