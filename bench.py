@@ -34,6 +34,16 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 CHUNK = 64
+# DRAM bytes (read + write) of one scan call (prep + chain kernels) on the benchmark workload,
+# from the ncu capture summarised in profiles/chunked_prefill_T4096.md; valid only for the
+# kernel source it was taken on (first 16 hex digits of its sha256).
+SCAN_TRAFFIC = {"04f0c0687cf454f6": 154.1e6}
+
+
+def source_digest(path: str) -> str:
+    import hashlib
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
 def peaks():
@@ -63,57 +73,70 @@ def scan_bytes(w: workloads.Workload, o_bytes=2) -> float:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """SM clock and clock-event (throttle) reasons sampled every millisecond through NVML
+    while the timed region runs (falls back to an nvidia-smi loop when NVML is missing)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+        self._handle = None
+
+    def _open(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.cuda_index)
+        if hasattr(props, "pci_bus_id"):
+            bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), props.pci_bus_id, props.pci_device_id)
+            self._handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        else:
+            self._handle = pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
+        self._nvml = pynvml
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM))
+
+    def _loop(self):
+        nv, h = self._nvml, self._handle
+        get_reasons = (getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None)
+                       or nv.nvmlDeviceGetCurrentClocksThrottleReasons)
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                reasons = get_reasons(h)
+                self.samples.append((float(mhz), int(reasons)))
+            except Exception:  # noqa: BLE001 - a failed sample is skipped
+                pass
+            time.sleep(0.001)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except OSError:
-            self.proc = None
+            self._open()
+            self._thread = threading.Thread(target=self._loop, daemon=True)
+            self._thread.start()
+        except Exception:  # noqa: BLE001 - no NVML: report no samples
+            self._thread = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [m for m, _ in self.samples]
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvml, 1 ms"}
 
 
 # ----------------------------------------------------------------- GPU arm ----
@@ -322,7 +345,9 @@ def run_gpu(args):
                      "peak_kind": pk_kind + " (bf16 dense burst; the scan's MMAs are fp16)",
                      "algorithmic_flops": fl, "algorithmic_bytes": scan_bytes(w),
                      "hbm_frac": scan_bytes(w) / scan_s / 1e9 / float(pk["hbm_gbs"]),
-                     "traffic": None},
+                     "traffic": SCAN_TRAFFIC.get(source_digest(os.path.join(
+                         ROOT, "gated_deltanet_03_b200", "csrc", "chunked.cu"))),
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, prep + chain"},
         "e2e": {"value": tokens / (e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
         "decode": {"workload": dw.name, "ms": dec, "GB/s": dec_bytes / (dec / 1e3) / 1e9,
