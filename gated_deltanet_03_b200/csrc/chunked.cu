@@ -148,6 +148,21 @@ __device__ __forceinline__ void locate(int id, const int32_t *cu, int num_seqs, 
     }
 }
 
+// Two fp16 values as one 32-bit register (first in the low half).
+__device__ __forceinline__ uint32_t pack_two_h(__half lo, __half hi) {
+    return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+
+// Warp-level 16 x 8 x 16 MMA, fp16 inputs, fp32 accumulation (row-major A, column-major B):
+// used only for the 16 x 16 blocks of the triangular inverse, where latency matters.
+__device__ __forceinline__ void mma_m16n8k16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // ===================================================================================
 // Prep kernel: one CTA per (chunk slot, value head); two CTAs per SM.
 // ===================================================================================
@@ -155,15 +170,17 @@ constexpr int P_OFF_KQ = 0;                       // [K_lo][Q_lo][K_hi][Q_hi], b
 constexpr int P_OFF_V = 4 * TILE;                 // [V_lo][V_hi]
 constexpr int P_OFF_TP = 6 * TILE;                // T'  [s][r] fp16, swizzled
 constexpr int P_OFF_TPP = 7 * TILE;               // T'' [s][r] fp16, swizzled
-constexpr int P_OFF_AF = 8 * TILE;                // A fp32 [64][65]
-constexpr int P_OFF_TF = P_OFF_AF + 64 * 65 * 4;  // T fp32 [64][65]
-constexpr int P_OFF_XF = P_OFF_TF + 64 * 65 * 4;  // X fp32 [3][256]
-constexpr int P_OFF_STG = P_OFF_AF;               // W and U~ staging once A and T are dead (32 KB)
-constexpr int P_OFF_VEC = P_OFF_XF + 3 * 256 * 4; // G, beta, rk, rq, gamma, decS (64 each), row sums of squares (128)
+constexpr int P_AH = 72;                          // fp16 row pitch of A and T copies (144 B)
+constexpr int P_OFF_AH = 8 * TILE;                // A fp16 [64][72]
+constexpr int P_OFF_TF = P_OFF_AH + 64 * P_AH * 2;  // T fp32 [64][65]
+constexpr int P_OFF_TH = P_OFF_TF + 64 * 65 * 4;  // T fp16 [64][72]
+constexpr int P_OFF_XH = P_OFF_TH + 64 * P_AH * 2;  // X fp16 [3 warps][16][24]
+constexpr int P_OFF_STG = P_OFF_AH;               // W and U~ staging once A and T are dead (32 KB)
+constexpr int P_OFF_VEC = P_OFF_XH + 3 * 16 * 24 * 2; // G, beta, rk, rq, gamma, decS (64 each), row sums of squares (128)
 constexpr int P_OFF_BAR = P_OFF_VEC + 8 * 64 * 4;
 constexpr int P_SMEM = P_OFF_BAR + 64 + 1024;
 static_assert(P_SMEM * 2 <= 228 * 1024, "two prep CTAs per SM");
-static_assert(P_OFF_XF - P_OFF_AF >= 4 * TILE, "staging fits in the A/T scratch");
+static_assert(P_OFF_VEC - P_OFF_AH >= 4 * TILE, "staging fits in the A/T scratch");
 constexpr uint32_t P_TM_D1 = 0, P_TM_D2 = 128, P_TM_D3 = 192;
 
 __global__ void __launch_bounds__(NT, 2)
@@ -188,9 +205,9 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + P_OFF_BAR);
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 2);
-    float *Af = reinterpret_cast<float *>(sm + P_OFF_AF);
+    __half *Ah = reinterpret_cast<__half *>(sm + P_OFF_AH);
     float *Tf = reinterpret_cast<float *>(sm + P_OFF_TF);
-    float *Xf = reinterpret_cast<float *>(sm + P_OFF_XF);
+    __half *Th = reinterpret_cast<__half *>(sm + P_OFF_TH);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int wg = warp / 4;
@@ -311,7 +328,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                         const int r = hcol * 32 + j;
                         float a = 0.0f;
                         if (s < r && r < L) a = sBeta[r] * __expf(sG[r] - Gs) * __uint_as_float(r32[j]) * sRk[r] * rks;
-                        Af[r * 65 + s] = a;
+                        Ah[r * P_AH + s] = __float2half_rn(a);
                     }
                 } else {
                     float pv[32];
@@ -329,8 +346,9 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     tc_fence_before();
     __syncthreads();
 
-    // ---- T = (I + A)^-1: 16 x 16 diagonal blocks by forward substitution, then the
-    //      off-diagonal blocks level by level, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.
+    // ---- T = (I + A)^-1: 16 x 16 diagonal blocks by forward substitution (fp32), then the
+    //      off-diagonal blocks level by level, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj, one
+    //      warp per block on the warp-level tensor-core MMA (fp16 inputs, fp32 accumulation).
     if (tid < 64) {
         const int bi = tid / 16, cc = tid % 16, o0 = bi * 16;
         float x[16];
@@ -338,33 +356,65 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         for (int r = 0; r < 16; ++r) {
             float acc = (r == cc) ? 1.0f : 0.0f;
 #pragma unroll
-            for (int s = 0; s < r; ++s) acc -= Af[(o0 + r) * 65 + o0 + s] * x[s];
+            for (int s = 0; s < r; ++s) acc -= __half2float(Ah[(o0 + r) * P_AH + o0 + s]) * x[s];
             x[r] = acc;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tf[(o0 + r) * 65 + o0 + cc] = x[r];
+        for (int r = 0; r < 16; ++r) {
+            Tf[(o0 + r) * 65 + o0 + cc] = x[r];
+            Th[(o0 + r) * P_AH + o0 + cc] = __float2half_rn(x[r]);
+        }
     }
     __syncthreads();
 #pragma unroll 1
     for (int lvl = 1; lvl < 4; ++lvl) {
-        const int nblk = 4 - lvl;
-        const int er = tid / 16, ec = tid % 16;
-        for (int bj = 0; bj < nblk; ++bj) {
-            const int bi = bj + lvl;
-            float acc = 0.0f;
-            for (int bk = bj; bk < bi; ++bk)
+        if (warp < 4 - lvl) {
+            const int bj = warp, bi = bj + lvl;
+            const int g = lane >> 2, t = lane & 3;
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int bk = bj; bk < bi; ++bk) {
+                const uint32_t *arow0 = reinterpret_cast<const uint32_t *>(Ah + (bi * 16 + g) * P_AH + bk * 16);
+                const uint32_t *arow1 = reinterpret_cast<const uint32_t *>(Ah + (bi * 16 + g + 8) * P_AH + bk * 16);
+                const uint32_t a0 = arow0[t], a1 = arow1[t], a2 = arow0[t + 4], a3 = arow1[t + 4];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    acc += Af[(bi * 16 + er) * 65 + bk * 16 + e] * Tf[(bk * 16 + e) * 65 + bj * 16 + ec];
-            Xf[bj * 256 + er * 16 + ec] = acc;
-        }
-        __syncthreads();
-        for (int bj = 0; bj < nblk; ++bj) {
-            const int bi = bj + lvl;
-            float acc = 0.0f;
+                for (int hn = 0; hn < 2; ++hn) {
+                    const int col = bj * 16 + hn * 8 + g;
+                    const uint32_t b0 = pack_two_h(Th[(bk * 16 + 2 * t) * P_AH + col], Th[(bk * 16 + 2 * t + 1) * P_AH + col]);
+                    const uint32_t b1 = pack_two_h(Th[(bk * 16 + 2 * t + 8) * P_AH + col], Th[(bk * 16 + 2 * t + 9) * P_AH + col]);
+                    mma_m16n8k16(acc[hn], a0, a1, a2, a3, b0, b1);
+                }
+            }
+            // X (fp16, per-warp scratch [16][24]) as the B operand of T_ij = -T_ii X
+            __half *Xh = reinterpret_cast<__half *>(sm + P_OFF_XH) + warp * 16 * 24;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) acc += Tf[(bi * 16 + er) * 65 + bi * 16 + e] * Xf[bj * 256 + e * 16 + ec];
-            Tf[(bi * 16 + er) * 65 + bj * 16 + ec] = -acc;
+            for (int hn = 0; hn < 2; ++hn) {
+                Xh[g * 24 + hn * 8 + 2 * t] = __float2half_rn(acc[hn][0]);
+                Xh[g * 24 + hn * 8 + 2 * t + 1] = __float2half_rn(acc[hn][1]);
+                Xh[(g + 8) * 24 + hn * 8 + 2 * t] = __float2half_rn(acc[hn][2]);
+                Xh[(g + 8) * 24 + hn * 8 + 2 * t + 1] = __float2half_rn(acc[hn][3]);
+            }
+            __syncwarp();
+            const uint32_t *trow0 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g) * P_AH + bi * 16);
+            const uint32_t *trow1 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g + 8) * P_AH + bi * 16);
+            const uint32_t a0 = trow0[t], a1 = trow1[t], a2 = trow0[t + 4], a3 = trow1[t + 4];
+#pragma unroll
+            for (int hn = 0; hn < 2; ++hn) {
+                const int col = hn * 8 + g;
+                const uint32_t b0 = pack_two_h(Xh[(2 * t) * 24 + col], Xh[(2 * t + 1) * 24 + col]);
+                const uint32_t b1 = pack_two_h(Xh[(2 * t + 8) * 24 + col], Xh[(2 * t + 9) * 24 + col]);
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_m16n8k16(d, a0, a1, a2, a3, b0, b1);
+                const int c0 = bj * 16 + hn * 8 + 2 * t;
+                const int r0 = bi * 16 + g;
+                Tf[r0 * 65 + c0] = -d[0];
+                Tf[r0 * 65 + c0 + 1] = -d[1];
+                Tf[(r0 + 8) * 65 + c0] = -d[2];
+                Tf[(r0 + 8) * 65 + c0 + 1] = -d[3];
+                Th[r0 * P_AH + c0] = __float2half_rn(-d[0]);
+                Th[r0 * P_AH + c0 + 1] = __float2half_rn(-d[1]);
+                Th[(r0 + 8) * P_AH + c0] = __float2half_rn(-d[2]);
+                Th[(r0 + 8) * P_AH + c0 + 1] = __float2half_rn(-d[3]);
+            }
         }
         __syncthreads();
     }
