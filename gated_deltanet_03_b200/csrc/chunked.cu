@@ -34,6 +34,8 @@
 // 128-byte swizzled), [K''; P^T] (fp16, three 64-wide MN-major blocks), U~ (fp16 [s][i]) and
 // gamma_C. Chunk c of sequence n uses slot cu_seqlens[n] / 64 + n + c, so slots never
 // collide and T / 64 + num_seqs slots per head suffice.
+#include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "common.cuh"
@@ -45,9 +47,37 @@ constexpr int kChunk = 64;
 constexpr int kWsItem = 74752;
 constexpr int kWsWQ = 0, kWsKP = 32768, kWsU = 57344, kWsVec = 73728;
 
+constexpr size_t kSegItemBytes = 196608;
+
+// Chunks per segment of the chain: the state chain of a sequence is split into segments that
+// run in parallel (state and transition passes), a short sequential combine, and the output
+// pass. Picks the length that minimises a cycle model of the three passes (per-chunk costs of
+// the chain modes and of one combine step, measured on B200, and the number of CTA waves on
+// 148 SMs), from the mean sequence length.
+int chunked_segment_chunks(int T, int num_seqs, int Hv) {
+    const double nch = (double)T / kChunk / (num_seqs > 0 ? num_seqs : 1);
+    const double c_state = 3.5, c_full = 4.7, c_comb = 2.5, sms = 148.0;
+    int best = 1 << 30;
+    double best_cost = 1e30;
+    for (int seg = 4; seg <= 4096; seg *= 2) {
+        const double nseg = nch / seg > 1.0 ? std::ceil(nch / seg) : 1.0;
+        const double ctas = (double)Hv * num_seqs * nseg;
+        double cost = std::ceil(ctas / sms) * std::min((double)seg, nch) * c_full;
+        if (nseg > 1.0) cost += std::ceil(2.0 * ctas / sms) * seg * c_state + (nseg - 2.0) * c_comb;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = seg;
+        }
+        if (seg >= nch) break;
+    }
+    return best;
+}
+
 size_t chunked_workspace_bytes(int T, int num_seqs, int Hk, int Hv) {
     (void)Hk;
-    return (size_t)Hv * (size_t)(T / kChunk + num_seqs) * kWsItem;
+    const int seg = chunked_segment_chunks(T, num_seqs, Hv);
+    return (size_t)Hv * (size_t)(T / kChunk + num_seqs) * kWsItem +
+           (size_t)Hv * (size_t)(T / (kChunk * seg) + num_seqs) * kSegItemBytes;
 }
 
 namespace {
@@ -522,10 +552,26 @@ __device__ __forceinline__ int workers_and(int pred) {
 }
 __device__ __forceinline__ void workers_sync() { asm volatile("barrier.cta.sync 2, 256;" ::: "memory"); }
 
+// Chain modes: the full chain with outputs from a segment's true start state; a segment's
+// state from S0 (first segment) or zero, with no outputs; a segment's transition matrix,
+// the state from the identity with U~ taken as zero (its final state is the map S -> S M).
+enum ChainMode { kChainFull = 0, kChainState = 1, kChainTransition = 2 };
+
+struct ChainParams {
+    const int32_t *cu_seqlens;
+    int32_t T, num_seqs, Hv, slots, seg_chunks, seg_slots, mode_base, out_bf16;
+    const float *S0g;
+    float *S_out;
+    void *o;
+    const uint8_t *ws;     // per-chunk operand items
+    uint8_t *ws_seg;       // per-segment B (fp32), M (fp16 hi/lo operand images), start state (fp32)
+    int *status;
+};
+constexpr size_t kSegItem = kSegItemBytes;
+constexpr size_t kSegB = 0, kSegMhi = 65536, kSegMlo = 98304, kSegS = 131072;
+
 __global__ void __launch_bounds__(CH_THREADS, 1)
-gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_t Hv, int32_t slots,
-                       int32_t out_bf16, const float *S0g, float *S_out, void *__restrict__ o,
-                       const uint8_t *__restrict__ ws, int *status) {
+gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CH_OFF_BAR);
@@ -533,15 +579,38 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int h = blockIdx.x, n = blockIdx.y;
-    int t_begin = 0, t_end = T;
-    if (cu_seqlens) {
-        t_begin = cu_seqlens[n];
-        t_end = cu_seqlens[n + 1];
+    const int h = blockIdx.x, id = blockIdx.y, mode = P.mode_base + (int)blockIdx.z;
+    const int T = P.T, Hv = P.Hv, SEG = P.seg_chunks;
+    int n = 0, t_begin = 0, t_end = T;
+    if (P.cu_seqlens) {
+        int lo = 0, hi = P.num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (P.cu_seqlens[mid] / (C * SEG) + mid <= id) lo = mid;
+            else hi = mid - 1;
+        }
+        n = lo;
+        t_begin = P.cu_seqlens[n];
+        t_end = P.cu_seqlens[n + 1];
     }
-    const int nchunks = (t_end - t_begin + C - 1) / C;
-    const int slot0 = t_begin / C + n;
-    const uint8_t *ws_h = ws + (size_t)h * slots * kWsItem;
+    const int nch_seq = (t_end - t_begin + C - 1) / C;
+    const int nseg = (nch_seq + SEG - 1) / SEG;
+    const int pseg = id - (t_begin / (C * SEG) + n);
+    // slots no segment uses; the state and transition passes skip the last segment, the
+    // transition pass also the first (its start state is known)
+    if (pseg < 0) return;
+    if (mode == kChainFull && pseg >= (nseg > 0 ? nseg : 1)) return;
+    if (mode != kChainFull && pseg >= nseg - 1) return;
+    if (mode == kChainTransition && pseg == 0) return;
+    const int c_first = pseg * SEG;
+    const int nchunks = max(0, min(nch_seq, c_first + SEG) - c_first);
+    const bool last_seg = pseg >= nseg - 1;
+    const uint8_t *seg_item = P.ws_seg + ((size_t)h * P.seg_slots + id) * kSegItem;
+    const int32_t slots = P.slots;
+    const float *S0g = P.S0g;
+    const int slot0 = t_begin / C + n + c_first;
+    const uint8_t *ws_h = P.ws + (size_t)h * slots * kWsItem;
+    int *status = P.status;
 
     if (tid == 0) {
         mbar_init(&full[0], 1);
@@ -570,8 +639,9 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
                 bulk_load(sm + (c & 1) * kWsItem, ws_h + (size_t)(slot0 + c) * kWsItem, kWsItem, bar);
             };
             if (nchunks > 0) issue_chunk(0);
-            const uint32_t id45 = idesc_f16(128, false, false, false);
-            const uint32_t id67 = idesc_f16(192, false, true, false);
+            const bool full_out = mode == kChainFull;   // the output halves only when o is produced
+            const uint32_t id45 = idesc_f16(full_out ? 128 : 64, false, false, false);
+            const uint32_t id67 = idesc_f16(full_out ? 192 : 128, false, true, false);
             for (int c = 0; c < nchunks; ++c) {
                 const int b = c & 1;
                 const uint8_t *buf = sm + b * kWsItem;
@@ -605,16 +675,24 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
         const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
         float S[64];   // S[i][64 wg .. 64 wg + 63], fp32
         {
-            const size_t base = (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
-            if (S0g) {
+            const float *src = nullptr;
+            size_t base = 0;
+            if (pseg == 0 && mode != kChainTransition && S0g) {
+                src = S0g;
+                base = (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
+            } else if (pseg > 0 && mode == kChainFull) {
+                src = reinterpret_cast<const float *>(seg_item + kSegS);
+                base = (size_t)row * D + 64 * wg;
+            }
+            if (src) {
 #pragma unroll
                 for (int c = 0; c < 64; c += 4) {
-                    float4 x = *reinterpret_cast<const float4 *>(S0g + base + c);
+                    float4 x = *reinterpret_cast<const float4 *>(src + base + c);
                     S[c] = x.x; S[c + 1] = x.y; S[c + 2] = x.z; S[c + 3] = x.w;
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) S[c] = 0.0f;
+                for (int c = 0; c < 64; ++c) S[c] = (mode == kChainTransition && row == 64 * wg + c) ? 1.0f : 0.0f;
             }
         }
         // fp16 copy of S as an A operand: row i on lane i, key index j two per column
@@ -635,7 +713,7 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
 
         bool alive = true;
         for (int c = 0; c < nchunks; ++c) {
-            const int t0 = t_begin + c * C;
+            const int t0 = t_begin + (c_first + c) * C;
             const int L = min(C, t_end - t0);
             const int b = c & 1;
             const uint8_t *buf = sm + b * kWsItem;
@@ -656,8 +734,10 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
 #pragma unroll
                 for (int w = 0; w < 16; ++w) {
                     const int s0 = wg * 32 + 2 * w;
-                    const float u0 = (s0 < L) ? __half2float(ut[s0 * D + row]) - __uint_as_float(r32[2 * w]) : 0.0f;
-                    const float u1 = (s0 + 1 < L) ? __half2float(ut[(s0 + 1) * D + row]) - __uint_as_float(r32[2 * w + 1]) : 0.0f;
+                    const float ut0 = mode == kChainTransition ? 0.0f : __half2float(ut[s0 * D + row]);
+                    const float ut1 = mode == kChainTransition ? 0.0f : __half2float(ut[(s0 + 1) * D + row]);
+                    const float u0 = (s0 < L) ? ut0 - __uint_as_float(r32[2 * w]) : 0.0f;
+                    const float u1 = (s0 + 1 < L) ? ut1 - __uint_as_float(r32[2 * w + 1]) : 0.0f;
                     ua[w] = pack_h2(u0, u1);
                 }
                 tmem_st16(tmem + lane_base + C_TM_UA + wg * 16, ua);
@@ -671,12 +751,14 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
             tc_fence_after();
             float ov[32];
             {
-                uint32_t a5[32], b5[32];
-                tmem_ld32(tmem + C_TM_D45 + lane_base + 64 + wg * 32, a5);
-                tmem_ld32(tmem + C_TM_D67 + lane_base + 128 + wg * 32, b5);
-                tmem_ld_wait();
+                if (mode == kChainFull) {
+                    uint32_t a5[32], b5[32];
+                    tmem_ld32(tmem + C_TM_D45 + lane_base + 64 + wg * 32, a5);
+                    tmem_ld32(tmem + C_TM_D67 + lane_base + 128 + wg * 32, b5);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) ov[j] = __uint_as_float(a5[j]) + __uint_as_float(b5[j]);
+                    for (int j = 0; j < 32; ++j) ov[j] = __uint_as_float(a5[j]) + __uint_as_float(b5[j]);
+                }
                 const float gC = reinterpret_cast<const float *>(buf + kWsVec)[0];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -688,8 +770,9 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
                 }
                 store_S(b ^ 1);   // S0 of chunk c + 1; releases the MMA warp
             }
-            {
+            if (mode == kChainFull) {
                 // o rows of this chunk: staged as [r][i], then 16-byte row stores (rows < L)
+                const int out_bf16 = P.out_bf16;
                 uint8_t *stage = sm + CH_OFF_STAGE;
                 if (out_bf16) {
                     __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(stage);
@@ -703,7 +786,7 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
                 workers_sync();
                 const int row_bytes = out_bf16 ? D * 2 : D * 4;
                 const int per_row = row_bytes / 16;
-                uint8_t *ob = static_cast<uint8_t *>(o);
+                uint8_t *ob = static_cast<uint8_t *>(P.o);
                 for (int e = tid; e < L * per_row; e += NT) {
                     const int r = e / per_row, ch = e % per_row;
                     const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + ch * 16);
@@ -712,11 +795,35 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
                 workers_sync();
             }
         }
-        if (alive && S_out) {
-            const size_t base = (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
+        if (alive) {
+            float *dst = nullptr;
+            if (mode == kChainFull && last_seg && P.S_out)
+                dst = P.S_out + (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
+            else if (mode == kChainState)
+                dst = reinterpret_cast<float *>(const_cast<uint8_t *>(seg_item) + kSegB) + (size_t)row * D + 64 * wg;
+            if (dst) {
 #pragma unroll
-            for (int c = 0; c < 64; c += 4)
-                *reinterpret_cast<float4 *>(S_out + base + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
+                for (int c = 0; c < 64; c += 4)
+                    *reinterpret_cast<float4 *>(dst + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
+            }
+            if (mode == kChainTransition) {
+                // the segment's map M (row j = this lane) as fp16 hi / lo B operand images,
+                // MN-major over the output column, 128-byte swizzled rows
+                uint8_t *mhi = const_cast<uint8_t *>(seg_item) + kSegMhi + wg * 16384;
+                uint8_t *mlo = const_cast<uint8_t *>(seg_item) + kSegMlo + wg * 16384;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    float hi8[8], lo8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float x = S[ch * 8 + e];
+                        hi8[e] = __half2float(__float2half_rn(x));
+                        lo8[e] = x - hi8[e];
+                    }
+                    st_h8(mhi + swz(row, ch), hi8);
+                    st_h8(mlo + swz(row, ch), lo8);
+                }
+            }
         }
     }
     tc_fence_before();
@@ -724,6 +831,150 @@ gdn_chunk_chain_kernel(const int32_t *__restrict__ cu_seqlens, int32_t T, int32_
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+
+// ===================================================================================
+// Segment combine: per (value head, sequence), S_start(p + 1) = S_start(p) M_p + B_p in order,
+// S_start(1) = B_0. The product runs on the tensor cores with S split into fp16 hi + lo and M
+// given as fp16 hi + lo operand images (S_hi M_hi + S_lo M_hi + S_hi M_lo, fp32 accumulation).
+// ===================================================================================
+constexpr int CB_OFF_BUF = 0;                   // two buffers of [M_hi | M_lo] images, 64 KB each
+constexpr int CB_OFF_BAR = 2 * 65536;
+constexpr int CB_SMEM = CB_OFF_BAR + 64 + 1024;
+constexpr uint32_t CB_TM_SHI = 0, CB_TM_SLO = 64, CB_TM_D = 128;
+
+__global__ void __launch_bounds__(NT, 1)
+gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
+    const int h = blockIdx.x, n = blockIdx.y;
+    const int SEG = P.seg_chunks;
+    int t_begin = 0, t_end = P.T;
+    if (P.cu_seqlens) {
+        t_begin = P.cu_seqlens[n];
+        t_end = P.cu_seqlens[n + 1];
+    }
+    const int nch = (t_end - t_begin + C - 1) / C;
+    const int nseg = (nch + SEG - 1) / SEG;
+    if (nseg <= 1) return;
+    const int base = t_begin / (C * SEG) + n;
+    auto seg = [&](int p) { return P.ws_seg + ((size_t)h * P.seg_slots + base + p) * kSegItem; };
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + CB_OFF_BAR);
+    uint64_t *bar_mma = full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 3);
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int wg = warp / 4, row = (warp % 4) * 32 + lane;
+    const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
+
+    if (tid == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_init(bar_mma, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    auto issue_m = [&](int p) {
+        uint64_t *bar = &full[(p - 1) & 1];
+        mbar_arrive_expect_tx(bar, 65536);
+        bulk_load(sm + CB_OFF_BUF + ((p - 1) & 1) * 65536, seg(p) + kSegMhi, 65536, bar);
+    };
+    if (tid == 0 && nseg > 2) issue_m(1);
+
+    float S[64];
+    {
+        const float *b0 = reinterpret_cast<const float *>(seg(0) + kSegB) + (size_t)row * D + 64 * wg;
+        float *s1 = reinterpret_cast<float *>(seg(1) + kSegS) + (size_t)row * D + 64 * wg;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(b0 + c);
+            S[c] = x.x; S[c + 1] = x.y; S[c + 2] = x.z; S[c + 3] = x.w;
+            *reinterpret_cast<float4 *>(s1 + c) = x;
+        }
+    }
+    const uint32_t idm = idesc_f16(128, false, true, false);
+    for (int p = 1; p + 1 < nseg; ++p) {
+        const int b = (p - 1) & 1;
+        uint8_t *buf = sm + CB_OFF_BUF + b * 65536;
+        // S -> fp16 hi / lo A operands
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+                const float x0 = S[part * 32 + 2 * w], x1 = S[part * 32 + 2 * w + 1];
+                const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+                hi[w] = pack_two_h(h0, h1);
+                lo[w] = pack_h2(x0 - __half2float(h0), x1 - __half2float(h1));
+            }
+            tmem_st16(tmem + lane_base + CB_TM_SHI + wg * 32 + part * 16, hi);
+            tmem_st16(tmem + lane_base + CB_TM_SLO + wg * 32 + part * 16, lo);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncthreads();
+        int ok = 1;
+        if (tid == 0) {
+            if (p + 2 < nseg) {
+                fence_proxy_async_smem();
+                issue_m(p + 1);
+            }
+            ok = mbar_wait(&full[b], (uint32_t)(((p - 1) >> 1) & 1), P.status) ? 1 : 0;
+            if (ok) {
+                tc_fence_after();
+                const uint8_t *mhi = buf, *mlo = buf + 32768;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tmem + CB_TM_D, tmem + CB_TM_SHI + kk * 8, mndesc(mhi + kk * 2048, 16384), idm, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tmem + CB_TM_D, tmem + CB_TM_SLO + kk * 8, mndesc(mhi + kk * 2048, 16384), idm, 1u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tmem + CB_TM_D, tmem + CB_TM_SHI + kk * 8, mndesc(mlo + kk * 2048, 16384), idm, 1u);
+                tc_commit(bar_mma);
+            }
+        }
+        float Bp[64];
+        {
+            const float *bp = reinterpret_cast<const float *>(seg(p) + kSegB) + (size_t)row * D + 64 * wg;
+#pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+                const float4 x = *reinterpret_cast<const float4 *>(bp + c);
+                Bp[c] = x.x; Bp[c + 1] = x.y; Bp[c + 2] = x.z; Bp[c + 3] = x.w;
+            }
+        }
+        if (tid == 0 && ok) ok = mbar_wait(bar_mma, (uint32_t)((p - 1) & 1), P.status) ? 1 : 0;
+        if (!__syncthreads_and(ok)) break;
+        tc_fence_after();
+        float *sn = reinterpret_cast<float *>(seg(p + 1) + kSegS) + (size_t)row * D + 64 * wg;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t r32[32];
+            tmem_ld32(tmem + CB_TM_D + lane_base + wg * 64 + half * 32, r32);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) S[half * 32 + j] = __uint_as_float(r32[j]) + Bp[half * 32 + j];
+        }
+#pragma unroll
+        for (int c = 0; c < 64; c += 4)
+            *reinterpret_cast<float4 *>(sn + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
+        tc_fence_before();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
     }
 }
 
@@ -769,18 +1020,31 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
         cudaError_t e = cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(gdn_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn_segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CB_SMEM);
         if (e != cudaSuccess) return e;
         attr = true;
     }
     const int slots = c.T / kChunk + c.num_seqs;
+    const int seg = chunked_segment_chunks(c.T, c.num_seqs, c.Hv);
+    const int seg_slots = c.T / (kChunk * seg) + c.num_seqs;
     uint8_t *ws = static_cast<uint8_t *>(c.ws);
     gdn_chunk_prep_kernel<<<dim3(slots, c.Hv), NT, P_SMEM, st>>>(maps, c.a, c.b, c.A_log, c.dt_bias, c.cu_seqlens, c.T,
                                                                  c.num_seqs, c.Hk, c.Hv, slots, c.scale, c.l2norm, ws,
                                                                  c.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    gdn_chunk_chain_kernel<<<dim3(c.Hv, c.num_seqs), CH_THREADS, CH_SMEM, st>>>(
-        c.cu_seqlens, c.T, c.Hv, slots, c.out_bf16 ? 1 : 0, c.S0, c.S_out, c.o, ws, c.status);
+    ChainParams P{c.cu_seqlens, c.T, c.num_seqs, c.Hv, slots, seg, seg_slots, kChainFull, c.out_bf16 ? 1 : 0, c.S0,
+                  c.S_out, c.o, ws, ws + (size_t)c.Hv * slots * kWsItem, c.status};
+    if (c.T > kChunk * seg) {   // some sequence may span several segments
+        P.mode_base = kChainState;   // z = 0: segment states (B), z = 1: segment transitions (M)
+        gdn_chunk_chain_kernel<<<dim3(c.Hv, seg_slots, 2), CH_THREADS, CH_SMEM, st>>>(P);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        gdn_segment_combine_kernel<<<dim3(c.Hv, c.num_seqs), NT, CB_SMEM, st>>>(P);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        P.mode_base = kChainFull;
+    }
+    gdn_chunk_chain_kernel<<<dim3(c.Hv, seg_slots, 1), CH_THREADS, CH_SMEM, st>>>(P);
     return cudaGetLastError();
 }
 
