@@ -323,25 +323,30 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     tc_fence_after();
     {
         // Q' rows (64 + r of the [W; Q'] image) and K'' (the first two blocks of [K''; P^T]):
-        // the converted tiles scaled row by row, swizzle positions unchanged
+        // the converted tiles scaled row by row, swizzle positions unchanged. Done by the four
+        // warps whose TMEM lanes (64-127) hold no needed D1 rows, while the other four read D1.
+        if (row >= 64) {
+            const int wt = (warp & 3) - 2 + 2 * wg;   // 0..3 over warps 2, 3, 6, 7
+            const int tt = wt * 32 + lane;
+#pragma unroll 4
+            for (int e = 0; e < 16; ++e) {
+                const int idx = e * 128 + tt;          // 2048 chunks: 1024 of Q, 1024 of K
+                const int isk = idx >> 10, w = idx & 1023, half = w >> 9, within = w & 511, r = within >> 3;
+                const uint8_t *src = sm + P_OFF_KQ + (2 * half + (isk ? 0 : 1)) * TILE + within * 16;
+                const float f = isk ? sDec[r] : sGam[r] * sRq[r];
+                const uint4 hv = *reinterpret_cast<const uint4 *>(src);
+                const __half2 *h2 = reinterpret_cast<const __half2 *>(&hv);
+                float x[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int idx = e * NT + tid;          // 2048 chunks: 1024 of Q, 1024 of K
-            const int isk = idx >> 10, w = idx & 1023, half = w >> 9, within = w & 511, r = within >> 3;
-            const uint8_t *src = sm + P_OFF_KQ + (2 * half + (isk ? 0 : 1)) * TILE + within * 16;
-            const float f = isk ? sDec[r] : sGam[r] * sRq[r];
-            const uint4 hv = *reinterpret_cast<const uint4 *>(src);
-            const __half2 *h2 = reinterpret_cast<const __half2 *>(&hv);
-            float x[8];
-#pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-                const float2 t = __half22float2(h2[q2]);
-                x[2 * q2] = t.x * f;
-                x[2 * q2 + 1] = t.y * f;
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const float2 t = __half22float2(h2[q2]);
+                    x[2 * q2] = t.x * f;
+                    x[2 * q2 + 1] = t.y * f;
+                }
+                uint8_t *dst = isk ? item + kWsKP + half * TILE + within * 16
+                                   : item + kWsWQ + half * 2 * TILE + TILE + within * 16;
+                st_h8(dst, x);
             }
-            uint8_t *dst = isk ? item + kWsKP + half * TILE + within * 16
-                               : item + kWsWQ + half * 2 * TILE + TILE + within * 16;
-            st_h8(dst, x);
         }
         // rows s of D1 (lanes 0-63): K K^T (warps 0-1) -> column s of A; K Q^T (warps 4-5) -> P^T row s
         if (row < 64) {
