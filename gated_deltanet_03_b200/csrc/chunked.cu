@@ -196,22 +196,24 @@ __device__ __forceinline__ void mma_m16n8k16(float (&c)[4], uint32_t a0, uint32_
 // ===================================================================================
 // Prep kernel: one CTA per (chunk slot, value head); two CTAs per SM.
 // ===================================================================================
-constexpr int P_OFF_KQ = 0;                       // [K_lo][Q_lo][K_hi][Q_hi], bf16 -> fp16 in place
-constexpr int P_OFF_V = 4 * TILE;                 // [V_lo][V_hi]
-constexpr int P_OFF_TP = 6 * TILE;                // T'  [s][r] fp16, swizzled
-constexpr int P_OFF_TPP = 7 * TILE;               // T'' [s][r] fp16, swizzled
-constexpr int P_AH = 72;                          // fp16 row pitch of A and T copies (144 B)
-constexpr int P_OFF_AH = 8 * TILE;                // A fp16 [64][72]
-constexpr int P_OFF_TF = P_OFF_AH + 64 * P_AH * 2;  // T fp32 [64][65]
-constexpr int P_OFF_TH = P_OFF_TF + 64 * 65 * 4;  // T fp16 [64][72]
-constexpr int P_OFF_XH = P_OFF_TH + 64 * P_AH * 2;  // X fp16 [3 warps][16][24]
-constexpr int P_OFF_STG = P_OFF_AH;               // W and U~ staging once A and T are dead (32 KB)
-constexpr int P_OFF_VEC = P_OFF_XH + 3 * 16 * 24 * 2; // G, beta, rk, rq, gamma, decS (64 each), row sums of squares (128)
+// Shared memory. [K_lo][Q_lo][K_hi][Q_hi] is the A operand [K; Q] (K-major, 128 rows); K_lo,
+// K_hi, V_lo, V_hi sit 2 TILE apart so that [K | V] is one MN-major B operand with N = 256.
+constexpr int P_OFF_KQ = 0;                        // staged bf16 tiles, converted to fp16 in place
+constexpr int P_OFF_VLO = 4 * TILE;
+constexpr int P_OFF_PST = 5 * TILE;                // P^T image, staged for the copy-out
+constexpr int P_OFF_VHI = 6 * TILE;
+constexpr int P_OFF_TP = 7 * TILE;                 // [T'; T''] fp16, K-major, 128-byte swizzled
+constexpr int P_OFF_TPP = 8 * TILE;
+constexpr int P_AH = 72;                           // fp16 row pitch of A and T (144 B)
+constexpr int P_OFF_AH = 9 * TILE;                 // A fp16 [64][72]
+constexpr int P_OFF_TH = P_OFF_AH + 64 * P_AH * 2; // T fp16 [64][72]
+constexpr int P_OFF_VEC = P_OFF_TH + 64 * P_AH * 2; // G, beta, rk, rq, gamma, decS (64 each), row sums of squares (128)
 constexpr int P_OFF_BAR = P_OFF_VEC + 8 * 64 * 4;
 constexpr int P_SMEM = P_OFF_BAR + 64 + 1024;
+constexpr int P_OFF_STG = 0;                       // W and U~ staging once the last MMA is done (32 KB)
 static_assert(P_SMEM * 2 <= 228 * 1024, "two prep CTAs per SM");
-static_assert(P_OFF_VEC - P_OFF_AH >= 4 * TILE, "staging fits in the A/T scratch");
-constexpr uint32_t P_TM_D1 = 0, P_TM_D2 = 128, P_TM_D3 = 192;
+// tensor memory: D1 = [K; Q] K^T (64 columns), then D2 = [T'; T''] [K | V] (256 columns) over it
+constexpr uint32_t P_TM_D1 = 0, P_TM_D2 = 0;
 
 __global__ void __launch_bounds__(NT, 2)
 gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict__ ga, const float *__restrict__ gb,
@@ -236,12 +238,11 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 2);
     __half *Ah = reinterpret_cast<__half *>(sm + P_OFF_AH);
-    float *Tf = reinterpret_cast<float *>(sm + P_OFF_TF);
     __half *Th = reinterpret_cast<__half *>(sm + P_OFF_TH);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int wg = warp / 4;
-    const int row = (warp % 4) * 32 + lane;
+    const int x = (warp % 4) * 32 + lane;   // this thread's TMEM lane
     const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
 
     if (tid == 0) {
@@ -253,8 +254,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         tma_load_3d(sm + P_OFF_KQ + 1 * TILE, &maps.q, bar_tma, 0, hk, t0);
         tma_load_3d(sm + P_OFF_KQ + 2 * TILE, &maps.k, bar_tma, 64, hk, t0);
         tma_load_3d(sm + P_OFF_KQ + 3 * TILE, &maps.q, bar_tma, 64, hk, t0);
-        tma_load_3d(sm + P_OFF_V + 0 * TILE, &maps.v, bar_tma, 0, h, t0);
-        tma_load_3d(sm + P_OFF_V + 1 * TILE, &maps.v, bar_tma, 64, h, t0);
+        tma_load_3d(sm + P_OFF_VLO, &maps.v, bar_tma, 0, h, t0);
+        tma_load_3d(sm + P_OFF_VHI, &maps.v, bar_tma, 64, h, t0);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 256);
@@ -264,13 +265,13 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     if (tid < 64) {
         float g = 0.0f, beta = 0.0f;
         if (tid < L) gdn_gates(ga[(size_t)(t0 + tid) * Hv + h], gb[(size_t)(t0 + tid) * Hv + h], A_log[h], dt_bias[h], g, beta);
-        float x = g;
+        float xs = g;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            float y = __shfl_up_sync(0xffffffffu, x, off);
-            if (lane >= off) x += y;
+            float y = __shfl_up_sync(0xffffffffu, xs, off);
+            if (lane >= off) xs += y;
         }
-        sG[tid] = x;
+        sG[tid] = xs;
         sBeta[tid] = beta;
     }
     tc_fence_before();
@@ -292,17 +293,21 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         ss += __shfl_xor_sync(0xffffffffu, ss, 1);
         if (half == 0) sSS[rho] = ss;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) convert16(sm + P_OFF_V + (e * NT + tid) * 16);
+        for (int e = 0; e < 4; ++e) {
+            const int idx = e * NT + tid;
+            convert16(sm + P_OFF_VLO + (idx >> 9) * 2 * TILE + (idx & 511) * 16);
+        }
     }
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
+        // D1 = [K; Q] K^T: lanes 0-63 K K^T, lanes 64-127 Q K^T (row = token, column = key token)
         tc_fence_after();
-        const uint32_t id1 = idesc_f16(128, false, false, false);
+        const uint32_t id1 = idesc_f16(64, false, false, false);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const uint8_t *abase = sm + P_OFF_KQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
-            mma_f16(tmem + P_TM_D1, kdesc(abase), kdesc(abase), id1, kk > 0 ? 1u : 0u);
+            const uint8_t *base = sm + P_OFF_KQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
+            mma_f16(tmem + P_TM_D1, kdesc(base), kdesc(base), id1, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar_mma);
     }
@@ -322,196 +327,194 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     if (!__syncthreads_and(ok)) goto teardown;
     tc_fence_after();
     {
-        // Q' rows (64 + r of the [W; Q'] image) and K'' (the first two blocks of [K''; P^T]):
-        // the converted tiles scaled row by row, swizzle positions unchanged. Done by the four
-        // warps whose TMEM lanes (64-127) hold no needed D1 rows, while the other four read D1.
-        if (row >= 64) {
-            const int wt = (warp & 3) - 2 + 2 * wg;   // 0..3 over warps 2, 3, 6, 7
-            const int tt = wt * 32 + lane;
-#pragma unroll 4
-            for (int e = 0; e < 16; ++e) {
-                const int idx = e * 128 + tt;          // 2048 chunks: 1024 of Q, 1024 of K
-                const int isk = idx >> 10, w = idx & 1023, half = w >> 9, within = w & 511, r = within >> 3;
-                const uint8_t *src = sm + P_OFF_KQ + (2 * half + (isk ? 0 : 1)) * TILE + within * 16;
-                const float f = isk ? sDec[r] : sGam[r] * sRq[r];
-                const uint4 hv = *reinterpret_cast<const uint4 *>(src);
-                const __half2 *h2 = reinterpret_cast<const __half2 *>(&hv);
-                float x[8];
+        // every warp reads 32 columns (key tokens s) of its 32 lanes
+        uint32_t r32[32];
+        tmem_ld32(tmem + P_TM_D1 + lane_base + wg * 32, r32);
+        tmem_ld_wait();
+        if (x < 64) {
+            // row r of A: A_rs = beta_r exp(G_r - G_s) k_r.k_s / (|k_r| |k_s|) for s < r < L
+            const int r = x;
+            const float Gr = sG[r], cr = sBeta[r] * sRk[r];
 #pragma unroll
-                for (int q2 = 0; q2 < 4; ++q2) {
-                    const float2 t = __half22float2(h2[q2]);
-                    x[2 * q2] = t.x * f;
-                    x[2 * q2 + 1] = t.y * f;
+            for (int q8 = 0; q8 < 4; ++q8) {
+                float a8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int s = wg * 32 + q8 * 8 + e;
+                    a8[e] = (s < r) ? cr * __expf(Gr - sG[s]) * __uint_as_float(r32[q8 * 8 + e]) * sRk[s] : 0.0f;
                 }
-                uint8_t *dst = isk ? item + kWsKP + half * TILE + within * 16
-                                   : item + kWsWQ + half * 2 * TILE + TILE + within * 16;
-                st_h8(dst, x);
+                st_h8(reinterpret_cast<uint8_t *>(Ah + r * P_AH + wg * 32 + q8 * 8), a8);
             }
-        }
-        // rows s of D1 (lanes 0-63): K K^T (warps 0-1) -> column s of A; K Q^T (warps 4-5) -> P^T row s
-        if (row < 64) {
-            const int s = row;
-            const float Gs = sG[s], rks = sRk[s];
+        } else {
+            // row r of P = (Q K^T o Gamma) scaled, into the P^T image [s][r] (MN-major over r)
+            const int r = x - 64;
+            const float Gr = sG[r], cr = sRq[r];
 #pragma unroll
-            for (int hcol = 0; hcol < 2; ++hcol) {
-                uint32_t r32[32];
-                tmem_ld32(tmem + P_TM_D1 + lane_base + wg * 64 + hcol * 32, r32);
-                tmem_ld_wait();
-                if (wg == 0) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int r = hcol * 32 + j;
-                        float a = 0.0f;
-                        if (s < r && r < L) a = sBeta[r] * __expf(sG[r] - Gs) * __uint_as_float(r32[j]) * sRk[r] * rks;
-                        Ah[r * P_AH + s] = __float2half_rn(a);
-                    }
-                } else {
-                    float pv[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int r = hcol * 32 + j;
-                        pv[j] = (s <= r && r < L) ? __uint_as_float(r32[j]) * sRq[r] * rks * __expf(sG[r] - Gs) : 0.0f;
-                    }
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) st_h8(item + kWsKP + 2 * TILE + swz(s, hcol * 4 + ch), &pv[ch * 8]);
-                }
+            for (int j = 0; j < 32; ++j) {
+                const int s = wg * 32 + j;
+                const float pv = (s <= r) ? cr * __expf(Gr - sG[s]) * __uint_as_float(r32[j]) * sRk[s] : 0.0f;
+                *reinterpret_cast<__half *>(sm + P_OFF_PST + swz(s, r >> 3) + (r & 7) * 2) = __float2half_rn(pv);
             }
         }
     }
     tc_fence_before();
     __syncthreads();
 
-    // ---- T = (I + A)^-1: 16 x 16 diagonal blocks by forward substitution (fp32), then the
-    //      off-diagonal blocks level by level, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj, one
-    //      warp per block on the warp-level tensor-core MMA (fp16 inputs, fp32 accumulation).
+    // ---- T = (I + A)^-1 (unit lower triangular), written as T (fp16, for the block products)
+    //      and as the B operands T'' = T diag(beta), T' = T diag(beta gamma / |k|). Two warps
+    //      solve the 16 x 16 diagonal blocks by forward substitution (fp32) while the other six
+    //      write the state-independent images: Q' and K'' from the converted tiles, P^T from its
+    //      staging, and the zero upper blocks of T' and T''.
     if (tid < 64) {
-        const int bi = tid / 16, cc = tid % 16, o0 = bi * 16;
-        float x[16];
+        const int bi = tid / 16, cc = tid % 16, o0 = bi * 16, r = o0 + cc;
+        float xv[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = (r == cc) ? 1.0f : 0.0f;
+        for (int rr = 0; rr < 16; ++rr) {
+            float acc = (rr == cc) ? 1.0f : 0.0f;
 #pragma unroll
-            for (int s = 0; s < r; ++s) acc -= __half2float(Ah[(o0 + r) * P_AH + o0 + s]) * x[s];
-            x[r] = acc;
+            for (int s = 0; s < rr; ++s) acc -= __half2float(Ah[(o0 + rr) * P_AH + o0 + s]) * xv[s];
+            xv[rr] = acc;
         }
+        const float fb = sBeta[r], fbg = fb * sGam[r] * sRk[r];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            Tf[(o0 + r) * 65 + o0 + cc] = x[r];
-            Th[(o0 + r) * P_AH + o0 + cc] = __float2half_rn(x[r]);
+        for (int rr = 0; rr < 16; ++rr) {
+            const int s = o0 + rr;
+            const uint32_t off = swz(s, r >> 3) + (r & 7) * 2;
+            Th[s * P_AH + r] = __float2half_rn(xv[rr]);
+            *reinterpret_cast<__half *>(sm + P_OFF_TPP + off) = __float2half_rn(xv[rr] * fb);
+            *reinterpret_cast<__half *>(sm + P_OFF_TP + off) = __float2half_rn(xv[rr] * fbg);
+        }
+    } else {
+        for (int idx = tid - 64; idx < 2048 + 512 + 384; idx += NT - 64) {
+            if (idx < 2048) {
+                // Q' rows (64 + r of the [W; Q'] image), K'' (the first two blocks of [K''; P^T]):
+                // converted tiles scaled row by row, swizzle positions unchanged
+                const int isk = idx >> 10, w = idx & 1023, half = w >> 9, within = w & 511, r = within >> 3;
+                const uint8_t *src = sm + P_OFF_KQ + (2 * half + (isk ? 0 : 1)) * TILE + within * 16;
+                const float f = isk ? sDec[r] : sGam[r] * sRq[r];
+                const uint4 hv = *reinterpret_cast<const uint4 *>(src);
+                const __half2 *h2 = reinterpret_cast<const __half2 *>(&hv);
+                float xv[8];
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const float2 t = __half22float2(h2[q2]);
+                    xv[2 * q2] = t.x * f;
+                    xv[2 * q2 + 1] = t.y * f;
+                }
+                uint8_t *dst = isk ? item + kWsKP + half * TILE + within * 16
+                                   : item + kWsWQ + half * 2 * TILE + TILE + within * 16;
+                st_h8(dst, xv);
+            } else if (idx < 2560) {
+                const int c16 = idx - 2048;
+                *reinterpret_cast<uint4 *>(item + kWsKP + 2 * TILE + c16 * 16) =
+                    *reinterpret_cast<const uint4 *>(sm + P_OFF_PST + c16 * 16);
+            } else {
+                // block (bi, bj), bj > bi, of T' and T'': 16 rows x two 16-byte chunks, zero
+                const int z = idx - 2560, img = z / 192, w = z % 192, blk = w >> 5, rr = (w >> 1) & 15, hc = w & 1;
+                const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                const int bj = bi + 1 + blk - (bi == 0 ? 0 : (bi == 1 ? 3 : 5));
+                *reinterpret_cast<uint4 *>(sm + (img ? P_OFF_TPP : P_OFF_TP) + swz(bi * 16 + rr, 2 * bj + hc)) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
         }
     }
     __syncthreads();
+    // off-diagonal blocks level by level, from T (I + A) = I:
+    //   T_ij = -(sum_{k=j+1}^{i} T_ik A_kj) T_jj,
+    // one warp per block on the warp-level tensor-core MMA (fp16 inputs, fp32 accumulation); the
+    // sum's accumulator fragments are directly the A fragments of the product with T_jj.
 #pragma unroll 1
     for (int lvl = 1; lvl < 4; ++lvl) {
         if (warp < 4 - lvl) {
             const int bj = warp, bi = bj + lvl;
             const int g = lane >> 2, t = lane & 3;
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            for (int bk = bj; bk < bi; ++bk) {
-                const uint32_t *arow0 = reinterpret_cast<const uint32_t *>(Ah + (bi * 16 + g) * P_AH + bk * 16);
-                const uint32_t *arow1 = reinterpret_cast<const uint32_t *>(Ah + (bi * 16 + g + 8) * P_AH + bk * 16);
-                const uint32_t a0 = arow0[t], a1 = arow1[t], a2 = arow0[t + 4], a3 = arow1[t + 4];
+            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int bk = bj + 1; bk <= bi; ++bk) {
+                const uint32_t *trow0 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g) * P_AH + bk * 16);
+                const uint32_t *trow1 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g + 8) * P_AH + bk * 16);
+                const uint32_t a0 = trow0[t], a1 = trow1[t], a2 = trow0[t + 4], a3 = trow1[t + 4];
 #pragma unroll
                 for (int hn = 0; hn < 2; ++hn) {
                     const int col = bj * 16 + hn * 8 + g;
-                    const uint32_t b0 = pack_two_h(Th[(bk * 16 + 2 * t) * P_AH + col], Th[(bk * 16 + 2 * t + 1) * P_AH + col]);
-                    const uint32_t b1 = pack_two_h(Th[(bk * 16 + 2 * t + 8) * P_AH + col], Th[(bk * 16 + 2 * t + 9) * P_AH + col]);
-                    mma_m16n8k16(acc[hn], a0, a1, a2, a3, b0, b1);
+                    const uint32_t b0 = pack_two_h(Ah[(bk * 16 + 2 * t) * P_AH + col], Ah[(bk * 16 + 2 * t + 1) * P_AH + col]);
+                    const uint32_t b1 = pack_two_h(Ah[(bk * 16 + 2 * t + 8) * P_AH + col], Ah[(bk * 16 + 2 * t + 9) * P_AH + col]);
+                    mma_m16n8k16(y[hn], a0, a1, a2, a3, b0, b1);
                 }
             }
-            // X (fp16, per-warp scratch [16][24]) as the B operand of T_ij = -T_ii X
-            __half *Xh = reinterpret_cast<__half *>(sm + P_OFF_XH) + warp * 16 * 24;
+            const uint32_t a0 = pack_h2(y[0][0], y[0][1]), a1 = pack_h2(y[0][2], y[0][3]);
+            const uint32_t a2 = pack_h2(y[1][0], y[1][1]), a3 = pack_h2(y[1][2], y[1][3]);
 #pragma unroll
             for (int hn = 0; hn < 2; ++hn) {
-                Xh[g * 24 + hn * 8 + 2 * t] = __float2half_rn(acc[hn][0]);
-                Xh[g * 24 + hn * 8 + 2 * t + 1] = __float2half_rn(acc[hn][1]);
-                Xh[(g + 8) * 24 + hn * 8 + 2 * t] = __float2half_rn(acc[hn][2]);
-                Xh[(g + 8) * 24 + hn * 8 + 2 * t + 1] = __float2half_rn(acc[hn][3]);
-            }
-            __syncwarp();
-            const uint32_t *trow0 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g) * P_AH + bi * 16);
-            const uint32_t *trow1 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g + 8) * P_AH + bi * 16);
-            const uint32_t a0 = trow0[t], a1 = trow1[t], a2 = trow0[t + 4], a3 = trow1[t + 4];
-#pragma unroll
-            for (int hn = 0; hn < 2; ++hn) {
-                const int col = hn * 8 + g;
-                const uint32_t b0 = pack_two_h(Xh[(2 * t) * 24 + col], Xh[(2 * t + 1) * 24 + col]);
-                const uint32_t b1 = pack_two_h(Xh[(2 * t + 8) * 24 + col], Xh[(2 * t + 9) * 24 + col]);
+                const int col = bj * 16 + hn * 8 + g;
+                const uint32_t b0 = pack_two_h(Th[(bj * 16 + 2 * t) * P_AH + col], Th[(bj * 16 + 2 * t + 1) * P_AH + col]);
+                const uint32_t b1 = pack_two_h(Th[(bj * 16 + 2 * t + 8) * P_AH + col], Th[(bj * 16 + 2 * t + 9) * P_AH + col]);
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
                 mma_m16n8k16(d, a0, a1, a2, a3, b0, b1);
                 const int c0 = bj * 16 + hn * 8 + 2 * t;
-                const int r0 = bi * 16 + g;
-                Tf[r0 * 65 + c0] = -d[0];
-                Tf[r0 * 65 + c0 + 1] = -d[1];
-                Tf[(r0 + 8) * 65 + c0] = -d[2];
-                Tf[(r0 + 8) * 65 + c0 + 1] = -d[3];
-                Th[r0 * P_AH + c0] = __float2half_rn(-d[0]);
-                Th[r0 * P_AH + c0 + 1] = __float2half_rn(-d[1]);
-                Th[(r0 + 8) * P_AH + c0] = __float2half_rn(-d[2]);
-                Th[(r0 + 8) * P_AH + c0 + 1] = __float2half_rn(-d[3]);
+                const float fb0 = sBeta[c0], fb1 = sBeta[c0 + 1];
+                const float fg0 = fb0 * sGam[c0] * sRk[c0], fg1 = fb1 * sGam[c0 + 1] * sRk[c0 + 1];
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int s = bi * 16 + g + 8 * hr;
+                    const float t0v = -d[2 * hr], t1v = -d[2 * hr + 1];
+                    const uint32_t off = swz(s, c0 >> 3) + (c0 & 7) * 2;
+                    *reinterpret_cast<uint32_t *>(Th + s * P_AH + c0) = pack_h2(t0v, t1v);
+                    *reinterpret_cast<uint32_t *>(sm + P_OFF_TPP + off) = pack_h2(t0v * fb0, t1v * fb1);
+                    *reinterpret_cast<uint32_t *>(sm + P_OFF_TP + off) = pack_h2(t0v * fg0, t1v * fg1);
+                }
             }
         }
         __syncthreads();
     }
-    {
-        // T' = T diag(beta gamma / |k|), T'' = T diag(beta): fp16 B operands [s][r] (r <= s)
-        const int s = tid % 64, part = tid / 64;
-        float tp[16], tpp[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int r = part * 16 + e;
-            const float t = (r <= s) ? Tf[s * 65 + r] : 0.0f;
-            tpp[e] = t * sBeta[r];
-            tp[e] = tpp[e] * sGam[r] * sRk[r];
-        }
-        st_h8(sm + P_OFF_TP + swz(s, part * 2), tp);
-        st_h8(sm + P_OFF_TP + swz(s, part * 2 + 1), tp + 8);
-        st_h8(sm + P_OFF_TPP + swz(s, part * 2), tpp);
-        st_h8(sm + P_OFF_TPP + swz(s, part * 2 + 1), tpp + 8);
-    }
     fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
     if (tid == 0) {
+        // D2 = [T'; T''] [K | V]: lanes 0-63 columns 0-127 hold W = T' K, lanes 64-127
+        // columns 128-255 hold U~ = T'' V (the other two quadrants are not used)
         tc_fence_after();
-        const uint32_t id_mn = idesc_f16(64, true, false, false);
+        const uint32_t id2 = idesc_f16(256, false, true, false);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)   // D2 = K^T T'^T  (A: K, MN-major over j)
-            mma_f16(tmem + P_TM_D2, mndesc(sm + P_OFF_KQ + kk * 2048, 2 * TILE), kdesc(sm + P_OFF_TP + kk * 32), id_mn,
-                    kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)   // D3 = V^T T''^T
-            mma_f16(tmem + P_TM_D3, mndesc(sm + P_OFF_V + kk * 2048, TILE), kdesc(sm + P_OFF_TPP + kk * 32), id_mn,
-                    kk > 0);
+        for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem + P_TM_D2, kdesc(sm + P_OFF_TP + kk * 32), mndesc(sm + P_OFF_KQ + kk * 2048, 2 * TILE), id2,
+                    kk > 0 ? 1u : 0u);
         tc_commit(bar_mma);
     }
     if (tid == 0) ok = mbar_wait(bar_mma, 1, status) ? 1 : 0;
     if (!__syncthreads_and(ok)) goto teardown;
     tc_fence_after();
     {
-        // W^T (lane j) -> W K-major [s][j] and U~^T (lane i) -> U~ [s][i], transposed through
-        // shared memory (the A/T scratch is dead), then copied out in 16-byte chunks
-        uint8_t *stg = sm + P_OFF_STG;
-        __half *uts = reinterpret_cast<__half *>(stg + 2 * TILE);
-        uint32_t wv32[32], uv32[32];
-        tmem_ld32(tmem + P_TM_D2 + lane_base + wg * 32, wv32);
-        tmem_ld32(tmem + P_TM_D3 + lane_base + wg * 32, uv32);
+        // W rows (K-major swizzled image halves) and U~ rows ([s][i], chunk positions XOR-swizzled
+        // by s & 7) staged in the dead tile area, then copied out in 16-byte chunks
+        uint32_t v0[32], v1[32];
+        const uint32_t col = (x < 64 ? 0u : 128u) + (uint32_t)wg * 64;
+        tmem_ld32(tmem + P_TM_D2 + lane_base + col, v0);
+        tmem_ld32(tmem + P_TM_D2 + lane_base + col + 32, v1);
         tmem_ld_wait();
-        const int j = row, hj = j >> 6, jj = j & 63;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const int s = wg * 32 + q;
-            *reinterpret_cast<__half *>(stg + hj * TILE + s * 128 + (((jj >> 3) ^ (s & 7)) << 4) + (jj & 7) * 2) =
-                __float2half_rn(__uint_as_float(wv32[q]));
+        for (int c = 0; c < 8; ++c) {
+            float f8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(c < 4 ? v0[c * 8 + e] : v1[(c - 4) * 8 + e]);
+            if (x < 64) st_h8(sm + P_OFF_STG + wg * TILE + swz(x, c), f8);
+            else {
+                const int s = x - 64;
+                st_h8(sm + P_OFF_STG + 2 * TILE + s * 256 + wg * 128 + ((c ^ (s & 7)) << 4), f8);
+            }
         }
-#pragma unroll
-        for (int q = 0; q < 32; ++q) uts[(wg * 32 + q) * D + row] = __float2half_rn(__uint_as_float(uv32[q]));
     }
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
         const int idx = e * NT + tid;   // 1024 chunks of W, then 1024 of U~
         const uint8_t *src = sm + P_OFF_STG + idx * 16;
-        uint8_t *dst = idx < 1024 ? item + kWsWQ + (idx >> 9) * 2 * TILE + (idx & 511) * 16 : item + kWsU + (idx - 1024) * 16;
+        uint8_t *dst;
+        if (idx < 1024) {
+            dst = item + kWsWQ + (idx >> 9) * 2 * TILE + (idx & 511) * 16;
+        } else {
+            const int u = idx - 1024, s = u >> 4, wgp = (u >> 3) & 1, c = (u & 7) ^ (s & 7);
+            dst = item + kWsU + s * 256 + wgp * 128 + c * 16;
+        }
         *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
     }
 teardown:
@@ -574,6 +577,29 @@ struct ChainParams {
 };
 constexpr size_t kSegItem = kSegItemBytes;
 constexpr size_t kSegB = 0, kSegMhi = 65536, kSegMlo = 98304, kSegS = 131072;
+
+// Segment states (B, start states) are stored lane-interleaved: the 16-byte group c4 of the
+// 64-column half wg of row i sits at ((wg * 16 + c4) * 128 + i) * 16, so that the thread owning
+// (row i, half wg) and its 31 neighbours touch 512 contiguous bytes per access.
+__device__ __forceinline__ size_t ilv_off(int row, int wg, int c4) {
+    return ((size_t)((wg * 16 + c4) * 128 + row)) * 16;
+}
+__device__ __forceinline__ void ilv_load(const uint8_t *base, int row, int wg, float (&S)[64]) {
+#pragma unroll
+    for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 x = *reinterpret_cast<const float4 *>(base + ilv_off(row, wg, c4));
+        S[4 * c4] = x.x; S[4 * c4 + 1] = x.y; S[4 * c4 + 2] = x.z; S[4 * c4 + 3] = x.w;
+    }
+}
+__device__ __forceinline__ void ilv_store(uint8_t *base, int row, int wg, const float (&S)[64]) {
+#pragma unroll
+    for (int c4 = 0; c4 < 16; ++c4)
+        *reinterpret_cast<float4 *>(base + ilv_off(row, wg, c4)) =
+            make_float4(S[4 * c4], S[4 * c4 + 1], S[4 * c4 + 2], S[4 * c4 + 3]);
+}
+// A row-major 128 x 128 fp32 state through shared memory (rows padded to 528 bytes, so both the
+// coalesced side and the row-per-thread side are free of bank conflicts); `tid` in 0..255.
+constexpr int kStgPitch = 528;
 
 __global__ void __launch_bounds__(CH_THREADS, 1)
 gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
@@ -679,26 +705,27 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
         const int row = (warp % 4) * 32 + lane;   // TMEM lane == value index i
         const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
         float S[64];   // S[i][64 wg .. 64 wg + 63], fp32
-        {
-            const float *src = nullptr;
-            size_t base = 0;
-            if (pseg == 0 && mode != kChainTransition && S0g) {
-                src = S0g;
-                base = (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
-            } else if (pseg > 0 && mode == kChainFull) {
-                src = reinterpret_cast<const float *>(seg_item + kSegS);
-                base = (size_t)row * D + 64 * wg;
+        if (pseg == 0 && mode != kChainTransition && S0g) {
+            // the caller's row-major initial state, staged in buffer 1 (its first chunk load is
+            // issued only after every worker has released S0 through bar_sready)
+            const float4 *src = reinterpret_cast<const float4 *>(S0g + ((size_t)n * Hv + h) * D * D);
+            uint8_t *stg = sm + kWsItem;
+#pragma unroll 4
+            for (int e = 0; e < 16; ++e) {
+                const int f = e * NT + tid;
+                *reinterpret_cast<float4 *>(stg + (f >> 5) * kStgPitch + (f & 31) * 16) = src[f];
             }
-            if (src) {
+            workers_sync();
 #pragma unroll
-                for (int c = 0; c < 64; c += 4) {
-                    float4 x = *reinterpret_cast<const float4 *>(src + base + c);
-                    S[c] = x.x; S[c + 1] = x.y; S[c + 2] = x.z; S[c + 3] = x.w;
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 64; ++c) S[c] = (mode == kChainTransition && row == 64 * wg + c) ? 1.0f : 0.0f;
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 x = *reinterpret_cast<const float4 *>(stg + row * kStgPitch + wg * 256 + c4 * 16);
+                S[4 * c4] = x.x; S[4 * c4 + 1] = x.y; S[4 * c4 + 2] = x.z; S[4 * c4 + 3] = x.w;
             }
+        } else if (pseg > 0 && mode == kChainFull) {
+            ilv_load(seg_item + kSegS, row, wg, S);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) S[c] = (mode == kChainTransition && row == 64 * wg + c) ? 1.0f : 0.0f;
         }
         // fp16 copy of S as an A operand: row i on lane i, key index j two per column
         auto store_S = [&](int slot) {
@@ -801,33 +828,43 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             }
         }
         if (alive) {
-            float *dst = nullptr;
-            if (mode == kChainFull && last_seg && P.S_out)
-                dst = P.S_out + (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
-            else if (mode == kChainState)
-                dst = reinterpret_cast<float *>(const_cast<uint8_t *>(seg_item) + kSegB) + (size_t)row * D + 64 * wg;
-            if (dst) {
+            // all chunks are consumed: both operand buffers are free for staging
+            if (mode == kChainFull && last_seg && P.S_out) {
+                uint8_t *stg = sm;
 #pragma unroll
-                for (int c = 0; c < 64; c += 4)
-                    *reinterpret_cast<float4 *>(dst + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
-            }
-            if (mode == kChainTransition) {
+                for (int c4 = 0; c4 < 16; ++c4)
+                    *reinterpret_cast<float4 *>(stg + row * kStgPitch + wg * 256 + c4 * 16) =
+                        make_float4(S[4 * c4], S[4 * c4 + 1], S[4 * c4 + 2], S[4 * c4 + 3]);
+                workers_sync();
+                float4 *dst = reinterpret_cast<float4 *>(P.S_out + ((size_t)n * Hv + h) * D * D);
+#pragma unroll 4
+                for (int e = 0; e < 16; ++e) {
+                    const int f = e * NT + tid;
+                    dst[f] = *reinterpret_cast<const float4 *>(stg + (f >> 5) * kStgPitch + (f & 31) * 16);
+                }
+            } else if (mode == kChainState) {
+                ilv_store(const_cast<uint8_t *>(seg_item) + kSegB, row, wg, S);
+            } else if (mode == kChainTransition) {
                 // the segment's map M (row j = this lane) as fp16 hi / lo B operand images,
-                // MN-major over the output column, 128-byte swizzled rows
-                uint8_t *mhi = const_cast<uint8_t *>(seg_item) + kSegMhi + wg * 16384;
-                uint8_t *mlo = const_cast<uint8_t *>(seg_item) + kSegMlo + wg * 16384;
+                // MN-major over the output column, 128-byte swizzled rows: built in shared
+                // memory, then copied out in 16-byte chunks
+                uint8_t *mhi = sm + wg * 16384, *mlo = sm + 32768 + wg * 16384;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
                     float hi8[8], lo8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float x = S[ch * 8 + e];
-                        hi8[e] = __half2float(__float2half_rn(x));
-                        lo8[e] = x - hi8[e];
+                        const float xv = S[ch * 8 + e];
+                        hi8[e] = __half2float(__float2half_rn(xv));
+                        lo8[e] = xv - hi8[e];
                     }
                     st_h8(mhi + swz(row, ch), hi8);
                     st_h8(mlo + swz(row, ch), lo8);
                 }
+                workers_sync();
+                uint4 *dst = reinterpret_cast<uint4 *>(const_cast<uint8_t *>(seg_item) + kSegMhi);
+#pragma unroll 4
+                for (int e = 0; e < 16; ++e) dst[e * NT + tid] = reinterpret_cast<const uint4 *>(sm)[e * NT + tid];
             }
         }
     }
@@ -896,16 +933,8 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
     if (tid == 0 && nseg > 2) issue_m(1);
 
     float S[64];
-    {
-        const float *b0 = reinterpret_cast<const float *>(seg(0) + kSegB) + (size_t)row * D + 64 * wg;
-        float *s1 = reinterpret_cast<float *>(seg(1) + kSegS) + (size_t)row * D + 64 * wg;
-#pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(b0 + c);
-            S[c] = x.x; S[c + 1] = x.y; S[c + 2] = x.z; S[c + 3] = x.w;
-            *reinterpret_cast<float4 *>(s1 + c) = x;
-        }
-    }
+    ilv_load(seg(0) + kSegB, row, wg, S);
+    ilv_store(seg(1) + kSegS, row, wg, S);
     const uint32_t idm = idesc_f16(128, false, true, false);
     for (int p = 1; p + 1 < nseg; ++p) {
         const int b = (p - 1) & 1;
@@ -950,18 +979,10 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
             }
         }
         float Bp[64];
-        {
-            const float *bp = reinterpret_cast<const float *>(seg(p) + kSegB) + (size_t)row * D + 64 * wg;
-#pragma unroll
-            for (int c = 0; c < 64; c += 4) {
-                const float4 x = *reinterpret_cast<const float4 *>(bp + c);
-                Bp[c] = x.x; Bp[c + 1] = x.y; Bp[c + 2] = x.z; Bp[c + 3] = x.w;
-            }
-        }
+        ilv_load(seg(p) + kSegB, row, wg, Bp);
         if (tid == 0 && ok) ok = mbar_wait(bar_mma, (uint32_t)((p - 1) & 1), P.status) ? 1 : 0;
         if (!__syncthreads_and(ok)) break;
         tc_fence_after();
-        float *sn = reinterpret_cast<float *>(seg(p + 1) + kSegS) + (size_t)row * D + 64 * wg;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             uint32_t r32[32];
@@ -970,9 +991,7 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) S[half * 32 + j] = __uint_as_float(r32[j]) + Bp[half * 32 + j];
         }
-#pragma unroll
-        for (int c = 0; c < 64; c += 4)
-            *reinterpret_cast<float4 *>(sn + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
+        ilv_store(seg(p + 1) + kSegS, row, wg, S);
         tc_fence_before();
     }
     tc_fence_before();

@@ -80,8 +80,10 @@ typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
  * Supported: Dk == Dv in {16, 32, 64, 128}; Hv % Hk == 0; T >= 0 (T == 0 only writes
  * final_state = initial_state). Dk == Dv == 128 with bf16 inputs runs the tensor-core
  * chunked path (64-token chunks; a prep kernel parallel over chunks writes the
- * state-independent operands to the workspace, a chain kernel walks the chunks of each
- * sequence; operands are staged in fp16, so |q|, |k|, |v| and the state must stay below
+ * state-independent operands to the workspace; long sequences are cut into segments whose
+ * states and transition matrices are computed in parallel and combined in order; a chain
+ * kernel then walks the chunks of each segment from its true start state; operands are
+ * staged in fp16, so |q|, |k|, |v| and the state must stay below
  * 6.5e4). Other sizes and fp32 inputs run the CUDA-core recurrent kernel (no workspace).
  */
 GDN_API gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v,
@@ -94,8 +96,13 @@ GDN_API gdn_status gdn_prefill_chunked(const void *q, const void *k, const void 
                                void *o, gdn_dtype out_dtype,
                                void *workspace, size_t workspace_bytes, gdn_stream_t stream);
 
-/* Scratch bytes the tensor-core path of gdn_prefill_chunked needs for these sizes:
- * Hv * (T / 64 + num_seqs) * 74752 when Dk == Dv == 128, else 0. Host-only, no CUDA call. */
+/* Scratch bytes the tensor-core path of gdn_prefill_chunked needs for these sizes, 0 unless
+ * Dk == Dv == 128. It is Hv * (T / 64 + num_seqs) * 74752 (state-independent operands, one
+ * item per 64-token chunk slot) plus Hv * (T / (64 * L) + num_seqs) * 196608 (per segment of
+ * L chunks: its state, its transition matrix, its start state), where the segment length L
+ * (a power of two, 4 <= L <= 4096) is picked on the host from T, num_seqs and Hv; so never
+ * more than Hv * (T / 64 + num_seqs) * 74752 + Hv * (T / 256 + num_seqs) * 196608.
+ * Host-only, no CUDA call. */
 GDN_API size_t gdn_prefill_workspace_bytes(int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv,
                                    int32_t Dk, int32_t Dv);
 
