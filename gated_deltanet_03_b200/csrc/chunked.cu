@@ -878,6 +878,228 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
 
 
 // ===================================================================================
+// Lean chain kernel for the state and transition passes (no outputs). A buffer holds only W,
+// K'', U~ and gamma_C of a chunk; 256 threads, thread 0 also issuing the copies and the MMAs;
+// 256 tensor-memory columns and at most 128 registers, so that two CTAs share an SM.
+// ===================================================================================
+constexpr int CL_W = 0, CL_K = 2 * TILE, CL_U = 4 * TILE, CL_VEC = 6 * TILE;
+constexpr int CL_BUF = 6 * TILE + 1024;
+constexpr int CL_OFF_BAR = 2 * CL_BUF;
+constexpr int CL_SMEM = CL_OFF_BAR + 64 + 1024;
+static_assert(2 * CL_SMEM <= 228 * 1024, "two lean chain CTAs per SM");
+// D4 (64 columns) and D7 (128) share columns: D4 is read out before MMA67 is issued
+constexpr uint32_t CL_TM_D4 = 0, CL_TM_D7 = 0, CL_TM_SA = 128, CL_TM_UA = 192;
+
+__global__ void __launch_bounds__(NT, 2)
+gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CL_OFF_BAR);
+    uint64_t *full = bars, *bar_mma = bars + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3);
+
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int h = blockIdx.x, id = blockIdx.y, mode = kChainState + (int)blockIdx.z;
+    const int T = P.T, Hv = P.Hv, SEG = P.seg_chunks;
+    int n = 0, t_begin = 0, t_end = T;
+    if (P.cu_seqlens) {
+        int lo = 0, hi = P.num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (P.cu_seqlens[mid] / (C * SEG) + mid <= id) lo = mid;
+            else hi = mid - 1;
+        }
+        n = lo;
+        t_begin = P.cu_seqlens[n];
+        t_end = P.cu_seqlens[n + 1];
+    }
+    const int nch_seq = (t_end - t_begin + C - 1) / C;
+    const int nseg = (nch_seq + SEG - 1) / SEG;
+    const int pseg = id - (t_begin / (C * SEG) + n);
+    // the last segment has no successor; the transition of the first is never needed
+    if (pseg < 0 || pseg >= nseg - 1) return;
+    if (mode == kChainTransition && pseg == 0) return;
+    const int c_first = pseg * SEG;
+    const int nchunks = max(0, min(nch_seq, c_first + SEG) - c_first);
+    const uint8_t *seg_item = P.ws_seg + ((size_t)h * P.seg_slots + id) * kSegItem;
+    const int slot0 = t_begin / C + n + c_first;
+    const uint8_t *ws_h = P.ws + (size_t)h * P.slots * kWsItem;
+    int *status = P.status;
+    const bool with_u = mode == kChainState;
+
+    if (tid == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_init(bar_mma, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    auto issue_chunk = [&](int c) {
+        uint64_t *bar = &full[c & 1];
+        uint8_t *dst = sm + (c & 1) * CL_BUF;
+        const uint8_t *item = ws_h + (size_t)(slot0 + c) * kWsItem;
+        mbar_arrive_expect_tx(bar, 4 * TILE + (with_u ? 2 * TILE : 0) + 16);
+        bulk_load(dst + CL_W, item + kWsWQ, TILE, bar);
+        bulk_load(dst + CL_W + TILE, item + kWsWQ + 2 * TILE, TILE, bar);
+        bulk_load(dst + CL_K, item + kWsKP, 2 * TILE, bar);
+        if (with_u) bulk_load(dst + CL_U, item + kWsU, 2 * TILE, bar);
+        bulk_load(dst + CL_VEC, item + kWsVec, 16, bar);
+    };
+    if (tid == 0) {
+        if (nchunks > 0) issue_chunk(0);
+        if (nchunks > 1) issue_chunk(1);
+    }
+
+    const int wg = warp / 4;
+    const int row = (warp % 4) * 32 + lane;   // TMEM lane == value index i
+    const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
+    float S[64];   // S[i][64 wg .. 64 wg + 63], fp32
+    if (mode == kChainState && pseg == 0 && P.S0g) {
+        const float *src = P.S0g + (((size_t)n * Hv + h) * D + row) * D + 64 * wg;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+            const float4 xv = *reinterpret_cast<const float4 *>(src + c);
+            S[c] = xv.x; S[c + 1] = xv.y; S[c + 2] = xv.z; S[c + 3] = xv.w;
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) S[c] = (mode == kChainTransition && row == 64 * wg + c) ? 1.0f : 0.0f;
+    }
+    // fp16 copy of S as the A operand of MMA45: row i on lane i, key index j two per column
+    auto store_S = [&]() {
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) pk[w] = pack_h2(S[part * 32 + 2 * w], S[part * 32 + 2 * w + 1]);
+            tmem_st16(tmem + lane_base + CL_TM_SA + wg * 32 + part * 16, pk);
+        }
+        tmem_st_wait();
+    };
+    store_S();
+
+    const uint32_t id45 = idesc_f16(64, false, false, false);
+    const uint32_t id67 = idesc_f16(128, false, true, false);
+    uint32_t mph = 0;
+    bool alive = true;
+    for (int c = 0; c < nchunks; ++c) {
+        const int L = min(C, t_end - (t_begin + (c_first + c) * C));
+        const int b = c & 1;
+        const uint8_t *buf = sm + b * CL_BUF;
+        tc_fence_before();
+        __syncthreads();   // S0 of this chunk is in tensor memory
+        int ok = 1;
+        if (tid == 0) {
+            ok = mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status) ? 1 : 0;
+            if (ok) {
+                tc_fence_after();
+                // D4 = S0 W^T   (B: W, K-major rows s, K = 128 key columns in two halves)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tmem + CL_TM_D4, tmem + CL_TM_SA + kk * 8,
+                               kdesc(buf + CL_W + (kk < 4 ? 0 : TILE) + (kk & 3) * 32), id45, kk > 0);
+                tc_commit(bar_mma);
+                ok = mbar_wait(bar_mma, mph, status) ? 1 : 0;
+            }
+            mph ^= 1u;
+        }
+        if (!__syncthreads_and(ok)) { alive = false; break; }
+        tc_fence_after();
+        const float gC = reinterpret_cast<const float *>(buf + CL_VEC)[0];
+        {
+            // U^T = U~^T - D4 (the transition pass takes U~ = 0) as the fp16 A operand of MMA67
+            const __half *ut = reinterpret_cast<const __half *>(buf + CL_U);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                uint32_t r16[16];
+                tmem_ld16(tmem + CL_TM_D4 + lane_base + wg * 32 + part * 16, r16);
+                tmem_ld_wait();
+                uint32_t ua[8];
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    const int s0 = wg * 32 + part * 16 + 2 * w;
+                    const float ut0 = with_u ? __half2float(ut[s0 * D + row]) : 0.0f;
+                    const float ut1 = with_u ? __half2float(ut[(s0 + 1) * D + row]) : 0.0f;
+                    const float u0 = (s0 < L) ? ut0 - __uint_as_float(r16[2 * w]) : 0.0f;
+                    const float u1 = (s0 + 1 < L) ? ut1 - __uint_as_float(r16[2 * w + 1]) : 0.0f;
+                    ua[w] = pack_h2(u0, u1);
+                }
+                tmem_st8(tmem + lane_base + CL_TM_UA + wg * 16 + part * 8, ua);
+            }
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncthreads();   // U is in tensor memory; D4 and this buffer's U~ are consumed
+        if (tid == 0) {
+            tc_fence_after();
+            // D7 = U^T K''   (B: K'', MN-major blocks of 64 keys, K = 64 tokens)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16_ts(tmem + CL_TM_D7, tmem + CL_TM_UA + kk * 8, mndesc(buf + CL_K + kk * 2048, TILE), id67,
+                           kk > 0);
+            tc_commit(bar_mma);
+            ok = mbar_wait(bar_mma, mph, status) ? 1 : 0;
+            mph ^= 1u;
+            if (ok && c + 2 < nchunks) {   // this buffer's last reader is done: refill it
+                fence_proxy_async_smem();
+                issue_chunk(c + 2);
+            }
+        }
+        if (!__syncthreads_and(ok)) { alive = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t r7[16];
+            tmem_ld16(tmem + CL_TM_D7 + lane_base + wg * 64 + q * 16, r7);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) S[q * 16 + j] = gC * S[q * 16 + j] + __uint_as_float(r7[j]);
+        }
+        store_S();
+    }
+    if (alive) {
+        if (mode == kChainState) {
+            ilv_store(const_cast<uint8_t *>(seg_item) + kSegB, row, wg, S);
+        } else {
+            // the segment's map M (row j = this lane) as fp16 hi / lo B operand images, MN-major
+            // over the output column, 128-byte swizzled rows: built in the (free) operand
+            // buffers, then copied out in 16-byte chunks
+            uint8_t *mhi = sm + wg * 16384, *mlo = sm + 32768 + wg * 16384;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                float hi8[8], lo8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float xv = S[ch * 8 + e];
+                    hi8[e] = __half2float(__float2half_rn(xv));
+                    lo8[e] = xv - hi8[e];
+                }
+                st_h8(mhi + swz(row, ch), hi8);
+                st_h8(mlo + swz(row, ch), lo8);
+            }
+            __syncthreads();
+            uint4 *dst = reinterpret_cast<uint4 *>(const_cast<uint8_t *>(seg_item) + kSegMhi);
+#pragma unroll 4
+            for (int e = 0; e < 16; ++e) dst[e * NT + tid] = reinterpret_cast<const uint4 *>(sm)[e * NT + tid];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+
+// ===================================================================================
 // Segment combine: per (value head, sequence), S_start(p + 1) = S_start(p) M_p + B_p in order,
 // S_start(1) = B_0. The product runs on the tensor cores with S split into fp16 hi + lo and M
 // given as fp16 hi + lo operand images (S_hi M_hi + S_lo M_hi + S_hi M_lo, fp32 accumulation).
@@ -1045,6 +1267,8 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(gdn_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
         if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn_chunk_lean_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CL_SMEM);
+        if (e == cudaSuccess)
             e = cudaFuncSetAttribute(gdn_segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CB_SMEM);
         if (e != cudaSuccess) return e;
         attr = true;
@@ -1062,7 +1286,7 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
                   c.S_out, c.o, ws, ws + (size_t)c.Hv * slots * kWsItem, c.status};
     if (c.T > kChunk * seg) {   // some sequence may span several segments
         P.mode_base = kChainState;   // z = 0: segment states (B), z = 1: segment transitions (M)
-        gdn_chunk_chain_kernel<<<dim3(c.Hv, seg_slots, 2), CH_THREADS, CH_SMEM, st>>>(P);
+        gdn_chunk_lean_kernel<<<dim3(c.Hv, seg_slots, 2), NT, CL_SMEM, st>>>(P);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         gdn_segment_combine_kernel<<<dim3(c.Hv, c.num_seqs), NT, CB_SMEM, st>>>(P);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
