@@ -33,6 +33,20 @@ METRIC = "GDN prefill tokens/s & decode GB/s (fraction of B200 roofline), 1 GPU"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+
+
+def make_l2_flush(torch, dev):
+    """L2 flush between timed steps: write a 256 MiB buffer (twice the 126 MB L2), then read a
+    second one, so the next step starts with neither its inputs nor dirty lines in L2 (the
+    write-back of the flush buffer happens here, outside the timed region)."""
+    wbuf = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
+    rbuf = torch.zeros((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush():
+        wbuf.zero_()
+        torch.sum(rbuf, dim=0, out=sink)
+    return flush
 CHUNK = 64
 # DRAM bytes (read + write) of one scan call (prep + chain kernels) on the benchmark workload,
 # from the ncu capture summarised in profiles/chunked_prefill_T4096.md; valid only for the
@@ -181,7 +195,7 @@ def run_gpu(args):
     gx = float(448.0 * 6.0 / y_cal.abs().max().item())
     alpha = float(np.float32(1.0) / (np.float32(gx) * np.float32(gw)))
     del y_cal
-    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=f32, device=dev)
+    flush = make_l2_flush(torch, dev)
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     ws = torch.empty((g.gdn_prefill_workspace_bytes(T, 1, w.Hk, Hv, D, D),), dtype=torch.uint8, device=dev)
@@ -201,7 +215,7 @@ def run_gpu(args):
         gemm()
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     assert g.gdn_get_device_status() == 0
@@ -223,7 +237,7 @@ def run_gpu(args):
     def timed(gr, n):
         out = []
         for _ in range(n):
-            flush.zero_()          # L2 flush between timed replays (outside the events)
+            flush()          # L2 flush between timed replays (outside the events)
             e0, e1 = ev(), ev()
             e0.record(stream)
             gr.replay()
@@ -274,7 +288,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     e2e_ms = []
     for _ in range(args.steps):
-        flush.zero_()
+        flush()
         s0, s1 = ev(), ev()
         s0.record(stream)
         e2e_step()
@@ -337,7 +351,7 @@ def run_gpu(args):
         "data": "synthetic (seeded; shapes of the pages' 1024-wide hybrid layer)",
         "config": {"workload": w.name, "T": T, "Hk": w.Hk, "Hv": Hv, "d": D, "chunk": CHUNK,
                    "out_proj": "NVFP4 W4A4 %d->%d" % (K, N), "global_batch": 1, "seq_len": T,
-                   "parallelism": "replicas x%d" % world, "l2": "flushed (256 MiB write) between timed steps"},
+                   "parallelism": "replicas x%d" % world, "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)"},
         "breakdown_ms": {"scan": statistics.mean(scan_ms), "gated_norm_nvfp4": statistics.mean(tail_ms),
                          "nvfp4_gemm": statistics.mean(gemm_ms), "timing": "CUDA graph replay per op"},
         "roofline": {"kernel": "gdn prefill scan (prep + chain kernels of one call)", "bound": "tensor", "achieved": achieved_tflops,
@@ -398,13 +412,13 @@ def run_only(args):
         "gemm": lambda: g.nvfp4_gemm(xq, xs, wq, ws, 1.0, y=Y),
         "decode": lambda: g.gdn_decode_step(q, k, v, a, b, A_log, dt_bias, S0, o=o),
     }[args.only]
-    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=f32, device=dev)
+    flush = make_l2_flush(torch, dev)
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
     times = []
     for _ in range(args.steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         fn()

@@ -7,13 +7,16 @@
 //
 // One CTA computes a 128 x 256 tile of y. Warp roles:
 //   warp 0   TMA producer: A (128 rows x 128 B) and B (256 rows x 128 B) tiles per stage,
-//            128-byte swizzle, into a 4-stage ring;
-//   warp 1   allocates tensor memory; lane 0 issues tcgen05.cp (scales) and tcgen05.mma;
-//   warp 2   scale re-layout: the stage's row-major [rows, 16 B] E4M3 scales (TMA-loaded with
-//            the tiles when K % 256 == 0, else gathered with plain loads and zero past K) are
-//            permuted in place into the 32x16-byte blocks the tensor core's scale copy reads
-//            (row r of a 128-row group at byte (r % 32) * 16 + (r / 32) * 4 + j);
-//   warps 4-7 epilogue: tensor memory -> registers -> alpha * acc -> y.
+//            128-byte swizzle, into a 4-stage ring, with the stage's row-major [rows, 16 B]
+//            E4M3 scales when K % 256 == 0;
+//   warp 1   allocates tensor memory; lane 0 issues tcgen05.mma;
+//   warps 4-7 scales, then the epilogue. Per stage each warp writes the scales into its lane
+//            quarter of the stage's tensor-memory scale slot with tcgen05.st (the layout the
+//            block-scaled MMA reads: for 32 rows r = 32 c + l, lane l, column 4 kb + c holds
+//            the four 16-value block scales of MMA k-step kb; the four lane quarters hold the
+//            same copy), read from the TMA-staged tile, or from global memory (zero past K)
+//            when the scales cannot be TMA-loaded. After the last stage: tensor memory ->
+//            registers -> alpha * acc -> 128-byte-swizzled shared-memory boxes -> TMA stores.
 // Every barrier wait is bounded (about 1 s); an expired wait records GDN_ERR_TIMEOUT and
 // the CTA finishes without issuing more work.
 #include <mutex>
@@ -36,8 +39,9 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barrier
 constexpr int THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0;             // accumulator: 128 lanes x 256 columns fp32
-constexpr uint32_t TM_SFA = 256;           // 4 k-blocks x 4 columns
-constexpr uint32_t TM_SFB = 272;           // 4 k-blocks x 8 columns
+constexpr uint32_t TM_SF = 256;            // per stage slot: A scales 4 x 4 columns, B scales 4 x 8
+constexpr uint32_t SF_SLOT = 48;
+static_assert(TM_SF + STAGES * SF_SLOT <= TMEM_COLS, "scale slots fit in tensor memory");
 
 // Instruction descriptor, kind::mxf4nvf4 block-scaled: A and B E2M1 (format 1), K-major,
 // scales UE4M3, M = 128, N = 256, dense K = 64 per instruction.
@@ -52,6 +56,13 @@ struct Smem {
     __device__ uint8_t *sfa(int s) const { return base + s * STAGE_BYTES + A_BYTES + B_BYTES; }
     __device__ uint8_t *sfb(int s) const { return base + s * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES; }
 };
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
 
 // 16 scale bytes of one row for the k-range of a stage (zero past K or past the last row).
 __device__ __forceinline__ uint4 load_scale_row(const uint8_t *sf, int row, int rows, int kblk16, int nblk16) {
@@ -71,47 +82,10 @@ __device__ __forceinline__ uint4 load_scale_row(const uint8_t *sf, int row, int 
     return r;
 }
 
-// Scatter one row's 16 scale bytes (4 k-blocks x 4 scales) into the per-k-block scale
-// copies: k-block kb of a group of 128 rows is a 512-byte block, row r at word
-// (r % 32) * 4 + r / 32.
-__device__ __forceinline__ void put_scale_row(uint8_t *dst, int row_in_tile, int groups, uint4 v) {
-    const int grp = row_in_tile / 128, r = row_in_tile % 128;
-    uint32_t *w = reinterpret_cast<uint32_t *>(dst);
-    const int word = (r % 32) * 4 + r / 32;
-    const uint32_t vals[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int kb = 0; kb < 4; ++kb) w[(kb * groups + grp) * 128 + word] = vals[kb];
-}
-
-// In-place permutation of one stage's scales from [rows][16 B] (row-major, as loaded) into
-// the per-k-block 512-byte blocks: every lane loads all its words first, then stores.
-__device__ __forceinline__ void relayout_scales(uint8_t *sf, int rows, int lane) {
-    uint32_t *w = reinterpret_cast<uint32_t *>(sf);
-    const int groups = rows / 128;
-    uint32_t v[BN / 32][4];
-#pragma unroll
-    for (int i = 0; i < BN / 32; ++i) {
-        if (i < rows / 32) {
-            const uint4 x = reinterpret_cast<const uint4 *>(sf)[i * 32 + lane];
-            v[i][0] = x.x; v[i][1] = x.y; v[i][2] = x.z; v[i][3] = x.w;
-        }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int i = 0; i < BN / 32; ++i) {
-        if (i < rows / 32) {
-            const int r = i * 32 + lane, grp = r / 128, rr = r % 128;
-            const int word = (rr % 32) * 4 + rr / 32;
-#pragma unroll
-            for (int kb = 0; kb < 4; ++kb) w[(kb * groups + grp) * 128 + word] = v[i][kb];
-        }
-    }
-}
-
 __global__ void __launch_bounds__(THREADS, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                   const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
-                  int sf_tma, const uint8_t *__restrict__ sfa_g, const uint8_t *__restrict__ sfb_g, float alpha,
+                  const __grid_constant__ CUtensorMap map_y, int sf_tma, const uint8_t *__restrict__ sfa_g, const uint8_t *__restrict__ sfb_g, float alpha,
                   int M, int N, int K, int out_bf16, void *__restrict__ y, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -129,7 +103,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);      // TMA producer's expect_tx arrive
             mbar_init(&empty[s], 1);     // tcgen05.commit of the MMAs that read the stage
-            mbar_init(&sf_ready[s], 1);  // scale warp: the stage's scales are in place
+            mbar_init(&sf_ready[s], 4);  // scale warps: the stage's scales are in tensor memory
         }
         mbar_init(acc_full, 1);
         fence_barrier_init();
@@ -160,32 +134,6 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 }
             }
         }
-    } else if (warp == 2) {
-        for (int kt = 0; kt < num_k; ++kt) {
-            const int s = kt % STAGES;
-            const uint32_t ph = (kt / STAGES) & 1;
-            bool ok = true;
-            if (sf_tma) {
-                // scales arrive with the tiles; permute them in place once they land
-                if (lane == 0) ok = mbar_wait(&full[s], ph, status);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                relayout_scales(sm.sfa(s), BM, lane);
-                relayout_scales(sm.sfb(s), BN, lane);
-            } else {
-                if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, status);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                const int kb16 = kt * (BK / 16);
-                for (int r = lane; r < BM; r += 32)
-                    put_scale_row(sm.sfa(s), r, BM / 128, load_scale_row(sfa_g, tile_m * BM + r, M, kb16, nblk16));
-                for (int r = lane; r < BN; r += 32)
-                    put_scale_row(sm.sfb(s), r, BN / 128, load_scale_row(sfb_g, tile_n * BN + r, N, kb16, nblk16));
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sf_ready[s]);
-        }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc();
@@ -195,21 +143,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 const uint32_t ph = (kt / STAGES) & 1;
                 if (!mbar_wait(&full[s], ph, status) || !mbar_wait(&sf_ready[s], ph, status)) { ok = false; break; }
                 tc_fence_after();
-                // scales of the 4 k-blocks into tensor memory (one 32x128-bit block each,
-                // broadcast to the four lane quarters)
-#pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
-                    const uint64_t da = smem_desc(smem_u32(sm.sfa(s) + kb * 512), 0, 128, 0);
-                    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem + TM_SFA + kb * 4),
-                                 "l"(da));
-#pragma unroll
-                    for (int g = 0; g < BN / 128; ++g) {
-                        const uint64_t db = smem_desc(smem_u32(sm.sfb(s) + (kb * (BN / 128) + g) * 512), 0, 128, 0);
-                        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(
-                                         tmem + TM_SFB + kb * (BN / 32) + g * 4),
-                                     "l"(db));
-                    }
-                }
+                const uint32_t sf = tmem + TM_SF + s * SF_SLOT;
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb) {
                     const uint64_t adesc = smem_desc(smem_u32(sm.a(s)) + kb * 32, 16, 1024, 2);
@@ -220,8 +154,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                         "setp.ne.b32 p, %4, 0;\n\t"
                         "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
                         "}" ::"r"(tmem + TM_ACC),
-                        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(tmem + TM_SFA + kb * 4),
-                        "r"(tmem + TM_SFB + kb * (BN / 32)));
+                        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(sf + kb * 4), "r"(sf + 16 + kb * 8));
                 }
                 tc_commit(&empty[s]);
             }
@@ -229,32 +162,111 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         }
     } else if (warp >= 4) {
         const int quarter = warp - 4;  // == warp % 4: this warp's lane quarter of tensor memory
+        const uint32_t lane_q = (uint32_t)(quarter * 32) << 16;
         bool ok = true;
-        if (lane == 0) ok = mbar_wait(acc_full, 0, status);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        // ---- scales of every stage into tensor memory
+        for (int kt = 0; kt < num_k; ++kt) {
+            const int s = kt % STAGES;
+            const uint32_t ph = (kt / STAGES) & 1;
+            uint32_t ra[16], rb[32];
+            if (sf_tma) {
+                // the stage's scale tiles have landed (which also means the slot's previous
+                // MMAs are complete: the producer refilled the stage after they released it)
+                if (lane == 0) ok = mbar_wait(&full[s], ph, status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 v = reinterpret_cast<const uint4 *>(sm.sfa(s))[c * 32 + lane];
+                    ra[c] = v.x; ra[4 + c] = v.y; ra[8 + c] = v.z; ra[12 + c] = v.w;
+                }
+#pragma unroll
+                for (int gc = 0; gc < 8; ++gc) {   // row g * 128 + c * 32 + lane, gc = g * 4 + c
+                    const uint4 v = reinterpret_cast<const uint4 *>(sm.sfb(s))[gc * 32 + lane];
+                    rb[gc] = v.x; rb[8 + gc] = v.y; rb[16 + gc] = v.z; rb[24 + gc] = v.w;
+                }
+            } else {
+                // the slot is free once the MMAs of its previous stage have completed
+                if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                const int kb16 = kt * (BK / 16);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 v = load_scale_row(sfa_g, tile_m * BM + c * 32 + lane, M, kb16, nblk16);
+                    ra[c] = v.x; ra[4 + c] = v.y; ra[8 + c] = v.z; ra[12 + c] = v.w;
+                }
+#pragma unroll
+                for (int gc = 0; gc < 8; ++gc) {
+                    const uint4 v = load_scale_row(sfb_g, tile_n * BN + gc * 32 + lane, N, kb16, nblk16);
+                    rb[gc] = v.x; rb[8 + gc] = v.y; rb[16 + gc] = v.z; rb[24 + gc] = v.w;
+                }
+            }
+            const uint32_t sf = tmem + lane_q + TM_SF + s * SF_SLOT;
+            tmem_st16(sf, ra);
+            tmem_st16(sf + 16, *reinterpret_cast<const uint32_t(*)[16]>(&rb[0]));
+            tmem_st16(sf + 32, *reinterpret_cast<const uint32_t(*)[16]>(&rb[16]));
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sf_ready[s]);
+        }
+        // ---- epilogue
+        if (ok) {
+            if (lane == 0) ok = mbar_wait(acc_full, 0, status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+        const int ept = threadIdx.x - 128;   // 0..127: this thread's row of the tile
+        // every stage is consumed by then: the ring holds the output boxes, [128 rows][128 B] each
+        uint8_t *obox = base;
         if (ok) {
             tc_fence_after();
-            const int row = tile_m * BM + quarter * 32 + lane;
+            const int r = ept;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + TM_ACC + ((uint32_t)(quarter * 32) << 16) + c0, r);
+            for (int c1 = 0; c1 < BN; c1 += 64) {
+                uint32_t rr[2][32];   // two loads in flight per wait
+                tmem_ld32(tmem + TM_ACC + lane_q + c1, rr[0]);
+                tmem_ld32(tmem + TM_ACC + lane_q + c1 + 32, rr[1]);
                 tmem_ld_wait();
-                const int n0 = tile_n * BN + c0;
-                if (row < M && n0 < N) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int c0 = c1 + 32 * hh;
                     float v[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * alpha;
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rr[hh][j]) * alpha;
+                    if (out_bf16) {
+                        uint8_t *box = obox + (c0 / 64) * 16384 + r * 128;
 #pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        if (n0 + j < N) {
-                            const float (&v8)[8] = *reinterpret_cast<const float(*)[8]>(&v[j]);
-                            if (out_bf16) store8<true>(y, (size_t)row * N + n0 + j, v8);
-                            else store8<false>(y, (size_t)row * N + n0 + j, v8);
+                        for (int i = 0; i < 4; ++i) {
+                            const int chunk = (c0 % 64) / 8 + i;
+                            uint4 u;
+                            __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                p2[e] = __floats2bfloat162_rn(v[8 * i + 2 * e], v[8 * i + 2 * e + 1]);
+                            *reinterpret_cast<uint4 *>(box + ((chunk ^ (r & 7)) << 4)) = u;
                         }
+                    } else {
+                        uint8_t *box = obox + (c0 / 32) * 16384 + r * 128;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            *reinterpret_cast<float4 *>(box + ((i ^ (r & 7)) << 4)) =
+                                make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                     }
                 }
             }
+            fence_proxy_async_smem();
+        }
+        asm volatile("barrier.cta.sync 1, 128;" ::: "memory");
+        if (ok && ept == 0) {
+            const int nbox = out_bf16 ? BN * 2 / 128 : BN * 4 / 128;
+            const int esz = out_bf16 ? 2 : 4;
+            for (int b = 0; b < nbox; ++b) {
+                const int x = tile_n * BN * esz + b * 128;
+                if (x < N * esz) tma_store_2d(&map_y, obox + b * 16384, x, tile_m * BM);
+            }
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }
     }
 
@@ -315,6 +327,9 @@ cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
         msa = ma;   // unused
         msb = mb;
     }
+    CUtensorMap my;
+    const uint64_t y_row_bytes = (uint64_t)g.N * (g.out_bf16 ? 2 : 4);
+    if (!make_map(&my, g.y, (uint64_t)g.M, y_row_bytes, BM)) return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
@@ -322,7 +337,7 @@ cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
         attr_set = true;
     }
     dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM);
-    nvfp4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, msa, msb, sf_tma ? 1 : 0, g.as, g.bs, g.alpha, g.M,
+    nvfp4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, msa, msb, my, sf_tma ? 1 : 0, g.as, g.bs, g.alpha, g.M,
                                                          g.N, g.K, g.out_bf16 ? 1 : 0, g.y, g.status);
     return cudaGetLastError();
 }

@@ -16,6 +16,39 @@ namespace gdn {
 
 constexpr int kTailThreads = 256;
 
+// Eight consecutive values as loaded (bf16: one 16-byte word; fp32: two), converted on use.
+template <bool BF16>
+struct Raw8 {
+    uint4 a, b;
+    __device__ __forceinline__ void load(const void *base, size_t idx) {
+        if constexpr (BF16) {
+            a = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(base) + idx);
+        } else {
+            const uint4 *p = reinterpret_cast<const uint4 *>(reinterpret_cast<const float *>(base) + idx);
+            a = p[0];
+            b = p[1];
+        }
+    }
+    __device__ __forceinline__ void get(float (&x)[8]) const {
+        if constexpr (BF16) {
+            const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&a);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(p[i]);
+                x[2 * i] = f.x;
+                x[2 * i + 1] = f.y;
+            }
+        } else {
+            x[0] = __uint_as_float(a.x); x[1] = __uint_as_float(a.y); x[2] = __uint_as_float(a.z); x[3] = __uint_as_float(a.w);
+            x[4] = __uint_as_float(b.x); x[5] = __uint_as_float(b.y); x[6] = __uint_as_float(b.z); x[7] = __uint_as_float(b.w);
+        }
+    }
+};
+
+// Rows handled per thread per pass: all their loads are issued before any is consumed, so
+// that enough bytes are in flight to cover the HBM latency.
+constexpr int kTailUnroll = 4;
+
 template <int D, bool IN_BF16, bool OUT_BF16, bool NVFP4>
 __global__ void __launch_bounds__(kTailThreads)
 gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
@@ -24,42 +57,57 @@ gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
                      uint8_t *__restrict__ xs) {
     constexpr int LANES = D / 8;                 // lanes per head row, 8 values each
     constexpr int RPB = kTailThreads / LANES;    // head rows per block pass
+    constexpr int U = kTailUnroll;
     const int lane_in_row = threadIdx.x % LANES;
     const int col = lane_in_row * 8;
     float wv[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) wv[j] = w[col + j];
     const float inv_d = 1.0f / (float)D;
+    const int64_t stride = (int64_t)gridDim.x * RPB;
 
-    for (int64_t row = (int64_t)blockIdx.x * RPB + threadIdx.x / LANES; row - threadIdx.x / LANES < rows;
-         row += (int64_t)gridDim.x * RPB) {
-        const bool live = row < rows;
-        const size_t base = (size_t)(live ? row : 0) * D + col;
-        float ov[8], zv[8];
-        load8<IN_BF16>(o, base, ov);
-        load8<IN_BF16>(z, base, zv);
-        float ss = 0.0f;
+    // the loop condition is uniform over the block (the shuffles below need whole warps)
+    for (int64_t row0 = (int64_t)blockIdx.x * RPB + threadIdx.x / LANES; row0 - threadIdx.x / LANES < rows;
+         row0 += U * stride) {
+        Raw8<IN_BF16> ro[U], rz[U];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) ss += ov[j] * ov[j];
-        ss = group_sum<LANES>(ss);
-        const float inv_rms = rsqrtf(ss * inv_d + eps);
-        float yv[8];
+        for (int u = 0; u < U; ++u) {
+            const int64_t row = row0 + u * stride;
+            const size_t base = (size_t)(row < rows ? row : 0) * D + col;
+            ro[u].load(o, base);
+            rz[u].load(z, base);
+        }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) yv[j] = ov[j] * inv_rms * wv[j] * silu_fast(zv[j]);
-        if constexpr (!NVFP4) {
-            if (live) store8<OUT_BF16>(y, base, yv);
-        } else {
-            // y as the bf16 tensor the two-call path would hand to the encoder
+        for (int u = 0; u < U; ++u) {
+            const int64_t row = row0 + u * stride;
+            const bool live = row < rows;
+            const size_t base = (size_t)(live ? row : 0) * D + col;
+            float ov[8], zv[8];
+            ro[u].get(ov);
+            rz[u].get(zv);
+            float ss = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) yv[j] = round_bf16(yv[j]);
-            float amax = amax8(yv);
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // partner lane: same block
-            float r;
-            const uint32_t sb = nvfp4_block_scale(amax, gs, r);
-            const uint32_t packed = nvfp4_pack8(yv, r);
-            if (live) {
-                reinterpret_cast<uint32_t *>(xq)[base / 8] = packed;
-                if ((lane_in_row & 1) == 0) xs[base / 16] = (uint8_t)sb;
+            for (int j = 0; j < 8; ++j) ss += ov[j] * ov[j];
+            ss = group_sum<LANES>(ss);
+            const float inv_rms = rsqrtf(ss * inv_d + eps);
+            float yv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) yv[j] = ov[j] * inv_rms * wv[j] * silu_fast(zv[j]);
+            if constexpr (!NVFP4) {
+                if (live) store8<OUT_BF16>(y, base, yv);
+            } else {
+                // y as the bf16 tensor the two-call path would hand to the encoder
+#pragma unroll
+                for (int j = 0; j < 8; ++j) yv[j] = round_bf16(yv[j]);
+                float amax = amax8(yv);
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // partner lane: same block
+                float r;
+                const uint32_t sb = nvfp4_block_scale(amax, gs, r);
+                const uint32_t packed = nvfp4_pack8(yv, r);
+                if (live) {
+                    reinterpret_cast<uint32_t *>(xq)[base / 8] = packed;
+                    if ((lane_in_row & 1) == 0) xs[base / 16] = (uint8_t)sb;
+                }
             }
         }
     }
@@ -70,8 +118,8 @@ static cudaError_t launch_tail_t(const TailArgs &t, cudaStream_t st) {
     const int64_t rows = (int64_t)t.M * t.Hv;
     if (rows == 0) return cudaSuccess;
     constexpr int RPB = kTailThreads / (D / 8);
-    int64_t blocks = (rows + RPB - 1) / RPB;
-    const int64_t cap = 148 * 16;
+    int64_t blocks = (rows + RPB * kTailUnroll - 1) / (RPB * kTailUnroll);
+    const int64_t cap = 148 * 8;
     if (blocks > cap) blocks = cap;
     gated_rmsnorm_kernel<D, IN_BF16, OUT_BF16, NVFP4><<<(unsigned)blocks, kTailThreads, 0, st>>>(
         t.o, t.z, t.w, t.eps, rows, t.y, t.gs, t.xq, t.xs);
@@ -100,22 +148,35 @@ static cudaError_t launch_tail(const TailArgs &t, cudaStream_t st) {
 cudaError_t launch_gated_rmsnorm(const TailArgs &t, cudaStream_t st) { return launch_tail<false>(t, st); }
 cudaError_t launch_gated_rmsnorm_nvfp4(const TailArgs &t, cudaStream_t st) { return launch_tail<true>(t, st); }
 
-// One thread per 16-value block: two 16-byte loads (bf16) or four (fp32), one 8-byte store of
-// codes and one byte of scale.
+// One thread per 16-value block and pass position: two 16-byte loads (bf16) or four (fp32), one
+// 8-byte store of codes and one byte of scale; four blocks per thread per pass, loads first.
 template <bool IN_BF16>
 __global__ void __launch_bounds__(256)
 nvfp4_quantize_kernel(const void *__restrict__ x, int64_t nblocks, float gs,
                       uint8_t *__restrict__ xq, uint8_t *__restrict__ xs) {
-    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblocks;
-         blk += (int64_t)gridDim.x * blockDim.x) {
-        float lo[8], hi[8];
-        load8<IN_BF16>(x, (size_t)blk * 16, lo);
-        load8<IN_BF16>(x, (size_t)blk * 16 + 8, hi);
-        float r;
-        const uint32_t sb = nvfp4_block_scale(fmaxf(amax8(lo), amax8(hi)), gs, r);
-        uint2 packed = make_uint2(nvfp4_pack8(lo, r), nvfp4_pack8(hi, r));
-        reinterpret_cast<uint2 *>(xq)[blk] = packed;
-        xs[blk] = (uint8_t)sb;
+    constexpr int U = 4;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b0 < nblocks; b0 += U * stride) {
+        Raw8<IN_BF16> rlo[U], rhi[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t blk = b0 + u * stride < nblocks ? b0 + u * stride : b0;
+            rlo[u].load(x, (size_t)blk * 16);
+            rhi[u].load(x, (size_t)blk * 16 + 8);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t blk = b0 + u * stride;
+            if (blk >= nblocks) break;
+            float lo[8], hi[8];
+            rlo[u].get(lo);
+            rhi[u].get(hi);
+            float r;
+            const uint32_t sb = nvfp4_block_scale(fmaxf(amax8(lo), amax8(hi)), gs, r);
+            const uint2 packed = make_uint2(nvfp4_pack8(lo, r), nvfp4_pack8(hi, r));
+            reinterpret_cast<uint2 *>(xq)[blk] = packed;
+            xs[blk] = (uint8_t)sb;
+        }
     }
 }
 
@@ -123,7 +184,7 @@ cudaError_t launch_nvfp4_quantize(const void *x, bool in_bf16, int32_t M, int32_
                                   uint8_t *xq, uint8_t *xs, cudaStream_t st) {
     const int64_t nblocks = (int64_t)M * (K / 16);
     if (nblocks == 0) return cudaSuccess;
-    int64_t grid = (nblocks + 255) / 256;
+    int64_t grid = (nblocks + 1023) / 1024;
     if (grid > 148 * 8) grid = 148 * 8;
     if (in_bf16) nvfp4_quantize_kernel<true><<<(unsigned)grid, 256, 0, st>>>(x, nblocks, gs, xq, xs);
     else nvfp4_quantize_kernel<false><<<(unsigned)grid, 256, 0, st>>>(x, nblocks, gs, xq, xs);
