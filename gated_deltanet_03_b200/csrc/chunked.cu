@@ -331,30 +331,37 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         uint32_t r32[32];
         tmem_ld32(tmem + P_TM_D1 + lane_base + wg * 32, r32);
         tmem_ld_wait();
+        // decay and key-norm factors of this warp's 32 columns (same for all lanes), then all 32
+        // values, then the stores
+        float gs[32], rks[32], vals[32];
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            const float4 g4 = *reinterpret_cast<const float4 *>(sG + wg * 32 + j);
+            const float4 k4 = *reinterpret_cast<const float4 *>(sRk + wg * 32 + j);
+            gs[j] = g4.x; gs[j + 1] = g4.y; gs[j + 2] = g4.z; gs[j + 3] = g4.w;
+            rks[j] = k4.x; rks[j + 1] = k4.y; rks[j + 2] = k4.z; rks[j + 3] = k4.w;
+        }
         if (x < 64) {
             // row r of A: A_rs = beta_r exp(G_r - G_s) k_r.k_s / (|k_r| |k_s|) for s < r < L
             const int r = x;
             const float Gr = sG[r], cr = sBeta[r] * sRk[r];
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-                float a8[8];
+            for (int j = 0; j < 32; ++j)
+                vals[j] = (wg * 32 + j < r) ? cr * __expf(Gr - gs[j]) * __uint_as_float(r32[j]) * rks[j] : 0.0f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int s = wg * 32 + q8 * 8 + e;
-                    a8[e] = (s < r) ? cr * __expf(Gr - sG[s]) * __uint_as_float(r32[q8 * 8 + e]) * sRk[s] : 0.0f;
-                }
-                st_h8(reinterpret_cast<uint8_t *>(Ah + r * P_AH + wg * 32 + q8 * 8), a8);
-            }
+            for (int q8 = 0; q8 < 4; ++q8)
+                st_h8(reinterpret_cast<uint8_t *>(Ah + r * P_AH + wg * 32 + q8 * 8), &vals[q8 * 8]);
         } else {
             // row r of P = (Q K^T o Gamma) scaled, into the P^T image [s][r] (MN-major over r)
             const int r = x - 64;
             const float Gr = sG[r], cr = sRq[r];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int s = wg * 32 + j;
-                const float pv = (s <= r) ? cr * __expf(Gr - sG[s]) * __uint_as_float(r32[j]) * sRk[s] : 0.0f;
-                *reinterpret_cast<__half *>(sm + P_OFF_PST + swz(s, r >> 3) + (r & 7) * 2) = __float2half_rn(pv);
-            }
+            for (int j = 0; j < 32; ++j)
+                vals[j] = (wg * 32 + j <= r) ? cr * __expf(Gr - gs[j]) * __uint_as_float(r32[j]) * rks[j] : 0.0f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                *reinterpret_cast<__half *>(sm + P_OFF_PST + swz(wg * 32 + j, r >> 3) + (r & 7) * 2) =
+                    __float2half_rn(vals[j]);
         }
     }
     tc_fence_before();
@@ -385,37 +392,61 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             *reinterpret_cast<__half *>(sm + P_OFF_TP + off) = __float2half_rn(xv[rr] * fbg);
         }
     } else {
-        for (int idx = tid - 64; idx < 2048 + 512 + 384; idx += NT - 64) {
-            if (idx < 2048) {
-                // Q' rows (64 + r of the [W; Q'] image), K'' (the first two blocks of [K''; P^T]):
-                // converted tiles scaled row by row, swizzle positions unchanged
-                const int isk = idx >> 10, w = idx & 1023, half = w >> 9, within = w & 511, r = within >> 3;
-                const uint8_t *src = sm + P_OFF_KQ + (2 * half + (isk ? 0 : 1)) * TILE + within * 16;
-                const float f = isk ? sDec[r] : sGam[r] * sRq[r];
-                const uint4 hv = *reinterpret_cast<const uint4 *>(src);
-                const __half2 *h2 = reinterpret_cast<const __half2 *>(&hv);
-                float xv[8];
+        // Q' rows (64 + r of the [W; Q'] image) and K'' (the first two blocks of [K''; P^T]): the
+        // converted tiles scaled row by row, swizzle positions unchanged; 2048 chunks over 192
+        // threads in two batches whose loads are issued before any store
+        const int t6 = tid - 64;
 #pragma unroll
-                for (int q2 = 0; q2 < 4; ++q2) {
-                    const float2 t = __half22float2(h2[q2]);
-                    xv[2 * q2] = t.x * f;
-                    xv[2 * q2 + 1] = t.y * f;
-                }
-                uint8_t *dst = isk ? item + kWsKP + half * TILE + within * 16
-                                   : item + kWsWQ + half * 2 * TILE + TILE + within * 16;
-                st_h8(dst, xv);
-            } else if (idx < 2560) {
-                const int c16 = idx - 2048;
-                *reinterpret_cast<uint4 *>(item + kWsKP + 2 * TILE + c16 * 16) =
-                    *reinterpret_cast<const uint4 *>(sm + P_OFF_PST + c16 * 16);
-            } else {
-                // block (bi, bj), bj > bi, of T' and T'': 16 rows x two 16-byte chunks, zero
-                const int z = idx - 2560, img = z / 192, w = z % 192, blk = w >> 5, rr = (w >> 1) & 15, hc = w & 1;
-                const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-                const int bj = bi + 1 + blk - (bi == 0 ? 0 : (bi == 1 ? 3 : 5));
-                *reinterpret_cast<uint4 *>(sm + (img ? P_OFF_TPP : P_OFF_TP) + swz(bi * 16 + rr, 2 * bj + hc)) =
-                    make_uint4(0u, 0u, 0u, 0u);
+        for (int batch = 0; batch < 2; ++batch) {
+            uint4 hv[6];
+            float f[6];
+#pragma unroll
+            for (int e = 0; e < 6; ++e) {
+                const int idx = (batch * 6 + e) * 192 + t6;
+                const int ic = idx < 2048 ? idx : 0;
+                const int isk = ic >> 10, w = ic & 1023, half = w >> 9, within = w & 511, r = within >> 3;
+                hv[e] = *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + (2 * half + (isk ? 0 : 1)) * TILE + within * 16);
+                f[e] = isk ? sDec[r] : sGam[r] * sRq[r];
             }
+#pragma unroll
+            for (int e = 0; e < 6; ++e) {
+                const int idx = (batch * 6 + e) * 192 + t6;
+                if (idx < 2048) {
+                    const int isk = idx >> 10, w = idx & 1023, half = w >> 9, within = w & 511;
+                    const __half2 *h2 = reinterpret_cast<const __half2 *>(&hv[e]);
+                    float xv[8];
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const float2 t = __half22float2(h2[q2]);
+                        xv[2 * q2] = t.x * f[e];
+                        xv[2 * q2 + 1] = t.y * f[e];
+                    }
+                    st_h8(isk ? item + kWsKP + half * TILE + within * 16 : item + kWsWQ + half * 2 * TILE + TILE + within * 16,
+                          xv);
+                }
+            }
+        }
+        // the P^T image from its staging (512 chunks)
+        uint4 pc[3];
+#pragma unroll
+        for (int e = 0; e < 3; ++e) {
+            const int c16 = e * 192 + t6;
+            pc[e] = *reinterpret_cast<const uint4 *>(sm + P_OFF_PST + (c16 < 512 ? c16 : 0) * 16);
+        }
+#pragma unroll
+        for (int e = 0; e < 3; ++e) {
+            const int c16 = e * 192 + t6;
+            if (c16 < 512) *reinterpret_cast<uint4 *>(item + kWsKP + 2 * TILE + c16 * 16) = pc[e];
+        }
+        // blocks (bi, bj), bj > bi, of T' and T'': 16 rows x two 16-byte chunks each, zero
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int z = e * 192 + t6;   // 384 chunks
+            const int img = z / 192, w = z % 192, blk = w >> 5, rr = (w >> 1) & 15, hc = w & 1;
+            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int bj = bi + 1 + blk - (bi == 0 ? 0 : (bi == 1 ? 3 : 5));
+            *reinterpret_cast<uint4 *>(sm + (img ? P_OFF_TPP : P_OFF_TP) + swz(bi * 16 + rr, 2 * bj + hc)) =
+                make_uint4(0u, 0u, 0u, 0u);
         }
     }
     __syncthreads();
