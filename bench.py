@@ -51,7 +51,7 @@ CHUNK = 64
 # DRAM bytes (read + write) of one scan call (prep + chain kernels) on the benchmark workload,
 # from the ncu capture summarised in profiles/chunked_prefill_T4096.md; valid only for the
 # kernel source it was taken on (first 16 hex digits of its sha256).
-SCAN_TRAFFIC = {"04f0c0687cf454f6": 154.1e6}
+SCAN_TRAFFIC = {"e8775da24552684d": 220.727e6}   # prep + lean + combine + chain, one call, ncu cold caches
 
 
 def source_digest(path: str) -> str:
