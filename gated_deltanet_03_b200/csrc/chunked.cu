@@ -347,7 +347,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             const float Gr = sG[r], cr = sBeta[r] * sRk[r];
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                vals[j] = (wg * 32 + j < r) ? cr * __expf(Gr - gs[j]) * __uint_as_float(r32[j]) * rks[j] : 0.0f;
+                vals[j] = (wg * 32 + j < r) ? cr * exp_approx(Gr - gs[j]) * __uint_as_float(r32[j]) * rks[j] : 0.0f;
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8)
                 st_h8(reinterpret_cast<uint8_t *>(Ah + r * P_AH + wg * 32 + q8 * 8), &vals[q8 * 8]);
@@ -357,7 +357,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             const float Gr = sG[r], cr = sRq[r];
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                vals[j] = (wg * 32 + j <= r) ? cr * __expf(Gr - gs[j]) * __uint_as_float(r32[j]) * rks[j] : 0.0f;
+                vals[j] = (wg * 32 + j <= r) ? cr * exp_approx(Gr - gs[j]) * __uint_as_float(r32[j]) * rks[j] : 0.0f;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
                 *reinterpret_cast<__half *>(sm + P_OFF_PST + swz(wg * 32 + j, r >> 3) + (r & 7) * 2) =
