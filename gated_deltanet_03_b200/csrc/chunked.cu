@@ -789,18 +789,24 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             tc_fence_after();
             {
                 // U^T = U~^T - D4 as the fp16 A operand of MMA67
+                const __half *ut = reinterpret_cast<const __half *>(buf + kWsU);
+                __half2 u2[16];
+#pragma unroll
+                for (int w = 0; w < 16; ++w) {
+                    const int s0 = wg * 32 + 2 * w;
+                    u2[w] = mode == kChainTransition ? __float2half2_rn(0.0f)
+                                                     : __halves2half2(ut[s0 * D + row], ut[(s0 + 1) * D + row]);
+                }
                 uint32_t r32[32];
                 tmem_ld32(tmem + C_TM_D45 + lane_base + wg * 32, r32);
                 tmem_ld_wait();
-                const __half *ut = reinterpret_cast<const __half *>(buf + kWsU);
                 uint32_t ua[16];
 #pragma unroll
                 for (int w = 0; w < 16; ++w) {
                     const int s0 = wg * 32 + 2 * w;
-                    const float ut0 = mode == kChainTransition ? 0.0f : __half2float(ut[s0 * D + row]);
-                    const float ut1 = mode == kChainTransition ? 0.0f : __half2float(ut[(s0 + 1) * D + row]);
-                    const float u0 = (s0 < L) ? ut0 - __uint_as_float(r32[2 * w]) : 0.0f;
-                    const float u1 = (s0 + 1 < L) ? ut1 - __uint_as_float(r32[2 * w + 1]) : 0.0f;
+                    const float2 uf = __half22float2(u2[w]);
+                    const float u0 = (s0 < L) ? uf.x - __uint_as_float(r32[2 * w]) : 0.0f;
+                    const float u1 = (s0 + 1 < L) ? uf.y - __uint_as_float(r32[2 * w + 1]) : 0.0f;
                     ua[w] = pack_h2(u0, u1);
                 }
                 tmem_st16(tmem + lane_base + C_TM_UA + wg * 16, ua);
@@ -884,10 +890,12 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
                 for (int ch = 0; ch < 8; ++ch) {
                     float hi8[8], lo8[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float xv = S[ch * 8 + e];
-                        hi8[e] = __half2float(__float2half_rn(xv));
-                        lo8[e] = xv - hi8[e];
+                    for (int e = 0; e < 8; e += 2) {
+                        const float2 hf = __half22float2(__floats2half2_rn(S[ch * 8 + e], S[ch * 8 + e + 1]));
+                        hi8[e] = hf.x;
+                        hi8[e + 1] = hf.y;
+                        lo8[e] = S[ch * 8 + e] - hf.x;
+                        lo8[e + 1] = S[ch * 8 + e + 1] - hf.y;
                     }
                     st_h8(mhi + swz(row, ch), hi8);
                     st_h8(mlo + swz(row, ch), lo8);
@@ -1046,7 +1054,15 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
         const float gC = reinterpret_cast<const float *>(buf + CL_VEC)[0];
         {
             // U^T = U~^T - D4 (the transition pass takes U~ = 0) as the fp16 A operand of MMA67
+            // this thread's 32 values of U~ (tokens 32 wg .. 32 wg + 31 of value row i), loaded
+            // before any tensor-memory access so that the loads overlap
             const __half *ut = reinterpret_cast<const __half *>(buf + CL_U);
+            __half2 u2[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+                const int s0 = wg * 32 + 2 * w;
+                u2[w] = with_u ? __halves2half2(ut[s0 * D + row], ut[(s0 + 1) * D + row]) : __float2half2_rn(0.0f);
+            }
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
                 uint32_t r16[16];
@@ -1056,10 +1072,9 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
 #pragma unroll
                 for (int w = 0; w < 8; ++w) {
                     const int s0 = wg * 32 + part * 16 + 2 * w;
-                    const float ut0 = with_u ? __half2float(ut[s0 * D + row]) : 0.0f;
-                    const float ut1 = with_u ? __half2float(ut[(s0 + 1) * D + row]) : 0.0f;
-                    const float u0 = (s0 < L) ? ut0 - __uint_as_float(r16[2 * w]) : 0.0f;
-                    const float u1 = (s0 + 1 < L) ? ut1 - __uint_as_float(r16[2 * w + 1]) : 0.0f;
+                    const float2 uf = __half22float2(u2[part * 8 + w]);
+                    const float u0 = (s0 < L) ? uf.x - __uint_as_float(r16[2 * w]) : 0.0f;
+                    const float u1 = (s0 + 1 < L) ? uf.y - __uint_as_float(r16[2 * w + 1]) : 0.0f;
                     ua[w] = pack_h2(u0, u1);
                 }
                 tmem_st8(tmem + lane_base + CL_TM_UA + wg * 16 + part * 8, ua);
@@ -1107,10 +1122,12 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
             for (int ch = 0; ch < 8; ++ch) {
                 float hi8[8], lo8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float xv = S[ch * 8 + e];
-                    hi8[e] = __half2float(__float2half_rn(xv));
-                    lo8[e] = xv - hi8[e];
+                for (int e = 0; e < 8; e += 2) {
+                    const float2 hf = __half22float2(__floats2half2_rn(S[ch * 8 + e], S[ch * 8 + e + 1]));
+                    hi8[e] = hf.x;
+                    hi8[e + 1] = hf.y;
+                    lo8[e] = S[ch * 8 + e] - hf.x;
+                    lo8[e + 1] = S[ch * 8 + e + 1] - hf.y;
                 }
                 st_h8(mhi + swz(row, ch), hi8);
                 st_h8(mlo + swz(row, ch), lo8);
@@ -1199,9 +1216,10 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
 #pragma unroll
             for (int w = 0; w < 16; ++w) {
                 const float x0 = S[part * 32 + 2 * w], x1 = S[part * 32 + 2 * w + 1];
-                const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-                hi[w] = pack_two_h(h0, h1);
-                lo[w] = pack_h2(x0 - __half2float(h0), x1 - __half2float(h1));
+                const __half2 h = __floats2half2_rn(x0, x1);
+                const float2 hf = __half22float2(h);
+                hi[w] = *reinterpret_cast<const uint32_t *>(&h);
+                lo[w] = pack_h2(x0 - hf.x, x1 - hf.y);
             }
             tmem_st16(tmem + lane_base + CB_TM_SHI + wg * 32 + part * 16, hi);
             tmem_st16(tmem + lane_base + CB_TM_SLO + wg * 32 + part * 16, lo);

@@ -145,11 +145,25 @@ GDN_DEV uint32_t cvt_e2m1x8(const float (&p)[8]) {
     return r;
 }
 
+// amax / 6 rounded to nearest even, as __fdiv_rn(amax, 6.0f) gives it: the product with the
+// rounded reciprocal corrected by one fused residual step (a division by a constant as in
+// Markstein's FMA division schemes). For finite amax >= 2^-125 this equals the correctly rounded
+// quotient for every input (checked exhaustively by tests/test_div6_cpu.py); below that, and
+// for inf or NaN, the plain division is used.
+GDN_DEV float div6_rn(float amax) {
+    if (amax >= 0x1p-125f && amax <= 3.4028235e38f) {
+        const float c = 1.0f / 6.0f;
+        const float q0 = amax * c;
+        return fmaf(fmaf(-q0, 6.0f, amax), c, q0);
+    }
+    return __fdiv_rn(amax, 6.0f);
+}
+
 // NVFP4 block scale from the block's largest magnitude and the global encode scale `gs`,
 // in this order of fp32 operations: s = (amax / 6) * gs; sb = E4M3(s); r = gs / sb
 // (r = 0 when sb == 0). Returns the E4M3 code; *r is the factor that maps values to codes.
 GDN_DEV uint32_t nvfp4_block_scale(float amax, float gs, float &r) {
-    float s = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+    float s = __fmul_rn(div6_rn(amax), gs);
     uint32_t sb = cvt_e4m3(s);
     r = (sb == 0u) ? 0.0f : __fdiv_rn(gs, e4m3_to_f32(sb));
     return sb;

@@ -16,6 +16,37 @@ namespace gdn {
 
 constexpr int kTailThreads = 256;
 
+// Two fp32 values in one 64-bit register pair (first value in the low half), for the packed
+// f32x2 arithmetic of sm_100: one instruction issues both lanes' multiply / add / fma.
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t f2(float a, float b) {
+    return (f2_t)__float_as_uint(a) | ((f2_t)__float_as_uint(b) << 32);
+}
+__device__ __forceinline__ float f2lo(f2_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2hi(f2_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ f2_t mul2(f2_t a, f2_t b) {
+    f2_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2_t add2(f2_t a, f2_t b) {
+    f2_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {
+    f2_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// bf16 word pair -> fp32 pair (exact: a bf16 is the high half of its fp32)
+__device__ __forceinline__ f2_t bf16x2_to_f2(uint32_t w) { return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)); }
+
 // Eight consecutive values as loaded (bf16: one 16-byte word; fp32: two), converted on use.
 template <bool BF16>
 struct Raw8 {
@@ -30,17 +61,20 @@ struct Raw8 {
         }
     }
     __device__ __forceinline__ void get(float (&x)[8]) const {
-        if constexpr (BF16) {
-            const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&a);
+        f2_t v[4];
+        get2(v);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f = __bfloat1622float2(p[i]);
-                x[2 * i] = f.x;
-                x[2 * i + 1] = f.y;
-            }
+        for (int k = 0; k < 4; ++k) {
+            x[2 * k] = f2lo(v[k]);
+            x[2 * k + 1] = f2hi(v[k]);
+        }
+    }
+    __device__ __forceinline__ void get2(f2_t (&v)[4]) const {
+        if constexpr (BF16) {
+            v[0] = bf16x2_to_f2(a.x); v[1] = bf16x2_to_f2(a.y); v[2] = bf16x2_to_f2(a.z); v[3] = bf16x2_to_f2(a.w);
         } else {
-            x[0] = __uint_as_float(a.x); x[1] = __uint_as_float(a.y); x[2] = __uint_as_float(a.z); x[3] = __uint_as_float(a.w);
-            x[4] = __uint_as_float(b.x); x[5] = __uint_as_float(b.y); x[6] = __uint_as_float(b.z); x[7] = __uint_as_float(b.w);
+            v[0] = f2(__uint_as_float(a.x), __uint_as_float(a.y)); v[1] = f2(__uint_as_float(a.z), __uint_as_float(a.w));
+            v[2] = f2(__uint_as_float(b.x), __uint_as_float(b.y)); v[3] = f2(__uint_as_float(b.z), __uint_as_float(b.w));
         }
     }
 };
@@ -58,12 +92,19 @@ gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
     constexpr int LANES = D / 8;                 // lanes per head row, 8 values each
     constexpr int RPB = kTailThreads / LANES;    // head rows per block pass
     constexpr int U = kTailUnroll;
+    // NVFP4: the per-block factor r = gs / E4M3(sb) for every scale code (sb = 0: r = 0)
+    __shared__ float r_tab[128];
+    if constexpr (NVFP4) {
+        if (threadIdx.x < 128) r_tab[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __fdiv_rn(gs, e4m3_to_f32(threadIdx.x));
+        __syncthreads();
+    }
     const int lane_in_row = threadIdx.x % LANES;
     const int col = lane_in_row * 8;
-    float wv[8];
+    f2_t w2[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) wv[j] = w[col + j];
+    for (int k = 0; k < 4; ++k) w2[k] = f2(w[col + 2 * k], w[col + 2 * k + 1]);
     const float inv_d = 1.0f / (float)D;
+    const f2_t nlog2e = f2(-kLog2e, -kLog2e), one2 = f2(1.0f, 1.0f);
     const int64_t stride = (int64_t)gridDim.x * RPB;
 
     // the loop condition is uniform over the block (the shuffles below need whole warps)
@@ -82,28 +123,62 @@ gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
             const int64_t row = row0 + u * stride;
             const bool live = row < rows;
             const size_t base = (size_t)(live ? row : 0) * D + col;
-            float ov[8], zv[8];
-            ro[u].get(ov);
-            rz[u].get(zv);
-            float ss = 0.0f;
+            f2_t o2[4], z2[4];
+            ro[u].get2(o2);
+            rz[u].get2(z2);
+            f2_t sq = mul2(o2[0], o2[0]);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) ss += ov[j] * ov[j];
-            ss = group_sum<LANES>(ss);
+            for (int k = 1; k < 4; ++k) sq = fma2(o2[k], o2[k], sq);
+            const float ss = group_sum<LANES>(f2lo(sq) + f2hi(sq));
             const float inv_rms = rsqrtf(ss * inv_d + eps);
-            float yv[8];
+            const f2_t ir2 = f2(inv_rms, inv_rms);
+            // y = o (w / rms) z sigma(z), sigma(z) = 1 / (1 + 2^(-z log2 e))
+            f2_t y2[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) yv[j] = ov[j] * inv_rms * wv[j] * silu_fast(zv[j]);
+            for (int k = 0; k < 4; ++k) {
+                const f2_t t = mul2(z2[k], nlog2e);
+                const f2_t d = add2(f2(exp2_approx(f2lo(t)), exp2_approx(f2hi(t))), one2);
+                const f2_t sl = mul2(z2[k], f2(rcp_approx(f2lo(d)), rcp_approx(f2hi(d))));
+                y2[k] = mul2(mul2(o2[k], mul2(w2[k], ir2)), sl);
+            }
             if constexpr (!NVFP4) {
-                if (live) store8<OUT_BF16>(y, base, yv);
+                if (live) {
+                    if constexpr (OUT_BF16) {
+                        uint4 u4;
+                        uint32_t *pw = reinterpret_cast<uint32_t *>(&u4);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const __nv_bfloat162 hb = __floats2bfloat162_rn(f2lo(y2[k]), f2hi(y2[k]));
+                            pw[k] = *reinterpret_cast<const uint32_t *>(&hb);
+                        }
+                        *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(y) + base) = u4;
+                    } else {
+                        float4 *p = reinterpret_cast<float4 *>(reinterpret_cast<float *>(y) + base);
+                        p[0] = make_float4(f2lo(y2[0]), f2hi(y2[0]), f2lo(y2[1]), f2hi(y2[1]));
+                        p[1] = make_float4(f2lo(y2[2]), f2hi(y2[2]), f2lo(y2[3]), f2hi(y2[3]));
+                    }
+                }
             } else {
                 // y as the bf16 tensor the two-call path would hand to the encoder
+                float amax = 0.0f;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) yv[j] = round_bf16(yv[j]);
-                float amax = amax8(yv);
+                for (int k = 0; k < 4; ++k) {
+                    const __nv_bfloat162 hb = __floats2bfloat162_rn(f2lo(y2[k]), f2hi(y2[k]));
+                    y2[k] = bf16x2_to_f2(*reinterpret_cast<const uint32_t *>(&hb));
+                    amax = fmaxf(amax, fmaxf(fabsf(f2lo(y2[k])), fabsf(f2hi(y2[k]))));
+                }
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // partner lane: same block
-                float r;
-                const uint32_t sb = nvfp4_block_scale(amax, gs, r);
-                const uint32_t packed = nvfp4_pack8(yv, r);
+                const uint32_t sb = cvt_e4m3(__fmul_rn(div6_rn(amax), gs));
+                const float r = r_tab[sb & 127u];
+                const f2_t r2 = f2(r, r);
+                float p[8];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const f2_t q = mul2(y2[k], r2);
+                    p[2 * k] = f2lo(q);
+                    p[2 * k + 1] = f2hi(q);
+                }
+                const uint32_t packed = cvt_e2m1x8(p);
                 if (live) {
                     reinterpret_cast<uint32_t *>(xq)[base / 8] = packed;
                     if ((lane_in_row & 1) == 0) xs[base / 16] = (uint8_t)sb;
