@@ -220,6 +220,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                       const float *__restrict__ A_log, const float *__restrict__ dt_bias,
                       const int32_t *__restrict__ cu_seqlens, int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv,
                       int32_t slots, float scale, int32_t l2norm, uint8_t *__restrict__ ws, int *status) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int id = blockIdx.x, h = blockIdx.y;
     int n, t_begin, t_end;
     locate(id, cu_seqlens, num_seqs, T, n, t_begin, t_end);
@@ -634,6 +636,8 @@ constexpr int kStgPitch = 528;
 
 __global__ void __launch_bounds__(CH_THREADS, 1)
 gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
+    pdl_launch_dependents();
+    pdl_wait();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CH_OFF_BAR);
@@ -931,6 +935,8 @@ constexpr uint32_t CL_TM_D4 = 0, CL_TM_D7 = 0, CL_TM_SA = 128, CL_TM_UA = 192;
 
 __global__ void __launch_bounds__(NT, 2)
 gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
+    pdl_launch_dependents();
+    pdl_wait();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CL_OFF_BAR);
@@ -1159,6 +1165,8 @@ constexpr uint32_t CB_TM_SHI = 0, CB_TM_SLO = 64, CB_TM_D = 128;
 
 __global__ void __launch_bounds__(NT, 1)
 gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int h = blockIdx.x, n = blockIdx.y;
     const int SEG = P.seg_chunks;
     int t_begin = 0, t_end = P.T;
@@ -1326,23 +1334,21 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
     const int seg = chunked_segment_chunks(c.T, c.num_seqs, c.Hv);
     const int seg_slots = c.T / (kChunk * seg) + c.num_seqs;
     uint8_t *ws = static_cast<uint8_t *>(c.ws);
-    gdn_chunk_prep_kernel<<<dim3(slots, c.Hv), NT, P_SMEM, st>>>(maps, c.a, c.b, c.A_log, c.dt_bias, c.cu_seqlens, c.T,
-                                                                 c.num_seqs, c.Hk, c.Hv, slots, c.scale, c.l2norm, ws,
-                                                                 c.status);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(gdn_chunk_prep_kernel, dim3(slots, c.Hv), dim3(NT), P_SMEM, st, maps, c.a, c.b, c.A_log,
+                               c.dt_bias, c.cu_seqlens, c.T, c.num_seqs, c.Hk, c.Hv, slots, c.scale, c.l2norm, ws,
+                               c.status);
     if (e != cudaSuccess) return e;
     ChainParams P{c.cu_seqlens, c.T, c.num_seqs, c.Hv, slots, seg, seg_slots, kChainFull, c.out_bf16 ? 1 : 0, c.S0,
                   c.S_out, c.o, ws, ws + (size_t)c.Hv * slots * kWsItem, c.status};
     if (c.T > kChunk * seg) {   // some sequence may span several segments
         P.mode_base = kChainState;   // z = 0: segment states (B), z = 1: segment transitions (M)
-        gdn_chunk_lean_kernel<<<dim3(c.Hv, seg_slots, 2), NT, CL_SMEM, st>>>(P);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        gdn_segment_combine_kernel<<<dim3(c.Hv, c.num_seqs), NT, CB_SMEM, st>>>(P);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_pdl(gdn_chunk_lean_kernel, dim3(c.Hv, seg_slots, 2), dim3(NT), CL_SMEM, st, P)) != cudaSuccess)
+            return e;
+        if ((e = launch_pdl(gdn_segment_combine_kernel, dim3(c.Hv, c.num_seqs), dim3(NT), CB_SMEM, st, P)) != cudaSuccess)
+            return e;
         P.mode_base = kChainFull;
     }
-    gdn_chunk_chain_kernel<<<dim3(c.Hv, seg_slots, 1), CH_THREADS, CH_SMEM, st>>>(P);
-    return cudaGetLastError();
+    return launch_pdl(gdn_chunk_chain_kernel, dim3(c.Hv, seg_slots, 1), dim3(CH_THREADS), CH_SMEM, st, P);
 }
 
 }  // namespace gdn

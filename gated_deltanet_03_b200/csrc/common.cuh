@@ -315,6 +315,14 @@ GDN_DEV void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr));
 }
+// Programmatic dependent launch. Every kernel of this library is launched with programmatic
+// stream serialization (launch_pdl): it may start while the previous kernel in the stream is
+// still running, so it calls pdl_wait() before its first global-memory access (which returns
+// once that kernel has finished and its writes are visible), and pdl_launch_dependents() at
+// entry so that the next kernel's CTAs can be placed on SMs this grid no longer needs.
+GDN_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+GDN_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 GDN_DEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Registers into 32 lanes x N consecutive 32-bit columns of tensor memory (this warp's

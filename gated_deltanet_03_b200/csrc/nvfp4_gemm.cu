@@ -87,6 +87,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                   const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                   const __grid_constant__ CUtensorMap map_y, int sf_tma, const uint8_t *__restrict__ sfa_g, const uint8_t *__restrict__ sfb_g, float alpha,
                   int M, int N, int K, int out_bf16, void *__restrict__ y, int *status) {
+    pdl_launch_dependents();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Smem sm{base};
@@ -118,6 +119,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();   // barriers and tensor memory are set up; now the predecessor's data
 
     if (warp == 0) {
         if (lane == 0) {
@@ -337,9 +339,8 @@ cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
         attr_set = true;
     }
     dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM);
-    nvfp4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, msa, msb, my, sf_tma ? 1 : 0, g.as, g.bs, g.alpha, g.M,
-                                                         g.N, g.K, g.out_bf16 ? 1 : 0, g.y, g.status);
-    return cudaGetLastError();
+    return launch_pdl(nvfp4_gemm_kernel, grid, dim3(THREADS), SMEM_BYTES, st, ma, mb, msa, msb, my, sf_tma ? 1 : 0,
+                      g.as, g.bs, g.alpha, g.M, g.N, g.K, g.out_bf16 ? 1 : 0, g.y, g.status);
 }
 
 }  // namespace gdn

@@ -39,6 +39,8 @@ gdn_recurrent_kernel(const void *__restrict__ q, const void *__restrict__ k,
                      const float *__restrict__ dt_bias, const int32_t *__restrict__ cu_seqlens,
                      int32_t tokens_per_seq, int32_t Hk, int32_t Hv, float scale, int32_t l2norm,
                      const float *S0, float *S_out, void *__restrict__ o) {
+    pdl_launch_dependents();
+    pdl_wait();
     using Sh = RecurrentShape<D>;
     constexpr int LANES = Sh::LANES, RPB = Sh::RPB, PASSES = Sh::PASSES, R = Sh::R;
     const int slice = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
@@ -125,10 +127,9 @@ template <int D, bool IN_BF16, bool OUT_BF16>
 static cudaError_t launch_recurrent_t(const RecurrentArgs &r, cudaStream_t st) {
     using Sh = RecurrentShape<D>;
     dim3 grid(Sh::SLICES, r.Hv, r.num_seqs);
-    gdn_recurrent_kernel<D, IN_BF16, OUT_BF16><<<grid, Sh::NT, 0, st>>>(
-        r.q, r.k, r.v, r.a, r.b, r.A_log, r.dt_bias, r.cu_seqlens, r.tokens_per_seq, r.Hk, r.Hv,
-        r.scale, r.l2norm, r.S0, r.S_out, r.o);
-    return cudaGetLastError();
+    return launch_pdl(gdn_recurrent_kernel<D, IN_BF16, OUT_BF16>, grid, dim3(Sh::NT), 0, st, r.q, r.k, r.v, r.a, r.b,
+                      r.A_log, r.dt_bias, r.cu_seqlens, r.tokens_per_seq, r.Hk, r.Hv, r.scale, r.l2norm, r.S0,
+                      r.S_out, r.o);
 }
 
 template <int D>

@@ -89,6 +89,8 @@ gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
                      const float *__restrict__ w, float eps, int64_t rows,
                      void *__restrict__ y, float gs, uint8_t *__restrict__ xq,
                      uint8_t *__restrict__ xs) {
+    pdl_launch_dependents();
+    pdl_wait();
     constexpr int LANES = D / 8;                 // lanes per head row, 8 values each
     constexpr int RPB = kTailThreads / LANES;    // head rows per block pass
     constexpr int U = kTailUnroll;
@@ -196,9 +198,8 @@ static cudaError_t launch_tail_t(const TailArgs &t, cudaStream_t st) {
     int64_t blocks = (rows + RPB * kTailUnroll - 1) / (RPB * kTailUnroll);
     const int64_t cap = 148 * 8;
     if (blocks > cap) blocks = cap;
-    gated_rmsnorm_kernel<D, IN_BF16, OUT_BF16, NVFP4><<<(unsigned)blocks, kTailThreads, 0, st>>>(
-        t.o, t.z, t.w, t.eps, rows, t.y, t.gs, t.xq, t.xs);
-    return cudaGetLastError();
+    return launch_pdl(gated_rmsnorm_kernel<D, IN_BF16, OUT_BF16, NVFP4>, dim3((unsigned)blocks), dim3(kTailThreads), 0,
+                      st, t.o, t.z, t.w, t.eps, rows, t.y, t.gs, t.xq, t.xs);
 }
 
 template <bool NVFP4, int D>
@@ -229,6 +230,8 @@ template <bool IN_BF16>
 __global__ void __launch_bounds__(256)
 nvfp4_quantize_kernel(const void *__restrict__ x, int64_t nblocks, float gs,
                       uint8_t *__restrict__ xq, uint8_t *__restrict__ xs) {
+    pdl_launch_dependents();
+    pdl_wait();
     constexpr int U = 4;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b0 < nblocks; b0 += U * stride) {
@@ -261,9 +264,8 @@ cudaError_t launch_nvfp4_quantize(const void *x, bool in_bf16, int32_t M, int32_
     if (nblocks == 0) return cudaSuccess;
     int64_t grid = (nblocks + 1023) / 1024;
     if (grid > 148 * 8) grid = 148 * 8;
-    if (in_bf16) nvfp4_quantize_kernel<true><<<(unsigned)grid, 256, 0, st>>>(x, nblocks, gs, xq, xs);
-    else nvfp4_quantize_kernel<false><<<(unsigned)grid, 256, 0, st>>>(x, nblocks, gs, xq, xs);
-    return cudaGetLastError();
+    if (in_bf16) return launch_pdl(nvfp4_quantize_kernel<true>, dim3((unsigned)grid), dim3(256), 0, st, x, nblocks, gs, xq, xs);
+    return launch_pdl(nvfp4_quantize_kernel<false>, dim3((unsigned)grid), dim3(256), 0, st, x, nblocks, gs, xq, xs);
 }
 
 }  // namespace gdn
