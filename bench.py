@@ -87,7 +87,7 @@ def scan_bytes(w: workloads.Workload, o_bytes=2) -> float:
 
 
 class ClockSampler:
-    """SM clock and clock-event (throttle) reasons sampled every millisecond through NVML
+    """SM clock and clock-event (throttle) reasons sampled every 0.2 ms through NVML
     while the timed region runs (falls back to an nvidia-smi loop when NVML is missing)."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
@@ -126,13 +126,17 @@ class ClockSampler:
                 self.samples.append((float(mhz), int(reasons)))
             except Exception:  # noqa: BLE001 - a failed sample is skipped
                 pass
-            time.sleep(0.001)
+            time.sleep(0.0002)
 
     def __enter__(self):
         try:
             self._open()
             self._thread = threading.Thread(target=self._loop, daemon=True)
             self._thread.start()
+            t0 = time.time()   # the timed region starts only once sampling runs
+            while not self.samples and time.time() - t0 < 2.0:
+                time.sleep(0.0005)
+            self.samples.clear()
         except Exception:  # noqa: BLE001 - no NVML: report no samples
             self._thread = None
         return self
@@ -150,7 +154,7 @@ class ClockSampler:
                 if r & bit:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(reasons), "samples": len(sm), "source": "nvml, 1 ms"}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvml, 0.2 ms"}
 
 
 # ----------------------------------------------------------------- GPU arm ----
@@ -487,7 +491,7 @@ def run_reference(args):
 def main():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")

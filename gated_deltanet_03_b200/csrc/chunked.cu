@@ -347,9 +347,15 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             // row r of A: A_rs = beta_r exp(G_r - G_s) k_r.k_s / (|k_r| |k_s|) for s < r < L
             const int r = x;
             const float Gr = sG[r], cr = sBeta[r] * sRk[r];
+            const f2_t cr2 = f2(cr, cr);
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                vals[j] = (wg * 32 + j < r) ? cr * exp_approx(Gr - gs[j]) * __uint_as_float(r32[j]) * rks[j] : 0.0f;
+            for (int j = 0; j < 32; j += 2) {
+                const f2_t v2 = mul2(mul2(f2(exp_approx(Gr - gs[j]), exp_approx(Gr - gs[j + 1])),
+                                          f2(__uint_as_float(r32[j]), __uint_as_float(r32[j + 1]))),
+                                     mul2(f2(rks[j], rks[j + 1]), cr2));
+                vals[j] = (wg * 32 + j < r) ? f2lo(v2) : 0.0f;
+                vals[j + 1] = (wg * 32 + j + 1 < r) ? f2hi(v2) : 0.0f;
+            }
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8)
                 st_h8(reinterpret_cast<uint8_t *>(Ah + r * P_AH + wg * 32 + q8 * 8), &vals[q8 * 8]);
@@ -357,9 +363,15 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             // row r of P = (Q K^T o Gamma) scaled, into the P^T image [s][r] (MN-major over r)
             const int r = x - 64;
             const float Gr = sG[r], cr = sRq[r];
+            const f2_t cr2 = f2(cr, cr);
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                vals[j] = (wg * 32 + j <= r) ? cr * exp_approx(Gr - gs[j]) * __uint_as_float(r32[j]) * rks[j] : 0.0f;
+            for (int j = 0; j < 32; j += 2) {
+                const f2_t v2 = mul2(mul2(f2(exp_approx(Gr - gs[j]), exp_approx(Gr - gs[j + 1])),
+                                          f2(__uint_as_float(r32[j]), __uint_as_float(r32[j + 1]))),
+                                     mul2(f2(rks[j], rks[j + 1]), cr2));
+                vals[j] = (wg * 32 + j <= r) ? f2lo(v2) : 0.0f;
+                vals[j + 1] = (wg * 32 + j + 1 <= r) ? f2hi(v2) : 0.0f;
+            }
 #pragma unroll
             for (int j = 0; j < 32; ++j)
                 *reinterpret_cast<__half *>(sm + P_OFF_PST + swz(wg * 32 + j, r >> 3) + (r & 7) * 2) =

@@ -315,6 +315,34 @@ GDN_DEV void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr));
 }
+// Two fp32 values in one 64-bit register pair (first value in the low half), for the packed
+// f32x2 arithmetic of sm_100: one instruction issues both lanes' multiply / add / fma.
+typedef unsigned long long f2_t;
+GDN_DEV f2_t f2(float a, float b) {
+    return (f2_t)__float_as_uint(a) | ((f2_t)__float_as_uint(b) << 32);
+}
+GDN_DEV float f2lo(f2_t v) { return __uint_as_float((uint32_t)v); }
+GDN_DEV float f2hi(f2_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+GDN_DEV f2_t mul2(f2_t a, f2_t b) {
+    f2_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+GDN_DEV f2_t add2(f2_t a, f2_t b) {
+    f2_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+GDN_DEV f2_t fma2(f2_t a, f2_t b, f2_t c) {
+    f2_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+GDN_DEV float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 // Programmatic dependent launch. Every kernel of this library is launched with programmatic
 // stream serialization (launch_pdl): it may start while the previous kernel in the stream is
 // still running, so it calls pdl_wait() before its first global-memory access (which returns

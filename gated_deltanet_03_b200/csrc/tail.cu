@@ -16,34 +16,6 @@ namespace gdn {
 
 constexpr int kTailThreads = 256;
 
-// Two fp32 values in one 64-bit register pair (first value in the low half), for the packed
-// f32x2 arithmetic of sm_100: one instruction issues both lanes' multiply / add / fma.
-typedef unsigned long long f2_t;
-__device__ __forceinline__ f2_t f2(float a, float b) {
-    return (f2_t)__float_as_uint(a) | ((f2_t)__float_as_uint(b) << 32);
-}
-__device__ __forceinline__ float f2lo(f2_t v) { return __uint_as_float((uint32_t)v); }
-__device__ __forceinline__ float f2hi(f2_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
-__device__ __forceinline__ f2_t mul2(f2_t a, f2_t b) {
-    f2_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ f2_t add2(f2_t a, f2_t b) {
-    f2_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {
-    f2_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ float rcp_approx(float x) {
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 // bf16 word pair -> fp32 pair (exact: a bf16 is the high half of its fp32)
 __device__ __forceinline__ f2_t bf16x2_to_f2(uint32_t w) { return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)); }
 
