@@ -1222,10 +1222,10 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
     };
     if (tid == 0 && nseg > 2) issue_m(1);
 
-    float S[64];
+    float S[64];   // S_start(p), starting from S_start(1) = B_0
     ilv_load(seg(0) + kSegB, row, wg, S);
-    ilv_store(seg(1) + kSegS, row, wg, S);
     const uint32_t idm = idesc_f16(128, false, true, false);
+    const f2_t neg1 = f2(-1.0f, -1.0f);
     for (int p = 1; p + 1 < nseg; ++p) {
         const int b = (p - 1) & 1;
         uint8_t *buf = sm + CB_OFF_BUF + b * 65536;
@@ -1235,11 +1235,12 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
             uint32_t hi[16], lo[16];
 #pragma unroll
             for (int w = 0; w < 16; ++w) {
-                const float x0 = S[part * 32 + 2 * w], x1 = S[part * 32 + 2 * w + 1];
-                const __half2 h = __floats2half2_rn(x0, x1);
+                const f2_t x2 = f2(S[part * 32 + 2 * w], S[part * 32 + 2 * w + 1]);
+                const __half2 h = __floats2half2_rn(f2lo(x2), f2hi(x2));
                 const float2 hf = __half22float2(h);
+                const f2_t r2 = fma2(f2(hf.x, hf.y), neg1, x2);
                 hi[w] = *reinterpret_cast<const uint32_t *>(&h);
-                lo[w] = pack_h2(x0 - hf.x, x1 - hf.y);
+                lo[w] = pack_h2(f2lo(r2), f2hi(r2));
             }
             tmem_st16(tmem + lane_base + CB_TM_SHI + wg * 32 + part * 16, hi);
             tmem_st16(tmem + lane_base + CB_TM_SLO + wg * 32 + part * 16, lo);
@@ -1269,22 +1270,27 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
                 tc_commit(bar_mma);
             }
         }
+        // while the MMAs run: publish S_start(p) for the output pass, fetch B_p
+        ilv_store(seg(p) + kSegS, row, wg, S);
         float Bp[64];
         ilv_load(seg(p) + kSegB, row, wg, Bp);
         if (tid == 0 && ok) ok = mbar_wait(bar_mma, (uint32_t)((p - 1) & 1), P.status) ? 1 : 0;
         if (!__syncthreads_and(ok)) break;
         tc_fence_after();
+        uint32_t r32[2][32];
+        tmem_ld32(tmem + CB_TM_D + lane_base + wg * 64, r32[0]);
+        tmem_ld32(tmem + CB_TM_D + lane_base + wg * 64 + 32, r32[1]);
+        tmem_ld_wait();
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t r32[32];
-            tmem_ld32(tmem + CB_TM_D + lane_base + wg * 64 + half * 32, r32);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) S[half * 32 + j] = __uint_as_float(r32[j]) + Bp[half * 32 + j];
+        for (int j = 0; j < 64; j += 2) {
+            const f2_t s2 = add2(f2(__uint_as_float(r32[j >> 5][j & 31]), __uint_as_float(r32[j >> 5][(j & 31) + 1])),
+                                 f2(Bp[j], Bp[j + 1]));
+            S[j] = f2lo(s2);
+            S[j + 1] = f2hi(s2);
         }
-        ilv_store(seg(p + 1) + kSegS, row, wg, S);
         tc_fence_before();
     }
+    ilv_store(seg(nseg - 1) + kSegS, row, wg, S);   // the last segment's start state
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
