@@ -952,8 +952,10 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CL_OFF_BAR);
-    uint64_t *full = bars, *bar_mma = bars + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3);
+    // full[2]: chunk copies; bar45 / bar67: MMA completion; bar_s / bar_u: the eight warps
+    // have stored S0 / U into tensor memory (one arrival per warp)
+    uint64_t *full = bars, *bar45 = bars + 2, *bar67 = bars + 3, *bar_s = bars + 4, *bar_u = bars + 5;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int h = blockIdx.x, id = blockIdx.y, mode = kChainState + (int)blockIdx.z;
@@ -987,7 +989,10 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
-        mbar_init(bar_mma, 1);
+        mbar_init(bar45, 1);
+        mbar_init(bar67, 1);
+        mbar_init(bar_s, 8);
+        mbar_init(bar_u, 8);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -1029,7 +1034,8 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) S[c] = (mode == kChainTransition && row == 64 * wg + c) ? 1.0f : 0.0f;
     }
-    // fp16 copy of S as the A operand of MMA45: row i on lane i, key index j two per column
+    // fp16 copy of S as the A operand of MMA45: row i on lane i, key index j two per column;
+    // each warp signals bar_s once its part is in tensor memory
     auto store_S = [&]() {
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -1039,41 +1045,46 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
             tmem_st16(tmem + lane_base + CL_TM_SA + wg * 32 + part * 16, pk);
         }
         tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_s);
+    };
+    // Every thread waits on the MMA barriers itself. A wait that runs out marks the thread
+    // dead: it records the status, stops waiting and issuing, and still takes every later step,
+    // so that no barrier is left short of arrivals.
+    bool dead = false;
+    auto wait = [&](uint64_t *bar, uint32_t parity) {
+        if (!dead && !mbar_wait(bar, parity, status)) dead = true;
     };
     store_S();
 
     const uint32_t id45 = idesc_f16(64, false, false, false);
     const uint32_t id67 = idesc_f16(128, false, true, false);
-    uint32_t mph = 0;
-    bool alive = true;
     for (int c = 0; c < nchunks; ++c) {
         const int L = min(C, t_end - (t_begin + (c_first + c) * C));
         const int b = c & 1;
+        const uint32_t ph = (uint32_t)(c & 1);
         const uint8_t *buf = sm + b * CL_BUF;
-        tc_fence_before();
-        __syncthreads();   // S0 of this chunk is in tensor memory
-        int ok = 1;
         if (tid == 0) {
-            ok = mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status) ? 1 : 0;
-            if (ok) {
+            wait(bar_s, ph);                                // S0 of this chunk is in tensor memory
+            wait(&full[b], (uint32_t)((c >> 1) & 1));
+            if (!dead) {
                 tc_fence_after();
                 // D4 = S0 W^T   (B: W, K-major rows s, K = 128 key columns in two halves)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_f16_ts(tmem + CL_TM_D4, tmem + CL_TM_SA + kk * 8,
                                kdesc(buf + CL_W + (kk < 4 ? 0 : TILE) + (kk & 3) * 32), id45, kk > 0);
-                tc_commit(bar_mma);
-                ok = mbar_wait(bar_mma, mph, status) ? 1 : 0;
+                tc_commit(bar45);
             }
-            mph ^= 1u;
         }
-        if (!__syncthreads_and(ok)) { alive = false; break; }
+        wait(&full[b], (uint32_t)((c >> 1) & 1));           // this chunk's U~ and gamma_C are visible
+        wait(bar45, ph);
         tc_fence_after();
         const float gC = reinterpret_cast<const float *>(buf + CL_VEC)[0];
         {
-            // U^T = U~^T - D4 (the transition pass takes U~ = 0) as the fp16 A operand of MMA67
-            // this thread's 32 values of U~ (tokens 32 wg .. 32 wg + 31 of value row i), loaded
-            // before any tensor-memory access so that the loads overlap
+            // U^T = U~^T - D4 (the transition pass takes U~ = 0) as the fp16 A operand of MMA67;
+            // this thread's 32 values of U~ are loaded before any tensor-memory access
             const __half *ut = reinterpret_cast<const __half *>(buf + CL_U);
             __half2 u2[16];
 #pragma unroll
@@ -1098,25 +1109,28 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
                 tmem_st8(tmem + lane_base + CL_TM_UA + wg * 16 + part * 8, ua);
             }
             tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_u);
         }
-        tc_fence_before();
-        __syncthreads();   // U is in tensor memory; D4 and this buffer's U~ are consumed
         if (tid == 0) {
-            tc_fence_after();
-            // D7 = U^T K''   (B: K'', MN-major blocks of 64 keys, K = 64 tokens)
+            wait(bar_u, ph);                                // U is in tensor memory, D4 is consumed
+            if (!dead) {
+                tc_fence_after();
+                // D7 = U^T K''   (B: K'', MN-major blocks of 64 keys, K = 64 tokens)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16_ts(tmem + CL_TM_D7, tmem + CL_TM_UA + kk * 8, mndesc(buf + CL_K + kk * 2048, TILE), id67,
-                           kk > 0);
-            tc_commit(bar_mma);
-            ok = mbar_wait(bar_mma, mph, status) ? 1 : 0;
-            mph ^= 1u;
-            if (ok && c + 2 < nchunks) {   // this buffer's last reader is done: refill it
-                fence_proxy_async_smem();
-                issue_chunk(c + 2);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16_ts(tmem + CL_TM_D7, tmem + CL_TM_UA + kk * 8, mndesc(buf + CL_K + kk * 2048, TILE),
+                               id67, kk > 0);
+                tc_commit(bar67);
             }
         }
-        if (!__syncthreads_and(ok)) { alive = false; break; }
+        wait(bar67, ph);
+        // this buffer's readers (both MMAs, every thread's U~ and gamma_C) are done: refill it
+        if (tid == 0 && !dead && c + 2 < nchunks) {
+            fence_proxy_async_smem();
+            issue_chunk(c + 2);
+        }
         tc_fence_after();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -1128,6 +1142,7 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
         }
         store_S();
     }
+    const bool alive = __syncthreads_and(!dead);
     if (alive) {
         if (mode == kChainState) {
             ilv_store(const_cast<uint8_t *>(seg_item) + kSegB, row, wg, S);
