@@ -159,6 +159,27 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- GPU arm ----
 
+def count_kernels(torch, fn):
+    """This library's kernels launched by one call of fn (CUPTI kernel records through the
+    profiler), and their names; falls back to the step's known launch sequence."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            fn()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events()
+                 if any(t in e.name for t in ("gdn_", "nvfp4_", "gated_rmsnorm"))]
+        if names:
+            def short(n):
+                n = n.replace("(anonymous namespace)::", "").replace("void ", "")
+                return n.split("(")[0].split("::")[-1]
+            return len(names), sorted({short(n) for n in names})
+    except Exception:  # noqa: BLE001 - no profiler: the static count below
+        pass
+    return 5, ["gdn_chunk_prep_kernel", "gdn_chunk_lean_kernel", "gdn_segment_combine_kernel",
+               "gdn_chunk_chain_kernel<true>", "nvfp4_gemm_kernel"]
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -213,9 +234,13 @@ def run_gpu(args):
     def gemm():
         g.nvfp4_gemm(xq, xs, wq, ws_w, alpha, y=Y)
 
+    def fused():
+        # the scan whose output pass also applies the gated RMSNorm and writes NVFP4 activations
+        g.gdn_prefill_chunked_gated_nvfp4(q, k, v, a, b, A_log, dt_bias, z, nw, gx, final_state=S, xq=xq, xs=xs,
+                                          workspace=ws)
+
     def step():
-        scan()
-        tail()
+        fused()
         gemm()
 
     for _ in range(args.warmup):
@@ -229,7 +254,7 @@ def run_gpu(args):
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
-        for name, fn in (("step", step), ("scan", scan), ("tail", tail), ("gemm", gemm)):
+        for name, fn in (("step", step), ("scan", scan), ("tail", tail), ("fused", fused), ("gemm", gemm)):
             fn()
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=side):
@@ -260,11 +285,12 @@ def run_gpu(args):
     torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     parts = {}
-    for name in ("scan", "tail", "gemm"):
+    for name in ("scan", "tail", "fused", "gemm"):
         evs = timed(graphs[name], args.steps)
         torch.cuda.synchronize()
         parts[name] = [a.elapsed_time(b) for a, b in evs]
-    scan_ms, tail_ms, gemm_ms = parts["scan"], parts["tail"], parts["gemm"]
+    scan_ms, tail_ms, fused_ms, gemm_ms = parts["scan"], parts["tail"], parts["fused"], parts["gemm"]
+    launches_per_step, kernel_names = count_kernels(torch, graphs["step"].replay)
     ms = statistics.mean(step_ms)
     ms_max = ms
     if world > 1:
@@ -356,8 +382,10 @@ def run_gpu(args):
         "config": {"workload": w.name, "T": T, "Hk": w.Hk, "Hv": Hv, "d": D, "chunk": CHUNK,
                    "out_proj": "NVFP4 W4A4 %d->%d" % (K, N), "global_batch": 1, "seq_len": T,
                    "parallelism": "replicas x%d" % world, "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)"},
-        "breakdown_ms": {"scan": statistics.mean(scan_ms), "gated_norm_nvfp4": statistics.mean(tail_ms),
-                         "nvfp4_gemm": statistics.mean(gemm_ms), "timing": "CUDA graph replay per op"},
+        "breakdown_ms": {"prefill_fused": statistics.mean(fused_ms), "nvfp4_gemm": statistics.mean(gemm_ms),
+                         "scan_alone": statistics.mean(scan_ms), "gated_norm_nvfp4_alone": statistics.mean(tail_ms),
+                         "step": "prefill_fused (scan + gated RMSNorm + NVFP4 encode in the output pass) + nvfp4_gemm",
+                         "timing": "CUDA graph replay per op"},
         "roofline": {"kernel": "gdn prefill scan (prep + chain kernels of one call)", "bound": "tensor", "achieved": achieved_tflops,
                      "peak": peak_tflops, "unit": "TFLOP/s", "frac": achieved_tflops / peak_tflops,
                      "peak_kind": pk_kind + " (bf16 dense burst; the scan's MMAs are fp16)",
@@ -371,7 +399,8 @@ def run_gpu(args):
         "decode": {"workload": dw.name, "ms": dec, "GB/s": dec_bytes / (dec / 1e3) / 1e9,
                    "frac": dec_bytes / (dec / 1e3) / 1e9 / float(pk["hbm_gbs"]),
                    "bytes": dec_bytes, "peak_gbs": float(pk["hbm_gbs"]), "peak_kind": pk_kind},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
+        "gpu_kernels_per_step": kernel_names,
         "clocks": clk.summary(),
     }
     if not args.no_cpu:
@@ -415,6 +444,8 @@ def run_only(args):
         "tail": lambda: g.gdn_gated_rmsnorm_silu_nvfp4(o, z, nw, 1.0, xq=xq, xs=xs),
         "gemm": lambda: g.nvfp4_gemm(xq, xs, wq, ws, 1.0, y=Y),
         "decode": lambda: g.gdn_decode_step(q, k, v, a, b, A_log, dt_bias, S0, o=o),
+        "fused": lambda: g.gdn_prefill_chunked_gated_nvfp4(q, k, v, a, b, A_log, dt_bias, z, nw, 1.0, cu_seqlens=cu,
+                                                           initial_state=S0, final_state=S, xq=xq, xs=xs),
     }[args.only]
     flush = make_l2_flush(torch, dev)
     for _ in range(args.warmup):
@@ -495,7 +526,7 @@ def main():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
-    p.add_argument("--only", choices=["scan", "tail", "gemm", "decode"],
+    p.add_argument("--only", choices=["scan", "tail", "gemm", "decode", "fused"],
                    help="time one kernel alone on its workload (for profiling); prints one JSON line")
     p.add_argument("--workload", default=None, help="workload name for --only scan (default: 1024-wide prefill)")
     args = p.parse_args()

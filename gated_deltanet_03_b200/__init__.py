@@ -5,7 +5,7 @@ PyTorch provides device memory (output tensors are allocated with torch) and the
 stream. There is no CPU fallback: if the library is missing, importing this package raises.
 
 Functions keep the C names:
-  gdn_prefill_chunked, gdn_decode_step, gdn_gated_rmsnorm_silu,
+  gdn_prefill_chunked, gdn_prefill_chunked_gated_nvfp4, gdn_decode_step, gdn_gated_rmsnorm_silu,
   gdn_gated_rmsnorm_silu_nvfp4, nvfp4_quantize_act, nvfp4_gemm,
   gdn_prefill_workspace_bytes, gdn_get_device_status.
 """
@@ -24,7 +24,7 @@ GDN_BF16, GDN_F32 = 0, 1
 
 # Exported C symbols, in the order include/gdn.h declares them.
 ABI_SYMBOLS = (
-    "gdn_prefill_chunked", "gdn_prefill_workspace_bytes", "gdn_decode_step",
+    "gdn_prefill_chunked", "gdn_prefill_workspace_bytes", "gdn_prefill_chunked_gated_nvfp4", "gdn_decode_step",
     "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act",
     "nvfp4_gemm", "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_status_string",
     "gdn_version",
@@ -45,6 +45,8 @@ def _load() -> ctypes.CDLL:
     P, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
     lib.gdn_prefill_chunked.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32,
                                         i32, P, P, P, i32, P, sz, P]
+    lib.gdn_prefill_chunked_gated_nvfp4.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32,
+                                                    i32, i32, P, P, P, P, P, f32, f32, P, P, P, sz, P]
     lib.gdn_prefill_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
     lib.gdn_prefill_workspace_bytes.restype = sz
     lib.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, P, P,
@@ -59,7 +61,7 @@ def _load() -> ctypes.CDLL:
     lib.gdn_status_string.argtypes = [i32]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_version.restype = i32
-    for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_static_ws", "gdn_decode_step", "gdn_gated_rmsnorm_silu",
+    for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_gated_nvfp4", "gdn_prefill_chunked_static_ws", "gdn_decode_step", "gdn_gated_rmsnorm_silu",
                  "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_gemm",
                  "gdn_get_device_status"):
         getattr(lib, name).restype = ctypes.c_int
@@ -134,6 +136,38 @@ def gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, initial_
                                  0 if workspace is None else workspace.numel(), _stream(stream))
     _check("gdn_prefill_chunked", st)
     return o, final_state
+
+
+def gdn_prefill_chunked_gated_nvfp4(q, k, v, a, b, A_log, dt_bias, z, norm_weight, global_scale: float,
+                                    cu_seqlens=None, initial_state=None, final_state=None, scale: float = 1.0,
+                                    qk_l2norm: bool = True, eps: float = 1e-6, o=None, write_o: bool = False,
+                                    xq=None, xs=None, workspace=None, stream=None):
+    """Prefill whose output pass also applies the gated RMSNorm and writes NVFP4 activations.
+    q, k [T, Hk, 128] bf16; v, z [T, Hv, 128] bf16; norm_weight [128] fp32.
+    Returns (xq [T, Hv*64] u8, xs [T, Hv*8] u8, final_state, o or None); o (bf16) is written only
+    when given or when write_o is set."""
+    T, Hk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if o is None and write_o:
+        o = torch.empty((T, Hv, Dv), dtype=torch.bfloat16, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((N, Hv, Dv, Dk), dtype=torch.float32, device=q.device)
+    if xq is None:
+        xq = torch.empty((T, Hv * Dv // 2), dtype=torch.uint8, device=q.device)
+    if xs is None:
+        xs = torch.empty((T, Hv * Dv // 16), dtype=torch.uint8, device=q.device)
+    _contig(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state, final_state, o, z, norm_weight, xq, xs)
+    ws_bytes = gdn_prefill_workspace_bytes(T, N, Hk, Hv, Dk, Dv)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=q.device)
+    st = LIB.gdn_prefill_chunked_gated_nvfp4(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(cu_seqlens), N, T, Hk, Hv,
+        Dk, Dv, float(scale), int(bool(qk_l2norm)), _dt(q), _ptr(initial_state), _ptr(final_state), _ptr(o),
+        _ptr(z), _ptr(norm_weight), float(eps), float(global_scale), _ptr(xq), _ptr(xs), _ptr(workspace),
+        0 if workspace is None else workspace.numel(), _stream(stream))
+    _check("gdn_prefill_chunked_gated_nvfp4", st)
+    return xq, xs, final_state, o
 
 
 def gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1.0,

@@ -104,6 +104,36 @@ gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v, cons
     return launched(gdn::launch_recurrent(r, st));
 }
 
+gdn_status gdn_prefill_chunked_gated_nvfp4(const void *q, const void *k, const void *v, const float *a,
+                                           const float *b, const float *A_log, const float *dt_bias,
+                                           const int32_t *cu_seqlens, int32_t num_seqs, int32_t T, int32_t Hk,
+                                           int32_t Hv, int32_t Dk, int32_t Dv, float scale, int32_t qk_l2norm,
+                                           gdn_dtype in_dtype, const float *initial_state, float *final_state,
+                                           void *o, const void *z, const float *norm_weight, float eps,
+                                           float global_scale, uint8_t *xq, uint8_t *xs, void *workspace,
+                                           size_t workspace_bytes, gdn_stream_t stream) {
+    if (T < 0 || num_seqs < 1 || Hk < 1 || Hv < 1 || Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens && num_seqs != 1) return GDN_ERR_INVALID_ARG;
+    if (Dk != 128 || Dv != 128 || in_dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (!A_log || !dt_bias) return GDN_ERR_INVALID_ARG;
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return GDN_ERR_INVALID_ARG;
+    if (T == 0)   // nothing to encode; the final state is the initial one
+        return gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens, num_seqs, T, Hk, Hv, Dk, Dv, scale,
+                                   qk_l2norm, in_dtype, initial_state, final_state, o, GDN_BF16, workspace,
+                                   workspace_bytes, stream);
+    if (!q || !k || !v || !a || !b || !z || !norm_weight || !xq || !xs) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) || (o && !aligned16(o)) ||
+        (reinterpret_cast<uintptr_t>(xq) & 3u))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn::chunked_workspace_bytes(T, num_seqs, Hk, Hv);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return GDN_ERR_WORKSPACE;
+    gdn::ChunkedArgs c{q, k, v, a, b, A_log, dt_bias, cu_seqlens, T, num_seqs, Hk, Hv, scale, qk_l2norm, true,
+                       initial_state, final_state, o, workspace, status_ptr(), z, norm_weight, eps, global_scale,
+                       xq, xs};
+    return launched(gdn::launch_chunked(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const float *a, const float *b,
                            const float *A_log, const float *dt_bias, int32_t B, int32_t Hk, int32_t Hv,
                            int32_t Dk, int32_t Dv, float scale, int32_t qk_l2norm, gdn_dtype in_dtype,

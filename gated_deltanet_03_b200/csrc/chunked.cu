@@ -580,6 +580,18 @@ constexpr int CH_OFF_STAGE = 2 * kWsItem;          // o staging, [r][i] (bf16 or
 constexpr int CH_OFF_BAR = CH_OFF_STAGE + 64 * 128 * 4;
 constexpr int CH_SMEM = CH_OFF_BAR + 128 + 1024;
 static_assert(CH_SMEM <= 232448, "chain shared memory");
+// Fused variant (gated RMSNorm + NVFP4 encode of each chunk's o rows): o staged in bf16 and
+// encoded by the workers while MMA45 of the next chunk runs; z tiles of three chunks in
+// flight (a chunk's tile is still read after the tile of the chunk after next is requested).
+constexpr int CHF_THREADS = CH_THREADS;
+constexpr int CHF_STAGE = 64 * 128 * 2;            // one chunk's o rows, bf16 [r][i]
+constexpr int CHF_OFF_Z = CH_OFF_STAGE + CHF_STAGE;
+constexpr int CHF_ZBYTES = 2 * TILE;               // [z_lo][z_hi], 64 tokens x 64 values each
+constexpr int CHF_OFF_RTAB = CHF_OFF_Z + 3 * CHF_ZBYTES;
+constexpr int CHF_OFF_BAR = CHF_OFF_RTAB + 128 * 4;
+constexpr int CHF_SMEM = CHF_OFF_BAR + 128 + 1024;
+static_assert(CHF_SMEM <= 232448, "fused chain shared memory");
+static_assert(CHF_OFF_Z % 1024 == 0, "TMA destination alignment");
 static_assert(kWsItem % 1024 == 0 && kWsKP % 1024 == 0, "1024-byte aligned operand tiles");
 // tensor memory: [D4 | D5a] (MMA45), [D7 | D5b] (MMA67), fp16 S0 (two slots) and U as A operands
 constexpr uint32_t C_TM_D45 = 0, C_TM_D67 = 128, C_TM_SA = 320, C_TM_UA = 448;
@@ -611,14 +623,18 @@ __device__ __forceinline__ void workers_sync() { asm volatile("barrier.cta.sync 
 enum ChainMode { kChainFull = 0, kChainState = 1, kChainTransition = 2 };
 
 struct ChainParams {
+    CUtensorMap zmap;      // fused output pass: z [T, Hv, 128] bf16, boxes of 64 values x 64 tokens
     const int32_t *cu_seqlens;
     int32_t T, num_seqs, Hv, slots, seg_chunks, seg_slots, mode_base, out_bf16;
     const float *S0g;
     float *S_out;
-    void *o;
+    void *o;               // may be null in the fused output pass
     const uint8_t *ws;     // per-chunk operand items
     uint8_t *ws_seg;       // per-segment B (fp32), M (fp16 hi/lo operand images), start state (fp32)
     int *status;
+    const float *norm_w;   // fused: RMSNorm weight [128], eps, NVFP4 encode scale and outputs
+    float eps, gs;
+    uint8_t *xq, *xs;
 };
 constexpr size_t kSegItem = kSegItemBytes;
 constexpr size_t kSegB = 0, kSegMhi = 65536, kSegMlo = 98304, kSegS = 131072;
@@ -646,13 +662,16 @@ __device__ __forceinline__ void ilv_store(uint8_t *base, int row, int wg, const 
 // coalesced side and the row-per-thread side are free of bank conflicts); `tid` in 0..255.
 constexpr int kStgPitch = 528;
 
-__global__ void __launch_bounds__(CH_THREADS, 1)
+// FUSED: the output pass also applies the gated RMSNorm to each chunk's o rows and writes them
+// NVFP4-encoded (o itself only when P.o is set).
+template <bool FUSED>
+__global__ void __launch_bounds__(FUSED ? CHF_THREADS : CH_THREADS, 1)
 gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
     pdl_launch_dependents();
     pdl_wait();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CH_OFF_BAR);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + (FUSED ? CHF_OFF_BAR : CH_OFF_BAR));
     uint64_t *full = bars, *bar_u = bars + 2, *bar_s = bars + 3, *bar_uready = bars + 4, *bar_sready = bars + 5;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
 
@@ -713,8 +732,14 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
         if (lane == 0) {
             auto issue_chunk = [&](int c) {
                 uint64_t *bar = &full[c & 1];
-                mbar_arrive_expect_tx(bar, kWsItem);
+                mbar_arrive_expect_tx(bar, kWsItem + (FUSED ? CHF_ZBYTES : 0));
                 bulk_load(sm + (c & 1) * kWsItem, ws_h + (size_t)(slot0 + c) * kWsItem, kWsItem, bar);
+                if constexpr (FUSED) {   // this chunk's z rows, two boxes of 64 values
+                    const int t0c = t_begin + (c_first + c) * C;
+                    uint8_t *zb = sm + CHF_OFF_Z + (c % 3) * CHF_ZBYTES;
+                    tma_load_3d(zb, &P.zmap, bar, 0, h, t0c);
+                    tma_load_3d(zb + TILE, &P.zmap, bar, 64, h, t0c);
+                }
             };
             if (nchunks > 0) issue_chunk(0);
             const bool full_out = mode == kChainFull;   // the output halves only when o is produced
@@ -752,6 +777,43 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
         const int row = (warp % 4) * 32 + lane;   // TMEM lane == value index i
         const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
         float S[64];   // S[i][64 wg .. 64 wg + 63], fp32
+        // fused: this thread's eight RMSNorm weights (16 threads per o row) and the encoder table
+        f2_t w2[4];
+        if constexpr (FUSED) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) w2[k] = f2(P.norm_w[(tid & 15) * 8 + 2 * k], P.norm_w[(tid & 15) * 8 + 2 * k + 1]);
+            nvfp4_fill_r_tab(reinterpret_cast<float *>(sm + CHF_OFF_RTAB), P.gs, tid);
+        }
+        // fused: gated RMSNorm + NVFP4 encode of rows [16 p0, 16 p1) of chunk cc, whose bf16 o rows
+        // are staged; 16 threads per row, eight values each (the same arithmetic as the
+        // standalone tail kernel); o written too when requested
+        auto epilogue = [&](int cc, int p0, int p1) {
+            const int t0e = t_begin + (c_first + cc) * C;
+            const int Le = min(C, t_end - t0e);
+            const uint8_t *stage = sm + CH_OFF_STAGE;
+            const uint8_t *zt = sm + CHF_OFF_Z + (cc % 3) * CHF_ZBYTES;
+            const float *r_tab = reinterpret_cast<const float *>(sm + CHF_OFF_RTAB);
+            uint8_t *ob = static_cast<uint8_t *>(P.o);
+            const int lr = tid & 15, col = lr * 8;
+#pragma unroll 1
+            for (int pass = p0; pass < p1; ++pass) {
+                const int r = pass * 16 + (tid >> 4);
+                const uint4 ou = *reinterpret_cast<const uint4 *>(stage + r * (D * 2) + col * 2);
+                const uint4 zu = *reinterpret_cast<const uint4 *>(zt + (col >> 6) * TILE + swz(r, (col & 63) >> 3));
+                const f2_t o2[4] = {bf16x2_to_f2(ou.x), bf16x2_to_f2(ou.y), bf16x2_to_f2(ou.z), bf16x2_to_f2(ou.w)};
+                const f2_t z2[4] = {bf16x2_to_f2(zu.x), bf16x2_to_f2(zu.y), bf16x2_to_f2(zu.z), bf16x2_to_f2(zu.w)};
+                f2_t y2[4];
+                gated_row8<16>(o2, z2, w2, 1.0f / (float)D, P.eps, y2);
+                uint32_t packed, sb;
+                nvfp4_encode_row8(y2, P.gs, r_tab, packed, sb);
+                if (r < Le) {
+                    const size_t base = ((size_t)(t0e + r) * Hv + h) * D + col;
+                    reinterpret_cast<uint32_t *>(P.xq)[base / 8] = packed;
+                    if ((lr & 1) == 0) P.xs[base / 16] = (uint8_t)sb;
+                    if (ob) *reinterpret_cast<uint4 *>(ob + base * 2) = ou;
+                }
+            }
+        };
         if (pseg == 0 && mode != kChainTransition && S0g) {
             // the caller's row-major initial state, staged in buffer 1 (its first chunk load is
             // issued only after every worker has released S0 through bar_sready)
@@ -855,7 +917,15 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
                 }
                 store_S(b ^ 1);   // S0 of chunk c + 1; releases the MMA warp
             }
-            if (mode == kChainFull) {
+            if (FUSED) {
+                // stage this chunk's o rows (bf16 [r][i]; the previous chunk's encode is done, a
+                // worker barrier has passed since) and encode them
+                __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(sm + CH_OFF_STAGE);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) st[(wg * 32 + j) * D + row] = __float2bfloat16_rn(ov[j]);
+                workers_sync();
+                epilogue(c, 0, 4);
+            } else if (mode == kChainFull) {
                 // o rows of this chunk: staged as [r][i], then 16-byte row stores (rows < L)
                 const int out_bf16 = P.out_bf16;
                 uint8_t *stage = sm + CH_OFF_STAGE;
@@ -1355,7 +1425,9 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gdn_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
+            e = cudaFuncSetAttribute(gdn_chunk_chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn_chunk_chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, CHF_SMEM);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(gdn_chunk_lean_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CL_SMEM);
         if (e == cudaSuccess)
@@ -1371,8 +1443,29 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
                                c.dt_bias, c.cu_seqlens, c.T, c.num_seqs, c.Hk, c.Hv, slots, c.scale, c.l2norm, ws,
                                c.status);
     if (e != cudaSuccess) return e;
-    ChainParams P{c.cu_seqlens, c.T, c.num_seqs, c.Hv, slots, seg, seg_slots, kChainFull, c.out_bf16 ? 1 : 0, c.S0,
-                  c.S_out, c.o, ws, ws + (size_t)c.Hv * slots * kWsItem, c.status};
+    ChainParams P{};
+    const bool fused = c.xq != nullptr;
+    if (fused && !make_map3(&P.zmap, c.z, c.T, c.Hv)) return cudaErrorInvalidValue;
+    P.cu_seqlens = c.cu_seqlens;
+    P.T = c.T;
+    P.num_seqs = c.num_seqs;
+    P.Hv = c.Hv;
+    P.slots = slots;
+    P.seg_chunks = seg;
+    P.seg_slots = seg_slots;
+    P.mode_base = kChainFull;
+    P.out_bf16 = c.out_bf16 ? 1 : 0;
+    P.S0g = c.S0;
+    P.S_out = c.S_out;
+    P.o = c.o;
+    P.ws = ws;
+    P.ws_seg = ws + (size_t)c.Hv * slots * kWsItem;
+    P.status = c.status;
+    P.norm_w = c.norm_w;
+    P.eps = c.eps;
+    P.gs = c.gs;
+    P.xq = c.xq;
+    P.xs = c.xs;
     if (c.T > kChunk * seg) {   // some sequence may span several segments
         P.mode_base = kChainState;   // z = 0: segment states (B), z = 1: segment transitions (M)
         if ((e = launch_pdl(gdn_chunk_lean_kernel, dim3(c.Hv, seg_slots, 2), dim3(NT), CL_SMEM, st, P)) != cudaSuccess)
@@ -1381,7 +1474,8 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
             return e;
         P.mode_base = kChainFull;
     }
-    return launch_pdl(gdn_chunk_chain_kernel, dim3(c.Hv, seg_slots, 1), dim3(CH_THREADS), CH_SMEM, st, P);
+    if (fused) return launch_pdl(gdn_chunk_chain_kernel<true>, dim3(c.Hv, seg_slots, 1), dim3(CHF_THREADS), CHF_SMEM, st, P);
+    return launch_pdl(gdn_chunk_chain_kernel<false>, dim3(c.Hv, seg_slots, 1), dim3(CH_THREADS), CH_SMEM, st, P);
 }
 
 }  // namespace gdn

@@ -343,6 +343,63 @@ GDN_DEV float rcp_approx(float x) {
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// bf16 word pair -> fp32 pair (exact: a bf16 is the high half of its fp32)
+GDN_DEV f2_t bf16x2_to_f2(uint32_t w) { return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)); }
+
+// Gated RMSNorm of one head row, eight values per thread, LANES threads per row (the row's
+// threads are consecutive lanes): y = o (w / rms(o)) z sigma(z), rms over the whole row,
+// sigma(z) = 1 / (1 + 2^(-z log2 e)). "Red Lite dev15d - DeltaNet gated tail", Pinned graph
+// semantics, steps 1-5. Shared by the standalone tail and the fused scan epilogue so that the
+// two agree bit for bit.
+template <int LANES>
+GDN_DEV void gated_row8(const f2_t (&o2)[4], const f2_t (&z2)[4], const f2_t (&w2)[4], float inv_d, float eps,
+                        f2_t (&y2)[4]) {
+    f2_t sq = mul2(o2[0], o2[0]);
+#pragma unroll
+    for (int k = 1; k < 4; ++k) sq = fma2(o2[k], o2[k], sq);
+    const float ss = group_sum<LANES>(f2lo(sq) + f2hi(sq));
+    const float inv_rms = rsqrtf(__fmaf_rn(ss, inv_d, eps));
+    const f2_t ir2 = f2(inv_rms, inv_rms), nlog2e = f2(-kLog2e, -kLog2e), one2 = f2(1.0f, 1.0f);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const f2_t t = mul2(z2[k], nlog2e);
+        const f2_t d = add2(f2(exp2_approx(f2lo(t)), exp2_approx(f2hi(t))), one2);
+        const f2_t sl = mul2(z2[k], f2(rcp_approx(f2lo(d)), rcp_approx(f2hi(d))));
+        y2[k] = mul2(mul2(o2[k], mul2(w2[k], ir2)), sl);
+    }
+}
+
+// NVFP4 encode of eight values of y (half of a 16-value block; the partner lane, lane ^ 1,
+// holds the other half): y rounded to bf16 first (the tensor the two-call path hands to the
+// encoder), block scale sb = E4M3((amax / 6) gs), codes E2M1(y r) with r = r_tab[sb] = gs / sb.
+GDN_DEV void nvfp4_encode_row8(f2_t (&y2)[4], float gs, const float *r_tab, uint32_t &packed, uint32_t &sb) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(f2lo(y2[k]), f2hi(y2[k]));
+        y2[k] = bf16x2_to_f2(*reinterpret_cast<const uint32_t *>(&hb));
+        amax = fmaxf(amax, fmaxf(fabsf(f2lo(y2[k])), fabsf(f2hi(y2[k]))));
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    sb = cvt_e4m3(__fmul_rn(div6_rn(amax), gs));
+    const float r = r_tab[sb & 127u];
+    const f2_t r2 = f2(r, r);
+    float p[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const f2_t q = mul2(y2[k], r2);
+        p[2 * k] = f2lo(q);
+        p[2 * k + 1] = f2hi(q);
+    }
+    packed = cvt_e2m1x8(p);
+}
+
+// The factor table of nvfp4_encode_row8 for encode scale gs: r_tab[c] = gs / E4M3(c), r_tab[0] = 0
+// (thread t < 128 of the block fills entry t; the caller synchronises).
+GDN_DEV void nvfp4_fill_r_tab(float *r_tab, float gs, int t) {
+    if (t < 128) r_tab[t] = t == 0 ? 0.0f : __fdiv_rn(gs, e4m3_to_f32((uint32_t)t));
+}
+
 // Programmatic dependent launch. Every kernel of this library is launched with programmatic
 // stream serialization (launch_pdl): it may start while the previous kernel in the stream is
 // still running, so it calls pdl_wait() before its first global-memory access (which returns

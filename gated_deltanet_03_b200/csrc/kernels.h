@@ -54,6 +54,11 @@ struct ChunkedArgs {
     void *o;
     void *ws;                    // workspace of chunked_workspace_bytes(T, num_seqs, Hk, Hv) bytes
     int *status;
+    // fused gated RMSNorm + NVFP4 encode of o (when xq is set; o may then be null):
+    const void *z;               // [T, Hv, 128] bf16
+    const float *norm_w;         // [128]
+    float eps, gs;
+    uint8_t *xq, *xs;            // [T, Hv * 64], [T, Hv * 8]
 };
 size_t chunked_workspace_bytes(int T, int num_seqs, int Hk, int Hv);
 cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st);

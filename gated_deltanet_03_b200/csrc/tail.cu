@@ -16,8 +16,6 @@ namespace gdn {
 
 constexpr int kTailThreads = 256;
 
-// bf16 word pair -> fp32 pair (exact: a bf16 is the high half of its fp32)
-__device__ __forceinline__ f2_t bf16x2_to_f2(uint32_t w) { return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)); }
 
 // Eight consecutive values as loaded (bf16: one 16-byte word; fp32: two), converted on use.
 template <bool BF16>
@@ -69,7 +67,7 @@ gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
     // NVFP4: the per-block factor r = gs / E4M3(sb) for every scale code (sb = 0: r = 0)
     __shared__ float r_tab[128];
     if constexpr (NVFP4) {
-        if (threadIdx.x < 128) r_tab[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __fdiv_rn(gs, e4m3_to_f32(threadIdx.x));
+        nvfp4_fill_r_tab(r_tab, gs, threadIdx.x);
         __syncthreads();
     }
     const int lane_in_row = threadIdx.x % LANES;
@@ -78,7 +76,6 @@ gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
 #pragma unroll
     for (int k = 0; k < 4; ++k) w2[k] = f2(w[col + 2 * k], w[col + 2 * k + 1]);
     const float inv_d = 1.0f / (float)D;
-    const f2_t nlog2e = f2(-kLog2e, -kLog2e), one2 = f2(1.0f, 1.0f);
     const int64_t stride = (int64_t)gridDim.x * RPB;
 
     // the loop condition is uniform over the block (the shuffles below need whole warps)
@@ -100,21 +97,8 @@ gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
             f2_t o2[4], z2[4];
             ro[u].get2(o2);
             rz[u].get2(z2);
-            f2_t sq = mul2(o2[0], o2[0]);
-#pragma unroll
-            for (int k = 1; k < 4; ++k) sq = fma2(o2[k], o2[k], sq);
-            const float ss = group_sum<LANES>(f2lo(sq) + f2hi(sq));
-            const float inv_rms = rsqrtf(ss * inv_d + eps);
-            const f2_t ir2 = f2(inv_rms, inv_rms);
-            // y = o (w / rms) z sigma(z), sigma(z) = 1 / (1 + 2^(-z log2 e))
             f2_t y2[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const f2_t t = mul2(z2[k], nlog2e);
-                const f2_t d = add2(f2(exp2_approx(f2lo(t)), exp2_approx(f2hi(t))), one2);
-                const f2_t sl = mul2(z2[k], f2(rcp_approx(f2lo(d)), rcp_approx(f2hi(d))));
-                y2[k] = mul2(mul2(o2[k], mul2(w2[k], ir2)), sl);
-            }
+            gated_row8<LANES>(o2, z2, w2, inv_d, eps, y2);
             if constexpr (!NVFP4) {
                 if (live) {
                     if constexpr (OUT_BF16) {
@@ -133,26 +117,8 @@ gated_rmsnorm_kernel(const void *__restrict__ o, const void *__restrict__ z,
                     }
                 }
             } else {
-                // y as the bf16 tensor the two-call path would hand to the encoder
-                float amax = 0.0f;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const __nv_bfloat162 hb = __floats2bfloat162_rn(f2lo(y2[k]), f2hi(y2[k]));
-                    y2[k] = bf16x2_to_f2(*reinterpret_cast<const uint32_t *>(&hb));
-                    amax = fmaxf(amax, fmaxf(fabsf(f2lo(y2[k])), fabsf(f2hi(y2[k]))));
-                }
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // partner lane: same block
-                const uint32_t sb = cvt_e4m3(__fmul_rn(div6_rn(amax), gs));
-                const float r = r_tab[sb & 127u];
-                const f2_t r2 = f2(r, r);
-                float p[8];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const f2_t q = mul2(y2[k], r2);
-                    p[2 * k] = f2lo(q);
-                    p[2 * k + 1] = f2hi(q);
-                }
-                const uint32_t packed = cvt_e2m1x8(p);
+                uint32_t packed, sb;
+                nvfp4_encode_row8(y2, gs, r_tab, packed, sb);
                 if (live) {
                     reinterpret_cast<uint32_t *>(xq)[base / 8] = packed;
                     if ((lane_in_row & 1) == 0) xs[base / 16] = (uint8_t)sb;

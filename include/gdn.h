@@ -106,6 +106,34 @@ GDN_API gdn_status gdn_prefill_chunked(const void *q, const void *k, const void 
 GDN_API size_t gdn_prefill_workspace_bytes(int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv,
                                    int32_t Dk, int32_t Dv);
 
+/* ------------------------------------------------- prefill + gated tail, fused ----
+ * [GDN] + [TAIL] "Pinned graph semantics", steps 1-5, with the NVFP4 activation encode of
+ * [GDN] mechanism i: the prefill above, whose output pass also applies the gated RMSNorm to
+ * every o row and writes it as NVFP4 activations for the output projection, so that neither o
+ * nor the gated y has to round-trip through HBM. The result is bit for bit that of
+ *   gdn_prefill_chunked(..., o bf16 ...) followed by gdn_gated_rmsnorm_silu_nvfp4(o, z, ...):
+ * the tail reads o rounded to bf16, as the two-call path stores it.
+ * Arguments as gdn_prefill_chunked, plus
+ * o            [T, Hv, 128] bf16 output, or NULL (o is then not written)
+ * z            [T, Hv, 128] bf16 gate input; norm_weight [128] fp32 (one weight for all heads); eps
+ * global_scale NVFP4 encode scale gs (block scale E4M3((amax / 6) gs), codes E2M1(y gs / scale))
+ * xq           [T, Hv * 64] u8: two E2M1 codes per byte, element 2j in the low nibble of byte j
+ * xs           [T, Hv * 8] E4M3 block scales, one per 16 consecutive values
+ * Supported: Dk == Dv == 128 and bf16 inputs (the tensor-core path), else GDN_ERR_UNSUPPORTED;
+ * the workspace is the one gdn_prefill_workspace_bytes gives. xq must be 4-byte aligned.
+ */
+GDN_API gdn_status gdn_prefill_chunked_gated_nvfp4(const void *q, const void *k, const void *v,
+                                           const float *a, const float *b,
+                                           const float *A_log, const float *dt_bias,
+                                           const int32_t *cu_seqlens, int32_t num_seqs,
+                                           int32_t T, int32_t Hk, int32_t Hv, int32_t Dk, int32_t Dv,
+                                           float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                                           const float *initial_state, float *final_state,
+                                           void *o, const void *z, const float *norm_weight,
+                                           float eps, float global_scale, uint8_t *xq, uint8_t *xs,
+                                           void *workspace, size_t workspace_bytes,
+                                           gdn_stream_t stream);
+
 /* ------------------------------------------------------------------- decode ----
  * [GDN]: one token per sequence; the state is read once and written once, in place.
  * q, k [B, Hk, Dk], v [B, Hv, Dv] in `in_dtype`; a, b [B, Hv] fp32; A_log, dt_bias [Hv];
