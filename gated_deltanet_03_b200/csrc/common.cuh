@@ -351,14 +351,17 @@ GDN_DEV f2_t bf16x2_to_f2(uint32_t w) { return f2(__uint_as_float(w << 16), __ui
 // sigma(z) = 1 / (1 + 2^(-z log2 e)). "Red Lite dev15d - DeltaNet gated tail", Pinned graph
 // semantics, steps 1-5. Shared by the standalone tail and the fused scan epilogue so that the
 // two agree bit for bit.
-template <int LANES>
-GDN_DEV void gated_row8(const f2_t (&o2)[4], const f2_t (&z2)[4], const f2_t (&w2)[4], float inv_d, float eps,
-                        f2_t (&y2)[4]) {
+// Sum of squares of eight values as the tail's threads form it: pairwise fp32x2 fma over the
+// four pairs, then the two lanes added.
+GDN_DEV float row_sumsq8(const f2_t (&o2)[4]) {
     f2_t sq = mul2(o2[0], o2[0]);
 #pragma unroll
     for (int k = 1; k < 4; ++k) sq = fma2(o2[k], o2[k], sq);
-    const float ss = group_sum<LANES>(f2lo(sq) + f2hi(sq));
-    const float inv_rms = rsqrtf(__fmaf_rn(ss, inv_d, eps));
+    return f2lo(sq) + f2hi(sq);
+}
+
+// y = o (w inv_rms) z sigma(z) for eight values, sigma(z) = 1 / (1 + 2^(-z log2 e)).
+GDN_DEV void gated_apply8(const f2_t (&o2)[4], const f2_t (&z2)[4], const f2_t (&w2)[4], float inv_rms, f2_t (&y2)[4]) {
     const f2_t ir2 = f2(inv_rms, inv_rms), nlog2e = f2(-kLog2e, -kLog2e), one2 = f2(1.0f, 1.0f);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -369,9 +372,21 @@ GDN_DEV void gated_row8(const f2_t (&o2)[4], const f2_t (&z2)[4], const f2_t (&w
     }
 }
 
+// Gated RMSNorm of one head row, eight values per thread, LANES threads per row (the row's
+// threads are consecutive lanes): y = o (w / rms(o)) z sigma(z), rms over the whole row.
+// "Red Lite dev15d - DeltaNet gated tail", Pinned graph semantics, steps 1-5. Shared by the
+// standalone tail and the fused kernels so that they agree bit for bit.
+template <int LANES>
+GDN_DEV void gated_row8(const f2_t (&o2)[4], const f2_t (&z2)[4], const f2_t (&w2)[4], float inv_d, float eps,
+                        f2_t (&y2)[4]) {
+    const float ss = group_sum<LANES>(row_sumsq8(o2));
+    gated_apply8(o2, z2, w2, rsqrtf(__fmaf_rn(ss, inv_d, eps)), y2);
+}
+
 // NVFP4 encode of eight values of y (half of a 16-value block; the partner lane, lane ^ 1,
 // holds the other half): y rounded to bf16 first (the tensor the two-call path hands to the
-// encoder), block scale sb = E4M3((amax / 6) gs), codes E2M1(y r) with r = r_tab[sb] = gs / sb.
+// encoder), block scale sb = E4M3((amax / 6) gs), codes E2M1(y r) with r = gs / sb (from r_tab
+// when given, else by division).
 GDN_DEV void nvfp4_encode_row8(f2_t (&y2)[4], float gs, const float *r_tab, uint32_t &packed, uint32_t &sb) {
     float amax = 0.0f;
 #pragma unroll
@@ -382,7 +397,8 @@ GDN_DEV void nvfp4_encode_row8(f2_t (&y2)[4], float gs, const float *r_tab, uint
     }
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     sb = cvt_e4m3(__fmul_rn(div6_rn(amax), gs));
-    const float r = r_tab[sb & 127u];
+    // r = gs / E4M3(sb) (0 for sb = 0), from the table when one is given
+    const float r = r_tab ? r_tab[sb & 127u] : ((sb & 127u) == 0 ? 0.0f : __fdiv_rn(gs, e4m3_to_f32(sb & 127u)));
     const f2_t r2 = f2(r, r);
     float p[8];
 #pragma unroll
