@@ -26,7 +26,7 @@ GDN_BF16, GDN_F32 = 0, 1
 ABI_SYMBOLS = (
     "gdn_prefill_chunked", "gdn_prefill_workspace_bytes", "gdn_prefill_chunked_gated_nvfp4", "gdn_decode_step",
     "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act",
-    "nvfp4_gemm", "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_status_string",
+    "nvfp4_gemm", "nvfp4_gemm_colscale", "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_status_string",
     "gdn_version",
 )
 
@@ -55,6 +55,7 @@ def _load() -> ctypes.CDLL:
     lib.gdn_gated_rmsnorm_silu_nvfp4.argtypes = [P, P, P, f32, i32, i32, i32, i32, f32, P, P, P]
     lib.nvfp4_quantize_act.argtypes = [P, i32, i32, i32, f32, P, P, P]
     lib.nvfp4_gemm.argtypes = [P, P, P, P, f32, i32, i32, i32, i32, P, P]
+    lib.nvfp4_gemm_colscale.argtypes = [P, P, P, P, P, i32, i32, i32, i32, P, P]
     lib.gdn_prefill_chunked_static_ws.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32,
                                                   i32, i32, P, P, P, i32, P]
     lib.gdn_get_device_status.argtypes = [P]
@@ -62,7 +63,7 @@ def _load() -> ctypes.CDLL:
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_version.restype = i32
     for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_gated_nvfp4", "gdn_prefill_chunked_static_ws", "gdn_decode_step", "gdn_gated_rmsnorm_silu",
-                 "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_gemm",
+                 "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_gemm_colscale",
                  "gdn_get_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -240,6 +241,28 @@ def nvfp4_gemm(aq, as_, bq, bs, alpha: float, out_dtype=torch.bfloat16, y=None, 
                         _stream(stream))
     _check("nvfp4_gemm", st)
     return y
+
+
+def nvfp4_gemm_colscale(aq, as_, bq, bs, col_alpha, out_dtype=torch.bfloat16, y=None, stream=None):
+    """nvfp4_gemm with a per-output-column factor col_alpha [N] fp32 (modules fused into one
+    weight, each with its own global scale)."""
+    M, K = aq.shape[0], aq.shape[1] * 2
+    N = bq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=aq.device)
+    _contig(aq, as_, bq, bs, col_alpha, y)
+    st = LIB.nvfp4_gemm_colscale(_ptr(aq), _ptr(as_), _ptr(bq), _ptr(bs), _ptr(col_alpha), M, N, K, _dt(y), _ptr(y),
+                                 _stream(stream))
+    _check("nvfp4_gemm_colscale", st)
+    return y
+
+
+def fused_module_col_alpha(widths, module_scales, act_scale: float, device=None):
+    """col_alpha for a weight made of modules of the given output widths, module i quantised with
+    global scale module_scales[i], activations with act_scale: 1 / (act_scale * module scale)."""
+    parts = [torch.full((int(n),), float(1.0 / (act_scale * float(s))), dtype=torch.float32)
+             for n, s in zip(widths, module_scales)]
+    return torch.cat(parts).to(device if device is not None else "cuda")
 
 
 def gdn_get_device_status(stream=None) -> int:

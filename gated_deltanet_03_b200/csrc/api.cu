@@ -203,7 +203,20 @@ gdn_status nvfp4_gemm(const uint8_t *aq, const uint8_t *as, const uint8_t *bq, c
     if (K == 0) return GDN_ERR_UNSUPPORTED;
     if (!aq || !as || !bq || !bs || !y) return GDN_ERR_INVALID_ARG;
     if (!aligned16(aq) || !aligned16(bq) || !aligned16(y)) return GDN_ERR_INVALID_ARG;
-    gdn::GemmArgs g{aq, as, bq, bs, alpha, M, N, K, out_dtype == GDN_BF16, y, status_ptr()};
+    gdn::GemmArgs g{aq, as, bq, bs, alpha, M, N, K, out_dtype == GDN_BF16, y, status_ptr(), nullptr};
+    return launched(gdn::launch_nvfp4_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gdn_status nvfp4_gemm_colscale(const uint8_t *aq, const uint8_t *as, const uint8_t *bq, const uint8_t *bs,
+                               const float *col_alpha, int32_t M, int32_t N, int32_t K, gdn_dtype out_dtype,
+                               void *y, gdn_stream_t stream) {
+    if (M < 0 || N < 0 || K < 0 || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
+    if (K % 32 != 0 || N % 16 != 0) return GDN_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return GDN_OK;
+    if (K == 0) return GDN_ERR_UNSUPPORTED;
+    if (!aq || !as || !bq || !bs || !y || !col_alpha) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(aq) || !aligned16(bq) || !aligned16(y)) return GDN_ERR_INVALID_ARG;
+    gdn::GemmArgs g{aq, as, bq, bs, 1.0f, M, N, K, out_dtype == GDN_BF16, y, status_ptr(), col_alpha};
     return launched(gdn::launch_nvfp4_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -87,6 +87,7 @@ struct GemmArgs {
     bool out_bf16;
     void *y;
     int *status;
+    const float *col_alpha;      // [N] per-column factor, or null: alpha for every column
 };
 cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st);
 

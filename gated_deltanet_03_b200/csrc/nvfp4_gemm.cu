@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                   const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                   const __grid_constant__ CUtensorMap map_y, int sf_tma, const uint8_t *__restrict__ sfa_g, const uint8_t *__restrict__ sfb_g, float alpha,
+                  const float *__restrict__ col_alpha,
                   int M, int N, int K, int out_bf16, void *__restrict__ y, int *status) {
     pdl_launch_dependents();
     extern __shared__ uint8_t smem_raw[];
@@ -235,7 +236,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     const int c0 = c1 + 32 * hh;
                     float v[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rr[hh][j]) * alpha;
+                    for (int j = 0; j < 32; ++j) {
+                        // per-column factor when the output columns come from modules with their
+                        // own global scales (clamped index: columns past N are never stored)
+                        const float al = col_alpha ? __ldg(col_alpha + min(tile_n * BN + c0 + j, N - 1)) : alpha;
+                        v[j] = __uint_as_float(rr[hh][j]) * al;
+                    }
                     if (out_bf16) {
                         uint8_t *box = obox + (c0 / 64) * 16384 + r * 128;
 #pragma unroll
@@ -340,7 +346,7 @@ cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
     }
     dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM);
     return launch_pdl(nvfp4_gemm_kernel, grid, dim3(THREADS), SMEM_BYTES, st, ma, mb, msa, msb, my, sf_tma ? 1 : 0,
-                      g.as, g.bs, g.alpha, g.M, g.N, g.K, g.out_bf16 ? 1 : 0, g.y, g.status);
+                      g.as, g.bs, g.alpha, g.col_alpha, g.M, g.N, g.K, g.out_bf16 ? 1 : 0, g.y, g.status);
 }
 
 }  // namespace gdn

@@ -195,6 +195,16 @@ GDN_API gdn_status nvfp4_gemm(const uint8_t *aq, const uint8_t *as, const uint8_
                       float alpha, int32_t M, int32_t N, int32_t K, gdn_dtype out_dtype, void *y,
                       gdn_stream_t stream);
 
+/* NVFP4 GEMM whose output columns come from several modules fused into one weight matrix,
+ * each quantised with its own calibrated global scale ([GDN] abstract: the global-scale
+ * mismatch of per-module-calibrated NVFP4 checkpoints served by kernels that fuse those modules
+ * into one GEMM, and its repair): column n is scaled by col_alpha[n] = 1 / (global_scale_a *
+ * global_scale of the module column n belongs to), instead of one alpha for the whole output.
+ * col_alpha: device fp32 [N]. Other arguments and limits as nvfp4_gemm. */
+GDN_API gdn_status nvfp4_gemm_colscale(const uint8_t *aq, const uint8_t *as, const uint8_t *bq,
+                                       const uint8_t *bs, const float *col_alpha, int32_t M, int32_t N,
+                                       int32_t K, gdn_dtype out_dtype, void *y, gdn_stream_t stream);
+
 /* ------------------------------------------------- allocation-free prefill ----
  * No counterpart in the paper. For callers that cannot allocate device memory - code that
  * runs where cudaMalloc is unavailable or not allowed, or a host framework that owns every

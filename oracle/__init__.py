@@ -17,7 +17,10 @@ Each function cites the passage it follows (page title, section):
   * gated tail: "Red Lite dev15d - DeltaNet gated tail" (Pinned graph semantics, 1-6);
   * NVFP4: "Why Gated DeltaNet Survives 4-Bit Quantization" (abstract, mechanism i:
     16-element block scaling), E2M1 values with E4M3 block scales and an fp32 global
-    scale.
+    scale;
+  * short convolution: "A Node-by-Node White-Box Walkthrough of a Quantized Hybrid Gated
+    DeltaNet Language Model" (Principais Contribuicoes, item 2: the short convolutions on the
+    layer's path), read as the depthwise causal convolution of width K followed by SiLU.
 
 Parity pins: every function here is checked by ``tests/test_oracle_pins.py`` against
 closed forms, invariants, library routines or brute force. None is "parity unpinned".
@@ -243,3 +246,31 @@ def e4m3_decode(codes):
     lib = _load()
     return np.array([lib.oracle_e4m3_decode(int(c)) for c in np.asarray(codes).ravel()],
                     dtype=np.float32)
+
+
+def short_conv1d_silu(x, weight, cu_seqlens=None, initial_state=None):
+    """Depthwise causal convolution of width K over each sequence, then SiLU, in fp64:
+    y[t, c] = SiLU(sum_{j<K} weight[c, j] x[t - (K - 1) + j, c]), where inputs before a
+    sequence's first token come from initial_state[n] ([K - 1, C], oldest first) or are zero.
+    x [T, C]; weight [C, K]; cu_seqlens [N + 1] or None (one sequence).
+    Returns (y [T, C] fp64, final_state [N, K - 1, C]: each sequence's last K - 1 inputs,
+    continuing the initial state when the sequence is shorter)."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(weight, dtype=np.float64)
+    T, C = x.shape
+    K = w.shape[1]
+    cu = np.array([0, T]) if cu_seqlens is None else np.asarray(cu_seqlens)
+    N = len(cu) - 1
+    y = np.zeros((T, C))
+    final = np.zeros((N, K - 1, C))
+    for n in range(N):
+        t0, t1 = int(cu[n]), int(cu[n + 1])
+        hist = np.zeros((K - 1, C)) if initial_state is None else np.asarray(initial_state[n], dtype=np.float64)
+        window = np.concatenate([hist, x[t0:t1]], axis=0)     # row K - 1 + i is token t0 + i
+        for i in range(t1 - t0):
+            acc = np.zeros(C)
+            for j in range(K):
+                acc += w[:, j] * window[i + j]
+            y[t0 + i] = acc / (1.0 + np.exp(-acc))
+        final[n] = window[len(window) - (K - 1):] if K > 1 else final[n]
+    return y, final

@@ -76,3 +76,42 @@ def test_gemm_full_size_sampled_rows(g, M, N, K):
     rows = np.concatenate([rows, [0, M - 1]])
     ref = oracle.nvfp4_gemm(aq, as_, gsa, wq, ws, gsw, rows=rows)
     assert rel_err(y[rows], ref) <= TOL_GEMM
+
+
+@pytest.mark.parametrize("M", [64, 300])
+def test_fused_modules_colscale(g, M):
+    """Several modules fused into one weight (as in a fused in_proj: q, k, v, z, a, b), each
+    calibrated and quantised with its own global scale; the gate modules an order of magnitude
+    smaller. With the per-column factor the fused GEMM matches the oracle module by module; with
+    one factor for the whole output (the mismatch) the modules whose scale differs are off."""
+    K = 512
+    widths = (128, 128, 256, 256, 16, 16)
+    mags = (0.02, 0.02, 0.02, 0.02, 0.001, 0.001)
+    rng = np.random.default_rng(M)
+    A = workloads.activations(M, K, seed=M + 1)
+    gsa = np.float32(448.0 * 6.0 / np.abs(A).max())
+    aq, as_ = oracle.nvfp4_quantize(A, gsa)
+    wqs, wss, gsws, refs = [], [], [], []
+    for n, mag in zip(widths, mags):
+        W = workloads.round_bf16(rng.standard_normal((n, K)).astype(np.float32) * mag)
+        gsw = np.float32(448.0 * 6.0 / np.abs(W).max())
+        wq, ws = oracle.nvfp4_quantize(W, gsw)
+        wqs.append(wq)
+        wss.append(ws)
+        gsws.append(gsw)
+        refs.append(oracle.nvfp4_gemm(aq, as_, gsa, wq, ws, gsw))
+    wq, ws, ref = np.concatenate(wqs), np.concatenate(wss), np.concatenate(refs, axis=1)
+    u8 = torch.uint8
+    ca = g.fused_module_col_alpha(widths, gsws, float(gsa))
+    y = to_np(g.nvfp4_gemm_colscale(dev(aq, u8), dev(as_, u8), dev(wq, u8), dev(ws, u8), ca, out_dtype=torch.float32))
+    torch.cuda.synchronize()
+    assert g.gdn_get_device_status() == 0
+    col = 0
+    for n in widths:
+        assert rel_err(y[:, col:col + n], ref[:, col:col + n]) <= TOL_GEMM
+        col += n
+    # one global scale (the first module's) for the fused output: the gate modules come out wrong
+    alpha0 = float(np.float32(1.0) / (gsa * gsws[0]))
+    y1 = _gpu(g, aq, as_, wq, ws, alpha0, torch.float32)
+    gate = slice(sum(widths[:4]), sum(widths))
+    assert rel_err(y1[:, gate], ref[:, gate]) > 100 * TOL_GEMM
