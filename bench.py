@@ -255,6 +255,17 @@ def run_gpu(args):
         fused()
         gemm()
 
+    # the causal short convolution in front of the scan (q|k|v channels of the same layer, K = 4),
+    # timed alone: not part of the step, whose inputs are the scan's
+    conv_C = 2 * w.Hk * D + Hv * D
+    cx = workloads.conv_inputs(T, conv_C, 4, seed=w.seed)
+    conv_x, conv_w = up(cx["x"], bf), up(cx["weight"], f32)
+    conv_y = torch.empty((T * conv_C,), dtype=bf, device=dev)
+    conv_parts = (w.Hk * D, w.Hk * D, Hv * D)
+
+    def conv():
+        g.gdn_short_conv1d_silu(conv_x, conv_w, parts=conv_parts, y=conv_y)
+
     for _ in range(args.warmup):
         flush()
         step()
@@ -266,7 +277,8 @@ def run_gpu(args):
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
-        for name, fn in (("step", step), ("scan", scan), ("tail", tail), ("fused", fused), ("gemm", gemm)):
+        for name, fn in (("step", step), ("scan", scan), ("tail", tail), ("fused", fused), ("gemm", gemm),
+                         ("conv", conv)):
             fn()
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=side):
@@ -297,7 +309,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     parts = {}
-    for name in ("scan", "tail", "fused", "gemm"):
+    for name in ("scan", "tail", "fused", "gemm", "conv"):
         evs = timed(graphs[name], args.steps)
         torch.cuda.synchronize()
         parts[name] = [a.elapsed_time(b) for a, b in evs]
@@ -351,20 +363,52 @@ def run_gpu(args):
     dA, ddt = up(dx["A_log"], f32), up(dx["dt_bias"], f32)
     dstate = up(dx["initial_state"], f32)
     dout = torch.empty((dw.num_seqs, dw.Hv, dw.D), dtype=bf, device=dev)
+
+    def graph_of(fn):
+        # device time of one launch, without the host's launch gap between the events
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=side):
+                fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        return gr
+
+    dec_graph = graph_of(lambda: g.gdn_decode_step(dq, dk, dv, da, db, dA, ddt, dstate, o=dout))
     for _ in range(max(3, args.warmup)):
-        g.gdn_decode_step(dq, dk, dv, da, db, dA, ddt, dstate, o=dout)
+        dec_graph.replay()
     torch.cuda.synchronize()
     dec_ms = []
     for _ in range(max(args.steps, 10)):
         s0, s1 = ev(), ev()
         s0.record(stream)
-        g.gdn_decode_step(dq, dk, dv, da, db, dA, ddt, dstate, o=dout)
+        dec_graph.replay()
         s1.record(stream)
         torch.cuda.synchronize()
         dec_ms.append(s0.elapsed_time(s1))
     dec = statistics.median(dec_ms)
     state_bytes = dstate.numel() * 4
     dec_bytes = 2 * state_bytes + sum(t.numel() * t.element_size() for t in (dq, dk, dv, da, db, dout))
+
+    # short convolution decode on the batched-decode workload's q|k|v channels (state in place)
+    dC = 2 * dw.Hk * dw.D + dw.Hv * dw.D
+    dcx = workloads.conv_inputs(dw.num_seqs, dC, 4, seed=dw.seed, num_seqs=dw.num_seqs, state=True)
+    dconv_x, dconv_w = up(dcx["x"], bf), up(dcx["weight"], f32)
+    dconv_s = up(dcx["initial_state"], bf)
+    dconv_y = torch.empty((dw.num_seqs * dC,), dtype=bf, device=dev)
+    dparts = (dw.Hk * dw.D, dw.Hk * dw.D, dw.Hv * dw.D)
+    cdec_graph = graph_of(lambda: g.gdn_short_conv1d_silu_decode(dconv_x, dconv_w, dconv_s, parts=dparts,
+                                                                  y=dconv_y))
+    for _ in range(max(3, args.warmup)):
+        cdec_graph.replay()
+    torch.cuda.synchronize()
+    cdec_ev = timed(cdec_graph, max(args.steps, 10))     # L2 flushed before each replay
+    torch.cuda.synchronize()
+    cdec = statistics.median(a.elapsed_time(b) for a, b in cdec_ev)
+    cdec_bytes = 2 * dconv_x.numel() * 2 + 2 * dconv_s.numel() * 2 + dconv_w.numel() * 4
+    assert g.gdn_get_device_status() == 0
 
     if world > 1:
         dist.barrier()
@@ -373,6 +417,7 @@ def run_gpu(args):
         return
 
     pk, pk_kind = peaks()
+    conv_bytes = 2 * T * conv_C * 2 + conv_w.numel() * 4     # x read once, y written once, weights
     scan_s = statistics.mean(fused_ms) / 1e3
     fl = scan_flops(w)
     achieved_tflops = fl / scan_s / 1e12
@@ -411,6 +456,14 @@ def run_gpu(args):
         "decode": {"workload": dw.name, "ms": dec, "GB/s": dec_bytes / (dec / 1e3) / 1e9,
                    "frac": dec_bytes / (dec / 1e3) / 1e9 / float(pk["hbm_gbs"]),
                    "bytes": dec_bytes, "peak_gbs": float(pk["hbm_gbs"]), "peak_kind": pk_kind},
+        "short_conv": {"workload": "%s q|k|v channels (T = %d, C = %d, K = 4), planes q, k, v" % (w.name, T, conv_C),
+                       "ms": statistics.mean(parts["conv"]),
+                       "GB/s": conv_bytes / (statistics.mean(parts["conv"]) / 1e3) / 1e9,
+                       "frac": conv_bytes / (statistics.mean(parts["conv"]) / 1e3) / 1e9 / float(pk["hbm_gbs"]),
+                       "bytes": conv_bytes, "bound": "hbm", "peak_kind": pk_kind,
+                       "decode": {"workload": "%s q|k|v channels (B = %d, C = %d, K = 4)" % (dw.name, dw.num_seqs, dC),
+                                  "ms": cdec, "bytes": cdec_bytes,
+                                  "GB/s": cdec_bytes / (cdec / 1e3) / 1e9}},
         "gpu_launches": launches_per_step * args.steps,
         "gpu_kernels_per_step": kernel_names,
         "clocks": clk.summary(),
@@ -429,7 +482,7 @@ def run_only(args):
     dev = torch.device("cuda", 0)
     bf, f32 = torch.bfloat16, torch.float32
     names = {wl.name: wl for wl in workloads.WORKLOADS}
-    w = names[args.workload] if args.workload else (workloads.DECODE_B256 if args.only == "decode"
+    w = names[args.workload] if args.workload else (workloads.DECODE_B256 if args.only in ("decode", "conv_decode")
                                                     else workloads.PREFILL_1K)
     x = workloads.generate(w)
 
@@ -450,7 +503,17 @@ def run_only(args):
     Y = torch.empty((w.T, w.n_out), dtype=bf, device=dev)
     g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=cu, initial_state=S0, final_state=S, o=o)
     g.gdn_gated_rmsnorm_silu_nvfp4(o, z, nw, 1.0, xq=xq, xs=xs)
+    conv_C = 2 * w.Hk * w.D + w.Hv * w.D
+    cx = workloads.conv_inputs(w.T, conv_C, 4, seed=w.seed)
+    conv_x, conv_w = up(cx["x"], bf), up(cx["weight"], f32)
+    conv_y = torch.empty((w.T * conv_C,), dtype=bf, device=dev)
+    dcx = workloads.conv_inputs(w.num_seqs, conv_C, 4, seed=w.seed, num_seqs=w.num_seqs, state=True)
+    dconv_x, dconv_s = up(dcx["x"], bf), up(dcx["initial_state"], bf)
     fn = {
+        "conv_decode": lambda: g.gdn_short_conv1d_silu_decode(dconv_x, conv_w, dconv_s,
+                                                              parts=(w.Hk * w.D, w.Hk * w.D, w.Hv * w.D)),
+        "conv": lambda: g.gdn_short_conv1d_silu(conv_x, conv_w, parts=(w.Hk * w.D, w.Hk * w.D, w.Hv * w.D),
+                                                y=conv_y),
         "scan": lambda: g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=cu, initial_state=S0,
                                               final_state=S, o=o),
         "tail": lambda: g.gdn_gated_rmsnorm_silu_nvfp4(o, z, nw, 1.0, xq=xq, xs=xs),
@@ -538,7 +601,7 @@ def main():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
-    p.add_argument("--only", choices=["scan", "tail", "gemm", "decode", "fused"],
+    p.add_argument("--only", choices=["scan", "tail", "gemm", "decode", "fused", "conv", "conv_decode"],
                    help="time one kernel alone on its workload (for profiling); prints one JSON line")
     p.add_argument("--workload", default=None, help="workload name for --only scan (default: 1024-wide prefill)")
     args = p.parse_args()

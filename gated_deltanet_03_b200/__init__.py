@@ -7,6 +7,7 @@ stream. There is no CPU fallback: if the library is missing, importing this pack
 Functions keep the C names:
   gdn_prefill_chunked, gdn_prefill_chunked_gated_nvfp4, gdn_decode_step, gdn_gated_rmsnorm_silu,
   gdn_gated_rmsnorm_silu_nvfp4, nvfp4_quantize_act, nvfp4_gemm,
+  nvfp4_gemm_colscale, gdn_short_conv1d_silu, gdn_short_conv1d_silu_decode,
   gdn_prefill_workspace_bytes, gdn_get_device_status.
 """
 from __future__ import annotations
@@ -26,7 +27,8 @@ GDN_BF16, GDN_F32 = 0, 1
 ABI_SYMBOLS = (
     "gdn_prefill_chunked", "gdn_prefill_workspace_bytes", "gdn_prefill_chunked_gated_nvfp4", "gdn_decode_step",
     "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act",
-    "nvfp4_gemm", "nvfp4_gemm_colscale", "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_status_string",
+    "nvfp4_gemm", "nvfp4_gemm_colscale", "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode",
+    "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_status_string",
     "gdn_version",
 )
 
@@ -56,6 +58,9 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_quantize_act.argtypes = [P, i32, i32, i32, f32, P, P, P]
     lib.nvfp4_gemm.argtypes = [P, P, P, P, f32, i32, i32, i32, i32, P, P]
     lib.nvfp4_gemm_colscale.argtypes = [P, P, P, P, P, i32, i32, i32, i32, P, P]
+    i64 = ctypes.c_int64
+    lib.gdn_short_conv1d_silu.argtypes = [P, i64, P, P, i32, i32, i32, i32, P, P, P, P, i32, P]
+    lib.gdn_short_conv1d_silu_decode.argtypes = [P, i64, P, i32, i32, i32, P, P, P, i32, P]
     lib.gdn_prefill_chunked_static_ws.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32,
                                                   i32, i32, P, P, P, i32, P]
     lib.gdn_get_device_status.argtypes = [P]
@@ -64,7 +69,7 @@ def _load() -> ctypes.CDLL:
     lib.gdn_version.restype = i32
     for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_gated_nvfp4", "gdn_prefill_chunked_static_ws", "gdn_decode_step", "gdn_gated_rmsnorm_silu",
                  "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_gemm_colscale",
-                 "gdn_get_device_status"):
+                 "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode", "gdn_get_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -263,6 +268,61 @@ def fused_module_col_alpha(widths, module_scales, act_scale: float, device=None)
     parts = [torch.full((int(n),), float(1.0 / (act_scale * float(s))), dtype=torch.float32)
              for n, s in zip(widths, module_scales)]
     return torch.cat(parts).to(device if device is not None else "cuda")
+
+
+def _conv_rows(x):
+    """(rows, C, ldx) of a bf16 [rows, C] tensor whose rows may be strided (a column slice of a
+    wider projection output)."""
+    if x.dim() != 2 or x.dtype != torch.bfloat16 or (x.shape[1] > 1 and x.stride(1) != 1):
+        raise ValueError("x must be bf16 [rows, C] with unit channel stride")
+    return x.shape[0], x.shape[1], x.stride(0) if x.shape[0] > 1 else x.shape[1]
+
+
+def _conv_planes(parts, rows, C, y, device):
+    """Output buffer and the views of its planes ([rows, width] each, one after another)."""
+    widths = [C] if parts is None else [int(p) for p in parts]
+    if y is None:
+        y = torch.empty((rows * C,), dtype=torch.bfloat16, device=device)
+    _contig(y)
+    arr = (ctypes.c_int32 * len(widths))(*widths)
+    views, off = [], 0
+    for wd in widths:
+        views.append(y.view(-1)[off:off + rows * wd].view(rows, wd))
+        off += rows * wd
+    return y, arr, views
+
+
+def gdn_short_conv1d_silu(x, weight, cu_seqlens=None, num_seqs=None, initial_state=None,
+                          final_state=None, output_final_state=False, parts=None, y=None, stream=None):
+    """Causal depthwise convolution (width K = weight.shape[1]) + SiLU over packed sequences.
+    x bf16 [T, C] (rows may be strided); weight fp32 [C, K]; states bf16 [N, K - 1, C]
+    (final_state may be initial_state: updated in place). parts: plane widths (e.g. q, k, v
+    channel counts) -> the outputs are [T, width] views of one buffer. Returns (y or the list of
+    plane views, final_state)."""
+    T, C, ldx = _conv_rows(x)
+    K = weight.shape[1]
+    N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (num_seqs or 1)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, K - 1, C), dtype=torch.bfloat16, device=x.device)
+    _contig(weight, cu_seqlens, initial_state, final_state)
+    buf, arr, views = _conv_planes(parts, T, C, y, x.device)
+    st = LIB.gdn_short_conv1d_silu(_ptr(x), ldx, _ptr(weight), _ptr(cu_seqlens), N, T, C, K, _ptr(initial_state),
+                                   _ptr(final_state), _ptr(buf), arr, len(arr), _stream(stream))
+    _check("gdn_short_conv1d_silu", st)
+    return (views[0] if parts is None else views), final_state
+
+
+def gdn_short_conv1d_silu_decode(x, weight, conv_state, parts=None, y=None, stream=None):
+    """One token per sequence: x bf16 [B, C]; conv_state bf16 [B, K - 1, C] shifted in place.
+    Returns y [B, C] (or the list of plane views)."""
+    B, C, ldx = _conv_rows(x)
+    K = weight.shape[1]
+    _contig(weight, conv_state)
+    buf, arr, views = _conv_planes(parts, B, C, y, x.device)
+    st = LIB.gdn_short_conv1d_silu_decode(_ptr(x), ldx, _ptr(weight), B, C, K, _ptr(conv_state), _ptr(buf), arr,
+                                          len(arr), _stream(stream))
+    _check("gdn_short_conv1d_silu_decode", st)
+    return views[0] if parts is None else views
 
 
 def gdn_get_device_status(stream=None) -> int:

@@ -220,4 +220,99 @@ gdn_status nvfp4_gemm_colscale(const uint8_t *aq, const uint8_t *as, const uint8
     return launched(gdn::launch_nvfp4_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+
+// Checks and fills the plane layout of a short-convolution output.
+bool conv_planes(const int32_t *part_widths, int32_t n_parts, int32_t C, gdn::ConvArgs &a) {
+    a.n_parts = 1;
+    for (int p = 0; p < 4; ++p) a.part_end[p] = C;
+    if (n_parts <= 1) return n_parts >= 0 && (n_parts == 0 || !part_widths || part_widths[0] == C);
+    if (n_parts > 4 || !part_widths) return false;
+    int64_t end = 0;
+    for (int p = 0; p < n_parts; ++p) {
+        if (part_widths[p] <= 0 || part_widths[p] % 8 != 0) return false;
+        end += part_widths[p];
+        a.part_end[p] = (int32_t)(end > C ? C : end);
+    }
+    a.n_parts = n_parts;
+    return end == C;
+}
+
+bool conv_common_ok(const void *x, int64_t ldx, const float *weight, int32_t C, int32_t K, const void *y) {
+    return K >= 1 && K <= 4 && C > 0 && C % 8 == 0 && ldx >= C && ldx % 8 == 0 && x && weight && y &&
+           aligned16(x) && aligned16(weight) && aligned16(y);
+}
+
+// [p0, p0 + n0) and [p1, p1 + n1) (bytes) overlap
+bool overlaps(const void *p0, size_t n0, const void *p1, size_t n1) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p0), b = reinterpret_cast<uintptr_t>(p1);
+    return n0 && n1 && a < b + n1 && b < a + n0;
+}
+
+}  // namespace
+
+gdn_status gdn_short_conv1d_silu(const void *x, int64_t ldx, const float *weight, const int32_t *cu_seqlens,
+                                 int32_t num_seqs, int32_t T, int32_t C, int32_t K, const void *initial_state,
+                                 void *final_state, void *y, const int32_t *part_widths, int32_t n_parts,
+                                 gdn_stream_t stream) {
+    if (T < 0 || num_seqs < 1 || K < 1 || C < 0) return GDN_ERR_INVALID_ARG;
+    if (K > 4) return GDN_ERR_UNSUPPORTED;
+    if (!cu_seqlens && T % num_seqs != 0) return GDN_ERR_INVALID_ARG;
+    if (C == 0) return GDN_OK;
+    if (C % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    gdn::ConvArgs a{};
+    if (!conv_planes(part_widths, n_parts, C, a)) return GDN_ERR_INVALID_ARG;
+    if (T > 0 && !conv_common_ok(x, ldx, weight, C, K, y)) return GDN_ERR_INVALID_ARG;
+    if (T == 0 && (ldx < C || !weight)) return GDN_ERR_INVALID_ARG;
+    const size_t state_bytes = (size_t)num_seqs * (K - 1) * C * 2;
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return GDN_ERR_INVALID_ARG;
+    if (final_state && (overlaps(final_state, state_bytes, x, (size_t)T * ldx * 2) ||
+                        overlaps(final_state, state_bytes, y, (size_t)T * C * 2)))
+        return GDN_ERR_INVALID_ARG;
+    if (T == 0 && (!final_state || K == 1)) return GDN_OK;
+    a.x = x;
+    a.ldx = ldx;
+    a.w = weight;
+    a.cu_seqlens = cu_seqlens;
+    a.tokens_per_seq = cu_seqlens ? 0 : T / num_seqs;
+    a.num_seqs = num_seqs;
+    a.T = T;
+    a.C = C;
+    a.K = K;
+    a.init_state = initial_state;
+    a.final_state = K > 1 ? final_state : nullptr;
+    a.y = y;
+    a.decode = false;
+    return launched(gdn::launch_short_conv(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gdn_status gdn_short_conv1d_silu_decode(const void *x, int64_t ldx, const float *weight, int32_t B, int32_t C,
+                                        int32_t K, void *conv_state, void *y, const int32_t *part_widths,
+                                        int32_t n_parts, gdn_stream_t stream) {
+    if (B < 0 || K < 1 || C < 0) return GDN_ERR_INVALID_ARG;
+    if (K > 4) return GDN_ERR_UNSUPPORTED;
+    if (B == 0 || C == 0) return GDN_OK;
+    if (C % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    gdn::ConvArgs a{};
+    if (!conv_planes(part_widths, n_parts, C, a)) return GDN_ERR_INVALID_ARG;
+    if (!conv_common_ok(x, ldx, weight, C, K, y)) return GDN_ERR_INVALID_ARG;
+    const size_t state_bytes = (size_t)B * (K - 1) * C * 2;
+    if (K > 1 && (!conv_state || !aligned16(conv_state))) return GDN_ERR_INVALID_ARG;
+    if (K > 1 && (overlaps(conv_state, state_bytes, x, (size_t)B * ldx * 2) ||
+                  overlaps(conv_state, state_bytes, y, (size_t)B * C * 2)))
+        return GDN_ERR_INVALID_ARG;
+    a.x = x;
+    a.ldx = ldx;
+    a.w = weight;
+    a.num_seqs = B;
+    a.T = B;
+    a.C = C;
+    a.K = K;
+    a.final_state = conv_state;
+    a.y = y;
+    a.decode = true;
+    return launched(gdn::launch_short_conv(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

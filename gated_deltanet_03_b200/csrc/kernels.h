@@ -91,4 +91,19 @@ struct GemmArgs {
 };
 cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st);
 
+struct ConvArgs {
+    const void *x;               // bf16 rows of ldx elements; channels [0, C) are convolved
+    int64_t ldx;
+    const float *w;              // [C, K]
+    const int32_t *cu_seqlens;   // device [num_seqs + 1], or null: num_seqs runs of tokens_per_seq
+    int32_t tokens_per_seq, num_seqs, T, C, K;
+    const void *init_state;      // bf16 [num_seqs, K - 1, C] or null (zero history)
+    void *final_state;           // bf16 [num_seqs, K - 1, C] or null; decode: the state, in place
+    void *y;                     // bf16, planes of [T, width] (one plane: [T, C])
+    int32_t part_end[4];
+    int32_t n_parts;
+    bool decode;                 // one token per sequence, state shifted in place
+};
+cudaError_t launch_short_conv(const ConvArgs &a, cudaStream_t st);
+
 }  // namespace gdn

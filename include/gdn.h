@@ -15,6 +15,10 @@
  *          "Pinned graph semantics", steps 1-6: per value head of 128, RMSNorm with one
  *          shared F32 weight, times SiLU(z), flattened head-major, then the output
  *          projection (here NVFP4 W4A4 instead of Q4_K).
+ *   [WALK] "A Node-by-Node White-Box Walkthrough of a Quantized Hybrid Gated DeltaNet Language
+ *          Model", Principais Contribuicoes, items 2 and 3: the short convolutions on the
+ *          layer's path and their window. The page gives no formula; the reading here is the
+ *          depthwise causal convolution of width K <= 4 without bias, followed by SiLU.
  *
  * Conventions for every entry point:
  *   - All pointers are DEVICE pointers owned by the caller, row-major and contiguous,
@@ -204,6 +208,44 @@ GDN_API gdn_status nvfp4_gemm(const uint8_t *aq, const uint8_t *as, const uint8_
 GDN_API gdn_status nvfp4_gemm_colscale(const uint8_t *aq, const uint8_t *as, const uint8_t *bq,
                                        const uint8_t *bs, const float *col_alpha, int32_t M, int32_t N,
                                        int32_t K, gdn_dtype out_dtype, void *y, gdn_stream_t stream);
+
+/* ------------------------------------------------------ short convolution ----
+ * [WALK]: the causal short convolution + SiLU on the layer's q, k, v channels before the scan:
+ *   y[t, c] = SiLU(sum_{j<K} weight[c, j] x[t - (K - 1) + j, c])
+ * per sequence; the inputs before a sequence's first token are its carried state (the last
+ * K - 1 inputs of what came before, oldest first) or zero.
+ *
+ * x           bf16 [T, ldx] (ldx >= C, ldx % 8 == 0): channels [0, C) of each row are used, so
+ *             x can be the q|k|v columns of a wider projection output in place
+ * weight      fp32 [C, K], K contiguous
+ * cu_seqlens  device int32 [num_seqs + 1] as for gdn_prefill_chunked (non-decreasing,
+ *             cu_seqlens[0] = 0, cu_seqlens[num_seqs] = T; empty sequences allowed), or NULL:
+ *             num_seqs sequences of T / num_seqs tokens each (T % num_seqs == 0)
+ * initial_state  bf16 [num_seqs, K - 1, C], or NULL (zero history)
+ * final_state    bf16 [num_seqs, K - 1, C] output, or NULL: each sequence's last K - 1
+ *             inputs (continuing initial_state when the sequence is shorter than K - 1). May
+ *             alias initial_state; must not overlap x or y.
+ * y           bf16, the output as n_parts planes: with part_widths = {w_0, w_1, ...} (host
+ *             array, each a multiple of 8, summing to C) plane p holds channels
+ *             [w_0 + .. + w_{p-1}, .. + w_p) as a contiguous [T, w_p] block, the planes one
+ *             after another (n_parts = 3 and widths {Hk*Dk, Hk*Dk, Hv*Dv} give q, k and v as
+ *             gdn_prefill_chunked reads them). n_parts 0 or 1 (part_widths NULL): y is [T, C].
+ * Supported: 1 <= K <= 4; C % 8 == 0; n_parts <= 4. A malformed cu_seqlens gives undefined
+ * values but no out-of-bounds access of cu_seqlens. */
+GDN_API gdn_status gdn_short_conv1d_silu(const void *x, int64_t ldx, const float *weight,
+                                         const int32_t *cu_seqlens, int32_t num_seqs, int32_t T,
+                                         int32_t C, int32_t K, const void *initial_state,
+                                         void *final_state, void *y, const int32_t *part_widths,
+                                         int32_t n_parts, gdn_stream_t stream);
+
+/* One decode token per sequence: x bf16 [B, ldx] (channels [0, C) used), conv_state bf16
+ * [B, K - 1, C] read and then shifted by one token in place (it ends as the last K - 1 inputs,
+ * x included), y as for gdn_short_conv1d_silu with T = B. conv_state must not overlap x or y.
+ * Continuing a prefill whose final_state was written gives the same y as one longer prefill. */
+GDN_API gdn_status gdn_short_conv1d_silu_decode(const void *x, int64_t ldx, const float *weight,
+                                                int32_t B, int32_t C, int32_t K, void *conv_state,
+                                                void *y, const int32_t *part_widths, int32_t n_parts,
+                                                gdn_stream_t stream);
 
 /* ------------------------------------------------- allocation-free prefill ----
  * No counterpart in the paper. For callers that cannot allocate device memory - code that

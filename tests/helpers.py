@@ -14,6 +14,11 @@ TOL_SCAN_BF16_OUT = 2e-3 + 2.0 ** -8
 # Gated RMSNorm in fp32 arithmetic (rsqrt, expf: a few ulp): 1e-5; bf16 output adds 2^-8.
 TOL_TAIL = 1e-5
 TOL_TAIL_BF16_OUT = 1e-5 + 2.0 ** -8
+# Short convolution + SiLU, element by element: bf16 storage rounding of y (half an ulp, 2^-9
+# relative) plus the fp32 sum of K products and the approximate exponential and reciprocal
+# (about 1e-6 relative of the pre-activation): |got - ref| <= 2^-8 |ref| + 1e-5.
+TOL_CONV_RTOL = 2.0 ** -8
+TOL_CONV_ATOL = 1e-5
 # NVFP4 GEMM against the fp64 product of the dequantised operands: the stated 1e-2.
 TOL_GEMM = 1e-2
 

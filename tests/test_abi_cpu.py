@@ -71,3 +71,38 @@ def test_host_validation_rejects_bad_arguments_without_cuda():
 def test_workspace_query_is_host_only():
     import gated_deltanet_03_b200 as g
     assert g.gdn_prefill_workspace_bytes(4096, 1, 16, 16, 128, 128) >= 0
+
+
+def test_short_conv_host_validation():
+    """Every case is rejected (or is a no-op) on the host, so nothing is launched; the fake
+    addresses are never dereferenced."""
+    import gated_deltanet_03_b200 as g
+    L = g.LIB
+    P = None
+    X, W, Y, S = 0x10000, 0x20000, 0x30000, 0x40000
+    parts3 = (ctypes.c_int32 * 3)(64, 64, 128)
+    bad_sum = (ctypes.c_int32 * 3)(64, 64, 120)
+    bad_mult = (ctypes.c_int32 * 3)(60, 68, 128)
+    # width 5 is beyond the supported 1..4; channels not a multiple of 8
+    assert L.gdn_short_conv1d_silu(X, 256, W, P, 1, 8, 256, 5, P, P, Y, P, 0, P) == g.GDN_ERR_UNSUPPORTED
+    assert L.gdn_short_conv1d_silu(X, 256, W, P, 1, 8, 252, 4, P, P, Y, P, 0, P) == g.GDN_ERR_UNSUPPORTED
+    # tokens not divisible into num_seqs equal runs without cu_seqlens; ldx < C; null output
+    assert L.gdn_short_conv1d_silu(X, 256, W, P, 3, 8, 256, 4, P, P, Y, P, 0, P) == g.GDN_ERR_INVALID_ARG
+    assert L.gdn_short_conv1d_silu(X, 128, W, P, 1, 8, 256, 4, P, P, Y, P, 0, P) == g.GDN_ERR_INVALID_ARG
+    assert L.gdn_short_conv1d_silu(X, 256, W, P, 1, 8, 256, 4, P, P, P, P, 0, P) == g.GDN_ERR_INVALID_ARG
+    # plane widths that do not sum to C or are not multiples of 8; too many planes
+    assert L.gdn_short_conv1d_silu(X, 256, W, P, 1, 8, 256, 4, P, P, Y, bad_sum, 3, P) == g.GDN_ERR_INVALID_ARG
+    assert L.gdn_short_conv1d_silu(X, 256, W, P, 1, 8, 256, 4, P, P, Y, bad_mult, 3, P) == g.GDN_ERR_INVALID_ARG
+    assert L.gdn_short_conv1d_silu(X, 256, W, P, 1, 8, 256, 4, P, P, Y, parts3, 5, P) == g.GDN_ERR_INVALID_ARG
+    # misaligned input; final state overlapping the input or the output
+    assert L.gdn_short_conv1d_silu(X + 2, 256, W, P, 1, 8, 256, 4, P, P, Y, P, 0, P) == g.GDN_ERR_INVALID_ARG
+    assert L.gdn_short_conv1d_silu(X, 256, W, P, 1, 8, 256, 4, P, X + 1024, Y, P, 0, P) == g.GDN_ERR_INVALID_ARG
+    assert L.gdn_short_conv1d_silu(X, 256, W, P, 1, 8, 256, 4, P, Y, Y, parts3, 3, P) == g.GDN_ERR_INVALID_ARG
+    # nothing to do: no tokens and no state requested; width 1 has no state
+    assert L.gdn_short_conv1d_silu(P, 256, W, P, 1, 0, 256, 4, P, P, P, P, 0, P) == g.GDN_OK
+    assert L.gdn_short_conv1d_silu(P, 256, W, P, 1, 0, 256, 1, P, S, P, P, 0, P) == g.GDN_OK
+    # decode: missing or overlapping state, unsupported width, empty batch
+    assert L.gdn_short_conv1d_silu_decode(X, 256, W, 4, 256, 4, P, Y, P, 0, P) == g.GDN_ERR_INVALID_ARG
+    assert L.gdn_short_conv1d_silu_decode(X, 256, W, 4, 256, 4, Y, Y, P, 0, P) == g.GDN_ERR_INVALID_ARG
+    assert L.gdn_short_conv1d_silu_decode(X, 256, W, 4, 256, 5, S, Y, P, 0, P) == g.GDN_ERR_UNSUPPORTED
+    assert L.gdn_short_conv1d_silu_decode(X, 256, W, 0, 256, 4, S, Y, P, 0, P) == g.GDN_OK

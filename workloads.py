@@ -10,7 +10,8 @@ flattened to 2048/4096 and projected to 1024/2048; d_model 1024 with 16+16 heads
   q, k, v, z ~ N(0, 1); a, b ~ N(0, 1); A_log ~ U(log 1, log 16); dt_bias = 0;
   norm weight ~ U(0.5, 1.5); projection weight ~ N(0, 0.02) (standard deviation);
   initial states, where non-zero, ~ N(0, 0.1) (standard deviation).
-Variable-length lengths are log-uniform in [1024, 65536], seeded.
+Variable-length lengths are log-uniform in [1024, 65536], seeded. Short convolution: x ~ N(0, 1),
+weight ~ N(0, 1/K), carried history ~ N(0, 1).
 """
 from __future__ import annotations
 
@@ -132,3 +133,14 @@ def activations(M: int, K: int, seed: int, std: float = 1.0, heavy_tail: bool = 
         xb[pick] = 0.0
         x = xb.reshape(M, K)
     return round_bf16(x) if bf16 else x
+
+
+def conv_inputs(T: int, C: int, K: int, seed: int, num_seqs: int = 1, state: bool = False) -> dict:
+    """Inputs of the causal short convolution: x [T, C] ~ N(0, 1) (bf16-rounded), weight [C, K]
+    ~ N(0, 1/K) fp32 (so the pre-activation is about unit scale), and, with state, a carried
+    input history [num_seqs, K - 1, C] ~ N(0, 1) (bf16-rounded)."""
+    rng = np.random.default_rng(seed)
+    out = {"x": round_bf16(_normal(rng, (T, C))),
+           "weight": _normal(rng, (C, K), 1.0 / math.sqrt(K))}
+    out["initial_state"] = round_bf16(_normal(rng, (num_seqs, K - 1, C))) if state else None
+    return out
