@@ -94,8 +94,6 @@ GDN_DEV float group_sum(float v) {
 // softplus(x) = log(1 + e^x), stable for large x; library expf / log1pf.
 GDN_DEV float softplus_f(float x) { return x > 20.0f ? x : log1pf(expf(x)); }
 GDN_DEV float sigmoid_f(float x) { return 1.0f / (1.0f + expf(-x)); }
-// z * sigmoid(z) with the fast exponential and division intrinsics (a few ulp; the tail's
-// tolerance is 1e-5 relative): the gated tail runs this once per element.
 // 2^x with the hardware approximation (relative error about 2^-22; results below the smallest
 // normal float are flushed to zero), and e^x through it.
 GDN_DEV float exp2_approx(float x) {
@@ -106,6 +104,8 @@ GDN_DEV float exp2_approx(float x) {
 constexpr float kLog2e = 1.4426950408889634f;
 GDN_DEV float exp_approx(float x) { return exp2_approx(x * kLog2e); }
 
+// z * sigmoid(z) with the fast exponential and division intrinsics (a few ulp; the tail's
+// tolerance is 1e-5 relative).
 GDN_DEV float silu_fast(float z) { return __fdividef(z, 1.0f + exp_approx(-z)); }
 
 // log of the decay gate, g = -exp(A_log) * softplus(a + dt_bias), and the write strength.
