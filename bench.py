@@ -392,6 +392,37 @@ def run_gpu(args):
     state_bytes = dstate.numel() * 4
     dec_bytes = 2 * state_bytes + sum(t.numel() * t.element_size() for t in (dq, dk, dv, da, db, dout))
 
+    # multi-token decode on the batched-decode workload's shape: verify 4 draft tokens per sequence
+    # (state read once), then commit a seeded number of accepted tokens (state read and written once)
+    mT = 4
+    mw = workloads.custom("verify_B%d_T%d" % (dw.num_seqs, mT), (mT,) * dw.num_seqs, dw.Hk, dw.Hv, dw.D,
+                          s0_std=0.1, seed=dw.seed)
+    mx = workloads.generate(mw)
+    mB = dw.num_seqs
+    mq = up(mx["q"], bf).view(mB, mT, dw.Hk, dw.D)
+    mk = up(mx["k"], bf).view(mB, mT, dw.Hk, dw.D)
+    mv = up(mx["v"], bf).view(mB, mT, dw.Hv, dw.D)
+    ma, mb = up(mx["a"], f32).view(mB, mT, dw.Hv), up(mx["b"], f32).view(mB, mT, dw.Hv)
+    mA, mdt = up(mx["A_log"], f32), up(mx["dt_bias"], f32)
+    mstate = up(mx["initial_state"], f32)
+    mo = torch.empty((mB, mT, dw.Hv, dw.D), dtype=bf, device=dev)
+    macc = torch.from_numpy(np.random.default_rng(dw.seed).integers(0, mT + 1, size=mB).astype(np.int32)).to(dev)
+    ver_graph = graph_of(lambda: g.gdn_decode_verify(mq, mk, mv, ma, mb, mA, mdt, mstate, o=mo))
+    com_graph = graph_of(lambda: g.gdn_decode_commit(mq, mk, mv, ma, mb, mA, mdt, mstate, macc))
+    for _ in range(max(3, args.warmup)):
+        ver_graph.replay()
+        com_graph.replay()
+    torch.cuda.synchronize()
+    ver_ev, com_ev = timed(ver_graph, max(args.steps, 10)), timed(com_graph, max(args.steps, 10))
+    torch.cuda.synchronize()
+    ver_ms = statistics.mean(a.elapsed_time(b) for a, b in ver_ev)
+    com_ms = statistics.mean(a.elapsed_time(b) for a, b in com_ev)
+    m_tok = sum(t.numel() * t.element_size() for t in (mq, mk, mv, ma, mb))
+    ver_bytes = mstate.numel() * 4 + m_tok + mo.numel() * mo.element_size()
+    com_bytes = 2 * mstate.numel() * 4 + m_tok
+    assert g.gdn_get_device_status() == 0
+    del mstate
+
     # short convolution decode on the batched-decode workload's q|k|v channels (state in place)
     dC = 2 * dw.Hk * dw.D + dw.Hv * dw.D
     dcx = workloads.conv_inputs(dw.num_seqs, dC, 4, seed=dw.seed, num_seqs=dw.num_seqs, state=True)
@@ -456,6 +487,14 @@ def run_gpu(args):
         "decode": {"workload": dw.name, "ms": dec, "GB/s": dec_bytes / (dec / 1e3) / 1e9,
                    "frac": dec_bytes / (dec / 1e3) / 1e9 / float(pk["hbm_gbs"]),
                    "bytes": dec_bytes, "peak_gbs": float(pk["hbm_gbs"]), "peak_kind": pk_kind},
+        "decode_multi": {"workload": "%s shape, %d draft tokens per sequence" % (dw.name, mT),
+                         "verify_ms": ver_ms, "verify_GB/s": ver_bytes / (ver_ms / 1e3) / 1e9,
+                         "verify_frac": ver_bytes / (ver_ms / 1e3) / 1e9 / float(pk["hbm_gbs"]),
+                         "commit_ms": com_ms, "commit_GB/s": com_bytes / (com_ms / 1e3) / 1e9,
+                         "commit_frac": com_bytes / (com_ms / 1e3) / 1e9 / float(pk["hbm_gbs"]),
+                         "bytes": {"verify": ver_bytes, "commit": com_bytes},
+                         "single_steps_ms": mT * dec,
+                         "timing": "CUDA graph replay, L2 flushed before each; commit of a seeded 0..4 accepted tokens"},
         "short_conv": {"workload": "%s q|k|v channels (T = %d, C = %d, K = 4), planes q, k, v" % (w.name, T, conv_C),
                        "ms": statistics.mean(parts["conv"]),
                        "GB/s": conv_bytes / (statistics.mean(parts["conv"]) / 1e3) / 1e9,

@@ -5,7 +5,8 @@ PyTorch provides device memory (output tensors are allocated with torch) and the
 stream. There is no CPU fallback: if the library is missing, importing this package raises.
 
 Functions keep the C names:
-  gdn_prefill_chunked, gdn_prefill_chunked_gated_nvfp4, gdn_decode_step, gdn_gated_rmsnorm_silu,
+  gdn_prefill_chunked, gdn_prefill_chunked_gated_nvfp4, gdn_decode_step, gdn_decode_verify,
+  gdn_decode_commit, gdn_gated_rmsnorm_silu,
   gdn_gated_rmsnorm_silu_nvfp4, nvfp4_quantize_act, nvfp4_gemm,
   nvfp4_gemm_colscale, gdn_short_conv1d_silu, gdn_short_conv1d_silu_decode,
   gdn_prefill_workspace_bytes, gdn_get_device_status.
@@ -26,6 +27,7 @@ GDN_BF16, GDN_F32 = 0, 1
 # Exported C symbols, in the order include/gdn.h declares them.
 ABI_SYMBOLS = (
     "gdn_prefill_chunked", "gdn_prefill_workspace_bytes", "gdn_prefill_chunked_gated_nvfp4", "gdn_decode_step",
+    "gdn_decode_verify", "gdn_decode_commit",
     "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act",
     "nvfp4_gemm", "nvfp4_gemm_colscale", "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode",
     "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_status_string",
@@ -53,6 +55,9 @@ def _load() -> ctypes.CDLL:
     lib.gdn_prefill_workspace_bytes.restype = sz
     lib.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, P, P,
                                     i32, P]
+    lib.gdn_decode_verify.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P, P, P,
+                                      i32, P]
+    lib.gdn_decode_commit.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P, P, P]
     lib.gdn_gated_rmsnorm_silu.argtypes = [P, P, P, f32, i32, i32, i32, i32, P, i32, P]
     lib.gdn_gated_rmsnorm_silu_nvfp4.argtypes = [P, P, P, f32, i32, i32, i32, i32, f32, P, P, P]
     lib.nvfp4_quantize_act.argtypes = [P, i32, i32, i32, f32, P, P, P]
@@ -67,7 +72,8 @@ def _load() -> ctypes.CDLL:
     lib.gdn_status_string.argtypes = [i32]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_version.restype = i32
-    for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_gated_nvfp4", "gdn_prefill_chunked_static_ws", "gdn_decode_step", "gdn_gated_rmsnorm_silu",
+    for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_gated_nvfp4", "gdn_prefill_chunked_static_ws", "gdn_decode_step", "gdn_decode_verify",
+                 "gdn_decode_commit", "gdn_gated_rmsnorm_silu",
                  "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_gemm_colscale",
                  "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode", "gdn_get_device_status"):
         getattr(lib, name).restype = ctypes.c_int
@@ -190,6 +196,40 @@ def gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1.0,
                              _ptr(state), _ptr(o), _dt(o), _stream(stream))
     _check("gdn_decode_step", st)
     return o
+
+
+def gdn_decode_verify(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1.0, qk_l2norm: bool = True,
+                      final_state=None, out_dtype=None, o=None, stream=None):
+    """T draft tokens per sequence: q, k [B, T, Hk, D], v [B, T, Hv, D], a, b [B, T, Hv];
+    `state` [B, Hv, D, D] fp32 is only read. Returns o [B, T, Hv, D] (final_state, if given,
+    receives the state after all T tokens)."""
+    B, T, Hk, Dk = q.shape
+    Hv, Dv = v.shape[2], v.shape[3]
+    out_dtype = out_dtype or q.dtype
+    if o is None:
+        o = torch.empty((B, T, Hv, Dv), dtype=out_dtype, device=q.device)
+    _contig(q, k, v, a, b, A_log, dt_bias, state, final_state, o)
+    st = LIB.gdn_decode_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
+                               B, T, Hk, Hv, Dk, Dv, float(scale), int(bool(qk_l2norm)), _dt(q), _ptr(state),
+                               _ptr(final_state), _ptr(o), _dt(o), _stream(stream))
+    _check("gdn_decode_verify", st)
+    return o
+
+
+def gdn_decode_commit(q, k, v, a, b, A_log, dt_bias, state, accepted, scale: float = 1.0,
+                      qk_l2norm: bool = True, stream=None):
+    """Advance `state` in place by the first accepted[b] (device int32 [B]) of each sequence's
+    T draft tokens (the same tensors as the gdn_decode_verify call)."""
+    B, T, Hk, Dk = q.shape
+    Hv, Dv = v.shape[2], v.shape[3]
+    _contig(q, k, v, a, b, A_log, dt_bias, state, accepted)
+    if accepted.dtype != torch.int32:
+        raise TypeError("accepted must be int32")
+    st = LIB.gdn_decode_commit(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
+                               B, T, Hk, Hv, Dk, Dv, float(scale), int(bool(qk_l2norm)), _dt(q), _ptr(accepted),
+                               _ptr(state), _stream(stream))
+    _check("gdn_decode_commit", st)
+    return state
 
 
 def gdn_gated_rmsnorm_silu(o, z, weight, eps: float = 1e-6, out_dtype=None, y=None, stream=None):

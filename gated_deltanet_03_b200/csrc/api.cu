@@ -1,6 +1,7 @@
 // C entry points declared in include/gdn.h: host-side argument checks, kernel variant
 // selection and launches on the caller's stream. No device memory is allocated here; the
 // only library-owned device object is the status word that bounded waits report into.
+#include <climits>
 #include <cstdio>
 
 #include "common.cuh"
@@ -147,6 +148,45 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const fl
         return GDN_ERR_INVALID_ARG;
     gdn::RecurrentArgs r{q, k, v, a, b, A_log, dt_bias, nullptr, 1, B, Hk, Hv, Dk, scale, qk_l2norm,
                          in_dtype == GDN_BF16, out_dtype == GDN_BF16, state, state, o};
+    return launched(gdn::launch_recurrent(r, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static gdn_status multi_check(const void *q, const void *k, const void *v, const float *a, const float *b,
+                              const float *A_log, const float *dt_bias, int32_t B, int32_t T, int32_t Hk, int32_t Hv,
+                              int32_t Dk, int32_t Dv, gdn_dtype in_dtype) {
+    if (B < 0 || T < 1 || Hk < 1 || Hv < 1 || Hv % Hk != 0 || !dtype_ok(in_dtype)) return GDN_ERR_INVALID_ARG;
+    if (Dk != Dv || !head_ok(Dk)) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)B * T > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !A_log || !dt_bias) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+gdn_status gdn_decode_verify(const void *q, const void *k, const void *v, const float *a, const float *b,
+                             const float *A_log, const float *dt_bias, int32_t B, int32_t T, int32_t Hk, int32_t Hv,
+                             int32_t Dk, int32_t Dv, float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                             const float *state, float *final_state, void *o, gdn_dtype out_dtype,
+                             gdn_stream_t stream) {
+    const gdn_status c = multi_check(q, k, v, a, b, A_log, dt_bias, B, T, Hk, Hv, Dk, Dv, in_dtype);
+    if (c != GDN_OK || B == 0) return c;
+    if (!dtype_ok(out_dtype) || !state || !o || !aligned16(state) || !aligned16(o) ||
+        (final_state && !aligned16(final_state)))
+        return GDN_ERR_INVALID_ARG;
+    gdn::RecurrentArgs r{q, k, v, a, b, A_log, dt_bias, nullptr, T, B, Hk, Hv, Dk, scale, qk_l2norm,
+                         in_dtype == GDN_BF16, out_dtype == GDN_BF16, state, final_state, o, nullptr};
+    return launched(gdn::launch_recurrent(r, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gdn_status gdn_decode_commit(const void *q, const void *k, const void *v, const float *a, const float *b,
+                             const float *A_log, const float *dt_bias, int32_t B, int32_t T, int32_t Hk, int32_t Hv,
+                             int32_t Dk, int32_t Dv, float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                             const int32_t *accepted, float *state, gdn_stream_t stream) {
+    const gdn_status c = multi_check(q, k, v, a, b, A_log, dt_bias, B, T, Hk, Hv, Dk, Dv, in_dtype);
+    if (c != GDN_OK || B == 0) return c;
+    if (!accepted || !state || !aligned16(state)) return GDN_ERR_INVALID_ARG;
+    gdn::RecurrentArgs r{q, k, v, a, b, A_log, dt_bias, nullptr, T, B, Hk, Hv, Dk, scale, qk_l2norm,
+                         in_dtype == GDN_BF16, true, state, state, nullptr, accepted};
     return launched(gdn::launch_recurrent(r, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -37,7 +37,8 @@ struct RecurrentArgs {
     bool in_bf16, out_bf16;
     const float *S0;             // may be null (zero state); may alias S_out
     float *S_out;                // may be null
-    void *o;
+    void *o;                     // may be null (no outputs)
+    const int32_t *n_apply;      // device [num_seqs] or null: sequence n takes only its first n_apply[n] tokens
 };
 cudaError_t launch_recurrent(const RecurrentArgs &r, cudaStream_t st);
 

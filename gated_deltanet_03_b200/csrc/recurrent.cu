@@ -7,10 +7,11 @@
 //     alpha = exp(-exp(A_log) softplus(a + dt_bias)),  beta = sigmoid(b),
 //     S <- alpha S (I - beta k k^T) + beta v k^T = alpha S + beta (v - alpha S k) k^T,
 //     o = S q.
-// The rows of S (value index i) evolve independently, so a CTA owns R rows of one
-// (sequence, value head) state and keeps them in registers across the sequence; each
-// row is spread over D/4 lanes holding 4 key columns each (128-bit loads), and the two
-// row dot products (S k and S q) are lane-group shuffle reductions.
+// The rows of S (value index i) evolve independently, so a CTA owns rows of one (sequence,
+// value head) state and keeps them in registers across the sequence; each row is spread over
+// a group of lanes, and the two row dot products (S k and S q) are lane-group shuffle
+// reductions. Head size 128 has its own layout (below); smaller heads spread a row over D/4
+// lanes holding 4 key columns each.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -38,7 +39,7 @@ gdn_recurrent_kernel(const void *__restrict__ q, const void *__restrict__ k,
                      const float *__restrict__ b, const float *__restrict__ A_log,
                      const float *__restrict__ dt_bias, const int32_t *__restrict__ cu_seqlens,
                      int32_t tokens_per_seq, int32_t Hk, int32_t Hv, float scale, int32_t l2norm,
-                     const float *S0, float *S_out, void *__restrict__ o) {
+                     const float *S0, float *S_out, void *__restrict__ o, const int32_t *__restrict__ n_apply) {
     pdl_launch_dependents();
     pdl_wait();
     using Sh = RecurrentShape<D>;
@@ -57,6 +58,7 @@ gdn_recurrent_kernel(const void *__restrict__ q, const void *__restrict__ k,
         t0 = n * tokens_per_seq;
         t1 = t0 + tokens_per_seq;
     }
+    if (n_apply) t1 = t0 + min(max(n_apply[n], 0), t1 - t0);   // only the first n_apply[n] tokens
     const size_t sbase = ((size_t)n * Hv + h) * D * D;
 
     float s[PASSES][4];
@@ -108,7 +110,7 @@ gdn_recurrent_kernel(const void *__restrict__ q, const void *__restrict__ k,
         for (int p = 0; p < PASSES; ++p) op[p] = dot4(s[p], qq);
 #pragma unroll
         for (int p = 0; p < PASSES; ++p) op[p] = group_sum<LANES>(op[p]);
-        if ((tid % LANES) == 0) {
+        if (o && (tid % LANES) == 0) {
 #pragma unroll
             for (int p = 0; p < PASSES; ++p) store1<OUT_BF16>(o, ((size_t)t * Hv + h) * D + row0 + p * RPB, op[p]);
         }
@@ -123,13 +125,168 @@ gdn_recurrent_kernel(const void *__restrict__ q, const void *__restrict__ k,
     }
 }
 
+// ---------------------------------------------------------------- d = 128 ----
+// A CTA of 128 threads owns 64 rows of one (sequence, value head) state: the 8 consecutive
+// lanes of a row group share 4 rows (slice*64 + tid/8 + 16 p, p < 4), and lane c of the group
+// holds key columns 32 j + 4 c + e (j, e < 4), so each of its four 16-byte state accesses per
+// row is part of one 128-byte run per row group. The arithmetic runs on packed f32 pairs; the
+// key norm is folded into the update's scalar (S k^ = kn (S k), and the rank-one write uses
+// u kn with the raw k); the gates of 32 tokens are computed once per warp, one per lane, and
+// broadcast per token.
+constexpr int kR128Threads = 128;
+constexpr unsigned kFull = 0xffffffffu;
+
+// Four per-thread values summed over the 8 lanes of a row group: after the exchange, lanes whose
+// bits 2 and 1 are (p >> 1, p & 1) hold the total of value p (4 shuffles instead of 12).
+GDN_DEV float group8_sum4_t(const float (&x)[4], int l8) {
+    const bool b2 = (l8 & 4) != 0, b1 = (l8 & 2) != 0;
+    const float r0 = __shfl_xor_sync(kFull, b2 ? x[0] : x[2], 4);
+    const float r1 = __shfl_xor_sync(kFull, b2 ? x[1] : x[3], 4);
+    const float k0 = (b2 ? x[2] : x[0]) + r0, k1 = (b2 ? x[3] : x[1]) + r1;
+    float v = (b1 ? k1 : k0) + __shfl_xor_sync(kFull, b1 ? k0 : k1, 2);
+    v += __shfl_xor_sync(kFull, v, 1);
+    return v;
+}
+
+// The 16 key-index values of lane c (columns 32 j + 4 c + e) of one 128-vector, as 8 pairs.
+template <bool BF16>
+GDN_DEV void load_cols16(const void *base, size_t row, int l8, f2_t (&x)[8]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const size_t idx = row + 32 * j + 4 * l8;
+        if constexpr (BF16) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(base) + idx);
+            x[2 * j] = bf16x2_to_f2(u.x);
+            x[2 * j + 1] = bf16x2_to_f2(u.y);
+        } else {
+            const float4 f = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(base) + idx);
+            x[2 * j] = f2(f.x, f.y);
+            x[2 * j + 1] = f2(f.z, f.w);
+        }
+    }
+}
+
+GDN_DEV float dot16(const f2_t (&a)[8], const f2_t (&b)[8]) {
+    f2_t acc = mul2(a[0], b[0]);
+#pragma unroll
+    for (int c = 1; c < 8; ++c) acc = fma2(a[c], b[c], acc);
+    return f2lo(acc) + f2hi(acc);
+}
+
+template <bool IN_BF16, bool OUT_BF16>
+__global__ void __launch_bounds__(kR128Threads)
+gdn_recurrent128_kernel(const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
+                        const float *__restrict__ a, const float *__restrict__ b, const float *__restrict__ A_log,
+                        const float *__restrict__ dt_bias, const int32_t *__restrict__ cu_seqlens,
+                        int32_t tokens_per_seq, int32_t Hk, int32_t Hv, float scale, int32_t l2norm,
+                        const float *S0, float *S_out, void *__restrict__ o, const int32_t *__restrict__ n_apply) {
+    pdl_launch_dependents();
+    pdl_wait();
+    constexpr int D = 128;
+    const int slice = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+    const int hk = h / (Hv / Hk);
+    const int tid = threadIdx.x, lane = tid & 31, l8 = tid & 7;
+    const int rbase = slice * 64 + (tid >> 3);
+    const int gbase = lane & ~7;
+
+    int t0, t1;
+    if (cu_seqlens) {
+        t0 = cu_seqlens[n];
+        t1 = cu_seqlens[n + 1];
+    } else {
+        t0 = n * tokens_per_seq;
+        t1 = t0 + tokens_per_seq;
+    }
+    if (n_apply) t1 = t0 + min(max(n_apply[n], 0), t1 - t0);   // only the first n_apply[n] tokens
+    const size_t sbase = ((size_t)n * Hv + h) * D * D;
+
+    f2_t s[4][8];
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (S0) x = __ldcs(reinterpret_cast<const float4 *>(S0 + sbase + (size_t)(rbase + 16 * p) * D + 32 * j + 4 * l8));
+            s[p][2 * j] = f2(x.x, x.y);
+            s[p][2 * j + 1] = f2(x.z, x.w);
+        }
+
+    const float Al = A_log[h], db = dt_bias[h];
+    float g_alpha = 0.0f, g_beta = 0.0f;   // gates of token (t - t0) / 32 * 32 + lane
+    for (int t = t0; t < t1; ++t) {
+        const int i = (t - t0) & 31;
+        if (i == 0) {
+            const int tt = t + lane;
+            if (tt < t1) {
+                float g;
+                gdn_gates(a[(size_t)tt * Hv + h], b[(size_t)tt * Hv + h], Al, db, g, g_beta);
+                g_alpha = expf(g);
+            }
+        }
+        const float alpha = __shfl_sync(kFull, g_alpha, i), beta = __shfl_sync(kFull, g_beta, i);
+        f2_t k2[8], q2[8];
+        load_cols16<IN_BF16>(k, ((size_t)t * Hk + hk) * D, l8, k2);
+        load_cols16<IN_BF16>(q, ((size_t)t * Hk + hk) * D, l8, q2);
+        float vv[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) vv[p] = load1<IN_BF16>(v, ((size_t)t * Hv + h) * D + rbase + 16 * p);
+
+        float kn = 1.0f, qn = scale;
+        if (l2norm) {
+            const float ks = group_sum<8>(dot16(k2, k2)), qs = group_sum<8>(dot16(q2, q2));
+            kn = rsqrtf(ks + 1e-6f);
+            qn = rsqrtf(qs + 1e-6f) * scale;
+        }
+        float part[4], sk[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) part[p] = dot16(s[p], k2);
+        const float skt = group8_sum4_t(part, l8);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) sk[p] = __shfl_sync(kFull, skt, gbase + 4 * (p >> 1) + 2 * (p & 1));
+        // S <- alpha S + beta (v - alpha S k^) k^T, k^ = kn k
+        const f2_t a2 = f2(alpha, alpha);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float u = beta * (vv[p] - alpha * kn * sk[p]) * kn;
+            const f2_t u2 = f2(u, u);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) s[p][c] = fma2(a2, s[p][c], mul2(u2, k2[c]));
+        }
+        // o = S q^, q^ = qn q (qn includes scale)
+#pragma unroll
+        for (int p = 0; p < 4; ++p) part[p] = dot16(s[p], q2);
+        const float ot = group8_sum4_t(part, l8);
+        if (o && (l8 & 1) == 0) {
+            const int p = 2 * ((l8 >> 2) & 1) + ((l8 >> 1) & 1);
+            store1<OUT_BF16>(o, ((size_t)t * Hv + h) * D + rbase + 16 * p, ot * qn);
+        }
+    }
+
+    if (S_out) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                __stcs(reinterpret_cast<float4 *>(S_out + sbase + (size_t)(rbase + 16 * p) * D + 32 * j + 4 * l8),
+                       make_float4(f2lo(s[p][2 * j]), f2hi(s[p][2 * j]), f2lo(s[p][2 * j + 1]), f2hi(s[p][2 * j + 1])));
+    }
+}
+
+template <bool IN_BF16, bool OUT_BF16>
+static cudaError_t launch_recurrent128_t(const RecurrentArgs &r, cudaStream_t st) {
+    dim3 grid(2, r.Hv, r.num_seqs);
+    return launch_pdl(gdn_recurrent128_kernel<IN_BF16, OUT_BF16>, grid, dim3(kR128Threads), 0, st, r.q, r.k, r.v,
+                      r.a, r.b, r.A_log, r.dt_bias, r.cu_seqlens, r.tokens_per_seq, r.Hk, r.Hv, r.scale, r.l2norm,
+                      r.S0, r.S_out, r.o, r.n_apply);
+}
+
 template <int D, bool IN_BF16, bool OUT_BF16>
 static cudaError_t launch_recurrent_t(const RecurrentArgs &r, cudaStream_t st) {
     using Sh = RecurrentShape<D>;
     dim3 grid(Sh::SLICES, r.Hv, r.num_seqs);
     return launch_pdl(gdn_recurrent_kernel<D, IN_BF16, OUT_BF16>, grid, dim3(Sh::NT), 0, st, r.q, r.k, r.v, r.a, r.b,
                       r.A_log, r.dt_bias, r.cu_seqlens, r.tokens_per_seq, r.Hk, r.Hv, r.scale, r.l2norm, r.S0,
-                      r.S_out, r.o);
+                      r.S_out, r.o, r.n_apply);
 }
 
 template <int D>
@@ -146,7 +303,11 @@ cudaError_t launch_recurrent(const RecurrentArgs &r, cudaStream_t st) {
         case 16: return launch_recurrent_d<16>(r, st);
         case 32: return launch_recurrent_d<32>(r, st);
         case 64: return launch_recurrent_d<64>(r, st);
-        case 128: return launch_recurrent_d<128>(r, st);
+        case 128:
+            if (r.in_bf16 && r.out_bf16) return launch_recurrent128_t<true, true>(r, st);
+            if (r.in_bf16) return launch_recurrent128_t<true, false>(r, st);
+            if (r.out_bf16) return launch_recurrent128_t<false, true>(r, st);
+            return launch_recurrent128_t<false, false>(r, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -151,6 +151,31 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
                            float *state, void *o, gdn_dtype out_dtype, gdn_stream_t stream);
 
+/* ------------------------------------------------ multi-token decode (verify) ----
+ * [GDN]: the same recurrence over T tokens per sequence (a draft of T tokens to check in one
+ * pass, e.g. speculative decoding), without changing the state: o for every draft token, the
+ * state read once. Sequence b's tokens are rows b*T .. b*T + T - 1 of q, k [B*T, Hk, Dk] and
+ * v, a, b, o [B*T, Hv, ...]; state [B, Hv, Dv, Dk] fp32 is read only. final_state: NULL, or
+ * [B, Hv, Dv, Dk] fp32 written with the state after all T tokens (may alias state: every
+ * CTA reads its rows before it writes them). Sizes and dtypes as gdn_decode_step; T >= 1.
+ * Equal to gdn_prefill_chunked over B sequences of T tokens from `state`. */
+GDN_API gdn_status gdn_decode_verify(const void *q, const void *k, const void *v, const float *a,
+                                     const float *b, const float *A_log, const float *dt_bias,
+                                     int32_t B, int32_t T, int32_t Hk, int32_t Hv, int32_t Dk,
+                                     int32_t Dv, float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                                     const float *state, float *final_state, void *o,
+                                     gdn_dtype out_dtype, gdn_stream_t stream);
+
+/* After gdn_decode_verify: advances each sequence's state, in place, by the first
+ * accepted[b] of its T draft tokens (device int32 [B]; values are clamped to [0, T]; 0
+ * leaves the state bit for bit unchanged). Same q, k, v, a, b as the verify call; no
+ * outputs are written. The state is read once and written once. */
+GDN_API gdn_status gdn_decode_commit(const void *q, const void *k, const void *v, const float *a,
+                                     const float *b, const float *A_log, const float *dt_bias,
+                                     int32_t B, int32_t T, int32_t Hk, int32_t Hv, int32_t Dk,
+                                     int32_t Dv, float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                                     const int32_t *accepted, float *state, gdn_stream_t stream);
+
 /* ------------------------------------------------------------ gated RMSNorm ----
  * [TAIL] steps 1-5: y[m, h*Dv + i] = o[m,h,i] / sqrt(mean_i o[m,h,:]^2 + eps) * w[i]
  *                                     * z[m,h,i] * sigmoid(z[m,h,i]).
