@@ -7,7 +7,7 @@ stream. There is no CPU fallback: if the library is missing, importing this pack
 Functions keep the C names:
   gdn_prefill_chunked, gdn_prefill_chunked_gated_nvfp4, gdn_decode_step, gdn_decode_verify,
   gdn_decode_commit, gdn_gated_rmsnorm_silu,
-  gdn_gated_rmsnorm_silu_nvfp4, nvfp4_quantize_act, nvfp4_gemm,
+  gdn_gated_rmsnorm_silu_nvfp4, nvfp4_quantize_act, nvfp4_dequantize_act, nvfp4_gemm,
   nvfp4_gemm_colscale, gdn_short_conv1d_silu, gdn_short_conv1d_silu_decode,
   gdn_prefill_workspace_bytes, gdn_get_device_status.
 """
@@ -28,7 +28,7 @@ GDN_BF16, GDN_F32 = 0, 1
 ABI_SYMBOLS = (
     "gdn_prefill_chunked", "gdn_prefill_workspace_bytes", "gdn_prefill_chunked_gated_nvfp4", "gdn_decode_step",
     "gdn_decode_verify", "gdn_decode_commit",
-    "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act",
+    "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_dequantize_act",
     "nvfp4_gemm", "nvfp4_gemm_colscale", "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode",
     "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_status_string",
     "gdn_version",
@@ -61,6 +61,7 @@ def _load() -> ctypes.CDLL:
     lib.gdn_gated_rmsnorm_silu.argtypes = [P, P, P, f32, i32, i32, i32, i32, P, i32, P]
     lib.gdn_gated_rmsnorm_silu_nvfp4.argtypes = [P, P, P, f32, i32, i32, i32, i32, f32, P, P, P]
     lib.nvfp4_quantize_act.argtypes = [P, i32, i32, i32, f32, P, P, P]
+    lib.nvfp4_dequantize_act.argtypes = [P, P, i32, i32, f32, i32, P, P]
     lib.nvfp4_gemm.argtypes = [P, P, P, P, f32, i32, i32, i32, i32, P, P]
     lib.nvfp4_gemm_colscale.argtypes = [P, P, P, P, P, i32, i32, i32, i32, P, P]
     i64 = ctypes.c_int64
@@ -74,7 +75,8 @@ def _load() -> ctypes.CDLL:
     lib.gdn_version.restype = i32
     for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_gated_nvfp4", "gdn_prefill_chunked_static_ws", "gdn_decode_step", "gdn_decode_verify",
                  "gdn_decode_commit", "gdn_gated_rmsnorm_silu",
-                 "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_gemm_colscale",
+                 "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_dequantize_act", "nvfp4_gemm",
+                 "nvfp4_gemm_colscale",
                  "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode", "gdn_get_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -273,6 +275,17 @@ def nvfp4_quantize_act(x, global_scale: float, xq=None, xs=None, stream=None):
                                 _stream(stream))
     _check("nvfp4_quantize_act", st)
     return xq, xs
+
+
+def nvfp4_dequantize_act(xq, xs, global_scale: float, out_dtype=torch.float32, y=None, stream=None):
+    """(xq [M, K/2], xs [M, K/16]) -> y [M, K] = E2M1 * E4M3 / global_scale."""
+    M, K = xq.shape[0], xq.shape[1] * 2
+    if y is None:
+        y = torch.empty((M, K), dtype=out_dtype, device=xq.device)
+    _contig(xq, xs, y)
+    st = LIB.nvfp4_dequantize_act(_ptr(xq), _ptr(xs), M, K, float(global_scale), _dt(y), _ptr(y), _stream(stream))
+    _check("nvfp4_dequantize_act", st)
+    return y
 
 
 def nvfp4_gemm(aq, as_, bq, bs, alpha: float, out_dtype=torch.bfloat16, y=None, stream=None):

@@ -235,6 +235,17 @@ gdn_status nvfp4_quantize_act(const void *x, gdn_dtype in_dtype, int32_t M, int3
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
+gdn_status nvfp4_dequantize_act(const uint8_t *xq, const uint8_t *xs, int32_t M, int32_t K, float global_scale,
+                                gdn_dtype out_dtype, void *y, gdn_stream_t stream) {
+    if (M < 0 || K < 0 || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
+    if (!(global_scale > 0.0f) || !(global_scale < 3.0e38f)) return GDN_ERR_INVALID_ARG;
+    if (K % 16 != 0) return GDN_ERR_UNSUPPORTED;
+    if (M == 0 || K == 0) return GDN_OK;
+    if (!xq || !xs || !y || (reinterpret_cast<uintptr_t>(xq) & 7u) || !aligned16(y)) return GDN_ERR_INVALID_ARG;
+    return launched(gdn::launch_nvfp4_dequantize(xq, xs, M, K, global_scale, out_dtype == GDN_BF16, y,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
 gdn_status nvfp4_gemm(const uint8_t *aq, const uint8_t *as, const uint8_t *bq, const uint8_t *bs, float alpha,
                       int32_t M, int32_t N, int32_t K, gdn_dtype out_dtype, void *y, gdn_stream_t stream) {
     if (M < 0 || N < 0 || K < 0 || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;

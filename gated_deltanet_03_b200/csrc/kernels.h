@@ -80,6 +80,8 @@ cudaError_t launch_gated_rmsnorm_nvfp4(const TailArgs &t, cudaStream_t st);
 
 cudaError_t launch_nvfp4_quantize(const void *x, bool in_bf16, int32_t M, int32_t K, float gs,
                                   uint8_t *xq, uint8_t *xs, cudaStream_t st);
+cudaError_t launch_nvfp4_dequantize(const uint8_t *xq, const uint8_t *xs, int32_t M, int32_t K, float gs,
+                                    bool out_bf16, void *y, cudaStream_t st);
 
 struct GemmArgs {
     const uint8_t *aq, *as, *bq, *bs;

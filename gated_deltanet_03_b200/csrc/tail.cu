@@ -196,6 +196,67 @@ nvfp4_quantize_kernel(const void *__restrict__ x, int64_t nblocks, float gs,
     }
 }
 
+// E2M1 and E4M3 values from their bit fields (the formats' definitions: E2M1 = sign, 2-bit
+// exponent with bias 1, 1-bit mantissa; E4M3 = sign, 4-bit exponent with bias 7, 3-bit mantissa,
+// exponent 0 subnormal, 0x7F / 0xFF NaN).
+GDN_DEV float e2m1_value(uint32_t c) {
+    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+    const float mag = e == 0 ? 0.5f * (float)m : (1.0f + 0.5f * (float)m) * (float)(1u << (e - 1));
+    return (c & 8u) ? -mag : mag;
+}
+GDN_DEV float e4m3_value(uint32_t b) {
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+    if (e == 15u && m == 7u) return __int_as_float(0x7fc00000);
+    const float mag = e == 0 ? (float)m * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+    return (b & 0x80u) ? -mag : mag;
+}
+
+// x_hat = E2M1(code) * E4M3(block scale) / gs: the product is exact in fp32 and the IEEE
+// division rounds it once, so each value is the correctly rounded fp32 quotient. One thread per
+// 16-value block (8 code bytes, 1 scale byte).
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256)
+nvfp4_dequantize_kernel(const uint8_t *__restrict__ xq, const uint8_t *__restrict__ xs, int64_t nblocks, float gs,
+                        void *__restrict__ y) {
+    pdl_launch_dependents();
+    pdl_wait();
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblocks;
+         blk += (int64_t)gridDim.x * blockDim.x) {
+        const uint2 codes = *reinterpret_cast<const uint2 *>(xq + blk * 8);
+        const float sc = e4m3_value(xs[blk]);
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t byte = ((i < 4 ? codes.x : codes.y) >> (8 * (i & 3))) & 0xFFu;
+            v[2 * i] = __fdiv_rn(e2m1_value(byte & 15u) * sc, gs);
+            v[2 * i + 1] = __fdiv_rn(e2m1_value(byte >> 4) * sc, gs);
+        }
+        if constexpr (OUT_BF16) {
+            uint4 u[2];
+            __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(u);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(y) + blk * 16);
+            dst[0] = u[0];
+            dst[1] = u[1];
+        } else {
+            float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(y) + blk * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+    }
+}
+
+cudaError_t launch_nvfp4_dequantize(const uint8_t *xq, const uint8_t *xs, int32_t M, int32_t K, float gs,
+                                    bool out_bf16, void *y, cudaStream_t st) {
+    const int64_t nblocks = (int64_t)M * (K / 16);
+    if (nblocks == 0) return cudaSuccess;
+    int64_t grid = (nblocks + 255) / 256;
+    if (grid > 148 * 8) grid = 148 * 8;
+    if (out_bf16) return launch_pdl(nvfp4_dequantize_kernel<true>, dim3((unsigned)grid), dim3(256), 0, st, xq, xs, nblocks, gs, y);
+    return launch_pdl(nvfp4_dequantize_kernel<false>, dim3((unsigned)grid), dim3(256), 0, st, xq, xs, nblocks, gs, y);
+}
+
 cudaError_t launch_nvfp4_quantize(const void *x, bool in_bf16, int32_t M, int32_t K, float gs,
                                   uint8_t *xq, uint8_t *xs, cudaStream_t st) {
     const int64_t nblocks = (int64_t)M * (K / 16);

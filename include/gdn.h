@@ -210,6 +210,15 @@ GDN_API gdn_status gdn_gated_rmsnorm_silu_nvfp4(const void *o, const void *z, co
 GDN_API gdn_status nvfp4_quantize_act(const void *x, gdn_dtype in_dtype, int32_t M, int32_t K,
                               float global_scale, uint8_t *xq, uint8_t *xs, gdn_stream_t stream);
 
+/* Inverse of nvfp4_quantize_act: y[m, k] = E2M1(code) * E4M3(scale of its 16-value block) /
+ * global_scale, each value the correctly rounded fp32 quotient (then rounded to bf16 for a bf16
+ * y). xq [M, K/2] (8-byte aligned), xs [M, K/16] as nvfp4_quantize_act writes them; y [M, K] in
+ * `out_dtype`. Used to measure what NVFP4 does to activations (quantise, then dequantise).
+ * Supported: K % 16 == 0. */
+GDN_API gdn_status nvfp4_dequantize_act(const uint8_t *xq, const uint8_t *xs, int32_t M, int32_t K,
+                                        float global_scale, gdn_dtype out_dtype, void *y,
+                                        gdn_stream_t stream);
+
 /* ------------------------------------------------------------ NVFP4 GEMM ----
  * [GDN] "NVFP4 W4A4 on all linear layers"; [TAIL] step 6 (ssm_out, 4096 -> 2048):
  *   y[m, n] = alpha * sum_k E2M1(a)[m,k] E4M3(as)[m,k/16] E2M1(b)[n,k] E4M3(bs)[n,k/16]
