@@ -48,6 +48,8 @@ def make_l2_flush(torch, dev):
         torch.sum(rbuf, dim=0, out=sink)
     return flush
 CHUNK = 64
+# FP4 (kind::mxf4nvf4) dense rate measured by a tcgen05 probe: 16368 MAC/cycle/SM x 148 SMs x 1965 MHz
+FP4_PROBE_TFLOPS = 2.0 * 16368 * 148 * 1.965e9 / 1e12
 # DRAM bytes (read + write) of one scan call (prep + chain kernels) on the benchmark workload,
 # from the ncu capture summarised in profiles/chunked_prefill_T4096.md; valid only for the
 # kernel source it was taken on (first 16 hex digits of its sha256).
@@ -423,6 +425,19 @@ def run_gpu(args):
     assert g.gdn_get_device_status() == 0
     del mstate
 
+    # the NVFP4 GEMM at the long-prefill layer's output projection (32768 x 2048 x 4096)
+    gM, gN, gK = 32768, 2048, 4096
+    ga = g.nvfp4_quantize_act(up(workloads.activations(gM, gK, seed=5, heavy_tail=False), bf), 448.0 * 6.0 / 6.0)
+    gw = g.nvfp4_quantize_act(up(workloads.activations(gN, gK, seed=6, heavy_tail=False), bf), 448.0 * 6.0 / 6.0)
+    gy = torch.empty((gM, gN), dtype=bf, device=dev)
+    big_graph = graph_of(lambda: g.nvfp4_gemm(ga[0], ga[1], gw[0], gw[1], 1.0, y=gy))
+    for _ in range(3):
+        big_graph.replay()
+    big_ev = timed(big_graph, max(args.steps, 10))
+    torch.cuda.synchronize()
+    big_ms = statistics.mean(a.elapsed_time(b) for a, b in big_ev)
+    del ga, gw, gy, big_graph
+
     # short convolution decode on the batched-decode workload's q|k|v channels (state in place)
     dC = 2 * dw.Hk * dw.D + dw.Hv * dw.D
     dcx = workloads.conv_inputs(dw.num_seqs, dC, 4, seed=dw.seed, num_seqs=dw.num_seqs, state=True)
@@ -487,6 +502,10 @@ def run_gpu(args):
         "decode": {"workload": dw.name, "ms": dec, "GB/s": dec_bytes / (dec / 1e3) / 1e9,
                    "frac": dec_bytes / (dec / 1e3) / 1e9 / float(pk["hbm_gbs"]),
                    "bytes": dec_bytes, "peak_gbs": float(pk["hbm_gbs"]), "peak_kind": pk_kind},
+        "gemm_long_prefill": {"shape": [gM, gN, gK], "ms": big_ms,
+                              "TFLOP/s": 2.0 * gM * gN * gK / (big_ms / 1e3) / 1e12,
+                              "frac_of_fp4_probe": 2.0 * gM * gN * gK / (big_ms / 1e3) / 1e12 / FP4_PROBE_TFLOPS,
+                              "peak_kind": "FP4 tensor rate measured by a tcgen05 probe (16368 MAC/cycle/SM at 1965 MHz)"},
         "decode_multi": {"workload": "%s shape, %d draft tokens per sequence" % (dw.name, mT),
                          "verify_ms": ver_ms, "verify_GB/s": ver_bytes / (ver_ms / 1e3) / 1e9,
                          "verify_frac": ver_bytes / (ver_ms / 1e3) / 1e9 / float(pk["hbm_gbs"]),

@@ -5,18 +5,24 @@
 // layer; "Red Lite dev15d - DeltaNet gated tail", Pinned graph semantics, step 6: the output
 // projection (4096 -> 2048 in the 27B-class layer).
 //
-// One CTA computes a 128 x 256 tile of y. Warp roles:
-//   warp 0   TMA producer: A (128 rows x 128 B) and B (256 rows x 128 B) tiles per stage,
-//            128-byte swizzle, into a 4-stage ring, with the stage's row-major [rows, 16 B]
-//            E4M3 scales when K % 256 == 0;
-//   warp 1   allocates tensor memory; lane 0 issues tcgen05.mma;
-//   warps 4-7 scales, then the epilogue. Per stage each warp writes the scales into its lane
-//            quarter of the stage's tensor-memory scale slot with tcgen05.st (the layout the
-//            block-scaled MMA reads: for 32 rows r = 32 c + l, lane l, column 4 kb + c holds
-//            the four 16-value block scales of MMA k-step kb; the four lane quarters hold the
-//            same copy), read from the TMA-staged tile, or from global memory (zero past K)
-//            when the scales cannot be TMA-loaded. After the last stage: tensor memory ->
-//            registers -> alpha * acc -> 128-byte-swizzled shared-memory boxes -> TMA stores.
+// Persistent: one CTA per SM walks 128 x 256 tiles of y (tile t = blockIdx.x, + gridDim.x, ...;
+// consecutive tiles share their A rows, so concurrent CTAs read each A tile from DRAM once).
+// The stage ring and its barriers run on one counter across tiles, so the producer fetches the
+// next tile's stages while the epilogue drains the current one. Warp roles:
+//   warp 0     TMA producer: A (128 rows x 128 B) and B (256 rows x 128 B) tiles per stage,
+//              128-byte swizzle, into a 4-stage ring, with the stage's row-major [rows, 16 B]
+//              E4M3 scales when K % 256 == 0;
+//   warp 1     allocates tensor memory; lane 0 issues tcgen05.mma, and before a tile's first
+//              MMA waits until the epilogue has read the previous tile's accumulator;
+//   warps 4-7  per stage each writes the scales into its lane quarter of the stage's
+//              tensor-memory scale slot with tcgen05.st (the layout the block-scaled MMA reads:
+//              for 32 rows r = 32 c + l, lane l, column 4 kb + c holds the four 16-value block
+//              scales of MMA k-step kb; the four lane quarters hold the same copy), read from the
+//              TMA-staged tile, or from global memory (zero past K) when the scales cannot be
+//              TMA-loaded;
+//   warps 8-15 the epilogue, two warps per lane quarter (column halves): tensor memory ->
+//              registers (64 columns at a time; after its last read the warp releases the
+//              accumulator) -> alpha * acc -> 16-byte stores of the thread's row.
 // Every barrier wait is bounded (about 1 s); an expired wait records GDN_ERR_TIMEOUT and
 // the CTA finishes without issuing more work.
 #include <mutex>
@@ -35,8 +41,10 @@ constexpr int B_BYTES = BN * BK / 2;       // 32 KB
 constexpr int SFA_BYTES = (BM / 128) * (BK / 64) * 512;   // 2 KB: 4 k-blocks x one 128-row block
 constexpr int SFB_BYTES = (BN / 128) * (BK / 64) * 512;   // 4 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr int THREADS = 256;
+constexpr int EPI_WARPS = 8;
+constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+constexpr int SMEM_BYTES = BAR_OFF + 256 /*barriers*/ + 1024 /*align*/;
+constexpr int THREADS = 512;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0;             // accumulator: 128 lanes x 256 columns fp32
 constexpr uint32_t TM_SF = 256;            // per stage slot: A scales 4 x 4 columns, B scales 4 x 8
@@ -92,12 +100,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Smem sm{base};
-    uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
-    uint64_t *full = bars, *empty = bars + STAGES, *sf_ready = bars + 2 * STAGES, *acc_full = bars + 3 * STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 1);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + BAR_OFF);
+    uint64_t *full = bars, *empty = bars + STAGES, *sf_ready = bars + 2 * STAGES;
+    uint64_t *acc_full = bars + 3 * STAGES, *acc_empty = bars + 3 * STAGES + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 2);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int tile_n = blockIdx.x, tile_m = blockIdx.y;
+    const int tiles_n = (N + BN - 1) / BN;
+    const int num_tiles = tiles_n * ((M + BM - 1) / BM);
     const int num_k = (K + BK - 1) / BK;
     const int nblk16 = K / 16;
 
@@ -107,7 +117,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             mbar_init(&empty[s], 1);     // tcgen05.commit of the MMAs that read the stage
             mbar_init(&sf_ready[s], 4);  // scale warps: the stage's scales are in tensor memory
         }
-        mbar_init(acc_full, 1);
+        mbar_init(acc_full, 1);          // tcgen05.commit after a tile's last MMA
+        mbar_init(acc_empty, EPI_WARPS); // every epilogue warp has read its part of the accumulator
         fence_barrier_init();
         tma_prefetch_desc(&map_a);
         tma_prefetch_desc(&map_b);
@@ -124,16 +135,21 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
 
     if (warp == 0) {
         if (lane == 0) {
-            for (int kt = 0; kt < num_k; ++kt) {
-                const int s = kt % STAGES;
-                const uint32_t ph = (kt / STAGES) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, status)) break;
-                mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + (sf_tma ? SFA_BYTES + SFB_BYTES : 0));
-                tma_load_2d(sm.a(s), &map_a, &full[s], kt * (BK / 2), tile_m * BM);
-                tma_load_2d(sm.b(s), &map_b, &full[s], kt * (BK / 2), tile_n * BN);
-                if (sf_tma) {
-                    tma_load_2d(sm.sfa(s), &map_sfa, &full[s], kt * (BK / 16), tile_m * BM);
-                    tma_load_2d(sm.sfb(s), &map_sfb, &full[s], kt * (BK / 16), tile_n * BN);
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                const int tile_m = t / tiles_n, tile_n = t % tiles_n;
+                for (int kt = 0; kt < num_k; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(&empty[s], ph ^ 1, status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + (sf_tma ? SFA_BYTES + SFB_BYTES : 0));
+                    tma_load_2d(sm.a(s), &map_a, &full[s], kt * (BK / 2), tile_m * BM);
+                    tma_load_2d(sm.b(s), &map_b, &full[s], kt * (BK / 2), tile_n * BN);
+                    if (sf_tma) {
+                        tma_load_2d(sm.sfa(s), &map_sfa, &full[s], kt * (BK / 16), tile_m * BM);
+                        tma_load_2d(sm.sfb(s), &map_sfb, &full[s], kt * (BK / 16), tile_n * BN);
+                    }
                 }
             }
         }
@@ -141,140 +157,153 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc();
             bool ok = true;
-            for (int kt = 0; kt < num_k && ok; ++kt) {
-                const int s = kt % STAGES;
-                const uint32_t ph = (kt / STAGES) & 1;
-                if (!mbar_wait(&full[s], ph, status) || !mbar_wait(&sf_ready[s], ph, status)) { ok = false; break; }
+            int it = 0, j = 0;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++j) {
+                // the accumulator is free once every epilogue warp has read the previous tile
+                if (j > 0 && !mbar_wait(acc_empty, (uint32_t)((j - 1) & 1), status)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t sf = tmem + TM_SF + s * SF_SLOT;
+                for (int kt = 0; kt < num_k; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(&full[s], ph, status) || !mbar_wait(&sf_ready[s], ph, status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sf = tmem + TM_SF + s * SF_SLOT;
 #pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
-                    const uint64_t adesc = smem_desc(smem_u32(sm.a(s)) + kb * 32, 16, 1024, 2);
-                    const uint64_t bdesc = smem_desc(smem_u32(sm.b(s)) + kb * 32, 16, 1024, 2);
-                    const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
-                    asm volatile(
-                        "{\n\t.reg .pred p;\n\t"
-                        "setp.ne.b32 p, %4, 0;\n\t"
-                        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
-                        "}" ::"r"(tmem + TM_ACC),
-                        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(sf + kb * 4), "r"(sf + 16 + kb * 8));
+                    for (int kb = 0; kb < 4; ++kb) {
+                        const uint64_t adesc = smem_desc(smem_u32(sm.a(s)) + kb * 32, 16, 1024, 2);
+                        const uint64_t bdesc = smem_desc(smem_u32(sm.b(s)) + kb * 32, 16, 1024, 2);
+                        const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
+                        asm volatile(
+                            "{\n\t.reg .pred p;\n\t"
+                            "setp.ne.b32 p, %4, 0;\n\t"
+                            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+                            "}" ::"r"(tmem + TM_ACC),
+                            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(sf + kb * 4), "r"(sf + 16 + kb * 8));
+                    }
+                    tc_commit(&empty[s]);
                 }
-                tc_commit(&empty[s]);
+                if (ok) tc_commit(acc_full);
             }
-            if (ok) tc_commit(acc_full);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 8) {
         const int quarter = warp - 4;  // == warp % 4: this warp's lane quarter of tensor memory
         const uint32_t lane_q = (uint32_t)(quarter * 32) << 16;
         bool ok = true;
+        int it = 0;
         // ---- scales of every stage into tensor memory
-        for (int kt = 0; kt < num_k; ++kt) {
-            const int s = kt % STAGES;
-            const uint32_t ph = (kt / STAGES) & 1;
-            uint32_t ra[16], rb[32];
-            if (sf_tma) {
-                // the stage's scale tiles have landed (which also means the slot's previous
-                // MMAs are complete: the producer refilled the stage after they released it)
-                if (lane == 0) ok = mbar_wait(&full[s], ph, status);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
+        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            const int tile_m = t / tiles_n, tile_n = t % tiles_n;
+            for (int kt = 0; kt < num_k; ++kt, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                uint32_t ra[16], rb[32];
+                if (sf_tma) {
+                    // the stage's scale tiles have landed (which also means the slot's previous
+                    // MMAs are complete: the producer refilled the stage after they released it)
+                    if (lane == 0) ok = mbar_wait(&full[s], ph, status);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 v = reinterpret_cast<const uint4 *>(sm.sfa(s))[c * 32 + lane];
-                    ra[c] = v.x; ra[4 + c] = v.y; ra[8 + c] = v.z; ra[12 + c] = v.w;
-                }
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 v = reinterpret_cast<const uint4 *>(sm.sfa(s))[c * 32 + lane];
+                        ra[c] = v.x; ra[4 + c] = v.y; ra[8 + c] = v.z; ra[12 + c] = v.w;
+                    }
 #pragma unroll
-                for (int gc = 0; gc < 8; ++gc) {   // row g * 128 + c * 32 + lane, gc = g * 4 + c
-                    const uint4 v = reinterpret_cast<const uint4 *>(sm.sfb(s))[gc * 32 + lane];
-                    rb[gc] = v.x; rb[8 + gc] = v.y; rb[16 + gc] = v.z; rb[24 + gc] = v.w;
-                }
-            } else {
-                // the slot is free once the MMAs of its previous stage have completed
-                if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, status);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                const int kb16 = kt * (BK / 16);
+                    for (int gc = 0; gc < 8; ++gc) {   // row g * 128 + c * 32 + lane, gc = g * 4 + c
+                        const uint4 v = reinterpret_cast<const uint4 *>(sm.sfb(s))[gc * 32 + lane];
+                        rb[gc] = v.x; rb[8 + gc] = v.y; rb[16 + gc] = v.z; rb[24 + gc] = v.w;
+                    }
+                } else {
+                    // the slot is free once the MMAs of its previous stage have completed
+                    if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, status);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    const int kb16 = kt * (BK / 16);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 v = load_scale_row(sfa_g, tile_m * BM + c * 32 + lane, M, kb16, nblk16);
-                    ra[c] = v.x; ra[4 + c] = v.y; ra[8 + c] = v.z; ra[12 + c] = v.w;
-                }
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 v = load_scale_row(sfa_g, tile_m * BM + c * 32 + lane, M, kb16, nblk16);
+                        ra[c] = v.x; ra[4 + c] = v.y; ra[8 + c] = v.z; ra[12 + c] = v.w;
+                    }
 #pragma unroll
-                for (int gc = 0; gc < 8; ++gc) {
-                    const uint4 v = load_scale_row(sfb_g, tile_n * BN + gc * 32 + lane, N, kb16, nblk16);
-                    rb[gc] = v.x; rb[8 + gc] = v.y; rb[16 + gc] = v.z; rb[24 + gc] = v.w;
+                    for (int gc = 0; gc < 8; ++gc) {
+                        const uint4 v = load_scale_row(sfb_g, tile_n * BN + gc * 32 + lane, N, kb16, nblk16);
+                        rb[gc] = v.x; rb[8 + gc] = v.y; rb[16 + gc] = v.z; rb[24 + gc] = v.w;
+                    }
                 }
+                const uint32_t sf = tmem + lane_q + TM_SF + s * SF_SLOT;
+                tmem_st16(sf, ra);
+                tmem_st16(sf + 16, *reinterpret_cast<const uint32_t(*)[16]>(&rb[0]));
+                tmem_st16(sf + 32, *reinterpret_cast<const uint32_t(*)[16]>(&rb[16]));
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_ready[s]);
             }
-            const uint32_t sf = tmem + lane_q + TM_SF + s * SF_SLOT;
-            tmem_st16(sf, ra);
-            tmem_st16(sf + 16, *reinterpret_cast<const uint32_t(*)[16]>(&rb[0]));
-            tmem_st16(sf + 32, *reinterpret_cast<const uint32_t(*)[16]>(&rb[16]));
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sf_ready[s]);
         }
-        // ---- epilogue
-        if (ok) {
-            if (lane == 0) ok = mbar_wait(acc_full, 0, status);
+    } else if (warp >= 8) {
+        // ---- epilogue: warp e owns rows 32 (e % 4) .. + 31 and columns 128 (e / 4) .. + 127;
+        // each thread stores its row's values straight from registers (16-byte stores; the row
+        // pieces of one warp instruction are scattered, the next instructions fill the sectors)
+        const int e = warp - 8, quarter = e % 4, half = e / 4;
+        const uint32_t lane_q = (uint32_t)(quarter * 32) << 16;
+        bool ok = true;
+        int j = 0;
+        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++j) {
+            const int tile_m = t / tiles_n, tile_n = t % tiles_n;
+            if (lane == 0) ok = mbar_wait(acc_full, (uint32_t)(j & 1), status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
-        }
-        const int ept = threadIdx.x - 128;   // 0..127: this thread's row of the tile
-        // every stage is consumed by then: the ring holds the output boxes, [128 rows][128 B] each
-        uint8_t *obox = base;
-        if (ok) {
+            if (!ok) break;
             tc_fence_after();
-            const int r = ept;
+            const int row = tile_m * BM + quarter * 32 + lane;
 #pragma unroll 1
-            for (int c1 = 0; c1 < BN; c1 += 64) {
-                uint32_t rr[2][32];   // two loads in flight per wait
-                tmem_ld32(tmem + TM_ACC + lane_q + c1, rr[0]);
-                tmem_ld32(tmem + TM_ACC + lane_q + c1 + 32, rr[1]);
+            for (int pr = 0; pr < 2; ++pr) {
+                uint32_t rr[2][32];
+                tmem_ld32(tmem + TM_ACC + lane_q + half * 128 + 64 * pr, rr[0]);
+                tmem_ld32(tmem + TM_ACC + lane_q + half * 128 + 64 * pr + 32, rr[1]);
                 tmem_ld_wait();
+                if (pr == 1) {
+                    // this warp's last read of the accumulator: release it to the next tile's MMAs
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(acc_empty);
+                }
+                if (row >= M) continue;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int c0 = c1 + 32 * hh;
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    const int c0 = tile_n * BN + half * 128 + 64 * pr + 32 * q2;   // first of these 32 columns
+                    if (c0 >= N) break;
                     float v[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        // per-column factor when the output columns come from modules with their
-                        // own global scales (clamped index: columns past N are never stored)
-                        const float al = col_alpha ? __ldg(col_alpha + min(tile_n * BN + c0 + j, N - 1)) : alpha;
-                        v[j] = __uint_as_float(rr[hh][j]) * al;
+                    for (int jj = 0; jj < 32; ++jj) {
+                        // per-column factor when the output columns come from modules with their own
+                        // global scales (clamped index: columns past N are never stored)
+                        const float al = col_alpha ? __ldg(col_alpha + min(c0 + jj, N - 1)) : alpha;
+                        v[jj] = __uint_as_float(rr[q2][jj]) * al;
                     }
+                    // N % 16 == 0, so every 8-column (bf16) or 4-column (fp32) piece is whole or absent
                     if (out_bf16) {
-                        uint8_t *box = obox + (c0 / 64) * 16384 + r * 128;
+                        __nv_bfloat16 *yr = reinterpret_cast<__nv_bfloat16 *>(y) + (size_t)row * N + c0;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const int chunk = (c0 % 64) / 8 + i;
+                            if (c0 + 8 * i >= N) break;
                             uint4 u;
                             __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&u);
 #pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                p2[e] = __floats2bfloat162_rn(v[8 * i + 2 * e], v[8 * i + 2 * e + 1]);
-                            *reinterpret_cast<uint4 *>(box + ((chunk ^ (r & 7)) << 4)) = u;
+                            for (int q = 0; q < 4; ++q)
+                                p2[q] = __floats2bfloat162_rn(v[8 * i + 2 * q], v[8 * i + 2 * q + 1]);
+                            *reinterpret_cast<uint4 *>(yr + 8 * i) = u;
                         }
                     } else {
-                        uint8_t *box = obox + (c0 / 32) * 16384 + r * 128;
+                        float *yr = reinterpret_cast<float *>(y) + (size_t)row * N + c0;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            *reinterpret_cast<float4 *>(box + ((i ^ (r & 7)) << 4)) =
+                        for (int i = 0; i < 8; ++i) {
+                            if (c0 + 4 * i >= N) break;
+                            *reinterpret_cast<float4 *>(yr + 4 * i) =
                                 make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        }
                     }
                 }
             }
-            fence_proxy_async_smem();
-        }
-        asm volatile("barrier.cta.sync 1, 128;" ::: "memory");
-        if (ok && ept == 0) {
-            const int nbox = out_bf16 ? BN * 2 / 128 : BN * 4 / 128;
-            const int esz = out_bf16 ? 2 : 4;
-            for (int b = 0; b < nbox; ++b) {
-                const int x = tile_n * BN * esz + b * 128;
-                if (x < N * esz) tma_store_2d(&map_y, obox + b * 16384, x, tile_m * BM);
-            }
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }
     }
 
@@ -337,14 +366,20 @@ cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
     }
     CUtensorMap my;
     const uint64_t y_row_bytes = (uint64_t)g.N * (g.out_bf16 ? 2 : 4);
-    if (!make_map(&my, g.y, (uint64_t)g.M, y_row_bytes, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&my, g.y, (uint64_t)g.M, y_row_bytes, 32)) return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM);
+    static int sms[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return cudaErrorInvalidDevice;
+    const int tiles = ((g.N + BN - 1) / BN) * ((g.M + BM - 1) / BM);
+    dim3 grid((unsigned)(tiles < sms[dev] ? tiles : sms[dev]));
     return launch_pdl(nvfp4_gemm_kernel, grid, dim3(THREADS), SMEM_BYTES, st, ma, mb, msa, msb, my, sf_tma ? 1 : 0,
                       g.as, g.bs, g.alpha, g.col_alpha, g.M, g.N, g.K, g.out_bf16 ? 1 : 0, g.y, g.status);
 }
