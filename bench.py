@@ -539,6 +539,8 @@ def run_only(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     bf, f32 = torch.bfloat16, torch.float32
+    if args.only == "gemm_long":
+        return run_gemm_long(args)
     names = {wl.name: wl for wl in workloads.WORKLOADS}
     w = names[args.workload] if args.workload else (workloads.DECODE_B256 if args.only in ("decode", "conv_decode")
                                                     else workloads.PREFILL_1K)
@@ -596,6 +598,41 @@ def run_only(args):
     assert g.gdn_get_device_status() == 0
     print(json.dumps({"only": args.only, "workload": w.name, "ms_median": statistics.median(times),
                       "ms_mean": statistics.mean(times), "steps": args.steps}))
+
+
+def run_gemm_long(args):
+    """The NVFP4 GEMM alone at the long-prefill layer's output projection (32768 x 2048 x 4096),
+    `warmup` + `steps` launches, CUDA-event timed with the L2 flushed between them."""
+    import torch
+
+    import gated_deltanet_03_b200 as g
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    gM, gN, gK = 32768, 2048, 4096
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, torch.bfloat16)
+
+    xa = g.nvfp4_quantize_act(up(workloads.activations(gM, gK, seed=5, heavy_tail=False)), 448.0)
+    xw = g.nvfp4_quantize_act(up(workloads.activations(gN, gK, seed=6, heavy_tail=False)), 448.0)
+    y = torch.empty((gM, gN), dtype=torch.bfloat16, device=dev)
+    flush = make_l2_flush(torch, dev)
+    for _ in range(args.warmup):
+        g.nvfp4_gemm(xa[0], xa[1], xw[0], xw[1], 1.0, y=y)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.nvfp4_gemm(xa[0], xa[1], xw[0], xw[1], 1.0, y=y)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    assert g.gdn_get_device_status() == 0
+    ms = statistics.median(times)
+    print(json.dumps({"only": "gemm_long", "shape": [gM, gN, gK], "ms_median": ms,
+                      "TFLOP/s": 2.0 * gM * gN * gK / (ms / 1e3) / 1e12, "steps": args.steps}))
 
 
 # ----------------------------------------------------------------- CPU arm ----
@@ -659,7 +696,7 @@ def main():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
-    p.add_argument("--only", choices=["scan", "tail", "gemm", "decode", "fused", "conv", "conv_decode"],
+    p.add_argument("--only", choices=["scan", "tail", "gemm", "gemm_long", "decode", "fused", "conv", "conv_decode"],
                    help="time one kernel alone on its workload (for profiling); prints one JSON line")
     p.add_argument("--workload", default=None, help="workload name for --only scan (default: 1024-wide prefill)")
     args = p.parse_args()

@@ -1254,6 +1254,11 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
 // Segment combine: per (value head, sequence), S_start(p + 1) = S_start(p) M_p + B_p in order,
 // S_start(1) = B_0. The product runs on the tensor cores with S split into fp16 hi + lo and M
 // given as fp16 hi + lo operand images (S_hi M_hi + S_lo M_hi + S_hi M_lo, fp32 accumulation).
+// Rows of S are independent in S M + B, so four CTAs share a (value head, sequence), each owning
+// 32 rows (blockIdx.z): each streams the whole M_p (64 KB) but only its quarter of B_p and of the
+// published states, 80 KB per step instead of 128 KB, which is what bounds a step (an SM takes
+// about 30 bytes per cycle from L2). Its rows sit in TMEM lanes 0-31, handled by warps 0 and 4;
+// the MMA's other 96 lanes carry no data and their results are not read.
 // ===================================================================================
 constexpr int CB_OFF_BUF = 0;                   // two buffers of [M_hi | M_lo] images, 64 KB each
 constexpr int CB_OFF_BAR = 2 * 65536;
@@ -1264,7 +1269,7 @@ __global__ void __launch_bounds__(NT, 1)
 gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
     pdl_launch_dependents();
     pdl_wait();
-    const int h = blockIdx.x, n = blockIdx.y;
+    const int h = blockIdx.x, n = blockIdx.y, rblk = blockIdx.z;
     const int SEG = P.seg_chunks;
     int t_begin = 0, t_end = P.T;
     if (P.cu_seqlens) {
@@ -1283,8 +1288,9 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
     uint64_t *bar_mma = full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 3);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int wg = warp / 4, row = (warp % 4) * 32 + lane;
-    const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
+    const int wg = warp / 4, row = rblk * 32 + lane;
+    const bool active = (warp % 4) == 0;   // warps 0 and 4: TMEM lanes 0-31, this CTA's rows
+    const uint32_t lane_base = 0;
 
     if (tid == 0) {
         mbar_init(&full[0], 1);
@@ -1308,7 +1314,7 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
     if (tid == 0 && nseg > 2) issue_m(1);
 
     float S[64];   // S_start(p), starting from S_start(1) = B_0
-    ilv_load(seg(0) + kSegB, row, wg, S);
+    if (active) ilv_load(seg(0) + kSegB, row, wg, S);
     const uint32_t idm = idesc_f16(128, false, true, false);
     const f2_t neg1 = f2(-1.0f, -1.0f);
     for (int p = 1; p + 1 < nseg; ++p) {
@@ -1316,7 +1322,7 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
         uint8_t *buf = sm + CB_OFF_BUF + b * 65536;
         // S -> fp16 hi / lo A operands
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
+        for (int part = 0; part < 2 && active; ++part) {
             uint32_t hi[16], lo[16];
 #pragma unroll
             for (int w = 0; w < 16; ++w) {
@@ -1356,12 +1362,15 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
             }
         }
         // while the MMAs run: publish S_start(p) for the output pass, fetch B_p
-        ilv_store(seg(p) + kSegS, row, wg, S);
         float Bp[64];
-        ilv_load(seg(p) + kSegB, row, wg, Bp);
+        if (active) {
+            ilv_store(seg(p) + kSegS, row, wg, S);
+            ilv_load(seg(p) + kSegB, row, wg, Bp);
+        }
         if (tid == 0 && ok) ok = mbar_wait(bar_mma, (uint32_t)((p - 1) & 1), P.status) ? 1 : 0;
         if (!__syncthreads_and(ok)) break;
         tc_fence_after();
+        if (!active) continue;
         uint32_t r32[2][32];
         tmem_ld32(tmem + CB_TM_D + lane_base + wg * 64, r32[0]);
         tmem_ld32(tmem + CB_TM_D + lane_base + wg * 64 + 32, r32[1]);
@@ -1375,7 +1384,7 @@ gdn_segment_combine_kernel(const __grid_constant__ ChainParams P) {
         }
         tc_fence_before();
     }
-    ilv_store(seg(nseg - 1) + kSegS, row, wg, S);   // the last segment's start state
+    if (active) ilv_store(seg(nseg - 1) + kSegS, row, wg, S);   // the last segment's start state
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -1470,7 +1479,7 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
         P.mode_base = kChainState;   // z = 0: segment states (B), z = 1: segment transitions (M)
         if ((e = launch_pdl(gdn_chunk_lean_kernel, dim3(c.Hv, seg_slots, 2), dim3(NT), CL_SMEM, st, P)) != cudaSuccess)
             return e;
-        if ((e = launch_pdl(gdn_segment_combine_kernel, dim3(c.Hv, c.num_seqs), dim3(NT), CB_SMEM, st, P)) != cudaSuccess)
+        if ((e = launch_pdl(gdn_segment_combine_kernel, dim3(c.Hv, c.num_seqs, 4), dim3(NT), CB_SMEM, st, P)) != cudaSuccess)
             return e;
         P.mode_base = kChainFull;
     }
