@@ -283,44 +283,30 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     if (tid >= 32 && tid < 64) sG[tid] += sG[31];
 
     int ok = 1;
-    if (tid == 0) ok = mbar_wait(bar_tma, 0, status) ? 1 : 0;
-    if (!__syncthreads_and(ok)) goto teardown;
-    {
-        // [K;Q] rows: thread -> (row rho = tid / 2, half = tid % 2); V: 4 chunks per thread
-        const int rho = tid >> 1, half = tid & 1;
-        uint8_t *rowp = sm + P_OFF_KQ + half * 2 * TILE + rho * 128;
-        float ss = 0.0f;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) ss += convert16(rowp + ((ch + rho) & 7) * 16);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        if (half == 0) sSS[rho] = ss;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int idx = e * NT + tid;
-            convert16(sm + P_OFF_VLO + (idx >> 9) * 2 * TILE + (idx & 511) * 16);
-        }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
     if (tid == 0) {
-        // D1 = [K; Q] K^T: lanes 0-63 K K^T, lanes 64-127 Q K^T (row = token, column = key token)
-        tc_fence_after();
-        const uint32_t id1 = idesc_f16(64, false, false, false);
+        ok = mbar_wait(bar_tma, 0, status) ? 1 : 0;
+        if (ok) {
+            // D1 = [K; Q] [K; Q]^T straight from the raw bf16 tiles: lanes 0-63 hold K K^T | K Q^T,
+            // lanes 64-127 Q K^T | Q Q^T (row = token, column = token). The diagonals are the
+            // squared norms |k_r|^2 and |q_r|^2 (exact bf16 products, fp32 sums).
+            tc_fence_after();
+            const uint32_t id1 = idesc_f16(128, false, false, false) | (1u << 7) | (1u << 10);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint8_t *base = sm + P_OFF_KQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
-            mma_f16(tmem + P_TM_D1, kdesc(base), kdesc(base), id1, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint8_t *base = sm + P_OFF_KQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
+                mma_f16(tmem + P_TM_D1, kdesc(base), kdesc(base), id1, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar_mma);
         }
-        tc_commit(bar_mma);
     }
-    if (tid < 64) {
-        const bool v = tid < L;
-        sRk[tid] = v ? (l2norm ? rsqrtf(sSS[tid] + 1e-6f) : 1.0f) : 0.0f;
-        sRq[tid] = v ? (l2norm ? rsqrtf(sSS[64 + tid] + 1e-6f) * scale : scale) : 0.0f;
-        sGam[tid] = v ? expf(sG[tid]) : 0.0f;
+    if (!__syncthreads_and(ok)) goto teardown;
+    // while MMA1 runs: V to fp16 in place (MMA1 reads only the K and Q tiles), decay factors
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int idx = e * NT + tid;
+        convert16(sm + P_OFF_VLO + (idx >> 9) * 2 * TILE + (idx & 511) * 16);
     }
-    __syncthreads();
-    if (tid < 64) sDec[tid] = tid < L ? __expf(sG[L - 1] - sG[tid]) * sRk[tid] : 0.0f;
+    if (tid < 64) sGam[tid] = tid < L ? expf(sG[tid]) : 0.0f;
     if (tid == 0) {
         float *wv = reinterpret_cast<float *>(item + kWsVec);
         wv[0] = __expf(sG[L - 1]);   // gamma_C
@@ -329,10 +315,34 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     if (!__syncthreads_and(ok)) goto teardown;
     tc_fence_after();
     {
-        // every warp reads 32 columns (key tokens s) of its 32 lanes
+        // every warp reads 32 columns (key tokens s) of its 32 lanes; warps 2 and 3 also read the
+        // Q Q^T block that holds their lanes' diagonal
         uint32_t r32[32];
         tmem_ld32(tmem + P_TM_D1 + lane_base + wg * 32, r32);
-        tmem_ld_wait();
+        const int quarter = warp % 4;
+        if (wg == 0 && quarter >= 2) {
+            uint32_t rq32[32];
+            tmem_ld32(tmem + P_TM_D1 + lane_base + 64 + (quarter - 2) * 32, rq32);
+            tmem_ld_wait();
+            float d = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) d = (j == lane) ? __uint_as_float(rq32[j]) : d;
+            const int r = x - 64;
+            sRq[r] = r < L ? (l2norm ? rsqrtf(d + 1e-6f) * scale : scale) : 0.0f;
+        } else {
+            tmem_ld_wait();
+        }
+        if (quarter < 2 && wg == quarter) {
+            // lanes 0-63: the K K^T diagonal sits in column x, i.e. this warp's column `lane`
+            float d = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) d = (j == lane) ? __uint_as_float(r32[j]) : d;
+            const int r = x;
+            const float rk = r < L ? (l2norm ? rsqrtf(d + 1e-6f) : 1.0f) : 0.0f;
+            sRk[r] = rk;
+            sDec[r] = r < L ? __expf(sG[L - 1] - sG[r]) * rk : 0.0f;
+        }
+        __syncthreads();
         // decay and key-norm factors of this warp's 32 columns (same for all lanes), then all 32
         // values, then the stores
         float gs[32], rks[32], vals[32];
@@ -384,8 +394,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     // ---- T = (I + A)^-1 (unit lower triangular), written as T (fp16, for the block products)
     //      and as the B operands T'' = T diag(beta), T' = T diag(beta gamma / |k|). Two warps
     //      solve the 16 x 16 diagonal blocks by forward substitution (fp32) while the other six
-    //      write the state-independent images: Q' and K'' from the converted tiles, P^T from its
-    //      staging, and the zero upper blocks of T' and T''.
+    //      copy the P^T image out of its staging and write the zero upper blocks of T' and T''.
     if (tid < 64) {
         const int bi = tid / 16, cc = tid % 16, o0 = bi * 16, r = o0 + cc;
         float xv[16];
@@ -406,40 +415,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             *reinterpret_cast<__half *>(sm + P_OFF_TP + off) = __float2half_rn(xv[rr] * fbg);
         }
     } else {
-        // Q' rows (64 + r of the [W; Q'] image) and K'' (the first two blocks of [K''; P^T]): the
-        // converted tiles scaled row by row, swizzle positions unchanged; 2048 chunks over 192
-        // threads in two batches whose loads are issued before any store
         const int t6 = tid - 64;
-#pragma unroll
-        for (int batch = 0; batch < 2; ++batch) {
-            uint4 hv[6];
-            float f[6];
-#pragma unroll
-            for (int e = 0; e < 6; ++e) {
-                const int idx = (batch * 6 + e) * 192 + t6;
-                const int ic = idx < 2048 ? idx : 0;
-                const int isk = ic >> 10, w = ic & 1023, half = w >> 9, within = w & 511, r = within >> 3;
-                hv[e] = *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + (2 * half + (isk ? 0 : 1)) * TILE + within * 16);
-                f[e] = isk ? sDec[r] : sGam[r] * sRq[r];
-            }
-#pragma unroll
-            for (int e = 0; e < 6; ++e) {
-                const int idx = (batch * 6 + e) * 192 + t6;
-                if (idx < 2048) {
-                    const int isk = idx >> 10, w = idx & 1023, half = w >> 9, within = w & 511;
-                    const __half2 *h2 = reinterpret_cast<const __half2 *>(&hv[e]);
-                    float xv[8];
-#pragma unroll
-                    for (int q2 = 0; q2 < 4; ++q2) {
-                        const float2 t = __half22float2(h2[q2]);
-                        xv[2 * q2] = t.x * f[e];
-                        xv[2 * q2 + 1] = t.y * f[e];
-                    }
-                    st_h8(isk ? item + kWsKP + half * TILE + within * 16 : item + kWsWQ + half * 2 * TILE + TILE + within * 16,
-                          xv);
-                }
-            }
-        }
         // the P^T image from its staging (512 chunks)
         uint4 pc[3];
 #pragma unroll
@@ -464,53 +440,96 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         }
     }
     __syncthreads();
-    // off-diagonal blocks level by level, from T (I + A) = I:
-    //   T_ij = -(sum_{k=j+1}^{i} T_ik A_kj) T_jj,
-    // one warp per block on the warp-level tensor-core MMA (fp16 inputs, fp32 accumulation); the
-    // sum's accumulator fragments are directly the A fragments of the product with T_jj.
+    if (warp < 3) {
+        // off-diagonal blocks level by level, from T (I + A) = I:
+        //   T_ij = -(sum_{k=j+1}^{i} T_ik A_kj) T_jj,
+        // one warp per block on the warp-level tensor-core MMA (fp16 inputs, fp32 accumulation);
+        // the sum's accumulator fragments are directly the A fragments of the product with T_jj.
+        // Warps 0-2 meet at a named barrier between levels.
 #pragma unroll 1
-    for (int lvl = 1; lvl < 4; ++lvl) {
-        if (warp < 4 - lvl) {
-            const int bj = warp, bi = bj + lvl;
-            const int g = lane >> 2, t = lane & 3;
-            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            for (int bk = bj + 1; bk <= bi; ++bk) {
-                const uint32_t *trow0 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g) * P_AH + bk * 16);
-                const uint32_t *trow1 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g + 8) * P_AH + bk * 16);
-                const uint32_t a0 = trow0[t], a1 = trow1[t], a2 = trow0[t + 4], a3 = trow1[t + 4];
+        for (int lvl = 1; lvl < 4; ++lvl) {
+            if (warp < 4 - lvl) {
+                const int bj = warp, bi = bj + lvl;
+                const int g = lane >> 2, t = lane & 3;
+                float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                for (int bk = bj + 1; bk <= bi; ++bk) {
+                    const uint32_t *trow0 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g) * P_AH + bk * 16);
+                    const uint32_t *trow1 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g + 8) * P_AH + bk * 16);
+                    const uint32_t a0 = trow0[t], a1 = trow1[t], a2 = trow0[t + 4], a3 = trow1[t + 4];
+#pragma unroll
+                    for (int hn = 0; hn < 2; ++hn) {
+                        const int col = bj * 16 + hn * 8 + g;
+                        const uint32_t b0 = pack_two_h(Ah[(bk * 16 + 2 * t) * P_AH + col], Ah[(bk * 16 + 2 * t + 1) * P_AH + col]);
+                        const uint32_t b1 = pack_two_h(Ah[(bk * 16 + 2 * t + 8) * P_AH + col], Ah[(bk * 16 + 2 * t + 9) * P_AH + col]);
+                        mma_m16n8k16(y[hn], a0, a1, a2, a3, b0, b1);
+                    }
+                }
+                const uint32_t a0 = pack_h2(y[0][0], y[0][1]), a1 = pack_h2(y[0][2], y[0][3]);
+                const uint32_t a2 = pack_h2(y[1][0], y[1][1]), a3 = pack_h2(y[1][2], y[1][3]);
 #pragma unroll
                 for (int hn = 0; hn < 2; ++hn) {
                     const int col = bj * 16 + hn * 8 + g;
-                    const uint32_t b0 = pack_two_h(Ah[(bk * 16 + 2 * t) * P_AH + col], Ah[(bk * 16 + 2 * t + 1) * P_AH + col]);
-                    const uint32_t b1 = pack_two_h(Ah[(bk * 16 + 2 * t + 8) * P_AH + col], Ah[(bk * 16 + 2 * t + 9) * P_AH + col]);
-                    mma_m16n8k16(y[hn], a0, a1, a2, a3, b0, b1);
+                    const uint32_t b0 = pack_two_h(Th[(bj * 16 + 2 * t) * P_AH + col], Th[(bj * 16 + 2 * t + 1) * P_AH + col]);
+                    const uint32_t b1 = pack_two_h(Th[(bj * 16 + 2 * t + 8) * P_AH + col], Th[(bj * 16 + 2 * t + 9) * P_AH + col]);
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_m16n8k16(d, a0, a1, a2, a3, b0, b1);
+                    const int c0 = bj * 16 + hn * 8 + 2 * t;
+                    const float fb0 = sBeta[c0], fb1 = sBeta[c0 + 1];
+                    const float fg0 = fb0 * sGam[c0] * sRk[c0], fg1 = fb1 * sGam[c0 + 1] * sRk[c0 + 1];
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int s = bi * 16 + g + 8 * hr;
+                        const float t0v = -d[2 * hr], t1v = -d[2 * hr + 1];
+                        const uint32_t off = swz(s, c0 >> 3) + (c0 & 7) * 2;
+                        *reinterpret_cast<uint32_t *>(Th + s * P_AH + c0) = pack_h2(t0v, t1v);
+                        *reinterpret_cast<uint32_t *>(sm + P_OFF_TPP + off) = pack_h2(t0v * fb0, t1v * fb1);
+                        *reinterpret_cast<uint32_t *>(sm + P_OFF_TP + off) = pack_h2(t0v * fg0, t1v * fg1);
+                    }
                 }
             }
-            const uint32_t a0 = pack_h2(y[0][0], y[0][1]), a1 = pack_h2(y[0][2], y[0][3]);
-            const uint32_t a2 = pack_h2(y[1][0], y[1][1]), a3 = pack_h2(y[1][2], y[1][3]);
+            asm volatile("barrier.cta.sync 1, 96;" ::: "memory");
+        }
+    } else {
+        // meanwhile warps 3-7: the Q' rows (64 + r of the [W; Q'] image) and K'' (the first two
+        // blocks of [K''; P^T]) from the raw bf16 tiles, scaled row by row with the swizzle
+        // positions unchanged, and K converted to fp16 in place (the B operand of MMA2); 2048
+        // chunks over 160 threads, in batches whose loads are issued before any store
+        const int t5 = tid - 96;
+#pragma unroll 1
+        for (int batch = 0; batch < 3; ++batch) {
+            uint4 hv[5];
+            float f[5];
 #pragma unroll
-            for (int hn = 0; hn < 2; ++hn) {
-                const int col = bj * 16 + hn * 8 + g;
-                const uint32_t b0 = pack_two_h(Th[(bj * 16 + 2 * t) * P_AH + col], Th[(bj * 16 + 2 * t + 1) * P_AH + col]);
-                const uint32_t b1 = pack_two_h(Th[(bj * 16 + 2 * t + 8) * P_AH + col], Th[(bj * 16 + 2 * t + 9) * P_AH + col]);
-                float d[4] = {0.f, 0.f, 0.f, 0.f};
-                mma_m16n8k16(d, a0, a1, a2, a3, b0, b1);
-                const int c0 = bj * 16 + hn * 8 + 2 * t;
-                const float fb0 = sBeta[c0], fb1 = sBeta[c0 + 1];
-                const float fg0 = fb0 * sGam[c0] * sRk[c0], fg1 = fb1 * sGam[c0 + 1] * sRk[c0 + 1];
+            for (int e = 0; e < 5; ++e) {
+                const int idx = (batch * 5 + e) * 160 + t5;
+                const int ic = idx < 2048 ? idx : 0;
+                const int isk = ic >> 10, w = ic & 1023, half = w >> 9, within = w & 511, r = within >> 3;
+                hv[e] = *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + (2 * half + (isk ? 0 : 1)) * TILE + within * 16);
+                f[e] = isk ? sDec[r] : sGam[r] * sRq[r];
+            }
 #pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const int s = bi * 16 + g + 8 * hr;
-                    const float t0v = -d[2 * hr], t1v = -d[2 * hr + 1];
-                    const uint32_t off = swz(s, c0 >> 3) + (c0 & 7) * 2;
-                    *reinterpret_cast<uint32_t *>(Th + s * P_AH + c0) = pack_h2(t0v, t1v);
-                    *reinterpret_cast<uint32_t *>(sm + P_OFF_TPP + off) = pack_h2(t0v * fb0, t1v * fb1);
-                    *reinterpret_cast<uint32_t *>(sm + P_OFF_TP + off) = pack_h2(t0v * fg0, t1v * fg1);
+            for (int e = 0; e < 5; ++e) {
+                const int idx = (batch * 5 + e) * 160 + t5;
+                if (idx < 2048) {
+                    const int isk = idx >> 10, w = idx & 1023, half = w >> 9, within = w & 511;
+                    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&hv[e]);
+                    float raw[8], xv[8];
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const float2 t = __bfloat1622float2(b2[q2]);
+                        raw[2 * q2] = t.x;
+                        raw[2 * q2 + 1] = t.y;
+                        xv[2 * q2] = t.x * f[e];
+                        xv[2 * q2 + 1] = t.y * f[e];
+                    }
+                    st_h8(isk ? item + kWsKP + half * TILE + within * 16 : item + kWsWQ + half * 2 * TILE + TILE + within * 16,
+                          xv);
+                    if (isk) st_h8(sm + P_OFF_KQ + 2 * half * TILE + within * 16, raw);
                 }
             }
         }
-        __syncthreads();
     }
+    __syncthreads();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
