@@ -394,7 +394,9 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     // ---- T = (I + A)^-1 (unit lower triangular), written as T (fp16, for the block products)
     //      and as the B operands T'' = T diag(beta), T' = T diag(beta gamma / |k|). Two warps
     //      solve the 16 x 16 diagonal blocks by forward substitution (fp32) while the other six
-    //      copy the P^T image out of its staging and write the zero upper blocks of T' and T''.
+    //      copy the P^T image out of its staging, write the zero upper blocks of T' and T'' and
+    //      the Q' rows (64 + r of the [W; Q'] image): the raw bf16 Q tile scaled row by row, the
+    //      swizzle positions unchanged.
     if (tid < 64) {
         const int bi = tid / 16, cc = tid % 16, o0 = bi * 16, r = o0 + cc;
         float xv[16];
@@ -416,6 +418,34 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         }
     } else {
         const int t6 = tid - 64;
+        // Q' (1024 chunks over 192 threads, loads issued before the stores)
+        {
+            uint4 hv[6];
+            float f[6];
+#pragma unroll
+            for (int e = 0; e < 6; ++e) {
+                const int idx = e * 192 + t6;
+                const int w = idx < 1024 ? idx : 0, half = w >> 9, within = w & 511, r = within >> 3;
+                hv[e] = *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + (2 * half + 1) * TILE + within * 16);
+                f[e] = sGam[r] * sRq[r];
+            }
+#pragma unroll
+            for (int e = 0; e < 6; ++e) {
+                const int idx = e * 192 + t6;
+                if (idx < 1024) {
+                    const int half = idx >> 9, within = idx & 511;
+                    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&hv[e]);
+                    float xv[8];
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const float2 t = __bfloat1622float2(b2[q2]);
+                        xv[2 * q2] = t.x * f[e];
+                        xv[2 * q2 + 1] = t.y * f[e];
+                    }
+                    st_h8(item + kWsWQ + half * 2 * TILE + TILE + within * 16, xv);
+                }
+            }
+        }
         // the P^T image from its staging (512 chunks)
         uint4 pc[3];
 #pragma unroll
@@ -490,28 +520,26 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             asm volatile("barrier.cta.sync 1, 96;" ::: "memory");
         }
     } else {
-        // meanwhile warps 3-7: the Q' rows (64 + r of the [W; Q'] image) and K'' (the first two
-        // blocks of [K''; P^T]) from the raw bf16 tiles, scaled row by row with the swizzle
-        // positions unchanged, and K converted to fp16 in place (the B operand of MMA2); 2048
-        // chunks over 160 threads, in batches whose loads are issued before any store
+        // meanwhile warps 3-7: K'' (the first two blocks of [K''; P^T]) from the raw bf16 K tile,
+        // scaled row by row with the swizzle positions unchanged, and K converted to fp16 in place
+        // (the B operand of MMA2); 1024 chunks over 160 threads, loads issued before the stores
         const int t5 = tid - 96;
 #pragma unroll 1
-        for (int batch = 0; batch < 3; ++batch) {
-            uint4 hv[5];
-            float f[5];
+        for (int batch = 0; batch < 2; ++batch) {
+            uint4 hv[4];
+            float f[4];
 #pragma unroll
-            for (int e = 0; e < 5; ++e) {
-                const int idx = (batch * 5 + e) * 160 + t5;
-                const int ic = idx < 2048 ? idx : 0;
-                const int isk = ic >> 10, w = ic & 1023, half = w >> 9, within = w & 511, r = within >> 3;
-                hv[e] = *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + (2 * half + (isk ? 0 : 1)) * TILE + within * 16);
-                f[e] = isk ? sDec[r] : sGam[r] * sRq[r];
+            for (int e = 0; e < 4; ++e) {
+                const int idx = (batch * 4 + e) * 160 + t5;
+                const int w = idx < 1024 ? idx : 0, half = w >> 9, within = w & 511, r = within >> 3;
+                hv[e] = *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + 2 * half * TILE + within * 16);
+                f[e] = sDec[r];
             }
 #pragma unroll
-            for (int e = 0; e < 5; ++e) {
-                const int idx = (batch * 5 + e) * 160 + t5;
-                if (idx < 2048) {
-                    const int isk = idx >> 10, w = idx & 1023, half = w >> 9, within = w & 511;
+            for (int e = 0; e < 4; ++e) {
+                const int idx = (batch * 4 + e) * 160 + t5;
+                if (idx < 1024) {
+                    const int half = idx >> 9, within = idx & 511;
                     const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&hv[e]);
                     float raw[8], xv[8];
 #pragma unroll
@@ -522,9 +550,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                         xv[2 * q2] = t.x * f[e];
                         xv[2 * q2 + 1] = t.y * f[e];
                     }
-                    st_h8(isk ? item + kWsKP + half * TILE + within * 16 : item + kWsWQ + half * 2 * TILE + TILE + within * 16,
-                          xv);
-                    if (isk) st_h8(sm + P_OFF_KQ + 2 * half * TILE + within * 16, raw);
+                    st_h8(item + kWsKP + half * TILE + within * 16, xv);
+                    st_h8(sm + P_OFF_KQ + 2 * half * TILE + within * 16, raw);
                 }
             }
         }
