@@ -207,7 +207,7 @@ constexpr int P_OFF_TPP = 8 * TILE;
 constexpr int P_AH = 72;                           // fp16 row pitch of A and T (144 B)
 constexpr int P_OFF_AH = 9 * TILE;                 // A fp16 [64][72]
 constexpr int P_OFF_TH = P_OFF_AH + 64 * P_AH * 2; // T fp16 [64][72]
-constexpr int P_OFF_VEC = P_OFF_TH + 64 * P_AH * 2; // G, beta, rk, rq, gamma, decS (64 each), row sums of squares (128)
+constexpr int P_OFF_VEC = P_OFF_TH + 64 * P_AH * 2; // G, beta, rk, rq, gamma, decS (64 each), spare (128)
 constexpr int P_OFF_BAR = P_OFF_VEC + 8 * 64 * 4;
 constexpr int P_SMEM = P_OFF_BAR + 64 + 1024;
 constexpr int P_OFF_STG = 0;                       // W and U~ staging once the last MMA is done (32 KB)
@@ -234,8 +234,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *vec = reinterpret_cast<float *>(sm + P_OFF_VEC);
-    float *sG = vec, *sBeta = vec + 64, *sRk = vec + 128, *sRq = vec + 192, *sGam = vec + 256, *sDec = vec + 320,
-          *sSS = vec + 384;
+    float *sG = vec, *sBeta = vec + 64, *sRk = vec + 128, *sRq = vec + 192, *sGam = vec + 256, *sDec = vec + 320;
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + P_OFF_BAR);
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 2);
@@ -621,7 +620,14 @@ teardown:
 // Chain kernel: one CTA per (value head, sequence), chunks in order, double-buffered.
 // Warps 0-7: element-wise work; warp 8: bulk copies and MMA issue.
 // ===================================================================================
-constexpr int CH_THREADS = NT + 32;
+// Output pass: 16 element-wise warps, four per tensor-memory lane quarter, each thread one state
+// row and 32 of its columns (half the per-thread work of eight warps, which shortens every
+// element-wise step of the chunk chain), plus the copy/MMA warp.
+constexpr int CH_WARPS = 16;
+constexpr int CH_WORKERS = CH_WARPS * 32;
+constexpr int CH_COLS = 128 / (CH_WARPS / 4);      // state columns per thread
+constexpr int CH_TOK = C / (CH_WARPS / 4);         // chunk tokens per thread in U and o
+constexpr int CH_THREADS = CH_WORKERS + 32;
 constexpr int CH_OFF_STAGE = 2 * kWsItem;          // o staging, [r][i] (bf16 or fp32)
 constexpr int CH_OFF_BAR = CH_OFF_STAGE + 64 * 128 * 4;
 constexpr int CH_SMEM = CH_OFF_BAR + 128 + 1024;
@@ -650,18 +656,18 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t
         "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
 
-// Barrier among the 256 element-wise threads only (named barrier 1), with an AND vote.
+// Barrier among the output pass's element-wise threads only (named barrier 1), with an AND vote.
 __device__ __forceinline__ int workers_and(int pred) {
     int r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
-        "barrier.cta.red.and.pred q, 1, 256, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
+        "barrier.cta.red.and.pred q, 1, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"(pred)
+        : "r"(pred), "n"(CH_WORKERS)
         : "memory");
     return r;
 }
-__device__ __forceinline__ void workers_sync() { asm volatile("barrier.cta.sync 2, 256;" ::: "memory"); }
+__device__ __forceinline__ void workers_sync() { asm volatile("barrier.cta.sync 2, %0;" ::"n"(CH_WORKERS) : "memory"); }
 
 // Chain modes: the full chain with outputs from a segment's true start state; a segment's
 // state from S0 (first segment) or zero, with no outputs; a segment's transition matrix,
@@ -684,6 +690,7 @@ struct ChainParams {
 };
 constexpr size_t kSegItem = kSegItemBytes;
 constexpr size_t kSegB = 0, kSegMhi = 65536, kSegMlo = 98304, kSegS = 131072;
+static_assert(kSegMlo == kSegMhi + 32768, "the combine reads M_lo right after M_hi");
 
 // Segment states (B, start states) are stored lane-interleaved: the 16-byte group c4 of the
 // 64-column half wg of row i sits at ((wg * 16 + c4) * 128 + i) * 16, so that the thread owning
@@ -704,8 +711,16 @@ __device__ __forceinline__ void ilv_store(uint8_t *base, int row, int wg, const 
         *reinterpret_cast<float4 *>(base + ilv_off(row, wg, c4)) =
             make_float4(S[4 * c4], S[4 * c4 + 1], S[4 * c4 + 2], S[4 * c4 + 3]);
 }
+// The 32-column quarter cq of row i (the same layout: 16-byte group cq * 8 + c4).
+__device__ __forceinline__ void ilv_load32(const uint8_t *base, int row, int cq, float (&S)[32]) {
+#pragma unroll
+    for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 x = *reinterpret_cast<const float4 *>(base + ((size_t)((cq * 8 + c4) * 128 + row)) * 16);
+        S[4 * c4] = x.x; S[4 * c4 + 1] = x.y; S[4 * c4 + 2] = x.z; S[4 * c4 + 3] = x.w;
+    }
+}
 // A row-major 128 x 128 fp32 state through shared memory (rows padded to 528 bytes, so both the
-// coalesced side and the row-per-thread side are free of bank conflicts); `tid` in 0..255.
+// coalesced side and the row-per-thread side are free of bank conflicts).
 constexpr int kStgPitch = 528;
 
 // FUSED: the output pass also applies the gated RMSNorm to each chunk's o rows and writes them
@@ -722,7 +737,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int h = blockIdx.x, id = blockIdx.y, mode = P.mode_base + (int)blockIdx.z;
+    const int h = blockIdx.x, id = blockIdx.y;
     const int T = P.T, Hv = P.Hv, SEG = P.seg_chunks;
     int n = 0, t_begin = 0, t_end = T;
     if (P.cu_seqlens) {
@@ -739,12 +754,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
     const int nch_seq = (t_end - t_begin + C - 1) / C;
     const int nseg = (nch_seq + SEG - 1) / SEG;
     const int pseg = id - (t_begin / (C * SEG) + n);
-    // slots no segment uses; the state and transition passes skip the last segment, the
-    // transition pass also the first (its start state is known)
-    if (pseg < 0) return;
-    if (mode == kChainFull && pseg >= (nseg > 0 ? nseg : 1)) return;
-    if (mode != kChainFull && pseg >= nseg - 1) return;
-    if (mode == kChainTransition && pseg == 0) return;
+    if (pseg < 0 || pseg >= (nseg > 0 ? nseg : 1)) return;   // a slot no segment uses
     const int c_first = pseg * SEG;
     const int nchunks = max(0, min(nch_seq, c_first + SEG) - c_first);
     const bool last_seg = pseg >= nseg - 1;
@@ -760,8 +770,8 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
         mbar_init(&full[1], 1);
         mbar_init(bar_u, 1);
         mbar_init(bar_s, 1);
-        mbar_init(bar_uready, 8);
-        mbar_init(bar_sready, 8);
+        mbar_init(bar_uready, CH_WARPS);
+        mbar_init(bar_sready, CH_WARPS);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -773,7 +783,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
+    if (warp == CH_WARPS) {
         // ------------------------------------------------ copy + MMA issue (one thread)
         if (lane == 0) {
             auto issue_chunk = [&](int c) {
@@ -788,9 +798,8 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
                 }
             };
             if (nchunks > 0) issue_chunk(0);
-            const bool full_out = mode == kChainFull;   // the output halves only when o is produced
-            const uint32_t id45 = idesc_f16(full_out ? 128 : 64, false, false, false);
-            const uint32_t id67 = idesc_f16(full_out ? 192 : 128, false, true, false);
+            const uint32_t id45 = idesc_f16(128, false, false, false);
+            const uint32_t id67 = idesc_f16(192, false, true, false);
             for (int c = 0; c < nchunks; ++c) {
                 const int b = c & 1;
                 const uint8_t *buf = sm + b * kWsItem;
@@ -818,11 +827,11 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             }
         }
     } else {
-        // ------------------------------------------------ element-wise work (256 threads)
-        const int wg = warp / 4;
+        // ------------------------------------------------ element-wise work (16 warps)
+        const int cq = warp / 4;                  // column quarter: state columns 32 cq .. 32 cq + 31
         const int row = (warp % 4) * 32 + lane;   // TMEM lane == value index i
         const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
-        float S[64];   // S[i][64 wg .. 64 wg + 63], fp32
+        float S[CH_COLS];   // S[i][32 cq .. 32 cq + 31], fp32
         // fused: this thread's eight RMSNorm weights (16 threads per o row) and the encoder table
         f2_t w2[4];
         if constexpr (FUSED) {
@@ -830,10 +839,10 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             for (int k = 0; k < 4; ++k) w2[k] = f2(P.norm_w[(tid & 15) * 8 + 2 * k], P.norm_w[(tid & 15) * 8 + 2 * k + 1]);
             nvfp4_fill_r_tab(reinterpret_cast<float *>(sm + CHF_OFF_RTAB), P.gs, tid);
         }
-        // fused: gated RMSNorm + NVFP4 encode of rows [16 p0, 16 p1) of chunk cc, whose bf16 o rows
-        // are staged; 16 threads per row, eight values each (the same arithmetic as the
+        // fused: gated RMSNorm + NVFP4 encode of chunk cc, whose bf16 o rows are staged; 16
+        // threads per row, eight values each, 32 rows per pass (the same arithmetic as the
         // standalone tail kernel); o written too when requested
-        auto epilogue = [&](int cc, int p0, int p1) {
+        auto epilogue = [&](int cc) {
             const int t0e = t_begin + (c_first + cc) * C;
             const int Le = min(C, t_end - t0e);
             const uint8_t *stage = sm + CH_OFF_STAGE;
@@ -842,8 +851,8 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             uint8_t *ob = static_cast<uint8_t *>(P.o);
             const int lr = tid & 15, col = lr * 8;
 #pragma unroll 1
-            for (int pass = p0; pass < p1; ++pass) {
-                const int r = pass * 16 + (tid >> 4);
+            for (int pass = 0; pass < C / (CH_WORKERS / 16); ++pass) {
+                const int r = pass * (CH_WORKERS / 16) + (tid >> 4);
                 const uint4 ou = *reinterpret_cast<const uint4 *>(stage + r * (D * 2) + col * 2);
                 const uint4 zu = *reinterpret_cast<const uint4 *>(zt + (col >> 6) * TILE + swz(r, (col & 63) >> 3));
                 const f2_t o2[4] = {bf16x2_to_f2(ou.x), bf16x2_to_f2(ou.y), bf16x2_to_f2(ou.z), bf16x2_to_f2(ou.w)};
@@ -860,37 +869,34 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
                 }
             }
         };
-        if (pseg == 0 && mode != kChainTransition && S0g) {
+        if (pseg == 0 && S0g) {
             // the caller's row-major initial state, staged in buffer 1 (its first chunk load is
             // issued only after every worker has released S0 through bar_sready)
             const float4 *src = reinterpret_cast<const float4 *>(S0g + ((size_t)n * Hv + h) * D * D);
             uint8_t *stg = sm + kWsItem;
 #pragma unroll 4
-            for (int e = 0; e < 16; ++e) {
-                const int f = e * NT + tid;
+            for (int e = 0; e < 4096 / CH_WORKERS; ++e) {
+                const int f = e * CH_WORKERS + tid;
                 *reinterpret_cast<float4 *>(stg + (f >> 5) * kStgPitch + (f & 31) * 16) = src[f];
             }
             workers_sync();
 #pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {
-                const float4 x = *reinterpret_cast<const float4 *>(stg + row * kStgPitch + wg * 256 + c4 * 16);
+            for (int c4 = 0; c4 < CH_COLS / 4; ++c4) {
+                const float4 x = *reinterpret_cast<const float4 *>(stg + row * kStgPitch + cq * CH_COLS * 4 + c4 * 16);
                 S[4 * c4] = x.x; S[4 * c4 + 1] = x.y; S[4 * c4 + 2] = x.z; S[4 * c4 + 3] = x.w;
             }
-        } else if (pseg > 0 && mode == kChainFull) {
-            ilv_load(seg_item + kSegS, row, wg, S);
+        } else if (pseg > 0) {
+            ilv_load32(seg_item + kSegS, row, cq, S);
         } else {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) S[c] = (mode == kChainTransition && row == 64 * wg + c) ? 1.0f : 0.0f;
+            for (int c = 0; c < CH_COLS; ++c) S[c] = 0.0f;
         }
         // fp16 copy of S as an A operand: row i on lane i, key index j two per column
         auto store_S = [&](int slot) {
+            uint32_t pk[16];
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int w = 0; w < 16; ++w) pk[w] = pack_h2(S[part * 32 + 2 * w], S[part * 32 + 2 * w + 1]);
-                tmem_st16(tmem + lane_base + C_TM_SA + slot * 64 + wg * 32 + part * 16, pk);
-            }
+            for (int w = 0; w < 16; ++w) pk[w] = pack_h2(S[2 * w], S[2 * w + 1]);
+            tmem_st16(tmem + lane_base + C_TM_SA + slot * 64 + cq * 16, pk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -912,28 +918,27 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             if (!workers_and(ok)) { alive = false; break; }
             tc_fence_after();
             {
-                // U^T = U~^T - D4 as the fp16 A operand of MMA67
+                // U^T = U~^T - D4 as the fp16 A operand of MMA67; this thread: tokens 16 cq .. + 15
                 const __half *ut = reinterpret_cast<const __half *>(buf + kWsU);
-                __half2 u2[16];
+                __half2 u2[CH_TOK / 2];
 #pragma unroll
-                for (int w = 0; w < 16; ++w) {
-                    const int s0 = wg * 32 + 2 * w;
-                    u2[w] = mode == kChainTransition ? __float2half2_rn(0.0f)
-                                                     : __halves2half2(ut[s0 * D + row], ut[(s0 + 1) * D + row]);
+                for (int w = 0; w < CH_TOK / 2; ++w) {
+                    const int s0 = cq * CH_TOK + 2 * w;
+                    u2[w] = __halves2half2(ut[s0 * D + row], ut[(s0 + 1) * D + row]);
                 }
-                uint32_t r32[32];
-                tmem_ld32(tmem + C_TM_D45 + lane_base + wg * 32, r32);
+                uint32_t r16[16];
+                tmem_ld16(tmem + C_TM_D45 + lane_base + cq * CH_TOK, r16);
                 tmem_ld_wait();
-                uint32_t ua[16];
+                uint32_t ua[8];
 #pragma unroll
-                for (int w = 0; w < 16; ++w) {
-                    const int s0 = wg * 32 + 2 * w;
+                for (int w = 0; w < CH_TOK / 2; ++w) {
+                    const int s0 = cq * CH_TOK + 2 * w;
                     const float2 uf = __half22float2(u2[w]);
-                    const float u0 = (s0 < L) ? uf.x - __uint_as_float(r32[2 * w]) : 0.0f;
-                    const float u1 = (s0 + 1 < L) ? uf.y - __uint_as_float(r32[2 * w + 1]) : 0.0f;
+                    const float u0 = (s0 < L) ? uf.x - __uint_as_float(r16[2 * w]) : 0.0f;
+                    const float u1 = (s0 + 1 < L) ? uf.y - __uint_as_float(r16[2 * w + 1]) : 0.0f;
                     ua[w] = pack_h2(u0, u1);
                 }
-                tmem_st16(tmem + lane_base + C_TM_UA + wg * 16, ua);
+                tmem_st8(tmem + lane_base + C_TM_UA + cq * (CH_TOK / 2), ua);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -942,53 +947,47 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             if (tid == 0) ok = mbar_wait(bar_s, ph, status) ? 1 : 0;
             if (!workers_and(ok)) { alive = false; break; }
             tc_fence_after();
-            float ov[32];
+            float ov[CH_TOK];
             {
-                if (mode == kChainFull) {
-                    uint32_t a5[32], b5[32];
-                    tmem_ld32(tmem + C_TM_D45 + lane_base + 64 + wg * 32, a5);
-                    tmem_ld32(tmem + C_TM_D67 + lane_base + 128 + wg * 32, b5);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) ov[j] = __uint_as_float(a5[j]) + __uint_as_float(b5[j]);
-                }
+                // o^T = D5a + D5b for tokens 16 cq .. + 15; S <- gamma_C S + D7 for this quarter
+                uint32_t a5[16], b5[16], r7[32];
+                tmem_ld16(tmem + C_TM_D45 + lane_base + 64 + cq * CH_TOK, a5);
+                tmem_ld16(tmem + C_TM_D67 + lane_base + 128 + cq * CH_TOK, b5);
+                tmem_ld32(tmem + C_TM_D67 + lane_base + cq * CH_COLS, r7);
+                tmem_ld_wait();
                 const float gC = reinterpret_cast<const float *>(buf + kWsVec)[0];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r7[32];
-                    tmem_ld32(tmem + C_TM_D67 + lane_base + wg * 64 + half * 32, r7);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) S[half * 32 + j] = gC * S[half * 32 + j] + __uint_as_float(r7[j]);
-                }
+                for (int j = 0; j < CH_COLS; ++j) S[j] = gC * S[j] + __uint_as_float(r7[j]);
                 store_S(b ^ 1);   // S0 of chunk c + 1; releases the MMA warp
+#pragma unroll
+                for (int j = 0; j < CH_TOK; ++j) ov[j] = __uint_as_float(a5[j]) + __uint_as_float(b5[j]);
             }
             if (FUSED) {
                 // stage this chunk's o rows (bf16 [r][i]; the previous chunk's encode is done, a
                 // worker barrier has passed since) and encode them
                 __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(sm + CH_OFF_STAGE);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) st[(wg * 32 + j) * D + row] = __float2bfloat16_rn(ov[j]);
+                for (int j = 0; j < CH_TOK; ++j) st[(cq * CH_TOK + j) * D + row] = __float2bfloat16_rn(ov[j]);
                 workers_sync();
-                epilogue(c, 0, 4);
-            } else if (mode == kChainFull) {
+                epilogue(c);
+            } else {
                 // o rows of this chunk: staged as [r][i], then 16-byte row stores (rows < L)
                 const int out_bf16 = P.out_bf16;
                 uint8_t *stage = sm + CH_OFF_STAGE;
                 if (out_bf16) {
                     __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(stage);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) st[(wg * 32 + j) * D + row] = __float2bfloat16_rn(ov[j]);
+                    for (int j = 0; j < CH_TOK; ++j) st[(cq * CH_TOK + j) * D + row] = __float2bfloat16_rn(ov[j]);
                 } else {
                     float *st = reinterpret_cast<float *>(stage);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) st[(wg * 32 + j) * D + row] = ov[j];
+                    for (int j = 0; j < CH_TOK; ++j) st[(cq * CH_TOK + j) * D + row] = ov[j];
                 }
                 workers_sync();
                 const int row_bytes = out_bf16 ? D * 2 : D * 4;
                 const int per_row = row_bytes / 16;
                 uint8_t *ob = static_cast<uint8_t *>(P.o);
-                for (int e = tid; e < L * per_row; e += NT) {
+                for (int e = tid; e < L * per_row; e += CH_WORKERS) {
                     const int r = e / per_row, ch = e % per_row;
                     const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + ch * 16);
                     *reinterpret_cast<uint4 *>(ob + (((size_t)(t0 + r) * Hv + h) * D) * (row_bytes / D) + ch * 16) = val;
@@ -996,46 +995,19 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
                 workers_sync();
             }
         }
-        if (alive) {
-            // all chunks are consumed: both operand buffers are free for staging
-            if (mode == kChainFull && last_seg && P.S_out) {
-                uint8_t *stg = sm;
+        if (alive && last_seg && P.S_out) {
+            // all chunks are consumed: both operand buffers are free for staging the final state
+            uint8_t *stg = sm;
 #pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4)
-                    *reinterpret_cast<float4 *>(stg + row * kStgPitch + wg * 256 + c4 * 16) =
-                        make_float4(S[4 * c4], S[4 * c4 + 1], S[4 * c4 + 2], S[4 * c4 + 3]);
-                workers_sync();
-                float4 *dst = reinterpret_cast<float4 *>(P.S_out + ((size_t)n * Hv + h) * D * D);
+            for (int c4 = 0; c4 < CH_COLS / 4; ++c4)
+                *reinterpret_cast<float4 *>(stg + row * kStgPitch + cq * CH_COLS * 4 + c4 * 16) =
+                    make_float4(S[4 * c4], S[4 * c4 + 1], S[4 * c4 + 2], S[4 * c4 + 3]);
+            workers_sync();
+            float4 *dst = reinterpret_cast<float4 *>(P.S_out + ((size_t)n * Hv + h) * D * D);
 #pragma unroll 4
-                for (int e = 0; e < 16; ++e) {
-                    const int f = e * NT + tid;
-                    dst[f] = *reinterpret_cast<const float4 *>(stg + (f >> 5) * kStgPitch + (f & 31) * 16);
-                }
-            } else if (mode == kChainState) {
-                ilv_store(const_cast<uint8_t *>(seg_item) + kSegB, row, wg, S);
-            } else if (mode == kChainTransition) {
-                // the segment's map M (row j = this lane) as fp16 hi / lo B operand images,
-                // MN-major over the output column, 128-byte swizzled rows: built in shared
-                // memory, then copied out in 16-byte chunks
-                uint8_t *mhi = sm + wg * 16384, *mlo = sm + 32768 + wg * 16384;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float hi8[8], lo8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const float2 hf = __half22float2(__floats2half2_rn(S[ch * 8 + e], S[ch * 8 + e + 1]));
-                        hi8[e] = hf.x;
-                        hi8[e + 1] = hf.y;
-                        lo8[e] = S[ch * 8 + e] - hf.x;
-                        lo8[e + 1] = S[ch * 8 + e + 1] - hf.y;
-                    }
-                    st_h8(mhi + swz(row, ch), hi8);
-                    st_h8(mlo + swz(row, ch), lo8);
-                }
-                workers_sync();
-                uint4 *dst = reinterpret_cast<uint4 *>(const_cast<uint8_t *>(seg_item) + kSegMhi);
-#pragma unroll 4
-                for (int e = 0; e < 16; ++e) dst[e * NT + tid] = reinterpret_cast<const uint4 *>(sm)[e * NT + tid];
+            for (int e = 0; e < 4096 / CH_WORKERS; ++e) {
+                const int f = e * CH_WORKERS + tid;
+                dst[f] = *reinterpret_cast<const float4 *>(stg + (f >> 5) * kStgPitch + (f & 31) * 16);
             }
         }
     }
