@@ -272,8 +272,149 @@ gdn_recurrent128_kernel(const void *__restrict__ q, const void *__restrict__ k, 
     }
 }
 
+// Draft verify in the chunk (WY) form: outputs for the T <= 8 draft tokens of each sequence from
+// the state S0, which is only read. With unit keys k^_t, queries q^_t (scale included), decay
+// gamma_t = alpha_1 ... alpha_t and c_st = gamma_t / gamma_s (a product of alphas), the token-by-token
+// rule S_t = alpha_t S_{t-1} + u_t k^_t^T, u_t = beta_t (v_t - alpha_t S_{t-1} k^_t), unrolls to
+//     S_{t-1} k^_t = gamma_{t-1} S0 k^_t + sum_{s<t} c_{s,t-1} u_s (k^_s . k^_t),
+//     o_t = S_t q^_t = gamma_t S0 q^_t + sum_{s<=t} c_{s,t} u_s (k^_s . q^_t),
+// so each state row needs only the 2 T products S0 k_t and S0 q_t (independent of one another,
+// no state update) and T x T scalars shared by the CTA (the Gram dots of the tokens' keys and
+// queries), instead of T dependent rank-one updates.
+constexpr int kVerifyMaxT = 8;
+
+template <bool IN_BF16, bool OUT_BF16>
+__global__ void __launch_bounds__(kR128Threads)
+gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
+                     const float *__restrict__ a, const float *__restrict__ b, const float *__restrict__ A_log,
+                     const float *__restrict__ dt_bias, int32_t T, int32_t Hk, int32_t Hv, float scale,
+                     int32_t l2norm, const float *__restrict__ S0, void *__restrict__ o) {
+    pdl_launch_dependents();
+    pdl_wait();
+    constexpr int D = 128;
+    const int slice = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+    const int hk = h / (Hv / Hk);
+    const int tid = threadIdx.x, l8 = tid & 7, grp = tid >> 3;
+    const int rbase = slice * 64 + grp;
+    const int t0 = n * T;
+    const size_t sbase = ((size_t)n * Hv + h) * D * D;
+    __shared__ float s_kk[kVerifyMaxT][kVerifyMaxT], s_kq[kVerifyMaxT][kVerifyMaxT];
+    __shared__ float s_qq[kVerifyMaxT], s_alpha[kVerifyMaxT], s_beta[kVerifyMaxT];
+
+    f2_t s[4][8];
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 x = __ldcs(reinterpret_cast<const float4 *>(S0 + sbase + (size_t)(rbase + 16 * p) * D + 32 * j + 4 * l8));
+            s[p][2 * j] = f2(x.x, x.y);
+            s[p][2 * j + 1] = f2(x.z, x.w);
+        }
+
+    // Gram dots of the tokens' raw keys and queries (k_s.k_t and k_s.q_t for s <= t, q_t.q_t),
+    // one 8-lane group per dot, and the gates
+    const int nkk = T * (T + 1) / 2, ndots = 2 * nkk + T;
+    // every lane runs the same number of rounds (the shuffles below take whole warps)
+    for (int base = 0; base < ndots; base += kR128Threads / 8) {
+        const bool live = base + grp < ndots;
+        const int d = live ? base + grp : 0;
+        int kind = d < nkk ? 0 : (d < 2 * nkk ? 1 : 2), e = kind == 0 ? d : (kind == 1 ? d - nkk : d - 2 * nkk);
+        int ss = 0, tt = e;
+        if (kind < 2) {   // e -> (s, t), s <= t, row-major over t
+            tt = 0;
+            while ((tt + 1) * (tt + 2) / 2 <= e) ++tt;
+            ss = e - tt * (tt + 1) / 2;
+        }
+        f2_t x2[8], y2[8];
+        load_cols16<IN_BF16>(kind == 2 ? q : k, ((size_t)(t0 + (kind == 2 ? tt : ss)) * Hk + hk) * D, l8, x2);
+        load_cols16<IN_BF16>(kind == 0 ? k : q, ((size_t)(t0 + tt) * Hk + hk) * D, l8, y2);
+        float part = dot16(x2, y2);
+        part += __shfl_xor_sync(kFull, part, 4);
+        part += __shfl_xor_sync(kFull, part, 2);
+        part += __shfl_xor_sync(kFull, part, 1);
+        if (live && l8 == 0) {
+            if (kind == 0) s_kk[ss][tt] = part;
+            else if (kind == 1) s_kq[ss][tt] = part;
+            else s_qq[tt] = part;
+        }
+    }
+    if (tid < T) {
+        float g, beta;
+        gdn_gates(a[(size_t)(t0 + tid) * Hv + h], b[(size_t)(t0 + tid) * Hv + h], A_log[h], dt_bias[h], g, beta);
+        s_alpha[tid] = expf(g);
+        s_beta[tid] = beta;
+    }
+
+    // S0 k_t and S0 q_t for this thread's four rows, reduced over the row's eight lanes: lanes
+    // whose bits 2 and 1 are (p >> 1, p & 1) hold row p's totals
+    float xk[kVerifyMaxT], xq[kVerifyMaxT];
+#pragma unroll
+    for (int t = 0; t < kVerifyMaxT; ++t) {
+        xk[t] = 0.0f;
+        xq[t] = 0.0f;
+        if (t < T) {
+            f2_t k2[8], q2[8];
+            load_cols16<IN_BF16>(k, ((size_t)(t0 + t) * Hk + hk) * D, l8, k2);
+            load_cols16<IN_BF16>(q, ((size_t)(t0 + t) * Hk + hk) * D, l8, q2);
+            float pk[4], pq[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                pk[p] = dot16(s[p], k2);
+                pq[p] = dot16(s[p], q2);
+            }
+            xk[t] = group8_sum4_t(pk, l8);
+            xq[t] = group8_sum4_t(pq, l8);
+        }
+    }
+    __syncthreads();
+
+    // per row: the T x T recurrence on the projections (lanes with l8 even own one row each)
+    const int prow = 2 * ((l8 >> 2) & 1) + ((l8 >> 1) & 1);
+    const int row = rbase + 16 * prow;
+    float kn[kVerifyMaxT], u[kVerifyMaxT], c[kVerifyMaxT];
+#pragma unroll
+    for (int t = 0; t < kVerifyMaxT; ++t) {
+        if (t >= T) break;
+        kn[t] = l2norm ? rsqrtf(s_kk[t][t] + 1e-6f) : 1.0f;
+        const float qn = l2norm ? rsqrtf(s_qq[t] + 1e-6f) * scale : scale;
+        const float alpha = s_alpha[t], beta = s_beta[t];
+        // c[s] = gamma_{t-1} / gamma_s before the update; gamma_{t-1} itself is c_{-1}
+        float proj = 0.0f, gam_prev = 1.0f;
+#pragma unroll
+        for (int r = 0; r < kVerifyMaxT; ++r)
+            if (r < t) proj += c[r] * u[r] * (kn[r] * kn[t] * s_kk[r][t]);
+#pragma unroll
+        for (int r = 0; r < kVerifyMaxT; ++r)
+            if (r < t) gam_prev *= s_alpha[r];
+        proj += gam_prev * kn[t] * xk[t];
+        const float vv = load1<IN_BF16>(v, ((size_t)(t0 + t) * Hv + h) * D + row);
+        u[t] = beta * (vv - alpha * proj);
+#pragma unroll
+        for (int r = 0; r < kVerifyMaxT; ++r)
+            if (r < t) c[r] *= alpha;
+        c[t] = 1.0f;
+        const float gam = gam_prev * alpha;
+        float ot = gam * qn * xq[t];
+#pragma unroll
+        for (int r = 0; r < kVerifyMaxT; ++r)
+            if (r <= t) ot += c[r] * u[r] * (kn[r] * qn * s_kq[r][t]);
+        if ((l8 & 1) == 0) store1<OUT_BF16>(o, ((size_t)(t0 + t) * Hv + h) * D + row, ot);
+    }
+}
+
+template <bool IN_BF16, bool OUT_BF16>
+static cudaError_t launch_verify128_t(const RecurrentArgs &r, cudaStream_t st) {
+    dim3 grid(2, r.Hv, r.num_seqs);
+    return launch_pdl(gdn_verify128_kernel<IN_BF16, OUT_BF16>, grid, dim3(kR128Threads), 0, st, r.q, r.k, r.v, r.a,
+                      r.b, r.A_log, r.dt_bias, r.tokens_per_seq, r.Hk, r.Hv, r.scale, r.l2norm, r.S0, r.o);
+}
+
 template <bool IN_BF16, bool OUT_BF16>
 static cudaError_t launch_recurrent128_t(const RecurrentArgs &r, cudaStream_t st) {
+    // outputs only, from a given state, for 2..8 tokens per sequence: the chunk form
+    if (!r.cu_seqlens && !r.S_out && r.o && r.S0 && !r.n_apply && r.tokens_per_seq >= 2 &&
+        r.tokens_per_seq <= kVerifyMaxT)
+        return launch_verify128_t<IN_BF16, OUT_BF16>(r, st);
     dim3 grid(2, r.Hv, r.num_seqs);
     return launch_pdl(gdn_recurrent128_kernel<IN_BF16, OUT_BF16>, grid, dim3(kR128Threads), 0, st, r.q, r.k, r.v,
                       r.a, r.b, r.A_log, r.dt_bias, r.cu_seqlens, r.tokens_per_seq, r.Hk, r.Hv, r.scale, r.l2norm,

@@ -59,6 +59,35 @@ def test_verify_matches_recurrence(g, B, T, Hk, Hv, D, io):
     assert torch.equal(S, S_before)
 
 
+@pytest.mark.parametrize("T,io,l2norm", [(2, "bf16", True), (3, "f32", True), (4, "bf16", True), (8, "bf16", True),
+                                         (5, "f32", False)])
+def test_verify_outputs_only_matches_recurrence(g, T, io, l2norm):
+    """Verify without a final state (d = 128, 2..8 tokens: the chunk-form kernel): every output
+    against the oracle's token-by-token recurrence, the state untouched, and against the
+    token-by-token kernel (the same call with a final state)."""
+    B, Hk, Hv, D = 9, 2, 4, 128
+    x, t, S = _setup(B, T, Hk, Hv, D, seed=300 + T, io=io)
+    scale = 1.0 if l2norm else 0.125
+    if not l2norm:   # raw q and k: keep the products of unit scale
+        for key in ("q", "k"):
+            t[key] = t[key] / float(np.sqrt(D))
+            x[key] = to_np(t[key].float()).reshape(x[key].shape)
+    S_before = S.clone()
+    o = g.gdn_decode_verify(t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], S, scale=scale,
+                            qk_l2norm=l2norm, out_dtype=torch.float32)
+    S_all = torch.empty_like(S)
+    o_seq = g.gdn_decode_verify(t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], S, scale=scale,
+                                qk_l2norm=l2norm, final_state=S_all, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert g.gdn_get_device_status() == 0
+    assert torch.equal(S, S_before)
+    o_ref, _ = oracle.gdn_scan(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                               cu_seqlens=x["cu_seqlens"], initial_state=x["initial_state"], scale=scale,
+                               qk_l2norm=l2norm)
+    assert rel_err(to_np(o).reshape(o_ref.shape), o_ref) <= TOL_SCAN
+    assert rel_err(to_np(o), to_np(o_seq)) <= TOL_SCAN
+
+
 def test_commit_takes_the_accepted_prefix(g):
     B, T, Hk, Hv, D = 7, 6, 2, 4, 128
     x, t, S = _setup(B, T, Hk, Hv, D, seed=77)
