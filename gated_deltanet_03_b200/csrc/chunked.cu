@@ -20,15 +20,17 @@
 // memory; the state itself stays fp32 in registers.
 //
 // Every MMA has M = 128 (value or key index on the TMEM lanes):
-//   prep   MMA1  D1 = [K; Q] [K; Q]^T      (rows 0-63: K K^T | K Q^T)
-//          MMA2  D2 = W^T  = K^T T'^T      T'  = T diag(beta gamma / |k|)
-//          MMA3  D3 = U~^T = V^T T''^T     T'' = T diag(beta)
+//   prep   MMA1  D1 = [K; Q] [K; Q]^T      on the raw bf16 tiles (rows 0-63: K K^T | K Q^T,
+//                                          rows 64-127: Q K^T | Q Q^T; the diagonals give the norms)
+//          MMA2  D2 = [T'; T''] [K | V]    rows 0-63: W = T' K, rows 64-127: U~ = T'' V, with
+//                                          T' = T diag(beta gamma / |k|), T'' = T diag(beta)
 //   chain  MMA45 [D4 | D5a] = S0 [W; Q']^T            Q' = diag(gamma scale / |q|) Q
 //          MMA67 [D7 | D5b] = U^T [K''; P^T]^T        K'' = diag(gamma_C / gamma / |k|) K
 //                                                     P^T[s][r] = k_s.q_r Gamma_rs scale / (|q_r| |k_s|)
 //   with U^T = U~^T - D4, S <- gamma_C S + D7, o^T = D5a + D5b. In the chain the fp16 copies of
-//   S0 and U live in tensor memory as the A operands; one warp issues the copies and MMAs,
-//   eight warps do the element-wise work, and they hand over through mbarriers.
+//   S0 and U live in tensor memory as the A operands; the element-wise warps (sixteen in the
+//   output pass, beside one copy/MMA warp; eight in the lean pass, one of whose threads issues)
+//   hand over to the issuing thread through mbarriers.
 //
 // Workspace: one 73 KB item per (value head, chunk slot): [W; Q'] (fp16, K-major, 128 rows,
 // 128-byte swizzled), [K''; P^T] (fp16, three 64-wide MN-major blocks), U~ (fp16 [s][i]) and
