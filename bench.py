@@ -541,6 +541,8 @@ def run_only(args):
     bf, f32 = torch.bfloat16, torch.float32
     if args.only == "gemm_long":
         return run_gemm_long(args)
+    if args.only == "verify":
+        return run_verify(args)
     names = {wl.name: wl for wl in workloads.WORKLOADS}
     w = names[args.workload] if args.workload else (workloads.DECODE_B256 if args.only in ("decode", "conv_decode")
                                                     else workloads.PREFILL_1K)
@@ -635,6 +637,47 @@ def run_gemm_long(args):
                       "TFLOP/s": 2.0 * gM * gN * gK / (ms / 1e3) / 1e12, "steps": args.steps}))
 
 
+def run_verify(args):
+    """Draft verify alone on the batched-decode shape (256 sequences x 4 draft tokens, 16/32
+    heads, d = 128, state read only), `warmup` + `steps` launches, L2 flushed between."""
+    import torch
+
+    import gated_deltanet_03_b200 as g
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    dw, mT = workloads.DECODE_B256, 4
+    mw = workloads.custom("verify_B%d_T%d" % (dw.num_seqs, mT), (mT,) * dw.num_seqs, dw.Hk, dw.Hv, dw.D,
+                          s0_std=0.1, seed=dw.seed)
+    mx = workloads.generate(mw)
+    B, bf, f32 = dw.num_seqs, torch.bfloat16, torch.float32
+
+    def up(a, dt):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+
+    q = up(mx["q"], bf).view(B, mT, dw.Hk, dw.D)
+    k = up(mx["k"], bf).view(B, mT, dw.Hk, dw.D)
+    v = up(mx["v"], bf).view(B, mT, dw.Hv, dw.D)
+    a, b = up(mx["a"], f32).view(B, mT, dw.Hv), up(mx["b"], f32).view(B, mT, dw.Hv)
+    A_log, dt_bias, state = up(mx["A_log"], f32), up(mx["dt_bias"], f32), up(mx["initial_state"], f32)
+    o = torch.empty((B, mT, dw.Hv, dw.D), dtype=bf, device=dev)
+    flush = make_l2_flush(torch, dev)
+    for _ in range(args.warmup):
+        g.gdn_decode_verify(q, k, v, a, b, A_log, dt_bias, state, o=o)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.gdn_decode_verify(q, k, v, a, b, A_log, dt_bias, state, o=o)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    assert g.gdn_get_device_status() == 0
+    print(json.dumps({"only": "verify", "workload": mw.name, "ms_median": statistics.median(times),
+                      "steps": args.steps}))
+
+
 # ----------------------------------------------------------------- CPU arm ----
 
 def cpu_pass(w, x, units=None):
@@ -703,7 +746,8 @@ def main():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
-    p.add_argument("--only", choices=["scan", "tail", "gemm", "gemm_long", "decode", "fused", "conv", "conv_decode"],
+    p.add_argument("--only", choices=["scan", "tail", "gemm", "gemm_long", "decode", "verify", "fused", "conv",
+                                      "conv_decode"],
                    help="time one kernel alone on its workload (for profiling); prints one JSON line")
     p.add_argument("--workload", default=None, help="workload name for --only scan (default: 1024-wide prefill)")
     args = p.parse_args()
