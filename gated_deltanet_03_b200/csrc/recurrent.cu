@@ -345,6 +345,13 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
         s_beta[tid] = beta;
     }
 
+    // the row this lane finishes (below) and its v values, loaded ahead of the dependent recurrence
+    const int prow = 2 * ((l8 >> 2) & 1) + ((l8 >> 1) & 1);
+    const int row = rbase + 16 * prow;
+    float vrow[kVerifyMaxT];
+#pragma unroll
+    for (int t = 0; t < kVerifyMaxT; ++t)
+        vrow[t] = t < T ? load1<IN_BF16>(v, ((size_t)(t0 + t) * Hv + h) * D + row) : 0.0f;
     // S0 k_t and S0 q_t for this thread's four rows, reduced over the row's eight lanes: lanes
     // whose bits 2 and 1 are (p >> 1, p & 1) hold row p's totals
     float xk[kVerifyMaxT], xq[kVerifyMaxT];
@@ -369,8 +376,6 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
     __syncthreads();
 
     // per row: the T x T recurrence on the projections (lanes with l8 even own one row each)
-    const int prow = 2 * ((l8 >> 2) & 1) + ((l8 >> 1) & 1);
-    const int row = rbase + 16 * prow;
     float kn[kVerifyMaxT], u[kVerifyMaxT], c[kVerifyMaxT];
 #pragma unroll
     for (int t = 0; t < kVerifyMaxT; ++t) {
@@ -387,8 +392,7 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
         for (int r = 0; r < kVerifyMaxT; ++r)
             if (r < t) gam_prev *= s_alpha[r];
         proj += gam_prev * kn[t] * xk[t];
-        const float vv = load1<IN_BF16>(v, ((size_t)(t0 + t) * Hv + h) * D + row);
-        u[t] = beta * (vv - alpha * proj);
+        u[t] = beta * (vrow[t] - alpha * proj);
 #pragma unroll
         for (int r = 0; r < kVerifyMaxT; ++r)
             if (r < t) c[r] *= alpha;
