@@ -620,7 +620,7 @@ teardown:
 
 // ===================================================================================
 // Chain kernel: one CTA per (value head, sequence), chunks in order, double-buffered.
-// Warps 0-7: element-wise work; warp 8: bulk copies and MMA issue.
+// Warps 0-15: element-wise work; warp 16: bulk copies and MMA issue.
 // ===================================================================================
 // Output pass: 16 element-wise warps, four per tensor-memory lane quarter, each thread one state
 // row and 32 of its columns (half the per-thread work of eight warps, which shortens every
