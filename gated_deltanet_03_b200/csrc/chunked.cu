@@ -239,7 +239,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     float *sG = vec, *sBeta = vec + 64, *sRk = vec + 128, *sRq = vec + 192, *sGam = vec + 256, *sDec = vec + 320;
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + P_OFF_BAR);
     uint64_t *bar_mma = bar_tma + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 2);
+    uint64_t *bar_v = bar_tma + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 3);
     __half *Ah = reinterpret_cast<__half *>(sm + P_OFF_AH);
     __half *Th = reinterpret_cast<__half *>(sm + P_OFF_TH);
 
@@ -251,14 +252,18 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_v, 1);
         fence_barrier_init();
-        mbar_arrive_expect_tx(bar_tma, 6 * TILE);
+        // K and Q on one barrier (MMA1 starts when they land), V on its own (not needed before
+        // the inverse's off-diagonal phase)
+        mbar_arrive_expect_tx(bar_tma, 4 * TILE);
         tma_load_3d(sm + P_OFF_KQ + 0 * TILE, &maps.k, bar_tma, 0, hk, t0);
         tma_load_3d(sm + P_OFF_KQ + 1 * TILE, &maps.q, bar_tma, 0, hk, t0);
         tma_load_3d(sm + P_OFF_KQ + 2 * TILE, &maps.k, bar_tma, 64, hk, t0);
         tma_load_3d(sm + P_OFF_KQ + 3 * TILE, &maps.q, bar_tma, 64, hk, t0);
-        tma_load_3d(sm + P_OFF_VLO, &maps.v, bar_tma, 0, h, t0);
-        tma_load_3d(sm + P_OFF_VHI, &maps.v, bar_tma, 64, h, t0);
+        mbar_arrive_expect_tx(bar_v, 2 * TILE);
+        tma_load_3d(sm + P_OFF_VLO, &maps.v, bar_v, 0, h, t0);
+        tma_load_3d(sm + P_OFF_VHI, &maps.v, bar_v, 64, h, t0);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 256);
@@ -283,7 +288,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     const uint32_t tmem = *tmem_slot;
     if (tid >= 32 && tid < 64) sG[tid] += sG[31];
 
-    int ok = 1;
+    int ok = 1, okv = 1;
     if (tid == 0) {
         ok = mbar_wait(bar_tma, 0, status) ? 1 : 0;
         if (ok) {
@@ -301,12 +306,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         }
     }
     if (!__syncthreads_and(ok)) goto teardown;
-    // while MMA1 runs: V to fp16 in place (MMA1 reads only the K and Q tiles), decay factors
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int idx = e * NT + tid;
-        convert16(sm + P_OFF_VLO + (idx >> 9) * 2 * TILE + (idx & 511) * 16);
-    }
+    // while MMA1 runs: the decay factors
     if (tid < 64) sGam[tid] = tid < L ? expf(sG[tid]) : 0.0f;
     if (tid == 0) {
         float *wv = reinterpret_cast<float *>(item + kWsVec);
@@ -521,10 +521,16 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             asm volatile("barrier.cta.sync 1, 96;" ::: "memory");
         }
     } else {
-        // meanwhile warps 3-7: K'' (the first two blocks of [K''; P^T]) from the raw bf16 K tile,
-        // scaled row by row with the swizzle positions unchanged, and K converted to fp16 in place
-        // (the B operand of MMA2); 1024 chunks over 160 threads, loads issued before the stores
+        // meanwhile warps 3-7: V converted to fp16 in place once its tiles have landed, then K''
+        // (the first two blocks of [K''; P^T]) from the raw bf16 K tile, scaled row by row with the
+        // swizzle positions unchanged, and K converted to fp16 in place (V and K are the B operand
+        // of MMA2); 1024 chunks over 160 threads, loads issued before the stores
         const int t5 = tid - 96;
+        okv = mbar_wait(bar_v, 0, status) ? 1 : 0;
+        if (okv) {
+            for (int idx = t5; idx < 1024; idx += 160)
+                convert16(sm + P_OFF_VLO + (idx >> 9) * 2 * TILE + (idx & 511) * 16);
+        }
 #pragma unroll 1
         for (int batch = 0; batch < 2; ++batch) {
             uint4 hv[4];
@@ -557,7 +563,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             }
         }
     }
-    __syncthreads();
+    if (!__syncthreads_and(okv)) goto teardown;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
