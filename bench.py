@@ -55,7 +55,7 @@ FP4_PROBE_TFLOPS = 2.0 * 16368 * 148 * 1.965e9 / 1e12
 # kernel source it was taken on (first 16 hex digits of its sha256).
 # DRAM bytes of one fused prefill call (prep + lean + combine + the output pass with the gated
 # tail), from one ncu capture with cold caches, keyed by the digest of the scan's source
-SCAN_TRAFFIC = {"9938c96fc4d676a6": 236.68e6}
+SCAN_TRAFFIC = {"8d0ca4422ce4682c": 237.57e6}
 
 
 def source_digest(path: str) -> str:
