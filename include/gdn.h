@@ -282,7 +282,7 @@ GDN_API gdn_status gdn_short_conv1d_silu_decode(const void *x, int64_t ldx, cons
                                                 gdn_stream_t stream);
 
 /* ------------------------------------------------- allocation-free prefill ----
- * No counterpart in the paper. For callers that cannot allocate device memory - code that
+ * No counterpart in the pages this library follows. For callers that cannot allocate device memory - code that
  * runs where cudaMalloc is unavailable or not allowed, or a host framework that owns every
  * allocation - this is gdn_prefill_chunked without the workspace argument: same inputs,
  * outputs, layouts and status codes. The tensor-core path uses a fixed scratch array inside
