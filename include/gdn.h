@@ -282,9 +282,9 @@ GDN_API gdn_status gdn_short_conv1d_silu_decode(const void *x, int64_t ldx, cons
                                                 gdn_stream_t stream);
 
 /* ------------------------------------------------- allocation-free prefill ----
- * No counterpart in the pages this library follows. For callers that cannot allocate device memory - code that
- * runs where cudaMalloc is unavailable or not allowed, or a host framework that owns every
- * allocation - this is gdn_prefill_chunked without the workspace argument: same inputs,
+ * No counterpart in the pages this library follows. For callers that cannot allocate device
+ * memory - code that runs where cudaMalloc is unavailable or not allowed, or a host framework
+ * that owns every allocation - this is gdn_prefill_chunked without the workspace argument: same inputs,
  * outputs, layouts and status codes. The tensor-core path uses a fixed scratch array inside
  * the library instead: 32 MiB (33554432 bytes), held on every GPU that loads the library
  * until the process exits. Sizes whose workspace (gdn_prefill_workspace_bytes) exceeds
