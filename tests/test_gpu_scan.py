@@ -80,6 +80,44 @@ def test_prefill_varlen_ragged(g):
     np.testing.assert_array_equal(S[4], x["initial_state"][4])
 
 
+_DEGENERATE = ["alpha1_beta1", "alpha1_beta0", "same_key_beta1", "same_key", "strong_decay",
+               "keys_in_4_directions"]
+
+
+@pytest.mark.parametrize("case", _DEGENERATE)
+def test_prefill_degenerate_gates(g, case):
+    """The gates at their limits and keys that repeat: alpha -> 1 (A_log = -30, no decay),
+    beta -> 1 (b = 20, each write replaces what the state held along k) or beta -> 0 (b = -20,
+    no write), one key for every token, decay of about e^-80 per token (every chunk's exp(G)
+    underflows), and keys drawn from four directions plus unit noise. Five 64-token chunks and
+    a ragged tail, nonzero initial state."""
+    w = workloads.custom("g", (300,), 2, 4, 128, io="bf16", s0_std=0.1, seed=300 + _DEGENERATE.index(case))
+    x = workloads.generate(w)
+    rng = np.random.default_rng(17)
+    T, Hk = x["k"].shape[0], x["k"].shape[1]
+    if case.startswith("alpha1"):
+        x["A_log"][:] = -30.0
+        x["b"][:] = 20.0 if case == "alpha1_beta1" else -20.0
+    elif case.startswith("same_key"):
+        x["k"][:] = workloads.round_bf16(np.broadcast_to(rng.standard_normal((1, Hk, 128)), x["k"].shape))
+        if case == "same_key_beta1":
+            x["A_log"][:] = -30.0
+            x["b"][:] = 20.0
+    elif case == "strong_decay":
+        x["a"][:] = 5.0
+        x["A_log"][:] = np.log(16.0)
+    else:
+        basis = rng.standard_normal((4, Hk, 128))
+        pick = rng.integers(0, 4, size=T)
+        x["k"][:] = workloads.round_bf16(basis[pick] + rng.standard_normal(x["k"].shape))
+        x["A_log"][:] = -30.0
+        x["b"][:] = 20.0
+    o_ref, S_ref = _full_oracle(x)
+    o, S = _run_prefill(g, x, w, torch.float32)
+    assert rel_err(o, o_ref) <= TOL_SCAN, rel_err(o, o_ref)
+    assert rel_err(S, S_ref) <= TOL_SCAN, rel_err(S, S_ref)
+
+
 def test_prefill_empty_batch_copies_state(g):
     w = workloads.custom("e", (0,), 1, 1, 128, io="bf16", s0_std=0.1, seed=3)
     x = workloads.generate(w)
