@@ -121,6 +121,31 @@ def _contig(*ts):
             raise ValueError("tensors must be contiguous")
 
 
+_F32, _I32, _U8 = (torch.float32,), (torch.int32,), (torch.uint8,)
+_IO = (torch.bfloat16, torch.float32)
+
+
+def _args(device, **named):
+    """Host-side checks before any launch, so that no kernel reads memory it was not given: a
+    (dtypes, min_elems) pair after a tensor checks its dtype and that it holds at least the
+    elements the call reads or writes (all tensors first), then every tensor must be a CUDA
+    tensor on `device`."""
+    given = [(name,) + (spec if isinstance(spec, tuple) else (spec, None, None)) for name, spec in named.items()]
+    given = [x for x in given if x[1] is not None]
+    for name, t, dtypes, need in given:
+        if not isinstance(t, torch.Tensor):
+            raise TypeError("%s must be a torch.Tensor" % name)
+        if dtypes is not None and t.dtype not in dtypes:
+            raise TypeError("%s must be %s (got %s)" % (name, " or ".join(map(str, dtypes)), t.dtype))
+        if need is not None and t.numel() < need:
+            raise ValueError("%s holds %d elements, the call needs %d" % (name, t.numel(), need))
+    for name, t, _, _ in given:
+        if t.device.type != "cuda":
+            raise ValueError("%s must be a CUDA tensor (got %s)" % (name, t.device))
+        if t.device != device:
+            raise ValueError("%s is on %s, the call's other tensors on %s" % (name, t.device, device))
+
+
 def gdn_prefill_workspace_bytes(T, num_seqs, Hk, Hv, Dk, Dv) -> int:
     return int(LIB.gdn_prefill_workspace_bytes(T, num_seqs, Hk, Hv, Dk, Dv))
 
@@ -135,6 +160,11 @@ def gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, initial_
     Hv, Dv = v.shape[1], v.shape[2]
     N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
     out_dtype = out_dtype or q.dtype
+    _args(q.device, q=(q, _IO, None), k=(k, (q.dtype,), T * Hk * Dk), v=(v, (q.dtype,), T * Hv * Dv),
+          a=(a, _F32, T * Hv), b=(b, _F32, T * Hv), A_log=(A_log, _F32, Hv), dt_bias=(dt_bias, _F32, Hv),
+          cu_seqlens=(cu_seqlens, _I32, None), initial_state=(initial_state, _F32, N * Hv * Dv * Dk),
+          final_state=(final_state, _F32, N * Hv * Dv * Dk), o=(o, _IO, T * Hv * Dv),
+          workspace=(workspace, _U8, None))
     if o is None:
         o = torch.empty((T, Hv, Dv), dtype=out_dtype, device=q.device)
     if final_state is None:
@@ -163,6 +193,12 @@ def gdn_prefill_chunked_gated_nvfp4(q, k, v, a, b, A_log, dt_bias, z, norm_weigh
     T, Hk, Dk = q.shape
     Hv, Dv = v.shape[1], v.shape[2]
     N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _args(q.device, q=(q, _IO, None), k=(k, (q.dtype,), T * Hk * Dk), v=(v, (q.dtype,), T * Hv * Dv),
+          a=(a, _F32, T * Hv), b=(b, _F32, T * Hv), A_log=(A_log, _F32, Hv), dt_bias=(dt_bias, _F32, Hv),
+          z=(z, (q.dtype,), T * Hv * Dv), norm_weight=(norm_weight, _F32, Dv),
+          cu_seqlens=(cu_seqlens, _I32, None), initial_state=(initial_state, _F32, N * Hv * Dv * Dk),
+          final_state=(final_state, _F32, N * Hv * Dv * Dk), o=(o, _IO, T * Hv * Dv),
+          xq=(xq, _U8, T * Hv * Dv // 2), xs=(xs, _U8, T * Hv * Dv // 16), workspace=(workspace, _U8, None))
     if o is None and write_o:
         o = torch.empty((T, Hv, Dv), dtype=torch.bfloat16, device=q.device)
     if final_state is None:
@@ -190,6 +226,11 @@ def gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1.0,
     B, Hk, Dk = q.shape
     Hv, Dv = v.shape[1], v.shape[2]
     out_dtype = out_dtype or q.dtype
+    _args(q.device, q=(q, _IO, None), k=(k, (q.dtype,), B * Hk * Dk), v=(v, (q.dtype,), B * Hv * Dv),
+          a=(a, _F32, B * Hv), b=(b, _F32, B * Hv), A_log=(A_log, _F32, Hv), dt_bias=(dt_bias, _F32, Hv),
+          state=(state, _F32, B * Hv * Dv * Dk), o=(o, _IO, B * Hv * Dv))
+    if state is None:
+        raise ValueError("state is required")
     if o is None:
         o = torch.empty((B, Hv, Dv), dtype=out_dtype, device=q.device)
     _contig(q, k, v, a, b, A_log, dt_bias, state, o)
@@ -208,6 +249,12 @@ def gdn_decode_verify(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1.0, 
     B, T, Hk, Dk = q.shape
     Hv, Dv = v.shape[2], v.shape[3]
     out_dtype = out_dtype or q.dtype
+    _args(q.device, q=(q, _IO, None), k=(k, (q.dtype,), B * T * Hk * Dk), v=(v, (q.dtype,), B * T * Hv * Dv),
+          a=(a, _F32, B * T * Hv), b=(b, _F32, B * T * Hv), A_log=(A_log, _F32, Hv), dt_bias=(dt_bias, _F32, Hv),
+          state=(state, _F32, B * Hv * Dv * Dk), final_state=(final_state, _F32, B * Hv * Dv * Dk),
+          o=(o, _IO, B * T * Hv * Dv))
+    if state is None:
+        raise ValueError("state is required")
     if o is None:
         o = torch.empty((B, T, Hv, Dv), dtype=out_dtype, device=q.device)
     _contig(q, k, v, a, b, A_log, dt_bias, state, final_state, o)
@@ -224,9 +271,12 @@ def gdn_decode_commit(q, k, v, a, b, A_log, dt_bias, state, accepted, scale: flo
     T draft tokens (the same tensors as the gdn_decode_verify call)."""
     B, T, Hk, Dk = q.shape
     Hv, Dv = v.shape[2], v.shape[3]
+    _args(q.device, q=(q, _IO, None), k=(k, (q.dtype,), B * T * Hk * Dk), v=(v, (q.dtype,), B * T * Hv * Dv),
+          a=(a, _F32, B * T * Hv), b=(b, _F32, B * T * Hv), A_log=(A_log, _F32, Hv), dt_bias=(dt_bias, _F32, Hv),
+          state=(state, _F32, B * Hv * Dv * Dk), accepted=(accepted, _I32, B))
+    if state is None or accepted is None:
+        raise ValueError("state and accepted are required")
     _contig(q, k, v, a, b, A_log, dt_bias, state, accepted)
-    if accepted.dtype != torch.int32:
-        raise TypeError("accepted must be int32")
     st = LIB.gdn_decode_commit(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
                                B, T, Hk, Hv, Dk, Dv, float(scale), int(bool(qk_l2norm)), _dt(q), _ptr(accepted),
                                _ptr(state), _stream(stream))
@@ -238,6 +288,8 @@ def gdn_gated_rmsnorm_silu(o, z, weight, eps: float = 1e-6, out_dtype=None, y=No
     """o, z [M, Hv, D] -> y [M, Hv * D]."""
     M, Hv, D = o.shape
     out_dtype = out_dtype or o.dtype
+    _args(o.device, o=(o, _IO, None), z=(z, (o.dtype,), M * Hv * D), weight=(weight, _F32, D),
+          y=(y, _IO, M * Hv * D))
     if y is None:
         y = torch.empty((M, Hv * D), dtype=out_dtype, device=o.device)
     _contig(o, z, weight, y)
@@ -252,6 +304,8 @@ def gdn_gated_rmsnorm_silu_nvfp4(o, z, weight, global_scale: float, eps: float =
     """o, z [M, Hv, D] -> (xq [M, K/2] uint8, xs [M, K/16] uint8), K = Hv * D."""
     M, Hv, D = o.shape
     K = Hv * D
+    _args(o.device, o=(o, _IO, None), z=(z, (o.dtype,), M * K), weight=(weight, _F32, D),
+          xq=(xq, _U8, M * K // 2), xs=(xs, _U8, M * K // 16))
     if xq is None:
         xq = torch.empty((M, K // 2), dtype=torch.uint8, device=o.device)
     if xs is None:
@@ -266,6 +320,7 @@ def gdn_gated_rmsnorm_silu_nvfp4(o, z, weight, global_scale: float, eps: float =
 def nvfp4_quantize_act(x, global_scale: float, xq=None, xs=None, stream=None):
     """x [M, K] bf16/fp32 -> (xq [M, K/2] uint8, xs [M, K/16] uint8)."""
     M, K = x.shape
+    _args(x.device, x=(x, _IO, None), xq=(xq, _U8, M * K // 2), xs=(xs, _U8, M * K // 16))
     if xq is None:
         xq = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
     if xs is None:
@@ -280,6 +335,7 @@ def nvfp4_quantize_act(x, global_scale: float, xq=None, xs=None, stream=None):
 def nvfp4_dequantize_act(xq, xs, global_scale: float, out_dtype=torch.float32, y=None, stream=None):
     """(xq [M, K/2], xs [M, K/16]) -> y [M, K] = E2M1 * E4M3 / global_scale."""
     M, K = xq.shape[0], xq.shape[1] * 2
+    _args(xq.device, xq=(xq, _U8, None), xs=(xs, _U8, M * K // 16), y=(y, _IO, M * K))
     if y is None:
         y = torch.empty((M, K), dtype=out_dtype, device=xq.device)
     _contig(xq, xs, y)
@@ -292,6 +348,8 @@ def nvfp4_gemm(aq, as_, bq, bs, alpha: float, out_dtype=torch.bfloat16, y=None, 
     """(aq [M, K/2], as [M, K/16]) x (bq [N, K/2], bs [N, K/16])^T * alpha -> y [M, N]."""
     M, K = aq.shape[0], aq.shape[1] * 2
     N = bq.shape[0]
+    _args(aq.device, aq=(aq, _U8, None), as_=(as_, _U8, M * K // 16), bq=(bq, _U8, N * K // 2),
+          bs=(bs, _U8, N * K // 16), y=(y, _IO, M * N))
     if y is None:
         y = torch.empty((M, N), dtype=out_dtype, device=aq.device)
     _contig(aq, as_, bq, bs, y)
@@ -306,6 +364,8 @@ def nvfp4_gemm_colscale(aq, as_, bq, bs, col_alpha, out_dtype=torch.bfloat16, y=
     weight, each with its own global scale)."""
     M, K = aq.shape[0], aq.shape[1] * 2
     N = bq.shape[0]
+    _args(aq.device, aq=(aq, _U8, None), as_=(as_, _U8, M * K // 16), bq=(bq, _U8, N * K // 2),
+          bs=(bs, _U8, N * K // 16), col_alpha=(col_alpha, _F32, N), y=(y, _IO, M * N))
     if y is None:
         y = torch.empty((M, N), dtype=out_dtype, device=aq.device)
     _contig(aq, as_, bq, bs, col_alpha, y)
@@ -355,6 +415,9 @@ def gdn_short_conv1d_silu(x, weight, cu_seqlens=None, num_seqs=None, initial_sta
     T, C, ldx = _conv_rows(x)
     K = weight.shape[1]
     N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (num_seqs or 1)
+    _args(x.device, x=x, weight=(weight, _F32, C * K), cu_seqlens=(cu_seqlens, _I32, None),
+          initial_state=(initial_state, (torch.bfloat16,), N * (K - 1) * C),
+          final_state=(final_state, (torch.bfloat16,), N * (K - 1) * C), y=(y, (torch.bfloat16,), T * C))
     if final_state is None and output_final_state:
         final_state = torch.empty((N, K - 1, C), dtype=torch.bfloat16, device=x.device)
     _contig(weight, cu_seqlens, initial_state, final_state)
@@ -370,6 +433,8 @@ def gdn_short_conv1d_silu_decode(x, weight, conv_state, parts=None, y=None, stre
     Returns y [B, C] (or the list of plane views)."""
     B, C, ldx = _conv_rows(x)
     K = weight.shape[1]
+    _args(x.device, x=x, weight=(weight, _F32, C * K), conv_state=(conv_state, (torch.bfloat16,), B * (K - 1) * C),
+          y=(y, (torch.bfloat16,), B * C))
     _contig(weight, conv_state)
     buf, arr, views = _conv_planes(parts, B, C, y, x.device)
     st = LIB.gdn_short_conv1d_silu_decode(_ptr(x), ldx, _ptr(weight), B, C, K, _ptr(conv_state), _ptr(buf), arr,
