@@ -50,9 +50,6 @@ def make_l2_flush(torch, dev):
 CHUNK = 64
 # FP4 (kind::mxf4nvf4) dense rate measured by a tcgen05 probe: 16368 MAC/cycle/SM x 148 SMs x 1965 MHz
 FP4_PROBE_TFLOPS = 2.0 * 16368 * 148 * 1.965e9 / 1e12
-# DRAM bytes (read + write) of one scan call (prep + chain kernels) on the benchmark workload,
-# from the ncu capture summarised in profiles/chunked_prefill_T4096.md; valid only for the
-# kernel source it was taken on (first 16 hex digits of its sha256).
 # DRAM bytes of one fused prefill call (prep + lean + combine + the output pass with the gated
 # tail), from one ncu capture with cold caches, keyed by the digest of the scan's source
 SCAN_TRAFFIC = {"8d0ca4422ce4682c": 237.57e6}

@@ -29,7 +29,7 @@ ABI_SYMBOLS = (
     "gdn_prefill_chunked", "gdn_prefill_workspace_bytes", "gdn_prefill_chunked_gated_nvfp4", "gdn_decode_step",
     "gdn_decode_verify", "gdn_decode_commit",
     "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_dequantize_act",
-    "nvfp4_gemm", "nvfp4_gemm_colscale", "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode",
+    "nvfp4_gemm", "nvfp4_gemm_colscale", "nvfp4_fused_col_alpha", "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode",
     "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_status_string",
     "gdn_version",
 )
@@ -64,6 +64,7 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_dequantize_act.argtypes = [P, P, i32, i32, f32, i32, P, P]
     lib.nvfp4_gemm.argtypes = [P, P, P, P, f32, i32, i32, i32, i32, P, P]
     lib.nvfp4_gemm_colscale.argtypes = [P, P, P, P, P, i32, i32, i32, i32, P, P]
+    lib.nvfp4_fused_col_alpha.argtypes = [P, P, i32, f32, P, P]
     i64 = ctypes.c_int64
     lib.gdn_short_conv1d_silu.argtypes = [P, i64, P, P, i32, i32, i32, i32, P, P, P, P, i32, P]
     lib.gdn_short_conv1d_silu_decode.argtypes = [P, i64, P, i32, i32, i32, P, P, P, i32, P]
@@ -76,7 +77,7 @@ def _load() -> ctypes.CDLL:
     for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_gated_nvfp4", "gdn_prefill_chunked_static_ws", "gdn_decode_step", "gdn_decode_verify",
                  "gdn_decode_commit", "gdn_gated_rmsnorm_silu",
                  "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_dequantize_act", "nvfp4_gemm",
-                 "nvfp4_gemm_colscale",
+                 "nvfp4_gemm_colscale", "nvfp4_fused_col_alpha",
                  "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode", "gdn_get_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -375,12 +376,22 @@ def nvfp4_gemm_colscale(aq, as_, bq, bs, col_alpha, out_dtype=torch.bfloat16, y=
     return y
 
 
-def fused_module_col_alpha(widths, module_scales, act_scale: float, device=None):
-    """col_alpha for a weight made of modules of the given output widths, module i quantised with
-    global scale module_scales[i], activations with act_scale: 1 / (act_scale * module scale)."""
-    parts = [torch.full((int(n),), float(1.0 / (act_scale * float(s))), dtype=torch.float32)
-             for n, s in zip(widths, module_scales)]
-    return torch.cat(parts).to(device if device is not None else "cuda")
+def nvfp4_fused_col_alpha(widths, module_scales, act_scale: float, col_alpha=None, device=None, stream=None):
+    """col_alpha [sum(widths)] fp32 for a weight made of modules of the given output widths,
+    module i quantised with global scale module_scales[i], activations with act_scale (computed
+    by the library: 1 / (act_scale * module scale) per column)."""
+    n = len(widths)
+    wa = (ctypes.c_int32 * n)(*[int(w) for w in widths])
+    sa = (ctypes.c_float * n)(*[float(s) for s in module_scales])
+    N = sum(int(w) for w in widths)
+    device = torch.device(device if device is not None else "cuda")
+    _args(device, col_alpha=(col_alpha, _F32, N))
+    if col_alpha is None:
+        col_alpha = torch.empty((N,), dtype=torch.float32, device=device)
+    _contig(col_alpha)
+    st = LIB.nvfp4_fused_col_alpha(wa, sa, n, float(act_scale), _ptr(col_alpha), _stream(stream))
+    _check("nvfp4_fused_col_alpha", st)
+    return col_alpha
 
 
 def _conv_rows(x):

@@ -2,6 +2,7 @@
 // selection and launches on the caller's stream. No device memory is allocated here; the
 // only library-owned device object is the status word that bounded waits report into.
 #include <climits>
+#include <cmath>
 #include <cstdio>
 
 #include "common.cuh"
@@ -11,19 +12,21 @@ namespace {
 
 __device__ int g_device_status = 0;
 
-constexpr int kMaxDevices = 64;
-int *g_status_ptr[kMaxDevices] = {nullptr};
-
-// Device address of the status word on the current device (looked up once per device).
+// Device address of the status word on the current device (looked up once per device, under a
+// lock; a device reset between calls is not supported, see gdn.h).
 int *status_ptr() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!g_status_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-        g_status_ptr[dev] = static_cast<int *>(p);
-    }
-    return g_status_ptr[dev];
+    static gdn::PerDevice<int *> addr;
+    int *p = nullptr;
+    if (addr.get(
+            [](int, int *&r) {
+                void *a = nullptr;
+                const cudaError_t e = cudaGetSymbolAddress(&a, g_device_status);
+                r = static_cast<int *>(a);
+                return e;
+            },
+            &p) != cudaSuccess)
+        return nullptr;
+    return p;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -269,6 +272,26 @@ gdn_status nvfp4_gemm_colscale(const uint8_t *aq, const uint8_t *as, const uint8
     if (!aligned16(aq) || !aligned16(bq) || !aligned16(y)) return GDN_ERR_INVALID_ARG;
     gdn::GemmArgs g{aq, as, bq, bs, 1.0f, M, N, K, out_dtype == GDN_BF16, y, status_ptr(), col_alpha};
     return launched(gdn::launch_nvfp4_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gdn_status nvfp4_fused_col_alpha(const int32_t *widths, const float *module_scales, int32_t n_modules,
+                                 float act_scale, float *col_alpha, gdn_stream_t stream) {
+    if (!widths || !module_scales || !col_alpha || n_modules < 1 || n_modules > gdn::kMaxModules)
+        return GDN_ERR_INVALID_ARG;
+    gdn::ColAlphaArgs c{};
+    int64_t end = 0;
+    for (int m = 0; m < n_modules; ++m) {
+        const float prod = act_scale * module_scales[m];
+        if (widths[m] < 1 || !(prod != 0.0f) || !std::isfinite(prod)) return GDN_ERR_INVALID_ARG;
+        end += widths[m];
+        if (end > INT32_MAX) return GDN_ERR_INVALID_ARG;
+        c.end[m] = (int32_t)end;
+        c.scale[m] = module_scales[m];
+    }
+    c.n_modules = n_modules;
+    c.act = act_scale;
+    c.col_alpha = col_alpha;
+    return launched(gdn::launch_fused_col_alpha(c, (int32_t)end, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 namespace {

@@ -1456,25 +1456,28 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
     if (!make_map3(&maps.q, c.q, c.T, c.Hk) || !make_map3(&maps.k, c.k, c.T, c.Hk) ||
         !make_map3(&maps.v, c.v, c.T, c.Hv))
         return cudaErrorInvalidValue;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gdn_chunk_chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gdn_chunk_chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, CHF_SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gdn_chunk_lean_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CL_SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gdn_segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CB_SMEM);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static PerDevice<int> attr;
+    int unused = 0;
+    cudaError_t e = attr.get(
+        [](int, int &) {
+            cudaError_t r = cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(gdn_chunk_chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(gdn_chunk_chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, CHF_SMEM);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(gdn_chunk_lean_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CL_SMEM);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(gdn_segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CB_SMEM);
+            return r;
+        },
+        &unused);
+    if (e != cudaSuccess) return e;
     const int slots = c.T / kChunk + c.num_seqs;
     const int seg = chunked_segment_chunks(c.T, c.num_seqs, c.Hv);
     const int seg_slots = c.T / (kChunk * seg) + c.num_seqs;
     uint8_t *ws = static_cast<uint8_t *>(c.ws);
-    cudaError_t e = launch_pdl(gdn_chunk_prep_kernel, dim3(slots, c.Hv), dim3(NT), P_SMEM, st, maps, c.a, c.b, c.A_log,
+    e = launch_pdl(gdn_chunk_prep_kernel, dim3(slots, c.Hv), dim3(NT), P_SMEM, st, maps, c.a, c.b, c.A_log,
                                c.dt_bias, c.cu_seqlens, c.T, c.num_seqs, c.Hk, c.Hv, slots, c.scale, c.l2norm, ws,
                                c.status);
     if (e != cudaSuccess) return e;

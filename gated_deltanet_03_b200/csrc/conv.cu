@@ -330,23 +330,26 @@ Planes make_planes(const ConvArgs &a) {
 // down to a whole number of channel blocks, but no more token shares than sub-tiles.
 template <int K>
 int conv_grid(int n_cblk, int T) {
-    static int per_sm[64] = {0};
-    static int sms[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
-    if (!per_sm[dev]) {
-        if (cudaFuncSetAttribute(short_conv_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kConvSmem) != cudaSuccess)
-            return -1;
-        int b = 0, m = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, short_conv_kernel<K>, kConvThreads, kConvSmem) !=
-                cudaSuccess ||
-            cudaDeviceGetAttribute(&m, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return -1;
-        sms[dev] = m;
-        per_sm[dev] = b > 0 ? b : 1;
-    }
-    const int shares = max(1, min(per_sm[dev] * sms[dev] / n_cblk, (T + kConvTile - 1) / kConvTile));
+    struct Occ {
+        int per_sm, sms;
+    };
+    static PerDevice<Occ> occ;
+    Occ o{};
+    const cudaError_t e = occ.get(
+        [](int dev, Occ &r) {
+            cudaError_t x = cudaFuncSetAttribute(short_conv_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)kConvSmem);
+            int b = 0, m = 0;
+            if (x == cudaSuccess)
+                x = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, short_conv_kernel<K>, kConvThreads, kConvSmem);
+            if (x == cudaSuccess) x = cudaDeviceGetAttribute(&m, cudaDevAttrMultiProcessorCount, dev);
+            r.per_sm = b > 0 ? b : 1;
+            r.sms = m;
+            return x;
+        },
+        &o);
+    if (e != cudaSuccess) return -1;
+    const int shares = max(1, min(o.per_sm * o.sms / n_cblk, (T + kConvTile - 1) / kConvTile));
     return shares * n_cblk;
 }
 

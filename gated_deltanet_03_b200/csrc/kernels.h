@@ -5,9 +5,39 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <utility>
 
 namespace gdn {
+
+// Per-device set-up (function attributes, occupancy queries): a kernel attribute such as the
+// dynamic shared-memory limit belongs to one device, so each launcher keeps one record per
+// device index and fills it under a lock the first time it runs with that device current.
+// A failed set-up is not recorded and runs again on the next call.
+constexpr int kMaxDevices = 64;
+template <typename Rec>
+struct PerDevice {
+    Rec rec[kMaxDevices] = {};
+    bool done[kMaxDevices] = {};
+    std::mutex mu;
+    // The current device's record, filled by init(dev, rec) on first use.
+    template <typename F>
+    cudaError_t get(F &&init, Rec *out) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev]) {
+            Rec r{};
+            if ((e = init(dev, r)) != cudaSuccess) return e;
+            rec[dev] = r;
+            done[dev] = true;
+        }
+        *out = rec[dev];
+        return cudaSuccess;
+    }
+};
 
 // Launch with programmatic stream serialization (see pdl_wait in common.cuh).
 template <typename... KArgs, typename... Args>
@@ -93,6 +123,17 @@ struct GemmArgs {
     const float *col_alpha;      // [N] per-column factor, or null: alpha for every column
 };
 cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st);
+
+// Per-column factors of a fused-module weight: column n of module m gets 1 / (act * scale[m]).
+constexpr int kMaxModules = 64;
+struct ColAlphaArgs {
+    int32_t end[kMaxModules];    // exclusive end column of each module
+    float scale[kMaxModules];
+    int32_t n_modules;
+    float act;
+    float *col_alpha;
+};
+cudaError_t launch_fused_col_alpha(const ColAlphaArgs &c, int32_t N, cudaStream_t st);
 
 struct ConvArgs {
     const void *x;               // bf16 rows of ldx elements; channels [0, C) are convolved

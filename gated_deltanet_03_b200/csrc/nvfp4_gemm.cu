@@ -395,6 +395,26 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t row_bytes
 
 }  // namespace
 
+namespace {
+
+// One thread per output column: find its module (a short linear search over the module ends)
+// and write 1 / (act * scale) with IEEE division.
+__global__ void fused_col_alpha_kernel(const __grid_constant__ ColAlphaArgs c, int32_t N) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= N) return;
+    int m = 0;
+    while (m + 1 < c.n_modules && n >= c.end[m]) ++m;
+    c.col_alpha[n] = __fdiv_rn(1.0f, __fmul_rn(c.act, c.scale[m]));
+}
+
+}  // namespace
+
+cudaError_t launch_fused_col_alpha(const ColAlphaArgs &c, int32_t N, cudaStream_t st) {
+    return launch_pdl(fused_col_alpha_kernel, dim3((unsigned)((N + 255) / 256)), dim3(256), 0, st, c, N);
+}
+
 cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
     CUtensorMap ma, mb, msa, msb;
     if (!make_map(&ma, g.aq, (uint64_t)g.M, (uint64_t)g.K / 2, 128)) return cudaErrorInvalidValue;
@@ -409,13 +429,6 @@ cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
         msa = ma;   // unused
         msb = mb;
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attrs[2];
     attrs[0].id = cudaLaunchAttributeClusterDimension;
@@ -429,19 +442,25 @@ cudaError_t launch_nvfp4_gemm(const GemmArgs &g, cudaStream_t st) {
     cfg.stream = st;
     cfg.attrs = attrs;
     cfg.numAttrs = 2;
-    // as many pairs as run at once (one CTA per SM), no more than there are 256 x 256 tiles
-    static int max_pairs[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!max_pairs[dev]) {
-        cfg.gridDim = dim3(2);
-        int clusters = 0;
-        const cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, nvfp4_gemm_kernel, &cfg);
-        if (e != cudaSuccess) return e;
-        max_pairs[dev] = clusters > 0 ? clusters : 1;
-    }
+    // as many pairs as run at once (one CTA per SM), no more than there are 256 x 256 tiles;
+    // the shared-memory attribute and the occupancy query are per device
+    static PerDevice<int> max_pairs;
+    int pairs = 0;
+    const cudaError_t e = max_pairs.get(
+        [&cfg](int, int &r) {
+            cudaError_t x = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+            if (x != cudaSuccess) return x;
+            cudaLaunchConfig_t q = cfg;
+            q.gridDim = dim3(2);
+            int clusters = 0;
+            if ((x = cudaOccupancyMaxActiveClusters(&clusters, nvfp4_gemm_kernel, &q)) != cudaSuccess) return x;
+            r = clusters > 0 ? clusters : 1;
+            return cudaSuccess;
+        },
+        &pairs);
+    if (e != cudaSuccess) return e;
     const int pair_tiles = ((g.N + 255) / 256) * ((g.M + 255) / 256);
-    cfg.gridDim = dim3((unsigned)(2 * (pair_tiles < max_pairs[dev] ? pair_tiles : max_pairs[dev])));
+    cfg.gridDim = dim3((unsigned)(2 * (pair_tiles < pairs ? pair_tiles : pairs)));
     return cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel, ma, mb, msa, msb, sf_tma ? 1 : 0, g.as, g.bs, g.alpha,
                               g.col_alpha, g.M, g.N, g.K, g.out_bf16 ? 1 : 0, g.y, g.status);
 }

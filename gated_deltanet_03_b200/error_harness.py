@@ -31,7 +31,8 @@ import math
 
 import torch
 
-from . import (gdn_prefill_chunked, gdn_prefill_workspace_bytes, nvfp4_dequantize_act, nvfp4_gemm_colscale,
+from . import (gdn_prefill_chunked, gdn_prefill_workspace_bytes, nvfp4_dequantize_act, nvfp4_fused_col_alpha,
+               nvfp4_gemm_colscale,
                nvfp4_quantize_act)
 
 E2M1_MAX = 6.0
@@ -75,8 +76,7 @@ def gate_compression(x: torch.Tensor, w_a: torch.Tensor, w_b: torch.Tensor, A_lo
     scales = [global_scale(w_a), global_scale(w_b)]
     wq_a, ws_a = nvfp4_quantize_act(w_a, scales[0])
     wq_b, ws_b = nvfp4_quantize_act(w_b, scales[1])
-    col_alpha = torch.cat([torch.full((Hv,), 1.0 / (gx * s), dtype=torch.float32, device=x.device)
-                           for s in scales])
+    col_alpha = nvfp4_fused_col_alpha((Hv, Hv), scales, gx, device=x.device)
     quant = nvfp4_gemm_colscale(xq, xs, torch.cat([wq_a, wq_b]), torch.cat([ws_a, ws_b]), col_alpha,
                                 out_dtype=torch.float32)
     a, b = exact[:, :Hv], exact[:, Hv:]

@@ -30,6 +30,9 @@
  *   - Kernels that wait on barriers bound every wait; on expiry they record
  *     GDN_ERR_TIMEOUT in a device status word and finish without deadlocking. Read (and
  *     clear) it with gdn_get_device_status().
+ *   - Per-device set-up (kernel attributes, the device addresses of the status word and of
+ *     the allocation-free scratch array) is done once per device on first use and kept:
+ *     resetting a device (cudaDeviceReset) between calls into this library is not supported.
  *   - Multi-head layouts: q, k [T, Hk, Dk]; v, o, z [T, Hv, Dv]; value head h reads key
  *     head h / (Hv / Hk) (contiguous groups). The state is [.., Hv, Dv, Dk] fp32, key index
  *     contiguous, so that o = S q.
@@ -243,6 +246,16 @@ GDN_API gdn_status nvfp4_gemm_colscale(const uint8_t *aq, const uint8_t *as, con
                                        const uint8_t *bs, const float *col_alpha, int32_t M, int32_t N,
                                        int32_t K, gdn_dtype out_dtype, void *y, gdn_stream_t stream);
 
+/* The col_alpha vector of nvfp4_gemm_colscale for a weight made of n_modules modules stacked
+ * along N: module m has widths[m] output columns and was quantised with global scale
+ * module_scales[m]; the activations with act_scale. Writes col_alpha[n] = 1 / (act_scale *
+ * module_scales[m]) (fp32 IEEE division) for every column n of module m, in order.
+ * widths, module_scales: HOST arrays of n_modules (1 <= n_modules <= 64, each width >= 1);
+ * col_alpha: device fp32 [sum of widths]. A zero or non-finite product act_scale * scale is
+ * GDN_ERR_INVALID_ARG. Enqueued on `stream`. */
+GDN_API gdn_status nvfp4_fused_col_alpha(const int32_t *widths, const float *module_scales, int32_t n_modules,
+                                         float act_scale, float *col_alpha, gdn_stream_t stream);
+
 /* ------------------------------------------------------ short convolution ----
  * [WALK]: the causal short convolution + SiLU on the layer's q, k, v channels before the scan:
  *   y[t, c] = SiLU(sum_{j<K} weight[c, j] x[t - (K - 1) + j, c])
@@ -289,8 +302,9 @@ GDN_API gdn_status gdn_short_conv1d_silu_decode(const void *x, int64_t ldx, cons
  * the library instead: 32 MiB (33554432 bytes), held on every GPU that loads the library
  * until the process exits. Sizes whose workspace (gdn_prefill_workspace_bytes) exceeds
  * 32 MiB return GDN_ERR_WORKSPACE before anything is launched. It allocates nothing.
- * The first call on a device looks up the array's device address for that device; make
- * that first call before any stream capture on the device.
+ * The first call on a device looks up the array's device address for that device and keeps
+ * it (so the device must not be reset between calls); make that first call before any stream
+ * capture on the device.
  * Every call uses the same array: calls that can overlap on the GPU (other streams, other
  * host threads) race on it and corrupt each other's results, so serialise them. What a
  * previous call left in the array does not matter: the path writes all it later reads.

@@ -31,7 +31,7 @@
  *   [FMT]  OCP Microscaling Formats (MX) v1.0 (E2M1 element encoding) and OCP 8-bit
  *          Floating Point (E4M3FN): value sets used below.
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent:
  *   - q/k are L2-normalised inside the path when qk_l2norm != 0: x * (sum x^2 + eps)^-1/2.
  *   - GQA: v-head h reads k-head h / (Hv / Hk).
  *   - the readout uses the updated state S_t.

@@ -102,7 +102,7 @@ def test_fused_modules_colscale(g, M):
         refs.append(oracle.nvfp4_gemm(aq, as_, gsa, wq, ws, gsw))
     wq, ws, ref = np.concatenate(wqs), np.concatenate(wss), np.concatenate(refs, axis=1)
     u8 = torch.uint8
-    ca = g.fused_module_col_alpha(widths, gsws, float(gsa))
+    ca = g.nvfp4_fused_col_alpha(widths, gsws, float(gsa))
     y = to_np(g.nvfp4_gemm_colscale(dev(aq, u8), dev(as_, u8), dev(wq, u8), dev(ws, u8), ca, out_dtype=torch.float32))
     torch.cuda.synchronize()
     assert g.gdn_get_device_status() == 0

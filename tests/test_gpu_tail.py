@@ -127,3 +127,26 @@ def test_tail_zero_rows_and_zero_blocks(g):
     xq, xs = g.gdn_gated_rmsnorm_silu_nvfp4(dev(o, torch.bfloat16), dev(z, torch.bfloat16),
                                             dev(w, torch.float32), 1.0)
     assert int(xs.abs().sum()) == 0 and int(xq.sum()) == 0
+
+
+def test_nvfp4_block_scale_order_on_ties(g):
+    """The encoder's block scale follows (amax / 6) * gs on the E4M3 tie cases of
+    tests/golden/nvfp4_scale_order.txt, where another order of the same operations picks a
+    different code; standalone encoder and fused tail both, bf16 and fp32 inputs."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "nvfp4_scale_order.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    for amax_s, gs_bits, want_s, _, _ in rows:
+        amax = float(amax_s)
+        gs = float(np.array([int(gs_bits, 16)], np.uint32).view(np.float32)[0])
+        want = int(want_s, 16)
+        x = np.zeros((4, 32), np.float32)
+        x[:, 5] = amax
+        x[:, 6] = -0.5 * amax
+        x[:, 16 + 3] = -amax
+        for dt in (torch.bfloat16, torch.float32):
+            xq, xs = g.nvfp4_quantize_act(dev(x, dt), gs)
+            xq_ref, xs_ref = oracle.nvfp4_quantize(x, np.float32(gs))
+            assert (xs.cpu().numpy() == want).all()
+            np.testing.assert_array_equal(xs.cpu().numpy(), xs_ref)
+            np.testing.assert_array_equal(xq.cpu().numpy(), xq_ref)

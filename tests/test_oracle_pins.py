@@ -378,6 +378,40 @@ def test_nvfp4_nibble_order_and_scale_layout():
     assert xs[0, 1] == 0x30 and xq[0, 8] == 7
 
 
+def _scale_order_cases():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "nvfp4_scale_order.txt")
+    cases = []
+    with open(path) as fh:
+        for line in fh:
+            if line.strip() and not line.startswith("#"):
+                amax, gs_bits, want, alt1, alt2 = line.split()
+                gs = np.array([int(gs_bits, 16)], np.uint32).view(np.float32)[0]
+                cases.append((float(amax), gs, int(want, 16), int(alt1, 16), int(alt2, 16)))
+    return cases
+
+
+@pytest.mark.parametrize("case", _scale_order_cases())
+def test_nvfp4_block_scale_order_of_operations(case):
+    """The block scale is (amax / 6) * gs in two fp32 roundings, then E4M3 ties-to-even
+    (tests/golden/nvfp4_scale_order.txt): each case sits on an E4M3 tie, where the other orders
+    of the same operations give a different code, so a wrong order fails here."""
+    amax, gs, want, alt1, alt2 = case
+    # the fixture's three codes, re-derived with torch's fp32 arithmetic and its E4M3 rounding
+    t = lambda x: torch.tensor(x, dtype=torch.float32)
+    e4 = lambda s: int(s.reshape(1).to(torch.float8_e4m3fn).view(torch.uint8)[0])
+    a, g = t(amax), t(float(gs))
+    assert e4((a / 6.0) * g) == want
+    assert e4(a * (g / 6.0)) == alt1 and e4((a * g) / 6.0) == alt2
+    assert want != alt1 and want != alt2
+    # the oracle on one block whose largest magnitude is amax (the sign must not matter)
+    x = np.zeros((2, 16), np.float32)
+    x[0, :4] = [0.25 * amax, -amax, 0.5, 0.0]
+    x[1, 7] = amax
+    xq, xs = oracle.nvfp4_quantize(x, gs)
+    assert int(xs[0, 0]) == want and int(xs[1, 0]) == want
+
+
 def test_nvfp4_exact_round_trip_of_grid_values():
     rng = np.random.default_rng(31)
     grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], np.float32)
