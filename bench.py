@@ -1,11 +1,12 @@
 """Benchmark of the Gated DeltaNet hot path on B200.
 
 One step = one pass of the whole layer path over one batch of synthetic input on the
-1024-wide hybrid-model prefill workload (T = 4096, 16 q/k and 16 v heads, d = 128, bf16):
-chunked gated delta-rule scan -> gated RMSNorm * SiLU(z) with the fused NVFP4 activation
-encode -> NVFP4 W4A4 output projection 2048 -> 1024. The decode step (B = 256 sequences,
-16 q/k / 32 v heads, fp32 state [256, 32, 128, 128] updated in place) is timed in the
-same run and reported under "decode".
+27B-class long-prefill workload (T = 32768, 16 q/k and 32 v heads, d = 128, bf16): chunked
+gated delta-rule scan -> gated RMSNorm * SiLU(z) with the fused NVFP4 activation encode ->
+NVFP4 W4A4 output projection 4096 -> 2048. The same step on the 1024-wide layer (T = 4096,
+16/16 heads, 2048 -> 1024) and on the variable-length batch (8 sequences, 16/32 heads) is
+reported under "prefill_1024_wide" and "varlen"; the decode step (B = 256 sequences, fp32
+state [256, 32, 128, 128] updated in place) under "decode".
 
 Launch: python bench.py [--gpus N --steps K --warmup W] (N > 1 under torchrun, one rank
 per GPU, each rank an independent replica of the workload: weak scaling, no collective
@@ -191,6 +192,120 @@ def count_kernels(torch, fn):
                "gdn_chunk_chain_kernel<true>", "nvfp4_gemm_kernel"]
 
 
+def prefill_case(torch, g, w, args, dev, flush, side, with_e2e=False, with_parts=False):
+    """One prefill workload end to end: the step (fused prefill = scan + gated RMSNorm + NVFP4
+    encode in the output pass, then the NVFP4 W4A4 output projection) captured in a CUDA graph
+    and replayed with the L2 flushed before each replay; the fused prefill and the GEMM alone the
+    same way. Returns the timings, the inputs (for the oracle baseline) and, when asked, the
+    end-to-end timing through the public API from pinned host buffers."""
+    x = workloads.generate(w)
+    bf, f32 = torch.bfloat16, torch.float32
+
+    def up(a, dt):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+
+    q, k, v, z = up(x["q"], bf), up(x["k"], bf), up(x["v"], bf), up(x["z"], bf)
+    a, b = up(x["a"], f32), up(x["b"], f32)
+    A_log, dt_bias, nw = up(x["A_log"], f32), up(x["dt_bias"], f32), up(x["norm_weight"], f32)
+    cu = up(x["cu_seqlens"], torch.int32) if w.num_seqs > 1 else None
+    S0 = None if x["initial_state"] is None else up(x["initial_state"], f32)
+    W = up(x["proj_weight"], bf)
+    gw = float(448.0 * 6.0 / W.float().abs().max().item())
+    wq, ws_w = g.nvfp4_quantize_act(W, gw)         # weights: quantised once, outside timing
+    T, Hv, D, K, N = w.T, w.Hv, w.D, w.K, w.n_out
+    S = torch.empty((w.num_seqs, Hv, D, D), dtype=f32, device=dev)
+    xq = torch.empty((T, K // 2), dtype=torch.uint8, device=dev)
+    xs = torch.empty((T, K // 16), dtype=torch.uint8, device=dev)
+    Y = torch.empty((T, N), dtype=bf, device=dev)
+    ws = torch.empty((g.gdn_prefill_workspace_bytes(T, w.num_seqs, w.Hk, Hv, D, D),), dtype=torch.uint8, device=dev)
+    # activation global scale: one calibration pass outside timing
+    o = torch.empty((T, Hv, D), dtype=bf, device=dev)
+    g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=cu, initial_state=S0, final_state=S, o=o,
+                          workspace=ws)
+    y_cal = g.gdn_gated_rmsnorm_silu(o, z, nw, out_dtype=f32)
+    gx = float(448.0 * 6.0 / y_cal.abs().max().item())
+    alpha = float(np.float32(1.0) / (np.float32(gx) * np.float32(gw)))
+    del y_cal
+    if not with_parts:
+        del o
+
+    def fused():
+        g.gdn_prefill_chunked_gated_nvfp4(q, k, v, a, b, A_log, dt_bias, z, nw, gx, cu_seqlens=cu, initial_state=S0,
+                                          final_state=S, xq=xq, xs=xs, workspace=ws)
+
+    def gemm():
+        g.nvfp4_gemm(xq, xs, wq, ws_w, alpha, y=Y)
+
+    def step():
+        fused()
+        gemm()
+
+    fns = [("step", step), ("fused", fused), ("gemm", gemm)]
+    if with_parts:
+        fns += [("scan", lambda: g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=cu, initial_state=S0,
+                                                        final_state=S, o=o, workspace=ws)),
+                ("tail", lambda: g.gdn_gated_rmsnorm_silu_nvfp4(o, z, nw, gx, xq=xq, xs=xs))]
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    assert g.gdn_get_device_status() == 0
+    graphs = {}
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for name, fn in fns:
+            fn()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=side):
+                fn()
+            graphs[name] = gr
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    res = {"w": w, "x": x, "graphs": graphs}
+    if with_e2e:
+        hq, hk, hv, hz = (t.cpu().pin_memory() for t in (q, k, v, z))
+        ha, hb = a.cpu().pin_memory(), b.cpu().pin_memory()
+        hY = torch.empty((T, N), dtype=bf, pin_memory=True)
+        res["h2d"] = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hz, ha, hb))
+        res["d2h"] = hY.numel() * hY.element_size()
+
+        def e2e_step():
+            # host -> device inputs, the whole path through the public API, result back to host
+            q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+            z.copy_(hz, non_blocking=True); a.copy_(ha, non_blocking=True); b.copy_(hb, non_blocking=True)
+            step()
+            hY.copy_(Y, non_blocking=True)
+        res["e2e_step"] = e2e_step
+    res["keep"] = (q, k, v, z, a, b, A_log, dt_bias, nw, cu, S0, wq, ws_w, S, xq, xs, Y, ws)
+    return res
+
+
+def timed_graph(torch, stream, flush, gr, n):
+    """Mean device time (ms) of n replays, the L2 flushed before each (outside the events)."""
+    out = []
+    for _ in range(n):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gr.replay()
+        e1.record(stream)
+        out.append((e0, e1))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in out]
+
+
+def prefill_summary(w, step_ms, fused_ms, gemm_ms, pk, pk_kind):
+    fl = scan_flops(w)
+    t = statistics.mean(fused_ms) / 1e3
+    return {"workload": w.name, "tokens": w.T, "tokens/s": w.T / (statistics.mean(step_ms) / 1e3),
+            "ms_per_step": statistics.mean(step_ms), "prefill_fused_ms": statistics.mean(fused_ms),
+            "nvfp4_gemm_ms": statistics.mean(gemm_ms),
+            "prefill_TFLOP/s": fl / t / 1e12, "prefill_tensor_frac": fl / t / 1e12 / float(pk["bf16_tflops"]),
+            "prefill_hbm_frac": fused_bytes(w) / t / 1e9 / float(pk["hbm_gbs"]),
+            "gemm_frac_of_fp4_probe": 2.0 * w.T * w.K * w.n_out / (statistics.mean(gemm_ms) / 1e3) / 1e12
+            / FP4_PROBE_TFLOPS, "peak_kind": pk_kind}
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -205,114 +320,30 @@ def run_gpu(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
-
-    w = workloads.PREFILL_1K
-    x = workloads.generate(w)
     bf, f32 = torch.bfloat16, torch.float32
 
     def up(a, dt):
         return torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
 
-    q, k, v, z = up(x["q"], bf), up(x["k"], bf), up(x["v"], bf), up(x["z"], bf)
-    a, b = up(x["a"], f32), up(x["b"], f32)
-    A_log, dt_bias, nw = up(x["A_log"], f32), up(x["dt_bias"], f32), up(x["norm_weight"], f32)
-    W = up(x["proj_weight"], bf)
-    gw = float(448.0 * 6.0 / W.float().abs().max().item())
-    wq, ws_w = g.nvfp4_quantize_act(W, gw)         # weights: quantised once, outside timing
-    T, Hv, D, K, N = w.T, w.Hv, w.D, w.K, w.n_out
-    o = torch.empty((T, Hv, D), dtype=bf, device=dev)
-    S = torch.empty((1, Hv, D, D), dtype=f32, device=dev)
-    xq = torch.empty((T, K // 2), dtype=torch.uint8, device=dev)
-    xs = torch.empty((T, K // 16), dtype=torch.uint8, device=dev)
-    Y = torch.empty((T, N), dtype=bf, device=dev)
-    # activation global scale: one calibration pass outside timing
-    g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, final_state=S, o=o)
-    y_cal = g.gdn_gated_rmsnorm_silu(o, z, nw, out_dtype=f32)
-    gx = float(448.0 * 6.0 / y_cal.abs().max().item())
-    alpha = float(np.float32(1.0) / (np.float32(gx) * np.float32(gw)))
-    del y_cal
     flush = make_l2_flush(torch, dev)
-
-    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    ws = torch.empty((g.gdn_prefill_workspace_bytes(T, 1, w.Hk, Hv, D, D),), dtype=torch.uint8, device=dev)
-
-    def scan():
-        g.gdn_prefill_chunked(q, k, v, a, b, A_log, dt_bias, final_state=S, o=o, workspace=ws)
-
-    def tail():
-        g.gdn_gated_rmsnorm_silu_nvfp4(o, z, nw, gx, xq=xq, xs=xs)
-
-    def gemm():
-        g.nvfp4_gemm(xq, xs, wq, ws_w, alpha, y=Y)
-
-    def fused():
-        # the scan whose output pass also applies the gated RMSNorm and writes NVFP4 activations
-        g.gdn_prefill_chunked_gated_nvfp4(q, k, v, a, b, A_log, dt_bias, z, nw, gx, final_state=S, xq=xq, xs=xs,
-                                          workspace=ws)
-
-    def step():
-        fused()
-        gemm()
-
-    # the causal short convolution in front of the scan (q|k|v channels of the same layer, K = 4),
-    # timed alone: not part of the step, whose inputs are the scan's
-    conv_C = 2 * w.Hk * D + Hv * D
-    cx = workloads.conv_inputs(T, conv_C, 4, seed=w.seed)
-    conv_x, conv_w = up(cx["x"], bf), up(cx["weight"], f32)
-    conv_y = torch.empty((T * conv_C,), dtype=bf, device=dev)
-    conv_parts = (w.Hk * D, w.Hk * D, Hv * D)
-
-    def conv():
-        g.gdn_short_conv1d_silu(conv_x, conv_w, parts=conv_parts, y=conv_y)
-
-    for _ in range(args.warmup):
-        flush()
-        step()
-    torch.cuda.synchronize()
-    assert g.gdn_get_device_status() == 0
-
-    # CUDA graphs: the step and each op alone, replayed so the timing is device time only
-    graphs = {}
     side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        for name, fn in (("step", step), ("scan", scan), ("tail", tail), ("fused", fused), ("gemm", gemm),
-                         ("conv", conv)):
-            fn()
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr, stream=side):
-                fn()
-            graphs[name] = gr
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
+    pk, pk_kind = peaks()
 
-    def timed(gr, n):
-        out = []
-        for _ in range(n):
-            flush()          # L2 flush between timed replays (outside the events)
-            e0, e1 = ev(), ev()
-            e0.record(stream)
-            gr.replay()
-            e1.record(stream)
-            out.append((e0, e1))
-        return out
-
+    # headline: the 27B-class long prefill (T = 32768, 16/32 heads, out_proj 4096 -> 2048)
+    w = workloads.PREFILL_LONG
+    main = prefill_case(torch, g, w, args, dev, flush, side, with_e2e=True)
+    graphs = main["graphs"]
+    T, Hv, D, K, N = w.T, w.Hv, w.D, w.K, w.n_out
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        step_ev = timed(graphs["step"], args.steps)
-        torch.cuda.synchronize()
+        step_ms = timed_graph(torch, stream, flush, graphs["step"], args.steps)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    parts = {}
-    for name in ("scan", "tail", "fused", "gemm", "conv"):
-        evs = timed(graphs[name], args.steps)
-        torch.cuda.synchronize()
-        parts[name] = [a.elapsed_time(b) for a, b in evs]
-    scan_ms, tail_ms, fused_ms, gemm_ms = parts["scan"], parts["tail"], parts["fused"], parts["gemm"]
+    fused_ms = timed_graph(torch, stream, flush, graphs["fused"], args.steps)
+    gemm_ms = timed_graph(torch, stream, flush, graphs["gemm"], args.steps)
     launches_per_step, kernel_names = count_kernels(torch, graphs["step"].replay)
     ms = statistics.mean(step_ms)
     ms_max = ms
@@ -321,28 +352,14 @@ def run_gpu(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_max = float(t.item())
     assert g.gdn_get_device_status() == 0
-
-    # end to end through the public API: pinned host inputs in, host result out
-    hq, hk, hv, hz = (t.cpu().pin_memory() for t in (q, k, v, z))
-    ha, hb = a.cpu().pin_memory(), b.cpu().pin_memory()
-    hY = torch.empty((T, N), dtype=bf, pin_memory=True)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hz, ha, hb))
-    d2h = hY.numel() * hY.element_size()
-
-    def e2e_step():
-        # host -> device inputs, the whole path through the public API, result back to host
-        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
-        z.copy_(hz, non_blocking=True); a.copy_(ha, non_blocking=True); b.copy_(hb, non_blocking=True)
-        step()
-        hY.copy_(Y, non_blocking=True)
-
+    e2e_step = main["e2e_step"]
     for _ in range(args.warmup):
         e2e_step()
     torch.cuda.synchronize()
     e2e_ms = []
     for _ in range(args.steps):
         flush()
-        s0, s1 = ev(), ev()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record(stream)
         e2e_step()
         s1.record(stream)
@@ -353,15 +370,35 @@ def run_gpu(args):
         t = torch.tensor([e2e], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e = float(t.item())
+    h2d, d2h, x_main = main["h2d"], main["d2h"], main["x"]
+    del main, graphs, e2e_step
+    torch.cuda.empty_cache()
 
-    # decode step on the batched-decode workload (state 512 MiB > L2: no flush needed)
-    dw = workloads.DECODE_B256
-    dx = workloads.generate(dw)
-    dq, dk, dv = up(dx["q"], bf), up(dx["k"], bf), up(dx["v"], bf)
-    da, db = up(dx["a"], f32), up(dx["b"], f32)
-    dA, ddt = up(dx["A_log"], f32), up(dx["dt_bias"], f32)
-    dstate = up(dx["initial_state"], f32)
-    dout = torch.empty((dw.num_seqs, dw.Hv, dw.D), dtype=bf, device=dev)
+    # the 1024-wide layer's prefill (T = 4096, 16/16 heads) and the variable-length batch
+    subs = {}
+    for name, wl, parts_too in (("prefill_1024_wide", workloads.PREFILL_1K, True), ("varlen", workloads.VARLEN_8, False)):
+        r = prefill_case(torch, g, wl, args, dev, flush, side, with_parts=parts_too)
+        n_rep = max(args.steps, 10)
+        st_ms = timed_graph(torch, stream, flush, r["graphs"]["step"], n_rep)
+        fu_ms = timed_graph(torch, stream, flush, r["graphs"]["fused"], n_rep)
+        ge_ms = timed_graph(torch, stream, flush, r["graphs"]["gemm"], n_rep)
+        subs[name] = prefill_summary(wl, st_ms, fu_ms, ge_ms, pk, pk_kind)
+        if parts_too:
+            subs[name]["scan_alone_ms"] = statistics.mean(timed_graph(torch, stream, flush, r["graphs"]["scan"], n_rep))
+            subs[name]["gated_norm_nvfp4_alone_ms"] = statistics.mean(
+                timed_graph(torch, stream, flush, r["graphs"]["tail"], n_rep))
+        assert g.gdn_get_device_status() == 0
+        del r
+        torch.cuda.empty_cache()
+
+    # the causal short convolution in front of the 1024-wide layer's scan (q|k|v channels,
+    # K = 4), timed alone: not part of the step, whose inputs are the scan's
+    cw = workloads.PREFILL_1K
+    conv_C = 2 * cw.Hk * cw.D + cw.Hv * cw.D
+    cx = workloads.conv_inputs(cw.T, conv_C, 4, seed=cw.seed)
+    conv_x, conv_w = up(cx["x"], bf), up(cx["weight"], f32)
+    conv_y = torch.empty((cw.T * conv_C,), dtype=bf, device=dev)
+    conv_parts = (cw.Hk * cw.D, cw.Hk * cw.D, cw.Hv * cw.D)
 
     def graph_of(fn):
         # device time of one launch, without the host's launch gap between the events
@@ -375,19 +412,25 @@ def run_gpu(args):
         torch.cuda.synchronize()
         return gr
 
+    conv_graph = graph_of(lambda: g.gdn_short_conv1d_silu(conv_x, conv_w, parts=conv_parts, y=conv_y))
+    conv_ms = timed_graph(torch, stream, flush, conv_graph, max(args.steps, 10))
+    del conv_graph
+
+    # decode step on the batched-decode workload (L2 flushed before each replay, as for every op)
+    dw = workloads.DECODE_B256
+    dx = workloads.generate(dw)
+    dq, dk, dv = up(dx["q"], bf), up(dx["k"], bf), up(dx["v"], bf)
+    da, db = up(dx["a"], f32), up(dx["b"], f32)
+    dA, ddt = up(dx["A_log"], f32), up(dx["dt_bias"], f32)
+    dstate = up(dx["initial_state"], f32)
+    dout = torch.empty((dw.num_seqs, dw.Hv, dw.D), dtype=bf, device=dev)
+
     dec_graph = graph_of(lambda: g.gdn_decode_step(dq, dk, dv, da, db, dA, ddt, dstate, o=dout))
     for _ in range(max(3, args.warmup)):
         dec_graph.replay()
     torch.cuda.synchronize()
-    dec_ms = []
-    for _ in range(max(args.steps, 10)):
-        s0, s1 = ev(), ev()
-        s0.record(stream)
-        dec_graph.replay()
-        s1.record(stream)
-        torch.cuda.synchronize()
-        dec_ms.append(s0.elapsed_time(s1))
-    dec = statistics.median(dec_ms)
+    dec_ms = timed_graph(torch, stream, flush, dec_graph, max(args.steps, 10))
+    dec = statistics.mean(dec_ms)
     state_bytes = dstate.numel() * 4
     dec_bytes = 2 * state_bytes + sum(t.numel() * t.element_size() for t in (dq, dk, dv, da, db, dout))
 
@@ -412,10 +455,8 @@ def run_gpu(args):
         ver_graph.replay()
         com_graph.replay()
     torch.cuda.synchronize()
-    ver_ev, com_ev = timed(ver_graph, max(args.steps, 10)), timed(com_graph, max(args.steps, 10))
-    torch.cuda.synchronize()
-    ver_ms = statistics.mean(a.elapsed_time(b) for a, b in ver_ev)
-    com_ms = statistics.mean(a.elapsed_time(b) for a, b in com_ev)
+    ver_ms = statistics.mean(timed_graph(torch, stream, flush, ver_graph, max(args.steps, 10)))
+    com_ms = statistics.mean(timed_graph(torch, stream, flush, com_graph, max(args.steps, 10)))
     m_tok = sum(t.numel() * t.element_size() for t in (mq, mk, mv, ma, mb))
     ver_bytes = mstate.numel() * 4 + m_tok + mo.numel() * mo.element_size()
     com_bytes = 2 * mstate.numel() * 4 + m_tok
@@ -430,9 +471,7 @@ def run_gpu(args):
     big_graph = graph_of(lambda: g.nvfp4_gemm(ga[0], ga[1], gw[0], gw[1], 1.0, y=gy))
     for _ in range(3):
         big_graph.replay()
-    big_ev = timed(big_graph, max(args.steps, 10))
-    torch.cuda.synchronize()
-    big_ms = statistics.mean(a.elapsed_time(b) for a, b in big_ev)
+    big_ms = statistics.mean(timed_graph(torch, stream, flush, big_graph, max(args.steps, 10)))
     del ga, gw, gy, big_graph
 
     # short convolution decode on the batched-decode workload's q|k|v channels (state in place)
@@ -447,9 +486,7 @@ def run_gpu(args):
     for _ in range(max(3, args.warmup)):
         cdec_graph.replay()
     torch.cuda.synchronize()
-    cdec_ev = timed(cdec_graph, max(args.steps, 10))     # L2 flushed before each replay
-    torch.cuda.synchronize()
-    cdec = statistics.median(a.elapsed_time(b) for a, b in cdec_ev)
+    cdec = statistics.mean(timed_graph(torch, stream, flush, cdec_graph, max(args.steps, 10)))
     cdec_bytes = 2 * dconv_x.numel() * 2 + 2 * dconv_s.numel() * 2 + dconv_w.numel() * 4
     assert g.gdn_get_device_status() == 0
 
@@ -459,8 +496,8 @@ def run_gpu(args):
     if rank != 0:
         return
 
-    pk, pk_kind = peaks()
-    conv_bytes = 2 * T * conv_C * 2 + conv_w.numel() * 4     # x read once, y written once, weights
+    conv_bytes = 2 * cw.T * conv_C * 2 + conv_w.numel() * 4     # x read once, y written once, weights
+    conv_mean = statistics.mean(conv_ms)
     scan_s = statistics.mean(fused_ms) / 1e3
     fl = scan_flops(w)
     achieved_tflops = fl / scan_s / 1e12
@@ -478,17 +515,18 @@ def run_gpu(args):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded; shapes of the pages' 1024-wide hybrid layer)",
+        "data": "synthetic (seeded; shapes of the pages' 27B-class hybrid layer: 32 x 128 -> 4096 -> 2048)",
         "config": {"workload": w.name, "T": T, "Hk": w.Hk, "Hv": Hv, "d": D, "chunk": CHUNK,
                    "out_proj": "NVFP4 W4A4 %d->%d" % (K, N), "global_batch": 1, "seq_len": T,
-                   "parallelism": "replicas x%d" % world, "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)"},
+                   "parallelism": "replicas x%d" % world,
+                   "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)"},
         "breakdown_ms": {"prefill_fused": statistics.mean(fused_ms), "nvfp4_gemm": statistics.mean(gemm_ms),
-                         "scan_alone": statistics.mean(scan_ms), "gated_norm_nvfp4_alone": statistics.mean(tail_ms),
                          "step": "prefill_fused (scan + gated RMSNorm + NVFP4 encode in the output pass) + nvfp4_gemm",
-                         "timing": "CUDA graph replay per op"},
-        "roofline": {"kernel": "fused prefill (prep, lean, combine and output-pass kernels of one call)", "bound": "tensor", "achieved": achieved_tflops,
+                         "timing": "CUDA graph replay per op, L2 flushed before each"},
+        "roofline": {"kernel": "fused prefill (prep, lean, combine and output-pass kernels of one call)",
+                     "bound": "tensor", "achieved": achieved_tflops,
                      "peak": peak_tflops, "unit": "TFLOP/s", "frac": achieved_tflops / peak_tflops,
-                     "peak_kind": pk_kind + " (bf16 dense burst; the scan's MMAs are fp16)",
+                     "peak_kind": pk_kind + " (bf16 dense burst; the scan's MMAs are fp16 and bf16)",
                      "algorithmic_flops": fl, "algorithmic_bytes": fused_bytes(w),
                      "hbm_frac": fused_bytes(w) / scan_s / 1e9 / float(pk["hbm_gbs"]),
                      "traffic": SCAN_TRAFFIC.get(source_digest(os.path.join(
@@ -498,7 +536,8 @@ def run_gpu(args):
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
         "decode": {"workload": dw.name, "ms": dec, "GB/s": dec_bytes / (dec / 1e3) / 1e9,
                    "frac": dec_bytes / (dec / 1e3) / 1e9 / float(pk["hbm_gbs"]),
-                   "bytes": dec_bytes, "peak_gbs": float(pk["hbm_gbs"]), "peak_kind": pk_kind},
+                   "bytes": dec_bytes, "peak_gbs": float(pk["hbm_gbs"]), "peak_kind": pk_kind,
+                   "timing": "CUDA graph replay, L2 flushed before each"},
         "gemm_long_prefill": {"shape": [gM, gN, gK], "ms": big_ms,
                               "TFLOP/s": 2.0 * gM * gN * gK / (big_ms / 1e3) / 1e12,
                               "frac_of_fp4_probe": 2.0 * gM * gN * gK / (big_ms / 1e3) / 1e12 / FP4_PROBE_TFLOPS,
@@ -511,10 +550,12 @@ def run_gpu(args):
                          "bytes": {"verify": ver_bytes, "commit": com_bytes},
                          "single_steps_ms": mT * dec,
                          "timing": "CUDA graph replay, L2 flushed before each; commit of a seeded 0..4 accepted tokens"},
-        "short_conv": {"workload": "%s q|k|v channels (T = %d, C = %d, K = 4), planes q, k, v" % (w.name, T, conv_C),
-                       "ms": statistics.mean(parts["conv"]),
-                       "GB/s": conv_bytes / (statistics.mean(parts["conv"]) / 1e3) / 1e9,
-                       "frac": conv_bytes / (statistics.mean(parts["conv"]) / 1e3) / 1e9 / float(pk["hbm_gbs"]),
+        "prefill_1024_wide": subs["prefill_1024_wide"],
+        "varlen": subs["varlen"],
+        "short_conv": {"workload": "%s q|k|v channels (T = %d, C = %d, K = 4), planes q, k, v" % (cw.name, cw.T, conv_C),
+                       "ms": conv_mean,
+                       "GB/s": conv_bytes / (conv_mean / 1e3) / 1e9,
+                       "frac": conv_bytes / (conv_mean / 1e3) / 1e9 / float(pk["hbm_gbs"]),
                        "bytes": conv_bytes, "bound": "hbm", "peak_kind": pk_kind,
                        "decode": {"workload": "%s q|k|v channels (B = %d, C = %d, K = 4)" % (dw.name, dw.num_seqs, dC),
                                   "ms": cdec, "bytes": cdec_bytes,
@@ -524,7 +565,7 @@ def run_gpu(args):
         "clocks": clk.summary(),
     }
     if not args.no_cpu:
-        out["cpu_baseline"] = cpu_baseline(w, x)
+        out["cpu_baseline"] = cpu_baseline(w, x_main)
     print(json.dumps(out))
 
 
@@ -677,12 +718,24 @@ def run_verify(args):
 
 # ----------------------------------------------------------------- CPU arm ----
 
+CPU_SAMPLE_TOKENS = 4096
+
+
+def token_prefix(w, x, n):
+    """The workload cut to its first n tokens (one sequence): the layer on a shorter input."""
+    y = dict(x)
+    for key in ("q", "k", "v", "z", "a", "b"):
+        y[key] = x[key][:n]
+    y["cu_seqlens"] = np.array([0, n], np.int32)
+    return y
+
+
 def cpu_pass(w, x, units=None):
     """The oracle over the same workload: scan (threaded over heads), gated tail, NVFP4
     encode and the fp64 GEMM over dequantised operands."""
     import oracle
     o, S = oracle.gdn_scan(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
-                           cu_seqlens=x["cu_seqlens"], units=units)
+                           cu_seqlens=x["cu_seqlens"], initial_state=x["initial_state"], units=units)
     y = oracle.gated_rmsnorm_silu(workloads.round_bf16(o.astype(np.float32)), x["z"], x["norm_weight"])
     gx = np.float32(448.0 * 6.0 / max(np.abs(y).max(), 1e-30))
     W = x["proj_weight"]
@@ -693,19 +746,27 @@ def cpu_pass(w, x, units=None):
 
 
 def cpu_baseline(w, x, min_seconds: float = 10.0):
-    """The oracle as it stands, on the host cores: whole passes over the workload (all heads, all
-    rows) repeated until about `min_seconds` of CPU work; tokens/s over all passes."""
+    """The oracle as it stands, on the host cores, on a bounded sample of the workload: whole
+    passes of the layer (all heads, all rows) over its first CPU_SAMPLE_TOKENS tokens, repeated
+    until about `min_seconds` of CPU work; tokens/s over all passes."""
     import oracle
+    n = min(CPU_SAMPLE_TOKENS, w.T)
+    xs = token_prefix(w, x, n) if w.num_seqs == 1 else x
+    n = n if w.num_seqs == 1 else w.T
     passes = 0
     t0 = time.perf_counter()
     while True:
-        cpu_pass(w, x)
+        cpu_pass(w, xs)
         passes += 1
         dt = time.perf_counter() - t0
         if dt >= min_seconds:
             break
-    return {"value": passes * w.T / dt, "unit": "tokens/s", "cores": oracle.default_threads(), "kind": "oracle",
-            "sample": "the whole workload (all %d heads, all rows), %d passes" % (w.Hv, passes), "seconds": dt}
+    return {"value": passes * n / dt, "unit": "tokens/s", "cores": oracle.default_threads(), "kind": "oracle",
+            "sample": "the layer (all %d heads, all rows) on the first %d of the %d tokens, %d passes"
+                      % (w.Hv, n, w.T, passes), "seconds": dt}
+
+
+REF_SAMPLE_TOKENS = 2048
 
 
 def run_reference(args):
@@ -713,25 +774,28 @@ def run_reference(args):
     if rank != 0:
         return
     import oracle
-    w = workloads.PREFILL_1K
+    w = workloads.PREFILL_LONG
     x = workloads.generate(w)
+    n = REF_SAMPLE_TOKENS
+    xs = token_prefix(w, x, n)
     for _ in range(args.warmup):
-        cpu_pass(w, x, units=[0])
+        cpu_pass(w, xs, units=[0])
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        cpu_pass(w, x)
+        cpu_pass(w, xs)
         times.append(time.perf_counter() - t0)
     dt = statistics.mean(times)
-    val = w.T / dt
+    val = n / dt
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 0,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded; shapes of the pages' 1024-wide hybrid layer)",
+        "data": "synthetic (seeded; shapes of the pages' 27B-class hybrid layer: 32 x 128 -> 4096 -> 2048)",
         "config": {"workload": w.name, "T": w.T, "Hk": w.Hk, "Hv": w.Hv, "d": w.D},
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": oracle.default_threads(), "kind": "oracle",
-                         "sample": "the whole workload per step (all heads, all rows)"},
+                         "sample": "each step: the layer (all heads, all rows) on the first %d of the %d tokens"
+                                   % (n, w.T)},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 

@@ -28,8 +28,8 @@ def test_reference_arm_prints_one_contract_line():
     assert d["unit"] == "tokens/s" and d["higher_is_better"] is True
     assert d["steps"] == 1 and d["warmup"] == 3
     assert d["value"] > 0 and d["ms_per_step"] > 0
-    assert abs(d["value"] - workloads.PREFILL_1K.T / (d["ms_per_step"] / 1e3)) <= 1e-6 * d["value"]
-    assert d["config"]["workload"] == workloads.PREFILL_1K.name
+    assert abs(d["value"] - bench.REF_SAMPLE_TOKENS / (d["ms_per_step"] / 1e3)) <= 1e-6 * d["value"]
+    assert d["config"]["workload"] == workloads.PREFILL_LONG.name
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,

@@ -118,6 +118,30 @@ def test_prefill_degenerate_gates(g, case):
     assert rel_err(S, S_ref) <= TOL_SCAN, rel_err(S, S_ref)
 
 
+@pytest.mark.parametrize("T", [512, 4096])
+@pytest.mark.parametrize("noise", [0.2, 0.05])
+def test_prefill_concentrated_keys_overwrite(g, T, noise):
+    """The overwrite regime ("Why Gated DeltaNet Survives 4-Bit Quantization", abstract,
+    mechanism iii: each write replaces the state along the current key) with keys concentrated
+    in four directions: key = one of four random directions + noise * N(0, 1), alpha -> 1
+    (A_log = -30), beta -> 1 (b = 20), nonzero initial state. Nearly parallel keys make the
+    state hold large components along their small differences, which is where a chunked form
+    with a low-precision staging loses accuracy; the bound is the stated 2e-3 on fp32 o and S."""
+    w = workloads.custom("ck", (T,), 2, 4, 128, io="bf16", s0_std=0.1, seed=700 + T + int(noise * 100))
+    x = workloads.generate(w)
+    rng = np.random.default_rng(23)
+    Hk = x["k"].shape[1]
+    basis = rng.standard_normal((4, Hk, 128))
+    pick = rng.integers(0, 4, size=T)
+    x["k"][:] = workloads.round_bf16(basis[pick] + noise * rng.standard_normal(x["k"].shape))
+    x["A_log"][:] = -30.0
+    x["b"][:] = 20.0
+    o_ref, S_ref = _full_oracle(x)
+    o, S = _run_prefill(g, x, w, torch.float32)
+    assert rel_err(o, o_ref) <= TOL_SCAN, rel_err(o, o_ref)
+    assert rel_err(S, S_ref) <= TOL_SCAN, rel_err(S, S_ref)
+
+
 def test_prefill_empty_batch_copies_state(g):
     w = workloads.custom("e", (0,), 1, 1, 128, io="bf16", s0_std=0.1, seed=3)
     x = workloads.generate(w)
