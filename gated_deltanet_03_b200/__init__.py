@@ -30,7 +30,7 @@ ABI_SYMBOLS = (
     "gdn_decode_verify", "gdn_decode_commit",
     "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_dequantize_act",
     "nvfp4_gemm", "nvfp4_gemm_colscale", "nvfp4_fused_col_alpha", "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode",
-    "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_status_string",
+    "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_debug_set_wait", "gdn_status_string",
     "gdn_version",
 )
 
@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
     lib.gdn_prefill_chunked_static_ws.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32,
                                                   i32, i32, P, P, P, i32, P]
     lib.gdn_get_device_status.argtypes = [P]
+    lib.gdn_debug_set_wait.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
     lib.gdn_status_string.argtypes = [i32]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_version.restype = i32
@@ -78,7 +79,7 @@ def _load() -> ctypes.CDLL:
                  "gdn_decode_commit", "gdn_gated_rmsnorm_silu",
                  "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_dequantize_act", "nvfp4_gemm",
                  "nvfp4_gemm_colscale", "nvfp4_fused_col_alpha",
-                 "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode", "gdn_get_device_status"):
+                 "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode", "gdn_get_device_status", "gdn_debug_set_wait"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -452,6 +453,15 @@ def gdn_short_conv1d_silu_decode(x, weight, conv_state, parts=None, y=None, stre
                                           len(arr), _stream(stream))
     _check("gdn_short_conv1d_silu_decode", st)
     return views[0] if parts is None else views
+
+
+INJECT_SKIP_PREP_LOADS = 1
+
+
+def gdn_debug_set_wait(wait_limit_ns: int = 0, inject_flags: int = 0) -> None:
+    """Test support: bounded-wait limit (0 = the default 1 s) and the switches that make a wait
+    run out with nothing in flight (INJECT_SKIP_PREP_LOADS) on the current device."""
+    _check("gdn_debug_set_wait", LIB.gdn_debug_set_wait(int(wait_limit_ns), int(inject_flags)))
 
 
 def gdn_get_device_status(stream=None) -> int:

@@ -1,6 +1,6 @@
 // C entry points declared in include/gdn.h: host-side argument checks, kernel variant
 // selection and launches on the caller's stream. No device memory is allocated here; the
-// only library-owned device object is the status word that bounded waits report into.
+// only library-owned device object is the control block (status word, wait limit, test switches).
 #include <climits>
 #include <cmath>
 #include <cstdio>
@@ -10,7 +10,7 @@
 
 namespace {
 
-__device__ int g_device_status = 0;
+__device__ gdn::DeviceCtl g_device_ctl = {0, 0u, gdn::kWaitLimitNs};
 
 // Device address of the status word on the current device (looked up once per device, under a
 // lock; a device reset between calls is not supported, see gdn.h).
@@ -20,7 +20,7 @@ int *status_ptr() {
     if (addr.get(
             [](int, int *&r) {
                 void *a = nullptr;
-                const cudaError_t e = cudaGetSymbolAddress(&a, g_device_status);
+                const cudaError_t e = cudaGetSymbolAddress(&a, g_device_ctl);
                 r = static_cast<int *>(a);
                 return e;
             },
@@ -65,6 +65,20 @@ gdn_status gdn_get_device_status(gdn_stream_t stream) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
     }
     return static_cast<gdn_status>(h);
+}
+
+gdn_status gdn_debug_set_wait(uint64_t wait_limit_ns, uint32_t inject_flags) {
+    int *p = status_ptr();
+    if (!p) return GDN_ERR_CUDA;
+    if (wait_limit_ns == 0) wait_limit_ns = gdn::kWaitLimitNs;
+    if (wait_limit_ns > gdn::kWaitLimitNs || (inject_flags & ~gdn::kInjectSkipPrepLoads) != 0u) return GDN_ERR_INVALID_ARG;
+    gdn::DeviceCtl *ctl = reinterpret_cast<gdn::DeviceCtl *>(p);
+    const unsigned long long lim = wait_limit_ns;
+    const unsigned int fl = inject_flags;
+    if (cudaMemcpy(&ctl->wait_limit_ns, &lim, sizeof(lim), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(&ctl->flags, &fl, sizeof(fl), cudaMemcpyHostToDevice) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    return GDN_OK;
 }
 
 size_t gdn_prefill_workspace_bytes(int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv, int32_t Dk,

@@ -1,6 +1,7 @@
-// Chunked gated delta-rule prefill on the fifth-generation tensor cores (tcgen05, TMEM),
-// as two kernels: a prep kernel that is parallel over (chunk, value head) and a chain
-// kernel that is sequential over the chunks of each (sequence, value head).
+// Chunked gated delta-rule prefill on the fifth-generation tensor cores (tcgen05, TMEM): a prep
+// kernel that is parallel over (chunk, value head), and the state chain, sequential over the
+// chunks of each (sequence, value head) and cut into segments (state and transition passes, a
+// short combine of the segments' maps, then the output pass from each segment's true start).
 //
 // "Why Gated DeltaNet Survives 4-Bit Quantization" (abstract, mechanisms ii-iii) describes
 // the recurrence; here it is evaluated 64 tokens at a time in the WY / UT form, which is
@@ -10,32 +11,38 @@
 //   W = T diag(beta gamma) K,   U~ = T diag(beta) V,     U = U~ - W S0^T,
 //   O = diag(gamma) Q S0^T + (Q K^T o Gamma) U,          Gamma_rs = exp(G_r - G_s), s <= r,
 //   S_C = gamma_C S0 + U^T diag(gamma_C / gamma) K.
-// W, U~, P = (Q K^T o Gamma) and the scaled Q and K do not depend on the state: the prep
-// kernel computes them for every chunk at once into the caller's workspace; the chain
-// kernel then runs two state-dependent MMAs per chunk.
+// W, U~, P = (Q K^T o Gamma), the scaled Q and the factors c_r = gamma_C / gamma_r / |k_r| do
+// not depend on the state: the prep kernel computes them for every chunk at once into the
+// caller's workspace; the chain kernels then run the state-dependent MMAs per chunk.
 //
-// The L2 norms of q and k never touch an MMA operand: raw bf16 inputs (exact in fp16) feed
-// the tensor cores and 1/|k|, scale/|q| enter as diagonal factors of the derived operands.
-// Derived operands are staged in fp16 (11-bit significand) with fp32 accumulation in tensor
-// memory; the state itself stays fp32 in registers.
+// Precision. The L2 norms of q and k never touch an MMA operand: the raw bf16 inputs feed the
+// tensor cores and 1/|k|, scale/|q| enter as diagonal factors. When keys are nearly parallel and
+// beta -> 1 (each write replaces the state along a key close to earlier ones), T has O(1)
+// entries of alternating sign and W, U are small differences, so a single 11-bit rounding of the
+// derived operands costs several 1e-3 of the result. The operands that carry this cancellation
+// are therefore kept to about 16 bits: the inverse is fp32, T' and T'' enter MMA2 as bf16 hi + lo
+// parts, U~ is stored in fp32, and in the chain U (with P^T) and U diag(c) (with the raw K) enter
+// as bf16 hi + lo parts (hi hi + hi lo + lo hi). W, Q' and the state's A-operand copy S0 stay
+// fp16, which the result tolerates; the state itself stays fp32 in registers.
 //
 // Every MMA has M = 128 (value or key index on the TMEM lanes):
 //   prep   MMA1  D1 = [K; Q] [K; Q]^T      on the raw bf16 tiles (rows 0-63: K K^T | K Q^T,
 //                                          rows 64-127: Q K^T | Q Q^T; the diagonals give the norms)
-//          MMA2  D2 = [T'; T''] [K | V]    rows 0-63: W = T' K, rows 64-127: U~ = T'' V, with
-//                                          T' = T diag(beta gamma / |k|), T'' = T diag(beta)
-//   chain  MMA45 [D4 | D5a] = S0 [W; Q']^T            Q' = diag(gamma scale / |q|) Q
-//          MMA67 [D7 | D5b] = U^T [K''; P^T]^T        K'' = diag(gamma_C / gamma / |k|) K
-//                                                     P^T[s][r] = k_s.q_r Gamma_rs scale / (|q_r| |k_s|)
-//   with U^T = U~^T - D4, S <- gamma_C S + D7, o^T = D5a + D5b. In the chain the fp16 copies of
-//   S0 and U live in tensor memory as the A operands; the element-wise warps (sixteen in the
-//   output pass, beside one copy/MMA warp; eight in the lean pass, one of whose threads issues)
-//   hand over to the issuing thread through mbarriers.
+//          MMA2  D2 = [T'; T''] [K | V]    bf16, hi then lo A parts; rows 0-63: W = T' K, rows
+//                                          64-127: U~ = T'' V; T' = T diag(beta gamma / |k|),
+//                                          T'' = T diag(beta)
+//   chain  MMA45 [D4 | D5a] = S0 [W; Q']^T      fp16; Q' = diag(gamma scale / |q|) Q
+//          MMA7  D7 = (U diag(c))^T K           bf16 hi / lo A, raw bf16 K
+//          MMA5b D5a += U^T P^T                 bf16 hi / lo, P^T[s][r] = k_s.q_r Gamma_rs scale / (|q_r| |k_s|)
+//   with U^T = U~^T - D4, S <- gamma_C S + D7, o^T = D5a. In the chain the copies of S0 and of U
+//   live in tensor memory as the A operands; the element-wise warps (sixteen in the output pass,
+//   beside one copy/MMA warp; eight in the lean pass, one of whose threads issues) hand over to
+//   the issuing thread through mbarriers.
 //
-// Workspace: one 73 KB item per (value head, chunk slot): [W; Q'] (fp16, K-major, 128 rows,
-// 128-byte swizzled), [K''; P^T] (fp16, three 64-wide MN-major blocks), U~ (fp16 [s][i]) and
-// gamma_C. Chunk c of sequence n uses slot cu_seqlens[n] / 64 + n + c, so slots never
-// collide and T / 64 + num_seqs slots per head suffice.
+// Workspace: one 81 KB item per (value head, chunk slot): [W; Q'] (fp16, K-major, 128 rows,
+// 128-byte swizzled), P^T hi and lo (bf16, MN-major over r), U~ (fp32 [s][i]), c[64] and
+// gamma_C. Chunk c of sequence n uses slot cu_seqlens[n] / 64 + n + c, so slots never collide
+// and T / 64 + num_seqs slots per head suffice. The chain reads the raw K tiles itself.
 #include <algorithm>
 #include <cmath>
 #include <mutex>
@@ -46,8 +53,8 @@
 namespace gdn {
 
 constexpr int kChunk = 64;
-constexpr int kWsItem = 74752;
-constexpr int kWsWQ = 0, kWsKP = 32768, kWsU = 57344, kWsVec = 73728;
+constexpr int kWsItem = 82944;
+constexpr int kWsWQ = 0, kWsP = 32768, kWsU = 49152, kWsVec = 81920;
 
 constexpr size_t kSegItemBytes = 196608;
 
@@ -143,23 +150,6 @@ struct Maps {
     CUtensorMap q, k, v;
 };
 
-// Convert a staged bf16 tile region to fp16 in place, 16 bytes per step. For the [K; Q]
-// area (4 tiles, rows of 128 B) also returns the thread's share of its row's sum of squares.
-__device__ __forceinline__ float convert16(uint8_t *p) {
-    uint4 u = *reinterpret_cast<const uint4 *>(p);
-    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
-    float f[8], ss = 0.0f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        float2 x = __bfloat1622float2(b2[e]);
-        f[2 * e] = x.x;
-        f[2 * e + 1] = x.y;
-        ss += x.x * x.x + x.y * x.y;
-    }
-    st_h8(p, f);
-    return ss;
-}
-
 // Chunk location: slot `id` of the workspace belongs to sequence n (the last n whose first
 // slot cu[n] / 64 + n is <= id) and is its chunk id - (cu[n] / 64 + n).
 __device__ __forceinline__ void locate(int id, const int32_t *cu, int num_seqs, int T, int &n, int &t_begin,
@@ -180,42 +170,37 @@ __device__ __forceinline__ void locate(int id, const int32_t *cu, int num_seqs, 
     }
 }
 
-// Two fp16 values as one 32-bit register (first in the low half).
-__device__ __forceinline__ uint32_t pack_two_h(__half lo, __half hi) {
-    return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-}
-
-// Warp-level 16 x 8 x 16 MMA, fp16 inputs, fp32 accumulation (row-major A, column-major B):
-// used only for the 16 x 16 blocks of the triangular inverse, where latency matters.
-__device__ __forceinline__ void mma_m16n8k16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                             uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 // ===================================================================================
 // Prep kernel: one CTA per (chunk slot, value head); two CTAs per SM.
 // ===================================================================================
-// Shared memory. [K_lo][Q_lo][K_hi][Q_hi] is the A operand [K; Q] (K-major, 128 rows); K_lo,
-// K_hi, V_lo, V_hi sit 2 TILE apart so that [K | V] is one MN-major B operand with N = 256.
-constexpr int P_OFF_KQ = 0;                        // staged bf16 tiles, converted to fp16 in place
-constexpr int P_OFF_VLO = 4 * TILE;
-constexpr int P_OFF_PST = 5 * TILE;                // P^T image, staged for the copy-out
-constexpr int P_OFF_VHI = 6 * TILE;
-constexpr int P_OFF_TP = 7 * TILE;                 // [T'; T''] fp16, K-major, 128-byte swizzled
-constexpr int P_OFF_TPP = 8 * TILE;
-constexpr int P_AH = 72;                           // fp16 row pitch of A and T (144 B)
-constexpr int P_OFF_AH = 9 * TILE;                 // A fp16 [64][72]
-constexpr int P_OFF_TH = P_OFF_AH + 64 * P_AH * 2; // T fp16 [64][72]
-constexpr int P_OFF_VEC = P_OFF_TH + 64 * P_AH * 2; // G, beta, rk, rq, gamma, decS (64 each), spare (128)
+// Shared memory (TILE = 8 KB). [K_lo; Q_lo] and [K_hi; Q_hi] are the two K-major column blocks
+// of the MMA1 operand [K; Q]; K_lo, K_hi, V_lo, V_hi sit 3 TILE apart so that [K | V] is one
+// MN-major B operand with N = 256 for MMA2. The A operands of MMA2 are [T'; T''] split into
+// bf16 hi and lo parts (16 KB each): hi in the free tiles 7-8, lo over Q_lo and the free tile 2
+// once the Q' image is written. After MMA2 the W (fp16) and U~ (fp32) staging reuses tiles 0-5.
+constexpr int P_OFF_KLO = 0, P_OFF_QLO = TILE, P_OFF_KHI = 3 * TILE, P_OFF_QHI = 4 * TILE;
+constexpr int P_OFF_ALO = TILE;                    // [T'_lo; T''_lo], after the Q' image
+constexpr int P_OFF_X = 5 * TILE;                  // inverse scratch (three 16 x 17 fp32 blocks)
+constexpr int P_OFF_VLO = 6 * TILE, P_OFF_AHI = 7 * TILE, P_OFF_VHI = 9 * TILE;
+constexpr int P_AT = 65;                           // fp32 row pitch of the A / T array (odd: no bank conflicts)
+constexpr int P_OFF_AT = 10 * TILE;                // A (strict lower, row-major) and T (strict lower, transposed)
+constexpr int P_OFF_VEC = P_OFF_AT + 64 * P_AT * 4; // G, beta, rk, rq, gamma, c, beta gamma rk, spare (64 each)
 constexpr int P_OFF_BAR = P_OFF_VEC + 8 * 64 * 4;
 constexpr int P_SMEM = P_OFF_BAR + 64 + 1024;
-constexpr int P_OFF_STG = 0;                       // W and U~ staging once the last MMA is done (32 KB)
-static_assert(P_SMEM * 2 <= 228 * 1024, "two prep CTAs per SM");
-// tensor memory: D1 = [K; Q] K^T (64 columns), then D2 = [T'; T''] [K | V] (256 columns) over it
+constexpr int P_OFF_WSTG = 0, P_OFF_USTG = 2 * TILE;   // W fp16 image, U~ fp32 rows (after MMA2)
+static_assert(P_SMEM * 2 + 2048 <= 233472, "two prep CTAs per SM");
+static_assert(P_OFF_USTG + 4 * TILE <= P_OFF_VLO, "staging stays clear of V_lo until MMA2 is done");
+// tensor memory: D1 = [K; Q] [K; Q]^T (128 columns), then D2 = [T'; T''] [K | V] (256) over it
 constexpr uint32_t P_TM_D1 = 0, P_TM_D2 = 0;
+
+// bf16 hi / lo split of two fp32 values, packed as bf16x2 words: hi = bf16(x), lo = bf16(x - hi).
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
 
 __global__ void __launch_bounds__(NT, 2)
 gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict__ ga, const float *__restrict__ gb,
@@ -237,33 +222,42 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *vec = reinterpret_cast<float *>(sm + P_OFF_VEC);
     float *sG = vec, *sBeta = vec + 64, *sRk = vec + 128, *sRq = vec + 192, *sGam = vec + 256, *sDec = vec + 320;
+    float *sBG = vec + 384;
+    float *AT = reinterpret_cast<float *>(sm + P_OFF_AT);
+    float *Xs = reinterpret_cast<float *>(sm + P_OFF_X);
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + P_OFF_BAR);
     uint64_t *bar_mma = bar_tma + 1;
     uint64_t *bar_v = bar_tma + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 3);
-    __half *Ah = reinterpret_cast<__half *>(sm + P_OFF_AH);
-    __half *Th = reinterpret_cast<__half *>(sm + P_OFF_TH);
+    uint64_t *bar_drain = bar_tma + 3;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 4);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int wg = warp / 4;
     const int x = (warp % 4) * 32 + lane;   // this thread's TMEM lane
     const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
+    // what thread 0 has issued, for the drain on the failure path
+    bool loads_issued = false;
+    int mmas_issued = 0;
+    bool failed = false;
 
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         mbar_init(bar_v, 1);
+        mbar_init(bar_drain, 1);
         fence_barrier_init();
-        // K and Q on one barrier (MMA1 starts when they land), V on its own (not needed before
-        // the inverse's off-diagonal phase)
-        mbar_arrive_expect_tx(bar_tma, 4 * TILE);
-        tma_load_3d(sm + P_OFF_KQ + 0 * TILE, &maps.k, bar_tma, 0, hk, t0);
-        tma_load_3d(sm + P_OFF_KQ + 1 * TILE, &maps.q, bar_tma, 0, hk, t0);
-        tma_load_3d(sm + P_OFF_KQ + 2 * TILE, &maps.k, bar_tma, 64, hk, t0);
-        tma_load_3d(sm + P_OFF_KQ + 3 * TILE, &maps.q, bar_tma, 64, hk, t0);
-        mbar_arrive_expect_tx(bar_v, 2 * TILE);
-        tma_load_3d(sm + P_OFF_VLO, &maps.v, bar_v, 0, h, t0);
-        tma_load_3d(sm + P_OFF_VHI, &maps.v, bar_v, 64, h, t0);
+        if (!(ctl_flags(status) & kInjectSkipPrepLoads)) {
+            // K and Q on one barrier (MMA1 starts when they land), V on its own (needed by MMA2)
+            mbar_arrive_expect_tx(bar_tma, 4 * TILE);
+            tma_load_3d(sm + P_OFF_KLO, &maps.k, bar_tma, 0, hk, t0);
+            tma_load_3d(sm + P_OFF_QLO, &maps.q, bar_tma, 0, hk, t0);
+            tma_load_3d(sm + P_OFF_KHI, &maps.k, bar_tma, 64, hk, t0);
+            tma_load_3d(sm + P_OFF_QHI, &maps.q, bar_tma, 64, hk, t0);
+            mbar_arrive_expect_tx(bar_v, 2 * TILE);
+            tma_load_3d(sm + P_OFF_VLO, &maps.v, bar_v, 0, h, t0);
+            tma_load_3d(sm + P_OFF_VHI, &maps.v, bar_v, 64, h, t0);
+            loads_issued = true;
+        }
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 256);
@@ -288,7 +282,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     const uint32_t tmem = *tmem_slot;
     if (tid >= 32 && tid < 64) sG[tid] += sG[31];
 
-    int ok = 1, okv = 1;
+    int ok = 1;
     if (tid == 0) {
         ok = mbar_wait(bar_tma, 0, status) ? 1 : 0;
         if (ok) {
@@ -299,21 +293,18 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             const uint32_t id1 = idesc_f16(128, false, false, false) | (1u << 7) | (1u << 10);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint8_t *base = sm + P_OFF_KQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32;
+                const uint8_t *base = sm + (kk < 4 ? P_OFF_KLO : P_OFF_KHI) + (kk & 3) * 32;
                 mma_f16(tmem + P_TM_D1, kdesc(base), kdesc(base), id1, kk > 0 ? 1u : 0u);
             }
             tc_commit(bar_mma);
+            mmas_issued = 1;
         }
     }
-    if (!__syncthreads_and(ok)) goto teardown;
+    if (!__syncthreads_and(ok)) { failed = true; goto teardown; }
     // while MMA1 runs: the decay factors
     if (tid < 64) sGam[tid] = tid < L ? expf(sG[tid]) : 0.0f;
-    if (tid == 0) {
-        float *wv = reinterpret_cast<float *>(item + kWsVec);
-        wv[0] = __expf(sG[L - 1]);   // gamma_C
-    }
     if (tid == 0) ok = mbar_wait(bar_mma, 0, status) ? 1 : 0;
-    if (!__syncthreads_and(ok)) goto teardown;
+    if (!__syncthreads_and(ok)) { failed = true; goto teardown; }
     tc_fence_after();
     {
         // every warp reads 32 columns (key tokens s) of its 32 lanes; warps 2 and 3 also read the
@@ -355,7 +346,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             rks[j] = k4.x; rks[j + 1] = k4.y; rks[j + 2] = k4.z; rks[j + 3] = k4.w;
         }
         if (x < 64) {
-            // row r of A: A_rs = beta_r exp(G_r - G_s) k_r.k_s / (|k_r| |k_s|) for s < r < L
+            // row r of A (fp32): A_rs = beta_r exp(G_r - G_s) k_r.k_s / (|k_r| |k_s|) for s < r < L
             const int r = x;
             const float Gr = sG[r], cr = sBeta[r] * sRk[r];
             const f2_t cr2 = f2(cr, cr);
@@ -368,10 +359,11 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                 vals[j + 1] = (wg * 32 + j + 1 < r) ? f2hi(v2) : 0.0f;
             }
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8)
-                st_h8(reinterpret_cast<uint8_t *>(Ah + r * P_AH + wg * 32 + q8 * 8), &vals[q8 * 8]);
+            for (int j = 0; j < 32; ++j)
+                if (wg * 32 + j < r) AT[r * P_AT + wg * 32 + j] = vals[j];
         } else {
-            // row r of P = (Q K^T o Gamma) scaled, into the P^T image [s][r] (MN-major over r)
+            // row r of P = (Q K^T o Gamma) scaled, as bf16 hi and lo P^T images [s][r] (MN-major
+            // over r, 128-byte swizzled), stored straight to the workspace item
             const int r = x - 64;
             const float Gr = sG[r], cr = sRq[r];
             const f2_t cr2 = f2(cr, cr);
@@ -384,39 +376,36 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                 vals[j + 1] = (wg * 32 + j + 1 <= r) ? f2hi(v2) : 0.0f;
             }
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                *reinterpret_cast<__half *>(sm + P_OFF_PST + swz(wg * 32 + j, r >> 3) + (r & 7) * 2) =
-                    __float2half_rn(vals[j]);
+            for (int j = 0; j < 32; ++j) {
+                const __nv_bfloat16 hb = __float2bfloat16_rn(vals[j]);
+                const __nv_bfloat16 lb = __float2bfloat16_rn(vals[j] - __bfloat162float(hb));
+                const uint32_t off = swz(wg * 32 + j, r >> 3) + (r & 7) * 2;
+                *reinterpret_cast<__nv_bfloat16 *>(item + kWsP + off) = hb;
+                *reinterpret_cast<__nv_bfloat16 *>(item + kWsP + TILE + off) = lb;
+            }
         }
     }
-    tc_fence_before();
     __syncthreads();
 
-    // ---- T = (I + A)^-1 (unit lower triangular), written as T (fp16, for the block products)
-    //      and as the B operands T'' = T diag(beta), T' = T diag(beta gamma / |k|). Two warps
-    //      solve the 16 x 16 diagonal blocks by forward substitution (fp32) while the other six
-    //      copy the P^T image out of its staging, write the zero upper blocks of T' and T'' and
-    //      the Q' rows (64 + r of the [W; Q'] image): the raw bf16 Q tile scaled row by row, the
-    //      swizzle positions unchanged.
+    // ---- T = (I + A)^-1 (unit lower triangular) in fp32. Its strict lower part is stored
+    //      transposed in the strict upper part of the A array: T[r][c] at AT[c][r] (r > c).
+    //      Two warps solve the 16 x 16 diagonal blocks by forward substitution while the other six
+    //      write the Q' rows (64 + r of the [W; Q'] image: the raw bf16 Q tile scaled row by row,
+    //      swizzle positions unchanged), the decay vector and the column factors of T'.
     if (tid < 64) {
-        const int bi = tid / 16, cc = tid % 16, o0 = bi * 16, r = o0 + cc;
+        const int bi = tid / 16, cc = tid % 16, o0 = bi * 16;
         float xv[16];
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) {
             float acc = (rr == cc) ? 1.0f : 0.0f;
 #pragma unroll
-            for (int s = 0; s < rr; ++s) acc -= __half2float(Ah[(o0 + rr) * P_AH + o0 + s]) * xv[s];
-            xv[rr] = acc;
+            for (int s = 0; s < rr; ++s)
+                if (s >= cc) acc -= AT[(o0 + rr) * P_AT + o0 + s] * xv[s];
+            xv[rr] = (rr < cc) ? 0.0f : acc;
         }
-        const float fb = sBeta[r], fbg = fb * sGam[r] * sRk[r];
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-            const int s = o0 + rr;
-            const uint32_t off = swz(s, r >> 3) + (r & 7) * 2;
-            Th[s * P_AH + r] = __float2half_rn(xv[rr]);
-            *reinterpret_cast<__half *>(sm + P_OFF_TPP + off) = __float2half_rn(xv[rr] * fb);
-            *reinterpret_cast<__half *>(sm + P_OFF_TP + off) = __float2half_rn(xv[rr] * fbg);
-        }
+        for (int rr = 0; rr < 16; ++rr)
+            if (rr > cc) AT[(o0 + cc) * P_AT + o0 + rr] = xv[rr];
     } else {
         const int t6 = tid - 64;
         // Q' (1024 chunks over 192 threads, loads issued before the stores)
@@ -427,7 +416,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             for (int e = 0; e < 6; ++e) {
                 const int idx = e * 192 + t6;
                 const int w = idx < 1024 ? idx : 0, half = w >> 9, within = w & 511, r = within >> 3;
-                hv[e] = *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + (2 * half + 1) * TILE + within * 16);
+                hv[e] = *reinterpret_cast<const uint4 *>(sm + (half ? P_OFF_QHI : P_OFF_QLO) + within * 16);
                 f[e] = sGam[r] * sRq[r];
             }
 #pragma unroll
@@ -447,175 +436,143 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                 }
             }
         }
-        // the P^T image from its staging (512 chunks)
-        uint4 pc[3];
-#pragma unroll
-        for (int e = 0; e < 3; ++e) {
-            const int c16 = e * 192 + t6;
-            pc[e] = *reinterpret_cast<const uint4 *>(sm + P_OFF_PST + (c16 < 512 ? c16 : 0) * 16);
-        }
-#pragma unroll
-        for (int e = 0; e < 3; ++e) {
-            const int c16 = e * 192 + t6;
-            if (c16 < 512) *reinterpret_cast<uint4 *>(item + kWsKP + 2 * TILE + c16 * 16) = pc[e];
-        }
-        // blocks (bi, bj), bj > bi, of T' and T'': 16 rows x two 16-byte chunks each, zero
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int z = e * 192 + t6;   // 384 chunks
-            const int img = z / 192, w = z % 192, blk = w >> 5, rr = (w >> 1) & 15, hc = w & 1;
-            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-            const int bj = bi + 1 + blk - (bi == 0 ? 0 : (bi == 1 ? 3 : 5));
-            *reinterpret_cast<uint4 *>(sm + (img ? P_OFF_TPP : P_OFF_TP) + swz(bi * 16 + rr, 2 * bj + hc)) =
-                make_uint4(0u, 0u, 0u, 0u);
-        }
+        // the per-token factors of the state update, c_r = gamma_C / gamma_r / |k_r|, and gamma_C
+        if (t6 < 64) reinterpret_cast<float *>(item + kWsVec)[t6] = sDec[t6];
+        if (t6 == 64) reinterpret_cast<float *>(item + kWsVec)[64] = L > 0 ? __expf(sG[L - 1]) : 1.0f;
+        // column factors of T' = T diag(beta gamma / |k|)
+        if (t6 >= 128) sBG[t6 - 128] = sBeta[t6 - 128] * sGam[t6 - 128] * sRk[t6 - 128];
     }
     __syncthreads();
-    if (warp < 3) {
-        // off-diagonal blocks level by level, from T (I + A) = I:
-        //   T_ij = -(sum_{k=j+1}^{i} T_ik A_kj) T_jj,
-        // one warp per block on the warp-level tensor-core MMA (fp16 inputs, fp32 accumulation);
-        // the sum's accumulator fragments are directly the A fragments of the product with T_jj.
-        // Warps 0-2 meet at a named barrier between levels.
+    // ---- off-diagonal blocks level by level, from T (I + A) = I:
+    //      X = sum_{k in blocks bj+1 .. bi} T[r][k] A[k][c],   T[r][c] = -(X T_jj)[r][c],
+    //      r in block bi, c in block bj; every thread one element of each block of the level.
 #pragma unroll 1
-        for (int lvl = 1; lvl < 4; ++lvl) {
-            if (warp < 4 - lvl) {
-                const int bj = warp, bi = bj + lvl;
-                const int g = lane >> 2, t = lane & 3;
-                float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                for (int bk = bj + 1; bk <= bi; ++bk) {
-                    const uint32_t *trow0 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g) * P_AH + bk * 16);
-                    const uint32_t *trow1 = reinterpret_cast<const uint32_t *>(Th + (bi * 16 + g + 8) * P_AH + bk * 16);
-                    const uint32_t a0 = trow0[t], a1 = trow1[t], a2 = trow0[t + 4], a3 = trow1[t + 4];
-#pragma unroll
-                    for (int hn = 0; hn < 2; ++hn) {
-                        const int col = bj * 16 + hn * 8 + g;
-                        const uint32_t b0 = pack_two_h(Ah[(bk * 16 + 2 * t) * P_AH + col], Ah[(bk * 16 + 2 * t + 1) * P_AH + col]);
-                        const uint32_t b1 = pack_two_h(Ah[(bk * 16 + 2 * t + 8) * P_AH + col], Ah[(bk * 16 + 2 * t + 9) * P_AH + col]);
-                        mma_m16n8k16(y[hn], a0, a1, a2, a3, b0, b1);
-                    }
-                }
-                const uint32_t a0 = pack_h2(y[0][0], y[0][1]), a1 = pack_h2(y[0][2], y[0][3]);
-                const uint32_t a2 = pack_h2(y[1][0], y[1][1]), a3 = pack_h2(y[1][2], y[1][3]);
-#pragma unroll
-                for (int hn = 0; hn < 2; ++hn) {
-                    const int col = bj * 16 + hn * 8 + g;
-                    const uint32_t b0 = pack_two_h(Th[(bj * 16 + 2 * t) * P_AH + col], Th[(bj * 16 + 2 * t + 1) * P_AH + col]);
-                    const uint32_t b1 = pack_two_h(Th[(bj * 16 + 2 * t + 8) * P_AH + col], Th[(bj * 16 + 2 * t + 9) * P_AH + col]);
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_m16n8k16(d, a0, a1, a2, a3, b0, b1);
-                    const int c0 = bj * 16 + hn * 8 + 2 * t;
-                    const float fb0 = sBeta[c0], fb1 = sBeta[c0 + 1];
-                    const float fg0 = fb0 * sGam[c0] * sRk[c0], fg1 = fb1 * sGam[c0 + 1] * sRk[c0 + 1];
-#pragma unroll
-                    for (int hr = 0; hr < 2; ++hr) {
-                        const int s = bi * 16 + g + 8 * hr;
-                        const float t0v = -d[2 * hr], t1v = -d[2 * hr + 1];
-                        const uint32_t off = swz(s, c0 >> 3) + (c0 & 7) * 2;
-                        *reinterpret_cast<uint32_t *>(Th + s * P_AH + c0) = pack_h2(t0v, t1v);
-                        *reinterpret_cast<uint32_t *>(sm + P_OFF_TPP + off) = pack_h2(t0v * fb0, t1v * fb1);
-                        *reinterpret_cast<uint32_t *>(sm + P_OFF_TP + off) = pack_h2(t0v * fg0, t1v * fg1);
-                    }
-                }
+    for (int lvl = 1; lvl < 4; ++lvl) {
+        const int nb = 4 - lvl;
+        const int rr = tid / 16, cc = tid % 16;
+        for (int m = 0; m < nb; ++m) {
+            const int bj = m, bi = m + lvl, r = bi * 16 + rr, c = bj * 16 + cc;
+            float acc = 0.0f;
+            for (int k = (bj + 1) * 16; k < bi * 16 + 16; ++k) {
+                const float t = (k < r) ? AT[k * P_AT + r] : (k == r ? 1.0f : 0.0f);
+                acc = fmaf(t, AT[k * P_AT + c], acc);
             }
-            asm volatile("barrier.cta.sync 1, 96;" ::: "memory");
+            Xs[m * 272 + rr * 17 + cc] = acc;
         }
-    } else {
-        // meanwhile warps 3-7: V converted to fp16 in place once its tiles have landed, then K''
-        // (the first two blocks of [K''; P^T]) from the raw bf16 K tile, scaled row by row with the
-        // swizzle positions unchanged, and K converted to fp16 in place (V and K are the B operand
-        // of MMA2); 1024 chunks over 160 threads, loads issued before the stores
-        const int t5 = tid - 96;
-        okv = mbar_wait(bar_v, 0, status) ? 1 : 0;
-        if (okv) {
-            for (int idx = t5; idx < 1024; idx += 160)
-                convert16(sm + P_OFF_VLO + (idx >> 9) * 2 * TILE + (idx & 511) * 16);
-        }
-#pragma unroll 1
-        for (int batch = 0; batch < 2; ++batch) {
-            uint4 hv[4];
-            float f[4];
+        __syncthreads();
+        for (int m = 0; m < nb; ++m) {
+            const int bj = m, bi = m + lvl, r = bi * 16 + rr, c = bj * 16 + cc;
+            float acc = 0.0f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int idx = (batch * 4 + e) * 160 + t5;
-                const int w = idx < 1024 ? idx : 0, half = w >> 9, within = w & 511, r = within >> 3;
-                hv[e] = *reinterpret_cast<const uint4 *>(sm + P_OFF_KQ + 2 * half * TILE + within * 16);
-                f[e] = sDec[r];
+            for (int k2 = 0; k2 < 16; ++k2) {
+                const int k = bj * 16 + k2;
+                const float t = (k > c) ? AT[c * P_AT + k] : (k == c ? 1.0f : 0.0f);
+                acc = fmaf(Xs[m * 272 + rr * 17 + k2], t, acc);
             }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int idx = (batch * 4 + e) * 160 + t5;
-                if (idx < 1024) {
-                    const int half = idx >> 9, within = idx & 511;
-                    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&hv[e]);
-                    float raw[8], xv[8];
-#pragma unroll
-                    for (int q2 = 0; q2 < 4; ++q2) {
-                        const float2 t = __bfloat1622float2(b2[q2]);
-                        raw[2 * q2] = t.x;
-                        raw[2 * q2 + 1] = t.y;
-                        xv[2 * q2] = t.x * f[e];
-                        xv[2 * q2 + 1] = t.y * f[e];
-                    }
-                    st_h8(item + kWsKP + half * TILE + within * 16, xv);
-                    st_h8(sm + P_OFF_KQ + 2 * half * TILE + within * 16, raw);
-                }
-            }
+            AT[c * P_AT + r] = -acc;
         }
+        __syncthreads();
     }
-    if (!__syncthreads_and(okv)) goto teardown;
+    // ---- the A operands of MMA2 as bf16 hi / lo K-major images (128-byte swizzle):
+    //      rows 0-63 T' = T diag(beta gamma / |k|), rows 64-127 T'' = T diag(beta)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int idx = e * NT + tid, r = idx >> 3, ch = idx & 7;
+        float t[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int s = ch * 8 + j;
+            t[j] = (s < r) ? AT[s * P_AT + r] : (s == r ? 1.0f : 0.0f);
+        }
+        uint32_t h1[4], l1[4], h2[4], l2[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int s = ch * 8 + 2 * j;
+            split_bf16x2(t[2 * j] * sBG[s], t[2 * j + 1] * sBG[s + 1], h1[j], l1[j]);
+            split_bf16x2(t[2 * j] * sBeta[s], t[2 * j + 1] * sBeta[s + 1], h2[j], l2[j]);
+        }
+        const uint32_t off = swz(r, ch);
+        *reinterpret_cast<uint4 *>(sm + P_OFF_AHI + off) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+        *reinterpret_cast<uint4 *>(sm + P_OFF_AHI + 8 * 1024 + off) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+        *reinterpret_cast<uint4 *>(sm + P_OFF_ALO + off) = make_uint4(l1[0], l1[1], l1[2], l1[3]);
+        *reinterpret_cast<uint4 *>(sm + P_OFF_ALO + 8 * 1024 + off) = make_uint4(l2[0], l2[1], l2[2], l2[3]);
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
-        // D2 = [T'; T''] [K | V]: lanes 0-63 columns 0-127 hold W = T' K, lanes 64-127
-        // columns 128-255 hold U~ = T'' V (the other two quadrants are not used)
-        tc_fence_after();
-        const uint32_t id2 = idesc_f16(256, false, true, false);
+        // D2 = [T'; T''] [K | V] with the hi and lo parts of the A operand accumulated: lanes 0-63
+        // columns 0-127 hold W = T' K, lanes 64-127 columns 128-255 hold U~ = T'' V (the other two
+        // quadrants are not used). K and V are the raw bf16 tiles.
+        ok = mbar_wait(bar_v, 0, status) ? 1 : 0;
+        if (ok) {
+            tc_fence_after();
+            const uint32_t id2 = idesc_f16(256, false, true, false) | (1u << 7) | (1u << 10);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tmem + P_TM_D2, kdesc(sm + P_OFF_TP + kk * 32), mndesc(sm + P_OFF_KQ + kk * 2048, 2 * TILE), id2,
-                    kk > 0 ? 1u : 0u);
-        tc_commit(bar_mma);
+            for (int kk = 0; kk < 8; ++kk)
+                mma_f16(tmem + P_TM_D2, kdesc(sm + (kk < 4 ? P_OFF_AHI : P_OFF_ALO) + (kk & 3) * 32),
+                        mndesc(sm + P_OFF_KLO + (kk & 3) * 2048, 3 * TILE), id2, kk > 0 ? 1u : 0u);
+            tc_commit(bar_mma);
+            mmas_issued = 2;
+            ok = mbar_wait(bar_mma, 1, status) ? 1 : 0;
+        }
     }
-    if (tid == 0) ok = mbar_wait(bar_mma, 1, status) ? 1 : 0;
-    if (!__syncthreads_and(ok)) goto teardown;
+    if (!__syncthreads_and(ok)) { failed = true; goto teardown; }
     tc_fence_after();
     {
-        // W rows (K-major swizzled image halves) and U~ rows ([s][i], chunk positions XOR-swizzled
-        // by s & 7) staged in the dead tile area, then copied out in 16-byte chunks
+        // W rows (fp16, K-major swizzled image halves) and U~ rows (fp32 [s][i], 16-byte groups
+        // XOR-swizzled by s & 7) staged in the dead tile area, then copied out in 16-byte chunks
         uint32_t v0[32], v1[32];
         const uint32_t col = (x < 64 ? 0u : 128u) + (uint32_t)wg * 64;
         tmem_ld32(tmem + P_TM_D2 + lane_base + col, v0);
         tmem_ld32(tmem + P_TM_D2 + lane_base + col + 32, v1);
         tmem_ld_wait();
+        if (x < 64) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            float f8[8];
+            for (int c = 0; c < 8; ++c) {
+                float f8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(c < 4 ? v0[c * 8 + e] : v1[(c - 4) * 8 + e]);
-            if (x < 64) st_h8(sm + P_OFF_STG + wg * TILE + swz(x, c), f8);
-            else {
-                const int s = x - 64;
-                st_h8(sm + P_OFF_STG + 2 * TILE + s * 256 + wg * 128 + ((c ^ (s & 7)) << 4), f8);
+                for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(c < 4 ? v0[c * 8 + e] : v1[(c - 4) * 8 + e]);
+                st_h8(sm + P_OFF_WSTG + wg * TILE + swz(x, c), f8);
+            }
+        } else {
+            const int s = x - 64;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const uint32_t *src = c < 8 ? &v0[c * 4] : &v1[(c - 8) * 4];
+                const int g16 = wg * 16 + c;
+                *reinterpret_cast<uint4 *>(sm + P_OFF_USTG + s * 512 + ((g16 ^ (s & 7)) << 4)) =
+                    make_uint4(src[0], src[1], src[2], src[3]);
             }
         }
     }
     __syncthreads();
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const int idx = e * NT + tid;   // 1024 chunks of W, then 1024 of U~
-        const uint8_t *src = sm + P_OFF_STG + idx * 16;
-        uint8_t *dst;
+    for (int e = 0; e < 12; ++e) {
+        const int idx = e * NT + tid;   // 1024 chunks of W, then 2048 of U~
         if (idx < 1024) {
-            dst = item + kWsWQ + (idx >> 9) * 2 * TILE + (idx & 511) * 16;
+            *reinterpret_cast<uint4 *>(item + kWsWQ + (idx >> 9) * 2 * TILE + (idx & 511) * 16) =
+                *reinterpret_cast<const uint4 *>(sm + P_OFF_WSTG + idx * 16);
         } else {
-            const int u = idx - 1024, s = u >> 4, wgp = (u >> 3) & 1, c = (u & 7) ^ (s & 7);
-            dst = item + kWsU + s * 256 + wgp * 128 + c * 16;
+            const int u = idx - 1024, s = u >> 5, g16 = u & 31;
+            *reinterpret_cast<uint4 *>(item + kWsU + u * 16) =
+                *reinterpret_cast<const uint4 *>(sm + P_OFF_USTG + s * 512 + ((g16 ^ (s & 7)) << 4));
         }
-        *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
     }
 teardown:
+    if (failed && tid == 0) {
+        // a wait ran out: before the tensor memory is freed and the CTA exits, wait (bounded) for
+        // what this thread issued - the MMAs through one more commit, the tile loads on their
+        // barriers (each armed once, so parity 0 names its only phase)
+        if (mmas_issued) {
+            tc_commit(bar_drain);
+            mbar_wait(bar_drain, 0, status);
+        }
+        if (loads_issued) {
+            mbar_wait(bar_tma, 0, status);
+            mbar_wait(bar_v, 0, status);
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -636,7 +593,13 @@ constexpr int CH_WORKERS = CH_WARPS * 32;
 constexpr int CH_COLS = 128 / (CH_WARPS / 4);      // state columns per thread
 constexpr int CH_TOK = C / (CH_WARPS / 4);         // chunk tokens per thread in U and o
 constexpr int CH_THREADS = CH_WORKERS + 32;
-constexpr int CH_OFF_STAGE = 2 * kWsItem;          // o staging, [r][i] (bf16 or fp32)
+// per-chunk buffer: [W; Q'] image (32 KB), P^T hi and lo images (16 KB), the raw bf16 K tile (16 KB)
+constexpr int CB_BUF = 65536, CB_WQ = 0, CB_P = 32768, CB_K = 49152;
+constexpr int kVecBytes = 272;                     // c[64] and gamma_C of a chunk
+constexpr int CH_OFF_VEC = 0;                      // two 512-byte slots
+constexpr int CH_OFF_BUF = 1024;                   // two chunk buffers
+constexpr int CH_OFF_U = CH_OFF_BUF + 2 * CB_BUF;  // U~ of the current chunk, fp32 [s][i] (one buffer)
+constexpr int CH_OFF_STAGE = CH_OFF_U + 32768;     // o staging, [r][i] (bf16 or fp32)
 constexpr int CH_OFF_BAR = CH_OFF_STAGE + 64 * 128 * 4;
 constexpr int CH_SMEM = CH_OFF_BAR + 128 + 1024;
 static_assert(CH_SMEM <= 232448, "chain shared memory");
@@ -651,10 +614,16 @@ constexpr int CHF_OFF_RTAB = CHF_OFF_Z + 3 * CHF_ZBYTES;
 constexpr int CHF_OFF_BAR = CHF_OFF_RTAB + 128 * 4;
 constexpr int CHF_SMEM = CHF_OFF_BAR + 128 + 1024;
 static_assert(CHF_SMEM <= 232448, "fused chain shared memory");
-static_assert(CHF_OFF_Z % 1024 == 0, "TMA destination alignment");
-static_assert(kWsItem % 1024 == 0 && kWsKP % 1024 == 0, "1024-byte aligned operand tiles");
-// tensor memory: [D4 | D5a] (MMA45), [D7 | D5b] (MMA67), fp16 S0 (two slots) and U as A operands
-constexpr uint32_t C_TM_D45 = 0, C_TM_D67 = 128, C_TM_SA = 320, C_TM_UA = 448;
+static_assert(CHF_OFF_Z % 1024 == 0 && CB_K % 1024 == 0 && CB_BUF % 1024 == 0 && CH_OFF_BUF % 1024 == 0,
+              "TMA destination alignment");
+static_assert(kWsItem % 1024 == 0 && kWsP % 1024 == 0 && kWsU % 16 == 0 && kWsVec % 16 == 0,
+              "1024-byte aligned operand tiles, 16-byte aligned bulk sources");
+// tensor memory: [D4 | o] (MMA45, then the intra-chunk output accumulated onto o), D7 (state
+// update), fp16 S0 (two slots), U as bf16 hi / lo A operands, U diag(c) as bf16 hi / lo
+constexpr uint32_t C_TM_D45 = 0, C_TM_D7 = 128, C_TM_SA = 256, C_TM_UA = 384, C_TM_UCA = 448;
+
+// kind::f16 instruction descriptor bits for bf16 A and B
+constexpr uint32_t kIdescBf16 = (1u << 7) | (1u << 10);
 
 // tcgen05.mma kind::f16 with the A operand in tensor memory (M = 128, K-major rows on lanes).
 __device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -683,9 +652,10 @@ __device__ __forceinline__ void workers_sync() { asm volatile("barrier.cta.sync 
 enum ChainMode { kChainFull = 0, kChainState = 1, kChainTransition = 2 };
 
 struct ChainParams {
+    CUtensorMap kmap;      // k [T, Hk, 128] bf16, boxes of 64 values x 64 tokens (the state update's B)
     CUtensorMap zmap;      // fused output pass: z [T, Hv, 128] bf16, boxes of 64 values x 64 tokens
     const int32_t *cu_seqlens;
-    int32_t T, num_seqs, Hv, slots, seg_chunks, seg_slots, mode_base, out_bf16;
+    int32_t T, num_seqs, Hk, Hv, slots, seg_chunks, seg_slots, mode_base, out_bf16;
     const float *S0g;
     float *S_out;
     void *o;               // may be null in the fused output pass
@@ -741,12 +711,14 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + (FUSED ? CHF_OFF_BAR : CH_OFF_BAR));
-    uint64_t *full = bars, *bar_u = bars + 2, *bar_s = bars + 3, *bar_uready = bars + 4, *bar_sready = bars + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+    uint64_t *full = bars, *full_u = bars + 2, *bar_u = bars + 3, *bar_s = bars + 4, *bar_uready = bars + 5,
+             *bar_sready = bars + 6, *bar_drain = bars + 7;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int h = blockIdx.x, id = blockIdx.y;
     const int T = P.T, Hv = P.Hv, SEG = P.seg_chunks;
+    const int hk = h / (Hv / P.Hk);
     int n = 0, t_begin = 0, t_end = T;
     if (P.cu_seqlens) {
         int lo = 0, hi = P.num_seqs - 1;
@@ -776,10 +748,12 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
+        mbar_init(full_u, 1);
         mbar_init(bar_u, 1);
         mbar_init(bar_s, 1);
         mbar_init(bar_uready, CH_WARPS);
         mbar_init(bar_sready, CH_WARPS);
+        mbar_init(bar_drain, 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -794,44 +768,94 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
     if (warp == CH_WARPS) {
         // ------------------------------------------------ copy + MMA issue (one thread)
         if (lane == 0) {
+            // issued phases per barrier, for the drain on the failure path
+            int n_full[2] = {0, 0}, n_u = 0, n_mma = 0;
+            bool ok = true;
             auto issue_chunk = [&](int c) {
-                uint64_t *bar = &full[c & 1];
-                mbar_arrive_expect_tx(bar, kWsItem + (FUSED ? CHF_ZBYTES : 0));
-                bulk_load(sm + (c & 1) * kWsItem, ws_h + (size_t)(slot0 + c) * kWsItem, kWsItem, bar);
+                const int b = c & 1;
+                uint64_t *bar = &full[b];
+                uint8_t *buf = sm + CH_OFF_BUF + b * CB_BUF;
+                const uint8_t *item = ws_h + (size_t)(slot0 + c) * kWsItem;
+                const int t0c = t_begin + (c_first + c) * C;
+                mbar_arrive_expect_tx(bar, CB_K + 2 * TILE + kVecBytes + (FUSED ? CHF_ZBYTES : 0));
+                bulk_load(buf + CB_WQ, item + kWsWQ, 4 * TILE, bar);
+                bulk_load(buf + CB_P, item + kWsP, 2 * TILE, bar);
+                bulk_load(sm + CH_OFF_VEC + b * 512, item + kWsVec, kVecBytes, bar);
+                tma_load_3d(buf + CB_K, &P.kmap, bar, 0, hk, t0c);
+                tma_load_3d(buf + CB_K + TILE, &P.kmap, bar, 64, hk, t0c);
                 if constexpr (FUSED) {   // this chunk's z rows, two boxes of 64 values
-                    const int t0c = t_begin + (c_first + c) * C;
                     uint8_t *zb = sm + CHF_OFF_Z + (c % 3) * CHF_ZBYTES;
                     tma_load_3d(zb, &P.zmap, bar, 0, h, t0c);
                     tma_load_3d(zb + TILE, &P.zmap, bar, 64, h, t0c);
                 }
+                ++n_full[b];
             };
-            if (nchunks > 0) issue_chunk(0);
+            auto issue_u = [&](int c) {
+                mbar_arrive_expect_tx(full_u, 4 * TILE);
+                bulk_load(sm + CH_OFF_U, ws_h + (size_t)(slot0 + c) * kWsItem + kWsU, 4 * TILE, full_u);
+                ++n_u;
+            };
+            // with a caller's initial state the workers stage it over buffer 1 and the head of the
+            // U~ buffer: the first U~ load then waits until they have released it (bar_sready)
+            const bool s0_staged = pseg == 0 && S0g;
+            if (nchunks > 0) {
+                issue_chunk(0);
+                if (!s0_staged) issue_u(0);
+            }
             const uint32_t id45 = idesc_f16(128, false, false, false);
-            const uint32_t id67 = idesc_f16(192, false, true, false);
+            const uint32_t id7 = idesc_f16(128, false, true, false) | kIdescBf16;
+            const uint32_t id5 = idesc_f16(64, false, true, false) | kIdescBf16;
             for (int c = 0; c < nchunks; ++c) {
                 const int b = c & 1;
-                const uint8_t *buf = sm + b * kWsItem;
-                if (!mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status)) break;
-                if (!mbar_wait(bar_sready, (uint32_t)(c & 1), status)) break;
+                const uint8_t *buf = sm + CH_OFF_BUF + b * CB_BUF;
+                if (!(ok = mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status))) break;
+                if (!(ok = mbar_wait(bar_sready, (uint32_t)(c & 1), status))) break;
+                if (c == 0 && s0_staged) issue_u(0);
                 tc_fence_after();
-                // [D4 | D5a] = S0 [W; Q']^T   (B: 128 K-major rows, K = 128 key columns)
+                // [D4 | D5a] = S0 [W; Q']^T   (fp16; B: 128 K-major rows, K = 128 key columns)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_f16_ts(tmem + C_TM_D45, tmem + C_TM_SA + b * 64 + kk * 8,
-                               kdesc(buf + kWsWQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32), id45, kk > 0);
+                               kdesc(buf + CB_WQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32), id45, kk > 0);
                 tc_commit(bar_u);
+                ++n_mma;
                 if (c + 1 < nchunks) {   // the other buffer's readers (chunk c-1) are done
                     fence_proxy_async_smem();
                     issue_chunk(c + 1);
                 }
-                if (!mbar_wait(bar_uready, (uint32_t)(c & 1), status)) break;
+                if (!(ok = mbar_wait(bar_uready, (uint32_t)(c & 1), status))) break;
+                if (c + 1 < nchunks) {   // every worker has read this chunk's U~
+                    fence_proxy_async_smem();
+                    issue_u(c + 1);
+                }
                 tc_fence_after();
-                // [D7 | D5b] = U^T [K''; P^T]^T   (B: three MN-major blocks of 64, K = 64 tokens)
+                // D7 = (U diag(c))^T K with U diag(c) as bf16 hi + lo and the raw bf16 K (MN-major,
+                // two blocks of 64 keys); then o += U^T P^T with U and P^T as bf16 hi / lo
+                // (hi hi + hi lo + lo hi), accumulated onto the D5a columns
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_f16_ts(tmem + C_TM_D67, tmem + C_TM_UA + kk * 8, mndesc(buf + kWsKP + kk * 2048, TILE), id67,
-                               kk > 0);
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16_ts(tmem + C_TM_D7, tmem + C_TM_UCA + part * 32 + kk * 8,
+                                   mndesc(buf + CB_K + kk * 2048, TILE), id7, (part | kk) ? 1u : 0u);
+#pragma unroll
+                for (int part = 0; part < 3; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16_ts(tmem + C_TM_D45 + 64, tmem + C_TM_UA + (part == 2 ? 32 : 0) + kk * 8,
+                                   mndesc(buf + CB_P + (part == 1 ? TILE : 0) + kk * 2048, TILE), id5, 1u);
                 tc_commit(bar_s);
+            }
+            if (!ok) {
+                // a wait ran out: wait (bounded) for this thread's MMAs and for the latest phase of
+                // every barrier it armed before the CTA frees its tensor memory and exits
+                if (n_mma) {
+                    tc_commit(bar_drain);
+                    mbar_wait(bar_drain, 0, status);
+                }
+                for (int b = 0; b < 2; ++b)
+                    if (n_full[b]) mbar_wait(&full[b], (uint32_t)((n_full[b] - 1) & 1), status);
+                if (n_u) mbar_wait(full_u, (uint32_t)((n_u - 1) & 1), status);
             }
         }
     } else {
@@ -878,10 +902,10 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             }
         };
         if (pseg == 0 && S0g) {
-            // the caller's row-major initial state, staged in buffer 1 (its first chunk load is
-            // issued only after every worker has released S0 through bar_sready)
+            // the caller's row-major initial state, staged over chunk buffer 1 and the head of the
+            // U~ buffer (neither is loaded before the workers release S0 through bar_sready)
             const float4 *src = reinterpret_cast<const float4 *>(S0g + ((size_t)n * Hv + h) * D * D);
-            uint8_t *stg = sm + kWsItem;
+            uint8_t *stg = sm + CH_OFF_BUF + CB_BUF;
 #pragma unroll 4
             for (int e = 0; e < 4096 / CH_WORKERS; ++e) {
                 const int f = e * CH_WORKERS + tid;
@@ -893,6 +917,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
                 const float4 x = *reinterpret_cast<const float4 *>(stg + row * kStgPitch + cq * CH_COLS * 4 + c4 * 16);
                 S[4 * c4] = x.x; S[4 * c4 + 1] = x.y; S[4 * c4 + 2] = x.z; S[4 * c4 + 3] = x.w;
             }
+            workers_sync();
         } else if (pseg > 0) {
             ilv_load32(seg_item + kSegS, row, cq, S);
         } else {
@@ -917,36 +942,42 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             const int t0 = t_begin + (c_first + c) * C;
             const int L = min(C, t_end - t0);
             const int b = c & 1;
-            const uint8_t *buf = sm + b * kWsItem;
+            const float *vecb = reinterpret_cast<const float *>(sm + CH_OFF_VEC + b * 512);
             const uint32_t ph = (uint32_t)(c & 1);
 
             int ok = 1;
             if (tid == 0)
-                ok = (mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status) && mbar_wait(bar_u, ph, status)) ? 1 : 0;
+                ok = (mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status) && mbar_wait(bar_u, ph, status) &&
+                      mbar_wait(full_u, ph, status))
+                         ? 1 : 0;
             if (!workers_and(ok)) { alive = false; break; }
             tc_fence_after();
             {
-                // U^T = U~^T - D4 as the fp16 A operand of MMA67; this thread: tokens 16 cq .. + 15
-                const __half *ut = reinterpret_cast<const __half *>(buf + kWsU);
-                __half2 u2[CH_TOK / 2];
+                // U^T = U~^T - D4 (fp32) for tokens 16 cq .. + 15 of this row, then U and U diag(c)
+                // as bf16 hi / lo A operands
+                const float *ut = reinterpret_cast<const float *>(sm + CH_OFF_U);
+                float uv[CH_TOK], cv[CH_TOK];
 #pragma unroll
-                for (int w = 0; w < CH_TOK / 2; ++w) {
-                    const int s0 = cq * CH_TOK + 2 * w;
-                    u2[w] = __halves2half2(ut[s0 * D + row], ut[(s0 + 1) * D + row]);
+                for (int w = 0; w < CH_TOK; ++w) {
+                    uv[w] = ut[(cq * CH_TOK + w) * D + row];
+                    cv[w] = vecb[cq * CH_TOK + w];
                 }
                 uint32_t r16[16];
                 tmem_ld16(tmem + C_TM_D45 + lane_base + cq * CH_TOK, r16);
                 tmem_ld_wait();
-                uint32_t ua[8];
+                uint32_t uh[8], ul[8], ch[8], cl[8];
 #pragma unroll
                 for (int w = 0; w < CH_TOK / 2; ++w) {
                     const int s0 = cq * CH_TOK + 2 * w;
-                    const float2 uf = __half22float2(u2[w]);
-                    const float u0 = (s0 < L) ? uf.x - __uint_as_float(r16[2 * w]) : 0.0f;
-                    const float u1 = (s0 + 1 < L) ? uf.y - __uint_as_float(r16[2 * w + 1]) : 0.0f;
-                    ua[w] = pack_h2(u0, u1);
+                    const float u0 = (s0 < L) ? uv[2 * w] - __uint_as_float(r16[2 * w]) : 0.0f;
+                    const float u1 = (s0 + 1 < L) ? uv[2 * w + 1] - __uint_as_float(r16[2 * w + 1]) : 0.0f;
+                    split_bf16x2(u0, u1, uh[w], ul[w]);
+                    split_bf16x2(u0 * cv[2 * w], u1 * cv[2 * w + 1], ch[w], cl[w]);
                 }
-                tmem_st8(tmem + lane_base + C_TM_UA + cq * (CH_TOK / 2), ua);
+                tmem_st8(tmem + lane_base + C_TM_UA + cq * (CH_TOK / 2), uh);
+                tmem_st8(tmem + lane_base + C_TM_UA + 32 + cq * (CH_TOK / 2), ul);
+                tmem_st8(tmem + lane_base + C_TM_UCA + cq * (CH_TOK / 2), ch);
+                tmem_st8(tmem + lane_base + C_TM_UCA + 32 + cq * (CH_TOK / 2), cl);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -957,18 +988,17 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             tc_fence_after();
             float ov[CH_TOK];
             {
-                // o^T = D5a + D5b for tokens 16 cq .. + 15; S <- gamma_C S + D7 for this quarter
-                uint32_t a5[16], b5[16], r7[32];
+                // o^T (D5a + the intra-chunk part) for tokens 16 cq .. + 15; S <- gamma_C S + D7
+                uint32_t a5[16], r7[32];
                 tmem_ld16(tmem + C_TM_D45 + lane_base + 64 + cq * CH_TOK, a5);
-                tmem_ld16(tmem + C_TM_D67 + lane_base + 128 + cq * CH_TOK, b5);
-                tmem_ld32(tmem + C_TM_D67 + lane_base + cq * CH_COLS, r7);
+                tmem_ld32(tmem + C_TM_D7 + lane_base + cq * CH_COLS, r7);
                 tmem_ld_wait();
-                const float gC = reinterpret_cast<const float *>(buf + kWsVec)[0];
+                const float gC = vecb[64];
 #pragma unroll
                 for (int j = 0; j < CH_COLS; ++j) S[j] = gC * S[j] + __uint_as_float(r7[j]);
                 store_S(b ^ 1);   // S0 of chunk c + 1; releases the MMA warp
 #pragma unroll
-                for (int j = 0; j < CH_TOK; ++j) ov[j] = __uint_as_float(a5[j]) + __uint_as_float(b5[j]);
+                for (int j = 0; j < CH_TOK; ++j) ov[j] = __uint_as_float(a5[j]);
             }
             if (FUSED) {
                 // stage this chunk's o rows (bf16 [r][i]; the previous chunk's encode is done, a
@@ -996,16 +1026,16 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
                 const int per_row = row_bytes / 16;
                 uint8_t *ob = static_cast<uint8_t *>(P.o);
                 for (int e = tid; e < L * per_row; e += CH_WORKERS) {
-                    const int r = e / per_row, ch = e % per_row;
-                    const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + ch * 16);
-                    *reinterpret_cast<uint4 *>(ob + (((size_t)(t0 + r) * Hv + h) * D) * (row_bytes / D) + ch * 16) = val;
+                    const int r = e / per_row, chn = e % per_row;
+                    const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + chn * 16);
+                    *reinterpret_cast<uint4 *>(ob + (((size_t)(t0 + r) * Hv + h) * D) * (row_bytes / D) + chn * 16) = val;
                 }
                 workers_sync();
             }
         }
         if (alive && last_seg && P.S_out) {
-            // all chunks are consumed: both operand buffers are free for staging the final state
-            uint8_t *stg = sm;
+            // all chunks are consumed: the chunk buffers are free for staging the final state
+            uint8_t *stg = sm + CH_OFF_BUF;
 #pragma unroll
             for (int c4 = 0; c4 < CH_COLS / 4; ++c4)
                 *reinterpret_cast<float4 *>(stg + row * kStgPitch + cq * CH_COLS * 4 + c4 * 16) =
@@ -1029,17 +1059,22 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
 
 
 // ===================================================================================
-// Lean chain kernel for the state and transition passes (no outputs). A buffer holds only W,
-// K'', U~ and gamma_C of a chunk; 256 threads, thread 0 also issuing the copies and the MMAs;
-// 256 tensor-memory columns and at most 128 registers, so that two CTAs share an SM.
+// Lean chain kernel for the state and transition passes (no outputs). A buffer holds W, the raw
+// K tile and the chunk's c and gamma_C; U~ (state pass only) has one buffer of its own, refilled
+// as soon as every thread has read it. 256 threads, thread 0 also issuing the copies and the
+// MMAs; 256 tensor-memory columns and at most 128 registers, so that two CTAs share an SM. The
+// two passes of a segment are adjacent blocks (blockIdx.x = 2 h + pass) and the two value heads
+// of a key head are neighbours too, so W and K reach the four CTAs from L2 after one HBM read.
 // ===================================================================================
-constexpr int CL_W = 0, CL_K = 2 * TILE, CL_U = 4 * TILE, CL_VEC = 6 * TILE;
-constexpr int CL_BUF = 6 * TILE + 1024;
-constexpr int CL_OFF_BAR = 2 * CL_BUF;
-constexpr int CL_SMEM = CL_OFF_BAR + 64 + 1024;
-static_assert(2 * CL_SMEM <= 228 * 1024, "two lean chain CTAs per SM");
-// D4 (64 columns) and D7 (128) share columns: D4 is read out before MMA67 is issued
-constexpr uint32_t CL_TM_D4 = 0, CL_TM_D7 = 0, CL_TM_SA = 128, CL_TM_UA = 192;
+constexpr int CL_W = 0, CL_K = 2 * TILE, CL_VEC = 4 * TILE;
+constexpr int CL_BUF = 4 * TILE + 1024;
+constexpr int CL_U = 2 * CL_BUF;
+constexpr int CL_OFF_BAR = CL_U + 4 * TILE;
+constexpr int CL_SMEM = CL_OFF_BAR + 128 + 1024;
+static_assert(2 * (CL_SMEM + 1024) <= 233472, "two lean chain CTAs per SM");
+static_assert(CL_BUF % 1024 == 0 && CL_K % 1024 == 0, "TMA destination alignment");
+// D4 (64 columns) and D7 (128) share columns: D4 is read out before MMA7 is issued
+constexpr uint32_t CL_TM_D4 = 0, CL_TM_D7 = 0, CL_TM_SA = 128, CL_TM_UCA = 192;
 
 __global__ void __launch_bounds__(NT, 2)
 gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
@@ -1048,14 +1083,16 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CL_OFF_BAR);
-    // full[2]: chunk copies; bar45 / bar67: MMA completion; bar_s / bar_u: the eight warps
-    // have stored S0 / U into tensor memory (one arrival per warp)
-    uint64_t *full = bars, *bar45 = bars + 2, *bar67 = bars + 3, *bar_s = bars + 4, *bar_u = bars + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+    // full[2]: chunk copies; full_u: U~; bar45 / bar67: MMA completion; bar_s / bar_u: the eight
+    // warps have stored S0 / U into tensor memory (one arrival per warp); bar_drain: failure path
+    uint64_t *full = bars, *full_u = bars + 2, *bar45 = bars + 3, *bar67 = bars + 4, *bar_s = bars + 5,
+             *bar_u = bars + 6, *bar_drain = bars + 7;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int h = blockIdx.x, id = blockIdx.y, mode = kChainState + (int)blockIdx.z;
+    const int h = blockIdx.x >> 1, id = blockIdx.y, mode = kChainState + (int)(blockIdx.x & 1);
     const int T = P.T, Hv = P.Hv, SEG = P.seg_chunks;
+    const int hk = h / (Hv / P.Hk);
     int n = 0, t_begin = 0, t_end = T;
     if (P.cu_seqlens) {
         int lo = 0, hi = P.num_seqs - 1;
@@ -1085,10 +1122,12 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
+        mbar_init(full_u, 1);
         mbar_init(bar45, 1);
         mbar_init(bar67, 1);
         mbar_init(bar_s, 8);
         mbar_init(bar_u, 8);
+        mbar_init(bar_drain, 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -1099,20 +1138,31 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // issued phases per barrier (thread 0), for the drain on the failure path
+    int n_full[2] = {0, 0}, n_u = 0, n_mma = 0;
     auto issue_chunk = [&](int c) {
-        uint64_t *bar = &full[c & 1];
-        uint8_t *dst = sm + (c & 1) * CL_BUF;
+        const int b = c & 1;
+        uint64_t *bar = &full[b];
+        uint8_t *dst = sm + b * CL_BUF;
         const uint8_t *item = ws_h + (size_t)(slot0 + c) * kWsItem;
-        mbar_arrive_expect_tx(bar, 4 * TILE + (with_u ? 2 * TILE : 0) + 16);
+        const int t0c = t_begin + (c_first + c) * C;
+        mbar_arrive_expect_tx(bar, 4 * TILE + kVecBytes);
         bulk_load(dst + CL_W, item + kWsWQ, TILE, bar);
         bulk_load(dst + CL_W + TILE, item + kWsWQ + 2 * TILE, TILE, bar);
-        bulk_load(dst + CL_K, item + kWsKP, 2 * TILE, bar);
-        if (with_u) bulk_load(dst + CL_U, item + kWsU, 2 * TILE, bar);
-        bulk_load(dst + CL_VEC, item + kWsVec, 16, bar);
+        tma_load_3d(dst + CL_K, &P.kmap, bar, 0, hk, t0c);
+        tma_load_3d(dst + CL_K + TILE, &P.kmap, bar, 64, hk, t0c);
+        bulk_load(dst + CL_VEC, item + kWsVec, kVecBytes, bar);
+        ++n_full[b];
+    };
+    auto issue_u = [&](int c) {
+        mbar_arrive_expect_tx(full_u, 4 * TILE);
+        bulk_load(sm + CL_U, ws_h + (size_t)(slot0 + c) * kWsItem + kWsU, 4 * TILE, full_u);
+        ++n_u;
     };
     if (tid == 0) {
         if (nchunks > 0) issue_chunk(0);
         if (nchunks > 1) issue_chunk(1);
+        if (with_u && nchunks > 0) issue_u(0);
     }
 
     const int wg = warp / 4;
@@ -1155,12 +1205,13 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
     store_S();
 
     const uint32_t id45 = idesc_f16(64, false, false, false);
-    const uint32_t id67 = idesc_f16(128, false, true, false);
+    const uint32_t id7 = idesc_f16(128, false, true, false) | kIdescBf16;
     for (int c = 0; c < nchunks; ++c) {
         const int L = min(C, t_end - (t_begin + (c_first + c) * C));
         const int b = c & 1;
         const uint32_t ph = (uint32_t)(c & 1);
         const uint8_t *buf = sm + b * CL_BUF;
+        const float *vecb = reinterpret_cast<const float *>(buf + CL_VEC);
         if (tid == 0) {
             wait(bar_s, ph);                                // S0 of this chunk is in tensor memory
             wait(&full[b], (uint32_t)((c >> 1) & 1));
@@ -1172,37 +1223,36 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
                     mma_f16_ts(tmem + CL_TM_D4, tmem + CL_TM_SA + kk * 8,
                                kdesc(buf + CL_W + (kk < 4 ? 0 : TILE) + (kk & 3) * 32), id45, kk > 0);
                 tc_commit(bar45);
+                ++n_mma;
             }
         }
-        wait(&full[b], (uint32_t)((c >> 1) & 1));           // this chunk's U~ and gamma_C are visible
+        wait(&full[b], (uint32_t)((c >> 1) & 1));           // this chunk's c and gamma_C are visible
+        if (with_u) wait(full_u, ph);
         wait(bar45, ph);
         tc_fence_after();
-        const float gC = reinterpret_cast<const float *>(buf + CL_VEC)[0];
+        const float gC = vecb[64];
         {
-            // U^T = U~^T - D4 (the transition pass takes U~ = 0) as the fp16 A operand of MMA67;
-            // this thread's 32 values of U~ are loaded before any tensor-memory access
-            const __half *ut = reinterpret_cast<const __half *>(buf + CL_U);
-            __half2 u2[16];
-#pragma unroll
-            for (int w = 0; w < 16; ++w) {
-                const int s0 = wg * 32 + 2 * w;
-                u2[w] = with_u ? __halves2half2(ut[s0 * D + row], ut[(s0 + 1) * D + row]) : __float2half2_rn(0.0f);
-            }
+            // U^T = U~^T - D4 (the transition pass takes U~ = 0), scaled per token by c, as the bf16
+            // hi / lo A operands of MMA7, 16 tokens at a time
+            const float *ut = reinterpret_cast<const float *>(sm + CL_U);
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
+                float u16v[16];
+#pragma unroll
+                for (int w = 0; w < 16; ++w) u16v[w] = with_u ? ut[(wg * 32 + part * 16 + w) * D + row] : 0.0f;
                 uint32_t r16[16];
                 tmem_ld16(tmem + CL_TM_D4 + lane_base + wg * 32 + part * 16, r16);
                 tmem_ld_wait();
-                uint32_t ua[8];
+                uint32_t uh[8], ul[8];
 #pragma unroll
                 for (int w = 0; w < 8; ++w) {
                     const int s0 = wg * 32 + part * 16 + 2 * w;
-                    const float2 uf = __half22float2(u2[part * 8 + w]);
-                    const float u0 = (s0 < L) ? uf.x - __uint_as_float(r16[2 * w]) : 0.0f;
-                    const float u1 = (s0 + 1 < L) ? uf.y - __uint_as_float(r16[2 * w + 1]) : 0.0f;
-                    ua[w] = pack_h2(u0, u1);
+                    const float u0 = (s0 < L) ? u16v[2 * w] - __uint_as_float(r16[2 * w]) : 0.0f;
+                    const float u1 = (s0 + 1 < L) ? u16v[2 * w + 1] - __uint_as_float(r16[2 * w + 1]) : 0.0f;
+                    split_bf16x2(u0 * vecb[s0], u1 * vecb[s0 + 1], uh[w], ul[w]);
                 }
-                tmem_st8(tmem + lane_base + CL_TM_UA + wg * 16 + part * 8, ua);
+                tmem_st8(tmem + lane_base + CL_TM_UCA + wg * 16 + part * 8, uh);
+                tmem_st8(tmem + lane_base + CL_TM_UCA + 32 + wg * 16 + part * 8, ul);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -1210,19 +1260,27 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
             if (lane == 0) mbar_arrive(bar_u);
         }
         if (tid == 0) {
-            wait(bar_u, ph);                                // U is in tensor memory, D4 is consumed
+            wait(bar_u, ph);                                // U is in tensor memory, D4 and U~ are consumed
             if (!dead) {
+                if (with_u && c + 1 < nchunks) {
+                    fence_proxy_async_smem();
+                    issue_u(c + 1);
+                }
                 tc_fence_after();
-                // D7 = U^T K''   (B: K'', MN-major blocks of 64 keys, K = 64 tokens)
+                // D7 = (U diag(c))^T K   (A: bf16 hi then lo; B: the raw K tile, MN-major blocks of
+                // 64 keys, K = 64 tokens)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_f16_ts(tmem + CL_TM_D7, tmem + CL_TM_UA + kk * 8, mndesc(buf + CL_K + kk * 2048, TILE),
-                               id67, kk > 0);
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16_ts(tmem + CL_TM_D7, tmem + CL_TM_UCA + part * 32 + kk * 8,
+                                   mndesc(buf + CL_K + kk * 2048, TILE), id7, (part | kk) ? 1u : 0u);
                 tc_commit(bar67);
+                ++n_mma;
             }
         }
         wait(bar67, ph);
-        // this buffer's readers (both MMAs, every thread's U~ and gamma_C) are done: refill it
+        // this buffer's readers (both MMAs, every thread's c and gamma_C) are done: refill it
         if (tid == 0 && !dead && c + 2 < nchunks) {
             fence_proxy_async_smem();
             issue_chunk(c + 2);
@@ -1239,6 +1297,17 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
         store_S();
     }
     const bool alive = __syncthreads_and(!dead);
+    if (!alive && tid == 0) {
+        // a wait ran out somewhere: wait (bounded) for this thread's MMAs and for the latest phase
+        // of every barrier it armed before the tensor memory is freed
+        if (n_mma) {
+            tc_commit(bar_drain);
+            mbar_wait(bar_drain, 0, status);
+        }
+        for (int b = 0; b < 2; ++b)
+            if (n_full[b]) mbar_wait(&full[b], (uint32_t)((n_full[b] - 1) & 1), status);
+        if (n_u) mbar_wait(full_u, (uint32_t)((n_u - 1) & 1), status);
+    }
     if (alive) {
         if (mode == kChainState) {
             ilv_store(const_cast<uint8_t *>(seg_item) + kSegB, row, wg, S);
@@ -1484,9 +1553,11 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
     ChainParams P{};
     const bool fused = c.xq != nullptr;
     if (fused && !make_map3(&P.zmap, c.z, c.T, c.Hv)) return cudaErrorInvalidValue;
+    P.kmap = maps.k;
     P.cu_seqlens = c.cu_seqlens;
     P.T = c.T;
     P.num_seqs = c.num_seqs;
+    P.Hk = c.Hk;
     P.Hv = c.Hv;
     P.slots = slots;
     P.seg_chunks = seg;
@@ -1505,8 +1576,8 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
     P.xq = c.xq;
     P.xs = c.xs;
     if (c.T > kChunk * seg) {   // some sequence may span several segments
-        P.mode_base = kChainState;   // z = 0: segment states (B), z = 1: segment transitions (M)
-        if ((e = launch_pdl(gdn_chunk_lean_kernel, dim3(c.Hv, seg_slots, 2), dim3(NT), CL_SMEM, st, P)) != cudaSuccess)
+        P.mode_base = kChainState;   // x = 2 h: segment states (B), x = 2 h + 1: segment transitions (M)
+        if ((e = launch_pdl(gdn_chunk_lean_kernel, dim3(2 * c.Hv, seg_slots, 1), dim3(NT), CL_SMEM, st, P)) != cudaSuccess)
             return e;
         if ((e = launch_pdl(gdn_segment_combine_kernel, dim3(c.Hv, c.num_seqs, 4), dim3(NT), CB_SMEM, st, P)) != cudaSuccess)
             return e;

@@ -186,8 +186,26 @@ GDN_DEV float amax8(const float (&x)[8]) {
 
 // -------------------------------------------------------------- device status ----
 
+// The library's device control block: the status word that bounded waits report into, the
+// wait limit in nanoseconds (1 s unless lowered for a test) and test switches that make a
+// kernel skip issuing its loads, so that a test can make a wait run out with nothing in flight.
+// Kernels receive the address of `status`; the other fields follow it.
+struct DeviceCtl {
+    int status;
+    unsigned int flags;
+    unsigned long long wait_limit_ns;
+};
+constexpr unsigned int kInjectSkipPrepLoads = 1u;   // the chunked prep kernel issues no tile loads
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
 GDN_DEV void report_status(int *status, int code) {
     if (status) atomicCAS(status, 0, code);
+}
+GDN_DEV unsigned long long ctl_wait_limit(const int *status) {
+    return status ? reinterpret_cast<const volatile DeviceCtl *>(status)->wait_limit_ns : kWaitLimitNs;
+}
+GDN_DEV unsigned int ctl_flags(const int *status) {
+    return status ? reinterpret_cast<const volatile DeviceCtl *>(status)->flags : 0u;
 }
 
 }  // namespace gdn
@@ -230,16 +248,17 @@ GDN_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete, for at most ~1 s of device time.
-// On expiry records GDN_ERR_TIMEOUT in the status word and returns false; callers then
-// stop issuing work and fall through to the kernel's teardown.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+// Wait for the phase with the given parity to complete, for at most the control block's wait
+// limit (1 s by default) of device time. On expiry records GDN_ERR_TIMEOUT in the status word
+// and returns false; callers then stop issuing work, drain what they issued and fall through
+// to the kernel's teardown.
 GDN_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+    const uint64_t limit = ctl_wait_limit(status);
     for (uint32_t i = 0;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u && global_timer_ns() - t0 > kWaitLimitNs) {
+        if ((i & 255u) == 255u && global_timer_ns() - t0 > limit) {
             report_status(status, GDN_ERR_TIMEOUT);
             return false;
         }

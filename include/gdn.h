@@ -325,6 +325,17 @@ GDN_API gdn_status gdn_prefill_chunked_static_ws(const void *q, const void *k, c
  * kernels set on an expired bounded wait, and clears it. */
 GDN_API gdn_status gdn_get_device_status(gdn_stream_t stream);
 
+/* Test support for the timeout path (no counterpart in the pages). Sets, for the current device,
+ * the limit of every bounded device-side wait (wait_limit_ns; 0 restores the default of 1 s, larger
+ * values are GDN_ERR_INVALID_ARG) and switches that make a kernel skip work so that one of its waits
+ * runs out with nothing in flight: GDN_INJECT_SKIP_PREP_LOADS (1) makes the chunked prefill's prep
+ * kernel issue none of its tile loads, so each of its CTAs times out waiting for them, records
+ * GDN_ERR_TIMEOUT and exits (the later kernels of the call then read an unwritten workspace, so
+ * that call's outputs are meaningless). Synchronous; call it with no work of this library in
+ * flight on the device, and call gdn_debug_set_wait(0, 0) to restore normal operation. */
+#define GDN_INJECT_SKIP_PREP_LOADS 1u
+GDN_API gdn_status gdn_debug_set_wait(uint64_t wait_limit_ns, uint32_t inject_flags);
+
 /* Static description of a status code. */
 GDN_API const char *gdn_status_string(gdn_status s);
 
