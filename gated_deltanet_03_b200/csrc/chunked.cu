@@ -170,20 +170,33 @@ __device__ __forceinline__ void locate(int id, const int32_t *cu, int num_seqs, 
     }
 }
 
+// Warp-level 16 x 8 x 16 MMA, bf16 inputs, fp32 accumulation (row-major A, column-major B): the
+// 16 x 16 blocks of the triangular inverse. Fragments: a = {A[g][2t..], A[g+8][2t..], A[g][2t+8..],
+// A[g+8][2t+8..]}, b = {B[2t..][g], B[2t+8..][g]}, c = {C[g][2t], C[g][2t+1], C[g+8][2t], C[g+8][2t+1]}
+// with g = lane / 4, t = lane % 4 (pairs in one 32-bit register, the lower index in the low half).
+__device__ __forceinline__ void mma_bf16_m16n8k16(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 // ===================================================================================
 // Prep kernel: one CTA per (chunk slot, value head); two CTAs per SM.
 // ===================================================================================
 // Shared memory (TILE = 8 KB). [K_lo; Q_lo] and [K_hi; Q_hi] are the two K-major column blocks
 // of the MMA1 operand [K; Q]; K_lo, K_hi, V_lo, V_hi sit 3 TILE apart so that [K | V] is one
 // MN-major B operand with N = 256 for MMA2. The A operands of MMA2 are [T'; T''] split into
-// bf16 hi and lo parts (16 KB each): hi in the free tiles 7-8, lo over Q_lo and the free tile 2
-// once the Q' image is written. After MMA2 the W (fp16) and U~ (fp32) staging reuses tiles 0-5.
+// bf16 hi and lo parts (16 KB each): hi in the free tiles 7-8, lo over Q_lo and tile 2 once the
+// Q' image is written. Tiles 5 and 2 first stage the P^T hi / lo images between the D1 readout
+// and their copy-out. After MMA2 the W (fp16) and U~ (fp32) staging reuses tiles 0-5.
 constexpr int P_OFF_KLO = 0, P_OFF_QLO = TILE, P_OFF_KHI = 3 * TILE, P_OFF_QHI = 4 * TILE;
 constexpr int P_OFF_ALO = TILE;                    // [T'_lo; T''_lo], after the Q' image
-constexpr int P_OFF_X = 5 * TILE;                  // inverse scratch (three 16 x 17 fp32 blocks)
+constexpr int P_OFF_PHI = 5 * TILE, P_OFF_PLO = 2 * TILE;   // P^T hi / lo staging (D1 readout -> copy-out)
 constexpr int P_OFF_VLO = 6 * TILE, P_OFF_AHI = 7 * TILE, P_OFF_VHI = 9 * TILE;
-constexpr int P_AT = 65;                           // fp32 row pitch of the A / T array (odd: no bank conflicts)
-constexpr int P_OFF_AT = 10 * TILE;                // A (strict lower, row-major) and T (strict lower, transposed)
+constexpr int P_AT = 72;                           // fp32 row pitch of the A / T array (8-byte fragment loads
+                                                   // of a warp-level MMA without bank conflicts)
+constexpr int P_OFF_AT = 10 * TILE;                // T (strict lower, row-major) and A (strict lower, transposed)
 constexpr int P_OFF_VEC = P_OFF_AT + 64 * P_AT * 4; // G, beta, rk, rq, gamma, c, beta gamma rk, spare (64 each)
 constexpr int P_OFF_BAR = P_OFF_VEC + 8 * 64 * 4;
 constexpr int P_SMEM = P_OFF_BAR + 64 + 1024;
@@ -224,7 +237,6 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     float *sG = vec, *sBeta = vec + 64, *sRk = vec + 128, *sRq = vec + 192, *sGam = vec + 256, *sDec = vec + 320;
     float *sBG = vec + 384;
     float *AT = reinterpret_cast<float *>(sm + P_OFF_AT);
-    float *Xs = reinterpret_cast<float *>(sm + P_OFF_X);
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + P_OFF_BAR);
     uint64_t *bar_mma = bar_tma + 1;
     uint64_t *bar_v = bar_tma + 2;
@@ -360,10 +372,10 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             }
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                if (wg * 32 + j < r) AT[r * P_AT + wg * 32 + j] = vals[j];
+                if (wg * 32 + j < r) AT[(wg * 32 + j) * P_AT + r] = vals[j];
         } else {
             // row r of P = (Q K^T o Gamma) scaled, as bf16 hi and lo P^T images [s][r] (MN-major
-            // over r, 128-byte swizzled), stored straight to the workspace item
+            // over r, 128-byte swizzled), staged for the copy-out
             const int r = x - 64;
             const float Gr = sG[r], cr = sRq[r];
             const f2_t cr2 = f2(cr, cr);
@@ -380,15 +392,15 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                 const __nv_bfloat16 hb = __float2bfloat16_rn(vals[j]);
                 const __nv_bfloat16 lb = __float2bfloat16_rn(vals[j] - __bfloat162float(hb));
                 const uint32_t off = swz(wg * 32 + j, r >> 3) + (r & 7) * 2;
-                *reinterpret_cast<__nv_bfloat16 *>(item + kWsP + off) = hb;
-                *reinterpret_cast<__nv_bfloat16 *>(item + kWsP + TILE + off) = lb;
+                *reinterpret_cast<__nv_bfloat16 *>(sm + P_OFF_PHI + off) = hb;
+                *reinterpret_cast<__nv_bfloat16 *>(sm + P_OFF_PLO + off) = lb;
             }
         }
     }
     __syncthreads();
 
-    // ---- T = (I + A)^-1 (unit lower triangular) in fp32. Its strict lower part is stored
-    //      transposed in the strict upper part of the A array: T[r][c] at AT[c][r] (r > c).
+    // ---- T = (I + A)^-1 (unit lower triangular) in fp32. A is stored transposed in the strict
+    //      upper part of the array (A[r][s] at AT[s][r]), T row-major in the strict lower part.
     //      Two warps solve the 16 x 16 diagonal blocks by forward substitution while the other six
     //      write the Q' rows (64 + r of the [W; Q'] image: the raw bf16 Q tile scaled row by row,
     //      swizzle positions unchanged), the decay vector and the column factors of T'.
@@ -400,12 +412,12 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             float acc = (rr == cc) ? 1.0f : 0.0f;
 #pragma unroll
             for (int s = 0; s < rr; ++s)
-                if (s >= cc) acc -= AT[(o0 + rr) * P_AT + o0 + s] * xv[s];
+                if (s >= cc) acc -= AT[(o0 + s) * P_AT + o0 + rr] * xv[s];
             xv[rr] = (rr < cc) ? 0.0f : acc;
         }
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr)
-            if (rr > cc) AT[(o0 + cc) * P_AT + o0 + rr] = xv[rr];
+            if (rr > cc) AT[(o0 + rr) * P_AT + o0 + cc] = xv[rr];
     } else {
         const int t6 = tid - 64;
         // Q' (1024 chunks over 192 threads, loads issued before the stores)
@@ -436,6 +448,20 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                 }
             }
         }
+        // the P^T hi and lo images from their staging (1024 chunks)
+        {
+            uint4 pc[6];
+#pragma unroll
+            for (int e = 0; e < 6; ++e) {
+                const int c16 = e * 192 + t6, w = c16 < 1024 ? c16 : 0;
+                pc[e] = *reinterpret_cast<const uint4 *>(sm + (w < 512 ? P_OFF_PHI : P_OFF_PLO) + (w & 511) * 16);
+            }
+#pragma unroll
+            for (int e = 0; e < 6; ++e) {
+                const int c16 = e * 192 + t6;
+                if (c16 < 1024) *reinterpret_cast<uint4 *>(item + kWsP + c16 * 16) = pc[e];
+            }
+        }
         // the per-token factors of the state update, c_r = gamma_C / gamma_r / |k_r|, and gamma_C
         if (t6 < 64) reinterpret_cast<float *>(item + kWsVec)[t6] = sDec[t6];
         if (t6 == 64) reinterpret_cast<float *>(item + kWsVec)[64] = L > 0 ? __expf(sG[L - 1]) : 1.0f;
@@ -446,30 +472,79 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     // ---- off-diagonal blocks level by level, from T (I + A) = I:
     //      X = sum_{k in blocks bj+1 .. bi} T[r][k] A[k][c],   T[r][c] = -(X T_jj)[r][c],
     //      r in block bi, c in block bj; every thread one element of each block of the level.
+    // ---- off-diagonal blocks level by level, from T (I + A) = I:
+    //      X = sum_{bk = bj+1 .. bi} T_{bi,bk} A_{bk,bj},   T_{bi,bj} = -X T_{bj,bj},
+    //      one warp per block on the warp-level tensor-core MMA (m16n8k16) with every operand split
+    //      into bf16 hi + lo parts (hi hi + hi lo + lo hi, fp32 accumulation: about 16 significant
+    //      bits per product, as the fp32 blocks need); the sum's accumulator fragments are
+    //      directly the A fragments of the product with T_jj.
 #pragma unroll 1
     for (int lvl = 1; lvl < 4; ++lvl) {
-        const int nb = 4 - lvl;
-        const int rr = tid / 16, cc = tid % 16;
-        for (int m = 0; m < nb; ++m) {
-            const int bj = m, bi = m + lvl, r = bi * 16 + rr, c = bj * 16 + cc;
-            float acc = 0.0f;
-            for (int k = (bj + 1) * 16; k < bi * 16 + 16; ++k) {
-                const float t = (k < r) ? AT[k * P_AT + r] : (k == r ? 1.0f : 0.0f);
-                acc = fmaf(t, AT[k * P_AT + c], acc);
-            }
-            Xs[m * 272 + rr * 17 + cc] = acc;
-        }
-        __syncthreads();
-        for (int m = 0; m < nb; ++m) {
-            const int bj = m, bi = m + lvl, r = bi * 16 + rr, c = bj * 16 + cc;
-            float acc = 0.0f;
+        if (warp < 4 - lvl) {
+            const int bj = warp, bi = bj + lvl;
+            const int g = lane >> 2, t = lane & 3;
+            const int r0 = bi * 16 + g, r1 = r0 + 8;
+            float xc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int bk = bj + 1; bk <= bi; ++bk) {
+                // A fragment: T[r][k] for r in block bi, k = 16 bk + {2t, 2t+1, 2t+8, 2t+9}
+                const int k0 = bk * 16 + 2 * t;
+                float2 e00 = *reinterpret_cast<const float2 *>(AT + r0 * P_AT + k0);
+                float2 e10 = *reinterpret_cast<const float2 *>(AT + r1 * P_AT + k0);
+                float2 e01 = *reinterpret_cast<const float2 *>(AT + r0 * P_AT + k0 + 8);
+                float2 e11 = *reinterpret_cast<const float2 *>(AT + r1 * P_AT + k0 + 8);
+                if (bk == bi) {   // the diagonal block: 1 on the diagonal, 0 above it
+                    auto fix = [](float v, int r, int k) { return k < r ? v : (k == r ? 1.0f : 0.0f); };
+                    e00 = make_float2(fix(e00.x, r0, k0), fix(e00.y, r0, k0 + 1));
+                    e10 = make_float2(fix(e10.x, r1, k0), fix(e10.y, r1, k0 + 1));
+                    e01 = make_float2(fix(e01.x, r0, k0 + 8), fix(e01.y, r0, k0 + 9));
+                    e11 = make_float2(fix(e11.x, r1, k0 + 8), fix(e11.y, r1, k0 + 9));
+                }
+                uint32_t ah[4], al[4];
+                split_bf16x2(e00.x, e00.y, ah[0], al[0]);
+                split_bf16x2(e10.x, e10.y, ah[1], al[1]);
+                split_bf16x2(e01.x, e01.y, ah[2], al[2]);
+                split_bf16x2(e11.x, e11.y, ah[3], al[3]);
 #pragma unroll
-            for (int k2 = 0; k2 < 16; ++k2) {
-                const int k = bj * 16 + k2;
-                const float t = (k > c) ? AT[c * P_AT + k] : (k == c ? 1.0f : 0.0f);
-                acc = fmaf(Xs[m * 272 + rr * 17 + k2], t, acc);
+                for (int hn = 0; hn < 2; ++hn) {
+                    // B fragment: A[k][c] (stored at AT[c][k]) for k = 16 bk + {2t, 2t+1, 2t+8, 2t+9}
+                    const int c = bj * 16 + hn * 8 + g;
+                    const float2 b0 = *reinterpret_cast<const float2 *>(AT + c * P_AT + k0);
+                    const float2 b1 = *reinterpret_cast<const float2 *>(AT + c * P_AT + k0 + 8);
+                    uint32_t bh[2], bl[2];
+                    split_bf16x2(b0.x, b0.y, bh[0], bl[0]);
+                    split_bf16x2(b1.x, b1.y, bh[1], bl[1]);
+                    mma_bf16_m16n8k16(xc[hn], ah, bh);
+                    mma_bf16_m16n8k16(xc[hn], ah, bl);
+                    mma_bf16_m16n8k16(xc[hn], al, bh);
+                }
             }
-            AT[c * P_AT + r] = -acc;
+            uint32_t ah[4], al[4];
+            split_bf16x2(xc[0][0], xc[0][1], ah[0], al[0]);
+            split_bf16x2(xc[0][2], xc[0][3], ah[1], al[1]);
+            split_bf16x2(xc[1][0], xc[1][1], ah[2], al[2]);
+            split_bf16x2(xc[1][2], xc[1][3], ah[3], al[3]);
+#pragma unroll
+            for (int hn = 0; hn < 2; ++hn) {
+                // B fragment: T_jj[k][c], k = 16 bj + {2t, 2t+1, 2t+8, 2t+9}, c = 16 bj + 8 hn + g
+                const int c = bj * 16 + hn * 8 + g, k0 = bj * 16 + 2 * t;
+                float bv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int k = k0 + (e & 1) + (e >> 1) * 8;
+                    const float v = AT[k * P_AT + c];
+                    bv[e] = k > c ? v : (k == c ? 1.0f : 0.0f);
+                }
+                uint32_t bh[2], bl[2];
+                split_bf16x2(bv[0], bv[1], bh[0], bl[0]);
+                split_bf16x2(bv[2], bv[3], bh[1], bl[1]);
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_bf16_m16n8k16(d, ah, bh);
+                mma_bf16_m16n8k16(d, ah, bl);
+                mma_bf16_m16n8k16(d, al, bh);
+                const int col = bj * 16 + hn * 8 + 2 * t;
+                *reinterpret_cast<float2 *>(AT + r0 * P_AT + col) = make_float2(-d[0], -d[1]);
+                *reinterpret_cast<float2 *>(AT + r1 * P_AT + col) = make_float2(-d[2], -d[3]);
+            }
         }
         __syncthreads();
     }
@@ -482,7 +557,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int s = ch * 8 + j;
-            t[j] = (s < r) ? AT[s * P_AT + r] : (s == r ? 1.0f : 0.0f);
+            t[j] = (s < r) ? AT[r * P_AT + s] : (s == r ? 1.0f : 0.0f);
         }
         uint32_t h1[4], l1[4], h2[4], l2[4];
 #pragma unroll
@@ -586,8 +661,10 @@ teardown:
 // Warps 0-15: element-wise work; warp 16: bulk copies and MMA issue.
 // ===================================================================================
 // Output pass: 16 element-wise warps, four per tensor-memory lane quarter, each thread one state
-// row and 32 of its columns (half the per-thread work of eight warps, which shortens every
-// element-wise step of the chunk chain), plus the copy/MMA warp.
+// row and 32 of its columns, plus the copy/MMA warp. The chain's critical path per chunk is
+// D4 -> U -> D7 -> S update; each chunk's outputs are finished one chunk later, in two halves
+// placed where the chain waits for its MMAs (while D7 of the next chunk runs, and while D4 of the
+// chunk after it runs), from o kept in two tensor-memory slots.
 constexpr int CH_WARPS = 16;
 constexpr int CH_WORKERS = CH_WARPS * 32;
 constexpr int CH_COLS = 128 / (CH_WARPS / 4);      // state columns per thread
@@ -603,9 +680,8 @@ constexpr int CH_OFF_STAGE = CH_OFF_U + 32768;     // o staging, [r][i] (bf16 or
 constexpr int CH_OFF_BAR = CH_OFF_STAGE + 64 * 128 * 4;
 constexpr int CH_SMEM = CH_OFF_BAR + 128 + 1024;
 static_assert(CH_SMEM <= 232448, "chain shared memory");
-// Fused variant (gated RMSNorm + NVFP4 encode of each chunk's o rows): o staged in bf16 and
-// encoded by the workers while MMA45 of the next chunk runs; z tiles of three chunks in
-// flight (a chunk's tile is still read after the tile of the chunk after next is requested).
+// Fused variant (gated RMSNorm + NVFP4 encode of each chunk's o rows): o staged in bf16; z tiles
+// of three chunks in flight (a chunk's tile is read while the chain works on the next chunk).
 constexpr int CHF_THREADS = CH_THREADS;
 constexpr int CHF_STAGE = 64 * 128 * 2;            // one chunk's o rows, bf16 [r][i]
 constexpr int CHF_OFF_Z = CH_OFF_STAGE + CHF_STAGE;
@@ -618,9 +694,10 @@ static_assert(CHF_OFF_Z % 1024 == 0 && CB_K % 1024 == 0 && CB_BUF % 1024 == 0 &&
               "TMA destination alignment");
 static_assert(kWsItem % 1024 == 0 && kWsP % 1024 == 0 && kWsU % 16 == 0 && kWsVec % 16 == 0,
               "1024-byte aligned operand tiles, 16-byte aligned bulk sources");
-// tensor memory: [D4 | o] (MMA45, then the intra-chunk output accumulated onto o), D7 (state
-// update), fp16 S0 (two slots), U as bf16 hi / lo A operands, U diag(c) as bf16 hi / lo
-constexpr uint32_t C_TM_D45 = 0, C_TM_D7 = 128, C_TM_SA = 256, C_TM_UA = 384, C_TM_UCA = 448;
+// tensor memory: D4 (U's state term), o in two slots (chunk c in slot c & 1: MMA5a, then the
+// intra-chunk part accumulated onto it), D7 (state update), the fp16 copy of S0, U as bf16 hi /
+// lo A operands, U diag(c) as bf16 hi / lo
+constexpr uint32_t C_TM_D4 = 0, C_TM_O = 64, C_TM_D7 = 192, C_TM_SA = 320, C_TM_UA = 384, C_TM_UCA = 448;
 
 // kind::f16 instruction descriptor bits for bf16 A and B
 constexpr uint32_t kIdescBf16 = (1u << 7) | (1u << 10);
@@ -701,8 +778,8 @@ __device__ __forceinline__ void ilv_load32(const uint8_t *base, int row, int cq,
 // coalesced side and the row-per-thread side are free of bank conflicts).
 constexpr int kStgPitch = 528;
 
-// FUSED: the output pass also applies the gated RMSNorm to each chunk's o rows and writes them
-// NVFP4-encoded (o itself only when P.o is set).
+// FUSED: the outputs are the gated RMSNorm of each chunk's o rows, NVFP4-encoded (o itself only
+// when P.o is set); otherwise o.
 template <bool FUSED>
 __global__ void __launch_bounds__(FUSED ? CHF_THREADS : CH_THREADS, 1)
 gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
@@ -711,9 +788,11 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + (FUSED ? CHF_OFF_BAR : CH_OFF_BAR));
+    // full[2]: chunk copies; full_u: U~; bar_u / bar_s: D4 / D7 done; bar_uready / bar_sready: the
+    // element-wise warps have stored U / S0; bar_o[2]: a chunk's o complete (per o slot)
     uint64_t *full = bars, *full_u = bars + 2, *bar_u = bars + 3, *bar_s = bars + 4, *bar_uready = bars + 5,
-             *bar_sready = bars + 6, *bar_drain = bars + 7;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
+             *bar_sready = bars + 6, *bar_drain = bars + 7, *bar_o = bars + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int h = blockIdx.x, id = blockIdx.y;
@@ -754,6 +833,8 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
         mbar_init(bar_uready, CH_WARPS);
         mbar_init(bar_sready, CH_WARPS);
         mbar_init(bar_drain, 1);
+        mbar_init(&bar_o[0], 1);
+        mbar_init(&bar_o[1], 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -795,31 +876,41 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
                 bulk_load(sm + CH_OFF_U, ws_h + (size_t)(slot0 + c) * kWsItem + kWsU, 4 * TILE, full_u);
                 ++n_u;
             };
-            // with a caller's initial state the workers stage it over buffer 1 and the head of the
-            // U~ buffer: the first U~ load then waits until they have released it (bar_sready)
+            // with a caller's initial state the element-wise warps stage it over buffer 1 and the
+            // head of the U~ buffer: the first U~ load waits until they have released it (bar_sready)
             const bool s0_staged = pseg == 0 && S0g;
             if (nchunks > 0) {
                 issue_chunk(0);
                 if (!s0_staged) issue_u(0);
             }
-            const uint32_t id45 = idesc_f16(128, false, false, false);
+            const uint32_t id4 = idesc_f16(64, false, false, false);
             const uint32_t id7 = idesc_f16(128, false, true, false) | kIdescBf16;
             const uint32_t id5 = idesc_f16(64, false, true, false) | kIdescBf16;
             for (int c = 0; c < nchunks; ++c) {
                 const int b = c & 1;
                 const uint8_t *buf = sm + CH_OFF_BUF + b * CB_BUF;
                 if (!(ok = mbar_wait(&full[b], (uint32_t)((c >> 1) & 1), status))) break;
+                // S0 of chunk c is in tensor memory, and the workers have read chunk c - 2's o
                 if (!(ok = mbar_wait(bar_sready, (uint32_t)(c & 1), status))) break;
                 if (c == 0 && s0_staged) issue_u(0);
                 tc_fence_after();
-                // [D4 | D5a] = S0 [W; Q']^T   (fp16; B: 128 K-major rows, K = 128 key columns)
+                // D4 = S0 W^T (fp16; B: the W rows of the [W; Q'] image, K = 128 key columns),
+                // committed alone; then o = S0 Q'^T into o slot b (both read the S0 copy before
+                // D7's commit, after which the state update rewrites it)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_f16_ts(tmem + C_TM_D45, tmem + C_TM_SA + b * 64 + kk * 8,
-                               kdesc(buf + CB_WQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32), id45, kk > 0);
+                    mma_f16_ts(tmem + C_TM_D4, tmem + C_TM_SA + kk * 8,
+                               kdesc(buf + CB_WQ + (kk < 4 ? 0 : 2 * TILE) + (kk & 3) * 32), id4, kk > 0);
                 tc_commit(bar_u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tmem + C_TM_O + b * 64, tmem + C_TM_SA + kk * 8,
+                               kdesc(buf + CB_WQ + (kk < 4 ? TILE : 3 * TILE) + (kk & 3) * 32), id4, kk > 0);
                 ++n_mma;
-                if (c + 1 < nchunks) {   // the other buffer's readers (chunk c-1) are done
+                if (c + 1 < nchunks) {
+                    // buffer (c + 1) & 1 was chunk c - 1's: its MMAs are done once its o is, its
+                    // readers among the workers (c, gamma_C, the z tile) before they handed on S0
+                    if (c > 0 && !(ok = mbar_wait(&bar_o[(c - 1) & 1], (uint32_t)(((c - 1) >> 1) & 1), status))) break;
                     fence_proxy_async_smem();
                     issue_chunk(c + 1);
                 }
@@ -830,21 +921,22 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
                 }
                 tc_fence_after();
                 // D7 = (U diag(c))^T K with U diag(c) as bf16 hi + lo and the raw bf16 K (MN-major,
-                // two blocks of 64 keys); then o += U^T P^T with U and P^T as bf16 hi / lo
-                // (hi hi + hi lo + lo hi), accumulated onto the D5a columns
+                // two blocks of 64 keys), committed alone: the state update waits only for it
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_f16_ts(tmem + C_TM_D7, tmem + C_TM_UCA + part * 32 + kk * 8,
                                    mndesc(buf + CB_K + kk * 2048, TILE), id7, (part | kk) ? 1u : 0u);
+                tc_commit(bar_s);
+                // o += U^T P^T with U and P^T as bf16 hi / lo (hi hi + hi lo + lo hi)
 #pragma unroll
                 for (int part = 0; part < 3; ++part)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f16_ts(tmem + C_TM_D45 + 64, tmem + C_TM_UA + (part == 2 ? 32 : 0) + kk * 8,
+                        mma_f16_ts(tmem + C_TM_O + b * 64, tmem + C_TM_UA + (part == 2 ? 32 : 0) + kk * 8,
                                    mndesc(buf + CB_P + (part == 1 ? TILE : 0) + kk * 2048, TILE), id5, 1u);
-                tc_commit(bar_s);
+                tc_commit(&bar_o[b]);
             }
             if (!ok) {
                 // a wait ran out: wait (bounded) for this thread's MMAs and for the latest phase of
@@ -865,28 +957,27 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
         const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
         float S[CH_COLS];   // S[i][32 cq .. 32 cq + 31], fp32
         // fused: this thread's eight RMSNorm weights (16 threads per o row) and the encoder table
+        const int lr = tid & 15, ecol = lr * 8;
         f2_t w2[4];
         if constexpr (FUSED) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) w2[k] = f2(P.norm_w[(tid & 15) * 8 + 2 * k], P.norm_w[(tid & 15) * 8 + 2 * k + 1]);
+            for (int k = 0; k < 4; ++k) w2[k] = f2(P.norm_w[ecol + 2 * k], P.norm_w[ecol + 2 * k + 1]);
             nvfp4_fill_r_tab(reinterpret_cast<float *>(sm + CHF_OFF_RTAB), P.gs, tid);
         }
-        // fused: gated RMSNorm + NVFP4 encode of chunk cc, whose bf16 o rows are staged; 16
-        // threads per row, eight values each, 32 rows per pass (the same arithmetic as the
-        // standalone tail kernel); o written too when requested
-        auto epilogue = [&](int cc) {
+        const int out_bf16 = FUSED ? 1 : P.out_bf16;
+        uint8_t *stage = sm + CH_OFF_STAGE;
+        // Outputs of chunk cc, first half: its o (done once bar_o has landed) out of tensor memory
+        // into the staging area as rows [r][i], then rows 0-31 finished (gated RMSNorm + NVFP4
+        // encode, or the o stores); the z values of the second half are kept in registers, so that
+        // the z tile is free when this half is done. Returns false if the wait ran out.
+        uint4 z_keep = make_uint4(0u, 0u, 0u, 0u);
+        auto out_rows = [&](int cc, int pass, const uint4 &zu) {
             const int t0e = t_begin + (c_first + cc) * C;
             const int Le = min(C, t_end - t0e);
-            const uint8_t *stage = sm + CH_OFF_STAGE;
-            const uint8_t *zt = sm + CHF_OFF_Z + (cc % 3) * CHF_ZBYTES;
-            const float *r_tab = reinterpret_cast<const float *>(sm + CHF_OFF_RTAB);
-            uint8_t *ob = static_cast<uint8_t *>(P.o);
-            const int lr = tid & 15, col = lr * 8;
-#pragma unroll 1
-            for (int pass = 0; pass < C / (CH_WORKERS / 16); ++pass) {
+            if constexpr (FUSED) {
                 const int r = pass * (CH_WORKERS / 16) + (tid >> 4);
-                const uint4 ou = *reinterpret_cast<const uint4 *>(stage + r * (D * 2) + col * 2);
-                const uint4 zu = *reinterpret_cast<const uint4 *>(zt + (col >> 6) * TILE + swz(r, (col & 63) >> 3));
+                const uint4 ou = *reinterpret_cast<const uint4 *>(stage + r * (D * 2) + ecol * 2);
+                const float *r_tab = reinterpret_cast<const float *>(sm + CHF_OFF_RTAB);
                 const f2_t o2[4] = {bf16x2_to_f2(ou.x), bf16x2_to_f2(ou.y), bf16x2_to_f2(ou.z), bf16x2_to_f2(ou.w)};
                 const f2_t z2[4] = {bf16x2_to_f2(zu.x), bf16x2_to_f2(zu.y), bf16x2_to_f2(zu.z), bf16x2_to_f2(zu.w)};
                 f2_t y2[4];
@@ -894,12 +985,50 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
                 uint32_t packed, sb;
                 nvfp4_encode_row8(y2, P.gs, r_tab, packed, sb);
                 if (r < Le) {
-                    const size_t base = ((size_t)(t0e + r) * Hv + h) * D + col;
+                    const size_t base = ((size_t)(t0e + r) * Hv + h) * D + ecol;
                     reinterpret_cast<uint32_t *>(P.xq)[base / 8] = packed;
                     if ((lr & 1) == 0) P.xs[base / 16] = (uint8_t)sb;
-                    if (ob) *reinterpret_cast<uint4 *>(ob + base * 2) = ou;
+                    if (P.o) *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(P.o) + base * 2) = ou;
+                }
+            } else {
+                const int row_bytes = out_bf16 ? D * 2 : D * 4;
+                const int per_row = row_bytes / 16;
+                uint8_t *ob = static_cast<uint8_t *>(P.o);
+                const int r_lo = pass * 32, r_hi = min(Le, r_lo + 32);
+                for (int e = r_lo * per_row + tid; e < r_hi * per_row; e += CH_WORKERS) {
+                    const int r = e / per_row, chn = e % per_row;
+                    const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + chn * 16);
+                    *reinterpret_cast<uint4 *>(ob + (((size_t)(t0e + r) * Hv + h) * D) * (row_bytes / D) + chn * 16) = val;
                 }
             }
+        };
+        auto out_first = [&](int cc) -> bool {
+            int ok = 1;
+            if (tid == 0) ok = mbar_wait(&bar_o[cc & 1], (uint32_t)((cc >> 1) & 1), status) ? 1 : 0;
+            if (!workers_and(ok)) return false;
+            tc_fence_after();
+            uint32_t a5[16];
+            tmem_ld16(tmem + C_TM_O + (cc & 1) * 64 + lane_base + cq * CH_TOK, a5);
+            tmem_ld_wait();
+            if (out_bf16) {
+                __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(stage);
+#pragma unroll
+                for (int j = 0; j < CH_TOK; ++j) st[(cq * CH_TOK + j) * D + row] = __float2bfloat16_rn(__uint_as_float(a5[j]));
+            } else {
+                float *st = reinterpret_cast<float *>(stage);
+#pragma unroll
+                for (int j = 0; j < CH_TOK; ++j) st[(cq * CH_TOK + j) * D + row] = __uint_as_float(a5[j]);
+            }
+            workers_sync();
+            uint4 zu0 = make_uint4(0u, 0u, 0u, 0u);
+            if constexpr (FUSED) {
+                const uint8_t *zt = sm + CHF_OFF_Z + (cc % 3) * CHF_ZBYTES;
+                const int r0 = tid >> 4, r1 = (CH_WORKERS / 16) + (tid >> 4);
+                zu0 = *reinterpret_cast<const uint4 *>(zt + (ecol >> 6) * TILE + swz(r0, (ecol & 63) >> 3));
+                z_keep = *reinterpret_cast<const uint4 *>(zt + (ecol >> 6) * TILE + swz(r1, (ecol & 63) >> 3));
+            }
+            out_rows(cc, 0, zu0);
+            return true;
         };
         if (pseg == 0 && S0g) {
             // the caller's row-major initial state, staged over chunk buffer 1 and the head of the
@@ -924,18 +1053,19 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
 #pragma unroll
             for (int c = 0; c < CH_COLS; ++c) S[c] = 0.0f;
         }
-        // fp16 copy of S as an A operand: row i on lane i, key index j two per column
-        auto store_S = [&](int slot) {
+        // fp16 copy of S as an A operand: row i on lane i, key index j two per column (one slot:
+        // the MMAs that read it have completed before the workers rewrite it)
+        auto store_S = [&]() {
             uint32_t pk[16];
 #pragma unroll
             for (int w = 0; w < 16; ++w) pk[w] = pack_h2(S[2 * w], S[2 * w + 1]);
-            tmem_st16(tmem + lane_base + C_TM_SA + slot * 64 + cq * 16, pk);
+            tmem_st16(tmem + lane_base + C_TM_SA + cq * 16, pk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_sready);
         };
-        store_S(0);
+        store_S();
 
         bool alive = true;
         for (int c = 0; c < nchunks; ++c) {
@@ -954,87 +1084,80 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams P) {
             tc_fence_after();
             {
                 // U^T = U~^T - D4 (fp32) for tokens 16 cq .. + 15 of this row, then U and U diag(c)
-                // as bf16 hi / lo A operands
+                // as bf16 hi / lo A operands (packed f32x2 arithmetic, eight tokens at a time)
                 const float *ut = reinterpret_cast<const float *>(sm + CH_OFF_U);
-                float uv[CH_TOK], cv[CH_TOK];
+                const f2_t neg1 = f2(-1.0f, -1.0f);
 #pragma unroll
-                for (int w = 0; w < CH_TOK; ++w) {
-                    uv[w] = ut[(cq * CH_TOK + w) * D + row];
-                    cv[w] = vecb[cq * CH_TOK + w];
-                }
-                uint32_t r16[16];
-                tmem_ld16(tmem + C_TM_D45 + lane_base + cq * CH_TOK, r16);
-                tmem_ld_wait();
-                uint32_t uh[8], ul[8], ch[8], cl[8];
+                for (int part = 0; part < 2; ++part) {
+                    const int sb = cq * CH_TOK + part * 8;
+                    f2_t u2[4], c2[4];
 #pragma unroll
-                for (int w = 0; w < CH_TOK / 2; ++w) {
-                    const int s0 = cq * CH_TOK + 2 * w;
-                    const float u0 = (s0 < L) ? uv[2 * w] - __uint_as_float(r16[2 * w]) : 0.0f;
-                    const float u1 = (s0 + 1 < L) ? uv[2 * w + 1] - __uint_as_float(r16[2 * w + 1]) : 0.0f;
-                    split_bf16x2(u0, u1, uh[w], ul[w]);
-                    split_bf16x2(u0 * cv[2 * w], u1 * cv[2 * w + 1], ch[w], cl[w]);
+                    for (int w = 0; w < 4; ++w) {
+                        const int s0 = sb + 2 * w;
+                        u2[w] = f2(s0 < L ? ut[s0 * D + row] : 0.0f, s0 + 1 < L ? ut[(s0 + 1) * D + row] : 0.0f);
+                        const float2 cc = *reinterpret_cast<const float2 *>(vecb + s0);
+                        c2[w] = f2(cc.x, cc.y);
+                    }
+                    uint32_t r8[8];
+                    tmem_ld8(tmem + C_TM_D4 + lane_base + sb, r8);
+                    tmem_ld_wait();
+                    uint32_t uh[4], ul[4], ch[4], cl[4];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const int s0 = sb + 2 * w;
+                        f2_t u = fma2(f2(__uint_as_float(r8[2 * w]), __uint_as_float(r8[2 * w + 1])), neg1, u2[w]);
+                        if (s0 >= L) u = f2(0.0f, 0.0f);
+                        else if (s0 + 1 >= L) u = f2(f2lo(u), 0.0f);
+                        const f2_t uc = mul2(u, c2[w]);
+                        split_bf16x2(f2lo(u), f2hi(u), uh[w], ul[w]);
+                        split_bf16x2(f2lo(uc), f2hi(uc), ch[w], cl[w]);
+                    }
+                    tmem_st4(tmem + lane_base + C_TM_UA + sb / 2, uh);
+                    tmem_st4(tmem + lane_base + C_TM_UA + 32 + sb / 2, ul);
+                    tmem_st4(tmem + lane_base + C_TM_UCA + sb / 2, ch);
+                    tmem_st4(tmem + lane_base + C_TM_UCA + 32 + sb / 2, cl);
                 }
-                tmem_st8(tmem + lane_base + C_TM_UA + cq * (CH_TOK / 2), uh);
-                tmem_st8(tmem + lane_base + C_TM_UA + 32 + cq * (CH_TOK / 2), ul);
-                tmem_st8(tmem + lane_base + C_TM_UCA + cq * (CH_TOK / 2), ch);
-                tmem_st8(tmem + lane_base + C_TM_UCA + 32 + cq * (CH_TOK / 2), cl);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_uready);
             }
+            // while D7 runs: the first half of chunk c - 1's outputs
+            if (c > 0 && !out_first(c - 1)) { alive = false; break; }
             if (tid == 0) ok = mbar_wait(bar_s, ph, status) ? 1 : 0;
             if (!workers_and(ok)) { alive = false; break; }
             tc_fence_after();
-            float ov[CH_TOK];
             {
-                // o^T (D5a + the intra-chunk part) for tokens 16 cq .. + 15; S <- gamma_C S + D7
-                uint32_t a5[16], r7[32];
-                tmem_ld16(tmem + C_TM_D45 + lane_base + 64 + cq * CH_TOK, a5);
-                tmem_ld32(tmem + C_TM_D7 + lane_base + cq * CH_COLS, r7);
-                tmem_ld_wait();
+                // S <- gamma_C S + D7 for this quarter, handed on at once
                 const float gC = vecb[64];
+                const f2_t g2 = f2(gC, gC);
 #pragma unroll
-                for (int j = 0; j < CH_COLS; ++j) S[j] = gC * S[j] + __uint_as_float(r7[j]);
-                store_S(b ^ 1);   // S0 of chunk c + 1; releases the MMA warp
+                for (int part = 0; part < 2; ++part) {
+                    uint32_t r7[16];
+                    tmem_ld16(tmem + C_TM_D7 + lane_base + cq * CH_COLS + part * 16, r7);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < CH_TOK; ++j) ov[j] = __uint_as_float(a5[j]);
-            }
-            if (FUSED) {
-                // stage this chunk's o rows (bf16 [r][i]; the previous chunk's encode is done, a
-                // worker barrier has passed since) and encode them
-                __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(sm + CH_OFF_STAGE);
-#pragma unroll
-                for (int j = 0; j < CH_TOK; ++j) st[(cq * CH_TOK + j) * D + row] = __float2bfloat16_rn(ov[j]);
-                workers_sync();
-                epilogue(c);
-            } else {
-                // o rows of this chunk: staged as [r][i], then 16-byte row stores (rows < L)
-                const int out_bf16 = P.out_bf16;
-                uint8_t *stage = sm + CH_OFF_STAGE;
-                if (out_bf16) {
-                    __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(stage);
-#pragma unroll
-                    for (int j = 0; j < CH_TOK; ++j) st[(cq * CH_TOK + j) * D + row] = __float2bfloat16_rn(ov[j]);
-                } else {
-                    float *st = reinterpret_cast<float *>(stage);
-#pragma unroll
-                    for (int j = 0; j < CH_TOK; ++j) st[(cq * CH_TOK + j) * D + row] = ov[j];
+                    for (int j = 0; j < 16; j += 2) {
+                        const int jj = part * 16 + j;
+                        const f2_t s2 = fma2(g2, f2(S[jj], S[jj + 1]), f2(__uint_as_float(r7[j]), __uint_as_float(r7[j + 1])));
+                        S[jj] = f2lo(s2);
+                        S[jj + 1] = f2hi(s2);
+                    }
                 }
-                workers_sync();
-                const int row_bytes = out_bf16 ? D * 2 : D * 4;
-                const int per_row = row_bytes / 16;
-                uint8_t *ob = static_cast<uint8_t *>(P.o);
-                for (int e = tid; e < L * per_row; e += CH_WORKERS) {
-                    const int r = e / per_row, chn = e % per_row;
-                    const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * row_bytes + chn * 16);
-                    *reinterpret_cast<uint4 *>(ob + (((size_t)(t0 + r) * Hv + h) * D) * (row_bytes / D) + chn * 16) = val;
-                }
-                workers_sync();
+                store_S();   // S0 of chunk c + 1; releases the MMA warp
             }
+            // while D4 of chunk c + 1 runs: the second half of chunk c - 1's outputs
+            if (c > 0) out_rows(c - 1, 1, z_keep);
+        }
+        // the last chunk's outputs
+        if (alive && nchunks > 0) {
+            if (!out_first(nchunks - 1)) alive = false;
+            else out_rows(nchunks - 1, 1, z_keep);
         }
         if (alive && last_seg && P.S_out) {
-            // all chunks are consumed: the chunk buffers are free for staging the final state
+            // every MMA is done (the last o was waited for): the chunk buffers are free for staging
+            // the final state
+            workers_sync();
             uint8_t *stg = sm + CH_OFF_BUF;
 #pragma unroll
             for (int c4 = 0; c4 < CH_COLS / 4; ++c4)
@@ -1233,26 +1356,26 @@ gdn_chunk_lean_kernel(const __grid_constant__ ChainParams P) {
         const float gC = vecb[64];
         {
             // U^T = U~^T - D4 (the transition pass takes U~ = 0), scaled per token by c, as the bf16
-            // hi / lo A operands of MMA7, 16 tokens at a time
+            // hi / lo A operands of MMA7, 8 tokens at a time
             const float *ut = reinterpret_cast<const float *>(sm + CL_U);
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                float u16v[16];
+            for (int part = 0; part < 4; ++part) {
+                float u8v[8];
 #pragma unroll
-                for (int w = 0; w < 16; ++w) u16v[w] = with_u ? ut[(wg * 32 + part * 16 + w) * D + row] : 0.0f;
-                uint32_t r16[16];
-                tmem_ld16(tmem + CL_TM_D4 + lane_base + wg * 32 + part * 16, r16);
+                for (int w = 0; w < 8; ++w) u8v[w] = with_u ? ut[(wg * 32 + part * 8 + w) * D + row] : 0.0f;
+                uint32_t r8[8];
+                tmem_ld8(tmem + CL_TM_D4 + lane_base + wg * 32 + part * 8, r8);
                 tmem_ld_wait();
-                uint32_t uh[8], ul[8];
+                uint32_t uh[4], ul[4];
 #pragma unroll
-                for (int w = 0; w < 8; ++w) {
-                    const int s0 = wg * 32 + part * 16 + 2 * w;
-                    const float u0 = (s0 < L) ? u16v[2 * w] - __uint_as_float(r16[2 * w]) : 0.0f;
-                    const float u1 = (s0 + 1 < L) ? u16v[2 * w + 1] - __uint_as_float(r16[2 * w + 1]) : 0.0f;
+                for (int w = 0; w < 4; ++w) {
+                    const int s0 = wg * 32 + part * 8 + 2 * w;
+                    const float u0 = (s0 < L) ? u8v[2 * w] - __uint_as_float(r8[2 * w]) : 0.0f;
+                    const float u1 = (s0 + 1 < L) ? u8v[2 * w + 1] - __uint_as_float(r8[2 * w + 1]) : 0.0f;
                     split_bf16x2(u0 * vecb[s0], u1 * vecb[s0 + 1], uh[w], ul[w]);
                 }
-                tmem_st8(tmem + lane_base + CL_TM_UCA + wg * 16 + part * 8, uh);
-                tmem_st8(tmem + lane_base + CL_TM_UCA + 32 + wg * 16 + part * 8, ul);
+                tmem_st4(tmem + lane_base + CL_TM_UCA + wg * 16 + part * 4, uh);
+                tmem_st4(tmem + lane_base + CL_TM_UCA + 32 + wg * 16 + part * 4, ul);
             }
             tmem_st_wait();
             tc_fence_before();
