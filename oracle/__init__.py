@@ -18,6 +18,8 @@ Each function cites the passage it follows (page title, section):
   * NVFP4: "Why Gated DeltaNet Survives 4-Bit Quantization" (abstract, mechanism i:
     16-element block scaling), E2M1 values with E4M3 block scales and an fp32 global
     scale;
+  * Q4_K weights: "Red Lite dev15d - DeltaNet gated tail + Q4_K output projection" (Q4_K
+    implementation: 256-value blocks of 144 bytes);
   * short convolution: "A Node-by-Node White-Box Walkthrough of a Quantized Hybrid Gated
     DeltaNet Language Model" (Principais Contribuicoes, item 2: the short convolutions on the
     layer's path), read as the depthwise causal convolution of width K followed by SiLU.
@@ -77,6 +79,10 @@ def _load():
     lib.oracle_e2m1_decode.restype = f32
     lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
     lib.oracle_e4m3_decode.restype = f32
+    lib.oracle_f16_decode.argtypes = [ctypes.c_uint16]
+    lib.oracle_f16_decode.restype = f64
+    lib.oracle_q4k_dequantize.argtypes = [i32, i32, P, P, i32, i32]
+    lib.oracle_q4k_dequantize.restype = None
     _lib = lib
     return lib
 
@@ -216,6 +222,42 @@ def nvfp4_gemm(aq, as_, gs_a: float, bq, bs, gs_b: float, rows=None):
     A = nvfp4_dequantize(aq, as_, gs_a)
     B = nvfp4_dequantize(bq, bs, gs_b)
     return A @ B.T
+
+
+def q4k_dequantize(w, K: int, threads: int | None = None):
+    """Q4_K weights w [N, K/256*144] uint8 -> fp64 [N, K] (exact): "Red Lite dev15d - DeltaNet
+    gated tail + Q4_K output projection", section "Q4_K implementation" (256-value blocks of
+    144 bytes: f16 d, f16 dmin, 12 bytes of 6-bit scales / mins, 128 bytes of 4-bit quants;
+    value = d * scale * q - dmin * min; bit positions as in gdn_oracle.c)."""
+    lib = _load()
+    w = _c(w, np.uint8)
+    N = w.shape[0]
+    if K % 256 or w.shape[1] != K // 256 * 144:
+        raise ValueError("w must be [N, K/256*144] with K % 256 == 0")
+    out = np.zeros((N, K), dtype=np.float64)
+
+    def run(r):
+        lib.oracle_q4k_dequantize(N, K, _ptr(w), _ptr(out), r[0], r[1])
+
+    with ThreadPoolExecutor(max_workers=threads or default_threads()) as ex:
+        list(ex.map(run, _split(N, threads or default_threads())))
+    return out
+
+
+def q4k_gemm(a, w, K: int, rows=None):
+    """Y = A @ W^T in fp64 with W the dequantised Q4_K weights (A [M, K] fp32 values, W [N, K]);
+    ``rows`` optionally selects rows of A. The product is a library fp64 matrix multiply."""
+    a = np.asarray(a, dtype=np.float64)
+    if rows is not None:
+        a = a[np.asarray(rows)]
+    return a @ q4k_dequantize(w, K).T
+
+
+def f16_decode(h):
+    """fp64 values of IEEE binary16 bit patterns."""
+    lib = _load()
+    h = np.asarray(h, dtype=np.uint16).ravel()
+    return np.array([lib.oracle_f16_decode(int(x)) for x in h], dtype=np.float64)
 
 
 def e2m1_encode(x):

@@ -29,7 +29,8 @@
  *          head with the one shared norm weight, SiLU(z), multiply, flatten, output
  *          projection; "Real layer-0 GGUF tensors": the norm weight is F32 [128].
  *   [FMT]  OCP Microscaling Formats (MX) v1.0 (E2M1 element encoding) and OCP 8-bit
- *          Floating Point (E4M3FN): value sets used below.
+ *          Floating Point (E4M3FN): value sets used below; IEEE 754 binary16 for the Q4_K
+ *          block scales.
  *
  * Readings where the pages are silent:
  *   - q/k are L2-normalised inside the path when qk_l2norm != 0: x * (sum x^2 + eps)^-1/2.
@@ -261,6 +262,61 @@ void oracle_nvfp4_dequantize(int32_t M, int32_t K, const uint8_t *xq, const uint
             uint8_t code = (kk & 1) ? (byte >> 4) : (byte & 15);
             double sc = oracle_e4m3_decode(xs[(size_t)m * (K / 16) + kk / 16]);
             out[(size_t)m * K + kk] = (double)oracle_e2m1_decode(code) * sc / (double)gs;
+        }
+}
+
+/* ----------------------------------------------------------------- Q4_K ---- */
+
+/* IEEE binary16: 1 sign, 5 exponent (bias 15), 10 mantissa bits; exponent 0 is subnormal,
+ * 31 is inf / NaN. Exact in fp64. */
+double oracle_f16_decode(uint16_t h) {
+    int e = (h >> 10) & 31, m = h & 1023;
+    double mag;
+    if (e == 31) mag = m ? NAN : INFINITY;
+    else if (e == 0) mag = ldexp((double)m, -24);
+    else mag = ldexp(1.0 + (double)m / 1024.0, e - 15);
+    return (h & 0x8000) ? -mag : mag;
+}
+
+/*
+ * [TAIL] "Q4_K implementation": blocks of 256 values in 144 bytes - f16 d, f16 dmin, 12 bytes of
+ * packed 6-bit scales and mins for the block's eight sub-blocks of 32 values, 128 bytes of 4-bit
+ * quants. The page fixes the sizes and calls the layout canonical; the bit positions read here
+ * are the GGUF K-quant ones:
+ *   bytes 0-1 d, 2-3 dmin (little-endian f16); bytes 4-15 = sc[12];
+ *   sub-block j < 4: scale = sc[j] & 63, min = sc[j + 4] & 63;
+ *   sub-block j >= 4: scale = (sc[j + 4] & 15) | ((sc[j - 4] >> 6) << 4),
+ *                     min = (sc[j + 4] >> 4) | ((sc[j] >> 6) << 4);
+ *   bytes 16-143 = qs[128]: value 64 g + i (g < 4, i < 32) is the low nibble of qs[32 g + i]
+ *   (sub-block 2 g), value 64 g + 32 + i its high nibble (sub-block 2 g + 1);
+ *   value = d * scale * q - dmin * min.
+ * w: rows [N, K / 256 * 144] bytes; out: [N, K] fp64 (exact), rows [row_begin, row_end).
+ */
+void oracle_q4k_dequantize(int32_t N, int32_t K, const uint8_t *w, double *out, int32_t row_begin,
+                           int32_t row_end) {
+    (void)N;
+    const int32_t nb = K / 256;
+    for (int32_t n = row_begin; n < row_end; ++n)
+        for (int32_t blk = 0; blk < nb; ++blk) {
+            const uint8_t *b = w + ((size_t)n * nb + blk) * 144;
+            const double d = oracle_f16_decode((uint16_t)(b[0] | (b[1] << 8)));
+            const double dmin = oracle_f16_decode((uint16_t)(b[2] | (b[3] << 8)));
+            const uint8_t *sc = b + 4, *qs = b + 16;
+            for (int j = 0; j < 8; ++j) {
+                int scale, mn;
+                if (j < 4) {
+                    scale = sc[j] & 63;
+                    mn = sc[j + 4] & 63;
+                } else {
+                    scale = (sc[j + 4] & 15) | ((sc[j - 4] >> 6) << 4);
+                    mn = (sc[j + 4] >> 4) | ((sc[j] >> 6) << 4);
+                }
+                const int g = j / 2, hi = j & 1;
+                for (int i = 0; i < 32; ++i) {
+                    const int q = hi ? (qs[32 * g + i] >> 4) : (qs[32 * g + i] & 15);
+                    out[(size_t)n * K + (size_t)blk * 256 + 32 * j + i] = d * (double)scale * (double)q - dmin * (double)mn;
+                }
+            }
         }
 }
 

@@ -135,6 +135,22 @@ def activations(M: int, K: int, seed: int, std: float = 1.0, heavy_tail: bool = 
     return round_bf16(x) if bf16 else x
 
 
+def q4k_weights(N: int, K: int, seed: int) -> np.ndarray:
+    """Synthetic Q4_K weights [N, K/256*144] uint8 (the page's 144-byte blocks of 256 values):
+    per block f16 d ~ |N(1e-4, 2e-5)| and dmin = 7.5 d U(0.5, 1.5) (so the values d*scale*q -
+    dmin*min spread around zero with a standard deviation of about 0.02), 12 random bytes of
+    6-bit scales / mins, 128 random bytes of 4-bit quants. Random bytes only; the packing is
+    whatever the bytes say."""
+    rng = np.random.default_rng(seed)
+    nb = N * (K // 256)
+    blocks = rng.integers(0, 256, size=(nb, 144), dtype=np.uint8)
+    d = np.abs(rng.normal(1e-4, 2e-5, size=nb)).astype(np.float16)
+    dmin = (d.astype(np.float32) * 7.5 * rng.uniform(0.5, 1.5, size=nb)).astype(np.float16)
+    blocks[:, 0:2] = d.view(np.uint8).reshape(nb, 2)
+    blocks[:, 2:4] = dmin.view(np.uint8).reshape(nb, 2)
+    return blocks.reshape(N, (K // 256) * 144)
+
+
 def conv_inputs(T: int, C: int, K: int, seed: int, num_seqs: int = 1, state: bool = False) -> dict:
     """Inputs of the causal short convolution: x [T, C] ~ N(0, 1) (bf16-rounded), weight [C, K]
     ~ N(0, 1/K) fp32 (so the pre-activation is about unit scale), and, with state, a carried
