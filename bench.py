@@ -433,6 +433,21 @@ def run_gpu(args):
     dec = statistics.mean(dec_ms)
     state_bytes = dstate.numel() * 4
     dec_bytes = 2 * state_bytes + sum(t.numel() * t.element_size() for t in (dq, dk, dv, da, db, dout))
+    # the decode step with the gated tail and the NVFP4 encode: fused kernel against the two calls
+    dz, dnw = up(dx["z"], bf), up(dx["norm_weight"], f32)
+    dxq = torch.empty((dw.num_seqs, dw.Hv * dw.D // 2), dtype=torch.uint8, device=dev)
+    dxs = torch.empty((dw.num_seqs, dw.Hv * dw.D // 16), dtype=torch.uint8, device=dev)
+    dgs = 448.0 * 6.0 / 4.0
+    fdec_graph = graph_of(lambda: g.gdn_decode_step_gated_nvfp4(dq, dk, dv, da, db, dA, ddt, dstate, dz, dnw, dgs,
+                                                                xq=dxq, xs=dxs))
+
+    def two_call():
+        g.gdn_decode_step(dq, dk, dv, da, db, dA, ddt, dstate, o=dout)
+        g.gdn_gated_rmsnorm_silu_nvfp4(dout, dz, dnw, dgs, xq=dxq, xs=dxs)
+    tdec_graph = graph_of(two_call)
+    fdec = statistics.mean(timed_graph(torch, stream, flush, fdec_graph, max(args.steps, 10)))
+    tdec = statistics.mean(timed_graph(torch, stream, flush, tdec_graph, max(args.steps, 10)))
+    del fdec_graph, tdec_graph
 
     # multi-token decode on the batched-decode workload's shape: verify 4 draft tokens per sequence
     # (state read once), then commit a seeded number of accepted tokens (state read and written once)
@@ -473,6 +488,18 @@ def run_gpu(args):
         big_graph.replay()
     big_ms = statistics.mean(timed_graph(torch, stream, flush, big_graph, max(args.steps, 10)))
     del ga, gw, gy, big_graph
+
+    # the Q4_K-weight output projection of the same layer (the tail page's comparison format)
+    q4w = up(workloads.q4k_weights(gN, gK, seed=7), torch.uint8)
+    q4_ms = {}
+    for qm in (gM, dw.num_seqs):
+        q4a = up(workloads.activations(qm, gK, seed=8, heavy_tail=False), bf)
+        q4y = torch.empty((qm, gN), dtype=bf, device=dev)
+        q4_graph = graph_of(lambda: g.q4k_gemm(q4a, q4w, y=q4y))
+        q4_ms[qm] = statistics.mean(timed_graph(torch, stream, flush, q4_graph, max(args.steps, 10)))
+        del q4a, q4y, q4_graph
+    del q4w
+    assert g.gdn_get_device_status() == 0
 
     # short convolution decode on the batched-decode workload's q|k|v channels (state in place)
     dC = 2 * dw.Hk * dw.D + dw.Hv * dw.D
@@ -537,11 +564,20 @@ def run_gpu(args):
         "decode": {"workload": dw.name, "ms": dec, "GB/s": dec_bytes / (dec / 1e3) / 1e9,
                    "frac": dec_bytes / (dec / 1e3) / 1e9 / float(pk["hbm_gbs"]),
                    "bytes": dec_bytes, "peak_gbs": float(pk["hbm_gbs"]), "peak_kind": pk_kind,
-                   "timing": "CUDA graph replay, L2 flushed before each"},
+                   "timing": "CUDA graph replay, L2 flushed before each",
+                   "with_gated_nvfp4_tail": {"fused_ms": fdec, "two_calls_ms": tdec,
+                                             "what": "decode step + gated RMSNorm + NVFP4 encode: one fused kernel "
+                                                     "against gdn_decode_step then gdn_gated_rmsnorm_silu_nvfp4"}},
         "gemm_long_prefill": {"shape": [gM, gN, gK], "ms": big_ms,
                               "TFLOP/s": 2.0 * gM * gN * gK / (big_ms / 1e3) / 1e12,
                               "frac_of_fp4_probe": 2.0 * gM * gN * gK / (big_ms / 1e3) / 1e12 / FP4_PROBE_TFLOPS,
                               "peak_kind": "FP4 tensor rate measured by a tcgen05 probe (16368 MAC/cycle/SM at 1965 MHz)"},
+        "q4k_out_proj": {"shape_prefill": [gM, gN, gK], "ms_prefill": q4_ms[gM],
+                         "TFLOP/s_prefill": 2.0 * gM * gN * gK / (q4_ms[gM] / 1e3) / 1e12,
+                         "tensor_frac_prefill": 2.0 * gM * gN * gK / (q4_ms[gM] / 1e3) / 1e12 / float(pk["bf16_tflops"]),
+                         "shape_decode": [dw.num_seqs, gN, gK], "ms_decode": q4_ms[dw.num_seqs],
+                         "weight_GB/s_decode": gN * (gK // 256) * 144 / (q4_ms[dw.num_seqs] / 1e3) / 1e9,
+                         "what": "Q4_K weights decoded to bf16 in the kernel, bf16 tensor-core MMA"},
         "decode_multi": {"workload": "%s shape, %d draft tokens per sequence" % (dw.name, mT),
                          "verify_ms": ver_ms, "verify_GB/s": ver_bytes / (ver_ms / 1e3) / 1e9,
                          "verify_frac": ver_bytes / (ver_ms / 1e3) / 1e9 / float(pk["hbm_gbs"]),

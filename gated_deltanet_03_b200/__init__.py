@@ -27,9 +27,10 @@ GDN_BF16, GDN_F32 = 0, 1
 # Exported C symbols, in the order include/gdn.h declares them.
 ABI_SYMBOLS = (
     "gdn_prefill_chunked", "gdn_prefill_workspace_bytes", "gdn_prefill_chunked_gated_nvfp4", "gdn_decode_step",
+    "gdn_decode_step_gated_nvfp4",
     "gdn_decode_verify", "gdn_decode_commit",
     "gdn_gated_rmsnorm_silu", "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_dequantize_act",
-    "nvfp4_gemm", "nvfp4_gemm_colscale", "nvfp4_fused_col_alpha", "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode",
+    "nvfp4_gemm", "nvfp4_gemm_colscale", "nvfp4_fused_col_alpha", "q4k_gemm", "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode",
     "gdn_prefill_chunked_static_ws", "gdn_get_device_status", "gdn_debug_set_wait", "gdn_status_string",
     "gdn_version",
 )
@@ -55,6 +56,8 @@ def _load() -> ctypes.CDLL:
     lib.gdn_prefill_workspace_bytes.restype = sz
     lib.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, P, P,
                                     i32, P]
+    lib.gdn_decode_step_gated_nvfp4.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, P, P, P,
+                                                f32, f32, P, P, P, P]
     lib.gdn_decode_verify.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P, P, P,
                                       i32, P]
     lib.gdn_decode_commit.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P, P, P]
@@ -65,6 +68,7 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_gemm.argtypes = [P, P, P, P, f32, i32, i32, i32, i32, P, P]
     lib.nvfp4_gemm_colscale.argtypes = [P, P, P, P, P, i32, i32, i32, i32, P, P]
     lib.nvfp4_fused_col_alpha.argtypes = [P, P, i32, f32, P, P]
+    lib.q4k_gemm.argtypes = [P, P, i32, i32, i32, i32, P, P]
     i64 = ctypes.c_int64
     lib.gdn_short_conv1d_silu.argtypes = [P, i64, P, P, i32, i32, i32, i32, P, P, P, P, i32, P]
     lib.gdn_short_conv1d_silu_decode.argtypes = [P, i64, P, i32, i32, i32, P, P, P, i32, P]
@@ -75,10 +79,11 @@ def _load() -> ctypes.CDLL:
     lib.gdn_status_string.argtypes = [i32]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_version.restype = i32
-    for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_gated_nvfp4", "gdn_prefill_chunked_static_ws", "gdn_decode_step", "gdn_decode_verify",
+    for name in ("gdn_prefill_chunked", "gdn_prefill_chunked_gated_nvfp4", "gdn_prefill_chunked_static_ws", "gdn_decode_step",
+                 "gdn_decode_step_gated_nvfp4", "gdn_decode_verify",
                  "gdn_decode_commit", "gdn_gated_rmsnorm_silu",
                  "gdn_gated_rmsnorm_silu_nvfp4", "nvfp4_quantize_act", "nvfp4_dequantize_act", "nvfp4_gemm",
-                 "nvfp4_gemm_colscale", "nvfp4_fused_col_alpha",
+                 "nvfp4_gemm_colscale", "nvfp4_fused_col_alpha", "q4k_gemm",
                  "gdn_short_conv1d_silu", "gdn_short_conv1d_silu_decode", "gdn_get_device_status", "gdn_debug_set_wait"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -243,6 +248,31 @@ def gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1.0,
     return o
 
 
+def gdn_decode_step_gated_nvfp4(q, k, v, a, b, A_log, dt_bias, state, z, norm_weight, global_scale: float,
+                                scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6, xq=None, xs=None,
+                                o=None, stream=None):
+    """One token per sequence (d = 128, bf16) with the gated RMSNorm and NVFP4 encode fused:
+    `state` [B, Hv, 128, 128] fp32 is updated in place. Returns (xq [B, Hv*64], xs [B, Hv*8], o or None)."""
+    B, Hk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    _args(q.device, q=(q, (torch.bfloat16,), None), k=(k, (torch.bfloat16,), B * Hk * Dk),
+          v=(v, (torch.bfloat16,), B * Hv * Dv), a=(a, _F32, B * Hv), b=(b, _F32, B * Hv), A_log=(A_log, _F32, Hv),
+          dt_bias=(dt_bias, _F32, Hv), state=(state, _F32, B * Hv * Dv * Dk), z=(z, (torch.bfloat16,), B * Hv * Dv),
+          norm_weight=(norm_weight, _F32, Dv), xq=(xq, _U8, B * Hv * Dv // 2), xs=(xs, _U8, B * Hv * Dv // 16),
+          o=(o, (torch.bfloat16,), B * Hv * Dv))
+    if xq is None:
+        xq = torch.empty((B, Hv * Dv // 2), dtype=torch.uint8, device=q.device)
+    if xs is None:
+        xs = torch.empty((B, Hv * Dv // 16), dtype=torch.uint8, device=q.device)
+    _contig(q, k, v, a, b, A_log, dt_bias, state, z, norm_weight, xq, xs, o)
+    st = LIB.gdn_decode_step_gated_nvfp4(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
+                                         B, Hk, Hv, Dk, Dv, float(scale), int(bool(qk_l2norm)), _dt(q), _ptr(state),
+                                         _ptr(z), _ptr(norm_weight), float(eps), float(global_scale), _ptr(xq),
+                                         _ptr(xs), _ptr(o), _stream(stream))
+    _check("gdn_decode_step_gated_nvfp4", st)
+    return xq, xs, o
+
+
 def gdn_decode_verify(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1.0, qk_l2norm: bool = True,
                       final_state=None, out_dtype=None, o=None, stream=None):
     """T draft tokens per sequence: q, k [B, T, Hk, D], v [B, T, Hv, D], a, b [B, T, Hv];
@@ -393,6 +423,21 @@ def nvfp4_fused_col_alpha(widths, module_scales, act_scale: float, col_alpha=Non
     st = LIB.nvfp4_fused_col_alpha(wa, sa, n, float(act_scale), _ptr(col_alpha), _stream(stream))
     _check("nvfp4_fused_col_alpha", st)
     return col_alpha
+
+
+def q4k_gemm(a, w, out_dtype=torch.bfloat16, y=None, stream=None):
+    """y [M, N] = a [M, K] (bf16) times the Q4_K weights w [N, K/256*144] (uint8) transposed."""
+    M, K = a.shape
+    N = w.shape[0]
+    if w.dim() != 2 or K % 256 or w.shape[1] != K // 256 * 144:
+        raise ValueError("w must be uint8 [N, K/256*144] with K % 256 == 0")
+    _args(a.device, a=(a, (torch.bfloat16,), None), w=(w, _U8, N * (K // 256) * 144), y=(y, _IO, M * N))
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _contig(a, w, y)
+    st = LIB.q4k_gemm(_ptr(a), _ptr(w), M, N, K, _dt(y), _ptr(y), _stream(stream))
+    _check("q4k_gemm", st)
+    return y
 
 
 def _conv_rows(x):

@@ -168,6 +168,25 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const fl
     return launched(gdn::launch_recurrent(r, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+gdn_status gdn_decode_step_gated_nvfp4(const void *q, const void *k, const void *v, const float *a, const float *b,
+                                       const float *A_log, const float *dt_bias, int32_t B, int32_t Hk, int32_t Hv,
+                                       int32_t Dk, int32_t Dv, float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                                       float *state, const void *z, const float *norm_weight, float eps,
+                                       float global_scale, uint8_t *xq, uint8_t *xs, void *o, gdn_stream_t stream) {
+    if (B < 0 || Hk < 1 || Hv < 1 || Hv % Hk != 0 || !dtype_ok(in_dtype)) return GDN_ERR_INVALID_ARG;
+    if (Dk != 128 || Dv != 128 || in_dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (!(eps >= 0.0f) || !(global_scale > 0.0f) || !std::isfinite(global_scale)) return GDN_ERR_INVALID_ARG;
+    if (B == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !A_log || !dt_bias || !state || !z || !norm_weight || !xq || !xs)
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(z) || !aligned16(xq) ||
+        (o && !aligned16(o)))
+        return GDN_ERR_INVALID_ARG;
+    gdn::DecodeTailArgs d{q, k, v, a, b, A_log, dt_bias, B, Hk, Hv, scale, qk_l2norm, state, z, norm_weight,
+                          eps, global_scale, xq, xs, o};
+    return launched(gdn::launch_decode_gated_nvfp4(d, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 static gdn_status multi_check(const void *q, const void *k, const void *v, const float *a, const float *b,
                               const float *A_log, const float *dt_bias, int32_t B, int32_t T, int32_t Hk, int32_t Hv,
                               int32_t Dk, int32_t Dv, gdn_dtype in_dtype) {
@@ -286,6 +305,17 @@ gdn_status nvfp4_gemm_colscale(const uint8_t *aq, const uint8_t *as, const uint8
     if (!aligned16(aq) || !aligned16(bq) || !aligned16(y)) return GDN_ERR_INVALID_ARG;
     gdn::GemmArgs g{aq, as, bq, bs, 1.0f, M, N, K, out_dtype == GDN_BF16, y, status_ptr(), col_alpha};
     return launched(gdn::launch_nvfp4_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gdn_status q4k_gemm(const void *a, const uint8_t *w, int32_t M, int32_t N, int32_t K, gdn_dtype out_dtype, void *y,
+                    gdn_stream_t stream) {
+    if (M < 0 || N < 0 || K < 0 || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
+    if (K % 256 != 0 || N % 128 != 0) return GDN_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return GDN_OK;
+    if (K == 0) return GDN_ERR_UNSUPPORTED;
+    if (!a || !w || !y || !aligned16(a) || !aligned16(w) || !aligned16(y)) return GDN_ERR_INVALID_ARG;
+    gdn::Q4kGemmArgs g{a, w, M, N, K, out_dtype == GDN_BF16, y, status_ptr()};
+    return launched(gdn::launch_q4k_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 gdn_status nvfp4_fused_col_alpha(const int32_t *widths, const float *module_scales, int32_t n_modules,

@@ -72,6 +72,22 @@ struct RecurrentArgs {
 };
 cudaError_t launch_recurrent(const RecurrentArgs &r, cudaStream_t st);
 
+// One decode token per sequence (d = 128, bf16) fused with the gated RMSNorm and the NVFP4 encode.
+struct DecodeTailArgs {
+    const void *q, *k, *v;       // [B, Hk, 128], [B, Hk, 128], [B, Hv, 128] bf16
+    const float *a, *b, *A_log, *dt_bias;
+    int32_t B, Hk, Hv;
+    float scale;
+    int32_t l2norm;
+    float *state;                // [B, Hv, 128, 128] fp32, in place
+    const void *z;               // [B, Hv, 128] bf16
+    const float *norm_w;         // [128]
+    float eps, gs;
+    uint8_t *xq, *xs;            // [B, Hv * 64], [B, Hv * 8]
+    void *o;                     // [B, Hv, 128] bf16 or null
+};
+cudaError_t launch_decode_gated_nvfp4(const DecodeTailArgs &d, cudaStream_t st);
+
 struct ChunkedArgs {
     const void *q, *k, *v;       // bf16
     const float *a, *b, *A_log, *dt_bias;
@@ -134,6 +150,17 @@ struct ColAlphaArgs {
     float *col_alpha;
 };
 cudaError_t launch_fused_col_alpha(const ColAlphaArgs &c, int32_t N, cudaStream_t st);
+
+// Output projection with Q4_K weights: y [M, N] = a [M, K] (bf16) times the decoded w [N, K]^T.
+struct Q4kGemmArgs {
+    const void *a;               // bf16 [M, K]
+    const uint8_t *w;            // [N, K / 256 * 144] Q4_K blocks
+    int32_t M, N, K;
+    bool out_bf16;
+    void *y;
+    int *status;
+};
+cudaError_t launch_q4k_gemm(const Q4kGemmArgs &g, cudaStream_t st);
 
 struct ConvArgs {
     const void *x;               // bf16 rows of ldx elements; channels [0, C) are convolved

@@ -35,8 +35,10 @@
 //              registers (64 columns at a time; after its last read the warp releases the
 //              accumulator) -> alpha * acc -> 16-byte stores of the thread's row.
 // Cross-CTA arrivals use mapa-mapped barrier addresses. Every barrier wait is bounded (about
-// 1 s); an expired wait records GDN_ERR_TIMEOUT and the CTA finishes without issuing more work;
-// both CTAs meet at a cluster barrier before tensor memory is freed.
+// 1 s); an expired wait records GDN_ERR_TIMEOUT and the CTA finishes without issuing more work.
+// Before tensor memory is freed the producer waits for the last load it armed on each stage and
+// the leader for a final commit of its MMAs (both bounded); then both CTAs meet at a cluster
+// barrier.
 #include <mutex>
 
 #include "common.cuh"
@@ -115,13 +117,15 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
         : "memory");
     return ok != 0;
 }
-// Bounded wait (about 1 s) on a barrier that receives arrivals from the peer CTA.
+// Bounded wait (the control block's limit, 1 s by default) on a barrier that receives arrivals
+// from the peer CTA.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, int *status) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+    const uint64_t limit = ctl_wait_limit(status);
     for (uint32_t i = 0;; ++i) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
-        if ((i & 255u) == 255u && global_timer_ns() - t0 > kWaitLimitNs) {
+        if ((i & 255u) == 255u && global_timer_ns() - t0 > limit) {
             report_status(status, GDN_ERR_TIMEOUT);
             return false;
         }
@@ -152,8 +156,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     auto ssfb = [&](int s) { return base + s * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES; };
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + BAR_OFF);
     uint64_t *full = bars, *empty = bars + STAGES, *sf_ready = bars + 2 * STAGES;
-    uint64_t *acc_full = bars + 3 * STAGES, *acc_empty = bars + 3 * STAGES + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 2);
+    uint64_t *acc_full = bars + 3 * STAGES, *acc_empty = bars + 3 * STAGES + 1, *drain = bars + 3 * STAGES + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 3);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cluster_rank();
@@ -171,6 +175,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         }
         mbar_init(acc_full, 1);          // the leader's commit after a tile's last MMA
         mbar_init(acc_empty, 2 * EPI_WARPS);   // leader only: every epilogue warp of both CTAs
+        mbar_init(drain, 1);             // the leader's last commit (every MMA of the pair done)
         fence_barrier_init();
         tma_prefetch_desc(&map_a);
         tma_prefetch_desc(&map_b);
@@ -206,6 +211,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     }
                 }
             }
+            // before the CTA may exit: the latest load armed on each stage has landed (bounded; on
+            // the normal path every one of them was consumed already)
+            for (int s = 0; s < STAGES && s < it; ++s) {
+                const int last = it - 1 - ((it - 1 - s) % STAGES);   // the last use of stage s
+                mbar_wait(&full[s], (uint32_t)((last / STAGES) & 1), status);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
@@ -236,6 +247,11 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     tc_commit_pair(&empty[s]);
                 }
                 if (ok) tc_commit_pair(acc_full);
+            }
+            // before the pair may free tensor memory: every MMA issued has completed (bounded)
+            if (it > 0) {
+                tc_commit_pair(drain);
+                mbar_wait(drain, 0, status);
             }
         }
     } else if (warp >= 4 && warp < 8) {

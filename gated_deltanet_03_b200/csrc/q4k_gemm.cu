@@ -1,0 +1,284 @@
+// Output projection with Q4_K weights (the comparison format of "Red Lite dev15d - DeltaNet gated
+// tail + Q4_K output projection", section "Q4_K implementation"): y[m, n] = sum_k a[m, k] w[n, k]
+// with a the bf16 activations and w decoded on the fly from 256-value blocks of 144 bytes (f16 d,
+// f16 dmin, twelve bytes of 6-bit sub-block scales and mins, 128 bytes of 4-bit quants;
+// w = d * scale * q - dmin * min; bit positions of the GGUF K-quant layout, which the page calls
+// canonical).
+//
+// tcgen05 kind::f16 (bf16 A and B, fp32 accumulation in tensor memory), CTA tile 128 x 128, 64
+// values of K per stage, a 3-stage ring, two CTAs per SM. Warp 0: TMA of the activation tile;
+// warp 1: tensor memory and the MMA issue (one thread); warps 4-7: one output column (weight row)
+// per thread - per stage it reads the row's 32 quant bytes for the stage (and the block header
+// once per block), decodes 64 weights in fp32, rounds them to bf16 and writes them into the
+// stage's K-major 128-byte-swizzled B tile; at the end the same warps read the accumulator (one
+// lane quarter each) and store y. The weights are decoded once per output tile; the 4.5 MB
+// weight of the 4096 -> 2048 projection stays in L2 across the M tiles.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gdn {
+namespace {
+
+constexpr int QK_BM = 128, QK_BN = 128, QK_BK = 64;
+constexpr int QK_STAGES = 3;
+constexpr int QK_TILE = QK_BM * QK_BK * 2;                  // 16 KB (A and B tiles alike)
+constexpr int QK_STAGE_BYTES = 2 * QK_TILE;
+constexpr int QK_OFF_BAR = QK_STAGES * QK_STAGE_BYTES;
+constexpr int QK_SMEM = QK_OFF_BAR + 128 + 1024;
+constexpr int QK_THREADS = 256;
+constexpr int QK_BLOCK_BYTES = 144;
+static_assert(2 * (QK_SMEM + 1024) <= 233472, "two Q4_K GEMM CTAs per SM");
+
+__device__ __forceinline__ uint32_t qk_swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
+
+__device__ __forceinline__ void qk_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// Scale and min of sub-block j from the twelve packed bytes (sc[0..11]).
+__device__ __forceinline__ void q4k_scale_min(const uint8_t (&sc)[12], int j, int &scale, int &mn) {
+    if (j < 4) {
+        scale = sc[j] & 63;
+        mn = sc[j + 4] & 63;
+    } else {
+        scale = (sc[j + 4] & 15) | ((sc[j - 4] >> 6) << 4);
+        mn = (sc[j + 4] >> 4) | ((sc[j] >> 6) << 4);
+    }
+}
+
+// fp32 of a 4-bit value: 2^23 + q as a float, minus 2^23 (exact).
+__device__ __forceinline__ float nib_f(uint32_t q) { return __uint_as_float(0x4B000000u | q) - 8388608.0f; }
+
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(QK_THREADS, 2)
+q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__restrict__ w, int M, int N, int K,
+                void *__restrict__ y, int *status) {
+    pdl_launch_dependents();
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + QK_OFF_BAR);
+    uint64_t *a_full = bars, *b_full = bars + QK_STAGES, *empty = bars + 2 * QK_STAGES;
+    uint64_t *acc_full = bars + 3 * QK_STAGES, *drain = bars + 3 * QK_STAGES + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * QK_STAGES + 2);
+    auto tile_a = [&](int s) { return sm + s * QK_STAGE_BYTES; };
+    auto tile_b = [&](int s) { return sm + s * QK_STAGE_BYTES + QK_TILE; };
+
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int n0 = blockIdx.x * QK_BN, m0 = blockIdx.y * QK_BM;
+    const int num_k = K / QK_BK, nb = K / 256;
+
+    if (tid == 0) {
+        for (int s = 0; s < QK_STAGES; ++s) {
+            mbar_init(&a_full[s], 1);
+            mbar_init(&b_full[s], 4);    // the four decoding warps
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int kt = 0; kt < num_k; ++kt) {
+                const int s = kt % QK_STAGES;
+                if (!mbar_wait(&empty[s], (uint32_t)(((kt / QK_STAGES) & 1) ^ 1), status)) break;
+                mbar_arrive_expect_tx(&a_full[s], QK_TILE);
+                tma_load_2d(tile_a(s), &map_a, &a_full[s], kt * QK_BK, m0);
+            }
+            // before the CTA may exit: the last load armed on each stage has landed
+            for (int s = 0; s < QK_STAGES && s < num_k; ++s) {
+                const int last = num_k - 1 - ((num_k - 1 - s) % QK_STAGES);
+                mbar_wait(&a_full[s], (uint32_t)((last / QK_STAGES) & 1), status);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // bf16 A and B, fp32 accumulation, both K-major, N = 128, M = 128
+            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(QK_BN >> 3) << 17) |
+                                   ((uint32_t)(QK_BM >> 4) << 24);
+            int issued = 0;
+            for (int kt = 0; kt < num_k; ++kt) {
+                const int s = kt % QK_STAGES;
+                const uint32_t ph = (uint32_t)((kt / QK_STAGES) & 1);
+                if (!mbar_wait(&a_full[s], ph, status) || !mbar_wait(&b_full[s], ph, status)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < QK_BK / 16; ++kk)
+                    qk_mma(tmem, smem_desc(smem_u32(tile_a(s)) + kk * 32, 16, 1024, 2),
+                           smem_desc(smem_u32(tile_b(s)) + kk * 32, 16, 1024, 2), idesc, (kt | kk) ? 1u : 0u);
+                tc_commit(&empty[s]);
+                ++issued;
+                if (kt == num_k - 1) tc_commit(acc_full);
+            }
+            // before tensor memory is freed: every MMA issued has completed (bounded)
+            if (issued) {
+                tc_commit(drain);
+                mbar_wait(drain, 0, status);
+            }
+        }
+    } else if (warp >= 4) {
+        const int quarter = warp - 4;
+        const int rl = quarter * 32 + lane;               // weight row within the tile
+        const int n = n0 + rl;
+        const uint8_t *wrow = w + (size_t)n * nb * QK_BLOCK_BYTES;
+        bool ok = true;
+        float ds[2] = {0.f, 0.f}, dm[2] = {0.f, 0.f};
+        for (int kt = 0; kt < num_k && ok; ++kt) {
+            const int s = kt % QK_STAGES, g = kt & 3;
+            const uint8_t *blk = wrow + (size_t)(kt >> 2) * QK_BLOCK_BYTES;
+            // the quant bytes of this stage's 64 values (sub-blocks 2 g and 2 g + 1) and, at a block's
+            // first stage, the block header, before the wait for the stage to be free
+            const uint4 q0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * g);
+            const uint4 q1 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * g + 16);
+            uint8_t sc[12];
+            float d = 0.f, dmin = 0.f;
+            {
+                const uint4 hd = *reinterpret_cast<const uint4 *>(blk);
+                d = __half2float(__ushort_as_half((unsigned short)(hd.x & 0xFFFFu)));
+                dmin = __half2float(__ushort_as_half((unsigned short)(hd.x >> 16)));
+                const uint32_t words[3] = {hd.y, hd.z, hd.w};
+#pragma unroll
+                for (int i = 0; i < 12; ++i) sc[i] = (uint8_t)(words[i >> 2] >> (8 * (i & 3)));
+            }
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                int scale, mn;
+                q4k_scale_min(sc, 2 * g + h2, scale, mn);
+                ds[h2] = d * (float)scale;
+                dm[h2] = dmin * (float)mn;
+            }
+            if (lane == 0) ok = mbar_wait(&empty[s], (uint32_t)(((kt / QK_STAGES) & 1) ^ 1), status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            // values 0-31 of the stage: low nibbles (sub-block 2 g); 32-63: high nibbles (2 g + 1)
+            const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+            uint8_t *brow = tile_b(s);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {   // 16-byte chunk c: values 8 c .. 8 c + 7
+                const int h2 = c >> 2, sh = h2 ? 4 : 0;
+                const uint32_t wa = qw[(c & 3) * 2], wb = qw[(c & 3) * 2 + 1];
+                uint32_t packed[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t src = e < 2 ? wa : wb;
+                    const int byte0 = (e & 1) * 2;
+                    const float x0 = fmaf(nib_f((src >> (8 * byte0 + sh)) & 15u), ds[h2], -dm[h2]);
+                    const float x1 = fmaf(nib_f((src >> (8 * byte0 + 8 + sh)) & 15u), ds[h2], -dm[h2]);
+                    const __nv_bfloat162 bb = __floats2bfloat162_rn(x0, x1);
+                    packed[e] = *reinterpret_cast<const uint32_t *>(&bb);
+                }
+                *reinterpret_cast<uint4 *>(brow + qk_swz(rl, c)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&b_full[s]);
+        }
+        // epilogue: this warp's lane quarter of the 128 x 128 accumulator, one output row per thread
+        if (ok) {
+            if (lane == 0) ok = mbar_wait(acc_full, 0, status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+        if (ok) {
+            tc_fence_after();
+            const int m = m0 + quarter * 32 + lane;
+            const uint32_t lb = ((uint32_t)(quarter * 32)) << 16;
+#pragma unroll 1
+            for (int c32 = 0; c32 < QK_BN / 32; ++c32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lb + c32 * 32, r);
+                tmem_ld_wait();
+                if (m < M) {
+                    if constexpr (OUT_BF16) {
+                        __nv_bfloat16 *yr = reinterpret_cast<__nv_bfloat16 *>(y) + (size_t)m * N + n0 + c32 * 32;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            uint4 u;
+                            __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                p2[q] = __floats2bfloat162_rn(__uint_as_float(r[8 * i + 2 * q]), __uint_as_float(r[8 * i + 2 * q + 1]));
+                            *reinterpret_cast<uint4 *>(yr + 8 * i) = u;
+                        }
+                    } else {
+                        float *yr = reinterpret_cast<float *>(y) + (size_t)m * N + n0 + c32 * 32;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            *reinterpret_cast<float4 *>(yr + 4 * i) =
+                                make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                            __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn qk_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+
+cudaError_t launch_q4k_gemm(const Q4kGemmArgs &g, cudaStream_t st) {
+    if (g.M == 0 || g.N == 0) return cudaSuccess;
+    EncodeTiledFn fn = qk_encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    CUtensorMap ma;
+    cuuint64_t dims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.M};
+    cuuint64_t strides[1] = {(cuuint64_t)g.K * 2};
+    cuuint32_t box[2] = {QK_BK, QK_BM};
+    cuuint32_t elem[2] = {1, 1};
+    if (fn(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(g.a), dims, strides, box, elem,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    static PerDevice<int> attr;
+    int unused = 0;
+    cudaError_t e = attr.get(
+        [](int, int &) {
+            cudaError_t r = cudaFuncSetAttribute(q4k_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, QK_SMEM);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(q4k_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, QK_SMEM);
+            return r;
+        },
+        &unused);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)(g.N / QK_BN), (unsigned)((g.M + QK_BM - 1) / QK_BM));
+    if (g.out_bf16)
+        return launch_pdl(q4k_gemm_kernel<true>, grid, dim3(QK_THREADS), QK_SMEM, st, ma, g.w, g.M, g.N, g.K, g.y, g.status);
+    return launch_pdl(q4k_gemm_kernel<false>, grid, dim3(QK_THREADS), QK_SMEM, st, ma, g.w, g.M, g.N, g.K, g.y, g.status);
+}
+
+}  // namespace gdn

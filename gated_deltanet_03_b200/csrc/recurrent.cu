@@ -406,6 +406,121 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
     }
 }
 
+// Decode step fused with the gated tail: one CTA of 256 threads per (sequence, value head) owns
+// all 128 rows of the state (the two 64-row halves of gdn_recurrent128_kernel, same thread layout
+// and arithmetic), so the head's o is complete inside the CTA. It is rounded to bf16 (the tensor
+// the two-call path hands to the tail), and one warp applies the gated RMSNorm and the NVFP4
+// encode with the tail kernel's row functions, so the codes and scales equal the two-call path's
+// bit for bit. "Red Lite dev15d - DeltaNet gated tail", Pinned graph semantics, steps 1-5.
+constexpr int kFusedDecThreads = 256;
+
+__global__ void __launch_bounds__(kFusedDecThreads)
+gdn_decode128_gated_nvfp4_kernel(const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
+                                 const float *__restrict__ a, const float *__restrict__ b,
+                                 const float *__restrict__ A_log, const float *__restrict__ dt_bias, int32_t Hk,
+                                 int32_t Hv, float scale, int32_t l2norm, float *state, const void *__restrict__ z,
+                                 const float *__restrict__ norm_w, float eps, float gs, uint8_t *__restrict__ xq,
+                                 uint8_t *__restrict__ xs, void *__restrict__ o) {
+    pdl_launch_dependents();
+    pdl_wait();
+    constexpr int D = 128;
+    const int h = blockIdx.x, n = blockIdx.y;          // sequence n decodes token n
+    const int hk = h / (Hv / Hk);
+    const int tid = threadIdx.x, lane = tid & 31, l8 = tid & 7;
+    const int rbase = (tid >> 7) * 64 + ((tid & 127) >> 3);
+    const int gbase = lane & ~7;
+    __shared__ __align__(16) __nv_bfloat16 o_s[D];
+    const size_t sbase = ((size_t)n * Hv + h) * D * D;
+
+    f2_t s[4][8];
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 x = __ldcs(reinterpret_cast<const float4 *>(state + sbase + (size_t)(rbase + 16 * p) * D + 32 * j + 4 * l8));
+            s[p][2 * j] = f2(x.x, x.y);
+            s[p][2 * j + 1] = f2(x.z, x.w);
+        }
+    float g_alpha = 0.0f, g_beta = 0.0f;
+    if (lane == 0) {
+        float g;
+        gdn_gates(a[(size_t)n * Hv + h], b[(size_t)n * Hv + h], A_log[h], dt_bias[h], g, g_beta);
+        g_alpha = expf(g);
+    }
+    const float alpha = __shfl_sync(kFull, g_alpha, 0), beta = __shfl_sync(kFull, g_beta, 0);
+    f2_t k2[8], q2[8];
+    load_cols16<true>(k, ((size_t)n * Hk + hk) * D, l8, k2);
+    load_cols16<true>(q, ((size_t)n * Hk + hk) * D, l8, q2);
+    float vv[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) vv[p] = load1<true>(v, ((size_t)n * Hv + h) * D + rbase + 16 * p);
+
+    float kn = 1.0f, qn = scale;
+    if (l2norm) {
+        const float ks = group_sum<8>(dot16(k2, k2)), qs = group_sum<8>(dot16(q2, q2));
+        kn = rsqrtf(ks + 1e-6f);
+        qn = rsqrtf(qs + 1e-6f) * scale;
+    }
+    float part[4], sk[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) part[p] = dot16(s[p], k2);
+    const float skt = group8_sum4_t(part, l8);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) sk[p] = __shfl_sync(kFull, skt, gbase + 4 * (p >> 1) + 2 * (p & 1));
+    const f2_t a2 = f2(alpha, alpha);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float u = beta * (vv[p] - alpha * kn * sk[p]) * kn;
+        const f2_t u2 = f2(u, u);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) s[p][c] = fma2(a2, s[p][c], mul2(u2, k2[c]));
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) part[p] = dot16(s[p], q2);
+    const float ot = group8_sum4_t(part, l8);
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            __stcs(reinterpret_cast<float4 *>(state + sbase + (size_t)(rbase + 16 * p) * D + 32 * j + 4 * l8),
+                   make_float4(f2lo(s[p][2 * j]), f2hi(s[p][2 * j]), f2lo(s[p][2 * j + 1]), f2hi(s[p][2 * j + 1])));
+    if ((l8 & 1) == 0) {
+        const int p = 2 * ((l8 >> 2) & 1) + ((l8 >> 1) & 1);
+        const __nv_bfloat16 ob = __float2bfloat16_rn(ot * qn);
+        o_s[rbase + 16 * p] = ob;
+        if (o) reinterpret_cast<__nv_bfloat16 *>(o)[((size_t)n * Hv + h) * D + rbase + 16 * p] = ob;
+    }
+    __syncthreads();
+    if (tid < 32) {
+        // the head row: 16 lanes x 8 values (lanes 16-31 repeat them, their results unused)
+        const int lr = lane & 15, col = lr * 8;
+        const uint4 ou = *reinterpret_cast<const uint4 *>(o_s + col);
+        const uint4 zu = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(z) +
+                                                          ((size_t)n * Hv + h) * D + col);
+        const f2_t o2[4] = {bf16x2_to_f2(ou.x), bf16x2_to_f2(ou.y), bf16x2_to_f2(ou.z), bf16x2_to_f2(ou.w)};
+        const f2_t z2[4] = {bf16x2_to_f2(zu.x), bf16x2_to_f2(zu.y), bf16x2_to_f2(zu.z), bf16x2_to_f2(zu.w)};
+        f2_t w2[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) w2[c] = f2(norm_w[col + 2 * c], norm_w[col + 2 * c + 1]);
+        f2_t y2[4];
+        gated_row8<16>(o2, z2, w2, 1.0f / (float)D, eps, y2);
+        uint32_t packed, sb;
+        nvfp4_encode_row8(y2, gs, nullptr, packed, sb);
+        if (lane < 16) {
+            const size_t base = ((size_t)n * Hv + h) * D + col;
+            reinterpret_cast<uint32_t *>(xq)[base / 8] = packed;
+            if ((lr & 1) == 0) xs[base / 16] = (uint8_t)sb;
+        }
+    }
+}
+
+cudaError_t launch_decode_gated_nvfp4(const DecodeTailArgs &d, cudaStream_t st) {
+    if (d.B == 0 || d.Hv == 0) return cudaSuccess;
+    return launch_pdl(gdn_decode128_gated_nvfp4_kernel, dim3(d.Hv, d.B), dim3(kFusedDecThreads), 0, st, d.q, d.k, d.v,
+                      d.a, d.b, d.A_log, d.dt_bias, d.Hk, d.Hv, d.scale, d.l2norm, d.state, d.z, d.norm_w, d.eps,
+                      d.gs, d.xq, d.xs, d.o);
+}
+
 template <bool IN_BF16, bool OUT_BF16>
 static cudaError_t launch_verify128_t(const RecurrentArgs &r, cudaStream_t st) {
     dim3 grid(2, r.Hv, r.num_seqs);

@@ -154,6 +154,21 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
                            float *state, void *o, gdn_dtype out_dtype, gdn_stream_t stream);
 
+/* gdn_decode_step fused with the gated tail and the NVFP4 encode (the survey's fused decode):
+ * [GDN] recurrence for one token per sequence, then [TAIL] steps 1-5 on each head's o and the
+ * 16-value NVFP4 block encode ([GDN] mechanism i) in the same kernel, so o never goes through
+ * HBM. Dk = Dv = 128, bf16 inputs. state [B, Hv, 128, 128] fp32 updated in place; z [B, Hv, 128]
+ * bf16; norm_weight [128] fp32; eps and global_scale as gdn_gated_rmsnorm_silu_nvfp4; outputs
+ * xq [B, Hv*64] u8 and xs [B, Hv*8] (E4M3), the same bytes as gdn_decode_step (bf16 o) followed by
+ * gdn_gated_rmsnorm_silu_nvfp4; o [B, Hv, 128] bf16 is also written when not NULL. */
+GDN_API gdn_status gdn_decode_step_gated_nvfp4(const void *q, const void *k, const void *v, const float *a,
+                                               const float *b, const float *A_log, const float *dt_bias,
+                                               int32_t B, int32_t Hk, int32_t Hv, int32_t Dk, int32_t Dv,
+                                               float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
+                                               float *state, const void *z, const float *norm_weight,
+                                               float eps, float global_scale, uint8_t *xq, uint8_t *xs,
+                                               void *o, gdn_stream_t stream);
+
 /* ------------------------------------------------ multi-token decode (verify) ----
  * [GDN]: the same recurrence over T tokens per sequence (a draft of T tokens to check in one
  * pass, e.g. speculative decoding), without changing the state: o for every draft token, the
@@ -255,6 +270,17 @@ GDN_API gdn_status nvfp4_gemm_colscale(const uint8_t *aq, const uint8_t *as, con
  * GDN_ERR_INVALID_ARG. Enqueued on `stream`. */
 GDN_API gdn_status nvfp4_fused_col_alpha(const int32_t *widths, const float *module_scales, int32_t n_modules,
                                          float act_scale, float *col_alpha, gdn_stream_t stream);
+
+/* ------------------------------------------------- Q4_K output projection ----
+ * [TAIL] "Q4_K implementation" (the page's comparison format for ssm_out): y [M, N] = a [M, K] w^T
+ * with w [N, K] held as Q4_K blocks of 256 values in 144 bytes (f16 d, f16 dmin, 12 bytes of
+ * 6-bit sub-block scales / mins, 128 bytes of 4-bit quants; w = d * scale * q - dmin * min; the
+ * GGUF K-quant bit positions, which the page calls canonical). The weights are decoded on the fly,
+ * rounded to bf16 and multiplied on the tensor cores with fp32 accumulation.
+ * a: bf16 [M, K] row-major; w: [N, K/256 * 144] bytes (row n: its K/256 blocks in order); y:
+ * [M, N] in out_dtype. Supported: K % 256 == 0, N % 128 == 0; a, w, y 16-byte aligned. */
+GDN_API gdn_status q4k_gemm(const void *a, const uint8_t *w, int32_t M, int32_t N, int32_t K, gdn_dtype out_dtype,
+                            void *y, gdn_stream_t stream);
 
 /* ------------------------------------------------------ short convolution ----
  * [WALK]: the causal short convolution + SiLU on the layer's q, k, v channels before the scan:

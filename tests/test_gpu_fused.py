@@ -87,3 +87,33 @@ def test_fused_rejects_unsupported(g):
         g.gdn_prefill_chunked_gated_nvfp4(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["A_log"],
                                           inp["dt_bias"], z, nw, 1.0)
     assert e.value.status == g.GDN_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("B,Hk,Hv", [(3, 1, 2), (256, 16, 32)])
+def test_fused_decode_equals_decode_then_tail(g, B, Hk, Hv):
+    """gdn_decode_step_gated_nvfp4 against gdn_decode_step (bf16 o) followed by
+    gdn_gated_rmsnorm_silu_nvfp4 on that o: the same state, o, codes and block scales, bit for bit
+    (the batched-decode shape and a small one)."""
+    w = workloads.custom("fd", (1,) * B, Hk, Hv, 128, io="bf16", s0_std=0.1, seed=400 + B, kind="decode")
+    x = workloads.generate(w)
+    d = upload_scan_inputs(x, True)
+    z = dev(x["z"], torch.bfloat16)
+    nw = dev(x["norm_weight"], torch.float32)
+    gs = 448.0 * 6.0 / 5.0
+    st_ref = d["initial_state"].clone()
+    o_ref = g.gdn_decode_step(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"], st_ref)
+    xq_ref, xs_ref = g.gdn_gated_rmsnorm_silu_nvfp4(o_ref, z, nw, gs)
+    st = d["initial_state"].clone()
+    o = torch.empty_like(o_ref)
+    xq, xs, _ = g.gdn_decode_step_gated_nvfp4(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"], st,
+                                              z, nw, gs, o=o)
+    torch.cuda.synchronize()
+    assert g.gdn_get_device_status() == 0
+    assert torch.equal(st, st_ref)
+    assert torch.equal(o, o_ref)
+    assert torch.equal(xq, xq_ref) and torch.equal(xs, xs_ref)
+    # without the o output
+    st2 = d["initial_state"].clone()
+    xq2, xs2, _ = g.gdn_decode_step_gated_nvfp4(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"],
+                                                st2, z, nw, gs)
+    assert torch.equal(xq2, xq_ref) and torch.equal(xs2, xs_ref) and torch.equal(st2, st_ref)

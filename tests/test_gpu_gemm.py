@@ -115,3 +115,23 @@ def test_fused_modules_colscale(g, M):
     y1 = _gpu(g, aq, as_, wq, ws, alpha0, torch.float32)
     gate = slice(sum(widths[:4]), sum(widths))
     assert rel_err(y1[:, gate], ref[:, gate]) > 100 * TOL_GEMM
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 256), (200, 256, 768), (256, 2048, 4096), (4096, 2048, 4096)])
+def test_q4k_gemm_matches_oracle(g, M, N, K):
+    """The Q4_K output projection ("Red Lite dev15d - DeltaNet gated tail + Q4_K output
+    projection", Q4_K implementation) against the fp64 product with the oracle's exact decode of
+    the same synthetic weights: within the GEMM tolerance (the kernel rounds each decoded weight
+    to bf16), for a ragged M, the batched-decode shape (M = 256, 4096 -> 2048) and a prefill-sized
+    M; bf16 and fp32 outputs."""
+    w = workloads.q4k_weights(N, K, seed=M + N + K)
+    a = workloads.activations(M, K, seed=M * 3 + 1, heavy_tail=False)
+    rows = np.arange(M) if M <= 256 else np.unique(np.concatenate([np.arange(0, M, 37), [M - 1]]))
+    ref = oracle.q4k_gemm(a, w, K, rows=rows)
+    aa, ww = dev(a, torch.bfloat16), dev(w, torch.uint8)
+    y32 = to_np(g.q4k_gemm(aa, ww, out_dtype=torch.float32))
+    yb = to_np(g.q4k_gemm(aa, ww, out_dtype=torch.bfloat16))
+    torch.cuda.synchronize()
+    assert g.gdn_get_device_status() == 0
+    assert rel_err(y32[rows], ref) <= TOL_GEMM
+    assert rel_err(yb[rows], ref) <= TOL_GEMM
