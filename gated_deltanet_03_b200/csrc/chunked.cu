@@ -60,19 +60,24 @@ constexpr size_t kSegItemBytes = 196608;
 
 // Chunks per segment of the chain: the state chain of a sequence is split into segments that
 // run in parallel (state and transition passes), a short sequential combine, and the output
-// pass. Picks the length that minimises a cycle model of the three passes (per-chunk costs of
-// the chain modes and of one combine step, measured on B200, and the number of CTA waves on
-// 148 SMs), from the mean sequence length.
+// pass. Picks the length that minimises a cost model of the three passes - per-chunk costs of
+// the output pass (one CTA per SM) and of the state / transition passes (two CTAs per SM) and the
+// cost of one combine step, fitted to fused-prefill timings on B200 over 4096 - 32768 tokens and
+// 16 - 32 value heads, with CTA waves counted fractionally above one - from the mean sequence
+// length (the host does not read cu_seqlens).
 int chunked_segment_chunks(int T, int num_seqs, int Hv) {
     const double nch = (double)T / kChunk / (num_seqs > 0 ? num_seqs : 1);
-    const double c_state = 3.5, c_full = 4.7, c_comb = 2.5, sms = 148.0;
+    const double c_full = 2.0, c_state = 0.5, c_comb = 4.0, sms = 148.0;
     int best = 1 << 30;
     double best_cost = 1e30;
     for (int seg = 4; seg <= 4096; seg *= 2) {
         const double nseg = nch / seg > 1.0 ? std::ceil(nch / seg) : 1.0;
         const double ctas = (double)Hv * num_seqs * nseg;
-        double cost = std::ceil(ctas / sms) * std::min((double)seg, nch) * c_full;
-        if (nseg > 1.0) cost += std::ceil(2.0 * ctas / sms) * seg * c_state + (nseg - 2.0) * c_comb;
+        double cost = std::max(1.0, ctas / sms) * std::min((double)seg, nch) * c_full;
+        if (nseg > 1.0) {
+            const double lean_ctas = 2.0 * Hv * num_seqs * (nseg - 1.0);
+            cost += std::max(1.0, lean_ctas / (2.0 * sms)) * seg * c_state + (nseg - 2.0) * c_comb;
+        }
         if (cost < best_cost) {
             best_cost = cost;
             best = seg;
