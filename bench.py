@@ -52,8 +52,9 @@ CHUNK = 64
 # FP4 (kind::mxf4nvf4) dense rate measured by a tcgen05 probe: 16368 MAC/cycle/SM x 148 SMs x 1965 MHz
 FP4_PROBE_TFLOPS = 2.0 * 16368 * 148 * 1.965e9 / 1e12
 # DRAM bytes of one fused prefill call (prep + lean + combine + the output pass with the gated
-# tail), from one ncu capture with cold caches, keyed by the digest of the scan's source
-SCAN_TRAFFIC = {"8d0ca4422ce4682c": 237.57e6}
+# tail) on the long-prefill workload, from one ncu capture with cold caches, keyed by the digest
+# of the scan's source (null in the line once the source has changed)
+SCAN_TRAFFIC = {"a812579e7fde3fe6": 4723.71e6}
 
 
 def source_digest(path: str) -> str:
