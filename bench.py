@@ -646,6 +646,10 @@ def run_only(args):
     conv_y = torch.empty((w.T * conv_C,), dtype=bf, device=dev)
     dcx = workloads.conv_inputs(w.num_seqs, conv_C, 4, seed=w.seed, num_seqs=w.num_seqs, state=True)
     dconv_x, dconv_s = up(dcx["x"], bf), up(dcx["initial_state"], bf)
+    if args.only == "q4k":
+        q4a = up(workloads.round_bf16(np.random.default_rng(3).standard_normal((w.T, w.K)).astype(np.float32)), bf)
+        q4w = up(workloads.q4k_weights(w.n_out, w.K, seed=7), torch.uint8)
+        q4y = torch.empty((w.T, w.n_out), dtype=bf, device=dev)
     fn = {
         "conv_decode": lambda: g.gdn_short_conv1d_silu_decode(dconv_x, conv_w, dconv_s,
                                                               parts=(w.Hk * w.D, w.Hk * w.D, w.Hv * w.D)),
@@ -655,6 +659,7 @@ def run_only(args):
                                               final_state=S, o=o),
         "tail": lambda: g.gdn_gated_rmsnorm_silu_nvfp4(o, z, nw, 1.0, xq=xq, xs=xs),
         "gemm": lambda: g.nvfp4_gemm(xq, xs, wq, ws, 1.0, y=Y),
+        "q4k": lambda: g.q4k_gemm(q4a, q4w, y=q4y),
         "decode": lambda: g.gdn_decode_step(q, k, v, a, b, A_log, dt_bias, S0, o=o),
         "fused": lambda: g.gdn_prefill_chunked_gated_nvfp4(q, k, v, a, b, A_log, dt_bias, z, nw, 1.0, cu_seqlens=cu,
                                                            initial_state=S0, final_state=S, xq=xq, xs=xs),
@@ -845,7 +850,7 @@ def main():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     p.add_argument("--only", choices=["scan", "tail", "gemm", "gemm_long", "decode", "verify", "fused", "conv",
-                                      "conv_decode"],
+                                      "conv_decode", "q4k"],
                    help="time one kernel alone on its workload (for profiling); prints one JSON line")
     p.add_argument("--workload", default=None, help="workload name for --only scan (default: 1024-wide prefill)")
     args = p.parse_args()

@@ -13,6 +13,14 @@
 // stage's K-major 128-byte-swizzled B tile; at the end the same warps read the accumulator (one
 // lane quarter each) and store y. The weights are decoded once per output tile; the 4.5 MB
 // weight of the 4096 -> 2048 projection stays in L2 across the M tiles.
+//
+// Split K for small M (the decode shapes, where the output tiles alone would leave most SMs
+// idle): a cluster of S CTAs (2, 4 or 8) along grid z shares one output tile, CTA r taking the
+// r-th of S equal K ranges. Each CTA writes its fp32 partial tile into its own shared memory
+// (over the then idle stage ring), and after a cluster barrier CTA r sums rows
+// [r 128/S, (r+1) 128/S) over the S partials in rank order (ld.shared::cluster) and stores them;
+// a second cluster barrier keeps every partial in place until all CTAs have read it. The order
+// of the sums is fixed, so results do not depend on scheduling.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -27,7 +35,30 @@ constexpr int QK_OFF_BAR = QK_STAGES * QK_STAGE_BYTES;
 constexpr int QK_SMEM = QK_OFF_BAR + 128 + 1024;
 constexpr int QK_THREADS = 256;
 constexpr int QK_BLOCK_BYTES = 144;
+constexpr int QK_PART_PITCH = QK_BN + 4;                   // fp32 row pitch of a partial tile (conflict-free rows)
+constexpr int QK_MAX_SPLIT = 8;
 static_assert(2 * (QK_SMEM + 1024) <= 233472, "two Q4_K GEMM CTAs per SM");
+static_assert(QK_BM * QK_PART_PITCH * 4 <= QK_OFF_BAR, "a partial tile fits over the stage ring");
+
+__device__ __forceinline__ uint32_t qk_cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void qk_cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 16 bytes at this CTA's shared address `p` as seen in CTA `rank` of the cluster.
+__device__ __forceinline__ float4 qk_ld_cluster(const void *p, uint32_t rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(a)
+                 : "memory");
+    return v;
+}
 
 __device__ __forceinline__ uint32_t qk_swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
@@ -55,7 +86,7 @@ __device__ __forceinline__ float nib_f(uint32_t q) { return __uint_as_float(0x4B
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(QK_THREADS, 2)
 q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__restrict__ w, int M, int N, int K,
-                void *__restrict__ y, int *status) {
+                void *__restrict__ y, int split, int *status) {
     pdl_launch_dependents();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -68,7 +99,10 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int n0 = blockIdx.x * QK_BN, m0 = blockIdx.y * QK_BM;
-    const int num_k = K / QK_BK, nb = K / 256;
+    const int nb = K / 256;
+    // this CTA's K range (all of K without split): k-tiles [kt0, kt0 + num_k)
+    const uint32_t crank = split > 1 ? qk_cluster_rank() : 0u;
+    const int num_k = K / QK_BK / split, kt0 = (int)crank * num_k;
 
     if (tid == 0) {
         for (int s = 0; s < QK_STAGES; ++s) {
@@ -92,11 +126,11 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
 
     if (warp == 0) {
         if (lane == 0) {
-            for (int kt = 0; kt < num_k; ++kt) {
-                const int s = kt % QK_STAGES;
-                if (!mbar_wait(&empty[s], (uint32_t)(((kt / QK_STAGES) & 1) ^ 1), status)) break;
+            for (int i = 0; i < num_k; ++i) {
+                const int s = i % QK_STAGES;
+                if (!mbar_wait(&empty[s], (uint32_t)(((i / QK_STAGES) & 1) ^ 1), status)) break;
                 mbar_arrive_expect_tx(&a_full[s], QK_TILE);
-                tma_load_2d(tile_a(s), &map_a, &a_full[s], kt * QK_BK, m0);
+                tma_load_2d(tile_a(s), &map_a, &a_full[s], (kt0 + i) * QK_BK, m0);
             }
             // before the CTA may exit: the last load armed on each stage has landed
             for (int s = 0; s < QK_STAGES && s < num_k; ++s) {
@@ -110,18 +144,18 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
             const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(QK_BN >> 3) << 17) |
                                    ((uint32_t)(QK_BM >> 4) << 24);
             int issued = 0;
-            for (int kt = 0; kt < num_k; ++kt) {
-                const int s = kt % QK_STAGES;
-                const uint32_t ph = (uint32_t)((kt / QK_STAGES) & 1);
+            for (int i = 0; i < num_k; ++i) {
+                const int s = i % QK_STAGES;
+                const uint32_t ph = (uint32_t)((i / QK_STAGES) & 1);
                 if (!mbar_wait(&a_full[s], ph, status) || !mbar_wait(&b_full[s], ph, status)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < QK_BK / 16; ++kk)
                     qk_mma(tmem, smem_desc(smem_u32(tile_a(s)) + kk * 32, 16, 1024, 2),
-                           smem_desc(smem_u32(tile_b(s)) + kk * 32, 16, 1024, 2), idesc, (kt | kk) ? 1u : 0u);
+                           smem_desc(smem_u32(tile_b(s)) + kk * 32, 16, 1024, 2), idesc, (i | kk) ? 1u : 0u);
                 tc_commit(&empty[s]);
                 ++issued;
-                if (kt == num_k - 1) tc_commit(acc_full);
+                if (i == num_k - 1) tc_commit(acc_full);
             }
             // before tensor memory is freed: every MMA issued has completed (bounded)
             if (issued) {
@@ -136,8 +170,9 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
         const uint8_t *wrow = w + (size_t)n * nb * QK_BLOCK_BYTES;
         bool ok = true;
         float ds[2] = {0.f, 0.f}, dm[2] = {0.f, 0.f};
-        for (int kt = 0; kt < num_k && ok; ++kt) {
-            const int s = kt % QK_STAGES, g = kt & 3;
+        for (int i = 0; i < num_k && ok; ++i) {
+            const int kt = kt0 + i;
+            const int s = i % QK_STAGES, g = kt & 3;
             const uint8_t *blk = wrow + (size_t)(kt >> 2) * QK_BLOCK_BYTES;
             // the quant bytes of this stage's 64 values (sub-blocks 2 g and 2 g + 1) and, at a block's
             // first stage, the block header, before the wait for the stage to be free
@@ -160,7 +195,7 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
                 ds[h2] = d * (float)scale;
                 dm[h2] = dmin * (float)mn;
             }
-            if (lane == 0) ok = mbar_wait(&empty[s], (uint32_t)(((kt / QK_STAGES) & 1) ^ 1), status);
+            if (lane == 0) ok = mbar_wait(&empty[s], (uint32_t)(((i / QK_STAGES) & 1) ^ 1), status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             // values 0-31 of the stage: low nibbles (sub-block 2 g); 32-63: high nibbles (2 g + 1)
@@ -191,7 +226,24 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
             if (lane == 0) ok = mbar_wait(acc_full, 0, status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
         }
-        if (ok) {
+        if (ok && split > 1) {
+            // the partial tile into this CTA's shared memory (the stage ring is idle: every load
+            // was consumed by an MMA that has completed), row = tensor-memory lane
+            tc_fence_after();
+            const uint32_t lb = ((uint32_t)(quarter * 32)) << 16;
+            float *prow = reinterpret_cast<float *>(sm) + (size_t)(quarter * 32 + lane) * QK_PART_PITCH;
+#pragma unroll 1
+            for (int c32 = 0; c32 < QK_BN / 32; ++c32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lb + c32 * 32, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<float4 *>(prow + c32 * 32 + 4 * i) =
+                        make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                    __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+            }
+        } else if (ok) {
             tc_fence_after();
             const int m = m0 + quarter * 32 + lane;
             const uint32_t lb = ((uint32_t)(quarter * 32)) << 16;
@@ -223,6 +275,38 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
                 }
             }
         }
+    }
+    if (split > 1) {
+        // every CTA of the cluster reaches both barriers, on the failure path too (its partial is
+        // then stale and the status word already says so)
+        qk_cluster_sync();
+        const int rows = QK_BM / split, r0 = (int)crank * rows;
+        for (int u = tid; u < rows * (QK_BN / 4); u += QK_THREADS) {
+            const int rr = r0 + u / (QK_BN / 4), c4 = u % (QK_BN / 4);
+            const float *src = reinterpret_cast<const float *>(sm) + (size_t)rr * QK_PART_PITCH + 4 * c4;
+            float4 acc = qk_ld_cluster(src, 0);
+            for (int z = 1; z < split; ++z) {
+                const float4 v = qk_ld_cluster(src, (uint32_t)z);
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+            }
+            const int m = m0 + rr;
+            if (m < M) {
+                if constexpr (OUT_BF16) {
+                    const __nv_bfloat162 p0 = __floats2bfloat162_rn(acc.x, acc.y);
+                    const __nv_bfloat162 p1 = __floats2bfloat162_rn(acc.z, acc.w);
+                    uint2 u2;
+                    u2.x = *reinterpret_cast<const uint32_t *>(&p0);
+                    u2.y = *reinterpret_cast<const uint32_t *>(&p1);
+                    *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(y) + (size_t)m * N + n0 + 4 * c4) = u2;
+                } else {
+                    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(y) + (size_t)m * N + n0 + 4 * c4) = acc;
+                }
+            }
+        }
+        qk_cluster_sync();
     }
     tc_fence_before();
     __syncthreads();
@@ -264,21 +348,41 @@ cudaError_t launch_q4k_gemm(const Q4kGemmArgs &g, cudaStream_t st) {
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    static PerDevice<int> attr;
-    int unused = 0;
-    cudaError_t e = attr.get(
-        [](int, int &) {
-            cudaError_t r = cudaFuncSetAttribute(q4k_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, QK_SMEM);
-            if (r == cudaSuccess)
-                r = cudaFuncSetAttribute(q4k_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, QK_SMEM);
-            return r;
+    static PerDevice<int> sm_count;   // the shared-memory attribute is set per device alongside
+    int sms = 0;
+    cudaError_t e = sm_count.get(
+        [](int dev, int &r) {
+            cudaError_t x = cudaFuncSetAttribute(q4k_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, QK_SMEM);
+            if (x == cudaSuccess)
+                x = cudaFuncSetAttribute(q4k_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, QK_SMEM);
+            if (x == cudaSuccess) x = cudaDeviceGetAttribute(&r, cudaDevAttrMultiProcessorCount, dev);
+            return x;
         },
-        &unused);
+        &sms);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)(g.N / QK_BN), (unsigned)((g.M + QK_BM - 1) / QK_BM));
+    const int tiles = (g.N / QK_BN) * ((g.M + QK_BM - 1) / QK_BM);
+    const int num_k = g.K / QK_BK;
+    int split = 1;   // double while the CTAs still fit at two per SM and every range keeps a whole block
+    while (split < QK_MAX_SPLIT && tiles * split * 2 <= 2 * sms && num_k % (2 * split) == 0 &&
+           num_k / (2 * split) >= 256 / QK_BK)
+        split *= 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(g.N / QK_BN), (unsigned)((g.M + QK_BM - 1) / QK_BM), (unsigned)split);
+    cfg.blockDim = dim3(QK_THREADS);
+    cfg.dynamicSmemBytes = QK_SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attrs[2];
+    attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[0].val.programmaticStreamSerializationAllowed = 1;
+    attrs[1].id = cudaLaunchAttributeClusterDimension;
+    attrs[1].val.clusterDim.x = 1;
+    attrs[1].val.clusterDim.y = 1;
+    attrs[1].val.clusterDim.z = (unsigned)split;
+    cfg.attrs = attrs;
+    cfg.numAttrs = split > 1 ? 2 : 1;
     if (g.out_bf16)
-        return launch_pdl(q4k_gemm_kernel<true>, grid, dim3(QK_THREADS), QK_SMEM, st, ma, g.w, g.M, g.N, g.K, g.y, g.status);
-    return launch_pdl(q4k_gemm_kernel<false>, grid, dim3(QK_THREADS), QK_SMEM, st, ma, g.w, g.M, g.N, g.K, g.y, g.status);
+        return cudaLaunchKernelEx(&cfg, q4k_gemm_kernel<true>, ma, g.w, g.M, g.N, g.K, g.y, split, g.status);
+    return cudaLaunchKernelEx(&cfg, q4k_gemm_kernel<false>, ma, g.w, g.M, g.N, g.K, g.y, split, g.status);
 }
 
 }  // namespace gdn
