@@ -109,6 +109,7 @@ gdn_status gdn_prefill_chunked(const void *q, const void *k, const void *v, cons
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (Dk == 128 && in_dtype == GDN_BF16 && T > 0) {
+        if (!gdn::chunked_size_ok(T, num_seqs)) return GDN_ERR_UNSUPPORTED;
         const size_t need = gdn::chunked_workspace_bytes(T, num_seqs, Hk, Hv);
         if (!workspace || workspace_bytes < need || !aligned16(workspace)) return GDN_ERR_WORKSPACE;
         gdn::ChunkedArgs c{q, k, v, a, b, A_log, dt_bias, cu_seqlens, T, num_seqs, Hk, Hv, scale, qk_l2norm,
@@ -144,6 +145,7 @@ gdn_status gdn_prefill_chunked_gated_nvfp4(const void *q, const void *k, const v
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) || (o && !aligned16(o)) ||
         (reinterpret_cast<uintptr_t>(xq) & 3u))
         return GDN_ERR_INVALID_ARG;
+    if (!gdn::chunked_size_ok(T, num_seqs)) return GDN_ERR_UNSUPPORTED;
     const size_t need = gdn::chunked_workspace_bytes(T, num_seqs, Hk, Hv);
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return GDN_ERR_WORKSPACE;
     gdn::ChunkedArgs c{q, k, v, a, b, A_log, dt_bias, cu_seqlens, T, num_seqs, Hk, Hv, scale, qk_l2norm, true,

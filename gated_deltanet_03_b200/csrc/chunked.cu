@@ -62,21 +62,27 @@ constexpr size_t kSegItemBytes = 196608;
 // run in parallel (state and transition passes), a short sequential combine, and the output
 // pass. Picks the length that minimises a cost model of the three passes - per-chunk costs of
 // the output pass (one CTA per SM) and of the state / transition passes (two CTAs per SM) and the
-// cost of one combine step, fitted to fused-prefill timings on B200 over 4096 - 32768 tokens and
-// 16 - 32 value heads, with CTA waves counted fractionally above one - from the mean sequence
-// length (the host does not read cu_seqlens).
+// cost of one combine step - fitted to fused-prefill timings on B200 over 8192 - 32768 tokens
+// (segment lengths 4 - 256, powers of two and others), within 1 % of every timing once a constant
+// per workload is allowed for the prep kernel. CTA waves above one count halfway between their
+// fraction and the next whole wave (a second wave of equal CTAs costs a whole wave, but CTAs
+// finish unevenly). A single sequence searches every length; a batch is planned from its mean
+// sequence length (the host does not read cu_seqlens) over powers of two only, since one long
+// sequence in a skewed batch sets the chain's length whatever the mean says.
 int chunked_segment_chunks(int T, int num_seqs, int Hv) {
-    const double nch = (double)T / kChunk / (num_seqs > 0 ? num_seqs : 1);
-    const double c_full = 2.0, c_state = 0.5, c_comb = 4.0, sms = 148.0;
+    const int nseq = num_seqs > 0 ? num_seqs : 1;
+    const double nch = (double)T / kChunk / nseq;
+    const double c_full = 2.0, c_state = 1.4, c_comb = 3.0, sms = 148.0;
+    auto waves = [](double x) { return x <= 1.0 ? 1.0 : 0.5 * (x + std::ceil(x)); };
     int best = 1 << 30;
     double best_cost = 1e30;
-    for (int seg = 4; seg <= 4096; seg *= 2) {
+    for (int seg = 4; seg <= 4096; seg = nseq == 1 ? seg + 1 : seg * 2) {
         const double nseg = nch / seg > 1.0 ? std::ceil(nch / seg) : 1.0;
-        const double ctas = (double)Hv * num_seqs * nseg;
-        double cost = std::max(1.0, ctas / sms) * std::min((double)seg, nch) * c_full;
+        const double ctas = (double)Hv * nseq * nseg;
+        double cost = waves(ctas / sms) * std::min((double)seg, nch) * c_full;
         if (nseg > 1.0) {
-            const double lean_ctas = 2.0 * Hv * num_seqs * (nseg - 1.0);
-            cost += std::max(1.0, lean_ctas / (2.0 * sms)) * seg * c_state + (nseg - 2.0) * c_comb;
+            const double lean_ctas = 2.0 * Hv * nseq * (nseg - 1.0);
+            cost += waves(lean_ctas / (2.0 * sms)) * seg * c_state + (nseg - 2.0) * c_comb;
         }
         if (cost < best_cost) {
             best_cost = cost;
@@ -187,28 +193,29 @@ __device__ __forceinline__ void mma_bf16_m16n8k16(float (&c)[4], const uint32_t 
 }
 
 // ===================================================================================
-// Prep kernel: one CTA per (chunk slot, value head); two CTAs per SM.
+// Prep kernel: one CTA per (chunk slot, value head); three CTAs per SM (68 KB of shared memory,
+// 128 tensor-memory columns, at most 80 registers a thread).
 // ===================================================================================
-// Shared memory (TILE = 8 KB). [K_lo; Q_lo] and [K_hi; Q_hi] are the two K-major column blocks
-// of the MMA1 operand [K; Q]; K_lo, K_hi, V_lo, V_hi sit 3 TILE apart so that [K | V] is one
-// MN-major B operand with N = 256 for MMA2. The A operands of MMA2 are [T'; T''] split into
-// bf16 hi and lo parts (16 KB each): hi in the free tiles 7-8, lo over Q_lo and tile 2 once the
-// Q' image is written. Tiles 5 and 2 first stage the P^T hi / lo images between the D1 readout
-// and their copy-out. After MMA2 the W (fp16) and U~ (fp32) staging reuses tiles 0-5.
-constexpr int P_OFF_KLO = 0, P_OFF_QLO = TILE, P_OFF_KHI = 3 * TILE, P_OFF_QHI = 4 * TILE;
-constexpr int P_OFF_ALO = TILE;                    // [T'_lo; T''_lo], after the Q' image
-constexpr int P_OFF_PHI = 5 * TILE, P_OFF_PLO = 2 * TILE;   // P^T hi / lo staging (D1 readout -> copy-out)
-constexpr int P_OFF_VLO = 6 * TILE, P_OFF_AHI = 7 * TILE, P_OFF_VHI = 9 * TILE;
+// Shared memory (TILE = 8 KB). [K_lo; Q_lo] (tiles 0-1) and [K_hi; Q_hi] (tiles 2-3) are the two
+// K-major column blocks of the MMA1 operand [K; Q]; K_lo and K_hi, 2 TILE apart, are also the
+// MN-major B operand K of MMA2a. Once MMA1 has completed and the Q' rows are written out, V is
+// loaded into the Q tiles (V_lo over Q_lo, V_hi over Q_hi: the B operand of MMA2b, blocks 2 TILE
+// apart as well). Tiles 4-6 hold the fp32 A / T array; once T is in registers, tiles 4-7 take
+// the bf16 hi (4-5) and lo (6-7) images of [T'; T''], the A operand of MMA2a and MMA2b. P^T, W
+// and U~ go from registers straight into the workspace item.
+constexpr int P_OFF_KLO = 0, P_OFF_QLO = TILE, P_OFF_KHI = 2 * TILE, P_OFF_QHI = 3 * TILE;
+constexpr int P_OFF_VLO = P_OFF_QLO, P_OFF_VHI = P_OFF_QHI;
 constexpr int P_AT = 72;                           // fp32 row pitch of the A / T array (8-byte fragment loads
                                                    // of a warp-level MMA without bank conflicts)
-constexpr int P_OFF_AT = 10 * TILE;                // T (strict lower, row-major) and A (strict lower, transposed)
-constexpr int P_OFF_VEC = P_OFF_AT + 64 * P_AT * 4; // G, beta, rk, rq, gamma, c, beta gamma rk, spare (64 each)
+constexpr int P_OFF_AT = 4 * TILE;                 // T (strict lower, row-major) and A (strict lower, transposed)
+constexpr int P_OFF_AHI = 4 * TILE, P_OFF_ALO = 6 * TILE;   // [T'; T''] hi / lo, after T is read
+constexpr int P_OFF_VEC = 8 * TILE;                // G, beta, rk, rq, gamma, c, beta gamma rk, spare (64 each)
 constexpr int P_OFF_BAR = P_OFF_VEC + 8 * 64 * 4;
 constexpr int P_SMEM = P_OFF_BAR + 64 + 1024;
-constexpr int P_OFF_WSTG = 0, P_OFF_USTG = 2 * TILE;   // W fp16 image, U~ fp32 rows (after MMA2)
-static_assert(P_SMEM * 2 + 2048 <= 233472, "two prep CTAs per SM");
-static_assert(P_OFF_USTG + 4 * TILE <= P_OFF_VLO, "staging stays clear of V_lo until MMA2 is done");
-// tensor memory: D1 = [K; Q] [K; Q]^T (128 columns), then D2 = [T'; T''] [K | V] (256) over it
+static_assert(P_OFF_AT + 64 * P_AT * 4 <= P_OFF_VEC, "the A / T array stays clear of the vectors");
+static_assert(3 * (P_SMEM + 1024) <= 233472, "three prep CTAs per SM");
+// tensor memory (128 columns): D1 = [K; Q] [K; Q]^T, then D2a = [T'; T''] K (rows 0-63: W) and
+// D2b = [T'; T''] V (rows 64-127: U~) in turn over it
 constexpr uint32_t P_TM_D1 = 0, P_TM_D2 = 0;
 
 // bf16 hi / lo split of two fp32 values, packed as bf16x2 words: hi = bf16(x), lo = bf16(x - hi).
@@ -220,14 +227,16 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uin
     lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
-__global__ void __launch_bounds__(NT, 2)
+__global__ void __launch_bounds__(NT, 3)
 gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict__ ga, const float *__restrict__ gb,
                       const float *__restrict__ A_log, const float *__restrict__ dt_bias,
                       const int32_t *__restrict__ cu_seqlens, int32_t T, int32_t num_seqs, int32_t Hk, int32_t Hv,
                       int32_t slots, float scale, int32_t l2norm, uint8_t *__restrict__ ws, int *status) {
     pdl_launch_dependents();
     pdl_wait();
-    const int id = blockIdx.x, h = blockIdx.y;
+    // heads fastest: the value heads of a chunk run together, so the gate rows they read and the
+    // K and Q tiles that value heads of one key head share come from DRAM once
+    const int h = blockIdx.x, id = blockIdx.y;
     int n, t_begin, t_end;
     locate(id, cu_seqlens, num_seqs, T, n, t_begin, t_end);
     const int t0 = t_begin + (id - (t_begin / C + n)) * C;
@@ -253,7 +262,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     const int x = (warp % 4) * 32 + lane;   // this thread's TMEM lane
     const uint32_t lane_base = ((uint32_t)((warp % 4) * 32)) << 16;
     // what thread 0 has issued, for the drain on the failure path
-    bool loads_issued = false;
+    bool loads_issued = false, v_issued = false;
     int mmas_issued = 0;
     bool failed = false;
 
@@ -264,20 +273,17 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         mbar_init(bar_drain, 1);
         fence_barrier_init();
         if (!(ctl_flags(status) & kInjectSkipPrepLoads)) {
-            // K and Q on one barrier (MMA1 starts when they land), V on its own (needed by MMA2)
+            // K and Q on one barrier (MMA1 starts when they land); V follows into the Q tiles later
             mbar_arrive_expect_tx(bar_tma, 4 * TILE);
             tma_load_3d(sm + P_OFF_KLO, &maps.k, bar_tma, 0, hk, t0);
             tma_load_3d(sm + P_OFF_QLO, &maps.q, bar_tma, 0, hk, t0);
             tma_load_3d(sm + P_OFF_KHI, &maps.k, bar_tma, 64, hk, t0);
             tma_load_3d(sm + P_OFF_QHI, &maps.q, bar_tma, 64, hk, t0);
-            mbar_arrive_expect_tx(bar_v, 2 * TILE);
-            tma_load_3d(sm + P_OFF_VLO, &maps.v, bar_v, 0, h, t0);
-            tma_load_3d(sm + P_OFF_VHI, &maps.v, bar_v, 64, h, t0);
             loads_issued = true;
         }
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 128);
         tmem_relinquish();
     }
     // gates and the warp-local part of the cumulative log decay, while the tiles stream in
@@ -324,23 +330,21 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
     if (!__syncthreads_and(ok)) { failed = true; goto teardown; }
     tc_fence_after();
     {
-        // every warp reads 32 columns (key tokens s) of its 32 lanes; warps 2 and 3 also read the
+        // every warp reads 32 columns (key tokens s) of its 32 lanes; warps 2 and 3 first read the
         // Q Q^T block that holds their lanes' diagonal
         uint32_t r32[32];
-        tmem_ld32(tmem + P_TM_D1 + lane_base + wg * 32, r32);
         const int quarter = warp % 4;
         if (wg == 0 && quarter >= 2) {
-            uint32_t rq32[32];
-            tmem_ld32(tmem + P_TM_D1 + lane_base + 64 + (quarter - 2) * 32, rq32);
+            tmem_ld32(tmem + P_TM_D1 + lane_base + 64 + (quarter - 2) * 32, r32);
             tmem_ld_wait();
             float d = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) d = (j == lane) ? __uint_as_float(rq32[j]) : d;
+            for (int j = 0; j < 32; ++j) d = (j == lane) ? __uint_as_float(r32[j]) : d;
             const int r = x - 64;
             sRq[r] = r < L ? (l2norm ? rsqrtf(d + 1e-6f) * scale : scale) : 0.0f;
-        } else {
-            tmem_ld_wait();
         }
+        tmem_ld32(tmem + P_TM_D1 + lane_base + wg * 32, r32);
+        tmem_ld_wait();
         if (quarter < 2 && wg == quarter) {
             // lanes 0-63: the K K^T diagonal sits in column x, i.e. this warp's column `lane`
             float d = 0.0f;
@@ -352,16 +356,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             sDec[r] = r < L ? __expf(sG[L - 1] - sG[r]) * rk : 0.0f;
         }
         __syncthreads();
-        // decay and key-norm factors of this warp's 32 columns (same for all lanes), then all 32
-        // values, then the stores
-        float gs[32], rks[32], vals[32];
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            const float4 g4 = *reinterpret_cast<const float4 *>(sG + wg * 32 + j);
-            const float4 k4 = *reinterpret_cast<const float4 *>(sRk + wg * 32 + j);
-            gs[j] = g4.x; gs[j + 1] = g4.y; gs[j + 2] = g4.z; gs[j + 3] = g4.w;
-            rks[j] = k4.x; rks[j + 1] = k4.y; rks[j + 2] = k4.z; rks[j + 3] = k4.w;
-        }
+        // this warp's 32 columns (key tokens s), two at a time; the decay and key-norm factors of a
+        // column pair come from shared memory (the same address for every lane)
         if (x < 64) {
             // row r of A (fp32): A_rs = beta_r exp(G_r - G_s) k_r.k_s / (|k_r| |k_s|) for s < r < L
             const int r = x;
@@ -369,36 +365,40 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
             const f2_t cr2 = f2(cr, cr);
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-                const f2_t v2 = mul2(mul2(f2(exp_approx(Gr - gs[j]), exp_approx(Gr - gs[j + 1])),
+                const int s0 = wg * 32 + j;
+                const float2 g2 = *reinterpret_cast<const float2 *>(sG + s0);
+                const float2 k2 = *reinterpret_cast<const float2 *>(sRk + s0);
+                const f2_t v2 = mul2(mul2(f2(exp_approx(Gr - g2.x), exp_approx(Gr - g2.y)),
                                           f2(__uint_as_float(r32[j]), __uint_as_float(r32[j + 1]))),
-                                     mul2(f2(rks[j], rks[j + 1]), cr2));
-                vals[j] = (wg * 32 + j < r) ? f2lo(v2) : 0.0f;
-                vals[j + 1] = (wg * 32 + j + 1 < r) ? f2hi(v2) : 0.0f;
+                                     mul2(f2(k2.x, k2.y), cr2));
+                if (s0 < r) AT[s0 * P_AT + r] = f2lo(v2);
+                if (s0 + 1 < r) AT[(s0 + 1) * P_AT + r] = f2hi(v2);
             }
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (wg * 32 + j < r) AT[(wg * 32 + j) * P_AT + r] = vals[j];
         } else {
-            // row r of P = (Q K^T o Gamma) scaled, as bf16 hi and lo P^T images [s][r] (MN-major
-            // over r, 128-byte swizzled), staged for the copy-out
+            // row r of P = (Q K^T o Gamma) scaled, as bf16 hi and lo P^T images [s][r] (MN-major over
+            // r, 128-byte swizzled), written straight into the workspace item (zeros above the
+            // diagonal, so the images are whole)
             const int r = x - 64;
             const float Gr = sG[r], cr = sRq[r];
             const f2_t cr2 = f2(cr, cr);
+            uint8_t *pimg = item + kWsP;
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-                const f2_t v2 = mul2(mul2(f2(exp_approx(Gr - gs[j]), exp_approx(Gr - gs[j + 1])),
+                const int s0 = wg * 32 + j;
+                const float2 g2 = *reinterpret_cast<const float2 *>(sG + s0);
+                const float2 k2 = *reinterpret_cast<const float2 *>(sRk + s0);
+                const f2_t v2 = mul2(mul2(f2(exp_approx(Gr - g2.x), exp_approx(Gr - g2.y)),
                                           f2(__uint_as_float(r32[j]), __uint_as_float(r32[j + 1]))),
-                                     mul2(f2(rks[j], rks[j + 1]), cr2));
-                vals[j] = (wg * 32 + j <= r) ? f2lo(v2) : 0.0f;
-                vals[j + 1] = (wg * 32 + j + 1 <= r) ? f2hi(v2) : 0.0f;
-            }
+                                     mul2(f2(k2.x, k2.y), cr2));
+                const float pv[2] = {s0 <= r ? f2lo(v2) : 0.0f, s0 + 1 <= r ? f2hi(v2) : 0.0f};
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const __nv_bfloat16 hb = __float2bfloat16_rn(vals[j]);
-                const __nv_bfloat16 lb = __float2bfloat16_rn(vals[j] - __bfloat162float(hb));
-                const uint32_t off = swz(wg * 32 + j, r >> 3) + (r & 7) * 2;
-                *reinterpret_cast<__nv_bfloat16 *>(sm + P_OFF_PHI + off) = hb;
-                *reinterpret_cast<__nv_bfloat16 *>(sm + P_OFF_PLO + off) = lb;
+                for (int e = 0; e < 2; ++e) {
+                    const __nv_bfloat16 hb = __float2bfloat16_rn(pv[e]);
+                    const __nv_bfloat16 lb = __float2bfloat16_rn(pv[e] - __bfloat162float(hb));
+                    const uint32_t off = swz(s0 + e, r >> 3) + (r & 7) * 2;
+                    *reinterpret_cast<__nv_bfloat16 *>(pimg + off) = hb;
+                    *reinterpret_cast<__nv_bfloat16 *>(pimg + TILE + off) = lb;
+                }
             }
         }
     }
@@ -453,20 +453,6 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
                 }
             }
         }
-        // the P^T hi and lo images from their staging (1024 chunks)
-        {
-            uint4 pc[6];
-#pragma unroll
-            for (int e = 0; e < 6; ++e) {
-                const int c16 = e * 192 + t6, w = c16 < 1024 ? c16 : 0;
-                pc[e] = *reinterpret_cast<const uint4 *>(sm + (w < 512 ? P_OFF_PHI : P_OFF_PLO) + (w & 511) * 16);
-            }
-#pragma unroll
-            for (int e = 0; e < 6; ++e) {
-                const int c16 = e * 192 + t6;
-                if (c16 < 1024) *reinterpret_cast<uint4 *>(item + kWsP + c16 * 16) = pc[e];
-            }
-        }
         // the per-token factors of the state update, c_r = gamma_C / gamma_r / |k_r|, and gamma_C
         if (t6 < 64) reinterpret_cast<float *>(item + kWsVec)[t6] = sDec[t6];
         if (t6 == 64) reinterpret_cast<float *>(item + kWsVec)[64] = L > 0 ? __expf(sG[L - 1]) : 1.0f;
@@ -474,9 +460,14 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         if (t6 >= 128) sBG[t6 - 128] = sBeta[t6 - 128] * sGam[t6 - 128] * sRk[t6 - 128];
     }
     __syncthreads();
-    // ---- off-diagonal blocks level by level, from T (I + A) = I:
-    //      X = sum_{k in blocks bj+1 .. bi} T[r][k] A[k][c],   T[r][c] = -(X T_jj)[r][c],
-    //      r in block bi, c in block bj; every thread one element of each block of the level.
+    // MMA1 has completed and the Q' rows are out: V into the Q tiles (needed by MMA2b)
+    if (tid == 0 && loads_issued) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar_v, 2 * TILE);
+        tma_load_3d(sm + P_OFF_VLO, &maps.v, bar_v, 0, h, t0);
+        tma_load_3d(sm + P_OFF_VHI, &maps.v, bar_v, 64, h, t0);
+        v_issued = true;
+    }
     // ---- off-diagonal blocks level by level, from T (I + A) = I:
     //      X = sum_{bk = bj+1 .. bi} T_{bi,bk} A_{bk,bj},   T_{bi,bj} = -X T_{bj,bj},
     //      one warp per block on the warp-level tensor-core MMA (m16n8k16) with every operand split
@@ -553,90 +544,108 @@ gdn_chunk_prep_kernel(const __grid_constant__ Maps maps, const float *__restrict
         }
         __syncthreads();
     }
-    // ---- the A operands of MMA2 as bf16 hi / lo K-major images (128-byte swizzle):
-    //      rows 0-63 T' = T diag(beta gamma / |k|), rows 64-127 T'' = T diag(beta)
+    // ---- the A operand of MMA2a / MMA2b as bf16 hi / lo K-major images (128-byte swizzle):
+    //      rows 0-63 T' = T diag(beta gamma / |k|), rows 64-127 T'' = T diag(beta). The images
+    //      overwrite the A / T array, so every thread first takes its 16 values of T.
+    {
+        float tv[2][8];
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        const int idx = e * NT + tid, r = idx >> 3, ch = idx & 7;
-        float t[8];
+        for (int e = 0; e < 2; ++e) {
+            const int idx = e * NT + tid, r = idx >> 3, ch = idx & 7;
+            // two 16-byte loads of row r (the eight lanes of a row read 256 contiguous bytes)
+            const float4 a0 = *reinterpret_cast<const float4 *>(AT + r * P_AT + ch * 8);
+            const float4 a1 = *reinterpret_cast<const float4 *>(AT + r * P_AT + ch * 8 + 4);
+            const float raw[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int s = ch * 8 + j;
-            t[j] = (s < r) ? AT[r * P_AT + s] : (s == r ? 1.0f : 0.0f);
+            for (int j = 0; j < 8; ++j) {
+                const int s0 = ch * 8 + j;
+                tv[e][j] = (s0 < r) ? raw[j] : (s0 == r ? 1.0f : 0.0f);
+            }
         }
-        uint32_t h1[4], l1[4], h2[4], l2[4];
+        __syncthreads();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int s = ch * 8 + 2 * j;
-            split_bf16x2(t[2 * j] * sBG[s], t[2 * j + 1] * sBG[s + 1], h1[j], l1[j]);
-            split_bf16x2(t[2 * j] * sBeta[s], t[2 * j + 1] * sBeta[s + 1], h2[j], l2[j]);
+        for (int e = 0; e < 2; ++e) {
+            const int idx = e * NT + tid, r = idx >> 3, ch = idx & 7;
+            uint32_t h1[4], l1[4], h2[4], l2[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int s0 = ch * 8 + 2 * j;
+                split_bf16x2(tv[e][2 * j] * sBG[s0], tv[e][2 * j + 1] * sBG[s0 + 1], h1[j], l1[j]);
+                split_bf16x2(tv[e][2 * j] * sBeta[s0], tv[e][2 * j + 1] * sBeta[s0 + 1], h2[j], l2[j]);
+            }
+            const uint32_t off = swz(r, ch);
+            *reinterpret_cast<uint4 *>(sm + P_OFF_AHI + off) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+            *reinterpret_cast<uint4 *>(sm + P_OFF_AHI + TILE + off) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+            *reinterpret_cast<uint4 *>(sm + P_OFF_ALO + off) = make_uint4(l1[0], l1[1], l1[2], l1[3]);
+            *reinterpret_cast<uint4 *>(sm + P_OFF_ALO + TILE + off) = make_uint4(l2[0], l2[1], l2[2], l2[3]);
         }
-        const uint32_t off = swz(r, ch);
-        *reinterpret_cast<uint4 *>(sm + P_OFF_AHI + off) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
-        *reinterpret_cast<uint4 *>(sm + P_OFF_AHI + 8 * 1024 + off) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
-        *reinterpret_cast<uint4 *>(sm + P_OFF_ALO + off) = make_uint4(l1[0], l1[1], l1[2], l1[3]);
-        *reinterpret_cast<uint4 *>(sm + P_OFF_ALO + 8 * 1024 + off) = make_uint4(l2[0], l2[1], l2[2], l2[3]);
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    // D2a = [T'; T''] K and then D2b = [T'; T''] V (N = 128 each, the hi and lo parts of the A
+    // operand accumulated; K and V are the raw bf16 tiles): lanes 0-63 of D2a hold W = T' K, lanes
+    // 64-127 of D2b hold U~ = T'' V. They share the tensor-memory columns, so W is read out between.
     if (tid == 0) {
-        // D2 = [T'; T''] [K | V] with the hi and lo parts of the A operand accumulated: lanes 0-63
-        // columns 0-127 hold W = T' K, lanes 64-127 columns 128-255 hold U~ = T'' V (the other two
-        // quadrants are not used). K and V are the raw bf16 tiles.
+        const uint32_t id2 = idesc_f16(128, false, true, false) | (1u << 7) | (1u << 10);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            mma_f16(tmem + P_TM_D2, kdesc(sm + (kk < 4 ? P_OFF_AHI : P_OFF_ALO) + (kk & 3) * 32),
+                    mndesc(sm + P_OFF_KLO + (kk & 3) * 2048, 2 * TILE), id2, kk > 0 ? 1u : 0u);
+        tc_commit(bar_mma);
+        mmas_issued = 2;
+        ok = mbar_wait(bar_mma, 1, status) ? 1 : 0;
+    }
+    if (!__syncthreads_and(ok)) { failed = true; goto teardown; }
+    tc_fence_after();
+    if (x < 64) {
+        // W row x (fp16): this warp group's 64 key columns are one half of the K-major swizzled
+        // [W; Q'] image
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            uint32_t v[32];
+            tmem_ld32(tmem + P_TM_D2 + lane_base + wg * 64 + hh * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float f8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(v[c * 8 + e]);
+                st_h8(item + kWsWQ + wg * 2 * TILE + swz(x, hh * 4 + c), f8);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
         ok = mbar_wait(bar_v, 0, status) ? 1 : 0;
         if (ok) {
+            const uint32_t id2 = idesc_f16(128, false, true, false) | (1u << 7) | (1u << 10);
             tc_fence_after();
-            const uint32_t id2 = idesc_f16(256, false, true, false) | (1u << 7) | (1u << 10);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
                 mma_f16(tmem + P_TM_D2, kdesc(sm + (kk < 4 ? P_OFF_AHI : P_OFF_ALO) + (kk & 3) * 32),
-                        mndesc(sm + P_OFF_KLO + (kk & 3) * 2048, 3 * TILE), id2, kk > 0 ? 1u : 0u);
+                        mndesc(sm + P_OFF_VLO + (kk & 3) * 2048, 2 * TILE), id2, kk > 0 ? 1u : 0u);
             tc_commit(bar_mma);
-            mmas_issued = 2;
-            ok = mbar_wait(bar_mma, 1, status) ? 1 : 0;
+            mmas_issued = 3;
+            ok = mbar_wait(bar_mma, 0, status) ? 1 : 0;
         }
     }
     if (!__syncthreads_and(ok)) { failed = true; goto teardown; }
     tc_fence_after();
-    {
-        // W rows (fp16, K-major swizzled image halves) and U~ rows (fp32 [s][i], 16-byte groups
-        // XOR-swizzled by s & 7) staged in the dead tile area, then copied out in 16-byte chunks
-        uint32_t v0[32], v1[32];
-        const uint32_t col = (x < 64 ? 0u : 128u) + (uint32_t)wg * 64;
-        tmem_ld32(tmem + P_TM_D2 + lane_base + col, v0);
-        tmem_ld32(tmem + P_TM_D2 + lane_base + col + 32, v1);
-        tmem_ld_wait();
-        if (x < 64) {
+    if (x >= 64) {
+        // U~ row s (fp32 [s][i]): this warp group's 64 value columns
+        const int s0 = x - 64;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float f8[8];
+        for (int hh = 0; hh < 2; ++hh) {
+            uint32_t v[32];
+            tmem_ld32(tmem + P_TM_D2 + lane_base + wg * 64 + hh * 32, v);
+            tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(c < 4 ? v0[c * 8 + e] : v1[(c - 4) * 8 + e]);
-                st_h8(sm + P_OFF_WSTG + wg * TILE + swz(x, c), f8);
-            }
-        } else {
-            const int s = x - 64;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const uint32_t *src = c < 8 ? &v0[c * 4] : &v1[(c - 8) * 4];
-                const int g16 = wg * 16 + c;
-                *reinterpret_cast<uint4 *>(sm + P_OFF_USTG + s * 512 + ((g16 ^ (s & 7)) << 4)) =
-                    make_uint4(src[0], src[1], src[2], src[3]);
-            }
-        }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < 12; ++e) {
-        const int idx = e * NT + tid;   // 1024 chunks of W, then 2048 of U~
-        if (idx < 1024) {
-            *reinterpret_cast<uint4 *>(item + kWsWQ + (idx >> 9) * 2 * TILE + (idx & 511) * 16) =
-                *reinterpret_cast<const uint4 *>(sm + P_OFF_WSTG + idx * 16);
-        } else {
-            const int u = idx - 1024, s = u >> 5, g16 = u & 31;
-            *reinterpret_cast<uint4 *>(item + kWsU + u * 16) =
-                *reinterpret_cast<const uint4 *>(sm + P_OFF_USTG + s * 512 + ((g16 ^ (s & 7)) << 4));
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(item + kWsU + s0 * 512 + (wg * 64 + hh * 32 + c * 4) * 4) =
+                    make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
         }
     }
 teardown:
@@ -648,16 +657,14 @@ teardown:
             tc_commit(bar_drain);
             mbar_wait(bar_drain, 0, status);
         }
-        if (loads_issued) {
-            mbar_wait(bar_tma, 0, status);
-            mbar_wait(bar_v, 0, status);
-        }
+        if (loads_issued) mbar_wait(bar_tma, 0, status);
+        if (v_issued) mbar_wait(bar_v, 0, status);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 128);
     }
 }
 
@@ -1674,7 +1681,8 @@ cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st) {
     const int seg = chunked_segment_chunks(c.T, c.num_seqs, c.Hv);
     const int seg_slots = c.T / (kChunk * seg) + c.num_seqs;
     uint8_t *ws = static_cast<uint8_t *>(c.ws);
-    e = launch_pdl(gdn_chunk_prep_kernel, dim3(slots, c.Hv), dim3(NT), P_SMEM, st, maps, c.a, c.b, c.A_log,
+    if (!chunked_size_ok(c.T, c.num_seqs)) return cudaErrorInvalidValue;
+    e = launch_pdl(gdn_chunk_prep_kernel, dim3(c.Hv, slots), dim3(NT), P_SMEM, st, maps, c.a, c.b, c.A_log,
                                c.dt_bias, c.cu_seqlens, c.T, c.num_seqs, c.Hk, c.Hv, slots, c.scale, c.l2norm, ws,
                                c.status);
     if (e != cudaSuccess) return e;

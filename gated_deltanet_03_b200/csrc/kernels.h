@@ -108,6 +108,8 @@ struct ChunkedArgs {
     uint8_t *xq, *xs;            // [T, Hv * 64], [T, Hv * 8]
 };
 size_t chunked_workspace_bytes(int T, int num_seqs, int Hk, int Hv);
+// The prep grid's y dimension counts the chunk slots (T / 64 + num_seqs), at most 65535.
+inline bool chunked_size_ok(int T, int num_seqs) { return (int64_t)T / 64 + num_seqs <= 65535; }
 cudaError_t launch_chunked(const ChunkedArgs &c, cudaStream_t st);
 
 struct TailArgs {

@@ -85,7 +85,8 @@ typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
  *             aligned, owned by the caller; its contents on entry do not matter and are
  *             overwritten. GDN_ERR_WORKSPACE if it is needed and missing or too small.
  * Supported: Dk == Dv in {16, 32, 64, 128}; Hv % Hk == 0; T >= 0 (T == 0 only writes
- * final_state = initial_state). Dk == Dv == 128 with bf16 inputs runs the tensor-core
+ * final_state = initial_state); on the tensor-core path T / 64 + num_seqs <= 65535 (about
+ * 4.19 M tokens; GDN_ERR_UNSUPPORTED beyond). Dk == Dv == 128 with bf16 inputs runs the tensor-core
  * chunked path (64-token chunks; a prep kernel parallel over chunks writes the
  * state-independent operands to the workspace; long sequences are cut into segments whose
  * states and transition matrices are computed in parallel and combined in order; a chain

@@ -46,6 +46,12 @@ def test_host_validation_rejects_bad_arguments_without_cuda():
     # several sequences without cu_seqlens
     assert L.gdn_prefill_chunked(P, P, P, P, P, P, P, P, 2, 8, 2, 4, 128, 128, 1.0, 1, 0, P, P, P, 0, P,
                                  0, P) == g.GDN_ERR_INVALID_ARG
+    # more chunk slots than the prep grid's y dimension holds (T / 64 + num_seqs > 65535): refused
+    # on the host, before any pointer is touched (the pointers are aligned placeholders)
+    A = 1 << 20
+    T_big = 64 * 65535
+    assert L.gdn_prefill_chunked(A, A, A, A, A, A, A, P, 1, T_big, 16, 32, 128, 128, 1.0, 1, 0, P, P, A, 0,
+                                 A, 1 << 40, P) == g.GDN_ERR_UNSUPPORTED
     # unsupported head size
     assert L.gdn_decode_step(P, P, P, P, P, P, P, 4, 1, 1, 96, 96, 1.0, 1, 0, P, P, 0,
                              P) == g.GDN_ERR_UNSUPPORTED
