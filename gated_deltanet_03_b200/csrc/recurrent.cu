@@ -280,11 +280,13 @@ gdn_recurrent128_kernel(const void *__restrict__ q, const void *__restrict__ k, 
 //     o_t = S_t q^_t = gamma_t S0 q^_t + sum_{s<=t} c_{s,t} u_s (k^_s . q^_t),
 // so each state row needs only the 2 T products S0 k_t and S0 q_t (independent of one another,
 // no state update) and T x T scalars shared by the CTA (the Gram dots of the tokens' keys and
-// queries), instead of T dependent rank-one updates.
+// queries), instead of T dependent rank-one updates. At most 96 registers a thread (a few spill),
+// so that five CTAs share an SM: a CTA computes only after its whole state slice has landed, and
+// the fifth CTA keeps more state loads in flight meanwhile.
 constexpr int kVerifyMaxT = 8;
 
 template <bool IN_BF16, bool OUT_BF16>
-__global__ void __launch_bounds__(kR128Threads)
+__global__ void __launch_bounds__(kR128Threads, 5)
 gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
                      const float *__restrict__ a, const float *__restrict__ b, const float *__restrict__ A_log,
                      const float *__restrict__ dt_bias, int32_t T, int32_t Hk, int32_t Hv, float scale,
@@ -414,7 +416,7 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
 // bit for bit. "Red Lite dev15d - DeltaNet gated tail", Pinned graph semantics, steps 1-5.
 constexpr int kFusedDecThreads = 256;
 
-__global__ void __launch_bounds__(kFusedDecThreads)
+__global__ void __launch_bounds__(kFusedDecThreads, 2)
 gdn_decode128_gated_nvfp4_kernel(const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
                                  const float *__restrict__ a, const float *__restrict__ b,
                                  const float *__restrict__ A_log, const float *__restrict__ dt_bias, int32_t Hk,
@@ -441,6 +443,12 @@ gdn_decode128_gated_nvfp4_kernel(const void *__restrict__ q, const void *__restr
             s[p][2 * j] = f2(x.x, x.y);
             s[p][2 * j + 1] = f2(x.z, x.w);
         }
+    // the tail's z row (warp 0: 16 lanes x 8 values), fetched with the state so that its DRAM latency
+    // is not added after the update (the norm weights, shared by every CTA, come from L2 later)
+    const int lr = lane & 15, col = lr * 8;
+    uint4 zu = make_uint4(0u, 0u, 0u, 0u);
+    if (tid < 32)
+        zu = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(z) + ((size_t)n * Hv + h) * D + col);
     float g_alpha = 0.0f, g_beta = 0.0f;
     if (lane == 0) {
         float g;
@@ -493,10 +501,7 @@ gdn_decode128_gated_nvfp4_kernel(const void *__restrict__ q, const void *__restr
     __syncthreads();
     if (tid < 32) {
         // the head row: 16 lanes x 8 values (lanes 16-31 repeat them, their results unused)
-        const int lr = lane & 15, col = lr * 8;
         const uint4 ou = *reinterpret_cast<const uint4 *>(o_s + col);
-        const uint4 zu = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(z) +
-                                                          ((size_t)n * Hv + h) * D + col);
         const f2_t o2[4] = {bf16x2_to_f2(ou.x), bf16x2_to_f2(ou.y), bf16x2_to_f2(ou.z), bf16x2_to_f2(ou.w)};
         const f2_t z2[4] = {bf16x2_to_f2(zu.x), bf16x2_to_f2(zu.y), bf16x2_to_f2(zu.z), bf16x2_to_f2(zu.w)};
         f2_t w2[4];
