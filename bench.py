@@ -266,17 +266,53 @@ def prefill_case(torch, g, w, args, dev, flush, side, with_e2e=False, with_parts
     if with_e2e:
         hq, hk, hv, hz = (t.cpu().pin_memory() for t in (q, k, v, z))
         ha, hb = a.cpu().pin_memory(), b.cpu().pin_memory()
-        hY = torch.empty((T, N), dtype=bf, pin_memory=True)
+        hY = [torch.empty((T, N), dtype=bf, pin_memory=True) for _ in range(2)]
         res["h2d"] = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hz, ha, hb))
-        res["d2h"] = hY.numel() * hY.element_size()
+        res["d2h"] = hY[0].numel() * hY[0].element_size()
+        # two device sets of the inputs and of the output: step i uses set i % 2, so that its
+        # compute overlaps the host -> device copies of step i + 1 and the device -> host copy of
+        # step i - 1 (PCIe carries both directions at once); the workspace and the NVFP4
+        # activations are used by the compute stream only and stay single
+        ins = [(q, k, v, z, a, b), tuple(torch.empty_like(t) for t in (q, k, v, z, a, b))]
+        outs = [Y, torch.empty_like(Y)]
+        cs_in, cs_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
-        def e2e_step():
-            # host -> device inputs, the whole path through the public API, result back to host
-            q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
-            z.copy_(hz, non_blocking=True); a.copy_(ha, non_blocking=True); b.copy_(hb, non_blocking=True)
-            step()
-            hY.copy_(Y, non_blocking=True)
-        res["e2e_step"] = e2e_step
+        def e2e_run(n):
+            """n steps through the public API, every step copying its inputs in from pinned host
+            memory and its output Y back; returns ms per step from the first copy in to the last
+            copy out."""
+            ready = [torch.cuda.Event() for _ in range(2)]
+            done = [torch.cuda.Event() for _ in range(2)]
+            drained = [torch.cuda.Event() for _ in range(2)]
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            cs_in.wait_stream(torch.cuda.current_stream())
+            t0.record(cs_in)
+            for i in range(n):
+                j = i % 2
+                dq, dk, dv, dz, da, db = ins[j]
+                if i >= 2:
+                    cs_in.wait_event(done[j])           # step i - 2 has consumed this input set
+                with torch.cuda.stream(cs_in):
+                    for dst, src in ((dq, hq), (dk, hk), (dv, hv), (dz, hz), (da, ha), (db, hb)):
+                        dst.copy_(src, non_blocking=True)
+                    ready[j].record(cs_in)
+                side.wait_event(ready[j])
+                if i >= 2:
+                    side.wait_event(drained[j])         # step i - 2's output has reached the host
+                with torch.cuda.stream(side):
+                    g.gdn_prefill_chunked_gated_nvfp4(dq, dk, dv, da, db, A_log, dt_bias, dz, nw, gx, cu_seqlens=cu,
+                                                      initial_state=S0, final_state=S, xq=xq, xs=xs, workspace=ws)
+                    g.nvfp4_gemm(xq, xs, wq, ws_w, alpha, y=outs[j])
+                    done[j].record(side)
+                cs_out.wait_event(done[j])
+                with torch.cuda.stream(cs_out):
+                    hY[j].copy_(outs[j], non_blocking=True)
+                    drained[j].record(cs_out)
+            t1.record(cs_out)
+            t1.synchronize()
+            torch.cuda.current_stream().wait_stream(cs_out)
+            return t0.elapsed_time(t1) / n
+        res["e2e_run"] = e2e_run
     res["keep"] = (q, k, v, z, a, b, A_log, dt_bias, nw, cu, S0, wq, ws_w, S, xq, xs, Y, ws)
     return res
 
@@ -353,26 +389,16 @@ def run_gpu(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_max = float(t.item())
     assert g.gdn_get_device_status() == 0
-    e2e_step = main["e2e_step"]
-    for _ in range(args.warmup):
-        e2e_step()
+    e2e_run = main["e2e_run"]
+    e2e_run(args.warmup)
     torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(args.steps):
-        flush()
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        e2e_step()
-        s1.record(stream)
-        s1.synchronize()
-        e2e_ms.append(s0.elapsed_time(s1))
-    e2e = statistics.mean(e2e_ms)
+    e2e = e2e_run(args.steps)
     if world > 1:
         t = torch.tensor([e2e], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e = float(t.item())
     h2d, d2h, x_main = main["h2d"], main["d2h"], main["x"]
-    del main, graphs, e2e_step
+    del main, graphs, e2e_run
     torch.cuda.empty_cache()
 
     # the 1024-wide layer's prefill (T = 4096, 16/16 heads) and the variable-length batch
@@ -561,7 +587,11 @@ def run_gpu(args):
                          ROOT, "gated_deltanet_03_b200", "csrc", "chunked.cu"))),
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over the call's four kernels"},
         "e2e": {"value": tokens / (e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e,
+                "how": "every step copies its inputs in from pinned host memory and its output back; "
+                       "copies in, compute and copies out of consecutive steps on three streams "
+                       "(double-buffered inputs and outputs), timed from the first copy in to the last "
+                       "copy out; inputs larger than L2"},
         "decode": {"workload": dw.name, "ms": dec, "GB/s": dec_bytes / (dec / 1e3) / 1e9,
                    "frac": dec_bytes / (dec / 1e3) / 1e9 / float(pk["hbm_gbs"]),
                    "bytes": dec_bytes, "peak_gbs": float(pk["hbm_gbs"]), "peak_kind": pk_kind,

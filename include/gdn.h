@@ -72,9 +72,10 @@ typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
  * q, k        [T, Hk, Dk] in `in_dtype`;  v [T, Hv, Dv] in `in_dtype`
  * a, b        [T, Hv] fp32 gate pre-activations; A_log, dt_bias [Hv] fp32
  * cu_seqlens  device int32 [num_seqs + 1], cumulative token offsets of the packed
- *             sequences (cu_seqlens[0] = 0, cu_seqlens[num_seqs] = T); NULL means one
- *             sequence of T tokens (then num_seqs must be 1). Every sequence starts from
- *             its own initial state.
+ *             sequences (cu_seqlens[0] = 0, non-decreasing, cu_seqlens[num_seqs] = T); NULL
+ *             means one sequence of T tokens (then num_seqs must be 1). Every sequence starts
+ *             from its own initial state. The array lives in device memory and is not checked:
+ *             entries outside that contract are undefined behaviour.
  * scale       multiplies q after normalisation (1.0 = the formula as written)
  * qk_l2norm   non-zero: q and k are L2-normalised per head inside the path,
  *             x * (sum x^2 + 1e-6)^-1/2, before use (the delta rule wants unit keys)
