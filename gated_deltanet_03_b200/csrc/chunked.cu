@@ -28,9 +28,9 @@
 // Every MMA has M = 128 (value or key index on the TMEM lanes):
 //   prep   MMA1  D1 = [K; Q] [K; Q]^T      on the raw bf16 tiles (rows 0-63: K K^T | K Q^T,
 //                                          rows 64-127: Q K^T | Q Q^T; the diagonals give the norms)
-//          MMA2  D2 = [T'; T''] [K | V]    bf16, hi then lo A parts; rows 0-63: W = T' K, rows
-//                                          64-127: U~ = T'' V; T' = T diag(beta gamma / |k|),
-//                                          T'' = T diag(beta)
+//          MMA2a D2 = [T'; T''] K          bf16, hi then lo A parts; rows 0-63: W = T' K
+//          MMA2b D2 = [T'; T''] V          then, over the same columns, rows 64-127: U~ = T'' V;
+//                                          T' = T diag(beta gamma / |k|), T'' = T diag(beta)
 //   chain  MMA45 [D4 | D5a] = S0 [W; Q']^T      fp16; Q' = diag(gamma scale / |q|) Q
 //          MMA7  D7 = (U diag(c))^T K           bf16 hi / lo A, raw bf16 K
 //          MMA5b D5a += U^T P^T                 bf16 hi / lo, P^T[s][r] = k_s.q_r Gamma_rs scale / (|q_r| |k_s|)

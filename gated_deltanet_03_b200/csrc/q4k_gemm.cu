@@ -8,9 +8,10 @@
 // tcgen05 kind::f16 (bf16 A and B, fp32 accumulation in tensor memory), CTA tile 128 x 128, 64
 // values of K per stage, a 3-stage ring, two CTAs per SM. Warp 0: TMA of the activation tile;
 // warp 1: tensor memory and the MMA issue (one thread); warps 4-7: one output column (weight row)
-// per thread - per stage it reads the row's 32 quant bytes for the stage (and the block header
-// once per block), decodes 64 weights in fp32, rounds them to bf16 and writes them into the
-// stage's K-major 128-byte-swizzled B tile; at the end the same warps read the accumulator (one
+// per thread - per stage it reads the row's 32 quant bytes for the stage and its block header
+// (one stage ahead of their use), decodes the 64 weights two at a time in bf16 arithmetic (the
+// sub-block factors d scale and dmin min rounded to bf16, one bf16x2 FMA per pair) and writes them
+// into the stage's K-major 128-byte-swizzled B tile; at the end the same warps read the accumulator (one
 // lane quarter each) and store y. The weights are decoded once per output tile; the 4.5 MB
 // weight of the 4096 -> 2048 projection stays in L2 across the M tiles.
 //
@@ -80,8 +81,6 @@ __device__ __forceinline__ void q4k_scale_min(const uint8_t (&sc)[12], int j, in
     }
 }
 
-// fp32 of a 4-bit value: 2^23 + q as a float, minus 2^23 (exact).
-__device__ __forceinline__ float nib_f(uint32_t q) { return __uint_as_float(0x4B000000u | q) - 8388608.0f; }
 
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(QK_THREADS, 2)
@@ -170,18 +169,26 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
         const uint8_t *wrow = w + (size_t)n * nb * QK_BLOCK_BYTES;
         bool ok = true;
         float ds[2] = {0.f, 0.f}, dm[2] = {0.f, 0.f};
+        // the quant bytes of a stage's 64 values (sub-blocks 2 g and 2 g + 1) and its block's
+        // header, loaded one stage ahead of their decode so that the L2 round trip overlaps it
+        auto load_stage = [&](int i, uint4 &q0, uint4 &q1, uint4 &hd) {
+            const int kt = kt0 + i, g = kt & 3;
+            const uint8_t *blk = wrow + (size_t)(kt >> 2) * QK_BLOCK_BYTES;
+            q0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * g);
+            q1 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * g + 16);
+            hd = *reinterpret_cast<const uint4 *>(blk);
+        };
+        uint4 nq0 = make_uint4(0u, 0u, 0u, 0u), nq1 = nq0, nhd = nq0;
+        if (num_k > 0) load_stage(0, nq0, nq1, nhd);
         for (int i = 0; i < num_k && ok; ++i) {
             const int kt = kt0 + i;
             const int s = i % QK_STAGES, g = kt & 3;
-            const uint8_t *blk = wrow + (size_t)(kt >> 2) * QK_BLOCK_BYTES;
-            // the quant bytes of this stage's 64 values (sub-blocks 2 g and 2 g + 1) and, at a block's
-            // first stage, the block header, before the wait for the stage to be free
-            const uint4 q0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * g);
-            const uint4 q1 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * g + 16);
+            const uint4 q0 = nq0, q1 = nq1;
             uint8_t sc[12];
             float d = 0.f, dmin = 0.f;
             {
-                const uint4 hd = *reinterpret_cast<const uint4 *>(blk);
+                const uint4 hd = nhd;
+                if (i + 1 < num_k) load_stage(i + 1, nq0, nq1, nhd);
                 d = __half2float(__ushort_as_half((unsigned short)(hd.x & 0xFFFFu)));
                 dmin = __half2float(__ushort_as_half((unsigned short)(hd.x >> 16)));
                 const uint32_t words[3] = {hd.y, hd.z, hd.w};
@@ -198,22 +205,28 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
             if (lane == 0) ok = mbar_wait(&empty[s], (uint32_t)(((i / QK_STAGES) & 1) ^ 1), status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            // values 0-31 of the stage: low nibbles (sub-block 2 g); 32-63: high nibbles (2 g + 1)
+            // values 0-31 of the stage: low nibbles (sub-block 2 g); 32-63: high nibbles (2 g + 1).
+            // Two quants at a time as bf16 pairs: a byte permute puts the nibbles of two adjacent
+            // bytes into the two 16-bit halves, OR-ing in the exponent of 128 makes them the bf16
+            // values 128 + q (exact, 7 mantissa bits), a bf16x2 subtraction gives q exactly, and one
+            // bf16x2 FMA gives d scale q - dmin min (d scale and dmin min rounded to bf16 first)
             const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
             uint8_t *brow = tile_b(s);
+            const __nv_bfloat162 c128 = __floats2bfloat162_rn(128.0f, 128.0f);
+            const __nv_bfloat162 ds2[2] = {__floats2bfloat162_rn(ds[0], ds[0]), __floats2bfloat162_rn(ds[1], ds[1])};
+            const __nv_bfloat162 nd2[2] = {__floats2bfloat162_rn(-dm[0], -dm[0]), __floats2bfloat162_rn(-dm[1], -dm[1])};
 #pragma unroll
             for (int c = 0; c < 8; ++c) {   // 16-byte chunk c: values 8 c .. 8 c + 7
                 const int h2 = c >> 2, sh = h2 ? 4 : 0;
-                const uint32_t wa = qw[(c & 3) * 2], wb = qw[(c & 3) * 2 + 1];
+                const uint32_t wa = qw[(c & 3) * 2] >> sh, wb = qw[(c & 3) * 2 + 1] >> sh;
                 uint32_t packed[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const uint32_t src = e < 2 ? wa : wb;
-                    const int byte0 = (e & 1) * 2;
-                    const float x0 = fmaf(nib_f((src >> (8 * byte0 + sh)) & 15u), ds[h2], -dm[h2]);
-                    const float x1 = fmaf(nib_f((src >> (8 * byte0 + 8 + sh)) & 15u), ds[h2], -dm[h2]);
-                    const __nv_bfloat162 bb = __floats2bfloat162_rn(x0, x1);
-                    packed[e] = *reinterpret_cast<const uint32_t *>(&bb);
+                    const uint32_t xb = (__byte_perm(src, 0u, (e & 1) ? 0x4342u : 0x4140u) & 0x000F000Fu) | 0x43004300u;
+                    const __nv_bfloat162 q2 = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&xb), c128);
+                    const __nv_bfloat162 w2 = __hfma2(q2, ds2[h2], nd2[h2]);
+                    packed[e] = *reinterpret_cast<const uint32_t *>(&w2);
                 }
                 *reinterpret_cast<uint4 *>(brow + qk_swz(rl, c)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
             }
