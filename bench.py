@@ -54,7 +54,7 @@ FP4_PROBE_TFLOPS = 2.0 * 16368 * 148 * 1.965e9 / 1e12
 # DRAM bytes of one fused prefill call (prep + lean + combine + the output pass with the gated
 # tail) on the long-prefill workload, from one ncu capture with cold caches, keyed by the digest
 # of the scan's source (null in the line once the source has changed)
-SCAN_TRAFFIC = {"868b6fff038ffaa5": 4581.67e6}
+SCAN_TRAFFIC = {"09b71335661839bc": 4580.83e6}
 
 
 def source_digest(path: str) -> str:

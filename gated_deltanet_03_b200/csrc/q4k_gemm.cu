@@ -169,14 +169,16 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
         const uint8_t *wrow = w + (size_t)n * nb * QK_BLOCK_BYTES;
         bool ok = true;
         float ds[2] = {0.f, 0.f}, dm[2] = {0.f, 0.f};
-        // the quant bytes of a stage's 64 values (sub-blocks 2 g and 2 g + 1) and its block's
-        // header, loaded one stage ahead of their decode so that the L2 round trip overlaps it
+        // the quant bytes of a stage's 64 values (sub-blocks 2 g and 2 g + 1), loaded one stage
+        // ahead of their decode so that the L2 round trip overlaps it; the block's 16-byte header
+        // only at the first stage of a block (or of this CTA's range) - each lane reads its own
+        // row, so every 16-byte load is a separate L1 wavefront
         auto load_stage = [&](int i, uint4 &q0, uint4 &q1, uint4 &hd) {
             const int kt = kt0 + i, g = kt & 3;
             const uint8_t *blk = wrow + (size_t)(kt >> 2) * QK_BLOCK_BYTES;
             q0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * g);
             q1 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * g + 16);
-            hd = *reinterpret_cast<const uint4 *>(blk);
+            if (g == 0 || i == 0) hd = *reinterpret_cast<const uint4 *>(blk);
         };
         uint4 nq0 = make_uint4(0u, 0u, 0u, 0u), nq1 = nq0, nhd = nq0;
         if (num_k > 0) load_stage(0, nq0, nq1, nhd);

@@ -79,6 +79,18 @@ def test_workspace_query_is_host_only():
     assert g.gdn_prefill_workspace_bytes(4096, 1, 16, 16, 128, 128) >= 0
 
 
+@pytest.mark.parametrize("T,Hk,Hv,seg", [(32768, 16, 32, 57), (16384, 16, 32, 29), (4096, 16, 16, 8)])
+def test_workspace_follows_the_segment_plan(T, Hk, Hv, seg):
+    """The workspace holds one 82,944-byte item per (value head, chunk slot) and one
+    196,608-byte segment item per (value head, segment slot), T / (64 L) + num_seqs slots for a
+    segment length of L chunks. The host plans L from its cost model: 57 chunks at T = 32768 with
+    32 value heads (288 output-pass CTAs, two whole waves on 148 SMs), 29 at T = 16384, 8 at
+    T = 4096 with 16 heads."""
+    import gated_deltanet_03_b200 as g
+    expect = Hv * (T // 64 + 1) * 82944 + Hv * (T // (64 * seg) + 1) * 196608
+    assert g.gdn_prefill_workspace_bytes(T, 1, Hk, Hv, 128, 128) == expect
+
+
 def test_short_conv_host_validation():
     """Every case is rejected (or is a no-op) on the host, so nothing is launched; the fake
     addresses are never dereferenced."""
