@@ -156,7 +156,7 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            float scale, int32_t qk_l2norm, gdn_dtype in_dtype,
                            float *state, void *o, gdn_dtype out_dtype, gdn_stream_t stream);
 
-/* gdn_decode_step fused with the gated tail and the NVFP4 encode (the survey's fused decode):
+/* gdn_decode_step fused with the gated tail and the NVFP4 encode:
  * [GDN] recurrence for one token per sequence, then [TAIL] steps 1-5 on each head's o and the
  * 16-value NVFP4 block encode ([GDN] mechanism i) in the same kernel, so o never goes through
  * HBM. Dk = Dv = 128, bf16 inputs. state [B, Hv, 128, 128] fp32 updated in place; z [B, Hv, 128]
