@@ -5,14 +5,19 @@
 // w = d * scale * q - dmin * min; bit positions of the GGUF K-quant layout, which the page calls
 // canonical).
 //
-// tcgen05 kind::f16 (bf16 A and B, fp32 accumulation in tensor memory), CTA tile 128 x 128, 64
-// values of K per stage, a 3-stage ring, two CTAs per SM. Warp 0: TMA of the activation tile;
-// warp 1: tensor memory and the MMA issue (one thread); warps 4-7: one output column (weight row)
-// per thread - per stage it reads the row's 32 quant bytes for the stage and its block header
-// (one stage ahead of their use), decodes the 64 weights two at a time in bf16 arithmetic (the
-// sub-block factors d scale and dmin min rounded to bf16, one bf16x2 FMA per pair) and writes them
-// into the stage's K-major 128-byte-swizzled B tile; at the end the same warps read the accumulator (one
-// lane quarter each) and store y. The weights are decoded once per output tile; the 4.5 MB
+// tcgen05 kind::f16 (bf16 A and B, fp32 accumulation in tensor memory), CTA tile 128 x BN, 64
+// values of K per stage, two CTAs per SM: BN = 128 with a 3-stage ring (small and medium M, and
+// the split-K form below), BN = 256 with a 2-stage ring for large M (each stage's MMA work doubles
+// while its shared-memory traffic - the activation tile written by TMA and read by the MMA, the
+// weight tile written by the decode warps and read by the MMA - grows by half, and that traffic is
+// what bounds the kernel). Warp 0: TMA of the activation tile; warp 1: tensor memory and the MMA
+// issue (one thread); warps 4 .. 4 + BN/32 - 1: one output column (weight row) per thread - per
+// stage it reads the row's 32 quant bytes for the stage (and the block header at a block's first
+// stage), one stage ahead of their use, decodes the 64 weights two at a time in bf16 arithmetic
+// (the sub-block factors d scale and dmin min rounded to bf16, one bf16x2 FMA per pair) and writes
+// them into the stage's K-major 128-byte-swizzled B tile; at the end the same warps read the
+// accumulator (one lane quarter and 128 columns each) and store y. The weights are decoded once
+// per output tile; the 4.5 MB
 // weight of the 4096 -> 2048 projection stays in L2 across the M tiles.
 //
 // Split K for small M (the decode shapes, where the output tiles alone would leave most SMs
@@ -28,18 +33,27 @@
 namespace gdn {
 namespace {
 
-constexpr int QK_BM = 128, QK_BN = 128, QK_BK = 64;
-constexpr int QK_STAGES = 3;
-constexpr int QK_TILE = QK_BM * QK_BK * 2;                  // 16 KB (A and B tiles alike)
-constexpr int QK_STAGE_BYTES = 2 * QK_TILE;
-constexpr int QK_OFF_BAR = QK_STAGES * QK_STAGE_BYTES;
-constexpr int QK_SMEM = QK_OFF_BAR + 128 + 1024;
-constexpr int QK_THREADS = 256;
+constexpr int QK_BM = 128, QK_BK = 64;
+constexpr int QK_TILE_A = QK_BM * QK_BK * 2;                // 16 KB activation tile per stage
 constexpr int QK_BLOCK_BYTES = 144;
-constexpr int QK_PART_PITCH = QK_BN + 4;                   // fp32 row pitch of a partial tile (conflict-free rows)
 constexpr int QK_MAX_SPLIT = 8;
-static_assert(2 * (QK_SMEM + 1024) <= 233472, "two Q4_K GEMM CTAs per SM");
-static_assert(QK_BM * QK_PART_PITCH * 4 <= QK_OFF_BAR, "a partial tile fits over the stage ring");
+// Two tile widths: N = 128 (three stages, the split-K form for small M) and N = 256 (two stages,
+// eight decode warps; half again as much MMA work per byte of shared-memory traffic, for large
+// M). Both keep two CTAs per SM.
+template <int BN>
+struct QkCfg {
+    static constexpr int STAGES = BN == 128 ? 3 : 2;
+    static constexpr int TILE_B = BN * QK_BK * 2;
+    static constexpr int STAGE_BYTES = QK_TILE_A + TILE_B;
+    static constexpr int PART_PITCH = BN + 4;                 // fp32 row pitch of a split-K partial tile
+    static constexpr int PART_BYTES = BN == 128 ? QK_BM * PART_PITCH * 4 : 0;
+    static constexpr int OFF_BAR = STAGES * STAGE_BYTES > PART_BYTES ? STAGES * STAGE_BYTES : PART_BYTES;
+    static constexpr int SMEM = OFF_BAR + 128 + 1024;
+    static constexpr int DEC_WARPS = BN / 32;                  // one weight row per decode thread
+    static constexpr int THREADS = 128 + BN;
+};
+static_assert(2 * (QkCfg<128>::SMEM + 1024) <= 233472 && 2 * (QkCfg<256>::SMEM + 1024) <= 233472,
+              "two Q4_K GEMM CTAs per SM");
 
 __device__ __forceinline__ uint32_t qk_cluster_rank() {
     uint32_t r;
@@ -82,22 +96,24 @@ __device__ __forceinline__ void q4k_scale_min(const uint8_t (&sc)[12], int j, in
 }
 
 
-template <bool OUT_BF16>
-__global__ void __launch_bounds__(QK_THREADS, 2)
+template <bool OUT_BF16, int BN>
+__global__ void __launch_bounds__(QkCfg<BN>::THREADS, 2)
 q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__restrict__ w, int M, int N, int K,
                 void *__restrict__ y, int split, int *status) {
+    using Cfg = QkCfg<BN>;
+    constexpr int QK_STAGES = Cfg::STAGES;
     pdl_launch_dependents();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + QK_OFF_BAR);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Cfg::OFF_BAR);
     uint64_t *a_full = bars, *b_full = bars + QK_STAGES, *empty = bars + 2 * QK_STAGES;
     uint64_t *acc_full = bars + 3 * QK_STAGES, *drain = bars + 3 * QK_STAGES + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * QK_STAGES + 2);
-    auto tile_a = [&](int s) { return sm + s * QK_STAGE_BYTES; };
-    auto tile_b = [&](int s) { return sm + s * QK_STAGE_BYTES + QK_TILE; };
+    auto tile_a = [&](int s) { return sm + s * Cfg::STAGE_BYTES; };
+    auto tile_b = [&](int s) { return sm + s * Cfg::STAGE_BYTES + QK_TILE_A; };
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int n0 = blockIdx.x * QK_BN, m0 = blockIdx.y * QK_BM;
+    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * QK_BM;
     const int nb = K / 256;
     // this CTA's K range (all of K without split): k-tiles [kt0, kt0 + num_k)
     const uint32_t crank = split > 1 ? qk_cluster_rank() : 0u;
@@ -106,7 +122,7 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
     if (tid == 0) {
         for (int s = 0; s < QK_STAGES; ++s) {
             mbar_init(&a_full[s], 1);
-            mbar_init(&b_full[s], 4);    // the four decoding warps
+            mbar_init(&b_full[s], Cfg::DEC_WARPS);
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
@@ -114,7 +130,7 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 128);
+        tmem_alloc(tmem_slot, BN);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -128,7 +144,7 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
             for (int i = 0; i < num_k; ++i) {
                 const int s = i % QK_STAGES;
                 if (!mbar_wait(&empty[s], (uint32_t)(((i / QK_STAGES) & 1) ^ 1), status)) break;
-                mbar_arrive_expect_tx(&a_full[s], QK_TILE);
+                mbar_arrive_expect_tx(&a_full[s], QK_TILE_A);
                 tma_load_2d(tile_a(s), &map_a, &a_full[s], (kt0 + i) * QK_BK, m0);
             }
             // before the CTA may exit: the last load armed on each stage has landed
@@ -139,8 +155,8 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // bf16 A and B, fp32 accumulation, both K-major, N = 128, M = 128
-            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(QK_BN >> 3) << 17) |
+            // bf16 A and B, fp32 accumulation, both K-major, N = BN, M = 128
+            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                    ((uint32_t)(QK_BM >> 4) << 24);
             int issued = 0;
             for (int i = 0; i < num_k; ++i) {
@@ -163,8 +179,9 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
             }
         }
     } else if (warp >= 4) {
-        const int quarter = warp - 4;
-        const int rl = quarter * 32 + lane;               // weight row within the tile
+        const int dw = warp - 4;                          // decode warp: weight rows 32 dw ..
+        const int quarter = dw & 3, col0 = (dw >> 2) * 128;   // its accumulator lanes and columns
+        const int rl = dw * 32 + lane;                    // weight row within the tile
         const int n = n0 + rl;
         const uint8_t *wrow = w + (size_t)n * nb * QK_BLOCK_BYTES;
         bool ok = true;
@@ -241,14 +258,14 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
             if (lane == 0) ok = mbar_wait(acc_full, 0, status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
         }
-        if (ok && split > 1) {
+        if (ok && BN == 128 && split > 1) {
             // the partial tile into this CTA's shared memory (the stage ring is idle: every load
             // was consumed by an MMA that has completed), row = tensor-memory lane
             tc_fence_after();
             const uint32_t lb = ((uint32_t)(quarter * 32)) << 16;
-            float *prow = reinterpret_cast<float *>(sm) + (size_t)(quarter * 32 + lane) * QK_PART_PITCH;
+            float *prow = reinterpret_cast<float *>(sm) + (size_t)(quarter * 32 + lane) * Cfg::PART_PITCH;
 #pragma unroll 1
-            for (int c32 = 0; c32 < QK_BN / 32; ++c32) {
+            for (int c32 = 0; c32 < 4; ++c32) {
                 uint32_t r[32];
                 tmem_ld32(tmem + lb + c32 * 32, r);
                 tmem_ld_wait();
@@ -263,13 +280,13 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
             const int m = m0 + quarter * 32 + lane;
             const uint32_t lb = ((uint32_t)(quarter * 32)) << 16;
 #pragma unroll 1
-            for (int c32 = 0; c32 < QK_BN / 32; ++c32) {
+            for (int c32 = 0; c32 < 4; ++c32) {   // this warp's 128 accumulator columns from col0
                 uint32_t r[32];
-                tmem_ld32(tmem + lb + c32 * 32, r);
+                tmem_ld32(tmem + lb + col0 + c32 * 32, r);
                 tmem_ld_wait();
                 if (m < M) {
                     if constexpr (OUT_BF16) {
-                        __nv_bfloat16 *yr = reinterpret_cast<__nv_bfloat16 *>(y) + (size_t)m * N + n0 + c32 * 32;
+                        __nv_bfloat16 *yr = reinterpret_cast<__nv_bfloat16 *>(y) + (size_t)m * N + n0 + col0 + c32 * 32;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             uint4 u;
@@ -280,7 +297,7 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
                             *reinterpret_cast<uint4 *>(yr + 8 * i) = u;
                         }
                     } else {
-                        float *yr = reinterpret_cast<float *>(y) + (size_t)m * N + n0 + c32 * 32;
+                        float *yr = reinterpret_cast<float *>(y) + (size_t)m * N + n0 + col0 + c32 * 32;
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             *reinterpret_cast<float4 *>(yr + 4 * i) =
@@ -291,14 +308,14 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
             }
         }
     }
-    if (split > 1) {
+    if (BN == 128 && split > 1) {
         // every CTA of the cluster reaches both barriers, on the failure path too (its partial is
         // then stale and the status word already says so)
         qk_cluster_sync();
         const int rows = QK_BM / split, r0 = (int)crank * rows;
-        for (int u = tid; u < rows * (QK_BN / 4); u += QK_THREADS) {
-            const int rr = r0 + u / (QK_BN / 4), c4 = u % (QK_BN / 4);
-            const float *src = reinterpret_cast<const float *>(sm) + (size_t)rr * QK_PART_PITCH + 4 * c4;
+        for (int u = tid; u < rows * (BN / 4); u += Cfg::THREADS) {
+            const int rr = r0 + u / (BN / 4), c4 = u % (BN / 4);
+            const float *src = reinterpret_cast<const float *>(sm) + (size_t)rr * Cfg::PART_PITCH + 4 * c4;
             float4 acc = qk_ld_cluster(src, 0);
             for (int z = 1; z < split; ++z) {
                 const float4 v = qk_ld_cluster(src, (uint32_t)z);
@@ -327,7 +344,7 @@ q4k_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const uint8_t *__rest
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 128);
+        tmem_dealloc(tmem, BN);
     }
 }
 
@@ -363,28 +380,37 @@ cudaError_t launch_q4k_gemm(const Q4kGemmArgs &g, cudaStream_t st) {
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    static PerDevice<int> sm_count;   // the shared-memory attribute is set per device alongside
+    static PerDevice<int> sm_count;   // the shared-memory attributes are set per device alongside
     int sms = 0;
     cudaError_t e = sm_count.get(
         [](int dev, int &r) {
-            cudaError_t x = cudaFuncSetAttribute(q4k_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, QK_SMEM);
+            cudaError_t x = cudaSuccess;
             if (x == cudaSuccess)
-                x = cudaFuncSetAttribute(q4k_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, QK_SMEM);
+                x = cudaFuncSetAttribute(q4k_gemm_kernel<true, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, QkCfg<128>::SMEM);
+            if (x == cudaSuccess)
+                x = cudaFuncSetAttribute(q4k_gemm_kernel<false, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, QkCfg<128>::SMEM);
+            if (x == cudaSuccess)
+                x = cudaFuncSetAttribute(q4k_gemm_kernel<true, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, QkCfg<256>::SMEM);
+            if (x == cudaSuccess)
+                x = cudaFuncSetAttribute(q4k_gemm_kernel<false, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, QkCfg<256>::SMEM);
             if (x == cudaSuccess) x = cudaDeviceGetAttribute(&r, cudaDevAttrMultiProcessorCount, dev);
             return x;
         },
         &sms);
     if (e != cudaSuccess) return e;
-    const int tiles = (g.N / QK_BN) * ((g.M + QK_BM - 1) / QK_BM);
+    const int mt = (g.M + QK_BM - 1) / QK_BM;
+    const int tiles = (g.N / 128) * mt;
     const int num_k = g.K / QK_BK;
     int split = 1;   // double while the CTAs still fit at two per SM and every range keeps a whole block
     while (split < QK_MAX_SPLIT && tiles * split * 2 <= 2 * sms && num_k % (2 * split) == 0 &&
            num_k / (2 * split) >= 256 / QK_BK)
         split *= 2;
+    // 256-wide tiles when K is not split and they still give every SM slot several tiles
+    const bool wide = split == 1 && g.N % 256 == 0 && (g.N / 256) * mt >= 4 * sms;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(g.N / QK_BN), (unsigned)((g.M + QK_BM - 1) / QK_BM), (unsigned)split);
-    cfg.blockDim = dim3(QK_THREADS);
-    cfg.dynamicSmemBytes = QK_SMEM;
+    cfg.gridDim = dim3((unsigned)(g.N / (wide ? 256 : 128)), (unsigned)mt, (unsigned)split);
+    cfg.blockDim = dim3(wide ? QkCfg<256>::THREADS : QkCfg<128>::THREADS);
+    cfg.dynamicSmemBytes = wide ? QkCfg<256>::SMEM : QkCfg<128>::SMEM;
     cfg.stream = st;
     cudaLaunchAttribute attrs[2];
     attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -395,9 +421,14 @@ cudaError_t launch_q4k_gemm(const Q4kGemmArgs &g, cudaStream_t st) {
     attrs[1].val.clusterDim.z = (unsigned)split;
     cfg.attrs = attrs;
     cfg.numAttrs = split > 1 ? 2 : 1;
+    if (wide) {
+        if (g.out_bf16)
+            return cudaLaunchKernelEx(&cfg, q4k_gemm_kernel<true, 256>, ma, g.w, g.M, g.N, g.K, g.y, split, g.status);
+        return cudaLaunchKernelEx(&cfg, q4k_gemm_kernel<false, 256>, ma, g.w, g.M, g.N, g.K, g.y, split, g.status);
+    }
     if (g.out_bf16)
-        return cudaLaunchKernelEx(&cfg, q4k_gemm_kernel<true>, ma, g.w, g.M, g.N, g.K, g.y, split, g.status);
-    return cudaLaunchKernelEx(&cfg, q4k_gemm_kernel<false>, ma, g.w, g.M, g.N, g.K, g.y, split, g.status);
+        return cudaLaunchKernelEx(&cfg, q4k_gemm_kernel<true, 128>, ma, g.w, g.M, g.N, g.K, g.y, split, g.status);
+    return cudaLaunchKernelEx(&cfg, q4k_gemm_kernel<false, 128>, ma, g.w, g.M, g.N, g.K, g.y, split, g.status);
 }
 
 }  // namespace gdn

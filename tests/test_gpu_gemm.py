@@ -117,14 +117,16 @@ def test_fused_modules_colscale(g, M):
     assert rel_err(y1[:, gate], ref[:, gate]) > 100 * TOL_GEMM
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 128, 256), (200, 256, 768), (130, 512, 1024), (256, 2048, 4096), (4096, 2048, 4096)])
+@pytest.mark.parametrize("M,N,K", [(1, 128, 256), (200, 256, 768), (130, 512, 1024), (256, 2048, 4096), (4096, 2048, 4096),
+                                   (10000, 2048, 4096)])
 def test_q4k_gemm_matches_oracle(g, M, N, K):
     """The Q4_K output projection ("Red Lite dev15d - DeltaNet gated tail + Q4_K output
     projection", Q4_K implementation) against the fp64 product with the oracle's exact decode of
     the same synthetic weights: within the GEMM tolerance (the kernel rounds each decoded weight
     to bf16), for ragged M, the batched-decode shape (M = 256, 4096 -> 2048) and a prefill-sized
     M; bf16 and fp32 outputs. The small-M shapes run split over K in clusters of 2 (200 x 256 x
-    768), 4 (130 x 512 x 1024) and 8 (256 x 2048 x 4096) CTAs; the others unsplit."""
+    768), 4 (130 x 512 x 1024) and 8 (256 x 2048 x 4096) CTAs; 4096 x 2048 x 4096 unsplit on
+    128-wide tiles, and the ragged 10000 x 2048 x 4096 on 256-wide tiles (the large-M form)."""
     w = workloads.q4k_weights(N, K, seed=M + N + K)
     a = workloads.activations(M, K, seed=M * 3 + 1, heavy_tail=False)
     rows = np.arange(M) if M <= 256 else np.unique(np.concatenate([np.arange(0, M, 37), [M - 1]]))
