@@ -649,7 +649,8 @@ def run_only(args):
     if args.only == "verify":
         return run_verify(args)
     names = {wl.name: wl for wl in workloads.WORKLOADS}
-    w = names[args.workload] if args.workload else (workloads.DECODE_B256 if args.only in ("decode", "conv_decode")
+    w = names[args.workload] if args.workload else (workloads.DECODE_B256 if args.only in ("decode", "decode_fused",
+                                                                                            "conv_decode")
                                                     else workloads.PREFILL_1K)
     x = workloads.generate(w)
 
@@ -691,6 +692,8 @@ def run_only(args):
         "gemm": lambda: g.nvfp4_gemm(xq, xs, wq, ws, 1.0, y=Y),
         "q4k": lambda: g.q4k_gemm(q4a, q4w, y=q4y),
         "decode": lambda: g.gdn_decode_step(q, k, v, a, b, A_log, dt_bias, S0, o=o),
+        "decode_fused": lambda: g.gdn_decode_step_gated_nvfp4(q, k, v, a, b, A_log, dt_bias, S0, z, nw, 1.0,
+                                                              xq=xq, xs=xs),
         "fused": lambda: g.gdn_prefill_chunked_gated_nvfp4(q, k, v, a, b, A_log, dt_bias, z, nw, 1.0, cu_seqlens=cu,
                                                            initial_state=S0, final_state=S, xq=xq, xs=xs),
     }[args.only]
@@ -880,7 +883,7 @@ def main():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     p.add_argument("--only", choices=["scan", "tail", "gemm", "gemm_long", "decode", "verify", "fused", "conv",
-                                      "conv_decode", "q4k"],
+                                      "conv_decode", "q4k", "decode_fused"],
                    help="time one kernel alone on its workload (for profiling); prints one JSON line")
     p.add_argument("--workload", default=None, help="workload name for --only scan (default: 1024-wide prefill)")
     args = p.parse_args()
