@@ -80,6 +80,36 @@ def test_prefill_varlen_ragged(g):
     np.testing.assert_array_equal(S[4], x["initial_state"][4])
 
 
+def _many_short_lengths(n, hi, seed):
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, hi + 1, size=n)
+    lens[::9] = 0          # every ninth sequence empty
+    lens[5::11] = 64       # some exactly one chunk
+    lens[7::13] = 1        # some a single token
+    return tuple(int(x) for x in lens)
+
+
+@pytest.mark.parametrize("seqlens", [
+    _many_short_lengths(120, 100, 31),
+    (2500,) + _many_short_lengths(40, 70, 32),
+    _many_short_lengths(20, 70, 33) + (1500, 0, 700),
+], ids=["120_short", "long_first_then_short", "short_then_long"])
+def test_prefill_varlen_many_sequences(g, seqlens):
+    """A packed batch of many sequences: most shorter than one 64-token chunk, empties and
+    single tokens among them, and one to two long sequences that the batch's segment plan
+    (sized from the mean length) cuts into several segments. Every sequence's chunk slots,
+    segment bounds and initial state are checked against the oracle's per-sequence scan."""
+    w = workloads.custom("m", seqlens, 2, 4, 128, io="bf16", s0_std=0.1, seed=len(seqlens))
+    x = workloads.generate(w)
+    o_ref, S_ref = _full_oracle(x)
+    o, S = _run_prefill(g, x, w, torch.float32)
+    assert rel_err(o, o_ref) <= TOL_SCAN, rel_err(o, o_ref)
+    assert rel_err(S, S_ref) <= TOL_SCAN, rel_err(S, S_ref)
+    for i, L in enumerate(seqlens):
+        if L == 0:
+            np.testing.assert_array_equal(S[i], x["initial_state"][i])
+
+
 _DEGENERATE = ["alpha1_beta1", "alpha1_beta0", "same_key_beta1", "same_key", "strong_decay",
                "keys_in_4_directions"]
 
