@@ -62,14 +62,6 @@ __device__ __forceinline__ void unpack8(uint4 u, f2_t (&x)[4]) {
     x[3] = bf16x2_to_f2(u.w);
 }
 
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
-    const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
-
 // Output planes: plane p holds channels [start_p, end_p) as a contiguous [rows, end_p - start_p]
 // block at offset rows * start_p.
 struct Planes {

@@ -166,6 +166,16 @@ GDN_DEV void load_cols16(const void *base, size_t row, int l8, f2_t (&x)[8]) {
     }
 }
 
+// The same 16 values of lane c from an fp32 row in shared memory.
+GDN_DEV void lds_cols16(const float *row, int l8, f2_t (&x)[8]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float4 f = *reinterpret_cast<const float4 *>(row + 32 * j + 4 * l8);
+        x[2 * j] = f2(f.x, f.y);
+        x[2 * j + 1] = f2(f.z, f.w);
+    }
+}
+
 GDN_DEV float dot16(const f2_t (&a)[8], const f2_t (&b)[8]) {
     f2_t acc = mul2(a[0], b[0]);
 #pragma unroll
@@ -302,6 +312,9 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
     const size_t sbase = ((size_t)n * Hv + h) * D * D;
     __shared__ float s_kk[kVerifyMaxT][kVerifyMaxT], s_kq[kVerifyMaxT][kVerifyMaxT];
     __shared__ float s_qq[kVerifyMaxT], s_alpha[kVerifyMaxT], s_beta[kVerifyMaxT];
+    // the T tokens' raw key (0) and query (1) rows as fp32, staged once for the Gram dots and the
+    // state products (every 8-lane group reads the same 16-byte pieces: broadcasts, no conflicts)
+    __shared__ __align__(16) float kq_s[2][kVerifyMaxT][D];
 
     f2_t s[4][8];
 #pragma unroll
@@ -312,6 +325,17 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
             s[p][2 * j] = f2(x.x, x.y);
             s[p][2 * j + 1] = f2(x.z, x.w);
         }
+
+    for (int e = tid; e < 2 * T * (D / 8); e += kR128Threads) {
+        const int which = e >= T * (D / 8) ? 1 : 0, rem = e - which * T * (D / 8);
+        const int t = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
+        float x[8];
+        load8<IN_BF16>(which ? q : k, ((size_t)(t0 + t) * Hk + hk) * D + c8, x);
+        float4 *dst = reinterpret_cast<float4 *>(&kq_s[which][t][c8]);
+        dst[0] = make_float4(x[0], x[1], x[2], x[3]);
+        dst[1] = make_float4(x[4], x[5], x[6], x[7]);
+    }
+    __syncthreads();
 
     // Gram dots of the tokens' raw keys and queries (k_s.k_t and k_s.q_t for s <= t, q_t.q_t),
     // one 8-lane group per dot, and the gates
@@ -328,8 +352,8 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
             ss = e - tt * (tt + 1) / 2;
         }
         f2_t x2[8], y2[8];
-        load_cols16<IN_BF16>(kind == 2 ? q : k, ((size_t)(t0 + (kind == 2 ? tt : ss)) * Hk + hk) * D, l8, x2);
-        load_cols16<IN_BF16>(kind == 0 ? k : q, ((size_t)(t0 + tt) * Hk + hk) * D, l8, y2);
+        lds_cols16(kq_s[kind == 2 ? 1 : 0][kind == 2 ? tt : ss], l8, x2);
+        lds_cols16(kq_s[kind == 0 ? 0 : 1][tt], l8, y2);
         float part = dot16(x2, y2);
         part += __shfl_xor_sync(kFull, part, 4);
         part += __shfl_xor_sync(kFull, part, 2);
@@ -363,8 +387,8 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
         xq[t] = 0.0f;
         if (t < T) {
             f2_t k2[8], q2[8];
-            load_cols16<IN_BF16>(k, ((size_t)(t0 + t) * Hk + hk) * D, l8, k2);
-            load_cols16<IN_BF16>(q, ((size_t)(t0 + t) * Hk + hk) * D, l8, q2);
+            lds_cols16(kq_s[0][t], l8, k2);
+            lds_cols16(kq_s[1][t], l8, q2);
             float pk[4], pq[4];
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
@@ -432,6 +456,14 @@ gdn_decode128_gated_nvfp4_kernel(const void *__restrict__ q, const void *__restr
     const int rbase = (tid >> 7) * 64 + ((tid & 127) >> 3);
     const int gbase = lane & ~7;
     __shared__ __align__(16) __nv_bfloat16 o_s[D];
+    // the tail's z row and norm weights, copied in asynchronously with the state loads so that
+    // neither their DRAM / L2 latency nor registers are spent after the update
+    __shared__ __align__(16) __nv_bfloat16 z_s[D];
+    __shared__ __align__(16) float w_s[D];
+    if (tid < D) cp_async4(w_s + tid, norm_w + tid);
+    else if (tid < D + D / 8)
+        cp_async16(z_s + (tid - D) * 8, reinterpret_cast<const __nv_bfloat16 *>(z) + ((size_t)n * Hv + h) * D + (tid - D) * 8);
+    cp_async_commit();
     const size_t sbase = ((size_t)n * Hv + h) * D * D;
 
     f2_t s[4][8];
@@ -443,12 +475,7 @@ gdn_decode128_gated_nvfp4_kernel(const void *__restrict__ q, const void *__restr
             s[p][2 * j] = f2(x.x, x.y);
             s[p][2 * j + 1] = f2(x.z, x.w);
         }
-    // the tail's z row (warp 0: 16 lanes x 8 values), fetched with the state so that its DRAM latency
-    // is not added after the update (the norm weights, shared by every CTA, come from L2 later)
     const int lr = lane & 15, col = lr * 8;
-    uint4 zu = make_uint4(0u, 0u, 0u, 0u);
-    if (tid < 32)
-        zu = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(z) + ((size_t)n * Hv + h) * D + col);
     float g_alpha = 0.0f, g_beta = 0.0f;
     if (lane == 0) {
         float g;
@@ -498,15 +525,16 @@ gdn_decode128_gated_nvfp4_kernel(const void *__restrict__ q, const void *__restr
         o_s[rbase + 16 * p] = ob;
         if (o) reinterpret_cast<__nv_bfloat16 *>(o)[((size_t)n * Hv + h) * D + rbase + 16 * p] = ob;
     }
+    cp_async_wait<0>();
     __syncthreads();
     if (tid < 32) {
         // the head row: 16 lanes x 8 values (lanes 16-31 repeat them, their results unused)
         const uint4 ou = *reinterpret_cast<const uint4 *>(o_s + col);
+        const uint4 zu = *reinterpret_cast<const uint4 *>(z_s + col);
         const f2_t o2[4] = {bf16x2_to_f2(ou.x), bf16x2_to_f2(ou.y), bf16x2_to_f2(ou.z), bf16x2_to_f2(ou.w)};
         const f2_t z2[4] = {bf16x2_to_f2(zu.x), bf16x2_to_f2(zu.y), bf16x2_to_f2(zu.z), bf16x2_to_f2(zu.w)};
-        f2_t w2[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) w2[c] = f2(norm_w[col + 2 * c], norm_w[col + 2 * c + 1]);
+        const float4 wa = *reinterpret_cast<const float4 *>(w_s + col), wb = *reinterpret_cast<const float4 *>(w_s + col + 4);
+        const f2_t w2[4] = {f2(wa.x, wa.y), f2(wa.z, wa.w), f2(wb.x, wb.y), f2(wb.z, wb.w)};
         f2_t y2[4];
         gated_row8<16>(o2, z2, w2, 1.0f / (float)D, eps, y2);
         uint32_t packed, sb;
