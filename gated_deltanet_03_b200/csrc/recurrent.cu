@@ -290,10 +290,34 @@ gdn_recurrent128_kernel(const void *__restrict__ q, const void *__restrict__ k, 
 //     o_t = S_t q^_t = gamma_t S0 q^_t + sum_{s<=t} c_{s,t} u_s (k^_s . q^_t),
 // so each state row needs only the 2 T products S0 k_t and S0 q_t (independent of one another,
 // no state update) and T x T scalars shared by the CTA (the Gram dots of the tokens' keys and
-// queries), instead of T dependent rank-one updates. At most 96 registers a thread (a few spill),
-// so that five CTAs share an SM: a CTA computes only after its whole state slice has landed, and
-// the fifth CTA keeps more state loads in flight meanwhile.
+// queries), instead of T dependent rank-one updates.
+//
+// The 2 T products are one small matrix product per CTA, [S0 rows] x [k_1..k_T | q_1..q_T], on
+// warp-level bf16 MMAs (m16n8k16, fp32 accumulation): each warp owns 16 state rows, the keys and
+// the queries are one 8-column tile each. S0 enters as bf16 hi + lo (hi = S0 rounded, lo = the
+// rounded remainder: the product misses S0 - hi - lo, at most 2^-17 of |S0| per element); bf16
+// keys and queries are exact in bf16, fp32 ones are split the same way and add the hi x lo term.
+// Within each 16-wide k-step a thread holds state columns 4c .. 4c + 3 (c = lane % 4) in the
+// places the MMA layout gives to columns 2c, 2c + 1, 2c + 8, 2c + 9; the key / query tiles use the
+// same column order, so the sums are those of the plain products.
 constexpr int kVerifyMaxT = 8;
+constexpr int kVerifyPairPitch = 72;   // bf16 pairs per staged row: 64 + 8, so B-fragment loads are conflict-free
+
+// D += A B on one m16n8k16 tile (bf16 inputs, fp32 accumulation)
+GDN_DEV void mma_bf16_m16n8k16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// (x, y) as a bf16 pair (x in the low half) and the pair of their rounded remainders
+GDN_DEV void split_bf16x2(float x, float y, uint32_t &hi, uint32_t &lo) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(x, y);
+    hi = *reinterpret_cast<const uint32_t *>(&p);
+    const f2_t w = bf16x2_to_f2(hi);
+    p = __floats2bfloat162_rn(x - f2lo(w), y - f2hi(w));
+    lo = *reinterpret_cast<const uint32_t *>(&p);
+}
 
 template <bool IN_BF16, bool OUT_BF16>
 __global__ void __launch_bounds__(kR128Threads, 5)
@@ -306,62 +330,75 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
     constexpr int D = 128;
     const int slice = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
     const int hk = h / (Hv / Hk);
-    const int tid = threadIdx.x, l8 = tid & 7, grp = tid >> 3;
-    const int rbase = slice * 64 + grp;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gq = lane >> 2, tig = lane & 3;         // MMA fragment row group, thread in group
+    const int r0 = slice * 64 + warp * 16 + gq;       // this thread's state rows r0 and r0 + 8
     const int t0 = n * T;
     const size_t sbase = ((size_t)n * Hv + h) * D * D;
     __shared__ float s_kk[kVerifyMaxT][kVerifyMaxT], s_kq[kVerifyMaxT][kVerifyMaxT];
     __shared__ float s_qq[kVerifyMaxT], s_alpha[kVerifyMaxT], s_beta[kVerifyMaxT];
-    // the T tokens' raw key (0) and query (1) rows as fp32, staged once for the Gram dots and the
-    // state products (every 8-lane group reads the same 16-byte pieces: broadcasts, no conflicts)
+    // the tokens' raw key (0) and query (1) rows: fp32 for the Gram dots, bf16 pairs (and for fp32
+    // inputs their remainders) for the MMA; rows of unused tokens are zero
     __shared__ __align__(16) float kq_s[2][kVerifyMaxT][D];
+    __shared__ __align__(16) uint32_t kq_hi[2][kVerifyMaxT][kVerifyPairPitch];
+    __shared__ __align__(16) uint32_t kq_lo[2][kVerifyMaxT][IN_BF16 ? 2 : kVerifyPairPitch];
 
-    f2_t s[4][8];
+    // state rows r0 and r0 + 8, columns 16 ks + 4 tig .. + 3 of each k-step ks (read once)
+    float4 sa[8], sb[8];
 #pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 x = __ldcs(reinterpret_cast<const float4 *>(S0 + sbase + (size_t)(rbase + 16 * p) * D + 32 * j + 4 * l8));
-            s[p][2 * j] = f2(x.x, x.y);
-            s[p][2 * j + 1] = f2(x.z, x.w);
-        }
+    for (int ks = 0; ks < 8; ++ks) {
+        sa[ks] = __ldcs(reinterpret_cast<const float4 *>(S0 + sbase + (size_t)r0 * D + 16 * ks + 4 * tig));
+        sb[ks] = __ldcs(reinterpret_cast<const float4 *>(S0 + sbase + (size_t)(r0 + 8) * D + 16 * ks + 4 * tig));
+    }
 
-    for (int e = tid; e < 2 * T * (D / 8); e += kR128Threads) {
-        const int which = e >= T * (D / 8) ? 1 : 0, rem = e - which * T * (D / 8);
+    // stage the keys and queries: 2 x 8 rows of 16 pieces of 8 values, two pieces a thread
+#pragma unroll
+    for (int e = tid; e < 2 * kVerifyMaxT * (D / 8); e += kR128Threads) {
+        const int which = e / (kVerifyMaxT * (D / 8)), rem = e % (kVerifyMaxT * (D / 8));
         const int t = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
-        float x[8];
-        load8<IN_BF16>(which ? q : k, ((size_t)(t0 + t) * Hk + hk) * D + c8, x);
+        float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+        if (t < T) load8<IN_BF16>(which ? q : k, ((size_t)(t0 + t) * Hk + hk) * D + c8, x);
         float4 *dst = reinterpret_cast<float4 *>(&kq_s[which][t][c8]);
         dst[0] = make_float4(x[0], x[1], x[2], x[3]);
         dst[1] = make_float4(x[4], x[5], x[6], x[7]);
+        uint4 hi, lo;
+        split_bf16x2(x[0], x[1], hi.x, lo.x);
+        split_bf16x2(x[2], x[3], hi.y, lo.y);
+        split_bf16x2(x[4], x[5], hi.z, lo.z);
+        split_bf16x2(x[6], x[7], hi.w, lo.w);
+        *reinterpret_cast<uint4 *>(&kq_hi[which][t][c8 / 2]) = hi;
+        if constexpr (!IN_BF16) *reinterpret_cast<uint4 *>(&kq_lo[which][t][c8 / 2]) = lo;
     }
     __syncthreads();
 
     // Gram dots of the tokens' raw keys and queries (k_s.k_t and k_s.q_t for s <= t, q_t.q_t),
     // one 8-lane group per dot, and the gates
-    const int nkk = T * (T + 1) / 2, ndots = 2 * nkk + T;
-    // every lane runs the same number of rounds (the shuffles below take whole warps)
-    for (int base = 0; base < ndots; base += kR128Threads / 8) {
-        const bool live = base + grp < ndots;
-        const int d = live ? base + grp : 0;
-        int kind = d < nkk ? 0 : (d < 2 * nkk ? 1 : 2), e = kind == 0 ? d : (kind == 1 ? d - nkk : d - 2 * nkk);
-        int ss = 0, tt = e;
-        if (kind < 2) {   // e -> (s, t), s <= t, row-major over t
-            tt = 0;
-            while ((tt + 1) * (tt + 2) / 2 <= e) ++tt;
-            ss = e - tt * (tt + 1) / 2;
-        }
-        f2_t x2[8], y2[8];
-        lds_cols16(kq_s[kind == 2 ? 1 : 0][kind == 2 ? tt : ss], l8, x2);
-        lds_cols16(kq_s[kind == 0 ? 0 : 1][tt], l8, y2);
-        float part = dot16(x2, y2);
-        part += __shfl_xor_sync(kFull, part, 4);
-        part += __shfl_xor_sync(kFull, part, 2);
-        part += __shfl_xor_sync(kFull, part, 1);
-        if (live && l8 == 0) {
-            if (kind == 0) s_kk[ss][tt] = part;
-            else if (kind == 1) s_kq[ss][tt] = part;
-            else s_qq[tt] = part;
+    {
+        const int l8 = tid & 7, grp = tid >> 3;
+        const int nkk = T * (T + 1) / 2, ndots = 2 * nkk + T;
+        // every lane runs the same number of rounds (the shuffles below take whole warps)
+        for (int base = 0; base < ndots; base += kR128Threads / 8) {
+            const bool live = base + grp < ndots;
+            const int d = live ? base + grp : 0;
+            int kind = d < nkk ? 0 : (d < 2 * nkk ? 1 : 2), e = kind == 0 ? d : (kind == 1 ? d - nkk : d - 2 * nkk);
+            int ss = 0, tt = e;
+            if (kind < 2) {   // e -> (s, t), s <= t, row-major over t
+                tt = 0;
+                while ((tt + 1) * (tt + 2) / 2 <= e) ++tt;
+                ss = e - tt * (tt + 1) / 2;
+            }
+            f2_t x2[8], y2[8];
+            lds_cols16(kq_s[kind == 2 ? 1 : 0][kind == 2 ? tt : ss], l8, x2);
+            lds_cols16(kq_s[kind == 0 ? 0 : 1][tt], l8, y2);
+            float part = dot16(x2, y2);
+            part += __shfl_xor_sync(kFull, part, 4);
+            part += __shfl_xor_sync(kFull, part, 2);
+            part += __shfl_xor_sync(kFull, part, 1);
+            if (live && l8 == 0) {
+                if (kind == 0) s_kk[ss][tt] = part;
+                else if (kind == 1) s_kq[ss][tt] = part;
+                else s_qq[tt] = part;
+            }
         }
     }
     if (tid < T) {
@@ -371,37 +408,56 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
         s_beta[tid] = beta;
     }
 
-    // the row this lane finishes (below) and its v values, loaded ahead of the dependent recurrence
-    const int prow = 2 * ((l8 >> 2) & 1) + ((l8 >> 1) & 1);
-    const int row = rbase + 16 * prow;
+    // the row this lane finishes (below: lanes 0, 1 of a group row r0, lanes 2, 3 row r0 + 8) and
+    // its v values, loaded ahead of the dependent recurrence
+    const int rsel = tig >> 1;
+    const int row = r0 + 8 * rsel;
     float vrow[kVerifyMaxT];
 #pragma unroll
     for (int t = 0; t < kVerifyMaxT; ++t)
         vrow[t] = t < T ? load1<IN_BF16>(v, ((size_t)(t0 + t) * Hv + h) * D + row) : 0.0f;
-    // S0 k_t and S0 q_t for this thread's four rows, reduced over the row's eight lanes: lanes
-    // whose bits 2 and 1 are (p >> 1, p & 1) hold row p's totals
+
+    // [S0 k_1 .. S0 k_8] and [S0 q_1 .. S0 q_8] for the warp's 16 rows: the D fragments hold
+    // (row r0, tokens 2 tig, 2 tig + 1) in [0], [1] and (row r0 + 8, the same tokens) in [2], [3]
+    float dk[4] = {0.0f, 0.0f, 0.0f, 0.0f}, dq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        uint32_t ahi[4], alo[4];
+        split_bf16x2(sa[ks].x, sa[ks].y, ahi[0], alo[0]);
+        split_bf16x2(sb[ks].x, sb[ks].y, ahi[1], alo[1]);
+        split_bf16x2(sa[ks].z, sa[ks].w, ahi[2], alo[2]);
+        split_bf16x2(sb[ks].z, sb[ks].w, ahi[3], alo[3]);
+        const int pc = 8 * ks + 2 * tig;
+        const uint2 bk = *reinterpret_cast<const uint2 *>(&kq_hi[0][gq][pc]);
+        const uint2 bq = *reinterpret_cast<const uint2 *>(&kq_hi[1][gq][pc]);
+        mma_bf16_m16n8k16(dk, ahi, bk.x, bk.y);
+        mma_bf16_m16n8k16(dk, alo, bk.x, bk.y);
+        mma_bf16_m16n8k16(dq, ahi, bq.x, bq.y);
+        mma_bf16_m16n8k16(dq, alo, bq.x, bq.y);
+        if constexpr (!IN_BF16) {
+            const uint2 lk = *reinterpret_cast<const uint2 *>(&kq_lo[0][gq][pc]);
+            const uint2 lq = *reinterpret_cast<const uint2 *>(&kq_lo[1][gq][pc]);
+            mma_bf16_m16n8k16(dk, ahi, lk.x, lk.y);
+            mma_bf16_m16n8k16(dq, ahi, lq.x, lq.y);
+        }
+    }
+    // this lane's row: token t's products sit in lane (group, t / 2), element t % 2 (+ 2 for r0 + 8)
     float xk[kVerifyMaxT], xq[kVerifyMaxT];
 #pragma unroll
     for (int t = 0; t < kVerifyMaxT; ++t) {
         xk[t] = 0.0f;
         xq[t] = 0.0f;
         if (t < T) {
-            f2_t k2[8], q2[8];
-            lds_cols16(kq_s[0][t], l8, k2);
-            lds_cols16(kq_s[1][t], l8, q2);
-            float pk[4], pq[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                pk[p] = dot16(s[p], k2);
-                pq[p] = dot16(s[p], q2);
-            }
-            xk[t] = group8_sum4_t(pk, l8);
-            xq[t] = group8_sum4_t(pq, l8);
+            const int src = (lane & ~3) | (t >> 1);
+            const float k0 = __shfl_sync(kFull, dk[t & 1], src), k1 = __shfl_sync(kFull, dk[2 + (t & 1)], src);
+            const float q0 = __shfl_sync(kFull, dq[t & 1], src), q1 = __shfl_sync(kFull, dq[2 + (t & 1)], src);
+            xk[t] = rsel ? k1 : k0;
+            xq[t] = rsel ? q1 : q0;
         }
     }
     __syncthreads();
 
-    // per row: the T x T recurrence on the projections (lanes with l8 even own one row each)
+    // per row: the T x T recurrence on the projections (lanes with tig even own one row each)
     float kn[kVerifyMaxT], u[kVerifyMaxT], c[kVerifyMaxT];
 #pragma unroll
     for (int t = 0; t < kVerifyMaxT; ++t) {
@@ -428,7 +484,7 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
 #pragma unroll
         for (int r = 0; r < kVerifyMaxT; ++r)
             if (r <= t) ot += c[r] * u[r] * (kn[r] * qn * s_kq[r][t]);
-        if ((l8 & 1) == 0) store1<OUT_BF16>(o, ((size_t)(t0 + t) * Hv + h) * D + row, ot);
+        if ((tig & 1) == 0) store1<OUT_BF16>(o, ((size_t)(t0 + t) * Hv + h) * D + row, ot);
     }
 }
 
