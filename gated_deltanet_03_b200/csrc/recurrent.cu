@@ -166,16 +166,6 @@ GDN_DEV void load_cols16(const void *base, size_t row, int l8, f2_t (&x)[8]) {
     }
 }
 
-// The same 16 values of lane c from an fp32 row in shared memory.
-GDN_DEV void lds_cols16(const float *row, int l8, f2_t (&x)[8]) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float4 f = *reinterpret_cast<const float4 *>(row + 32 * j + 4 * l8);
-        x[2 * j] = f2(f.x, f.y);
-        x[2 * j + 1] = f2(f.z, f.w);
-    }
-}
-
 GDN_DEV float dot16(const f2_t (&a)[8], const f2_t (&b)[8]) {
     f2_t acc = mul2(a[0], b[0]);
 #pragma unroll
@@ -337,12 +327,17 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
     const size_t sbase = ((size_t)n * Hv + h) * D * D;
     __shared__ float s_kk[kVerifyMaxT][kVerifyMaxT], s_kq[kVerifyMaxT][kVerifyMaxT];
     __shared__ float s_qq[kVerifyMaxT], s_alpha[kVerifyMaxT], s_beta[kVerifyMaxT];
-    // the tokens' raw key (0) and query (1) rows: fp32 for the Gram dots, bf16 pairs (and for fp32
-    // inputs their remainders) for the MMA; rows of unused tokens are zero
-    __shared__ __align__(16) float kq_s[2][kVerifyMaxT][D];
+    // the tokens' raw key (0) and query (1) rows as bf16 pairs (and for fp32 inputs the pairs of
+    // their rounded remainders), the MMAs' operands; rows of unused tokens are zero
     __shared__ __align__(16) uint32_t kq_hi[2][kVerifyMaxT][kVerifyPairPitch];
     __shared__ __align__(16) uint32_t kq_lo[2][kVerifyMaxT][IN_BF16 ? 2 : kVerifyPairPitch];
 
+    // the gate inputs of token `lane` (warp 2), fetched before the state
+    float ga_raw = 0.0f, gb_raw = 0.0f;
+    if (warp == 2 && lane < T) {
+        ga_raw = a[(size_t)(t0 + lane) * Hv + h];
+        gb_raw = b[(size_t)(t0 + lane) * Hv + h];
+    }
     // state rows r0 and r0 + 8, columns 16 ks + 4 tig .. + 3 of each k-step ks (read once)
     float4 sa[8], sb[8];
 #pragma unroll
@@ -358,9 +353,6 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
         const int t = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
         float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
         if (t < T) load8<IN_BF16>(which ? q : k, ((size_t)(t0 + t) * Hk + hk) * D + c8, x);
-        float4 *dst = reinterpret_cast<float4 *>(&kq_s[which][t][c8]);
-        dst[0] = make_float4(x[0], x[1], x[2], x[3]);
-        dst[1] = make_float4(x[4], x[5], x[6], x[7]);
         uint4 hi, lo;
         split_bf16x2(x[0], x[1], hi.x, lo.x);
         split_bf16x2(x[2], x[3], hi.y, lo.y);
@@ -371,41 +363,47 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
     }
     __syncthreads();
 
-    // Gram dots of the tokens' raw keys and queries (k_s.k_t and k_s.q_t for s <= t, q_t.q_t),
-    // one 8-lane group per dot, and the gates
-    {
-        const int l8 = tid & 7, grp = tid >> 3;
-        const int nkk = T * (T + 1) / 2, ndots = 2 * nkk + T;
-        // every lane runs the same number of rounds (the shuffles below take whole warps)
-        for (int base = 0; base < ndots; base += kR128Threads / 8) {
-            const bool live = base + grp < ndots;
-            const int d = live ? base + grp : 0;
-            int kind = d < nkk ? 0 : (d < 2 * nkk ? 1 : 2), e = kind == 0 ? d : (kind == 1 ? d - nkk : d - 2 * nkk);
-            int ss = 0, tt = e;
-            if (kind < 2) {   // e -> (s, t), s <= t, row-major over t
-                tt = 0;
-                while ((tt + 1) * (tt + 2) / 2 <= e) ++tt;
-                ss = e - tt * (tt + 1) / 2;
-            }
-            f2_t x2[8], y2[8];
-            lds_cols16(kq_s[kind == 2 ? 1 : 0][kind == 2 ? tt : ss], l8, x2);
-            lds_cols16(kq_s[kind == 0 ? 0 : 1][tt], l8, y2);
-            float part = dot16(x2, y2);
-            part += __shfl_xor_sync(kFull, part, 4);
-            part += __shfl_xor_sync(kFull, part, 2);
-            part += __shfl_xor_sync(kFull, part, 1);
-            if (live && l8 == 0) {
-                if (kind == 0) s_kk[ss][tt] = part;
-                else if (kind == 1) s_kq[ss][tt] = part;
-                else s_qq[tt] = part;
+    // Gram dots of the tokens' raw keys and queries, X X^T with X = [k_1 .. k_8; q_1 .. q_8] (rows
+    // of unused tokens zero): warp 0 multiplies X by its key tile (n = k_1 .. k_8: k.k and q.k),
+    // warp 1 by its query tile (n = q_1 .. q_8: q.q). The A fragments of X are, pair for pair, the
+    // B fragments of both tiles. Two accumulators (even and odd k-steps) halve the dependent chain.
+    if (warp < 2) {
+        float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const int pc = 8 * ks + 2 * tig;
+            const uint2 xk = *reinterpret_cast<const uint2 *>(&kq_hi[0][gq][pc]);
+            const uint2 xq = *reinterpret_cast<const uint2 *>(&kq_hi[1][gq][pc]);
+            const uint2 xn = warp == 0 ? xk : xq;
+            const uint32_t ax[4] = {xk.x, xq.x, xk.y, xq.y};
+            mma_bf16_m16n8k16(acc[ks & 1], ax, xn.x, xn.y);
+            if constexpr (!IN_BF16) {
+                const uint2 lk = *reinterpret_cast<const uint2 *>(&kq_lo[0][gq][pc]);
+                const uint2 lq = *reinterpret_cast<const uint2 *>(&kq_lo[1][gq][pc]);
+                const uint2 ln = warp == 0 ? lk : lq;
+                const uint32_t al[4] = {lk.x, lq.x, lk.y, lq.y};
+                mma_bf16_m16n8k16(acc[ks & 1], ax, ln.x, ln.y);
+                mma_bf16_m16n8k16(acc[ks & 1], al, xn.x, xn.y);
             }
         }
-    }
-    if (tid < T) {
+        // rows gq (k_gq) in [0], [1] and gq + 8 (q_gq) in [2], [3]; columns n = 2 tig, 2 tig + 1
+        const int n0 = 2 * tig;
+        const float g0 = acc[0][0] + acc[1][0], g1 = acc[0][1] + acc[1][1];
+        const float g2 = acc[0][2] + acc[1][2], g3 = acc[0][3] + acc[1][3];
+        if (warp == 0) {
+            s_kk[gq][n0] = g0;
+            s_kk[gq][n0 + 1] = g1;
+            s_kq[n0][gq] = g2;
+            s_kq[n0 + 1][gq] = g3;
+        } else {
+            if (n0 == gq) s_qq[gq] = g2;
+            if (n0 + 1 == gq) s_qq[gq] = g3;
+        }
+    } else if (warp == 2 && lane < T) {
         float g, beta;
-        gdn_gates(a[(size_t)(t0 + tid) * Hv + h], b[(size_t)(t0 + tid) * Hv + h], A_log[h], dt_bias[h], g, beta);
-        s_alpha[tid] = expf(g);
-        s_beta[tid] = beta;
+        gdn_gates(ga_raw, gb_raw, A_log[h], dt_bias[h], g, beta);
+        s_alpha[lane] = expf(g);
+        s_beta[lane] = beta;
     }
 
     // the row this lane finishes (below: lanes 0, 1 of a group row r0, lanes 2, 3 row r0 + 8) and
