@@ -338,6 +338,21 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
         ga_raw = a[(size_t)(t0 + lane) * Hv + h];
         gb_raw = b[(size_t)(t0 + lane) * Hv + h];
     }
+    // stage the keys and queries: 2 x 8 rows of 16 pieces of 8 values, two pieces a thread. bf16
+    // rows are their own hi pairs: they are copied in asynchronously, ahead of the state loads.
+    if constexpr (IN_BF16) {
+#pragma unroll
+        for (int e = tid; e < 2 * kVerifyMaxT * (D / 8); e += kR128Threads) {
+            const int which = e / (kVerifyMaxT * (D / 8)), rem = e % (kVerifyMaxT * (D / 8));
+            const int t = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
+            uint32_t *dst = &kq_hi[which][t][c8 / 2];
+            if (t < T)
+                cp_async16(dst, reinterpret_cast<const __nv_bfloat16 *>(which ? q : k) + ((size_t)(t0 + t) * Hk + hk) * D + c8);
+            else
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        cp_async_commit();
+    }
     // state rows r0 and r0 + 8, columns 16 ks + 4 tig .. + 3 of each k-step ks (read once)
     float4 sa[8], sb[8];
 #pragma unroll
@@ -345,21 +360,23 @@ gdn_verify128_kernel(const void *__restrict__ q, const void *__restrict__ k, con
         sa[ks] = __ldcs(reinterpret_cast<const float4 *>(S0 + sbase + (size_t)r0 * D + 16 * ks + 4 * tig));
         sb[ks] = __ldcs(reinterpret_cast<const float4 *>(S0 + sbase + (size_t)(r0 + 8) * D + 16 * ks + 4 * tig));
     }
-
-    // stage the keys and queries: 2 x 8 rows of 16 pieces of 8 values, two pieces a thread
+    if constexpr (IN_BF16) {
+        cp_async_wait<0>();
+    } else {
 #pragma unroll
-    for (int e = tid; e < 2 * kVerifyMaxT * (D / 8); e += kR128Threads) {
-        const int which = e / (kVerifyMaxT * (D / 8)), rem = e % (kVerifyMaxT * (D / 8));
-        const int t = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
-        float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-        if (t < T) load8<IN_BF16>(which ? q : k, ((size_t)(t0 + t) * Hk + hk) * D + c8, x);
-        uint4 hi, lo;
-        split_bf16x2(x[0], x[1], hi.x, lo.x);
-        split_bf16x2(x[2], x[3], hi.y, lo.y);
-        split_bf16x2(x[4], x[5], hi.z, lo.z);
-        split_bf16x2(x[6], x[7], hi.w, lo.w);
-        *reinterpret_cast<uint4 *>(&kq_hi[which][t][c8 / 2]) = hi;
-        if constexpr (!IN_BF16) *reinterpret_cast<uint4 *>(&kq_lo[which][t][c8 / 2]) = lo;
+        for (int e = tid; e < 2 * kVerifyMaxT * (D / 8); e += kR128Threads) {
+            const int which = e / (kVerifyMaxT * (D / 8)), rem = e % (kVerifyMaxT * (D / 8));
+            const int t = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
+            float x[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+            if (t < T) load8<false>(which ? q : k, ((size_t)(t0 + t) * Hk + hk) * D + c8, x);
+            uint4 hi, lo;
+            split_bf16x2(x[0], x[1], hi.x, lo.x);
+            split_bf16x2(x[2], x[3], hi.y, lo.y);
+            split_bf16x2(x[4], x[5], hi.z, lo.z);
+            split_bf16x2(x[6], x[7], hi.w, lo.w);
+            *reinterpret_cast<uint4 *>(&kq_hi[which][t][c8 / 2]) = hi;
+            *reinterpret_cast<uint4 *>(&kq_lo[which][t][c8 / 2]) = lo;
+        }
     }
     __syncthreads();
 
